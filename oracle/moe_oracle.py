@@ -1,0 +1,360 @@
+"""CPU oracle for the sparse Mixture-of-Experts FFN forward pass.
+
+TEST INFRASTRUCTURE ONLY. This module is the plain, slow, fp64 statement of
+what the block computes. Only the test suite, ``__graft_entry__.smoke()`` and
+the CPU-baseline / reference arm of ``bench.py`` may import it. The product
+path (the CUDA library and its Python binding) never imports, calls or links
+anything here, and this module imports nothing from the product package.
+
+Sources (web pages, cited by title and section):
+
+* [CS]  "Mixture of Experts and Hybrid Architectures" cheat sheet
+        (aiengineeringfromscratch.com), sections "One MoE layer", "The router
+        in code", "Troubleshooting", "Aux-loss-free balance loop".
+* [KB]  "Mixture of experts and architecture families" knowledge-base page
+        (cv-page-czj.pages.dev), section "The router and load balancing".
+* [DS]  "Sparse MoE FFN" DeepSeek-V3 study note (ai-engineer-exhaustive),
+        section "How it works": eq. 12 (residual form), the SwiGLU equation,
+        the "Routing" paragraph and the "Packed forward (official)" paragraph.
+* [L2]  "Lesson 2 - From the Dense FFN to a Layer of Experts" (fanfani.net),
+        section 2 (boxed MoE equation) and section 4 (shared experts equation).
+
+Everything is computed in float64 from the exact input values (bf16 inputs
+are widened exactly by the caller). No intermediate is rounded. Library
+primitives used as single steps: ``numpy`` matmul, ``exp``, stable
+``argsort``, ``bincount``, ``cumsum``.
+
+Readings taken where the pages are silent or ambiguous (each one is listed
+again in the design notes):
+
+* route_scale multiplies the renormalised gates in both gating modes; the
+  softmax workloads use 1.0, so their gates sum to 1 as [CS] states.
+* The group score is the sum of the two largest biased scores of the group
+  (bias 0 when absent); groups are runs of E/n_groups consecutive experts.
+* Every tie (experts or groups) goes to the lower index, as a stable sort on
+  the negated score gives ([CS] "The router in code" sorts with a key).
+* The k winners are reported in ascending expert id.
+* In softmax mode the bias is added to the raw logit; the gates are the
+  max-subtracted softmax of the selected raw logits ([CS]). [KB]'s
+  softmax-over-all-then-renormalise form is the same number in exact
+  arithmetic; ``moe_forward_dense_loop`` restates it and a test checks it.
+* Sigmoid mode always renormalises over the winners ([DS] "Routing").
+* W1 sits inside SiLU, W3 is the multiplier, W2 projects down ([DS] SwiGLU
+  equation); experts carry no bias vectors.
+* The block returns shared + routed, without the residual ([DS] eq. 12 and
+  the note under it).
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional, Sequence
+
+import numpy as np
+
+GATE_SOFTMAX = 0
+GATE_SIGMOID = 1
+
+__all__ = [
+    "GATE_SOFTMAX", "GATE_SIGMOID", "router_logits", "affinity", "biased_scores",
+    "group_scores", "group_eligibility", "select_experts", "gate_values", "route",
+    "silu", "swiglu_ffn", "expert_outputs", "moe_forward", "moe_forward_dense_loop",
+    "expert_counts_offsets", "permutation_rows", "near_tie_tokens",
+]
+
+
+def _f64(a) -> np.ndarray:
+    return np.asarray(a, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Routing
+# ---------------------------------------------------------------------------
+
+def router_logits(x, w_router) -> np.ndarray:
+    """Router linear layer: ``l[t, e] = u_t . e_e`` for every expert.
+
+    [DS] "Routing": the affinity argument is u_t^T e_i. [CS] "The router in
+    code": one dot product of the hidden state with each router row.
+    x: (T, d); w_router: (E, d). Returns (T, E).
+    """
+    return _f64(x) @ _f64(w_router).T
+
+
+def affinity(logits, gate_mode: int) -> np.ndarray:
+    """Token-to-expert affinity.
+
+    Sigmoid mode: s = 1 / (1 + exp(-l))  ([DS] "Routing").
+    Softmax mode: the raw logit itself; the softmax is taken over the
+    selected experts only, after selection ([CS] "The router in code").
+    """
+    logits = _f64(logits)
+    if gate_mode == GATE_SIGMOID:
+        with np.errstate(over="ignore"):
+            return 1.0 / (1.0 + np.exp(-logits))
+    if gate_mode == GATE_SOFTMAX:
+        return logits.copy()
+    raise ValueError(f"unknown gate mode {gate_mode}")
+
+
+def biased_scores(scores, bias) -> np.ndarray:
+    """Selection score ``s + b``: the bias moves selection only.
+
+    [CS] "The router in code" (bias added before the sort, gates from the
+    unbiased values) and "Troubleshooting" (gate with the raw scores);
+    [DS] "Routing" (top-K on s + b_i).
+    """
+    scores = _f64(scores)
+    if bias is None:
+        return scores.copy()
+    return scores + _f64(bias)[None, :]
+
+
+def group_scores(biased, n_groups: int) -> np.ndarray:
+    """Score of each expert group: the sum of its two largest biased scores.
+
+    [DS] "Routing": 8 groups, keep 4, group score = sum of top-2.
+    Group G holds experts [G*E/n_groups, (G+1)*E/n_groups). Returns (T, n_groups).
+    """
+    biased = _f64(biased)
+    T, E = biased.shape
+    size = E // n_groups
+    per_group = biased.reshape(T, n_groups, size)
+    two_largest = np.sort(per_group, axis=2)[:, :, -2:]
+    return two_largest.sum(axis=2)
+
+
+def _kept_groups(gscore, topk_groups: int) -> np.ndarray:
+    """Indices of the best ``topk_groups`` groups per token, ties to lower index."""
+    order = np.argsort(-gscore, axis=1, kind="stable")
+    return order[:, :topk_groups]
+
+
+def group_eligibility(biased, n_groups: int, topk_groups: int) -> np.ndarray:
+    """Boolean (T, E) mask of experts that sit in a kept group.
+
+    With ``n_groups <= 1`` every expert is eligible (plain top-k).
+    """
+    biased = _f64(biased)
+    T, E = biased.shape
+    if n_groups <= 1:
+        return np.ones((T, E), dtype=bool)
+    keep = np.zeros((T, n_groups), dtype=bool)
+    kept = _kept_groups(group_scores(biased, n_groups), topk_groups)
+    keep[np.arange(T)[:, None], kept] = True
+    return np.repeat(keep, E // n_groups, axis=1)
+
+
+def select_experts(biased, eligible, k: int) -> np.ndarray:
+    """Top-k of the biased scores among eligible experts, ascending expert id.
+
+    A stable sort of the negated scores puts equal scores in index order, so a
+    tie goes to the lower expert index. Returns int64 (T, k).
+    """
+    masked = np.where(eligible, _f64(biased), -np.inf)
+    winners = np.argsort(-masked, axis=1, kind="stable")[:, :k]
+    return np.sort(winners, axis=1)
+
+
+def gate_values(logits, scores, idx, gate_mode: int, route_scale: float) -> np.ndarray:
+    """Gate weight of each selected expert, from the UNBIASED values.
+
+    Softmax: exp(l_i - max) / sum over the k selected raw logits
+    ([CS] "The router in code": softmax over the chosen original scores).
+    Sigmoid: s_i / sum of the k selected s ([DS] "Routing": renormalised
+    over the K_r winners). Both are then multiplied by ``route_scale``
+    ([DS] "Routing": route_scale = 2.5). Returns (T, k).
+    """
+    rows = np.arange(idx.shape[0])[:, None]
+    if gate_mode == GATE_SOFTMAX:
+        chosen = _f64(logits)[rows, idx]
+        top = chosen.max(axis=1, keepdims=True)
+        ex = np.exp(chosen - top)
+        g = ex / ex.sum(axis=1, keepdims=True)
+    elif gate_mode == GATE_SIGMOID:
+        chosen = _f64(scores)[rows, idx]
+        g = chosen / chosen.sum(axis=1, keepdims=True)
+    else:
+        raise ValueError(f"unknown gate mode {gate_mode}")
+    return g * float(route_scale)
+
+
+def route(x, w_router, bias, k: int, gate_mode: int, n_groups: int = 1,
+          topk_groups: int = 1, route_scale: float = 1.0) -> dict:
+    """The whole gate: logits, affinity, biased group-limited top-k, gates.
+
+    Returns a dict with ``idx`` (T, k) ascending expert ids, ``gates`` (T, k),
+    and the intermediates ``logits``, ``scores``, ``biased``, ``eligible``.
+    """
+    logits = router_logits(x, w_router)
+    scores = affinity(logits, gate_mode)
+    biased = biased_scores(scores, bias)
+    eligible = group_eligibility(biased, n_groups, topk_groups)
+    idx = select_experts(biased, eligible, k)
+    gates = gate_values(logits, scores, idx, gate_mode, route_scale)
+    return dict(idx=idx, gates=gates, logits=logits, scores=scores,
+                biased=biased, eligible=eligible)
+
+
+# ---------------------------------------------------------------------------
+# Experts
+# ---------------------------------------------------------------------------
+
+def silu(z) -> np.ndarray:
+    """SiLU(z) = z * sigmoid(z)."""
+    z = _f64(z)
+    with np.errstate(over="ignore"):
+        return z / (1.0 + np.exp(-z))
+
+
+def swiglu_ffn(u, w1, w3, w2) -> np.ndarray:
+    """FFN(u) = W2 (SiLU(W1 u) * W3 u), row-wise over u.
+
+    [DS] SwiGLU equation: W1, W3 in R^{f x d}, W2 in R^{d x f}.
+    u: (n, d). Returns (n, d).
+    """
+    u = _f64(u)
+    h = silu(u @ _f64(w1).T) * (u @ _f64(w3).T)
+    return h @ _f64(w2).T
+
+
+def expert_outputs(x, idx, gates, w1, w3, w2, ws1=None, ws3=None, ws2=None) -> np.ndarray:
+    """Routed sum plus shared expert, per the packed forward.
+
+    [DS] "Packed forward (official)": for each expert, gather the tokens that
+    chose it, run the SwiGLU, scale by the matching gate and scatter-add into
+    a zero buffer; then add the shared FFN over all tokens; no residual
+    ([DS] eq. 12 and the note under it). [L2] section 4 gives the same sum:
+    shared experts with unit weight plus gated routed experts.
+
+    ``w1``/``w3``/``w2`` may be any object whose ``[e]`` gives expert e's
+    matrix (an array stack, or a lazy loader for large workloads).
+    """
+    x = _f64(x)
+    T = x.shape[0]
+    idx = np.asarray(idx)
+    gates = _f64(gates)
+    y = np.zeros_like(x)
+    for e in np.unique(idx):
+        tok, slot = np.nonzero(idx == e)
+        out = swiglu_ffn(x[tok], w1[e], w3[e], w2[e])
+        np.add.at(y, tok, gates[tok, slot][:, None] * out)
+    if ws1 is not None:
+        y += swiglu_ffn(x, ws1, ws3, ws2)
+    return y
+
+
+def moe_forward(x, w_router, bias, w1, w3, w2, k: int, gate_mode: int,
+                n_groups: int = 1, topk_groups: int = 1, route_scale: float = 1.0,
+                ws1=None, ws3=None, ws2=None) -> np.ndarray:
+    """MoE(u) = sum_shared FFN_s(u) + sum_{i in TopK} g_i FFN_i(u).
+
+    [DS] eq. 12 without the u_t skip term; [L2] section 4 shared-expert form.
+    """
+    r = route(x, w_router, bias, k, gate_mode, n_groups, topk_groups, route_scale)
+    return expert_outputs(x, r["idx"], r["gates"], w1, w3, w2, ws1, ws3, ws2)
+
+
+def moe_forward_dense_loop(x, w_router, w1, w3, w2, k: int) -> np.ndarray:
+    """The per-expert loop form with softmax over ALL experts, then renormalise.
+
+    [KB] "The router and load balancing": probabilities from a softmax over
+    all E logits, keep the k largest, divide by their sum, then visit each
+    expert in turn and add its weighted output to the tokens that chose it.
+    No bias, no groups, no shared expert (the page's form has none).
+    """
+    x = _f64(x)
+    logits = router_logits(x, w_router)
+    shifted = logits - logits.max(axis=1, keepdims=True)
+    p = np.exp(shifted)
+    p /= p.sum(axis=1, keepdims=True)
+    T, E = p.shape
+    chosen = np.argsort(-p, axis=1, kind="stable")[:, :k]
+    weight = np.zeros((T, E))
+    rows = np.arange(T)[:, None]
+    weight[rows, chosen] = p[rows, chosen]
+    weight /= weight.sum(axis=1, keepdims=True)
+    out = np.zeros_like(x)
+    for e in range(E):
+        tok = np.nonzero(weight[:, e] > 0)[0]
+        if tok.size == 0:
+            continue
+        out[tok] += weight[tok, e][:, None] * swiglu_ffn(x[tok], w1[e], w3[e], w2[e])
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Packing: counts, offsets, permutation
+# ---------------------------------------------------------------------------
+
+def expert_counts_offsets(idx, E: int):
+    """counts[e] = #tokens that chose e; offsets = exclusive prefix sum (E+1).
+
+    The packed forward gathers, per expert, the tokens whose indices equal it
+    ([DS] "Packed forward"); laying those groups end to end in expert order
+    gives these offsets.
+    """
+    counts = np.bincount(np.asarray(idx).ravel(), minlength=E).astype(np.int64)
+    offsets = np.zeros(E + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(counts)
+    return counts, offsets
+
+
+def permutation_rows(idx, offsets):
+    """Packed row of every (token, slot) pair, tokens in index order per expert.
+
+    row(t, j) = offsets[e] + #{t' < t : e in sel(t')} with e = idx[t, j].
+    Returns (inv_row (T, k), perm_src (T*k,)): ``perm_src[inv_row[t, j]] == t``.
+    """
+    idx = np.asarray(idx)
+    T, k = idx.shape
+    next_free = np.asarray(offsets[:-1], dtype=np.int64).copy()
+    inv_row = np.empty((T, k), dtype=np.int64)
+    perm_src = np.full(int(offsets[-1]), -1, dtype=np.int64)
+    for t in range(T):
+        for j in range(k):
+            e = idx[t, j]
+            inv_row[t, j] = next_free[e]
+            perm_src[next_free[e]] = t
+            next_free[e] += 1
+    return inv_row, perm_src
+
+
+# ---------------------------------------------------------------------------
+# Near ties (which tokens a finite-precision router may legitimately route
+# differently from this fp64 statement)
+# ---------------------------------------------------------------------------
+
+def near_tie_tokens(routed: dict, k: int, n_groups: int = 1, topk_groups: int = 1,
+                    eps: float = 1e-5) -> np.ndarray:
+    """Boolean (T,) flags for tokens whose selection rests on a gap below eps.
+
+    A token is flagged when the k-th and (k+1)-th largest eligible biased
+    scores differ by less than ``eps``, or, with group-limited routing, when
+    the last kept and first dropped group scores differ by less than ``eps``
+    AND swapping those two groups changes the selected set.
+    """
+    biased = routed["biased"]
+    eligible = routed["eligible"]
+    T, E = biased.shape
+    flags = np.zeros(T, dtype=bool)
+    masked = np.where(eligible, biased, -np.inf)
+    srt = -np.sort(-masked, axis=1)
+    n_elig = eligible.sum(axis=1)
+    for t in range(T):
+        if k < n_elig[t] and srt[t, k - 1] - srt[t, k] < eps:
+            flags[t] = True
+    if n_groups > 1 and topk_groups < n_groups:
+        gscore = group_scores(biased, n_groups)
+        order = np.argsort(-gscore, axis=1, kind="stable")
+        size = E // n_groups
+        for t in range(T):
+            last, first_out = order[t, topk_groups - 1], order[t, topk_groups]
+            if gscore[t, last] - gscore[t, first_out] >= eps:
+                continue
+            alt = np.zeros(E, dtype=bool)
+            for g in list(order[t, :topk_groups - 1]) + [first_out]:
+                alt[g * size:(g + 1) * size] = True
+            alt_sel = select_experts(biased[t:t + 1], alt[None, :], k)[0]
+            if not np.array_equal(alt_sel, routed["idx"][t]):
+                flags[t] = True
+    return flags

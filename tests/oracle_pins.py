@@ -1,0 +1,370 @@
+"""Pins of the CPU oracle to facts outside itself.
+
+Each ``pin_*`` function raises AssertionError when the oracle disagrees with a
+closed form, a hand-worked case, an invariant stated on the pages, a brute
+force search, or an independent library routine. ``test_oracle_pins.py`` runs
+them; ``test_oracle_mutations.py`` plants mistakes in the oracle and checks
+that at least one pin catches each.
+
+The hand cases use d = E = f = 2, an identity router and identity expert
+matrices (expert 1's down projection doubled), so every value has a closed
+form in the logistic function: SiLU(u) * u = u^2 * sigma(u) per coordinate,
+and a 2-way softmax is sigma of the logit difference.
+"""
+from __future__ import annotations
+
+import itertools
+import math
+
+import numpy as np
+import torch
+
+import oracle.moe_oracle as orc
+
+
+def sigma(z: float) -> float:
+    return 1.0 / (1.0 + math.exp(-z))
+
+
+def _close(a, b, tol=1e-12):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    assert a.shape == b.shape, (a.shape, b.shape)
+    err = np.max(np.abs(a - b)) if a.size else 0.0
+    assert err <= tol * max(1.0, float(np.max(np.abs(b))) if b.size else 1.0), (a, b, err)
+
+
+# ---------------------------------------------------------------- hand cases
+HAND_X = np.array([[1.0, 0.0], [0.0, 1.0], [2.0, -1.0]])
+HAND_WR = np.eye(2)
+HAND_W1 = np.stack([np.eye(2), np.eye(2)])
+HAND_W3 = np.stack([np.eye(2), np.eye(2)])
+HAND_W2 = np.stack([np.eye(2), 2.0 * np.eye(2)])
+
+
+def _ffn_closed(u, scale):
+    """Identity-weight SwiGLU: scale * u^2 * sigma(u), per coordinate."""
+    return np.array([scale * v * v * sigma(v) for v in u])
+
+
+def _hand(k, gate_mode, bias, route_scale):
+    r = orc.route(HAND_X, HAND_WR, bias, k, gate_mode, route_scale=route_scale)
+    y = orc.moe_forward(HAND_X, HAND_WR, bias, HAND_W1, HAND_W3, HAND_W2, k, gate_mode,
+                        route_scale=route_scale)
+    return r, y
+
+
+def pin_hand_softmax_k1():
+    r, y = _hand(1, orc.GATE_SOFTMAX, None, 1.0)
+    assert r["idx"].ravel().tolist() == [0, 1, 0]
+    _close(r["gates"], np.ones((3, 1)))
+    _close(y[0], _ffn_closed(HAND_X[0], 1.0))
+    _close(y[1], _ffn_closed(HAND_X[1], 2.0))
+    _close(y[2], _ffn_closed(HAND_X[2], 1.0))
+    _close(y[0], [0.731059, 0.0], tol=1e-6)
+    _close(y[2], [3.523188, 0.268941], tol=1e-6)
+
+
+def pin_hand_softmax_k2():
+    r, y = _hand(2, orc.GATE_SOFTMAX, None, 1.0)
+    assert r["idx"].tolist() == [[0, 1]] * 3
+    for t, u in enumerate(HAND_X):
+        g0 = sigma(u[0] - u[1])            # two-way softmax of logits (u0, u1)
+        _close(r["gates"][t], [g0, 1.0 - g0])
+        _close(y[t], _ffn_closed(u, g0 * 1.0 + (1.0 - g0) * 2.0))
+    _close(y[0], [0.927671, 0.0], tol=1e-6)
+    _close(y[1], [0.0, 1.265505], tol=1e-6)
+
+
+def pin_hand_sigmoid_bias_moves_selection():
+    # Without bias token 0 picks expert 0 (sigma(1) > sigma(0)); a +0.3 bias on
+    # expert 1 lifts sigma(0) + 0.3 = 0.8 above sigma(1) = 0.731: selection flips,
+    # the single gate is still route_scale (renormalised over one winner).
+    r0, y0 = _hand(1, orc.GATE_SIGMOID, np.array([0.0, 0.0]), 2.5)
+    r1, y1 = _hand(1, orc.GATE_SIGMOID, np.array([0.0, 0.3]), 2.5)
+    assert r0["idx"].ravel().tolist() == [0, 1, 0]
+    assert r1["idx"].ravel().tolist() == [1, 1, 0]
+    _close(r1["gates"], np.full((3, 1), 2.5))
+    _close(y0[0], _ffn_closed(HAND_X[0], 2.5 * 1.0))
+    _close(y1[0], _ffn_closed(HAND_X[0], 2.5 * 2.0))
+    _close(y1[0], [3.655293, 0.0], tol=1e-6)
+    _close(y1[2], [8.807971, 0.672354], tol=1e-6)
+
+
+def pin_hand_sigmoid_k2_gates_ignore_bias():
+    # k = E: both experts always win; the gates come from the raw sigmoid and
+    # must not move with the bias.
+    ra, ya = _hand(2, orc.GATE_SIGMOID, np.array([0.0, 0.0]), 2.5)
+    rb, yb = _hand(2, orc.GATE_SIGMOID, np.array([0.0, 0.3]), 2.5)
+    for t, u in enumerate(HAND_X):
+        s0, s1 = sigma(u[0]), sigma(u[1])
+        g = [2.5 * s0 / (s0 + s1), 2.5 * s1 / (s0 + s1)]
+        _close(ra["gates"][t], g)
+        _close(rb["gates"][t], g)
+        _close(ya[t], _ffn_closed(u, g[0] + 2.0 * g[1]))
+    _close(ya, yb)
+    _close(ra["gates"][0], [1.484614, 1.015386], tol=1e-6)
+    _close(ya[2], [10.86829, 0.829627], tol=1e-6)
+
+
+def pin_tie_goes_to_lower_index():
+    x = np.array([[1.0, 1.0], [0.5, 0.5]])
+    for mode in (orc.GATE_SOFTMAX, orc.GATE_SIGMOID):
+        r = orc.route(x, np.eye(2), None, 1, mode, route_scale=1.0)
+        assert r["idx"].ravel().tolist() == [0, 0]
+    # Group tie: two groups with identical scores, keep one -> the lower group.
+    b = np.array([[0.5, 0.1, 0.5, 0.1]])
+    el = orc.group_eligibility(b, 2, 1)
+    assert el.tolist() == [[True, True, False, False]]
+
+
+# ------------------------------------------------------------ closed forms
+def pin_router_is_u_dot_e():
+    # A permutation router: e_e = unit vector of coordinate perm[e], so the
+    # logit of expert e is u[perm[e]]. A transposed operand gives perm^-1.
+    perm = [2, 0, 3, 1]
+    wr = np.zeros((4, 4))
+    for e, c in enumerate(perm):
+        wr[e, c] = 1.0
+    x = np.array([[10.0, 20.0, 30.0, 40.0], [1.0, -2.0, 3.0, -4.0]])
+    _close(orc.router_logits(x, wr), x[:, perm])
+    # Non-square: E=3 experts over d=5 hidden.
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((4, 5))
+    wr = rng.standard_normal((3, 5))
+    expect = np.array([[sum(x[t, c] * wr[e, c] for c in range(5)) for e in range(3)]
+                       for t in range(4)])
+    _close(orc.router_logits(x, wr), expect, tol=1e-12)
+
+
+def pin_sigmoid_values():
+    l = np.array([[0.0, math.log(3.0), -math.log(3.0), 40.0, -40.0]])
+    s = orc.affinity(l, orc.GATE_SIGMOID)
+    _close(s[0, :3], [0.5, 0.75, 0.25])
+    assert 1.0 - 1e-15 < s[0, 3] <= 1.0 and 0.0 <= s[0, 4] < 1e-17
+    _close(orc.affinity(l, orc.GATE_SOFTMAX), l)
+
+
+def pin_softmax_two_way_is_logistic():
+    rng = np.random.default_rng(5)
+    lg = rng.standard_normal((16, 6)) * 3
+    idx = np.sort(np.stack([rng.choice(6, 2, replace=False) for _ in range(16)]), axis=1)
+    g = orc.gate_values(lg, lg, idx, orc.GATE_SOFTMAX, 1.0)
+    for t in range(16):
+        a, b = lg[t, idx[t, 0]], lg[t, idx[t, 1]]
+        _close(g[t], [sigma(a - b), sigma(b - a)])
+
+
+# -------------------------------------------------------------- invariants
+def _random_case(rng, T=12, d=6, E=8, f=5, shared=0):
+    return dict(
+        x=rng.standard_normal((T, d)),
+        wr=rng.standard_normal((E, d)) / math.sqrt(d),
+        w1=rng.standard_normal((E, f, d)) / math.sqrt(d),
+        w3=rng.standard_normal((E, f, d)) / math.sqrt(d),
+        w2=rng.standard_normal((E, d, f)) / math.sqrt(f),
+        ws1=rng.standard_normal((shared, d)) if shared else None,
+        ws3=rng.standard_normal((shared, d)) if shared else None,
+        ws2=rng.standard_normal((d, shared)) if shared else None,
+    )
+
+
+def pin_gate_sums():
+    rng = np.random.default_rng(11)
+    c = _random_case(rng, T=40, E=16)
+    bias = rng.uniform(-0.3, 0.3, 16)
+    for k in (1, 2, 5, 16):
+        r = orc.route(c["x"], c["wr"], bias, k, orc.GATE_SOFTMAX)
+        _close(r["gates"].sum(axis=1), np.ones(40))
+        assert np.all(r["gates"] > 0)
+        for scale in (1.0, 2.5):
+            r = orc.route(c["x"], c["wr"], bias, k, orc.GATE_SIGMOID, 4, 2 if k <= 8 else 4,
+                          route_scale=scale)
+            _close(r["gates"].sum(axis=1), np.full(40, scale))
+
+
+def pin_bias_moves_selection_not_gates():
+    rng = np.random.default_rng(12)
+    c = _random_case(rng, T=50, E=8)
+    for mode in (orc.GATE_SOFTMAX, orc.GATE_SIGMOID):
+        base = orc.route(c["x"], c["wr"], None, 3, mode, route_scale=2.5)
+        # A constant shift never changes the order: same winners, same gates.
+        shifted = orc.route(c["x"], c["wr"], np.full(8, 0.7), 3, mode, route_scale=2.5)
+        assert np.array_equal(base["idx"], shifted["idx"])
+        _close(base["gates"], shifted["gates"])
+        # A bias that changes selection: wherever a token keeps its winners,
+        # its gates are unchanged; some tokens must move.
+        b = np.zeros(8)
+        b[7] = 5.0
+        moved = orc.route(c["x"], c["wr"], b, 3, mode, route_scale=2.5)
+        assert np.all(moved["idx"][:, -1] == 7)
+        same = np.all(moved["idx"] == base["idx"], axis=1)
+        assert same.sum() < 50
+        _close(moved["gates"][same], base["gates"][same])
+        # Gates of a moved token are the unbiased renormalisation over its winners.
+        rows = np.arange(50)[:, None]
+        if mode == orc.GATE_SIGMOID:
+            s = moved["scores"][rows, moved["idx"]]
+            _close(moved["gates"], 2.5 * s / s.sum(axis=1, keepdims=True))
+        else:
+            l = moved["logits"][rows, moved["idx"]]
+            ex = np.exp(l - l.max(axis=1, keepdims=True))
+            _close(moved["gates"], 2.5 * ex / ex.sum(axis=1, keepdims=True))
+
+
+def pin_k_equals_E_bias_irrelevant():
+    rng = np.random.default_rng(13)
+    c = _random_case(rng, T=10, E=4)
+    for mode in (orc.GATE_SOFTMAX, orc.GATE_SIGMOID):
+        ya = orc.moe_forward(c["x"], c["wr"], None, c["w1"], c["w3"], c["w2"], 4, mode,
+                             route_scale=2.5)
+        yb = orc.moe_forward(c["x"], c["wr"], rng.uniform(-3, 3, 4), c["w1"], c["w3"],
+                             c["w2"], 4, mode, route_scale=2.5)
+        _close(ya, yb, tol=1e-12)
+
+
+# ------------------------------------------------------------- brute force
+def _brute_topk(vals, allowed, k):
+    best, best_set = None, None
+    for combo in itertools.combinations([e for e in range(len(vals)) if allowed[e]], k):
+        s = math.fsum(vals[e] for e in combo)
+        if best is None or s > best:
+            best, best_set = s, combo
+    return list(best_set)
+
+
+def pin_brute_force_topk():
+    rng = np.random.default_rng(21)
+    for trial in range(60):
+        E = int(rng.integers(2, 9))
+        k = int(rng.integers(1, E + 1))
+        vals = rng.integers(-3, 4, size=E).astype(np.float64)   # many exact ties
+        got = orc.select_experts(vals[None, :], np.ones((1, E), bool), k)[0]
+        assert got.tolist() == _brute_topk(vals.tolist(), [True] * E, k), (vals, k, got)
+
+
+def _brute_group_route(vals, n_groups, topk_groups, k):
+    E = len(vals)
+    size = E // n_groups
+    gscore = []
+    for g in range(n_groups):
+        mem = range(g * size, (g + 1) * size)
+        gscore.append(max(vals[a] + vals[b] for a in mem for b in mem if a < b))
+    kept = _brute_topk(gscore, [True] * n_groups, topk_groups)
+    allowed = [e // size in kept for e in range(E)]
+    return _brute_topk(vals, allowed, k)
+
+
+def pin_brute_force_group_limited():
+    # Hand case: expert 0 has the single best score but group 1 has the best
+    # top-2 sum (0.6 + 0.5 > 0.9 + 0.0); keeping one group selects expert 2.
+    b = np.array([[0.9, 0.0, 0.6, 0.5]])
+    assert orc.select_experts(b, orc.group_eligibility(b, 2, 1), 1)[0].tolist() == [2]
+    rng = np.random.default_rng(22)
+    for trial in range(60):
+        n_groups = int(rng.choice([2, 4]))
+        size = int(rng.choice([2, 3]))
+        E = n_groups * size
+        tg = int(rng.integers(1, n_groups + 1))
+        k = int(rng.integers(1, tg * size + 1))
+        vals = rng.integers(-4, 5, size=E).astype(np.float64) / 2
+        got = orc.select_experts(vals[None, :], orc.group_eligibility(vals[None, :], n_groups, tg), k)
+        assert got[0].tolist() == _brute_group_route(vals.tolist(), n_groups, tg, k), (vals, n_groups, tg, k)
+
+
+# --------------------------------------------------- library special cases
+def _torch_swiglu(u, w1, w3, w2):
+    u, w1, w3, w2 = (torch.as_tensor(a, dtype=torch.float64) for a in (u, w1, w3, w2))
+    return torch.nn.functional.linear(
+        torch.nn.functional.silu(torch.nn.functional.linear(u, w1)) * torch.nn.functional.linear(u, w3),
+        w2).numpy()
+
+
+def pin_single_expert_is_dense_swiglu():
+    rng = np.random.default_rng(31)
+    T, d, f = 9, 7, 5
+    x = rng.standard_normal((T, d))
+    w1, w3 = rng.standard_normal((1, f, d)), rng.standard_normal((1, f, d))
+    w2 = rng.standard_normal((1, d, f))
+    y = orc.moe_forward(x, rng.standard_normal((1, d)), None, w1, w3, w2, 1, orc.GATE_SOFTMAX)
+    _close(y, _torch_swiglu(x, w1[0], w3[0], w2[0]), tol=1e-12)
+    _close(orc.swiglu_ffn(x, w1[0], w3[0], w2[0]), _torch_swiglu(x, w1[0], w3[0], w2[0]), tol=1e-12)
+
+
+def pin_shared_expert_added_no_residual():
+    rng = np.random.default_rng(32)
+    c = _random_case(rng, T=8, d=6, E=4, f=3, shared=10)
+    zero_w2 = np.zeros_like(c["w2"])
+    y = orc.moe_forward(c["x"], c["wr"], None, c["w1"], c["w3"], zero_w2, 2, orc.GATE_SIGMOID,
+                        route_scale=2.5, ws1=c["ws1"], ws3=c["ws3"], ws2=c["ws2"])
+    _close(y, _torch_swiglu(c["x"], c["ws1"], c["ws3"], c["ws2"]), tol=1e-12)
+    # All-zero weights give a zero output: the block adds no residual.
+    yz = orc.moe_forward(c["x"], c["wr"], None, np.zeros_like(c["w1"]), np.zeros_like(c["w3"]),
+                         zero_w2, 2, orc.GATE_SOFTMAX, ws1=np.zeros_like(c["ws1"]),
+                         ws3=np.zeros_like(c["ws3"]), ws2=np.zeros_like(c["ws2"]))
+    _close(yz, np.zeros_like(c["x"]))
+    # Shared + routed splits additively.
+    yr = orc.moe_forward(c["x"], c["wr"], None, c["w1"], c["w3"], c["w2"], 2, orc.GATE_SIGMOID,
+                         route_scale=2.5)
+    ys = orc.moe_forward(c["x"], c["wr"], None, c["w1"], c["w3"], c["w2"], 2, orc.GATE_SIGMOID,
+                         route_scale=2.5, ws1=c["ws1"], ws3=c["ws3"], ws2=c["ws2"])
+    _close(ys - yr, _torch_swiglu(c["x"], c["ws1"], c["ws3"], c["ws2"]), tol=1e-12)
+
+
+def pin_routed_sum_per_token_by_hand():
+    rng = np.random.default_rng(33)
+    c = _random_case(rng, T=6, d=5, E=5, f=4)
+    r = orc.route(c["x"], c["wr"], None, 2, orc.GATE_SIGMOID, route_scale=2.5)
+    y = orc.expert_outputs(c["x"], r["idx"], r["gates"], c["w1"], c["w3"], c["w2"])
+    for t in range(6):
+        acc = np.zeros(5)
+        for j in range(2):
+            e = r["idx"][t, j]
+            acc += r["gates"][t, j] * _torch_swiglu(c["x"][t:t + 1], c["w1"][e], c["w3"][e], c["w2"][e])[0]
+        _close(y[t], acc, tol=1e-12)
+
+
+def pin_packed_equals_dense_loop():
+    rng = np.random.default_rng(41)
+    for E, k in ((4, 1), (6, 2), (8, 3), (5, 5)):
+        c = _random_case(rng, T=15, d=6, E=E, f=4)
+        packed = orc.moe_forward(c["x"], c["wr"], None, c["w1"], c["w3"], c["w2"], k, orc.GATE_SOFTMAX)
+        loop = orc.moe_forward_dense_loop(c["x"], c["wr"], c["w1"], c["w3"], c["w2"], k)
+        _close(packed, loop, tol=1e-11)
+
+
+# ------------------------------------------------------------ packing
+def pin_counts_offsets_rows():
+    rng = np.random.default_rng(51)
+    T, E, k = 37, 9, 3
+    idx = np.sort(np.stack([rng.choice(E, k, replace=False) for _ in range(T)]), axis=1)
+    counts, offsets = orc.expert_counts_offsets(idx, E)
+    assert counts.sum() == T * k and offsets[0] == 0 and offsets[-1] == T * k
+    for e in range(E):
+        assert counts[e] == sum(int(e in idx[t]) for t in range(T))
+        assert offsets[e] == sum(counts[:e])
+    inv_row, perm_src = orc.permutation_rows(idx, offsets)
+    # Independent statement: sort the (expert, token) pairs lexicographically;
+    # a pair's position in that order is its packed row.
+    pairs = sorted((idx[t, j], t, j) for t in range(T) for j in range(k))
+    for row, (e, t, j) in enumerate(pairs):
+        assert inv_row[t, j] == row and perm_src[row] == t
+    assert sorted(perm_src.tolist()) == sorted([t for t in range(T) for _ in range(k)])
+
+
+def pin_near_tie_flags():
+    # Token 0: an exact tie between the 2nd and 3rd score (k = 2) -> flagged.
+    # Token 1: wide gaps -> not flagged.
+    lg = np.array([[3.0, 1.0, 1.0, -2.0], [3.0, 2.0, 0.0, -2.0]])
+    r = orc.route(lg, np.eye(4), None, 2, orc.GATE_SOFTMAX)
+    assert orc.near_tie_tokens(r, 2).tolist() == [True, False]
+    # Group boundary tie that changes the selection is flagged; one that does
+    # not (both candidate groups lose to the kept group's experts) is not.
+    b = np.array([[0.9, 0.8, 0.5, 0.1, 0.5, 0.1], [0.9, 0.8, 0.5, 0.1, 0.5, 0.1]])
+    r = orc.route(b, np.eye(6), None, 3, orc.GATE_SOFTMAX, n_groups=3, topk_groups=2)
+    assert orc.near_tie_tokens(r, 3, 3, 2).tolist() == [True, True]
+    r = orc.route(b, np.eye(6), None, 2, orc.GATE_SOFTMAX, n_groups=3, topk_groups=2)
+    assert orc.near_tie_tokens(r, 2, 3, 2).tolist() == [False, False]
+
+
+ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]

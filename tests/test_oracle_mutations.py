@@ -1,0 +1,158 @@
+"""Plant plausible mistakes in the CPU oracle and check the pins catch each.
+
+Every mutation replaces one oracle function (through the module's globals,
+so the oracle's own callers see it) with a variant that carries one error:
+a dropped term, a wrong sign or index, a transposed or swapped operand, a
+missing step. The pins must fail (raise) for every one of them.
+"""
+import numpy as np
+import pytest
+
+import oracle.moe_oracle as orc
+import oracle_pins
+
+_orig = {name: getattr(orc, name) for name in dir(orc) if callable(getattr(orc, name))}
+
+
+def _swiglu_swapped(u, w1, w3, w2):
+    return _orig["swiglu_ffn"](u, w3, w1, w2)
+
+
+def _swiglu_no_silu(u, w1, w3, w2):
+    u = np.asarray(u, np.float64)
+    h = (u @ np.asarray(w1, np.float64).T) * (u @ np.asarray(w3, np.float64).T)
+    return h @ np.asarray(w2, np.float64).T
+
+
+def _swiglu_down_transposed(u, w1, w3, w2):
+    return _orig["swiglu_ffn"](u, w1, w3, np.swapaxes(np.asarray(w2), -1, -2))
+
+
+def _silu_dropped_z(z):
+    return 1.0 / (1.0 + np.exp(-np.asarray(z, np.float64)))
+
+
+def _sigmoid_wrong_sign(logits, gate_mode):
+    if gate_mode == orc.GATE_SIGMOID:
+        return 1.0 / (1.0 + np.exp(np.asarray(logits, np.float64)))
+    return _orig["affinity"](logits, gate_mode)
+
+
+def _router_transposed(x, w_router):
+    x = np.asarray(x, np.float64)
+    w = np.asarray(w_router, np.float64)
+    if w.shape[0] == w.shape[1]:
+        return x @ w
+    return x @ w.T[:, ::-1]
+
+
+def _route_gates_use_biased(x, w_router, bias, k, gate_mode, n_groups=1, topk_groups=1,
+                            route_scale=1.0):
+    r = _orig["route"](x, w_router, bias, k, gate_mode, n_groups, topk_groups, route_scale)
+    r["gates"] = _orig["gate_values"](r["biased"], r["biased"], r["idx"], gate_mode, route_scale)
+    return r
+
+
+def _gates_no_renorm(logits, scores, idx, gate_mode, route_scale):
+    if gate_mode == orc.GATE_SIGMOID:
+        rows = np.arange(idx.shape[0])[:, None]
+        return np.asarray(scores, np.float64)[rows, idx] * route_scale
+    return _orig["gate_values"](logits, scores, idx, gate_mode, route_scale)
+
+
+def _gates_no_scale(logits, scores, idx, gate_mode, route_scale):
+    return _orig["gate_values"](logits, scores, idx, gate_mode, 1.0)
+
+
+def _group_max(biased, n_groups):
+    b = np.asarray(biased, np.float64)
+    T, E = b.shape
+    return b.reshape(T, n_groups, E // n_groups).max(axis=2)
+
+
+def _select_ties_high(biased, eligible, k):
+    masked = np.where(eligible, np.asarray(biased, np.float64), -np.inf)
+    rev = masked[:, ::-1]
+    win = np.argsort(-rev, axis=1, kind="stable")[:, :k]
+    return np.sort(masked.shape[1] - 1 - win, axis=1)
+
+
+def _select_biggest_last(biased, eligible, k):
+    masked = np.where(eligible, np.asarray(biased, np.float64), -np.inf)
+    win = np.argsort(-masked, axis=1, kind="stable")[:, 1:k + 1]
+    return np.sort(win, axis=1)
+
+
+def _outputs_no_shared(x, idx, gates, w1, w3, w2, ws1=None, ws3=None, ws2=None):
+    return _orig["expert_outputs"](x, idx, gates, w1, w3, w2)
+
+
+def _outputs_with_residual(x, idx, gates, w1, w3, w2, ws1=None, ws3=None, ws2=None):
+    return _orig["expert_outputs"](x, idx, gates, w1, w3, w2, ws1, ws3, ws2) + np.asarray(x, np.float64)
+
+
+def _outputs_slot_swapped(x, idx, gates, w1, w3, w2, ws1=None, ws3=None, ws2=None):
+    return _orig["expert_outputs"](x, idx, np.asarray(gates)[:, ::-1], w1, w3, w2, ws1, ws3, ws2)
+
+
+def _rows_reverse_tokens(idx, offsets):
+    inv_row, perm_src = _orig["permutation_rows"](np.asarray(idx)[::-1], offsets)
+    return inv_row[::-1], (len(idx) - 1 - perm_src)
+
+
+def _counts_off_by_one(idx, E):
+    counts, offsets = _orig["expert_counts_offsets"](idx, E)
+    offsets = offsets.copy()
+    offsets[1:-1] += 1
+    return counts, offsets
+
+
+def _near_tie_none(routed, k, n_groups=1, topk_groups=1, eps=1e-5):
+    return np.zeros(routed["idx"].shape[0], dtype=bool)
+
+
+def _loop_no_renorm(x, w_router, w1, w3, w2, k):
+    # Dense-loop form that forgets to renormalise the kept probabilities.
+    x = np.asarray(x, np.float64)
+    lg = _orig["router_logits"](x, w_router)
+    p = np.exp(lg - lg.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    idx = np.sort(np.argsort(-p, axis=1, kind="stable")[:, :k], axis=1)
+    rows = np.arange(x.shape[0])[:, None]
+    return _orig["expert_outputs"](x, idx, p[rows, idx], w1, w3, w2)
+
+
+MUTATIONS = {
+    "swiglu_w1_w3_swapped": ("swiglu_ffn", _swiglu_swapped),
+    "swiglu_no_silu": ("swiglu_ffn", _swiglu_no_silu),
+    "swiglu_down_transposed": ("swiglu_ffn", _swiglu_down_transposed),
+    "silu_drops_z": ("silu", _silu_dropped_z),
+    "sigmoid_wrong_sign": ("affinity", _sigmoid_wrong_sign),
+    "router_transposed": ("router_logits", _router_transposed),
+    "gates_from_biased": ("route", _route_gates_use_biased),
+    "gates_not_renormalised": ("gate_values", _gates_no_renorm),
+    "route_scale_dropped": ("gate_values", _gates_no_scale),
+    "group_score_max": ("group_scores", _group_max),
+    "ties_to_higher_index": ("select_experts", _select_ties_high),
+    "topk_off_by_one": ("select_experts", _select_biggest_last),
+    "shared_expert_dropped": ("expert_outputs", _outputs_no_shared),
+    "residual_added": ("expert_outputs", _outputs_with_residual),
+    "gate_slot_mismatch": ("expert_outputs", _outputs_slot_swapped),
+    "rows_reverse_token_order": ("permutation_rows", _rows_reverse_tokens),
+    "offsets_off_by_one": ("expert_counts_offsets", _counts_off_by_one),
+    "near_ties_never_flagged": ("near_tie_tokens", _near_tie_none),
+    "dense_loop_no_renorm": ("moe_forward_dense_loop", _loop_no_renorm),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_mutation_is_caught(name, monkeypatch):
+    attr, fn = MUTATIONS[name]
+    monkeypatch.setattr(orc, attr, fn)
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin()
+        except Exception as exc:  # AssertionError, or a shape error from a transposed operand
+            caught.append((pin.__name__, type(exc).__name__))
+    assert caught, f"mutation {name} passed every pin"
