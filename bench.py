@@ -1,0 +1,448 @@
+#!/usr/bin/env python
+"""Throughput of the sparse MoE FFN block forward on B200.
+
+One step = one whole forward pass of the block (router GEMM, top-k and
+gates, offsets, permute, SwiGLU expert GEMMs, down GEMMs, combine with the
+shared expert) over one batch of T tokens, through ``moe_forward`` of the C
+ABI. Default workload: the DeepSeek-V3-shaped layer (T=4096, d=7168, 256
+routed experts + 1 shared, inner 2048, top-8, sigmoid, 8 groups keep 4,
+route_scale 2.5), bf16 storage with fp32 accumulation, synthetic seeded data.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl mine|reference]
+
+With N > 1 (launched by torch.distributed.run) every rank runs an
+independent replica on its own GPU (the block has no exchange step on one
+node's data-parallel path): weak scaling, value = all ranks' tokens / the
+slowest rank's time. Rank 0 prints one JSON line.
+
+``--impl reference`` times the CPU oracle (the plain fp64 statement of the
+block) on a bounded sample of the same workload: the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "MoE-layer tokens/s and active TFLOP/s at DeepSeek-V3 shape; % bf16 / HBM roofline"
+KERNELS_PER_FORWARD = 8   # router GEMM, top-k, chunk scan, offsets, permute, gate/up, down, combine
+CPU_SAMPLE_TOKENS = {"tiny_fp32": 64, "decode_fine": 32, "deepseek_v3": 16, "mixtral_8x7b": 8,
+                     "deepseek_v3_skewed": 64}
+REF_STEP_TOKENS = {"tiny_fp32": 64, "decode_fine": 8, "deepseek_v3": 2, "mixtral_8x7b": 2,
+                   "deepseek_v3_skewed": 8}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="deepseek_v3")
+    ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
+    ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of a CUDA graph")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], tensor=d["bf16_tflops"], tensor_sustained=d["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm=6650.0, tensor=1590.0, tensor_sustained=1400.0, source="fallback")
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while work runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.proc = None
+        self.dev = device_index
+
+    def start(self):
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:
+            sel = str(self.dev)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", sel, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), [v.strip() for v in line.split(",")]))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        rows = [s for t, s in self.samples if t0 <= t <= t1]
+        window = "timed region"
+        if len(rows) < 3:
+            rows = [s for _, s in self.samples]
+            window = "warm-up and timed region (timed region shorter than 3 samples)"
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [num(r[0]) for r in rows if num(r[0]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if len(r) > 4 + i and r[4 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": num(rows[0][1]), "reasons": reasons, "samples": len(rows), "window": window,
+                "power_w_max": max((num(r[2]) or 0.0) for r in rows)}
+
+
+# ------------------------------------------------------------ work accounting
+def stage_work(cfg, counts):
+    """Algorithmic bytes and flops of each stage (the design doc lists the formulas)."""
+    es = cfg.elem_bytes
+    T, d, E, k, f, fs = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.f_shared
+    touched = int((counts > 0).sum())
+    rows, srows = T * k, (T if fs else 0)
+    w = {}
+    w["route"] = dict(bytes=(T * d + E * d) * es + T * k * 8 + T * E * 4 * 2, flops=2.0 * T * E * d)
+    w["permute"] = dict(bytes=(T * d + rows * d) * es + rows * 8, flops=0.0)
+    w["gate_up"] = dict(bytes=(touched * 2 * f * d + 2 * fs * d) * es + (rows * d + srows * d) * es
+                        + (rows * f + srows * fs) * es,
+                        flops=4.0 * (rows * f + srows * fs) * d)
+    w["down"] = dict(bytes=(touched * d * f + d * fs) * es + (rows * f + srows * fs) * es
+                     + (rows * d + srows * d) * es,
+                     flops=2.0 * (rows * f + srows * fs) * d)
+    w["combine"] = dict(bytes=(rows * d + srows * d + T * d) * es + rows * 8, flops=0.0)
+    return w, touched
+
+
+def source_sha(path):
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+
+def traffic_for(workload, stage):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel is unchanged."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+        e = d.get(workload, {}).get(stage)
+        if not e:
+            return None
+        src = os.path.join(ROOT, e["source"])
+        if source_sha(src) != e["source_sha256_16"]:
+            return None
+        return e["bytes_per_launch"]
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------- oracle arm
+def oracle_sample_time(cfg, inp, n_tokens, seed):
+    """Run the CPU oracle on ``n_tokens`` seeded tokens; returns (seconds, threads)."""
+    import numpy as np
+    import oracle.moe_oracle as orc
+    from mixture_experts_ffn_sigmoid_b200.inputs import sample_token_ids
+
+    def f64(t):
+        return None if t is None else t.detach().to("cpu").to(torch.float64).numpy()
+
+    class Lazy:
+        def __init__(self, t):
+            self.t = t
+
+        def __getitem__(self, e):
+            return f64(self.t[int(e)])
+
+    tok = sample_token_ids(cfg.T, n_tokens, seed=seed)
+    x = inp["x"][tok.to(inp["x"].device)]
+    wr = f64(inp["w_router"])
+    bias = f64(inp["bias"])
+    shared = [f64(inp[k]) for k in ("ws1", "ws3", "ws2")]
+    t0 = time.perf_counter()
+    r = orc.route(f64(x), wr, bias, cfg.k, cfg.gate_mode, cfg.n_groups, cfg.topk_groups, cfg.route_scale)
+    orc.expert_outputs(f64(x), r["idx"], r["gates"], Lazy(inp["w1"]), Lazy(inp["w3"]), Lazy(inp["w2"]),
+                       *shared)
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        threads = os.cpu_count() or 1
+    return dt, threads
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from mixture_experts_ffn_sigmoid_b200.inputs import CONFIGS, make_inputs
+    cfg = CONFIGS[args.config]
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0"))) if torch.cuda.is_available() \
+        else torch.device("cpu")
+    inp = make_inputs(cfg, dev, seed=0)
+    n = min(REF_STEP_TOKENS.get(cfg.name, 4), cfg.T)
+    for i in range(args.warmup):
+        oracle_sample_time(cfg, inp, n, seed=100 + i)
+    times, threads = [], 1
+    for i in range(args.steps):
+        dt, threads = oracle_sample_time(cfg, inp, n, seed=1000 + i)
+        times.append(dt)
+    total = sum(times)
+    value = n * args.steps / total
+    sample = f"{n} seeded tokens of the {cfg.name} workload per step (routing over all experts, " \
+             f"FFN of every selected expert and the shared expert, fp64)"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k, "f": cfg.f,
+                       "f_shared": cfg.f_shared},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------- our arm
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    from mixture_experts_ffn_sigmoid_b200 import binding as B
+    from mixture_experts_ffn_sigmoid_b200.inputs import CONFIGS, make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    cfg = CONFIGS[args.config]
+    B.lib()
+    inp = make_inputs(cfg, dev, seed=0)
+    if rank > 0:
+        inp["x"] = make_inputs(cfg, dev, seed=rank, x_only=True)["x"]
+    T, d = cfg.T, cfg.d
+    ws = B.alloc_workspace(cfg, dev)
+    y = torch.empty((T, d), dtype=cfg.torch_dtype, device=dev)
+
+    def forward():
+        B.moe_forward(cfg, inp["x"], inp["w_router"], inp["bias"], inp["w1"], inp["w3"], inp["w2"],
+                      inp["ws1"], inp["ws3"], inp["ws2"], y, ws)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    for _ in range(max(args.warmup, 3)):
+        forward()
+    torch.cuda.synchronize()
+    assert B.moe_get_device_error(ws) == B.MOE_OK
+
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            forward()
+        graph.replay()
+        torch.cuda.synchronize()
+    run = graph.replay if graph is not None else forward
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    # ---- timed region: K whole forward passes --------------------------------
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        run()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier()
+    ms_total = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_total = t.item()
+    ms_step = ms_total / args.steps
+    value = world * T / (ms_step / 1e3)
+    assert B.moe_get_device_error(ws) == B.MOE_OK
+    sampler.stop()
+    clocks = sampler.summary(t_wall0, t_wall1)
+
+    # ---- stage breakdown: the same kernels through the per-stage entry points,
+    # one CUDA event between stages on the launching stream ----------------------
+    k, E = cfg.k, cfg.E
+    rows = T * k
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    gate = torch.empty((T, k), dtype=torch.float32, device=dev)
+    counts = torch.empty((E,), dtype=torch.int32, device=dev)
+    offsets = torch.empty((E + 1,), dtype=torch.int32, device=dev)
+    x_perm = torch.empty((rows, d), dtype=cfg.torch_dtype, device=dev)
+    perm_src = torch.empty((rows,), dtype=torch.int32, device=dev)
+    inv_row = torch.empty((T, k), dtype=torch.int32, device=dev)
+    h = torch.empty((rows, cfg.f), dtype=cfg.torch_dtype, device=dev)
+    sh = cfg.f_shared > 0
+    h_s = torch.empty((T, cfg.f_shared), dtype=cfg.torch_dtype, device=dev) if sh else None
+    y_perm = torch.empty((rows, d), dtype=cfg.torch_dtype, device=dev)
+    y_s = torch.empty((T, d), dtype=cfg.torch_dtype, device=dev) if sh else None
+    y2 = torch.empty_like(y)
+    names = ["route", "permute", "gate_up", "down", "combine"]
+    calls = [
+        lambda: B.moe_route(cfg, inp["x"], inp["w_router"], inp["bias"], idx, gate, counts, offsets, ws),
+        lambda: B.moe_permute(cfg, inp["x"], idx, offsets, x_perm, perm_src, inv_row, ws),
+        lambda: B.moe_expert_gate_up(cfg, x_perm, offsets, inp["w1"], inp["w3"], inp["x"] if sh else None,
+                                     inp["ws1"], inp["ws3"], h, h_s, ws),
+        lambda: B.moe_expert_down(cfg, h, offsets, inp["w2"], h_s, inp["ws2"], y_perm, y_s, ws),
+        lambda: B.moe_combine(cfg, y_perm, inv_row, gate, y_s, y2),
+    ]
+    for _ in range(2):
+        for c in calls:
+            c()
+    torch.cuda.synchronize()
+    n_stage = max(3, min(args.steps, 50))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(n_stage)]
+    for i in range(n_stage):
+        evs[i][0].record(stream)
+        for j, c in enumerate(calls):
+            c()
+            evs[i][j + 1].record(stream)
+    torch.cuda.synchronize()
+    stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(n_stage))
+                for j, n in enumerate(names)}
+    assert torch.equal(y2, y), "per-stage chain and moe_forward disagree"
+    work, touched = stage_work(cfg, counts.cpu())
+    peaks = measured_peaks()
+    dom = max(names, key=lambda n: stage_ms[n])
+    wd = work[dom]
+    t_dom = stage_ms[dom] / 1e3
+    hbm_time = wd["bytes"] / (peaks["hbm"] * 1e9)
+    tc_time = wd["flops"] / (peaks["tensor_sustained"] * 1e12)
+    if tc_time > hbm_time:
+        roof = {"bound": "tensor", "achieved": wd["flops"] / t_dom / 1e12, "peak": peaks["tensor_sustained"],
+                "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": wd["bytes"] / t_dom / 1e9, "peak": peaks["hbm"], "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = traffic_for(cfg.name, dom)
+    roof.update({"kernel": dom, "peak_source": peaks["source"], "algorithmic_bytes": wd["bytes"],
+                 "algorithmic_flops": wd["flops"], "kernel_ms": stage_ms[dom]})
+    expert_ms = stage_ms["gate_up"] + stage_ms["down"]
+    expert_flops = work["gate_up"]["flops"] + work["down"]["flops"]
+    expert_bytes = work["gate_up"]["bytes"] + work["down"]["bytes"]
+
+    # ---- end to end through the public call with host buffers ------------------
+    x_host = inp["x"].cpu().pin_memory()
+    y_host = torch.empty((T, d), dtype=cfg.torch_dtype).pin_memory()
+    x_dev = torch.empty_like(inp["x"])
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        B.moe_forward(cfg, x_dev, inp["w_router"], inp["bias"], inp["w1"], inp["w3"], inp["w2"],
+                      inp["ws1"], inp["ws3"], inp["ws2"], y, ws)
+        y_host.copy_(y, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = t.item()
+    barrier()
+
+    # ---- CPU oracle baseline (rank 0, one GPU only) --------------------------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n = min(CPU_SAMPLE_TOKENS.get(cfg.name, 16), T)
+        dt, threads = oracle_sample_time(cfg, inp, n, seed=7)
+        cpu = {"value": n / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n} seeded tokens of {cfg.name}: fp64 routing over all {E} experts and the "
+                         f"FFN of each selected and shared expert ({dt:.1f} s)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": {"workload": cfg.name, "T": T, "d": d, "E": E, "k": k, "f": cfg.f,
+                       "f_shared": cfg.f_shared, "gate": "sigmoid" if cfg.gate_mode else "softmax",
+                       "n_groups": cfg.n_groups, "topk_groups": cfg.topk_groups,
+                       "route_scale": cfg.route_scale, "parallelism": f"replicas x{world}",
+                       "cuda_graph": graph is not None,
+                       "l2": "inputs larger than L2: every step streams the touched expert weights "
+                             f"({(touched * 3 * cfg.f * d + 3 * cfg.f_shared * d) * cfg.elem_bytes / 1e9:.2f} GB)"},
+            "active_tflops": cfg.active_flops() * world / (ms_step / 1e3) / 1e12,
+            "experts_touched": touched,
+            "expert_gemm": {"ms": expert_ms, "tflops": expert_flops / (expert_ms / 1e3) / 1e12,
+                            "gbs": expert_bytes / (expert_ms / 1e3) / 1e9,
+                            "frac_tensor": expert_flops / (expert_ms / 1e3) / 1e12 / peaks["tensor_sustained"],
+                            "frac_hbm": expert_bytes / (expert_ms / 1e3) / 1e9 / peaks["hbm"]},
+            "stages_ms": stage_ms,
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": T * d * cfg.elem_bytes, "d2h_bytes_per_step": T * d * cfg.elem_bytes,
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": KERNELS_PER_FORWARD * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if graph is not None:
+        del graph
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

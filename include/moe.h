@@ -1,0 +1,259 @@
+/*
+ * moe.h - C ABI of the sparse Mixture-of-Experts FFN forward pass on B200.
+ *
+ * The block computed here (the forward pass, without the residual):
+ *
+ *   MoE(u_t) = sum_{s in shared} FFN_s(u_t) + sum_{i in TopK(t)} g_{i,t} FFN_i(u_t)
+ *   FFN(u)   = W2 (SiLU(W1 u) * W3 u)
+ *
+ * Sources, cited by page title and section:
+ *   [DS] "Sparse MoE FFN" DeepSeek-V3 study note, "How it works": eq. 12
+ *        (residual form; the module returns shared + routed without u_t),
+ *        the SwiGLU equation (W1, W3 in R^{f x d}, W2 in R^{d x f}), the
+ *        "Routing" paragraph (sigmoid affinities, top-K on s + b, 8 groups
+ *        keep 4 with group score = sum of top-2, gates = unbiased selected s
+ *        renormalised, times route_scale = 2.5) and "Packed forward
+ *        (official)" (flatten to (T, d); weights and indices (T, K_r);
+ *        per-expert gather, SwiGLU, scale, scatter-add; shared FFN over all T;
+ *        no token dropped).
+ *   [CS] "Mixture of Experts and Hybrid Architectures" cheat sheet, "The
+ *        router in code": route(hidden, W_router, top_k, bias) ->
+ *        (top_idx, gates); bias moves selection only; softmax over the chosen
+ *        original scores, which sums to 1.
+ *   [KB] "Mixture of experts and architecture families", "The router and
+ *        load balancing": moe_layer(x, router, experts, k) over x: [tokens, d].
+ *   [L2] "Lesson 2 - From the Dense FFN to a Layer of Experts", sections 2
+ *        and 4 (routed sum; shared experts with unit weight).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every data pointer is a DEVICE pointer to a row-major, contiguous array
+ *    owned by the caller. The library keeps no pointer after a call returns
+ *    and allocates no memory: scratch lives in the caller's workspace, sized
+ *    by moe_workspace_size().
+ *  - Activations, weights, x_perm, y_perm, y_shared, y and the workspace must
+ *    be 16-byte aligned; d and f (and f_shared) must be multiples of 8 for
+ *    bf16 and of 4 for fp32. Otherwise the call returns MOE_ERR_MISALIGNED.
+ *  - dtype selects the storage type of activations and weights (fp32 or
+ *    bf16). Router logits, bias, gates and every accumulation are fp32.
+ *  - stream is a cudaStream_t (NULL = the legacy default stream). Calls only
+ *    enqueue work: none synchronises the host, none copies device data to
+ *    the host, so a call may be captured in a CUDA graph.
+ *  - Arguments are validated before anything is enqueued. T = 0 is valid:
+ *    moe_route then only zeroes expert_counts and expert_offsets, and the
+ *    other entry points enqueue nothing.
+ *  - Every entry point that takes a workspace needs at least
+ *    moe_workspace_size(cfg) bytes of it, else MOE_ERR_WORKSPACE_TOO_SMALL.
+ *  - Calls on distinct workspaces are independent and thread-safe. No C++
+ *    exception crosses this interface.
+ *  - Device-side waits are bounded (about 2 s). A wait that runs out records
+ *    MOE_ERR_TIMEOUT in the workspace's error word and its kernel returns;
+ *    moe_get_device_error() reports it.
+ */
+#ifndef MOE_B200_H_
+#define MOE_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,        /* a size or mode outside the documented range */
+  MOE_ERR_MISALIGNED = 2,         /* a pointer or a row stride breaks the 16-byte rule */
+  MOE_ERR_UNSUPPORTED = 3,        /* valid, but beyond this build's limits (E, k, groups) */
+  MOE_ERR_WORKSPACE_TOO_SMALL = 4,
+  MOE_ERR_CUDA = 5,               /* a CUDA runtime call or launch failed */
+  MOE_ERR_TIMEOUT = 6             /* a device-side wait ran out (see moe_get_device_error) */
+} moe_status;
+
+typedef enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 } moe_dtype;
+
+typedef enum {
+  /* gates = route_scale * softmax of the selected RAW logits (max-subtracted) [CS] */
+  MOE_GATE_SOFTMAX = 0,
+  /* gates = route_scale * s_i / sum_selected s, s = sigmoid(logit)           [DS] */
+  MOE_GATE_SIGMOID = 1
+} moe_gate_mode;
+
+/* Shape and routing settings of one MoE FFN block. All fields are plain
+ * 32-bit values so that the struct has the same layout from any language. */
+typedef struct {
+  int32_t T;            /* tokens (rows of x)                                      */
+  int32_t d;            /* hidden width                                            */
+  int32_t E;            /* routed experts, 1..1024                                 */
+  int32_t k;            /* experts per token, 1..min(E, 32)                        */
+  int32_t f;            /* routed expert inner width (rows of W1, W3)              */
+  int32_t dtype;        /* moe_dtype                                               */
+  int32_t gate_mode;    /* moe_gate_mode                                           */
+  int32_t n_groups;     /* expert groups; 1 = no group limit. E % n_groups == 0,   */
+                        /* 1..32, and E / n_groups >= 2 when n_groups > 1          */
+  int32_t topk_groups;  /* groups kept per token, 1..n_groups, with                */
+                        /* topk_groups * E / n_groups >= k                         */
+  float route_scale;    /* > 0; multiplies the renormalised gates (1.0 = none)     */
+  int32_t f_shared;     /* shared-expert inner width; 0 = no shared expert         */
+} moe_config;
+
+/* Checks a configuration without touching any device. Returns MOE_OK,
+ * MOE_ERR_INVALID_ARG or MOE_ERR_UNSUPPORTED. Host-only. */
+MOE_API moe_status moe_check_config(const moe_config* cfg);
+
+/* Bytes of workspace that every entry point below accepts for cfg (the
+ * largest any of them needs; moe_forward needs all of it). 0 if cfg is not
+ * valid. Host-only. Worst case: T*k packed rows plus T shared rows. */
+MOE_API size_t moe_workspace_size(const moe_config* cfg);
+
+/*
+ * moe_route - the gate: router logits, affinities, biased (optionally
+ * group-limited) top-k, gates, and the packing offsets.  [DS] "Routing";
+ * [CS] "The router in code".
+ *
+ *   x            [T][d]     dtype     activations u_t
+ *   w_router     [E][d]     dtype     router rows e_i
+ *   bias         [E]        fp32      selection bias b_i, or NULL (= 0)
+ *   topk_idx     [T][k]     int32     OUT: selected experts, ascending id;
+ *                                     ties go to the lower expert / group index
+ *   topk_gate    [T][k]     fp32      OUT: gate of each selected expert, from
+ *                                     the unbiased affinity
+ *   expert_counts  [E]      int32     OUT: tokens per expert
+ *   expert_offsets [E+1]    int32     OUT: exclusive prefix sum of counts
+ *
+ * Selection: b'_e = s_e + bias_e, with s = sigmoid(logit) (MOE_GATE_SIGMOID)
+ * or s = logit (MOE_GATE_SOFTMAX). With n_groups > 1, group G = experts
+ * [G*E/n_groups, (G+1)*E/n_groups) scores the sum of its two largest b';
+ * only the topk_groups best groups stay eligible. Then the k largest
+ * eligible b' win.
+ */
+MOE_API moe_status moe_route(const moe_config* cfg, const void* x, const void* w_router,
+                     const float* bias, int32_t* topk_idx, float* topk_gate,
+                     int32_t* expert_counts, int32_t* expert_offsets,
+                     void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * moe_permute - gather token rows into expert-contiguous order.
+ * [DS] "Packed forward": for each expert, gather the tokens whose indices
+ * equal it; [KB] the per-expert mask loop.
+ *
+ *   x              [T][d]     dtype   activations
+ *   topk_idx       [T][k]     int32   from moe_route (each row: k distinct ids)
+ *   expert_offsets [E+1]      int32   from moe_route
+ *   x_perm         [T*k][d]   dtype   OUT: row offsets[e] + r holds the r-th
+ *                                     token (in token order) that chose e
+ *   perm_src       [T*k]      int32   OUT: source token of each packed row
+ *   inv_row        [T][k]     int32   OUT: packed row of (token, slot)
+ */
+MOE_API moe_status moe_permute(const moe_config* cfg, const void* x, const int32_t* topk_idx,
+                       const int32_t* expert_offsets, void* x_perm, int32_t* perm_src,
+                       int32_t* inv_row, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * moe_expert_swiglu - every expert's SwiGLU FFN over its packed rows, plus
+ * the shared expert over all T tokens.  [DS] SwiGLU equation and "Packed
+ * forward" (the shared FFN runs on all T tokens).
+ *
+ *   x_perm         [T*k][d]      dtype  packed activations (moe_permute)
+ *   expert_offsets [E+1]         int32  segment e = rows [off[e], off[e+1])
+ *   w1, w3         [E][f][d]     dtype  W1 (inside SiLU), W3 (multiplier)
+ *   w2             [E][d][f]     dtype  W2 (down projection)
+ *   x_shared       [T][d]        dtype  shared-expert input, NULL if f_shared == 0
+ *   ws1, ws3       [f_shared][d] dtype  shared W1, W3 (NULL if f_shared == 0)
+ *   ws2            [d][f_shared] dtype  shared W2     (NULL if f_shared == 0)
+ *   y_perm         [T*k][d]      dtype  OUT: FFN_e(row), gate NOT applied
+ *   y_shared       [T][d]        dtype  OUT: FFN_shared(x_t) (NULL if f_shared == 0)
+ *
+ * bf16 runs on tcgen05 tensor cores with fp32 accumulation; the SwiGLU
+ * intermediate is rounded to bf16 once. fp32 runs fp32 FMA throughout.
+ */
+MOE_API moe_status moe_expert_swiglu(const moe_config* cfg, const void* x_perm,
+                             const int32_t* expert_offsets, const void* w1, const void* w3,
+                             const void* w2, const void* x_shared, const void* ws1,
+                             const void* ws3, const void* ws2, void* y_perm, void* y_shared,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * moe_expert_gate_up - first half of moe_expert_swiglu: the SwiGLU inner
+ * activation of every segment.  [DS] SwiGLU equation, SiLU(W1 u) * W3 u.
+ *
+ *   x_perm, expert_offsets, w1, w3, x_shared, ws1, ws3   as in moe_expert_swiglu
+ *   h              [T*k][f]          dtype  OUT: SiLU(W1_e row) * (W3_e row)
+ *   h_shared       [T][f_shared]     dtype  OUT: same for the shared expert
+ *                                           (NULL if f_shared == 0)
+ *
+ * bf16: one persistent tcgen05 kernel; both products accumulate in TMEM in
+ * fp32, the epilogue applies SiLU and the product in fp32 and rounds once.
+ */
+MOE_API moe_status moe_expert_gate_up(const moe_config* cfg, const void* x_perm,
+                              const int32_t* expert_offsets, const void* w1, const void* w3,
+                              const void* x_shared, const void* ws1, const void* ws3, void* h,
+                              void* h_shared, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * moe_expert_down - second half of moe_expert_swiglu: the down projection
+ * W2 h of every segment.  [DS] SwiGLU equation, W2 in R^{d x f}.
+ *
+ *   h              [T*k][f]          dtype  from moe_expert_gate_up
+ *   expert_offsets [E+1]             int32
+ *   w2             [E][d][f]         dtype
+ *   h_shared       [T][f_shared]     dtype  (NULL if f_shared == 0)
+ *   ws2            [d][f_shared]     dtype  (NULL if f_shared == 0)
+ *   y_perm         [T*k][d]          dtype  OUT
+ *   y_shared       [T][d]            dtype  OUT (NULL if f_shared == 0)
+ */
+MOE_API moe_status moe_expert_down(const moe_config* cfg, const void* h,
+                           const int32_t* expert_offsets, const void* w2, const void* h_shared,
+                           const void* ws2, void* y_perm, void* y_shared, void* workspace,
+                           size_t ws_bytes, void* stream);
+
+/*
+ * moe_combine - gate-weighted sum of each token's k expert rows, plus the
+ * shared row.  [KB] out[rows] += w * expert(x[rows]); [DS] "Packed forward"
+ * (scale by the matching weights, scatter-add into a zero buffer, return y+z).
+ *
+ *   y[t] = sum_{j<k} topk_gate[t][j] * y_perm[inv_row[t][j]]  (+ y_shared[t])
+ *
+ * Summed in fp32 in slot order j = 0..k-1, then the shared row, then
+ * rounded once to dtype. y_shared may be NULL. y is [T][d] dtype.
+ */
+MOE_API moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t* inv_row,
+                       const float* topk_gate, const void* y_shared, void* y, void* stream);
+
+/*
+ * moe_forward - the whole block: route, permute, experts, combine.
+ * Inputs as above; y [T][d] dtype receives shared + routed (no residual,
+ * [DS] eq. 12). ws1/ws3/ws2 are NULL when f_shared == 0.
+ */
+MOE_API moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_router,
+                       const float* bias, const void* w1, const void* w3, const void* w2,
+                       const void* ws1, const void* ws3, const void* ws2, void* y,
+                       void* workspace, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, reads and clears the workspace's device error word.
+ * Returns MOE_OK, MOE_ERR_TIMEOUT (a bounded device wait ran out during an
+ * earlier call on this workspace) or MOE_ERR_CUDA. Every entry point that
+ * takes a workspace clears the word when it starts. */
+MOE_API moe_status moe_get_device_error(void* workspace, void* stream);
+
+/* Launches one kernel that waits on a barrier nothing ever arrives at,
+ * with a bound of timeout_ns nanoseconds, so that the bounded-wait path can
+ * be exercised without hanging or faulting the GPU. The kernel records
+ * MOE_ERR_TIMEOUT in the workspace's error word and returns. */
+MOE_API moe_status moe_selftest_wait_timeout(void* workspace, size_t ws_bytes, int64_t timeout_ns,
+                                     void* stream);
+
+/* Static description of a status code. Never NULL. */
+MOE_API const char* moe_status_string(moe_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H_ */

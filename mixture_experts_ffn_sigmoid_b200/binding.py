@@ -1,0 +1,231 @@
+"""ctypes binding of ``libmoe_b200.so`` (declared in ``include/moe.h``).
+
+Argument marshalling only: every function here checks shapes and dtypes of
+torch tensors, passes their device pointers and the current CUDA stream to
+the C entry point of the same name, and raises ``MoEError`` on a non-OK
+status. All compute runs in the library's CUDA kernels; there is no other
+path. If the library is missing or cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+from .inputs import MoEConfig
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_MISALIGNED = 2
+MOE_ERR_UNSUPPORTED = 3
+MOE_ERR_WORKSPACE_TOO_SMALL = 4
+MOE_ERR_CUDA = 5
+MOE_ERR_TIMEOUT = 6
+
+MOE_DTYPE_F32 = 0
+MOE_DTYPE_BF16 = 1
+
+EXPORTED = ("moe_check_config", "moe_workspace_size", "moe_route", "moe_permute",
+            "moe_expert_swiglu", "moe_expert_gate_up", "moe_expert_down", "moe_combine", "moe_forward", "moe_get_device_error",
+            "moe_selftest_wait_timeout", "moe_status_string")
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class CConfig(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("f", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("gate_mode", ctypes.c_int32), ("n_groups", ctypes.c_int32),
+                ("topk_groups", ctypes.c_int32), ("route_scale", ctypes.c_float),
+                ("f_shared", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """Load the CUDA library once; raise if it is not there."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                               "`python -m mixture_experts_ffn_sigmoid_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        vp, sz, i32p, f32p = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p
+        cfgp = ctypes.POINTER(CConfig)
+        sig = {
+            "moe_check_config": (ctypes.c_int, [cfgp]),
+            "moe_workspace_size": (sz, [cfgp]),
+            "moe_route": (ctypes.c_int, [cfgp, vp, vp, f32p, i32p, f32p, i32p, i32p, vp, sz, vp]),
+            "moe_permute": (ctypes.c_int, [cfgp, vp, i32p, i32p, vp, i32p, i32p, vp, sz, vp]),
+            "moe_expert_swiglu": (ctypes.c_int, [cfgp, vp, i32p, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                                 vp, sz, vp]),
+            "moe_expert_gate_up": (ctypes.c_int, [cfgp, vp, i32p, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+            "moe_expert_down": (ctypes.c_int, [cfgp, vp, i32p, vp, vp, vp, vp, vp, vp, sz, vp]),
+            "moe_combine": (ctypes.c_int, [cfgp, vp, i32p, f32p, vp, vp, vp]),
+            "moe_forward": (ctypes.c_int, [cfgp, vp, vp, f32p, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+            "moe_get_device_error": (ctypes.c_int, [vp, vp]),
+            "moe_selftest_wait_timeout": (ctypes.c_int, [vp, sz, ctypes.c_int64, vp]),
+            "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().moe_status_string(int(status)).decode()
+
+
+def make_config(cfg: MoEConfig, T: Optional[int] = None) -> CConfig:
+    return CConfig(T=cfg.T if T is None else T, d=cfg.d, E=cfg.E, k=cfg.k, f=cfg.f,
+                   dtype=MOE_DTYPE_F32 if cfg.dtype == "f32" else MOE_DTYPE_BF16,
+                   gate_mode=cfg.gate_mode, n_groups=cfg.n_groups, topk_groups=cfg.topk_groups,
+                   route_scale=cfg.route_scale, f_shared=cfg.f_shared)
+
+
+def _cfg(c) -> CConfig:
+    return c if isinstance(c, CConfig) else make_config(c)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(status: int, where: str):
+    if status != MOE_OK:
+        raise MoEError(status, where)
+
+
+def check_config(cfg) -> int:
+    return lib().moe_check_config(ctypes.byref(_cfg(cfg)))
+
+
+def workspace_size(cfg) -> int:
+    return lib().moe_workspace_size(ctypes.byref(_cfg(cfg)))
+
+
+def alloc_workspace(cfg, device="cuda") -> torch.Tensor:
+    n = workspace_size(cfg)
+    if n == 0:
+        raise MoEError(check_config(cfg) or MOE_ERR_INVALID_ARG, "moe_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def moe_route(cfg, x, w_router, bias, topk_idx, topk_gate, expert_counts, expert_offsets,
+              workspace, stream=None):
+    c = _cfg(cfg)
+    _check(lib().moe_route(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(topk_idx),
+                           _ptr(topk_gate), _ptr(expert_counts), _ptr(expert_offsets),
+                           _ptr(workspace), workspace.numel(), _stream(stream)), "moe_route")
+
+
+def moe_permute(cfg, x, topk_idx, expert_offsets, x_perm, perm_src, inv_row, workspace, stream=None):
+    c = _cfg(cfg)
+    _check(lib().moe_permute(ctypes.byref(c), _ptr(x), _ptr(topk_idx), _ptr(expert_offsets),
+                             _ptr(x_perm), _ptr(perm_src), _ptr(inv_row), _ptr(workspace),
+                             workspace.numel(), _stream(stream)), "moe_permute")
+
+
+def moe_expert_swiglu(cfg, x_perm, expert_offsets, w1, w3, w2, x_shared, ws1, ws3, ws2, y_perm,
+                      y_shared, workspace, stream=None):
+    c = _cfg(cfg)
+    _check(lib().moe_expert_swiglu(ctypes.byref(c), _ptr(x_perm), _ptr(expert_offsets), _ptr(w1),
+                                   _ptr(w3), _ptr(w2), _ptr(x_shared), _ptr(ws1), _ptr(ws3),
+                                   _ptr(ws2), _ptr(y_perm), _ptr(y_shared), _ptr(workspace),
+                                   workspace.numel(), _stream(stream)), "moe_expert_swiglu")
+
+
+def moe_expert_gate_up(cfg, x_perm, expert_offsets, w1, w3, x_shared, ws1, ws3, h, h_shared,
+                       workspace, stream=None):
+    c = _cfg(cfg)
+    _check(lib().moe_expert_gate_up(ctypes.byref(c), _ptr(x_perm), _ptr(expert_offsets), _ptr(w1),
+                                    _ptr(w3), _ptr(x_shared), _ptr(ws1), _ptr(ws3), _ptr(h),
+                                    _ptr(h_shared), _ptr(workspace), workspace.numel(),
+                                    _stream(stream)), "moe_expert_gate_up")
+
+
+def moe_expert_down(cfg, h, expert_offsets, w2, h_shared, ws2, y_perm, y_shared, workspace,
+                    stream=None):
+    c = _cfg(cfg)
+    _check(lib().moe_expert_down(ctypes.byref(c), _ptr(h), _ptr(expert_offsets), _ptr(w2),
+                                 _ptr(h_shared), _ptr(ws2), _ptr(y_perm), _ptr(y_shared),
+                                 _ptr(workspace), workspace.numel(), _stream(stream)),
+           "moe_expert_down")
+
+
+def moe_combine(cfg, y_perm, inv_row, topk_gate, y_shared, y, stream=None):
+    c = _cfg(cfg)
+    _check(lib().moe_combine(ctypes.byref(c), _ptr(y_perm), _ptr(inv_row), _ptr(topk_gate),
+                             _ptr(y_shared), _ptr(y), _stream(stream)), "moe_combine")
+
+
+def moe_forward(cfg, x, w_router, bias, w1, w3, w2, ws1, ws3, ws2, y, workspace, stream=None):
+    c = _cfg(cfg)
+    _check(lib().moe_forward(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w1),
+                             _ptr(w3), _ptr(w2), _ptr(ws1), _ptr(ws3), _ptr(ws2), _ptr(y),
+                             _ptr(workspace), workspace.numel(), _stream(stream)), "moe_forward")
+
+
+def moe_get_device_error(workspace, stream=None) -> int:
+    return lib().moe_get_device_error(_ptr(workspace), _stream(stream))
+
+
+def moe_selftest_wait_timeout(workspace, timeout_ns: int, stream=None):
+    _check(lib().moe_selftest_wait_timeout(_ptr(workspace), workspace.numel(), int(timeout_ns),
+                                           _stream(stream)), "moe_selftest_wait_timeout")
+
+
+class MoEBlock:
+    """Convenience wrapper holding one block's weights and workspace on the GPU.
+
+    ``forward(x)`` returns a new ``[T, d]`` tensor (shared + routed, no
+    residual) computed by ``moe_forward``.
+    """
+
+    def __init__(self, cfg: MoEConfig, weights: dict, device="cuda"):
+        self.cfg = cfg
+        self.w = weights
+        self.device = torch.device(device)
+        self._ws = {}
+
+    def workspace(self, T: int) -> torch.Tensor:
+        if T not in self._ws:
+            self._ws[T] = alloc_workspace(make_config(self.cfg, T), self.device)
+        return self._ws[T]
+
+    def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        T = x.shape[0]
+        if out is None:
+            out = torch.empty_like(x)
+        w = self.w
+        moe_forward(make_config(self.cfg, T), x, w["w_router"], w.get("bias"), w["w1"], w["w3"], w["w2"],
+                    w.get("ws1"), w.get("ws3"), w.get("ws2"), out, self.workspace(T), stream)
+        return out

@@ -1,0 +1,495 @@
+// C ABI of the MoE FFN forward pass: argument checks, workspace carving and
+// kernel enqueue. No entry point allocates, synchronises or copies to the
+// host (moe_get_device_error excepted, which exists to do exactly that).
+#include <math.h>
+#include <string.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+
+int device_sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  return n;
+}
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+struct Layout {
+  size_t err, logits, ccount, cbase, idx, gate, counts, offsets, inv_row, perm_src;
+  size_t x_perm, h, h_s, y_perm, y_s, total;
+};
+
+// Workspace regions, each 256-byte aligned. Sizes cover the worst case of
+// T*k packed rows plus T shared rows.
+Layout layout_of(const moe_config& c) {
+  Layout L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += (bytes + kAlign - 1) / kAlign * kAlign;
+    return o;
+  };
+  const size_t es = c.dtype == MOE_DTYPE_F32 ? 4 : 2;
+  const size_t T = (size_t)c.T, k = (size_t)c.k, E = (size_t)c.E, d = (size_t)c.d, f = (size_t)c.f;
+  const size_t fs = (size_t)c.f_shared;
+  const size_t nch = (T + kChunk - 1) / kChunk;
+  L.err = take(kAlign);
+  L.logits = take(T * E * 4);
+  L.ccount = take(nch * E * 4);
+  L.cbase = take(nch * E * 4);
+  L.idx = take(T * k * 4);
+  L.gate = take(T * k * 4);
+  L.counts = take(E * 4);
+  L.offsets = take((E + 1) * 4);
+  L.inv_row = take(T * k * 4);
+  L.perm_src = take(T * k * 4);
+  L.x_perm = take(T * k * d * es);
+  L.h = take(T * k * f * es);
+  L.h_s = take(T * fs * es);
+  L.y_perm = take(T * k * d * es);
+  L.y_s = take(fs > 0 ? T * d * es : 0);
+  L.total = off;
+  return L;
+}
+
+moe_status check_config(const moe_config* c) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->T < 0 || c->d <= 0 || c->E <= 0 || c->k <= 0 || c->f <= 0 || c->f_shared < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (c->dtype != MOE_DTYPE_F32 && c->dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+  if (c->gate_mode != MOE_GATE_SOFTMAX && c->gate_mode != MOE_GATE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (c->k > c->E) return MOE_ERR_INVALID_ARG;
+  if (!(c->route_scale > 0.0f) || !isfinite(c->route_scale)) return MOE_ERR_INVALID_ARG;
+  if (c->n_groups < 1 || c->topk_groups < 1 || c->topk_groups > c->n_groups) return MOE_ERR_INVALID_ARG;
+  if (c->E % c->n_groups != 0) return MOE_ERR_INVALID_ARG;
+  if (c->n_groups > 1 && c->E / c->n_groups < 2) return MOE_ERR_INVALID_ARG;
+  if ((long long)c->topk_groups * (c->E / c->n_groups) < c->k) return MOE_ERR_INVALID_ARG;
+  if (c->E > kMaxExperts || c->k > kMaxTopK || c->n_groups > kMaxGroups) return MOE_ERR_UNSUPPORTED;
+  const int v = c->dtype == MOE_DTYPE_F32 ? 4 : 8;
+  if (c->d % v || c->f % v || c->f_shared % v) return MOE_ERR_MISALIGNED;
+  // Row indices (packed rows, weight rows) travel as 32-bit TMA coordinates.
+  const long long lim = 0x7fffffffLL;
+  if ((long long)c->T * (c->k + 1) >= lim || (long long)c->E * c->f >= lim ||
+      (long long)c->E * c->d >= lim)
+    return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// A required pointer: NULL -> invalid, not 16-byte aligned -> misaligned.
+moe_status need(const void* p) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  return aligned16(p) ? MOE_OK : MOE_ERR_MISALIGNED;
+}
+moe_status need4(const void* p) {   // int32 / fp32 side arrays: 4-byte alignment
+  if (!p) return MOE_ERR_INVALID_ARG;
+  return (reinterpret_cast<uintptr_t>(p) & 3u) == 0 ? MOE_OK : MOE_ERR_MISALIGNED;
+}
+
+#define MOE_TRY(expr)                   \
+  do {                                  \
+    const moe_status _st = (expr);      \
+    if (_st != MOE_OK) return _st;      \
+  } while (0)
+#define MOE_CUDA(expr)                          \
+  do {                                          \
+    if ((expr) != cudaSuccess) return MOE_ERR_CUDA; \
+  } while (0)
+
+template <typename T>
+T* at(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(ws) + off); }
+
+moe_status check_ws(const moe_config& c, void* ws, size_t ws_bytes) {
+  MOE_TRY(need(ws));
+  if (ws_bytes < layout_of(c).total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  return MOE_OK;
+}
+
+// Router logits -> top-k, gates, chunk histograms -> counts, chunk bases, offsets.
+moe_status enqueue_route(const moe_config& c, const void* x, const void* w_router, const float* bias,
+                         int* idx, float* gate, int* counts, int* offsets, void* ws, cudaStream_t s) {
+  const Layout L = layout_of(c);
+  float* logits = at<float>(ws, L.logits);
+  const int num_sms = device_sm_count();
+  if (c.dtype == MOE_DTYPE_BF16) {
+    UmmaGemmParams g = {};
+    g.mode = kUmmaRouter;
+    g.n_routed = 0;
+    g.shared_rows = c.T;
+    g.m_rows_s = c.E;
+    g.K_s = c.d;
+    int bn = 256;
+    while (bn > 32 && (long long)ceil_div(c.E, 128) * ceil_div(c.T, bn) < num_sms) bn >>= 1;
+    g.bn_max = bn;
+    g.a_s = w_router;
+    g.b_s = x;
+    g.out_s = logits;
+    g.out_s_ld = c.E;
+    g.err = at<uint32_t>(ws, L.err);
+    g.timeout_ns = kDefaultTimeoutNs;
+    MOE_CUDA(launch_umma_gemm(g, num_sms, s));
+  } else {
+    SimtGemmParams g = {};
+    g.dual = 0;
+    g.n_routed = 0;
+    g.shared_rows = c.T;
+    g.a_s = x;
+    g.b1_s = w_router;
+    g.out_s = logits;
+    g.N_s = c.E;
+    g.K_s = c.d;
+    MOE_CUDA(launch_simt_gemm(c.dtype, 1, g, s));
+  }
+  RouteParams r;
+  r.T = c.T; r.E = c.E; r.k = c.k; r.gate_mode = c.gate_mode;
+  r.n_groups = c.n_groups; r.topk_groups = c.topk_groups; r.route_scale = c.route_scale;
+  r.logits = logits; r.bias = bias; r.topk_idx = idx; r.topk_gate = gate;
+  r.chunk_counts = at<int>(ws, L.ccount);
+  MOE_CUDA(launch_router_topk(r, s));
+  const int nch = ceil_div(c.T, kChunk);
+  MOE_CUDA(launch_chunk_scan(at<int>(ws, L.ccount), nch, c.E, at<int>(ws, L.cbase), counts, s));
+  MOE_CUDA(launch_offsets(counts, c.E, offsets, s));
+  return MOE_OK;
+}
+
+// SwiGLU inner activation of every segment: h = SiLU(x W1^T) * (x W3^T).
+moe_status enqueue_gate_up(const moe_config& c, const void* x_perm, const int* offsets, const void* w1,
+                           const void* w3, const void* x_sh, const void* ws1, const void* ws3, void* h,
+                           void* h_s, uint32_t* err, cudaStream_t s) {
+  const bool shared = c.f_shared > 0;
+  const int rows = c.T * c.k;
+  if (c.dtype == MOE_DTYPE_BF16) {
+    UmmaGemmParams g = {};
+    g.mode = kUmmaSwiGLU;
+    g.n_routed = c.E;
+    g.offsets = offsets;
+    g.m_rows = c.f;
+    g.K = c.d;
+    g.shared_rows = shared ? c.T : 0;
+    g.m_rows_s = c.f_shared;
+    g.K_s = c.d;
+    g.bn_max = 256;
+    g.a = w1; g.a3 = w3; g.b = x_perm;
+    g.a_rows_total = (long long)c.E * c.f;
+    g.b_rows_total = rows;
+    g.a_s = ws1; g.a3_s = ws3; g.b_s = x_sh;
+    g.out = h; g.out_ld = c.f;
+    g.out_s = h_s; g.out_s_ld = c.f_shared;
+    g.err = err;
+    g.timeout_ns = kDefaultTimeoutNs;
+    g.max_routed_rows = rows;
+    MOE_CUDA(launch_umma_gemm(g, device_sm_count(), s));
+  } else {
+    SimtGemmParams g = {};
+    g.dual = 1;
+    g.n_routed = c.E;
+    g.offsets = offsets;
+    g.a = x_perm; g.b1 = w1; g.b3 = w3; g.out = h;
+    g.N = c.f; g.K = c.d;
+    g.shared_rows = shared ? c.T : 0;
+    g.a_s = x_sh; g.b1_s = ws1; g.b3_s = ws3; g.out_s = h_s;
+    g.N_s = c.f_shared; g.K_s = c.d;
+    g.max_rows = rows;
+    MOE_CUDA(launch_simt_gemm(c.dtype, 0, g, s));
+  }
+  return MOE_OK;
+}
+
+// Down projection of every segment: y = h W2^T.
+moe_status enqueue_down(const moe_config& c, const void* h, const int* offsets, const void* w2,
+                        const void* h_s, const void* ws2, void* y_perm, void* y_sh, uint32_t* err,
+                        cudaStream_t s) {
+  const bool shared = c.f_shared > 0;
+  const int rows = c.T * c.k;
+  if (c.dtype == MOE_DTYPE_BF16) {
+    UmmaGemmParams q = {};
+    q.mode = kUmmaDown;
+    q.n_routed = c.E;
+    q.offsets = offsets;
+    q.m_rows = c.d;
+    q.K = c.f;
+    q.shared_rows = shared ? c.T : 0;
+    q.m_rows_s = c.d;
+    q.K_s = c.f_shared;
+    q.bn_max = 256;
+    q.a = w2; q.b = h;
+    q.a_rows_total = (long long)c.E * c.d;
+    q.b_rows_total = rows;
+    q.a_s = ws2; q.b_s = h_s;
+    q.out = y_perm; q.out_ld = c.d;
+    q.out_s = y_sh; q.out_s_ld = c.d;
+    q.err = err;
+    q.timeout_ns = kDefaultTimeoutNs;
+    q.max_routed_rows = rows;
+    MOE_CUDA(launch_umma_gemm(q, device_sm_count(), s));
+  } else {
+    SimtGemmParams q = {};
+    q.dual = 0;
+    q.n_routed = c.E;
+    q.offsets = offsets;
+    q.a = h; q.b1 = w2; q.out = y_perm;
+    q.N = c.d; q.K = c.f;
+    q.shared_rows = shared ? c.T : 0;
+    q.a_s = h_s; q.b1_s = ws2; q.out_s = y_sh;
+    q.N_s = c.d; q.K_s = c.f_shared;
+    q.max_rows = rows;
+    MOE_CUDA(launch_simt_gemm(c.dtype, 0, q, s));
+  }
+  return MOE_OK;
+}
+
+moe_status enqueue_experts(const moe_config& c, const void* x_perm, const int* offsets, const void* w1,
+                           const void* w3, const void* w2, const void* x_sh, const void* ws1,
+                           const void* ws3, const void* ws2, void* y_perm, void* y_sh, void* ws,
+                           cudaStream_t s) {
+  const Layout L = layout_of(c);
+  void* h = at<char>(ws, L.h);
+  void* h_s = at<char>(ws, L.h_s);
+  uint32_t* err = at<uint32_t>(ws, L.err);
+  MOE_TRY(enqueue_gate_up(c, x_perm, offsets, w1, w3, x_sh, ws1, ws3, h, h_s, err, s));
+  return enqueue_down(c, h, offsets, w2, h_s, ws2, y_perm, y_sh, err, s);
+}
+
+moe_status clear_error_word(void* ws, cudaStream_t s) {
+  MOE_CUDA(cudaMemsetAsync(at<char>(ws, 0), 0, kAlign, s));
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+moe_status moe_check_config(const moe_config* cfg) { return check_config(cfg); }
+
+size_t moe_workspace_size(const moe_config* cfg) {
+  if (check_config(cfg) != MOE_OK) return 0;
+  return layout_of(*cfg).total;
+}
+
+moe_status moe_route(const moe_config* cfg, const void* x, const void* w_router, const float* bias,
+                     int32_t* topk_idx, float* topk_gate, int32_t* expert_counts,
+                     int32_t* expert_offsets, void* workspace, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_config(cfg));
+  const moe_config& c = *cfg;
+  MOE_TRY(need4(expert_counts));
+  MOE_TRY(need4(expert_offsets));
+  MOE_TRY(check_ws(c, workspace, ws_bytes));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (c.T == 0) {
+    MOE_CUDA(cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * c.E, s));
+    MOE_CUDA(cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (c.E + 1), s));
+    return MOE_OK;
+  }
+  MOE_TRY(need(x));
+  MOE_TRY(need(w_router));
+  MOE_TRY(need4(topk_idx));
+  MOE_TRY(need4(topk_gate));
+  if (bias) MOE_TRY(need4(bias));
+  MOE_TRY(clear_error_word(workspace, s));
+  return enqueue_route(c, x, w_router, bias, topk_idx, topk_gate, expert_counts, expert_offsets,
+                       workspace, s);
+}
+
+moe_status moe_permute(const moe_config* cfg, const void* x, const int32_t* topk_idx,
+                       const int32_t* expert_offsets, void* x_perm, int32_t* perm_src,
+                       int32_t* inv_row, void* workspace, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_config(cfg));
+  const moe_config& c = *cfg;
+  MOE_TRY(check_ws(c, workspace, ws_bytes));
+  if (c.T == 0) return MOE_OK;
+  MOE_TRY(need(x));
+  MOE_TRY(need(x_perm));
+  MOE_TRY(need4(topk_idx));
+  MOE_TRY(need4(expert_offsets));
+  MOE_TRY(need4(perm_src));
+  MOE_TRY(need4(inv_row));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  MOE_TRY(clear_error_word(workspace, s));
+  const Layout L = layout_of(c);
+  const int nch = ceil_div(c.T, kChunk);
+  MOE_CUDA(launch_chunk_counts(topk_idx, c.T, c.k, c.E, at<int>(workspace, L.ccount), s));
+  MOE_CUDA(launch_chunk_scan(at<int>(workspace, L.ccount), nch, c.E, at<int>(workspace, L.cbase),
+                             at<int>(workspace, L.counts), s));
+  MOE_CUDA(launch_permute(c.dtype, x, topk_idx, expert_offsets, at<int>(workspace, L.cbase), c.T, c.d,
+                          c.E, c.k, x_perm, perm_src, inv_row, device_sm_count(), s));
+  return MOE_OK;
+}
+
+moe_status moe_expert_swiglu(const moe_config* cfg, const void* x_perm, const int32_t* expert_offsets,
+                             const void* w1, const void* w3, const void* w2, const void* x_shared,
+                             const void* ws1, const void* ws3, const void* ws2, void* y_perm,
+                             void* y_shared, void* workspace, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_config(cfg));
+  const moe_config& c = *cfg;
+  MOE_TRY(check_ws(c, workspace, ws_bytes));
+  if (c.T == 0) return MOE_OK;
+  MOE_TRY(need(x_perm));
+  MOE_TRY(need4(expert_offsets));
+  MOE_TRY(need(w1));
+  MOE_TRY(need(w3));
+  MOE_TRY(need(w2));
+  MOE_TRY(need(y_perm));
+  if (c.f_shared > 0) {
+    MOE_TRY(need(x_shared));
+    MOE_TRY(need(ws1));
+    MOE_TRY(need(ws3));
+    MOE_TRY(need(ws2));
+    MOE_TRY(need(y_shared));
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  MOE_TRY(clear_error_word(workspace, s));
+  return enqueue_experts(c, x_perm, expert_offsets, w1, w3, w2, x_shared, ws1, ws3, ws2, y_perm,
+                         y_shared, workspace, s);
+}
+
+moe_status moe_expert_gate_up(const moe_config* cfg, const void* x_perm, const int32_t* expert_offsets,
+                              const void* w1, const void* w3, const void* x_shared, const void* ws1,
+                              const void* ws3, void* h, void* h_shared, void* workspace,
+                              size_t ws_bytes, void* stream) {
+  MOE_TRY(check_config(cfg));
+  const moe_config& c = *cfg;
+  MOE_TRY(check_ws(c, workspace, ws_bytes));
+  if (c.T == 0) return MOE_OK;
+  MOE_TRY(need(x_perm));
+  MOE_TRY(need4(expert_offsets));
+  MOE_TRY(need(w1));
+  MOE_TRY(need(w3));
+  MOE_TRY(need(h));
+  if (c.f_shared > 0) {
+    MOE_TRY(need(x_shared));
+    MOE_TRY(need(ws1));
+    MOE_TRY(need(ws3));
+    MOE_TRY(need(h_shared));
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  MOE_TRY(clear_error_word(workspace, s));
+  return enqueue_gate_up(c, x_perm, expert_offsets, w1, w3, x_shared, ws1, ws3, h, h_shared,
+                         at<uint32_t>(workspace, 0), s);
+}
+
+moe_status moe_expert_down(const moe_config* cfg, const void* h, const int32_t* expert_offsets,
+                           const void* w2, const void* h_shared, const void* ws2, void* y_perm,
+                           void* y_shared, void* workspace, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_config(cfg));
+  const moe_config& c = *cfg;
+  MOE_TRY(check_ws(c, workspace, ws_bytes));
+  if (c.T == 0) return MOE_OK;
+  MOE_TRY(need(h));
+  MOE_TRY(need4(expert_offsets));
+  MOE_TRY(need(w2));
+  MOE_TRY(need(y_perm));
+  if (c.f_shared > 0) {
+    MOE_TRY(need(h_shared));
+    MOE_TRY(need(ws2));
+    MOE_TRY(need(y_shared));
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  MOE_TRY(clear_error_word(workspace, s));
+  return enqueue_down(c, h, expert_offsets, w2, h_shared, ws2, y_perm, y_shared,
+                      at<uint32_t>(workspace, 0), s);
+}
+
+moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t* inv_row,
+                       const float* topk_gate, const void* y_shared, void* y, void* stream) {
+  MOE_TRY(check_config(cfg));
+  const moe_config& c = *cfg;
+  if (c.T == 0) return MOE_OK;
+  MOE_TRY(need(y_perm));
+  MOE_TRY(need4(inv_row));
+  MOE_TRY(need4(topk_gate));
+  MOE_TRY(need(y));
+  if (y_shared) MOE_TRY(need(y_shared));
+  MOE_CUDA(launch_combine(c.dtype, y_perm, inv_row, topk_gate, y_shared, y, c.T, c.d, c.k,
+                          device_sm_count(), static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_router, const float* bias,
+                       const void* w1, const void* w3, const void* w2, const void* ws1,
+                       const void* ws3, const void* ws2, void* y, void* workspace, size_t ws_bytes,
+                       void* stream) {
+  MOE_TRY(check_config(cfg));
+  const moe_config& c = *cfg;
+  MOE_TRY(check_ws(c, workspace, ws_bytes));
+  if (c.T == 0) return MOE_OK;
+  MOE_TRY(need(x));
+  MOE_TRY(need(w_router));
+  if (bias) MOE_TRY(need4(bias));
+  MOE_TRY(need(w1));
+  MOE_TRY(need(w3));
+  MOE_TRY(need(w2));
+  MOE_TRY(need(y));
+  if (c.f_shared > 0) {
+    MOE_TRY(need(ws1));
+    MOE_TRY(need(ws3));
+    MOE_TRY(need(ws2));
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const Layout L = layout_of(c);
+  void* ws = workspace;
+  MOE_TRY(clear_error_word(ws, s));
+  int* idx = at<int>(ws, L.idx);
+  float* gate = at<float>(ws, L.gate);
+  int* offsets = at<int>(ws, L.offsets);
+  MOE_TRY(enqueue_route(c, x, w_router, bias, idx, gate, at<int>(ws, L.counts), offsets, ws, s));
+  MOE_CUDA(launch_permute(c.dtype, x, idx, offsets, at<int>(ws, L.cbase), c.T, c.d, c.E, c.k,
+                          at<char>(ws, L.x_perm), at<int>(ws, L.perm_src), at<int>(ws, L.inv_row),
+                          device_sm_count(), s));
+  const bool shared = c.f_shared > 0;
+  void* y_s = shared ? at<char>(ws, L.y_s) : nullptr;
+  MOE_TRY(enqueue_experts(c, at<char>(ws, L.x_perm), offsets, w1, w3, w2, shared ? x : nullptr, ws1,
+                          ws3, ws2, at<char>(ws, L.y_perm), y_s, ws, s));
+  MOE_CUDA(launch_combine(c.dtype, at<char>(ws, L.y_perm), at<int>(ws, L.inv_row), gate, y_s, y, c.T,
+                          c.d, c.k, device_sm_count(), s));
+  return MOE_OK;
+}
+
+moe_status moe_get_device_error(void* workspace, void* stream) {
+  MOE_TRY(need(workspace));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaMemset(workspace, 0, sizeof(word)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (word & kErrTimeoutWait) return MOE_ERR_TIMEOUT;
+  return MOE_OK;
+}
+
+moe_status moe_selftest_wait_timeout(void* workspace, size_t ws_bytes, int64_t timeout_ns,
+                                     void* stream) {
+  MOE_TRY(need(workspace));
+  if (ws_bytes < kAlign || timeout_ns <= 0) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  MOE_TRY(clear_error_word(workspace, s));
+  MOE_CUDA(launch_wait_timeout_selftest(static_cast<uint32_t*>(workspace), timeout_ns, s));
+  return MOE_OK;
+}
+
+const char* moe_status_string(moe_status status) {
+  switch (status) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_MISALIGNED: return "pointer or row stride not 16-byte aligned";
+    case MOE_ERR_UNSUPPORTED: return "configuration beyond this build's limits";
+    case MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA runtime error";
+    case MOE_ERR_TIMEOUT: return "a bounded device wait timed out";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

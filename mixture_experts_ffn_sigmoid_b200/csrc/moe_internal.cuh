@@ -1,0 +1,107 @@
+// Internal declarations shared by the kernels and the C-ABI layer.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+constexpr int kChunk = 32;            // tokens per routing chunk (one warp's worth)
+constexpr int kMaxExperts = 1024;
+constexpr int kMaxTopK = 32;
+constexpr int kMaxGroups = 32;
+constexpr long long kDefaultTimeoutNs = 2000000000LL;   // 2 s per device wait
+
+// Error word codes written by kernels (bit flags, OR-ed together).
+constexpr uint32_t kErrTimeoutWait = 1u << 0;
+constexpr uint32_t kErrBadIndex = 1u << 1;
+
+__host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+__host__ __device__ inline long long ceil_div_ll(long long a, long long b) { return (a + b - 1) / b; }
+
+template <typename T> struct Vec16;            // 16-byte vector of T
+template <> struct Vec16<float> { static constexpr int N = 4; };
+template <> struct Vec16<__nv_bfloat16> { static constexpr int N = 8; };
+
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+
+// ---------------------------------------------------------------- launchers
+// Routing (route_kernels.cu)
+struct RouteParams {
+  int T, E, k, gate_mode, n_groups, topk_groups;
+  float route_scale;
+  const float* logits;     // [T][E]
+  const float* bias;       // [E] or null
+  int* topk_idx;           // [T][k]
+  float* topk_gate;        // [T][k]
+  int* chunk_counts;       // [nchunks][E] or null
+};
+cudaError_t launch_router_topk(const RouteParams& p, cudaStream_t s);
+cudaError_t launch_chunk_counts(const int* topk_idx, int T, int k, int E, int* chunk_counts,
+                                cudaStream_t s);
+cudaError_t launch_chunk_scan(const int* chunk_counts, int nchunks, int E, int* chunk_base,
+                              int* counts, cudaStream_t s);
+cudaError_t launch_offsets(const int* counts, int E, int* offsets, cudaStream_t s);
+
+// Permute / combine (permute_kernels.cu)
+cudaError_t launch_permute(int dtype, const void* x, const int* topk_idx, const int* offsets,
+                           const int* chunk_base, int T, int d, int E, int k, void* x_perm,
+                           int* perm_src, int* inv_row, int num_sms, cudaStream_t s);
+cudaError_t launch_combine(int dtype, const void* y_perm, const int* inv_row, const float* gate,
+                           const void* y_shared, void* y, int T, int d, int k, int num_sms,
+                           cudaStream_t s);
+
+// SIMT grouped GEMM (simt_gemm.cu): fp32 experts and fp32 router logits.
+struct SimtGemmParams {
+  int dual;                 // 1: out = SiLU(A B1^T) * (A B3^T); 0: out = A B1^T
+  int n_routed;             // routed segments (E), 0 for a single dense segment
+  const int* offsets;       // [n_routed+1] packed-row offsets
+  const void* a;            // routed A rows [rows][K]
+  const void* b1;           // routed B1 [n_routed][N][K]
+  const void* b3;           // routed B3 (dual)
+  void* out;                // routed out [rows][N]
+  int N, K;
+  int shared_rows;          // rows of the dense (shared) segment, 0 = none
+  const void* a_s; const void* b1_s; const void* b3_s; void* out_s;
+  int N_s, K_s;
+  int max_rows;             // upper bound on routed rows (T*k) for the grid
+};
+cudaError_t launch_simt_gemm(int in_dtype, int out_f32, const SimtGemmParams& p, cudaStream_t s);
+
+// tcgen05 grouped GEMM (umma_gemm.cu)
+enum UmmaMode { kUmmaRouter = 0, kUmmaSwiGLU = 1, kUmmaDown = 2 };
+struct UmmaGemmParams {
+  int mode;
+  int n_routed;             // routed segments
+  const int* offsets;       // [n_routed+1]
+  int m_rows;               // weight rows per routed expert
+  int K;                    // reduction length of routed segments
+  int shared_rows;          // tokens of the dense segment (0 = none)
+  int m_rows_s;             // weight rows of the dense segment
+  int K_s;
+  int bn_max;               // token tile cap, multiple of 16, <= 256
+  // tensor sources (bf16, row-major)
+  const void* a; const void* a3; const void* b;        // routed: [n_routed*m_rows][K], ..., [rows][K]
+  long long a_rows_total, b_rows_total;
+  const void* a_s; const void* a3_s; const void* b_s;  // dense: [m_rows_s][K_s], ..., [shared_rows][K_s]
+  void* out; long long out_ld;                          // routed out [rows][out_ld]
+  void* out_s; long long out_s_ld;                      // dense out
+  uint32_t* err;
+  long long timeout_ns;
+  int max_routed_rows;      // upper bound on routed rows (T*k) for the grid
+};
+cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t s);
+cudaError_t launch_wait_timeout_selftest(uint32_t* err, long long timeout_ns, cudaStream_t s);
+
+int device_sm_count();
+
+}  // namespace moe

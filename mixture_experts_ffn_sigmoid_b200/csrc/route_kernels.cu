@@ -1,0 +1,259 @@
+// Routing kernels: biased, optionally group-limited top-k over router logits,
+// gates from the unbiased affinities, and the deterministic packing offsets.
+//
+// Sparse MoE FFN (DeepSeek-V3 note), "How it works", Routing paragraph:
+//   s = sigmoid(u . e_i); top-K on s + b (after group masking: 8 groups,
+//   keep 4, group score = sum of top-2); gates = unbiased selected s,
+//   renormalised over the winners, times route_scale.
+// MoE cheat sheet, "The router in code": bias moves selection only; softmax
+//   over the chosen raw scores (max-subtracted), which sums to 1.
+//
+// Layout: one warp per token, lane l holds experts l, l+32, l+64, ...; a
+// block of 32 warps is one chunk of 32 tokens, so the same block can also
+// emit the chunk's per-expert histogram (a bit mask per expert: bit w set
+// when token w of the chunk chose the expert). Histograms are exact and the
+// scan below gives every (token, expert) pair the packed row
+// offsets[e] + #{earlier tokens that chose e}: deterministic, atomic-free.
+#include <math.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+__device__ __forceinline__ float sigmoid_f32(float l) { return 1.0f / (1.0f + expf(-l)); }
+
+template <int NPL>
+__global__ void __launch_bounds__(1024, 1) router_topk_kernel(RouteParams p) {
+  __shared__ uint32_t s_mask[kMaxExperts];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x;
+  const int t = chunk * kChunk + warp;
+  const int E = p.E, k = p.k;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_mask[e] = 0u;
+  __syncthreads();
+
+  if (t < p.T) {                       // warp-uniform
+    const float* lrow = p.logits + (size_t)t * E;
+    float v[NPL];                      // biased selection score b' = s + bias
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      const int e = lane + 32 * i;
+      float b = -INFINITY;
+      if (e < E) {
+        const float l = lrow[e];
+        const float s = (p.gate_mode == MOE_GATE_SIGMOID) ? sigmoid_f32(l) : l;
+        b = s + (p.bias ? p.bias[e] : 0.0f);
+      }
+      v[i] = b;
+    }
+
+    if (p.n_groups > 1) {
+      // Group score = sum of the two largest b' of the group; lane G ends up
+      // holding group G's score.
+      const int gsz = E / p.n_groups;
+      float my_gscore = -INFINITY;
+      for (int G = 0; G < p.n_groups; ++G) {
+        float m1 = -INFINITY, m2 = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+          const int e = lane + 32 * i;
+          if (e < E && e / gsz == G) {
+            const float x = v[i];
+            if (x > m1) { m2 = m1; m1 = x; } else if (x > m2) { m2 = x; }
+          }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          const float o1 = __shfl_xor_sync(kFull, m1, off);
+          const float o2 = __shfl_xor_sync(kFull, m2, off);
+          const float hi = fmaxf(m1, o1);
+          const float lo = fmaxf(fminf(m1, o1), fmaxf(m2, o2));
+          m1 = hi;
+          m2 = lo;
+        }
+        if (lane == G) my_gscore = m1 + m2;
+      }
+      // Keep the topk_groups best groups; ties go to the lower group index.
+      int rank = 0;
+      for (int G = 0; G < p.n_groups; ++G) {
+        const float o = __shfl_sync(kFull, my_gscore, G);
+        if (o > my_gscore || (o == my_gscore && G < lane)) ++rank;
+      }
+      const unsigned kept = __ballot_sync(kFull, lane < p.n_groups && rank < p.topk_groups);
+#pragma unroll
+      for (int i = 0; i < NPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E && !((kept >> (e / gsz)) & 1u)) v[i] = -INFINITY;
+      }
+    }
+
+    // k rounds of a warp arg-max: largest b' first, equal b' to the lower id.
+    unsigned taken = 0u;
+    int my_e = -1;                     // lane j < k ends with the j-th winner
+    for (int r = 0; r < k; ++r) {
+      float bv = -INFINITY;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < NPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E && !((taken >> i) & 1u)) {
+          if (v[i] > bv || (v[i] == bv && e < be)) { bv = v[i]; be = e; }
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(kFull, bv, off);
+        const int oe = __shfl_xor_sync(kFull, be, off);
+        if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+      }
+      if ((be & 31) == lane) taken |= 1u << (be >> 5);
+      if (lane == r) my_e = be;
+    }
+
+    // Report winners in ascending expert id.
+    int pos = 0;
+    for (int j = 0; j < k; ++j) {
+      const int o = __shfl_sync(kFull, my_e, j);
+      if (o < my_e) ++pos;
+    }
+    // Gates from the UNBIASED value of each winner.
+    const bool act = lane < k;
+    const float l = act ? lrow[my_e] : 0.0f;
+    float num;
+    if (p.gate_mode == MOE_GATE_SIGMOID) {
+      num = act ? sigmoid_f32(l) : 0.0f;
+    } else {
+      float m = act ? l : -INFINITY;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
+      num = act ? expf(l - m) : 0.0f;
+    }
+    float sum = num;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(kFull, sum, off);
+    if (act) {
+      p.topk_idx[(size_t)t * k + pos] = my_e;
+      p.topk_gate[(size_t)t * k + pos] = p.route_scale * (num / sum);
+      atomicOr(&s_mask[my_e], 1u << warp);
+    }
+  }
+  if (p.chunk_counts) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+      p.chunk_counts[(size_t)chunk * E + e] = __popc(s_mask[e]);
+  }
+}
+
+// Per-chunk histograms from a caller-supplied topk_idx (used by the
+// stand-alone permute entry point). Out-of-range ids are skipped.
+__global__ void __launch_bounds__(256) chunk_count_kernel(const int* __restrict__ idx, int T, int k,
+                                                          int E, int* __restrict__ chunk_counts) {
+  __shared__ uint32_t s_mask[kMaxExperts];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_mask[e] = 0u;
+  __syncthreads();
+  const int t = blockIdx.x * kChunk + threadIdx.x;
+  if (threadIdx.x < kChunk && t < T) {
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(size_t)t * k + j];
+      if (e >= 0 && e < E) atomicOr(&s_mask[e], 1u << threadIdx.x);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    chunk_counts[(size_t)blockIdx.x * E + e] = __popc(s_mask[e]);
+}
+
+// Inclusive block scan of one int per thread (blockDim a multiple of 32, <= 1024).
+__device__ int block_inclusive_scan(int v, int* s_warp, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(kFull, v, off);
+    if (lane >= off) v += o;
+  }
+  if (lane == 31) s_warp[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < nwarps ? s_warp[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(kFull, w, off);
+      if (lane >= off) w += o;
+    }
+    if (lane < nwarps) s_warp[lane] = w;
+  }
+  __syncthreads();
+  const int before = warp > 0 ? s_warp[warp - 1] : 0;
+  *total = s_warp[nwarps - 1];
+  __syncthreads();
+  return v + before;
+}
+
+// One block per expert: exclusive scan of its per-chunk counts over chunks.
+__global__ void __launch_bounds__(256) chunk_scan_kernel(const int* __restrict__ cc, int nch, int E,
+                                                         int* __restrict__ base, int* __restrict__ counts) {
+  __shared__ int s_warp[32];
+  const int e = blockIdx.x;
+  int carry = 0;
+  for (int c0 = 0; c0 < nch; c0 += blockDim.x) {
+    const int c = c0 + threadIdx.x;
+    const int v = c < nch ? cc[(size_t)c * E + e] : 0;
+    int total;
+    const int incl = block_inclusive_scan(v, s_warp, &total);
+    if (c < nch) base[(size_t)c * E + e] = carry + incl - v;
+    carry += total;
+  }
+  if (threadIdx.x == 0) counts[e] = carry;
+}
+
+// Exclusive scan of counts over experts: offsets[0..E].
+__global__ void __launch_bounds__(1024) offsets_kernel(const int* __restrict__ counts, int E,
+                                                       int* __restrict__ offsets) {
+  __shared__ int s_warp[32];
+  const int e = threadIdx.x;
+  const int v = e < E ? counts[e] : 0;
+  int total;
+  const int incl = block_inclusive_scan(v, s_warp, &total);
+  if (e < E) offsets[e] = incl - v;
+  if (e == 0) offsets[E] = total;
+}
+
+}  // namespace
+
+cudaError_t launch_router_topk(const RouteParams& p, cudaStream_t s) {
+  if (p.T <= 0) return cudaSuccess;
+  const int nch = ceil_div(p.T, kChunk);
+  const int per_lane = ceil_div(p.E, 32);
+  dim3 grid(nch), block(1024);
+  if (per_lane <= 1) router_topk_kernel<1><<<grid, block, 0, s>>>(p);
+  else if (per_lane <= 2) router_topk_kernel<2><<<grid, block, 0, s>>>(p);
+  else if (per_lane <= 4) router_topk_kernel<4><<<grid, block, 0, s>>>(p);
+  else if (per_lane <= 8) router_topk_kernel<8><<<grid, block, 0, s>>>(p);
+  else if (per_lane <= 16) router_topk_kernel<16><<<grid, block, 0, s>>>(p);
+  else router_topk_kernel<32><<<grid, block, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_counts(const int* topk_idx, int T, int k, int E, int* chunk_counts,
+                                cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  chunk_count_kernel<<<ceil_div(T, kChunk), 256, 0, s>>>(topk_idx, T, k, E, chunk_counts);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_scan(const int* chunk_counts, int nchunks, int E, int* chunk_base,
+                              int* counts, cudaStream_t s) {
+  chunk_scan_kernel<<<E, 256, 0, s>>>(chunk_counts, nchunks, E, chunk_base, counts);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_offsets(const int* counts, int E, int* offsets, cudaStream_t s) {
+  const int threads = ceil_div(E, 32) * 32;
+  offsets_kernel<<<1, threads, 0, s>>>(counts, E, offsets);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,580 @@
+// Persistent grouped GEMM on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// What it computes (SwiGLU equation of the Sparse MoE FFN note, "How it
+// works": FFN(u) = W2 (SiLU(W1 u) * W3 u), W1, W3 in R^{f x d}, W2 in
+// R^{d x f}; the router linear of the "Routing" paragraph, u . e_i):
+//
+//   kUmmaSwiGLU: h[r][m]   = SiLU(sum_c W1_e[m][c] x[r][c]) * (sum_c W3_e[m][c] x[r][c])
+//   kUmmaDown:   y[r][m]   = sum_c W2_e[m][c] h[r][c]
+//   kUmmaRouter: l[t][e]   = sum_c Wr[e][c] x[t][c]          (fp32 out)
+//
+// for every packed row r of every segment. Segment e < n_routed is expert e
+// over packed rows [offsets[e], offsets[e+1]); segment n_routed is the dense
+// segment (shared expert over all T tokens, or the router over all tokens).
+//
+// Orientation ("swap AB"): the weight rows are the MMA's M side (128 per
+// tile) and the tokens are its N side (16..256 per tile, a multiple of 16).
+// A DeepSeek-V3 expert sees ~128 tokens, so putting tokens on N wastes at
+// most 15 columns per tile instead of padding every expert to 128 or 256
+// rows; a weight tile is read from HBM once per token tile.
+//
+// Roles (192 threads, one CTA per SM, persistent over a static tile list):
+//   warp 0 lane 0 : TMA producer, STAGES-deep ring of (A [, A3], B) tiles
+//   warp 1        : TMEM allocator; lane 0 issues tcgen05.mma (kind::f16,
+//                   bf16 x bf16 -> fp32 in TMEM) and tcgen05.commit
+//   warps 2..5    : epilogue; tcgen05.ld of their 32-lane quarter, SiLU*gate
+//                   in fp32, one rounding to the output type, masked stores
+// Shared-memory tiles use the 128-byte swizzle written by TMA and read by
+// the MMA through K-major SW128 descriptors (8-row atoms, 1024 B apart).
+// TMA loads past a segment's end read neighbouring rows or zero fill; such
+// columns (tokens) and rows (weights past m_rows) are never stored.
+//
+// Every wait is bounded; on expiry the CTA records kErrTimeoutWait in the
+// error word, raises a shared abort flag, drains its in-flight copies and
+// MMAs (again bounded), frees TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128;          // weight rows per tile (MMA M)
+constexpr int BK = 64;           // K per stage: one 128-byte swizzle row of bf16
+constexpr int UMMA_K = 16;       // K per tcgen05.mma for 16-bit inputs
+constexpr int BN_MAX = 256;      // token columns per tile (MMA N)
+constexpr int BOX_N = 32;        // token rows per TMA box
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN_MAX * BK * 2;
+constexpr int MAX_SEG = kMaxExperts + 1;
+constexpr int NUM_THREADS = 192;
+constexpr int TMEM_COLS = 512;
+
+template <bool DUAL>
+struct Cfg {
+  static constexpr int STAGES = DUAL ? 3 : 4;
+  static constexpr int A_PER_STAGE = DUAL ? 2 : 1;
+  static constexpr int STAGE_BYTES = A_PER_STAGE * A_BYTES + B_BYTES;
+  static constexpr int ACC_STAGES = DUAL ? 1 : 2;
+  static constexpr int TABLE_BYTES = 2 * (MAX_SEG + 1) * 4;
+  static constexpr int BAR_BYTES = (2 * STAGES + 2 * 2 + 1) * 8 + 16;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + TABLE_BYTES + BAR_BYTES;
+};
+
+// ------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait on an mbarrier phase. Returns false when the CTA is aborting
+// (if honour_abort) or when timeout_ns elapses; the latter raises the abort
+// flag and records the timeout in the error word.
+__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
+                                          uint32_t* err, long long timeout_ns, bool honour_abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0u) {
+      if (honour_abort && *abort_flag) return false;
+      if ((long long)(global_ns() - t0) > timeout_ns) {
+        *abort_flag = 1u;
+        if (err) atomicOr(err, kErrTimeoutWait);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm, int c0, int c1,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tmap_prefetch(const CUtensorMap* tm) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm)) : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t slot_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// D[tmem] (+)= A[smem] * B[smem]^T, M=128, N from the instruction descriptor.
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on `bar` once every tcgen05.mma issued so far by this thread completes.
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+// 32 lanes x 16 consecutive fp32 columns: thread i gets lane (base + i).
+// The load and its wait::ld sit in one asm statement, so no use of the
+// destination registers can be scheduled before the data has landed.
+#define MOE_R16(r) "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), \
+    "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),   \
+    "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+__device__ __forceinline__ void tmem_ld16_wait(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : MOE_R16(r)
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld16x2_wait(uint32_t ta, uint32_t tb, uint32_t (&ra)[16],
+                                                 uint32_t (&rb)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%32];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%33];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : MOE_R16(ra), MOE_R16(rb)
+      : "r"(ta), "r"(tb)
+      : "memory");
+}
+#undef MOE_R16
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row atoms
+// 1024 bytes apart (stride byte offset), descriptor version 1 (sm_100).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) |
+         ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
+// K-major, N >> 3 at bit 17, M >> 4 at bit 24.
+__device__ __forceinline__ uint32_t idesc_bf16_f32(int m, int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
+         ((uint32_t)(m >> 4) << 24);
+}
+
+// ------------------------------------------------------------ tile list
+struct Tile {
+  int seg, wt, tt;
+  int rows;      // tokens in the segment
+  int mrows;     // weight rows of the segment
+  int K;
+  int b_row0;    // first packed row (token) of the segment in the B tensor
+  bool dense;
+};
+
+__device__ __forceinline__ void seg_dims(const UmmaGemmParams& p, const int* s_off, int s, int& rows,
+                                         int& mrows) {
+  if (s < p.n_routed) {
+    rows = s_off[s + 1] - s_off[s];
+    mrows = p.m_rows;
+  } else {
+    rows = p.shared_rows;
+    mrows = p.m_rows_s;
+  }
+}
+
+__device__ __forceinline__ Tile decode_tile(const UmmaGemmParams& p, const int* s_off,
+                                            const int* s_start, int nseg, int tile) {
+  int lo = 0, hi = nseg - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_start[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
+  Tile t;
+  t.seg = lo;
+  seg_dims(p, s_off, lo, t.rows, t.mrows);
+  t.dense = lo >= p.n_routed;
+  t.K = t.dense ? p.K_s : p.K;
+  t.b_row0 = t.dense ? 0 : s_off[lo];
+  const int nwt = ceil_div(t.mrows, BM), ntt = ceil_div(t.rows, p.bn_max);
+  const int local = tile - s_start[lo];
+  if (t.rows <= t.mrows) {   // weights dominate: keep one weight tile's token tiles together
+    t.wt = local / ntt;
+    t.tt = local - t.wt * ntt;
+  } else {                   // tokens dominate: sweep the expert's weights per token tile
+    t.tt = local / nwt;
+    t.wt = local - t.tt * nwt;
+  }
+  return t;
+}
+
+template <bool DUAL>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA3,
+                     const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmAs,
+                     const __grid_constant__ CUtensorMap tmA3s, const __grid_constant__ CUtensorMap tmBs,
+                     const UmmaGemmParams p) {
+  using C = Cfg<DUAL>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* stage_base = smem;
+  int* s_start = reinterpret_cast<int*>(smem + C::STAGES * C::STAGE_BYTES);
+  int* s_off = s_start + (MAX_SEG + 1);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_off + (MAX_SEG + 1));
+  uint64_t* full_bar = bars;
+  uint64_t* empty_bar = bars + C::STAGES;
+  uint64_t* accf_bar = bars + 2 * C::STAGES;
+  uint64_t* acce_bar = accf_bar + 2;
+  uint64_t* drain_bar = acce_bar + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nseg = p.n_routed + (p.shared_rows > 0 ? 1 : 0);
+
+  for (int s = threadIdx.x; s <= p.n_routed; s += blockDim.x)
+    s_off[s] = p.n_routed > 0 ? p.offsets[s] : 0;
+  if (threadIdx.x == 64) {
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(smem_u32(&full_bar[i]), 1);
+      mbar_init(smem_u32(&empty_bar[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&accf_bar[i]), 1);
+      mbar_init(smem_u32(&acce_bar[i]), 4 * 32);
+    }
+    mbar_init(smem_u32(drain_bar), 1);
+    *abort_flag = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    tmap_prefetch(&tmA); tmap_prefetch(&tmB); tmap_prefetch(&tmAs); tmap_prefetch(&tmBs);
+    if (DUAL) { tmap_prefetch(&tmA3); tmap_prefetch(&tmA3s); }
+  }
+  __syncthreads();
+  // Tiles per segment -> exclusive prefix s_start[0..nseg] (warp 0).
+  if (warp == 0) {
+    const int per = ceil_div(nseg, 32);
+    const int s0 = min(nseg, lane * per), s1 = min(nseg, s0 + per);
+    int sum = 0;
+    for (int s = s0; s < s1; ++s) {
+      int rows, mrows;
+      seg_dims(p, s_off, s, rows, mrows);
+      sum += rows > 0 ? ceil_div(mrows, BM) * ceil_div(rows, p.bn_max) : 0;
+    }
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    int run = incl - sum;
+    for (int s = s0; s < s1; ++s) {
+      s_start[s] = run;
+      int rows, mrows;
+      seg_dims(p, s_off, s, rows, mrows);
+      run += rows > 0 ? ceil_div(mrows, BM) * ceil_div(rows, p.bn_max) : 0;
+    }
+    if (lane == 31) s_start[nseg] = incl;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total_tiles = s_start[nseg];
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    int stage = 0;
+    uint32_t phase = 0, armed = 0, armed_parity = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+      const Tile t = decode_tile(p, s_off, s_start, nseg, tile);
+      const CUtensorMap* mA = t.dense ? &tmAs : &tmA;
+      const CUtensorMap* mA3 = t.dense ? &tmA3s : &tmA3;
+      const CUtensorMap* mB = t.dense ? &tmBs : &tmB;
+      const int a_row = (t.dense ? 0 : t.seg * p.m_rows) + t.wt * BM;
+      const int b_row = t.b_row0 + t.tt * p.bn_max;
+      const int n_valid = min(p.bn_max, t.rows - t.tt * p.bn_max);
+      const int n_mma = (n_valid + 15) & ~15;
+      const int nbox = ceil_div(n_mma, BOX_N);
+      const uint32_t bytes = C::A_PER_STAGE * A_BYTES + nbox * BOX_N * BK * 2;
+      const int nk = ceil_div(t.K, BK);
+      bool ok = true;
+      for (int kb = 0; kb < nk; ++kb) {
+        if (!wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag, p.err, p.timeout_ns, true)) {
+          ok = false;
+          break;
+        }
+        const uint32_t fb = smem_u32(&full_bar[stage]);
+        mbar_expect_tx(fb, bytes);
+        uint8_t* sb = stage_base + stage * C::STAGE_BYTES;
+        tma_load_2d(smem_u32(sb), mA, kb * BK, a_row, fb);
+        if (DUAL) tma_load_2d(smem_u32(sb + A_BYTES), mA3, kb * BK, a_row, fb);
+        uint8_t* bb = sb + C::A_PER_STAGE * A_BYTES;
+        for (int bx = 0; bx < nbox; ++bx)
+          tma_load_2d(smem_u32(bb + bx * BOX_N * BK * 2), mB, kb * BK, b_row + bx * BOX_N, fb);
+        armed |= 1u << stage;
+        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+    }
+    // Let every copy this thread started land before the CTA can exit.
+    for (int s = 0; s < C::STAGES; ++s)
+      if ((armed >> s) & 1u)
+        wait_bounded(smem_u32(&full_bar[s]), (armed_parity >> s) & 1u, abort_flag, p.err,
+                     p.timeout_ns, false);
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    int stage = 0, acc = 0;
+    uint32_t phase = 0, acc_phase = 0;
+    bool issued = false;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+      const Tile t = decode_tile(p, s_off, s_start, nseg, tile);
+      const int n_valid = min(p.bn_max, t.rows - t.tt * p.bn_max);
+      const int n_mma = (n_valid + 15) & ~15;
+      const int nk = ceil_div(t.K, BK);
+      if (!wait_bounded(smem_u32(&acce_bar[acc]), acc_phase ^ 1u, abort_flag, p.err, p.timeout_ns, true))
+        break;
+      tc_fence_after();
+      const uint32_t idesc = idesc_bf16_f32(BM, n_mma);
+      const uint32_t d1 = tmem_base + (uint32_t)(acc * BN_MAX);
+      const uint32_t d3 = tmem_base + (uint32_t)BN_MAX;
+      bool ok = true;
+      for (int kb = 0; kb < nk; ++kb) {
+        if (!wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, p.err, p.timeout_ns, true)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sb = smem_u32(stage_base + stage * C::STAGE_BYTES);
+        const uint64_t a_desc = sw128_desc(sb);
+        const uint64_t a3_desc = sw128_desc(sb + A_BYTES);
+        const uint64_t b_desc = sw128_desc(sb + C::A_PER_STAGE * A_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+          const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+          const uint64_t koff = (uint64_t)((kk * UMMA_K * 2) >> 4);
+          umma_bf16(d1, a_desc + koff, b_desc + koff, idesc, accum);
+          if (DUAL) umma_bf16(d3, a3_desc + koff, b_desc + koff, idesc, accum);
+        }
+        issued = true;
+        umma_commit(smem_u32(&empty_bar[stage]));
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+      umma_commit(smem_u32(&accf_bar[acc]));
+      if (C::ACC_STAGES == 2) {
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      } else {
+        acc_phase ^= 1u;
+      }
+    }
+    if (issued) {   // every MMA this thread issued completes before TMEM is freed
+      umma_commit(smem_u32(drain_bar));
+      wait_bounded(smem_u32(drain_bar), 0u, abort_flag, p.err, p.timeout_ns, false);
+    }
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                  // TMEM lane quarter this warp may read
+    const int row = q * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+      const Tile t = decode_tile(p, s_off, s_start, nseg, tile);
+      const int n_valid = min(p.bn_max, t.rows - t.tt * p.bn_max);
+      const int n_mma = (n_valid + 15) & ~15;
+      if (!wait_bounded(smem_u32(&accf_bar[acc]), acc_phase, abort_flag, p.err, p.timeout_ns, true))
+        break;
+      tc_fence_after();
+      const int m = t.wt * BM + row;
+      const bool m_ok = m < t.mrows;
+      const long long ld = t.dense ? p.out_s_ld : p.out_ld;
+      void* out = t.dense ? p.out_s : p.out;
+      const long long r0 = (long long)t.b_row0 + (long long)t.tt * p.bn_max;
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MAX);
+      for (int c0 = 0; c0 < n_mma; c0 += 16) {
+        uint32_t r1[16], r3[16];
+        if (DUAL) tmem_ld16x2_wait(taddr + c0, taddr + BN_MAX + c0, r1, r3);
+        else tmem_ld16_wait(taddr + c0, r1);
+        if (m_ok) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int col = c0 + j;
+            if (col < n_valid) {
+              float v = __uint_as_float(r1[j]);
+              if (DUAL) v = (v / (1.0f + __expf(-v))) * __uint_as_float(r3[j]);
+              const long long o = (r0 + col) * ld + m;
+              if (p.mode == kUmmaRouter) reinterpret_cast<float*>(out)[o] = v;
+              else reinterpret_cast<__nv_bfloat16*>(out)[o] = __float2bfloat16_rn(v);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(&acce_bar[acc]));
+      if (C::ACC_STAGES == 2) {
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      } else {
+        acc_phase ^= 1u;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+__global__ void wait_timeout_selftest_kernel(uint32_t* err, long long timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0u;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // Nothing ever arrives on `bar`: phase 0 never completes, the wait runs out.
+  if (threadIdx.x == 0)
+    wait_bounded(smem_u32(&bar), 0u, &abort_flag, err, timeout_ns, false);
+  __syncthreads();
+}
+
+// ------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// bf16 [outer][inner] row-major, 128-byte swizzle, box = 64 x box_rows.
+bool make_tmap(CUtensorMap* tm, const void* base, long long inner, long long outer, int box_rows) {
+  auto fn = get_encode_fn();
+  if (!fn || outer <= 0 || inner <= 0) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+  cuuint64_t strides[1] = {(cuuint64_t)inner * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <bool DUAL>
+cudaError_t ensure_smem_attr() {
+  static int done_mask = 0;   // one bit per device ordinal (< 32)
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 32 && ((done_mask >> dev) & 1)) return cudaSuccess;
+  e = cudaFuncSetAttribute(umma_gemm_kernel<DUAL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           Cfg<DUAL>::SMEM_BYTES);
+  if (e == cudaSuccess && dev < 32) done_mask |= 1 << dev;
+  return e;
+}
+
+}  // namespace
+
+cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t s) {
+  const bool dual = p.mode == kUmmaSwiGLU;
+  const bool has_dense = p.shared_rows > 0;
+  if (p.n_routed == 0 && !has_dense) return cudaSuccess;
+  CUtensorMap tA, tA3, tB, tAs, tA3s, tBs;
+  if (has_dense) {
+    if (!make_tmap(&tAs, p.a_s, p.K_s, p.m_rows_s, BM)) return cudaErrorInvalidValue;
+    if (!make_tmap(&tBs, p.b_s, p.K_s, p.shared_rows, BOX_N)) return cudaErrorInvalidValue;
+    if (dual && !make_tmap(&tA3s, p.a3_s, p.K_s, p.m_rows_s, BM)) return cudaErrorInvalidValue;
+    if (!dual) tA3s = tAs;
+  }
+  if (p.n_routed > 0) {
+    if (!make_tmap(&tA, p.a, p.K, p.a_rows_total, BM)) return cudaErrorInvalidValue;
+    if (!make_tmap(&tB, p.b, p.K, p.b_rows_total, BOX_N)) return cudaErrorInvalidValue;
+    if (dual && !make_tmap(&tA3, p.a3, p.K, p.a_rows_total, BM)) return cudaErrorInvalidValue;
+    if (!dual) tA3 = tA;
+  } else {
+    tA = tAs; tA3 = tA3s; tB = tBs;
+  }
+  if (!has_dense) { tAs = tA; tA3s = tA3; tBs = tB; }
+
+  long long tiles = 0;
+  if (p.n_routed > 0)
+    tiles += (long long)ceil_div(p.m_rows, BM) * (ceil_div(p.max_routed_rows, p.bn_max) + p.n_routed);
+  if (has_dense) tiles += (long long)ceil_div(p.m_rows_s, BM) * ceil_div(p.shared_rows, p.bn_max);
+  const int grid = (int)(tiles < num_sms ? tiles : num_sms);
+  if (grid <= 0) return cudaSuccess;
+  cudaError_t e;
+  if (dual) {
+    if ((e = ensure_smem_attr<true>()) != cudaSuccess) return e;
+    umma_gemm_kernel<true><<<grid, NUM_THREADS, Cfg<true>::SMEM_BYTES, s>>>(tA, tA3, tB, tAs, tA3s, tBs, p);
+  } else {
+    if ((e = ensure_smem_attr<false>()) != cudaSuccess) return e;
+    umma_gemm_kernel<false><<<grid, NUM_THREADS, Cfg<false>::SMEM_BYTES, s>>>(tA, tA3, tB, tAs, tA3s, tBs, p);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wait_timeout_selftest(uint32_t* err, long long timeout_ns, cudaStream_t s) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, s>>>(err, timeout_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

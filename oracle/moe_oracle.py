@@ -57,7 +57,7 @@ GATE_SIGMOID = 1
 __all__ = [
     "GATE_SOFTMAX", "GATE_SIGMOID", "router_logits", "affinity", "biased_scores",
     "group_scores", "group_eligibility", "select_experts", "gate_values", "route",
-    "silu", "swiglu_ffn", "expert_outputs", "moe_forward", "moe_forward_dense_loop",
+    "silu", "swiglu_hidden", "swiglu_ffn", "expert_outputs", "moe_forward", "moe_forward_dense_loop",
     "expert_counts_offsets", "permutation_rows", "near_tie_tokens",
 ]
 
@@ -206,15 +206,21 @@ def silu(z) -> np.ndarray:
         return z / (1.0 + np.exp(-z))
 
 
+def swiglu_hidden(u, w1, w3) -> np.ndarray:
+    """The SwiGLU inner activation SiLU(W1 u) * W3 u, row-wise over u.
+
+    [DS] SwiGLU equation: W1, W3 in R^{f x d}. u: (n, d). Returns (n, f).
+    """
+    u = _f64(u)
+    return silu(u @ _f64(w1).T) * (u @ _f64(w3).T)
+
+
 def swiglu_ffn(u, w1, w3, w2) -> np.ndarray:
     """FFN(u) = W2 (SiLU(W1 u) * W3 u), row-wise over u.
 
-    [DS] SwiGLU equation: W1, W3 in R^{f x d}, W2 in R^{d x f}.
-    u: (n, d). Returns (n, d).
+    [DS] SwiGLU equation: W2 in R^{d x f}. u: (n, d). Returns (n, d).
     """
-    u = _f64(u)
-    h = silu(u @ _f64(w1).T) * (u @ _f64(w3).T)
-    return h @ _f64(w2).T
+    return swiglu_hidden(u, w1, w3) @ _f64(w2).T
 
 
 def expert_outputs(x, idx, gates, w1, w3, w2, ws1=None, ws3=None, ws2=None) -> np.ndarray:

@@ -289,6 +289,8 @@ def pin_single_expert_is_dense_swiglu():
     y = orc.moe_forward(x, rng.standard_normal((1, d)), None, w1, w3, w2, 1, orc.GATE_SOFTMAX)
     _close(y, _torch_swiglu(x, w1[0], w3[0], w2[0]), tol=1e-12)
     _close(orc.swiglu_ffn(x, w1[0], w3[0], w2[0]), _torch_swiglu(x, w1[0], w3[0], w2[0]), tol=1e-12)
+    # The inner activation alone: the down projection with W2 = I.
+    _close(orc.swiglu_hidden(x, w1[0], w3[0]), _torch_swiglu(x, w1[0], w3[0], np.eye(f)), tol=1e-12)
 
 
 def pin_shared_expert_added_no_residual():

@@ -1,0 +1,104 @@
+"""Edge and degenerate cases of the block on the GPU, each against the oracle:
+one token, a token count that leaves a ragged 32-token chunk, k = E (every
+expert fires, bias irrelevant), all tokens on one expert (all other experts
+empty), a single expert (a dense SwiGLU), group limits that keep one group,
+no tokens at all, and the bounded-wait error path."""
+import numpy as np
+import pytest
+import torch
+
+import oracle.moe_oracle as orc
+from mixture_experts_ffn_sigmoid_b200 import binding as B
+from mixture_experts_ffn_sigmoid_b200.inputs import GATE_SIGMOID, GATE_SOFTMAX, MoEConfig
+
+import gpu_harness as H
+
+pytestmark = pytest.mark.gpu
+
+EDGE = {
+    "one_token": MoEConfig("one_token", T=1, d=256, E=16, k=4, f=256, gate_mode=GATE_SIGMOID,
+                           route_scale=2.5, f_shared=128, bias="uniform"),
+    "ragged_chunk": MoEConfig("ragged_chunk", T=33, d=128, E=8, k=2, f=128),
+    "k_equals_E": MoEConfig("k_equals_E", T=40, d=128, E=4, k=4, f=64, gate_mode=GATE_SIGMOID,
+                            route_scale=2.5, bias="uniform"),
+    "single_expert": MoEConfig("single_expert", T=100, d=192, E=1, k=1, f=320),
+    "one_group_kept": MoEConfig("one_group_kept", T=96, d=128, E=64, k=6, f=128, gate_mode=GATE_SIGMOID,
+                                n_groups=8, topk_groups=1, route_scale=2.5, bias="uniform"),
+    "k1_fp32": MoEConfig("k1_fp32", T=50, d=64, E=5, k=1, f=48, dtype="f32"),
+    "many_experts": MoEConfig("many_experts", T=64, d=128, E=1024, k=32, f=64),
+}
+
+
+@pytest.mark.parametrize("name", sorted(EDGE))
+def test_edge_forward(name):
+    cfg = EDGE[name]
+    inp = H.gpu_inputs(cfg)
+    got = H.gpu_route(cfg, inp)
+    H.check_route(cfg, H.oracle_route(cfg, inp), got)
+    y = H.gpu_forward(cfg, inp)
+    H.check_forward(cfg, inp, y)
+
+
+def test_all_tokens_on_one_expert():
+    # A +10 bias on expert 3 with k = 1: expert 3 gets every token (a segment
+    # spanning several 256-token tiles), the other experts are empty.
+    cfg = MoEConfig("hot_expert", T=600, d=128, E=8, k=1, f=128, gate_mode=GATE_SIGMOID, route_scale=1.0,
+                    bias="uniform")
+    inp = H.gpu_inputs(cfg)
+    inp["bias"] = torch.zeros(8, device="cuda")
+    inp["bias"][3] = 10.0
+    got = H.gpu_route(cfg, inp)
+    counts = got["counts"].cpu().numpy()
+    assert counts[3] == 600 and counts.sum() == 600
+    H.check_route(cfg, H.oracle_route(cfg, inp), got)
+    y = H.gpu_forward(cfg, inp)
+    H.check_forward(cfg, inp, y)
+
+
+def test_zero_tokens():
+    cfg = MoEConfig("empty", T=0, d=128, E=8, k=2, f=128)
+    c = B.make_config(cfg)
+    ws = B.alloc_workspace(c)
+    counts = torch.full((8,), 5, dtype=torch.int32, device="cuda")
+    offsets = torch.full((9,), 5, dtype=torch.int32, device="cuda")
+    empty = torch.empty((0, 128), dtype=torch.bfloat16, device="cuda")
+    wr = torch.zeros((8, 128), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((0, 2), dtype=torch.int32, device="cuda")
+    gate = torch.empty((0, 2), dtype=torch.float32, device="cuda")
+    B.lib()
+    st = B.lib().moe_route(B.ctypes.byref(c), None, B._ptr(wr), None, None, None, B._ptr(counts),
+                           B._ptr(offsets), B._ptr(ws), ws.numel(), B._stream(None))
+    assert st == B.MOE_OK
+    torch.cuda.synchronize()
+    assert counts.sum().item() == 0 and offsets.sum().item() == 0
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    cfg = MoEConfig("after_timeout", T=64, d=128, E=8, k=2, f=128)
+    ws = B.alloc_workspace(cfg)
+    B.moe_selftest_wait_timeout(ws, 50_000_000)          # 50 ms bound, nothing ever arrives
+    assert B.moe_get_device_error(ws) == B.MOE_ERR_TIMEOUT
+    assert B.moe_get_device_error(ws) == B.MOE_OK         # the word was cleared
+    inp = H.gpu_inputs(cfg)
+    y = H.gpu_forward(cfg, inp, ws)                       # the context is still usable
+    H.check_forward(cfg, inp, y)
+
+
+def test_bad_indices_are_skipped_not_dereferenced():
+    # Out-of-range expert ids from a caller: the permute skips them and
+    # reports row -1 instead of writing out of bounds.
+    cfg = MoEConfig("bad_idx", T=32, d=128, E=8, k=2, f=128)
+    inp = H.gpu_inputs(cfg)
+    got = H.gpu_route(cfg, inp)
+    idx = got["idx"].clone()
+    idx[5, 1] = 99
+    idx[7, 0] = -3
+    rows = cfg.T * cfg.k
+    x_perm = torch.zeros((rows, cfg.d), dtype=cfg.torch_dtype, device="cuda")
+    perm_src = torch.full((rows,), -1, dtype=torch.int32, device="cuda")
+    inv_row = torch.zeros((cfg.T, cfg.k), dtype=torch.int32, device="cuda")
+    B.moe_permute(cfg, inp["x"], idx, got["offsets"], x_perm, perm_src, inv_row, got["ws"])
+    torch.cuda.synchronize()
+    inv = inv_row.cpu().numpy()
+    assert inv[5, 1] == -1 and inv[7, 0] == -1
+    assert inv.max() < rows

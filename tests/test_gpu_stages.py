@@ -1,0 +1,156 @@
+"""Per-stage parity on the GPU: route, permute, experts, combine, each called
+through the C ABI and compared with the CPU oracle on the same inputs.
+
+Shapes are small enough for the full oracle, yet span several tiles and a
+ragged tail: T not a multiple of the 32-token chunk, expert segments longer
+than one 256-token tile, hidden and inner widths that are not multiples of
+the 64-wide K step or the 128-row weight tile.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.moe_oracle as orc
+from mixture_experts_ffn_sigmoid_b200 import binding as B
+from mixture_experts_ffn_sigmoid_b200.inputs import CONFIGS, GATE_SIGMOID, GATE_SOFTMAX, MoEConfig
+
+import gpu_harness as H
+
+pytestmark = pytest.mark.gpu
+
+STAGE_CASES = {
+    "tiny_fp32": CONFIGS["tiny_fp32"],
+    "ds_like_small_bf16": MoEConfig("ds_like_small", T=300, d=256, E=32, k=4, f=384, gate_mode=GATE_SIGMOID,
+                                    n_groups=8, topk_groups=4, route_scale=2.5, f_shared=256, bias="uniform"),
+    "long_segments_bf16": MoEConfig("long_segments", T=700, d=320, E=4, k=2, f=136),
+    "ragged_dims_bf16": MoEConfig("ragged_dims", T=77, d=200, E=12, k=3, f=72, gate_mode=GATE_SIGMOID,
+                                  route_scale=1.0, f_shared=40, bias="uniform"),
+    "ragged_dims_fp32": MoEConfig("ragged_dims_f32", T=77, d=200, E=12, k=3, f=72, dtype="f32",
+                                  gate_mode=GATE_SIGMOID, f_shared=40, bias="uniform"),
+}
+
+
+@pytest.fixture(scope="module")
+def cases():
+    out = {}
+    for name, cfg in STAGE_CASES.items():
+        out[name] = (cfg, H.gpu_inputs(cfg))
+    return out
+
+
+@pytest.mark.parametrize("name", sorted(STAGE_CASES))
+def test_route(cases, name):
+    cfg, inp = cases[name]
+    got = H.gpu_route(cfg, inp)
+    rep = H.check_route(cfg, H.oracle_route(cfg, inp), got)
+    assert rep["near_ties"] <= max(1, cfg.T // 100)
+
+
+@pytest.mark.parametrize("name", sorted(STAGE_CASES))
+def test_permute(cases, name):
+    cfg, inp = cases[name]
+    got = H.gpu_route(cfg, inp)
+    rows = cfg.T * cfg.k
+    x_perm = torch.full((rows, cfg.d), float("nan"), dtype=cfg.torch_dtype, device="cuda")
+    perm_src = torch.full((rows,), -7, dtype=torch.int32, device="cuda")
+    inv_row = torch.full((cfg.T, cfg.k), -7, dtype=torch.int32, device="cuda")
+    B.moe_permute(cfg, inp["x"], got["idx"], got["offsets"], x_perm, perm_src, inv_row, got["ws"])
+    assert B.moe_get_device_error(got["ws"]) == B.MOE_OK
+    gi = got["idx"].cpu().numpy()
+    inv_ref, src_ref = orc.permutation_rows(gi, got["offsets"].cpu().numpy())
+    assert np.array_equal(inv_row.cpu().numpy(), inv_ref)
+    assert np.array_equal(perm_src.cpu().numpy(), src_ref)
+    # Copies are exact: packed row r is x[perm_src[r]] byte for byte.
+    assert torch.equal(x_perm, inp["x"][perm_src.long()])
+
+
+def _packed(cfg, inp):
+    got = H.gpu_route(cfg, inp)
+    rows = cfg.T * cfg.k
+    x_perm = torch.empty((rows, cfg.d), dtype=cfg.torch_dtype, device="cuda")
+    perm_src = torch.empty((rows,), dtype=torch.int32, device="cuda")
+    inv_row = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device="cuda")
+    B.moe_permute(cfg, inp["x"], got["idx"], got["offsets"], x_perm, perm_src, inv_row, got["ws"])
+    return got, x_perm, perm_src, inv_row
+
+
+@pytest.mark.parametrize("name", sorted(STAGE_CASES))
+def test_expert_swiglu(cases, name):
+    cfg, inp = cases[name]
+    got, x_perm, perm_src, inv_row = _packed(cfg, inp)
+    rows = cfg.T * cfg.k
+    y_perm = torch.full((rows, cfg.d), float("nan"), dtype=cfg.torch_dtype, device="cuda")
+    y_sh = torch.full((cfg.T, cfg.d), float("nan"), dtype=cfg.torch_dtype, device="cuda") \
+        if cfg.f_shared else None
+    B.moe_expert_swiglu(cfg, x_perm, got["offsets"], inp["w1"], inp["w3"], inp["w2"],
+                        inp["x"] if cfg.f_shared else None, inp["ws1"], inp["ws3"], inp["ws2"],
+                        y_perm, y_sh, got["ws"])
+    assert B.moe_get_device_error(got["ws"]) == B.MOE_OK
+    # Reference: FFN of the expert that owns each packed row, on that row.
+    offs = got["offsets"].cpu().numpy()
+    xp = H.f64(x_perm)
+    w1, w3, w2 = H.f64(inp["w1"]), H.f64(inp["w3"]), H.f64(inp["w2"])
+    ref = np.zeros((rows, cfg.d))
+    for e in range(cfg.E):
+        a, b = offs[e], offs[e + 1]
+        if b > a:
+            ref[a:b] = orc.swiglu_ffn(xp[a:b], w1[e], w3[e], w2[e])
+    H.compare_outputs(cfg, H.f64(y_perm), ref, "y_perm")
+    if cfg.f_shared:
+        ref_s = orc.swiglu_ffn(H.f64(inp["x"]), H.f64(inp["ws1"]), H.f64(inp["ws3"]), H.f64(inp["ws2"]))
+        H.compare_outputs(cfg, H.f64(y_sh), ref_s, "y_shared")
+
+
+@pytest.mark.parametrize("name", sorted(STAGE_CASES))
+def test_combine(cases, name):
+    cfg, inp = cases[name]
+    got, x_perm, perm_src, inv_row = _packed(cfg, inp)
+    rows = cfg.T * cfg.k
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5)
+    y_perm = torch.randn((rows, cfg.d), generator=g, device="cuda").to(cfg.torch_dtype)
+    y_sh = torch.randn((cfg.T, cfg.d), generator=g, device="cuda").to(cfg.torch_dtype) if cfg.f_shared else None
+    y = torch.full((cfg.T, cfg.d), float("nan"), dtype=cfg.torch_dtype, device="cuda")
+    B.moe_combine(cfg, y_perm, inv_row, got["gate"], y_sh, y)
+    torch.cuda.synchronize()
+    yp, inv, gate = H.f64(y_perm), inv_row.cpu().numpy(), got["gate"].cpu().numpy().astype(np.float64)
+    ref = np.zeros((cfg.T, cfg.d))
+    for j in range(cfg.k):
+        ref += gate[:, j:j + 1] * yp[inv[:, j]]
+    if cfg.f_shared:
+        ref += H.f64(y_sh)
+    # Only the final rounding to the storage type separates the two.
+    err = np.abs(H.f64(y) - ref)
+    bound = (2.0 ** -8 if cfg.dtype == "bf16" else 2.0 ** -22) * np.abs(ref) + 1e-6
+    assert np.all(err <= bound), float((err - bound).max())
+
+
+@pytest.mark.parametrize("name", sorted(STAGE_CASES))
+def test_forward_full_oracle(cases, name):
+    cfg, inp = cases[name]
+    y = H.gpu_forward(cfg, inp)
+    rep = H.check_forward(cfg, inp, y)
+    assert rep["compared"] >= cfg.T - max(1, cfg.T // 100)
+
+
+def test_forward_equals_stage_chain(cases):
+    # moe_forward and the four stage calls give the same bytes.
+    cfg, inp = cases["ds_like_small_bf16"]
+    y_fwd = H.gpu_forward(cfg, inp)
+    got, x_perm, perm_src, inv_row = _packed(cfg, inp)
+    rows = cfg.T * cfg.k
+    y_perm = torch.empty((rows, cfg.d), dtype=cfg.torch_dtype, device="cuda")
+    y_sh = torch.empty((cfg.T, cfg.d), dtype=cfg.torch_dtype, device="cuda")
+    B.moe_expert_swiglu(cfg, x_perm, got["offsets"], inp["w1"], inp["w3"], inp["w2"], inp["x"],
+                        inp["ws1"], inp["ws3"], inp["ws2"], y_perm, y_sh, got["ws"])
+    y = torch.empty_like(y_fwd)
+    B.moe_combine(cfg, y_perm, inv_row, got["gate"], y_sh, y)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_fwd)
+
+
+def test_forward_is_deterministic(cases):
+    cfg, inp = cases["ds_like_small_bf16"]
+    a = H.gpu_forward(cfg, inp)
+    b = H.gpu_forward(cfg, inp)
+    assert torch.equal(a, b)

@@ -28,6 +28,10 @@ def _swiglu_down_transposed(u, w1, w3, w2):
     return _orig["swiglu_ffn"](u, w1, w3, np.swapaxes(np.asarray(w2), -1, -2))
 
 
+def _hidden_swapped(u, w1, w3):
+    return _orig["swiglu_hidden"](u, w3, w1)
+
+
 def _silu_dropped_z(z):
     return 1.0 / (1.0 + np.exp(-np.asarray(z, np.float64)))
 
@@ -127,6 +131,7 @@ MUTATIONS = {
     "swiglu_no_silu": ("swiglu_ffn", _swiglu_no_silu),
     "swiglu_down_transposed": ("swiglu_ffn", _swiglu_down_transposed),
     "silu_drops_z": ("silu", _silu_dropped_z),
+    "hidden_w1_w3_swapped": ("swiglu_hidden", _hidden_swapped),
     "sigmoid_wrong_sign": ("affinity", _sigmoid_wrong_sign),
     "router_transposed": ("router_logits", _router_transposed),
     "gates_from_biased": ("route", _route_gates_use_biased),
