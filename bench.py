@@ -54,7 +54,18 @@ def parse_args():
     ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--T", type=int, default=None, help="override the token count (profiling cases)")
+    ap.add_argument("--E", type=int, default=None, help="override the routed expert count (profiling cases)")
     return ap.parse_args()
+
+
+def workload(args):
+    from mixture_experts_ffn_sigmoid_b200.inputs import CONFIGS
+    cfg = CONFIGS[args.config]
+    if args.T is not None or args.E is not None:
+        cfg = cfg.with_(T=args.T or cfg.T, E=args.E or cfg.E,
+                        name=f"{cfg.name}_T{args.T or cfg.T}_E{args.E or cfg.E}")
+    return cfg
 
 
 def measured_peaks():
@@ -131,7 +142,7 @@ class ClockSampler:
 
 # ------------------------------------------------------------ work accounting
 def stage_work(cfg, counts):
-    """Algorithmic bytes and flops of each stage (the design doc lists the formulas)."""
+    """Algorithmic bytes (compulsory HBM traffic) and flops of each stage for one forward."""
     es = cfg.elem_bytes
     T, d, E, k, f, fs = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.f_shared
     touched = int((counts > 0).sum())
@@ -210,12 +221,12 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    from mixture_experts_ffn_sigmoid_b200.inputs import CONFIGS, make_inputs
-    cfg = CONFIGS[args.config]
+    from mixture_experts_ffn_sigmoid_b200.inputs import make_inputs
+    cfg = workload(args)
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0"))) if torch.cuda.is_available() \
         else torch.device("cpu")
     inp = make_inputs(cfg, dev, seed=0)
-    n = min(REF_STEP_TOKENS.get(cfg.name, 4), cfg.T)
+    n = min(REF_STEP_TOKENS.get(args.config, 4), cfg.T)
     for i in range(args.warmup):
         oracle_sample_time(cfg, inp, n, seed=100 + i)
     times, threads = [], 1
@@ -245,7 +256,7 @@ def main():
         run_reference(args)
         return
     from mixture_experts_ffn_sigmoid_b200 import binding as B
-    from mixture_experts_ffn_sigmoid_b200.inputs import CONFIGS, make_inputs
+    from mixture_experts_ffn_sigmoid_b200.inputs import make_inputs
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -255,7 +266,7 @@ def main():
     if world > 1:
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
-    cfg = CONFIGS[args.config]
+    cfg = workload(args)
     B.lib()
     inp = make_inputs(cfg, dev, seed=0)
     if rank > 0:
@@ -404,7 +415,7 @@ def main():
     # ---- CPU oracle baseline (rank 0, one GPU only) --------------------------
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n = min(CPU_SAMPLE_TOKENS.get(cfg.name, 16), T)
+        n = min(CPU_SAMPLE_TOKENS.get(args.config, 16), T)
         dt, threads = oracle_sample_time(cfg, inp, n, seed=7)
         cpu = {"value": n / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                "sample": f"{n} seeded tokens of {cfg.name}: fp64 routing over all {E} experts and the "
