@@ -236,6 +236,34 @@ MOE_API moe_status moe_forward(const moe_config* cfg, const void* x, const void*
                        const void* ws1, const void* ws3, const void* ws2, void* y,
                        void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * moe_route_noalloc - moe_route for callers that cannot allocate device
+ * memory (no workspace argument). Same arguments and outputs as moe_route
+ * minus the workspace. The pages have no counterpart: this entry point only
+ * changes where the router's scratch lives.
+ *
+ * Some callers have no way to obtain device scratch when they route: code
+ * inside another runtime's allocation-free region, a plugin host that only
+ * hands over the tensors it owns, or a process that must not grow its device
+ * footprint mid-run. Here the scratch (router logits, per-chunk histograms
+ * and bases, error word) is one fixed 24 MiB array in the library's device
+ * image, present on every GPU that loads the library until the process
+ * exits; the call itself allocates nothing.
+ *  - Capacity: the call needs 256 + 4*T*E + 8*E*ceil(T/32) bytes (each term
+ *    rounded up to 256); beyond 24 MiB it returns MOE_ERR_WORKSPACE_TOO_SMALL
+ *    before enqueuing anything.
+ *  - The first call on each device looks up the array's device address
+ *    (with that device current) and caches it; make that first call before
+ *    any stream capture on the device.
+ *  - Every call on a device shares the one array and leaves its contents
+ *    behind; each call clears the error word first and overwrites the rest.
+ *    Calls whose work overlaps on the GPU (two streams, two threads) race on
+ *    the array and must be serialised by the caller.
+ */
+MOE_API moe_status moe_route_noalloc(const moe_config* cfg, const void* x, const void* w_router,
+                             const float* bias, int32_t* topk_idx, float* topk_gate,
+                             int32_t* expert_counts, int32_t* expert_offsets, void* stream);
+
 /* Synchronises `stream`, reads and clears the workspace's device error word.
  * Returns MOE_OK, MOE_ERR_TIMEOUT (a bounded device wait ran out during an
  * earlier call on this workspace) or MOE_ERR_CUDA. Every entry point that

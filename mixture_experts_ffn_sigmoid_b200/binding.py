@@ -31,7 +31,7 @@ MOE_DTYPE_BF16 = 1
 
 EXPORTED = ("moe_check_config", "moe_workspace_size", "moe_route", "moe_permute",
             "moe_expert_swiglu", "moe_expert_gate_up", "moe_expert_down", "moe_combine", "moe_forward", "moe_get_device_error",
-            "moe_selftest_wait_timeout", "moe_status_string")
+            "moe_selftest_wait_timeout", "moe_route_noalloc", "moe_status_string")
 
 
 class MoEError(RuntimeError):
@@ -78,6 +78,7 @@ def lib() -> ctypes.CDLL:
             "moe_forward": (ctypes.c_int, [cfgp, vp, vp, f32p, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
             "moe_get_device_error": (ctypes.c_int, [vp, vp]),
             "moe_selftest_wait_timeout": (ctypes.c_int, [vp, sz, ctypes.c_int64, vp]),
+            "moe_route_noalloc": (ctypes.c_int, [cfgp, vp, vp, f32p, i32p, f32p, i32p, i32p, vp]),
             "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         }
         for name, (res, args) in sig.items():
@@ -192,6 +193,15 @@ def moe_forward(cfg, x, w_router, bias, w1, w3, w2, ws1, ws3, ws2, y, workspace,
     _check(lib().moe_forward(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w1),
                              _ptr(w3), _ptr(w2), _ptr(ws1), _ptr(ws3), _ptr(ws2), _ptr(y),
                              _ptr(workspace), workspace.numel(), _stream(stream)), "moe_forward")
+
+
+def moe_route_noalloc(cfg, x, w_router, bias, topk_idx, topk_gate, expert_counts, expert_offsets,
+                      stream=None):
+    """moe_route with the router's scratch in the library's fixed device array."""
+    c = _cfg(cfg)
+    _check(lib().moe_route_noalloc(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(bias),
+                                   _ptr(topk_idx), _ptr(topk_gate), _ptr(expert_counts),
+                                   _ptr(expert_offsets), _stream(stream)), "moe_route_noalloc")
 
 
 def moe_get_device_error(workspace, stream=None) -> int:

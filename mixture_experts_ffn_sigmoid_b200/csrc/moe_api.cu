@@ -493,3 +493,73 @@ const char* moe_status_string(moe_status status) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Router without a caller workspace.
+//
+// Some callers cannot allocate device memory at the point where they route:
+// code running inside another framework's allocator-free region, a plugin
+// host that hands out only the tensors it owns, or a call made while the
+// process must not grow its device footprint. For them, moe_route_noalloc
+// keeps the router's scratch (logits, per-chunk histograms and bases, and the
+// error word) in one fixed array that lives in this library's device image.
+// The array is created with the library's module on every GPU that loads it
+// and stays until the process exits. Its host-side name is only a stand-in
+// for the symbol, never a device address: the address is looked up once per
+// device with cudaGetSymbolAddress while that device is current.
+// ---------------------------------------------------------------------------
+#include <atomic>
+
+namespace {
+constexpr size_t kRouteScratchBytes = size_t(24) << 20;   // 24 MiB per device
+constexpr int kMaxDevices = 64;
+std::atomic<void*> g_route_scratch_addr[kMaxDevices];
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_route_scratch[kRouteScratchBytes];
+
+namespace {
+// Device address of the scratch array on the current device (set-up on the
+// first call per device; needs no allocation).
+moe_status route_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+  void* p = g_route_scratch_addr[dev].load(std::memory_order_acquire);
+  if (!p) {
+    if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
+    g_route_scratch_addr[dev].store(p, std::memory_order_release);
+  }
+  *out = p;
+  return MOE_OK;
+}
+}  // namespace
+
+extern "C" moe_status moe_route_noalloc(const moe_config* cfg, const void* x, const void* w_router,
+                                        const float* bias, int32_t* topk_idx, float* topk_gate,
+                                        int32_t* expert_counts, int32_t* expert_offsets,
+                                        void* stream) {
+  MOE_TRY(check_config(cfg));
+  const moe_config& c = *cfg;
+  MOE_TRY(need4(expert_counts));
+  MOE_TRY(need4(expert_offsets));
+  // The router uses the leading regions of the workspace layout (error word,
+  // logits, chunk histograms, chunk bases); they must fit in the array.
+  if (layout_of(c).idx > kRouteScratchBytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (c.T == 0) {
+    MOE_CUDA(cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * c.E, s));
+    MOE_CUDA(cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (c.E + 1), s));
+    return MOE_OK;
+  }
+  MOE_TRY(need(x));
+  MOE_TRY(need(w_router));
+  MOE_TRY(need4(topk_idx));
+  MOE_TRY(need4(topk_gate));
+  if (bias) MOE_TRY(need4(bias));
+  void* scratch = nullptr;
+  MOE_TRY(route_scratch(&scratch));
+  MOE_TRY(clear_error_word(scratch, s));   // the only region that must start at zero
+  return enqueue_route(c, x, w_router, bias, topk_idx, topk_gate, expert_counts, expert_offsets,
+                       scratch, s);
+}
