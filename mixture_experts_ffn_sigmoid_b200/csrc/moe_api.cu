@@ -131,6 +131,7 @@ moe_status enqueue_route(const moe_config& c, const void* x, const void* w_route
     int bn = 256;
     while (bn > 32 && (long long)ceil_div(c.E, 128) * ceil_div(c.T, bn) < num_sms) bn >>= 1;
     g.bn_max = bn;
+    g.max_inflight = 3;
     g.a_s = w_router;
     g.b_s = x;
     g.out_s = logits;
@@ -162,6 +163,23 @@ moe_status enqueue_route(const moe_config& c, const void* x, const void* w_route
   return MOE_OK;
 }
 
+// Token-tile width of the expert GEMMs. Weight bytes dominate: every token
+// tile of an expert streams that expert's weights once more, so tiles are as
+// wide as the MMA allows (256) unless experts see only a handful of tokens
+// (decode), where a narrow tile leaves shared memory for deeper pipelining.
+// Slots in flight per CTA. With wide token tiles every slot also carries
+// L2-resident token rows, and measurements on B200 (DeepSeek-V3 shape) show
+// more than three outstanding weight slots slowing those loads down; narrow
+// tiles (decode) carry almost only weights and gain from a deeper queue.
+int inflight_for(int bn) { return bn >= 128 ? 3 : 8; }
+
+int expert_tile_n(const moe_config& c) {
+  const double m = (double)c.T * c.k / c.E;
+  int bn = (int)ceil(4.0 * m + 16.0);
+  bn = (bn + 31) / 32 * 32;
+  return bn < 32 ? 32 : (bn > 256 ? 256 : bn);
+}
+
 // SwiGLU inner activation of every segment: h = SiLU(x W1^T) * (x W3^T).
 moe_status enqueue_gate_up(const moe_config& c, const void* x_perm, const int* offsets, const void* w1,
                            const void* w3, const void* x_sh, const void* ws1, const void* ws3, void* h,
@@ -178,7 +196,8 @@ moe_status enqueue_gate_up(const moe_config& c, const void* x_perm, const int* o
     g.shared_rows = shared ? c.T : 0;
     g.m_rows_s = c.f_shared;
     g.K_s = c.d;
-    g.bn_max = 256;
+    g.bn_max = expert_tile_n(c);
+    g.max_inflight = inflight_for(g.bn_max);
     g.a = w1; g.a3 = w3; g.b = x_perm;
     g.a_rows_total = (long long)c.E * c.f;
     g.b_rows_total = rows;
@@ -221,7 +240,8 @@ moe_status enqueue_down(const moe_config& c, const void* h, const int* offsets, 
     q.shared_rows = shared ? c.T : 0;
     q.m_rows_s = c.d;
     q.K_s = c.f_shared;
-    q.bn_max = 256;
+    q.bn_max = expert_tile_n(c);
+    q.max_inflight = inflight_for(q.bn_max);
     q.a = w2; q.b = h;
     q.a_rows_total = (long long)c.E * c.d;
     q.b_rows_total = rows;

@@ -89,6 +89,7 @@ struct UmmaGemmParams {
   int m_rows_s;             // weight rows of the dense segment
   int K_s;
   int bn_max;               // token tile cap, multiple of 16, <= 256
+  int max_inflight;         // slots a CTA keeps loading at once (2..8)
   // tensor sources (bf16, row-major)
   const void* a; const void* a3; const void* b;        // routed: [n_routed*m_rows][K], ..., [rows][K]
   long long a_rows_total, b_rows_total;

@@ -4,30 +4,43 @@
 // works": FFN(u) = W2 (SiLU(W1 u) * W3 u), W1, W3 in R^{f x d}, W2 in
 // R^{d x f}; the router linear of the "Routing" paragraph, u . e_i):
 //
-//   kUmmaSwiGLU: h[r][m]   = SiLU(sum_c W1_e[m][c] x[r][c]) * (sum_c W3_e[m][c] x[r][c])
-//   kUmmaDown:   y[r][m]   = sum_c W2_e[m][c] h[r][c]
-//   kUmmaRouter: l[t][e]   = sum_c Wr[e][c] x[t][c]          (fp32 out)
+//   kUmmaSwiGLU: h[r][m] = SiLU(sum_c W1_e[m][c] x[r][c]) * (sum_c W3_e[m][c] x[r][c])
+//   kUmmaDown:   y[r][m] = sum_c W2_e[m][c] h[r][c]
+//   kUmmaRouter: l[t][e] = sum_c Wr[e][c] x[t][c]            (fp32 out)
 //
 // for every packed row r of every segment. Segment e < n_routed is expert e
 // over packed rows [offsets[e], offsets[e+1]); segment n_routed is the dense
-// segment (shared expert over all T tokens, or the router over all tokens).
+// segment (the shared expert over all T tokens, or the router over all tokens).
 //
-// Orientation ("swap AB"): the weight rows are the MMA's M side (128 per
-// tile) and the tokens are its N side (16..256 per tile, a multiple of 16).
-// A DeepSeek-V3 expert sees ~128 tokens, so putting tokens on N wastes at
-// most 15 columns per tile instead of padding every expert to 128 or 256
-// rows; a weight tile is read from HBM once per token tile.
+// Orientation ("swap AB"): weight rows are the MMA's M side (128 per MMA) and
+// tokens its N side (16..256 per tile, a multiple of 16). A DeepSeek-V3 expert
+// sees a few dozen to a few hundred tokens; putting tokens on N pads them to
+// 16, not to a 128-row M tile, and each weight tile is read from HBM once per
+// token tile. Each tile pairs two 128-row weight blocks with one token block
+// (SwiGLU: the W1 and W3 rows of the same f range; down: 256 consecutive W2
+// rows), so two MMAs share every token tile that is staged.
 //
 // Roles (192 threads, one CTA per SM, persistent over a static tile list):
-//   warp 0 lane 0 : TMA producer, STAGES-deep ring of (A [, A3], B) tiles
+//   warp 0 lane 0 : TMA producer into a ring of variable-size slots
 //   warp 1        : TMEM allocator; lane 0 issues tcgen05.mma (kind::f16,
 //                   bf16 x bf16 -> fp32 in TMEM) and tcgen05.commit
-//   warps 2..5    : epilogue; tcgen05.ld of their 32-lane quarter, SiLU*gate
+//   warps 2..5    : epilogue; tcgen05.ld of their 32-lane quarter, SiLU * up
 //                   in fp32, one rounding to the output type, masked stores
-// Shared-memory tiles use the 128-byte swizzle written by TMA and read by
-// the MMA through K-major SW128 descriptors (8-row atoms, 1024 B apart).
-// TMA loads past a segment's end read neighbouring rows or zero fill; such
-// columns (tokens) and rows (weights past m_rows) are never stored.
+//
+// The slot ring: a k-step needs (weights) + (its token rows, rounded to 32)
+// bytes, so slots are sized per tile and packed into one shared-memory ring
+// (wrapping to the start when the tail is too short), with at most
+// max_inflight slots loading or waiting at a time. Slot addresses depend
+// only on the sequence of slot sizes, so the producer and the MMA issuer
+// compute them independently; the producer reuses bytes only after the MMA
+// released (tcgen05.commit) every slot that overlaps them. Narrow token
+// tiles thus buy more weight bytes in flight, the quantity that bounds a
+// weight-streaming GEMM.
+//
+// Shared-memory tiles use the 128-byte swizzle written by TMA and read by the
+// MMA through K-major SW128 descriptors (8-row atoms 1024 B apart). TMA loads
+// past a segment's end read neighbouring rows or zero fill; such columns
+// (tokens) and rows (weights past m_rows) are never stored.
 //
 // Every wait is bounded; on expiry the CTA records kErrTimeoutWait in the
 // error word, raises a shared abort flag, drains its in-flight copies and
@@ -40,26 +53,47 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 128;          // weight rows per tile (MMA M)
-constexpr int BK = 64;           // K per stage: one 128-byte swizzle row of bf16
+constexpr int BM = 128;          // weight rows per MMA (M)
+constexpr int BK = 64;           // K per slot: one 128-byte swizzle row of bf16
 constexpr int UMMA_K = 16;       // K per tcgen05.mma for 16-bit inputs
-constexpr int BN_MAX = 256;      // token columns per tile (MMA N)
+constexpr int BN_MAX = 256;      // token columns per tile (MMA N), upper bound
 constexpr int BOX_N = 32;        // token rows per TMA box
 constexpr int A_BYTES = BM * BK * 2;
-constexpr int B_BYTES = BN_MAX * BK * 2;
-constexpr int MAX_SEG = kMaxExperts + 1;
+constexpr int BOX_BYTES = BOX_N * BK * 2;
 constexpr int NUM_THREADS = 192;
 constexpr int TMEM_COLS = 512;
+constexpr int NSLOT = 8;            // barrier pairs of the slot ring
+constexpr int SMEM_LIMIT = 232448;  // 227 KB of dynamic shared memory per block
 
-template <bool DUAL>
-struct Cfg {
-  static constexpr int STAGES = DUAL ? 3 : 4;
-  static constexpr int A_PER_STAGE = DUAL ? 2 : 1;
-  static constexpr int STAGE_BYTES = A_PER_STAGE * A_BYTES + B_BYTES;
-  static constexpr int ACC_STAGES = DUAL ? 1 : 2;
-  static constexpr int TABLE_BYTES = 2 * (MAX_SEG + 1) * 4;
-  static constexpr int BAR_BYTES = (2 * STAGES + 2 * 2 + 1) * 8 + 16;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + TABLE_BYTES + BAR_BYTES;
+// Shared-memory plan of one launch: [header page | tile tables | slot ring],
+// the ring 1024-byte aligned (128-byte swizzle atoms).
+struct SmemPlan {
+  int table_bytes, ring_bytes, total;
+};
+
+__host__ __device__ inline SmemPlan smem_plan(int n_routed, int nseg) {
+  SmemPlan sp;
+  sp.table_bytes = ((nseg + 1 + n_routed + 1) * 4 + 1023) / 1024 * 1024;
+  sp.ring_bytes = (SMEM_LIMIT - 1024 - 1024 - sp.table_bytes) / 1024 * 1024;
+  sp.total = 1024 + 1024 + sp.table_bytes + sp.ring_bytes;
+  return sp;
+}
+
+// Deterministic slot allocation shared by producer and MMA issuer.
+struct RingCursor {
+  uint32_t head = 0;    // next free byte (before wrap check)
+  uint32_t count = 0;   // slots allocated so far
+  __device__ __forceinline__ uint32_t peek(uint32_t size, uint32_t cap) const {
+    return head + size > cap ? 0u : head;
+  }
+  __device__ __forceinline__ void take(uint32_t size, uint32_t cap, uint32_t& off, uint32_t& slot,
+                                       uint32_t& parity) {
+    off = peek(size, cap);
+    head = off + size;
+    slot = count % NSLOT;
+    parity = (count / NSLOT) & 1u;
+    ++count;
+  }
 };
 
 // ------------------------------------------------------------ PTX wrappers
@@ -204,6 +238,11 @@ __device__ __forceinline__ uint32_t idesc_bf16_f32(int m, int n) {
 }
 
 // ------------------------------------------------------------ tile list
+template <int MODE> struct Kind;
+template <> struct Kind<kUmmaRouter> { static constexpr int A_TILES = 1; static constexpr int WROWS = 128; static constexpr int ACC_STAGES = 2; };
+template <> struct Kind<kUmmaSwiGLU> { static constexpr int A_TILES = 2; static constexpr int WROWS = 128; static constexpr int ACC_STAGES = 1; };
+template <> struct Kind<kUmmaDown>   { static constexpr int A_TILES = 2; static constexpr int WROWS = 256; static constexpr int ACC_STAGES = 1; };
+
 struct Tile {
   int seg, wt, tt;
   int rows;      // tokens in the segment
@@ -225,7 +264,7 @@ __device__ __forceinline__ void seg_dims(const UmmaGemmParams& p, const int* s_o
 }
 
 __device__ __forceinline__ Tile decode_tile(const UmmaGemmParams& p, const int* s_off,
-                                            const int* s_start, int nseg, int tile) {
+                                            const int* s_start, int nseg, int tile, int wrows) {
   int lo = 0, hi = nseg - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -237,7 +276,7 @@ __device__ __forceinline__ Tile decode_tile(const UmmaGemmParams& p, const int* 
   t.dense = lo >= p.n_routed;
   t.K = t.dense ? p.K_s : p.K;
   t.b_row0 = t.dense ? 0 : s_off[lo];
-  const int nwt = ceil_div(t.mrows, BM), ntt = ceil_div(t.rows, p.bn_max);
+  const int nwt = ceil_div(t.mrows, wrows), ntt = ceil_div(t.rows, p.bn_max);
   const int local = tile - s_start[lo];
   if (t.rows <= t.mrows) {   // weights dominate: keep one weight tile's token tiles together
     t.wt = local / ntt;
@@ -249,35 +288,42 @@ __device__ __forceinline__ Tile decode_tile(const UmmaGemmParams& p, const int* 
   return t;
 }
 
-template <bool DUAL>
+template <int MODE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA3,
                      const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmAs,
                      const __grid_constant__ CUtensorMap tmA3s, const __grid_constant__ CUtensorMap tmBs,
                      const UmmaGemmParams p) {
-  using C = Cfg<DUAL>;
+  using KD = Kind<MODE>;
+  constexpr int A_TILES = KD::A_TILES;
+  constexpr int WROWS = KD::WROWS;
+  constexpr int ACC_STAGES = KD::ACC_STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* stage_base = smem;
-  int* s_start = reinterpret_cast<int*>(smem + C::STAGES * C::STAGE_BYTES);
-  int* s_off = s_start + (MAX_SEG + 1);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(s_off + (MAX_SEG + 1));
+  const int nseg = p.n_routed + (p.shared_rows > 0 ? 1 : 0);
+  const SmemPlan sp = smem_plan(p.n_routed, nseg);
+  const uint32_t cap = (uint32_t)sp.ring_bytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
   uint64_t* full_bar = bars;
-  uint64_t* empty_bar = bars + C::STAGES;
-  uint64_t* accf_bar = bars + 2 * C::STAGES;
+  uint64_t* empty_bar = bars + NSLOT;
+  uint64_t* accf_bar = bars + 2 * NSLOT;
   uint64_t* acce_bar = accf_bar + 2;
   uint64_t* drain_bar = acce_bar + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
+  uint32_t* fl_off = tmem_slot + 2;             // producer's record of slots in flight
+  uint32_t* fl_size = fl_off + NSLOT;
+  int* s_start = reinterpret_cast<int*>(smem + 1024);
+  int* s_off = s_start + (nseg + 1);
+  uint8_t* ring = smem + 1024 + sp.table_bytes;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nseg = p.n_routed + (p.shared_rows > 0 ? 1 : 0);
 
   for (int s = threadIdx.x; s <= p.n_routed; s += blockDim.x)
     s_off[s] = p.n_routed > 0 ? p.offsets[s] : 0;
   if (threadIdx.x == 64) {
-    for (int i = 0; i < C::STAGES; ++i) {
+    for (int i = 0; i < NSLOT; ++i) {
       mbar_init(smem_u32(&full_bar[i]), 1);
       mbar_init(smem_u32(&empty_bar[i]), 1);
     }
@@ -295,7 +341,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
   if (threadIdx.x == 0) {
     tmap_prefetch(&tmA); tmap_prefetch(&tmB); tmap_prefetch(&tmAs); tmap_prefetch(&tmBs);
-    if (DUAL) { tmap_prefetch(&tmA3); tmap_prefetch(&tmA3s); }
+    if (MODE == kUmmaSwiGLU) { tmap_prefetch(&tmA3); tmap_prefetch(&tmA3s); }
   }
   __syncthreads();
   // Tiles per segment -> exclusive prefix s_start[0..nseg] (warp 0).
@@ -306,7 +352,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int s = s0; s < s1; ++s) {
       int rows, mrows;
       seg_dims(p, s_off, s, rows, mrows);
-      sum += rows > 0 ? ceil_div(mrows, BM) * ceil_div(rows, p.bn_max) : 0;
+      sum += rows > 0 ? ceil_div(mrows, WROWS) * ceil_div(rows, p.bn_max) : 0;
     }
     int incl = sum;
 #pragma unroll
@@ -319,7 +365,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       s_start[s] = run;
       int rows, mrows;
       seg_dims(p, s_off, s, rows, mrows);
-      run += rows > 0 ? ceil_div(mrows, BM) * ceil_div(rows, p.bn_max) : 0;
+      run += rows > 0 ? ceil_div(mrows, WROWS) * ceil_div(rows, p.bn_max) : 0;
     }
     if (lane == 31) s_start[nseg] = incl;
   }
@@ -331,54 +377,74 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
-    int stage = 0;
-    uint32_t phase = 0, armed = 0, armed_parity = 0;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-      const Tile t = decode_tile(p, s_off, s_start, nseg, tile);
+    RingCursor cur;
+    uint32_t inflight = 0;
+    const uint32_t max_inflight = (uint32_t)min(max(p.max_inflight, 2), NSLOT);
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+      const Tile t = decode_tile(p, s_off, s_start, nseg, tile, WROWS);
       const CUtensorMap* mA = t.dense ? &tmAs : &tmA;
       const CUtensorMap* mA3 = t.dense ? &tmA3s : &tmA3;
       const CUtensorMap* mB = t.dense ? &tmBs : &tmB;
-      const int a_row = (t.dense ? 0 : t.seg * p.m_rows) + t.wt * BM;
+      const int a_row = (t.dense ? 0 : t.seg * p.m_rows) + t.wt * WROWS;
       const int b_row = t.b_row0 + t.tt * p.bn_max;
       const int n_valid = min(p.bn_max, t.rows - t.tt * p.bn_max);
-      const int n_mma = (n_valid + 15) & ~15;
-      const int nbox = ceil_div(n_mma, BOX_N);
-      const uint32_t bytes = C::A_PER_STAGE * A_BYTES + nbox * BOX_N * BK * 2;
+      const int nbox = (n_valid + BOX_N - 1) / BOX_N;
+      const uint32_t bytes = A_TILES * A_BYTES + nbox * BOX_BYTES;
       const int nk = ceil_div(t.K, BK);
-      bool ok = true;
       for (int kb = 0; kb < nk; ++kb) {
-        if (!wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag, p.err, p.timeout_ns, true)) {
-          ok = false;
-          break;
+        // Make room: the barrier pair and the bytes of the new slot must be free.
+        const uint32_t off_new = cur.peek(bytes, cap);
+        while (true) {
+          bool clash = inflight >= max_inflight;
+          for (uint32_t i = 0; i < inflight && !clash; ++i) {
+            const uint32_t j = (cur.count - inflight + i) % NSLOT;
+            clash = off_new < fl_off[j] + fl_size[j] && fl_off[j] < off_new + bytes;
+          }
+          if (!clash) break;
+          const uint32_t oldest = cur.count - inflight;
+          if (!wait_bounded(smem_u32(&empty_bar[oldest % NSLOT]), (oldest / NSLOT) & 1u, abort_flag,
+                            p.err, p.timeout_ns, true)) {
+            ok = false;
+            break;
+          }
+          --inflight;
         }
-        const uint32_t fb = smem_u32(&full_bar[stage]);
+        if (!ok) break;
+        uint32_t off, slot, parity;
+        cur.take(bytes, cap, off, slot, parity);
+        fl_off[slot] = off;
+        fl_size[slot] = bytes;
+        ++inflight;
+        const uint32_t fb = smem_u32(&full_bar[slot]);
         mbar_expect_tx(fb, bytes);
-        uint8_t* sb = stage_base + stage * C::STAGE_BYTES;
-        tma_load_2d(smem_u32(sb), mA, kb * BK, a_row, fb);
-        if (DUAL) tma_load_2d(smem_u32(sb + A_BYTES), mA3, kb * BK, a_row, fb);
-        uint8_t* bb = sb + C::A_PER_STAGE * A_BYTES;
+        const uint32_t sb = smem_u32(ring + off);
+        tma_load_2d(sb, mA, kb * BK, a_row, fb);
+        if (MODE == kUmmaSwiGLU) tma_load_2d(sb + A_BYTES, mA3, kb * BK, a_row, fb);
+        if (MODE == kUmmaDown) tma_load_2d(sb + A_BYTES, mA, kb * BK, a_row + BM, fb);
+        const uint32_t bb = sb + A_TILES * A_BYTES;
         for (int bx = 0; bx < nbox; ++bx)
-          tma_load_2d(smem_u32(bb + bx * BOX_N * BK * 2), mB, kb * BK, b_row + bx * BOX_N, fb);
-        armed |= 1u << stage;
-        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+          tma_load_2d(bb + bx * BOX_BYTES, mB, kb * BK, b_row + bx * BOX_N, fb);
       }
-      if (!ok) break;
     }
     // Let every copy this thread started land before the CTA can exit.
-    for (int s = 0; s < C::STAGES; ++s)
-      if ((armed >> s) & 1u)
-        wait_bounded(smem_u32(&full_bar[s]), (armed_parity >> s) & 1u, abort_flag, p.err,
-                     p.timeout_ns, false);
+    for (uint32_t i = 0; i < inflight; ++i) {
+      const uint32_t u = cur.count - inflight + i;
+      wait_bounded(smem_u32(&full_bar[u % NSLOT]), (u / NSLOT) & 1u, abort_flag, p.err, p.timeout_ns,
+                   false);
+    }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
-    int stage = 0, acc = 0;
-    uint32_t phase = 0, acc_phase = 0;
+    RingCursor cur;
+    int acc = 0;
+    uint32_t acc_phase = 0;
     bool issued = false;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-      const Tile t = decode_tile(p, s_off, s_start, nseg, tile);
+      const Tile t = decode_tile(p, s_off, s_start, nseg, tile, WROWS);
       const int n_valid = min(p.bn_max, t.rows - t.tt * p.bn_max);
       const int n_mma = (n_valid + 15) & ~15;
+      const int nbox = (n_valid + BOX_N - 1) / BOX_N;
+      const uint32_t bytes = A_TILES * A_BYTES + nbox * BOX_BYTES;
       const int nk = ceil_div(t.K, BK);
       if (!wait_bounded(smem_u32(&acce_bar[acc]), acc_phase ^ 1u, abort_flag, p.err, p.timeout_ns, true))
         break;
@@ -388,29 +454,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t d3 = tmem_base + (uint32_t)BN_MAX;
       bool ok = true;
       for (int kb = 0; kb < nk; ++kb) {
-        if (!wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, p.err, p.timeout_ns, true)) {
+        uint32_t off, slot, parity;
+        cur.take(bytes, cap, off, slot, parity);
+        if (!wait_bounded(smem_u32(&full_bar[slot]), parity, abort_flag, p.err, p.timeout_ns, true)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t sb = smem_u32(stage_base + stage * C::STAGE_BYTES);
+        const uint32_t sb = smem_u32(ring + off);
         const uint64_t a_desc = sw128_desc(sb);
         const uint64_t a3_desc = sw128_desc(sb + A_BYTES);
-        const uint64_t b_desc = sw128_desc(sb + C::A_PER_STAGE * A_BYTES);
+        const uint64_t b_desc = sw128_desc(sb + A_TILES * A_BYTES);
 #pragma unroll
         for (int kk = 0; kk < BK / UMMA_K; ++kk) {
           const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
           const uint64_t koff = (uint64_t)((kk * UMMA_K * 2) >> 4);
           umma_bf16(d1, a_desc + koff, b_desc + koff, idesc, accum);
-          if (DUAL) umma_bf16(d3, a3_desc + koff, b_desc + koff, idesc, accum);
+          if (A_TILES == 2) umma_bf16(d3, a3_desc + koff, b_desc + koff, idesc, accum);
         }
         issued = true;
-        umma_commit(smem_u32(&empty_bar[stage]));
-        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        umma_commit(smem_u32(&empty_bar[slot]));
       }
       if (!ok) break;
       umma_commit(smem_u32(&accf_bar[acc]));
-      if (C::ACC_STAGES == 2) {
+      if (ACC_STAGES == 2) {
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       } else {
@@ -428,39 +495,89 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-      const Tile t = decode_tile(p, s_off, s_start, nseg, tile);
+      const Tile t = decode_tile(p, s_off, s_start, nseg, tile, WROWS);
       const int n_valid = min(p.bn_max, t.rows - t.tt * p.bn_max);
       const int n_mma = (n_valid + 15) & ~15;
       if (!wait_bounded(smem_u32(&accf_bar[acc]), acc_phase, abort_flag, p.err, p.timeout_ns, true))
         break;
       tc_fence_after();
-      const int m = t.wt * BM + row;
+      const int m = t.wt * WROWS + row;
       const bool m_ok = m < t.mrows;
       const long long ld = t.dense ? p.out_s_ld : p.out_ld;
       void* out = t.dense ? p.out_s : p.out;
       const long long r0 = (long long)t.b_row0 + (long long)t.tt * p.bn_max;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MAX);
-      for (int c0 = 0; c0 < n_mma; c0 += 16) {
-        uint32_t r1[16], r3[16];
-        if (DUAL) tmem_ld16x2_wait(taddr + c0, taddr + BN_MAX + c0, r1, r3);
-        else tmem_ld16_wait(taddr + c0, r1);
+      if (MODE == kUmmaSwiGLU) {
+        // Drain both accumulators into registers as packed bf16 h, hand TMEM
+        // back to the MMA warp, then store while the next tile accumulates.
+        uint32_t hp[BN_MAX / 2];
+#pragma unroll
+        for (int c = 0; c < BN_MAX / 16; ++c) {
+          if (c * 16 < n_mma) {
+            uint32_t r1[16], r3[16];
+            tmem_ld16x2_wait(taddr + c * 16, taddr + BN_MAX + c * 16, r1, r3);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float g0 = __uint_as_float(r1[2 * j]), g1 = __uint_as_float(r1[2 * j + 1]);
+              const float h0 = (g0 / (1.0f + __expf(-g0))) * __uint_as_float(r3[2 * j]);
+              const float h1 = (g1 / (1.0f + __expf(-g1))) * __uint_as_float(r3[2 * j + 1]);
+              const __nv_bfloat162 hb = __floats2bfloat162_rn(h0, h1);
+              hp[c * 8 + j] = *reinterpret_cast<const uint32_t*>(&hb);
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&acce_bar[acc]));
         if (m_ok) {
+          unsigned short* o = reinterpret_cast<unsigned short*>(out) + r0 * ld + m;
+#pragma unroll
+          for (int c = 0; c < BN_MAX / 16; ++c) {
+            if (c * 16 < n_valid) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const int col = c * 16 + j;
+                if (col < n_valid)
+                  o[(long long)col * ld] = (unsigned short)(hp[c * 8 + (j >> 1)] >> ((j & 1) * 16));
+              }
+            }
+          }
+        }
+      } else if (MODE == kUmmaDown) {
+        // Two 128-row blocks of the same 256-row weight tile.
+        const int m2 = m + BM;
+        const bool m2_ok = m2 < t.mrows;
+        __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out) + r0 * ld;
+        for (int c0 = 0; c0 < n_mma; c0 += 16) {
+          uint32_t r1[16], r3[16];
+          tmem_ld16x2_wait(taddr + c0, taddr + BN_MAX + c0, r1, r3);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int col = c0 + j;
             if (col < n_valid) {
-              float v = __uint_as_float(r1[j]);
-              if (DUAL) v = (v / (1.0f + __expf(-v))) * __uint_as_float(r3[j]);
-              const long long o = (r0 + col) * ld + m;
-              if (p.mode == kUmmaRouter) reinterpret_cast<float*>(out)[o] = v;
-              else reinterpret_cast<__nv_bfloat16*>(out)[o] = __float2bfloat16_rn(v);
+              if (m_ok) o[(long long)col * ld + m] = __float2bfloat16_rn(__uint_as_float(r1[j]));
+              if (m2_ok) o[(long long)col * ld + m2] = __float2bfloat16_rn(__uint_as_float(r3[j]));
             }
           }
         }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&acce_bar[acc]));
+      } else {
+        float* o = reinterpret_cast<float*>(out) + r0 * ld;
+        for (int c0 = 0; c0 < n_mma; c0 += 16) {
+          uint32_t r1[16];
+          tmem_ld16_wait(taddr + c0, r1);
+          if (m_ok) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int col = c0 + j;
+              if (col < n_valid) o[(long long)col * ld + m] = __uint_as_float(r1[j]);
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&acce_bar[acc]));
       }
-      tc_fence_before();
-      mbar_arrive(smem_u32(&acce_bar[acc]));
-      if (C::ACC_STAGES == 2) {
+      if (ACC_STAGES == 2) {
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       } else {
@@ -519,37 +636,54 @@ bool make_tmap(CUtensorMap* tm, const void* base, long long inner, long long out
   return r == CUDA_SUCCESS;
 }
 
-template <bool DUAL>
+template <int MODE>
 cudaError_t ensure_smem_attr() {
   static int done_mask = 0;   // one bit per device ordinal (< 32)
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 32 && ((done_mask >> dev) & 1)) return cudaSuccess;
-  e = cudaFuncSetAttribute(umma_gemm_kernel<DUAL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           Cfg<DUAL>::SMEM_BYTES);
+  e = cudaFuncSetAttribute(umma_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           SMEM_LIMIT);
   if (e == cudaSuccess && dev < 32) done_mask |= 1 << dev;
   return e;
+}
+
+template <int MODE>
+cudaError_t launch_mode(const CUtensorMap& tA, const CUtensorMap& tA3, const CUtensorMap& tB,
+                        const CUtensorMap& tAs, const CUtensorMap& tA3s, const CUtensorMap& tBs,
+                        const UmmaGemmParams& p, int grid, int smem, cudaStream_t s) {
+  cudaError_t e = ensure_smem_attr<MODE>();
+  if (e != cudaSuccess) return e;
+  umma_gemm_kernel<MODE><<<grid, NUM_THREADS, smem, s>>>(tA, tA3, tB, tAs, tA3s, tBs, p);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t s) {
-  const bool dual = p.mode == kUmmaSwiGLU;
   const bool has_dense = p.shared_rows > 0;
   if (p.n_routed == 0 && !has_dense) return cudaSuccess;
+  if (p.bn_max < 16 || p.bn_max > BN_MAX || p.bn_max % 16) return cudaErrorInvalidValue;
+  const int nseg = p.n_routed + (has_dense ? 1 : 0);
+  const SmemPlan sp = smem_plan(p.n_routed, nseg);
+  const int a_tiles = p.mode == kUmmaRouter ? 1 : 2;
+  const int wrows = p.mode == kUmmaDown ? 256 : 128;
+  if (sp.ring_bytes < 2 * (a_tiles * A_BYTES + ceil_div(p.bn_max, BOX_N) * BOX_BYTES))
+    return cudaErrorInvalidValue;
+  const bool swiglu = p.mode == kUmmaSwiGLU;
   CUtensorMap tA, tA3, tB, tAs, tA3s, tBs;
   if (has_dense) {
     if (!make_tmap(&tAs, p.a_s, p.K_s, p.m_rows_s, BM)) return cudaErrorInvalidValue;
     if (!make_tmap(&tBs, p.b_s, p.K_s, p.shared_rows, BOX_N)) return cudaErrorInvalidValue;
-    if (dual && !make_tmap(&tA3s, p.a3_s, p.K_s, p.m_rows_s, BM)) return cudaErrorInvalidValue;
-    if (!dual) tA3s = tAs;
+    if (swiglu && !make_tmap(&tA3s, p.a3_s, p.K_s, p.m_rows_s, BM)) return cudaErrorInvalidValue;
+    if (!swiglu) tA3s = tAs;
   }
   if (p.n_routed > 0) {
     if (!make_tmap(&tA, p.a, p.K, p.a_rows_total, BM)) return cudaErrorInvalidValue;
     if (!make_tmap(&tB, p.b, p.K, p.b_rows_total, BOX_N)) return cudaErrorInvalidValue;
-    if (dual && !make_tmap(&tA3, p.a3, p.K, p.a_rows_total, BM)) return cudaErrorInvalidValue;
-    if (!dual) tA3 = tA;
+    if (swiglu && !make_tmap(&tA3, p.a3, p.K, p.a_rows_total, BM)) return cudaErrorInvalidValue;
+    if (!swiglu) tA3 = tA;
   } else {
     tA = tAs; tA3 = tA3s; tB = tBs;
   }
@@ -557,19 +691,16 @@ cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t 
 
   long long tiles = 0;
   if (p.n_routed > 0)
-    tiles += (long long)ceil_div(p.m_rows, BM) * (ceil_div(p.max_routed_rows, p.bn_max) + p.n_routed);
-  if (has_dense) tiles += (long long)ceil_div(p.m_rows_s, BM) * ceil_div(p.shared_rows, p.bn_max);
+    tiles += (long long)ceil_div(p.m_rows, wrows) * (ceil_div(p.max_routed_rows, p.bn_max) + p.n_routed);
+  if (has_dense) tiles += (long long)ceil_div(p.m_rows_s, wrows) * ceil_div(p.shared_rows, p.bn_max);
   const int grid = (int)(tiles < num_sms ? tiles : num_sms);
   if (grid <= 0) return cudaSuccess;
-  cudaError_t e;
-  if (dual) {
-    if ((e = ensure_smem_attr<true>()) != cudaSuccess) return e;
-    umma_gemm_kernel<true><<<grid, NUM_THREADS, Cfg<true>::SMEM_BYTES, s>>>(tA, tA3, tB, tAs, tA3s, tBs, p);
-  } else {
-    if ((e = ensure_smem_attr<false>()) != cudaSuccess) return e;
-    umma_gemm_kernel<false><<<grid, NUM_THREADS, Cfg<false>::SMEM_BYTES, s>>>(tA, tA3, tB, tAs, tA3s, tBs, p);
+  switch (p.mode) {
+    case kUmmaRouter: return launch_mode<kUmmaRouter>(tA, tA3, tB, tAs, tA3s, tBs, p, grid, sp.total, s);
+    case kUmmaSwiGLU: return launch_mode<kUmmaSwiGLU>(tA, tA3, tB, tAs, tA3s, tBs, p, grid, sp.total, s);
+    case kUmmaDown: return launch_mode<kUmmaDown>(tA, tA3, tB, tAs, tA3s, tBs, p, grid, sp.total, s);
   }
-  return cudaGetLastError();
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_wait_timeout_selftest(uint32_t* err, long long timeout_ns, cudaStream_t s) {
