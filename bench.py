@@ -140,6 +140,21 @@ class ClockSampler:
                 "power_w_max": max((num(r[2]) or 0.0) for r in rows)}
 
 
+# ------------------------------------------------------- multi-rank timing
+def reduce_max(value: float, device, world: int) -> float:
+    """The slowest rank's value: every rank contributes, every rank gets the max."""
+    if world <= 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.item()
+
+
+def whole_job_rate(tokens_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Tokens per second of all ranks together (each rank runs its own replica)."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
 # ------------------------------------------------------------ work accounting
 def stage_work(cfg, counts):
     """Algorithmic bytes (compulsory HBM traffic) and flops of each stage for one forward."""
@@ -312,13 +327,9 @@ def main():
     torch.cuda.synchronize()
     t_wall1 = time.time()
     barrier()
-    ms_total = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_total = t.item()
+    ms_total = reduce_max(ev0.elapsed_time(ev1), dev, world)
     ms_step = ms_total / args.steps
-    value = world * T / (ms_step / 1e3)
+    value = whole_job_rate(T, world, ms_step)
     assert B.moe_get_device_error(ws) == B.MOE_OK
     sampler.stop()
     clocks = sampler.summary(t_wall0, t_wall1)
@@ -385,31 +396,52 @@ def main():
     expert_bytes = work["gate_up"]["bytes"] + work["down"]["bytes"]
 
     # ---- end to end through the public call with host buffers ------------------
-    x_host = inp["x"].cpu().pin_memory()
-    y_host = torch.empty((T, d), dtype=cfg.torch_dtype).pin_memory()
-    x_dev = torch.empty_like(inp["x"])
+    # Every step copies its x from pinned host memory, runs moe_forward and copies
+    # y back to pinned host memory. Copies run on their own streams with two
+    # buffers, so step i's compute overlaps step i+1's upload and step i-1's
+    # download, as a serving loop would.
+    x_host = [inp["x"].cpu().pin_memory() for _ in range(2)]
+    y_host = [torch.empty((T, d), dtype=cfg.torch_dtype).pin_memory() for _ in range(2)]
+    x_dev = [torch.empty_like(inp["x"]) for _ in range(2)]
+    y_dev = [torch.empty_like(y) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev = lambda: torch.cuda.Event(enable_timing=False)
+    in_done, comp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
 
-    def e2e_step():
-        x_dev.copy_(x_host, non_blocking=True)
-        B.moe_forward(cfg, x_dev, inp["w_router"], inp["bias"], inp["w1"], inp["w3"], inp["w2"],
-                      inp["ws1"], inp["ws3"], inp["ws2"], y, ws)
-        y_host.copy_(y, non_blocking=True)
+    def e2e_run(n_steps, t_start, t_end):
+        t_start.record(stream)
+        s_in.wait_event(t_start)
+        s_out.wait_event(t_start)
+        for i in range(n_steps):
+            b = i & 1
+            if i >= 2:
+                s_in.wait_event(comp_done[b])        # x_dev[b] no longer read
+            with torch.cuda.stream(s_in):
+                x_dev[b].copy_(x_host[b], non_blocking=True)
+            in_done[b].record(s_in)
+            stream.wait_event(in_done[b])
+            if i >= 2:
+                stream.wait_event(out_done[b])       # y_dev[b] already downloaded
+            B.moe_forward(cfg, x_dev[b], inp["w_router"], inp["bias"], inp["w1"], inp["w3"], inp["w2"],
+                          inp["ws1"], inp["ws3"], inp["ws2"], y_dev[b], ws, stream)
+            comp_done[b].record(stream)
+            s_out.wait_event(comp_done[b])
+            with torch.cuda.stream(s_out):
+                y_host[b].copy_(y_dev[b], non_blocking=True)
+            out_done[b].record(s_out)
+        stream.wait_event(out_done[(n_steps - 1) & 1])
+        if n_steps > 1:
+            stream.wait_event(out_done[n_steps & 1])
+        t_end.record(stream)
 
-    for _ in range(2):
-        e2e_step()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_run(3, e0, e1)
     torch.cuda.synchronize()
     barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
+    e2e_run(args.steps, e0, e1)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = t.item()
+    assert torch.equal(y_host[(args.steps - 1) & 1], y.cpu()), "end-to-end output differs"
+    e2e_ms = reduce_max(e0.elapsed_time(e1) / args.steps, dev, world)
     barrier()
 
     # ---- CPU oracle baseline (rank 0, one GPU only) --------------------------
@@ -442,7 +474,7 @@ def main():
             "stages_ms": stage_ms,
             "roofline": roof,
             "cpu_baseline": cpu,
-            "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": "tokens/s",
+            "e2e": {"value": whole_job_rate(T, world, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": T * d * cfg.elem_bytes, "d2h_bytes_per_step": T * d * cfg.elem_bytes,
                     "ms_per_step": e2e_ms},
             "gpu_launches": KERNELS_PER_FORWARD * args.steps,
