@@ -224,6 +224,67 @@ __device__ __forceinline__ void tmem_ld16x2_wait(uint32_t ta, uint32_t tb, uint3
 }
 #undef MOE_R16
 
+// ---- CTA-pair (cluster of 2) forms used by the two-SM MMA path.
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_cta(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+// TMA into this CTA's shared memory, completing on a barrier that may sit in
+// the peer CTA (the pair leader's).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* tm, int c0, int c1,
+                                                 uint32_t cluster_bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(cluster_bar)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t slot_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+// D (M=256 across the pair) (+)= A * B^T; each CTA holds 128 rows of A and
+// half of B's rows at the same shared-memory offsets, and 128 lanes of D.
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on the barrier at this offset in every CTA of `mask` once the pair
+// MMAs issued so far complete.
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
+}
+
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row atoms
 // 1024 bytes apart (stride byte offset), descriptor version 1 (sm_100).
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
@@ -238,10 +299,18 @@ __device__ __forceinline__ uint32_t idesc_bf16_f32(int m, int n) {
 }
 
 // ------------------------------------------------------------ tile list
+// Per mode: weight blocks (128 rows each) per CTA and accumulator stages.
+// With PAIR the two CTAs of a cluster run one M=256 MMA: each holds 128 rows
+// of every weight block and half of the token tile.
 template <int MODE> struct Kind;
-template <> struct Kind<kUmmaRouter> { static constexpr int A_TILES = 1; static constexpr int WROWS = 128; static constexpr int ACC_STAGES = 2; };
-template <> struct Kind<kUmmaSwiGLU> { static constexpr int A_TILES = 2; static constexpr int WROWS = 128; static constexpr int ACC_STAGES = 1; };
-template <> struct Kind<kUmmaDown>   { static constexpr int A_TILES = 2; static constexpr int WROWS = 256; static constexpr int ACC_STAGES = 1; };
+template <> struct Kind<kUmmaRouter> { static constexpr int A_TILES = 1; static constexpr int ACC_STAGES = 2; };
+template <> struct Kind<kUmmaSwiGLU> { static constexpr int A_TILES = 2; static constexpr int ACC_STAGES = 1; };
+template <> struct Kind<kUmmaDown>   { static constexpr int A_TILES = 2; static constexpr int ACC_STAGES = 1; };
+
+// Weight rows covered by one tile (all CTAs of the group together).
+__host__ __device__ constexpr int tile_rows(int mode, bool pair) {
+  return (mode == kUmmaDown ? 256 : 128) * (pair ? 2 : 1);
+}
 
 struct Tile {
   int seg, wt, tt;
@@ -288,7 +357,22 @@ __device__ __forceinline__ Tile decode_tile(const UmmaGemmParams& p, const int* 
   return t;
 }
 
-template <int MODE>
+// Token rows this CTA stages for a tile, and how many TMA boxes that takes.
+struct TokenSlice {
+  int n_valid, n_mma, row, nbox;
+};
+template <bool PAIR>
+__device__ __forceinline__ TokenSlice token_slice(const UmmaGemmParams& p, const Tile& t, uint32_t rank) {
+  TokenSlice ts;
+  ts.n_valid = min(p.bn_max, t.rows - t.tt * p.bn_max);
+  ts.n_mma = (ts.n_valid + 15) & ~15;
+  const int mine = PAIR ? ts.n_mma / 2 : ts.n_valid;
+  ts.row = t.b_row0 + t.tt * p.bn_max + (PAIR ? (int)rank * (ts.n_mma / 2) : 0);
+  ts.nbox = (mine + BOX_N - 1) / BOX_N;
+  return ts;
+}
+
+template <int MODE, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA3,
                      const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmAs,
@@ -296,8 +380,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                      const UmmaGemmParams p) {
   using KD = Kind<MODE>;
   constexpr int A_TILES = KD::A_TILES;
-  constexpr int WROWS = KD::WROWS;
   constexpr int ACC_STAGES = KD::ACC_STAGES;
+  constexpr int WROWS = tile_rows(MODE, PAIR);
+  // Row offset of weight block a (0 or 1) inside a tile, for CTA rank r.
+  constexpr int BLOCK_STEP = (MODE == kUmmaDown) ? (PAIR ? 256 : 128) : 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -319,6 +405,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* ring = smem + 1024 + sp.table_bytes;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_rank() : 0u;
+  const bool leader = rank == 0;
+  const int group = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int ngroups = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   for (int s = threadIdx.x; s <= p.n_routed; s += blockDim.x)
     s_off[s] = p.n_routed > 0 ? p.offsets[s] : 0;
@@ -329,15 +419,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&accf_bar[i]), 1);
-      mbar_init(smem_u32(&acce_bar[i]), 4 * 32);
+      mbar_init(smem_u32(&acce_bar[i]), (PAIR ? 2 : 1) * 4);   // one arrival per epilogue warp
     }
     mbar_init(smem_u32(drain_bar), 1);
     *abort_flag = 0u;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   if (threadIdx.x == 0) {
     tmap_prefetch(&tmA); tmap_prefetch(&tmB); tmap_prefetch(&tmAs); tmap_prefetch(&tmBs);
@@ -370,7 +465,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 31) s_start[nseg] = incl;
   }
   tc_fence_before();
-  __syncthreads();
+  if (PAIR) cluster_sync_all(); else __syncthreads();   // barriers of both CTAs exist from here on
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total_tiles = s_start[nseg];
@@ -381,16 +476,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t inflight = 0;
     const uint32_t max_inflight = (uint32_t)min(max(p.max_inflight, 2), NSLOT);
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+    for (int tile = group; tile < total_tiles && ok; tile += ngroups) {
       const Tile t = decode_tile(p, s_off, s_start, nseg, tile, WROWS);
+      const TokenSlice ts = token_slice<PAIR>(p, t, rank);
       const CUtensorMap* mA = t.dense ? &tmAs : &tmA;
       const CUtensorMap* mA3 = t.dense ? &tmA3s : &tmA3;
       const CUtensorMap* mB = t.dense ? &tmBs : &tmB;
-      const int a_row = (t.dense ? 0 : t.seg * p.m_rows) + t.wt * WROWS;
-      const int b_row = t.b_row0 + t.tt * p.bn_max;
-      const int n_valid = min(p.bn_max, t.rows - t.tt * p.bn_max);
-      const int nbox = (n_valid + BOX_N - 1) / BOX_N;
-      const uint32_t bytes = A_TILES * A_BYTES + nbox * BOX_BYTES;
+      const int a_row = (t.dense ? 0 : t.seg * p.m_rows) + t.wt * WROWS + (int)rank * BM;
+      const uint32_t bytes = A_TILES * A_BYTES + ts.nbox * BOX_BYTES;
       const int nk = ceil_div(t.K, BK);
       for (int kb = 0; kb < nk; ++kb) {
         // Make room: the barrier pair and the bytes of the new slot must be free.
@@ -416,40 +509,55 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         fl_off[slot] = off;
         fl_size[slot] = bytes;
         ++inflight;
-        const uint32_t fb = smem_u32(&full_bar[slot]);
-        mbar_expect_tx(fb, bytes);
+        const uint32_t fb_local = smem_u32(&full_bar[slot]);
         const uint32_t sb = smem_u32(ring + off);
-        tma_load_2d(sb, mA, kb * BK, a_row, fb);
-        if (MODE == kUmmaSwiGLU) tma_load_2d(sb + A_BYTES, mA3, kb * BK, a_row, fb);
-        if (MODE == kUmmaDown) tma_load_2d(sb + A_BYTES, mA, kb * BK, a_row + BM, fb);
         const uint32_t bb = sb + A_TILES * A_BYTES;
-        for (int bx = 0; bx < nbox; ++bx)
-          tma_load_2d(bb + bx * BOX_BYTES, mB, kb * BK, b_row + bx * BOX_N, fb);
+        if (PAIR) {
+          // Both CTAs' copies complete on the leader's barrier, which the leader
+          // arms for both halves (the halves are the same size).
+          const uint32_t fb = map_to_cta(fb_local, 0);
+          if (leader) mbar_expect_tx(fb_local, 2 * bytes);
+          tma_load_2d_pair(sb, mA, kb * BK, a_row, fb);
+          if (MODE == kUmmaSwiGLU) tma_load_2d_pair(sb + A_BYTES, mA3, kb * BK, a_row, fb);
+          if (MODE == kUmmaDown) tma_load_2d_pair(sb + A_BYTES, mA, kb * BK, a_row + BLOCK_STEP, fb);
+          for (int bx = 0; bx < ts.nbox; ++bx)
+            tma_load_2d_pair(bb + bx * BOX_BYTES, mB, kb * BK, ts.row + bx * BOX_N, fb);
+        } else {
+          mbar_expect_tx(fb_local, bytes);
+          tma_load_2d(sb, mA, kb * BK, a_row, fb_local);
+          if (MODE == kUmmaSwiGLU) tma_load_2d(sb + A_BYTES, mA3, kb * BK, a_row, fb_local);
+          if (MODE == kUmmaDown) tma_load_2d(sb + A_BYTES, mA, kb * BK, a_row + BLOCK_STEP, fb_local);
+          for (int bx = 0; bx < ts.nbox; ++bx)
+            tma_load_2d(bb + bx * BOX_BYTES, mB, kb * BK, ts.row + bx * BOX_N, fb_local);
+        }
       }
     }
-    // Let every copy this thread started land before the CTA can exit.
+    // Let every copy this thread started land before the CTA can exit: its
+    // slot is released only after the MMA consumed it.
     for (uint32_t i = 0; i < inflight; ++i) {
       const uint32_t u = cur.count - inflight + i;
-      wait_bounded(smem_u32(&full_bar[u % NSLOT]), (u / NSLOT) & 1u, abort_flag, p.err, p.timeout_ns,
-                   false);
+      if (PAIR)
+        wait_bounded(smem_u32(&empty_bar[u % NSLOT]), (u / NSLOT) & 1u, abort_flag, p.err,
+                     p.timeout_ns, false);
+      else
+        wait_bounded(smem_u32(&full_bar[u % NSLOT]), (u / NSLOT) & 1u, abort_flag, p.err,
+                     p.timeout_ns, false);
     }
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == 1 && lane == 0 && leader) {
     // ------------------------------------------------------------ MMA issuer
     RingCursor cur;
     int acc = 0;
     uint32_t acc_phase = 0;
     bool issued = false;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+    for (int tile = group; tile < total_tiles; tile += ngroups) {
       const Tile t = decode_tile(p, s_off, s_start, nseg, tile, WROWS);
-      const int n_valid = min(p.bn_max, t.rows - t.tt * p.bn_max);
-      const int n_mma = (n_valid + 15) & ~15;
-      const int nbox = (n_valid + BOX_N - 1) / BOX_N;
-      const uint32_t bytes = A_TILES * A_BYTES + nbox * BOX_BYTES;
+      const TokenSlice ts = token_slice<PAIR>(p, t, 0);
+      const uint32_t bytes = A_TILES * A_BYTES + ts.nbox * BOX_BYTES;
       const int nk = ceil_div(t.K, BK);
       if (!wait_bounded(smem_u32(&acce_bar[acc]), acc_phase ^ 1u, abort_flag, p.err, p.timeout_ns, true))
         break;
       tc_fence_after();
-      const uint32_t idesc = idesc_bf16_f32(BM, n_mma);
+      const uint32_t idesc = idesc_bf16_f32(PAIR ? 2 * BM : BM, ts.n_mma);
       const uint32_t d1 = tmem_base + (uint32_t)(acc * BN_MAX);
       const uint32_t d3 = tmem_base + (uint32_t)BN_MAX;
       bool ok = true;
@@ -469,14 +577,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int kk = 0; kk < BK / UMMA_K; ++kk) {
           const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
           const uint64_t koff = (uint64_t)((kk * UMMA_K * 2) >> 4);
-          umma_bf16(d1, a_desc + koff, b_desc + koff, idesc, accum);
-          if (A_TILES == 2) umma_bf16(d3, a3_desc + koff, b_desc + koff, idesc, accum);
+          if (PAIR) {
+            umma_bf16_pair(d1, a_desc + koff, b_desc + koff, idesc, accum);
+            if (A_TILES == 2) umma_bf16_pair(d3, a3_desc + koff, b_desc + koff, idesc, accum);
+          } else {
+            umma_bf16(d1, a_desc + koff, b_desc + koff, idesc, accum);
+            if (A_TILES == 2) umma_bf16(d3, a3_desc + koff, b_desc + koff, idesc, accum);
+          }
         }
         issued = true;
-        umma_commit(smem_u32(&empty_bar[slot]));
+        if (PAIR) umma_commit_pair(smem_u32(&empty_bar[slot]), 0x3);
+        else umma_commit(smem_u32(&empty_bar[slot]));
       }
       if (!ok) break;
-      umma_commit(smem_u32(&accf_bar[acc]));
+      if (PAIR) umma_commit_pair(smem_u32(&accf_bar[acc]), 0x3);
+      else umma_commit(smem_u32(&accf_bar[acc]));
       if (ACC_STAGES == 2) {
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
@@ -485,28 +600,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
     if (issued) {   // every MMA this thread issued completes before TMEM is freed
-      umma_commit(smem_u32(drain_bar));
+      if (PAIR) umma_commit_pair(smem_u32(drain_bar), 0x1);
+      else umma_commit(smem_u32(drain_bar));
       wait_bounded(smem_u32(drain_bar), 0u, abort_flag, p.err, p.timeout_ns, false);
     }
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                  // TMEM lane quarter this warp may read
     const int row = q * 32 + lane;
+    // The accumulator is released to the leader's barrier (remote for the peer).
+    const uint32_t acce0 = PAIR ? map_to_cta(smem_u32(&acce_bar[0]), 0) : smem_u32(&acce_bar[0]);
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+    for (int tile = group; tile < total_tiles; tile += ngroups) {
       const Tile t = decode_tile(p, s_off, s_start, nseg, tile, WROWS);
-      const int n_valid = min(p.bn_max, t.rows - t.tt * p.bn_max);
-      const int n_mma = (n_valid + 15) & ~15;
+      const TokenSlice ts = token_slice<PAIR>(p, t, 0);
+      const int n_valid = ts.n_valid, n_mma = ts.n_mma;
       if (!wait_bounded(smem_u32(&accf_bar[acc]), acc_phase, abort_flag, p.err, p.timeout_ns, true))
         break;
       tc_fence_after();
-      const int m = t.wt * WROWS + row;
+      const int m = t.wt * WROWS + (int)rank * BM + row;
       const bool m_ok = m < t.mrows;
       const long long ld = t.dense ? p.out_s_ld : p.out_ld;
       void* out = t.dense ? p.out_s : p.out;
       const long long r0 = (long long)t.b_row0 + (long long)t.tt * p.bn_max;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MAX);
+      const uint32_t acce = acce0 + (uint32_t)(acc * 8);
       if (MODE == kUmmaSwiGLU) {
         // Drain both accumulators into registers as packed bf16 h, hand TMEM
         // back to the MMA warp, then store while the next tile accumulates.
@@ -527,7 +646,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
         tc_fence_before();
-        mbar_arrive(smem_u32(&acce_bar[acc]));
+        __syncwarp();
+        if (lane == 0) { if (PAIR) mbar_arrive_cluster(acce); else mbar_arrive(acce); }
         if (m_ok) {
           unsigned short* o = reinterpret_cast<unsigned short*>(out) + r0 * ld + m;
 #pragma unroll
@@ -543,8 +663,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       } else if (MODE == kUmmaDown) {
-        // Two 128-row blocks of the same 256-row weight tile.
-        const int m2 = m + BM;
+        // Two 128-row blocks of the tile's weight rows, BLOCK_STEP apart.
+        const int m2 = m + BLOCK_STEP;
         const bool m2_ok = m2 < t.mrows;
         __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out) + r0 * ld;
         for (int c0 = 0; c0 < n_mma; c0 += 16) {
@@ -560,7 +680,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
         tc_fence_before();
-        mbar_arrive(smem_u32(&acce_bar[acc]));
+        __syncwarp();
+        if (lane == 0) { if (PAIR) mbar_arrive_cluster(acce); else mbar_arrive(acce); }
       } else {
         float* o = reinterpret_cast<float*>(out) + r0 * ld;
         for (int c0 = 0; c0 < n_mma; c0 += 16) {
@@ -575,7 +696,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
         tc_fence_before();
-        mbar_arrive(smem_u32(&acce_bar[acc]));
+        __syncwarp();
+        if (lane == 0) { if (PAIR) mbar_arrive_cluster(acce); else mbar_arrive(acce); }
       }
       if (ACC_STAGES == 2) {
         acc ^= 1;
@@ -586,11 +708,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   }
   tc_fence_before();
-  __syncthreads();
+  if (PAIR) cluster_sync_all(); else __syncthreads();   // peer smem and TMEM stay live until here
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    if (PAIR) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
@@ -636,27 +759,42 @@ bool make_tmap(CUtensorMap* tm, const void* base, long long inner, long long out
   return r == CUDA_SUCCESS;
 }
 
-template <int MODE>
+template <int MODE, bool PAIR>
 cudaError_t ensure_smem_attr() {
   static int done_mask = 0;   // one bit per device ordinal (< 32)
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 32 && ((done_mask >> dev) & 1)) return cudaSuccess;
-  e = cudaFuncSetAttribute(umma_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(umma_gemm_kernel<MODE, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            SMEM_LIMIT);
   if (e == cudaSuccess && dev < 32) done_mask |= 1 << dev;
   return e;
 }
 
-template <int MODE>
+template <int MODE, bool PAIR>
 cudaError_t launch_mode(const CUtensorMap& tA, const CUtensorMap& tA3, const CUtensorMap& tB,
                         const CUtensorMap& tAs, const CUtensorMap& tA3s, const CUtensorMap& tBs,
                         const UmmaGemmParams& p, int grid, int smem, cudaStream_t s) {
-  cudaError_t e = ensure_smem_attr<MODE>();
+  cudaError_t e = ensure_smem_attr<MODE, PAIR>();
   if (e != cudaSuccess) return e;
-  umma_gemm_kernel<MODE><<<grid, NUM_THREADS, smem, s>>>(tA, tA3, tB, tAs, tA3s, tBs, p);
-  return cudaGetLastError();
+  if (!PAIR) {
+    umma_gemm_kernel<MODE, false><<<grid, NUM_THREADS, smem, s>>>(tA, tA3, tB, tAs, tA3s, tBs, p);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, umma_gemm_kernel<MODE, true>, tA, tA3, tB, tAs, tA3s, tBs, p);
 }
 
 }  // namespace
@@ -668,7 +806,11 @@ cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t 
   const int nseg = p.n_routed + (has_dense ? 1 : 0);
   const SmemPlan sp = smem_plan(p.n_routed, nseg);
   const int a_tiles = p.mode == kUmmaRouter ? 1 : 2;
-  const int wrows = p.mode == kUmmaDown ? 256 : 128;
+  // Expert GEMMs with wide token tiles run on CTA pairs (M=256 MMAs: each CTA
+  // stages half the token tile, halving token traffic per weight byte). Narrow
+  // tiles (decode) and the router stay on single CTAs.
+  const bool pair = p.mode != kUmmaRouter && p.bn_max >= 128 && num_sms >= 2;
+  const int wrows = tile_rows(p.mode, pair);
   if (sp.ring_bytes < 2 * (a_tiles * A_BYTES + ceil_div(p.bn_max, BOX_N) * BOX_BYTES))
     return cudaErrorInvalidValue;
   const bool swiglu = p.mode == kUmmaSwiGLU;
@@ -693,12 +835,19 @@ cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t 
   if (p.n_routed > 0)
     tiles += (long long)ceil_div(p.m_rows, wrows) * (ceil_div(p.max_routed_rows, p.bn_max) + p.n_routed);
   if (has_dense) tiles += (long long)ceil_div(p.m_rows_s, wrows) * ceil_div(p.shared_rows, p.bn_max);
-  const int grid = (int)(tiles < num_sms ? tiles : num_sms);
-  if (grid <= 0) return cudaSuccess;
+  const int groups = pair ? num_sms / 2 : num_sms;
+  const int ngroup = (int)(tiles < groups ? tiles : groups);
+  if (ngroup <= 0) return cudaSuccess;
+  const int grid = pair ? 2 * ngroup : ngroup;
   switch (p.mode) {
-    case kUmmaRouter: return launch_mode<kUmmaRouter>(tA, tA3, tB, tAs, tA3s, tBs, p, grid, sp.total, s);
-    case kUmmaSwiGLU: return launch_mode<kUmmaSwiGLU>(tA, tA3, tB, tAs, tA3s, tBs, p, grid, sp.total, s);
-    case kUmmaDown: return launch_mode<kUmmaDown>(tA, tA3, tB, tAs, tA3s, tBs, p, grid, sp.total, s);
+    case kUmmaRouter:
+      return launch_mode<kUmmaRouter, false>(tA, tA3, tB, tAs, tA3s, tBs, p, grid, sp.total, s);
+    case kUmmaSwiGLU:
+      return pair ? launch_mode<kUmmaSwiGLU, true>(tA, tA3, tB, tAs, tA3s, tBs, p, grid, sp.total, s)
+                  : launch_mode<kUmmaSwiGLU, false>(tA, tA3, tB, tAs, tA3s, tBs, p, grid, sp.total, s);
+    case kUmmaDown:
+      return pair ? launch_mode<kUmmaDown, true>(tA, tA3, tB, tAs, tA3s, tBs, p, grid, sp.total, s)
+                  : launch_mode<kUmmaDown, false>(tA, tA3, tB, tAs, tA3s, tBs, p, grid, sp.total, s);
   }
   return cudaErrorInvalidValue;
 }
