@@ -59,6 +59,7 @@ __all__ = [
     "group_scores", "group_eligibility", "select_experts", "gate_values", "route",
     "silu", "swiglu_hidden", "swiglu_ffn", "expert_outputs", "moe_forward", "moe_forward_dense_loop",
     "expert_counts_offsets", "permutation_rows", "near_tie_tokens",
+    "balance_target", "update_bias", "routing_entropy",
 ]
 
 
@@ -364,3 +365,43 @@ def near_tie_tokens(routed: dict, k: int, n_groups: int = 1, topk_groups: int = 
             if not np.array_equal(alt_sel, routed["idx"][t]):
                 flags[t] = True
     return flags
+
+
+# ---------------------------------------------------------------------------
+# Aux-loss-free load balancing (the step that follows routing in training)
+# ---------------------------------------------------------------------------
+
+def balance_target(T: int, k: int, E: int) -> float:
+    """Per-expert target usage: n_tokens * top_k / n_experts.
+
+    [CS] "Aux-loss-free balance loop", step 1.
+    """
+    return T * k / E
+
+
+def update_bias(bias, counts, target: float, gamma: float) -> np.ndarray:
+    """One bias update: experts over target lose gamma, experts under gain it.
+
+    [CS] "Aux-loss-free balance loop", step 5 (over target: bias -= gamma;
+    under target: bias += gamma). An expert exactly on target keeps its bias
+    (the page names only the two strict cases).
+    """
+    bias = _f64(bias).copy()
+    counts = np.asarray(counts, dtype=np.float64)
+    bias[counts > target] -= gamma
+    bias[counts < target] += gamma
+    return bias
+
+
+def routing_entropy(counts) -> float:
+    """Shannon entropy (nats) of the expert-usage distribution counts / sum.
+
+    [CS] "Aux-loss-free balance loop", step 7: it rises toward ln(n_experts),
+    the value for uniform usage. Experts with zero count contribute 0.
+    """
+    c = np.asarray(counts, dtype=np.float64)
+    total = c.sum()
+    if total <= 0:
+        return 0.0
+    p = c[c > 0] / total
+    return float(-(p * np.log(p)).sum())

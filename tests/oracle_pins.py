@@ -369,4 +369,43 @@ def pin_near_tie_flags():
     assert orc.near_tie_tokens(r, 2, 3, 2).tolist() == [False, False]
 
 
+# ------------------------------------------------------- balance loop
+def pin_entropy_closed_forms():
+    for E in (1, 2, 7, 256):
+        _close(orc.routing_entropy(np.full(E, 5)), math.log(E), tol=1e-14)
+    _close(orc.routing_entropy([0, 0, 9, 0]), 0.0)
+    _close(orc.routing_entropy([3, 1]), -(0.75 * math.log(0.75) + 0.25 * math.log(0.25)))
+    _close(orc.routing_entropy([2, 0, 2]), math.log(2.0))
+    assert orc.routing_entropy([0, 0]) == 0.0
+
+
+def pin_bias_update_direction():
+    # target = 12 * 2 / 4 = 6: experts at 9, 6, 3, 6 tokens.
+    t = orc.balance_target(12, 2, 4)
+    assert t == 6.0
+    b = orc.update_bias([0.5, -0.25, 0.0, 1.0], [9, 6, 3, 6], t, 0.15)
+    _close(b, [0.35, -0.25, 0.15, 1.0], tol=1e-15)
+
+
+def pin_balance_loop_raises_entropy():
+    # The cheat sheet's loop: route with scores + bias, count, update with
+    # gamma = 0.15, 10 iterations; entropy rises toward ln(E). A router whose
+    # first experts are favoured starts far from uniform.
+    rng = np.random.default_rng(61)
+    T, d, E, k = 256, 16, 8, 2
+    x = rng.standard_normal((T, d))
+    wr = rng.standard_normal((E, d)) / math.sqrt(d)
+    skew = np.linspace(1.5, -1.5, E)
+    bias = np.zeros(E)
+    ent = []
+    for it in range(10):
+        r = orc.route(x, wr, skew + bias, k, orc.GATE_SOFTMAX)
+        counts, _ = orc.expert_counts_offsets(r["idx"], E)
+        ent.append(orc.routing_entropy(counts))
+        bias = orc.update_bias(bias, counts, orc.balance_target(T, k, E), 0.15)
+    assert ent[-1] > ent[0] + 0.2, ent
+    assert max(ent) <= math.log(E) + 1e-12
+    assert ent[-1] > 0.95 * math.log(E), ent
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]

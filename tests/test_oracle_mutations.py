@@ -126,7 +126,22 @@ def _loop_no_renorm(x, w_router, w1, w3, w2, k):
     return _orig["expert_outputs"](x, idx, p[rows, idx], w1, w3, w2)
 
 
+def _bias_update_wrong_sign(bias, counts, target, gamma):
+    return _orig["update_bias"](bias, counts, target, -gamma)
+
+
+def _entropy_log2(counts):
+    return _orig["routing_entropy"](counts) / np.log(2.0)
+
+
+def _target_no_k(T, k, E):
+    return T / E
+
+
 MUTATIONS = {
+    "bias_update_wrong_sign": ("update_bias", _bias_update_wrong_sign),
+    "entropy_in_bits": ("routing_entropy", _entropy_log2),
+    "target_without_k": ("balance_target", _target_no_k),
     "swiglu_w1_w3_swapped": ("swiglu_ffn", _swiglu_swapped),
     "swiglu_no_silu": ("swiglu_ffn", _swiglu_no_silu),
     "swiglu_down_transposed": ("swiglu_ffn", _swiglu_down_transposed),
