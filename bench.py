@@ -375,6 +375,29 @@ def main():
     stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(n_stage))
                 for j, n in enumerate(names)}
     assert torch.equal(y2, y), "per-stage chain and moe_forward disagree"
+    # ---- aux-loss-free balancing step that follows routing in training: one
+    # small kernel over the E counts (launch-latency bound); timed on its own.
+    bias_scratch = inp["bias"].clone() if inp["bias"] is not None else torch.zeros(E, device=dev)
+    ent = torch.empty(1, device=dev)
+    # 100 calls captured in one CUDA graph, so the device time per call is
+    # measured rather than the host's launch rate.
+    for _ in range(3):
+        B.moe_balance_update(cfg, counts, bias_scratch, 0.15, ent)
+    torch.cuda.synchronize()
+    bal_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(bal_graph):
+        for _ in range(100):
+            B.moe_balance_update(cfg, counts, bias_scratch, 0.15, ent)
+    bal_graph.replay()
+    torch.cuda.synchronize()
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b0.record(stream)
+    bal_graph.replay()
+    b1.record(stream)
+    torch.cuda.synchronize()
+    del bal_graph
+    balance = {"us_per_call": b0.elapsed_time(b1) * 10.0, "entropy": ent.item(),
+               "ln_E": math.log(E), "gamma": 0.15, "bound": "launch latency (E-element kernel)"}
     work, touched = stage_work(cfg, counts.cpu())
     peaks = measured_peaks()
     dom = max(names, key=lambda n: stage_ms[n])
@@ -472,6 +495,7 @@ def main():
                             "frac_tensor": expert_flops / (expert_ms / 1e3) / 1e12 / peaks["tensor_sustained"],
                             "frac_hbm": expert_bytes / (expert_ms / 1e3) / 1e9 / peaks["hbm"]},
             "stages_ms": stage_ms,
+            "balance_update": balance,
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": {"value": whole_job_rate(T, world, e2e_ms), "unit": "tokens/s",

@@ -264,6 +264,25 @@ MOE_API moe_status moe_route_noalloc(const moe_config* cfg, const void* x, const
                              const float* bias, int32_t* topk_idx, float* topk_gate,
                              int32_t* expert_counts, int32_t* expert_offsets, void* stream);
 
+/*
+ * moe_balance_update - the aux-loss-free balancing step that follows routing
+ * in training, and the routing entropy.  [CS] "Aux-loss-free balance loop":
+ * target usage = n_tokens * top_k / n_experts; over target, bias -= gamma;
+ * under target, bias += gamma; entropy of the usage rises toward ln(E).
+ *
+ *   expert_counts [E]  int32  tokens per expert (moe_route's output for cfg->T tokens)
+ *   bias          [E]  fp32   IN/OUT selection bias, updated in place (NULL: skip)
+ *   gamma                     step size >= 0 (the page's demo uses 0.15)
+ *   entropy       [1]  fp32   OUT: -sum_e p_e ln p_e, p = counts / sum(counts),
+ *                             accumulated in fp64 (NULL: skip)
+ *
+ * An expert exactly on target keeps its bias; over/under is decided exactly
+ * (count * E against T * k in integers). At least one of bias and entropy
+ * must be given. One small kernel; asynchronous on `stream`.
+ */
+MOE_API moe_status moe_balance_update(const moe_config* cfg, const int32_t* expert_counts,
+                              float* bias, float gamma, float* entropy, void* stream);
+
 /* Synchronises `stream`, reads and clears the workspace's device error word.
  * Returns MOE_OK, MOE_ERR_TIMEOUT (a bounded device wait ran out during an
  * earlier call on this workspace) or MOE_ERR_CUDA. Every entry point that

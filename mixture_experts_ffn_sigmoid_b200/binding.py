@@ -31,7 +31,8 @@ MOE_DTYPE_BF16 = 1
 
 EXPORTED = ("moe_check_config", "moe_workspace_size", "moe_route", "moe_permute",
             "moe_expert_swiglu", "moe_expert_gate_up", "moe_expert_down", "moe_combine", "moe_forward", "moe_get_device_error",
-            "moe_selftest_wait_timeout", "moe_route_noalloc", "moe_status_string")
+            "moe_selftest_wait_timeout", "moe_route_noalloc", "moe_balance_update",
+            "moe_status_string")
 
 
 class MoEError(RuntimeError):
@@ -79,6 +80,7 @@ def lib() -> ctypes.CDLL:
             "moe_get_device_error": (ctypes.c_int, [vp, vp]),
             "moe_selftest_wait_timeout": (ctypes.c_int, [vp, sz, ctypes.c_int64, vp]),
             "moe_route_noalloc": (ctypes.c_int, [cfgp, vp, vp, f32p, i32p, f32p, i32p, i32p, vp]),
+            "moe_balance_update": (ctypes.c_int, [cfgp, i32p, f32p, ctypes.c_float, f32p, vp]),
             "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         }
         for name, (res, args) in sig.items():
@@ -202,6 +204,13 @@ def moe_route_noalloc(cfg, x, w_router, bias, topk_idx, topk_gate, expert_counts
     _check(lib().moe_route_noalloc(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(bias),
                                    _ptr(topk_idx), _ptr(topk_gate), _ptr(expert_counts),
                                    _ptr(expert_offsets), _stream(stream)), "moe_route_noalloc")
+
+
+def moe_balance_update(cfg, expert_counts, bias, gamma: float, entropy=None, stream=None):
+    """Aux-loss-free bias step in place on `bias` and/or the routing entropy."""
+    c = _cfg(cfg)
+    _check(lib().moe_balance_update(ctypes.byref(c), _ptr(expert_counts), _ptr(bias), float(gamma),
+                                    _ptr(entropy), _stream(stream)), "moe_balance_update")
 
 
 def moe_get_device_error(workspace, stream=None) -> int:

@@ -477,6 +477,20 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
   return MOE_OK;
 }
 
+moe_status moe_balance_update(const moe_config* cfg, const int32_t* expert_counts, float* bias,
+                              float gamma, float* entropy, void* stream) {
+  MOE_TRY(check_config(cfg));
+  const moe_config& c = *cfg;
+  MOE_TRY(need4(expert_counts));
+  if (!bias && !entropy) return MOE_ERR_INVALID_ARG;
+  if (bias) MOE_TRY(need4(bias));
+  if (entropy) MOE_TRY(need4(entropy));
+  if (bias && (!(gamma >= 0.0f) || !isfinite(gamma))) return MOE_ERR_INVALID_ARG;
+  MOE_CUDA(launch_balance_update(expert_counts, c.E, (long long)c.T * c.k, gamma, bias, entropy,
+                                 static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
 moe_status moe_get_device_error(void* workspace, void* stream) {
   MOE_TRY(need(workspace));
   cudaStream_t s = static_cast<cudaStream_t>(stream);

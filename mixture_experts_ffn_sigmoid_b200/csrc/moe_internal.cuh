@@ -51,6 +51,8 @@ cudaError_t launch_chunk_counts(const int* topk_idx, int T, int k, int E, int* c
 cudaError_t launch_chunk_scan(const int* chunk_counts, int nchunks, int E, int* chunk_base,
                               int* counts, cudaStream_t s);
 cudaError_t launch_offsets(const int* counts, int E, int* offsets, cudaStream_t s);
+cudaError_t launch_balance_update(const int* counts, int E, long long tk, float gamma, float* bias,
+                                  float* entropy, cudaStream_t s);
 
 // Permute / combine (permute_kernels.cu)
 cudaError_t launch_permute(int dtype, const void* x, const int* topk_idx, const int* offsets,

@@ -221,7 +221,58 @@ __global__ void __launch_bounds__(1024) offsets_kernel(const int* __restrict__ c
   if (e == 0) offsets[E] = total;
 }
 
+// Aux-loss-free balancing step (MoE cheat sheet, "Aux-loss-free balance
+// loop"): target = T*k/E; an expert over target loses gamma of bias, one
+// under target gains gamma, one on target keeps its bias (decided in exact
+// integer arithmetic, count*E vs T*k). Also the entropy (nats) of the usage
+// distribution counts/sum, accumulated in fp64.
+__global__ void __launch_bounds__(1024) balance_update_kernel(const int* __restrict__ counts, int E,
+                                                              long long tk, float gamma,
+                                                              float* __restrict__ bias,
+                                                              float* __restrict__ entropy) {
+  __shared__ double s_red[32];
+  __shared__ long long s_tot[32];
+  const int e = threadIdx.x;
+  const int lane = e & 31, warp = e >> 5, nwarps = blockDim.x >> 5;
+  const long long c = e < E ? (long long)counts[e] : 0;
+  if (e < E && bias) {
+    const long long scaled = c * E;
+    if (scaled > tk) bias[e] -= gamma;
+    else if (scaled < tk) bias[e] += gamma;
+  }
+  if (!entropy) return;
+  // Total count, then -sum p ln p.
+  long long tot = c;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) tot += __shfl_xor_sync(kFull, tot, off);
+  if (lane == 0) s_tot[warp] = tot;
+  __syncthreads();
+  long long all = 0;
+  for (int w = 0; w < nwarps; ++w) all += s_tot[w];
+  double h = 0.0;
+  if (c > 0 && all > 0) {
+    const double pr = (double)c / (double)all;
+    h = -pr * log(pr);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) h += __shfl_xor_sync(kFull, h, off);
+  if (lane == 0) s_red[warp] = h;
+  __syncthreads();
+  if (e == 0) {
+    double sum = 0.0;
+    for (int w = 0; w < nwarps; ++w) sum += s_red[w];
+    *entropy = (float)sum;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_balance_update(const int* counts, int E, long long tk, float gamma, float* bias,
+                                  float* entropy, cudaStream_t s) {
+  const int threads = ceil_div(E, 32) * 32;
+  balance_update_kernel<<<1, threads, 0, s>>>(counts, E, tk, gamma, bias, entropy);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_router_topk(const RouteParams& p, cudaStream_t s) {
   if (p.T <= 0) return cudaSuccess;

@@ -142,6 +142,10 @@ def test_host_side_rejections_before_any_launch():
                          None) == B.MOE_ERR_MISALIGNED
     assert L.moe_expert_swiglu(ctypes.byref(cfg), fake, fake, fake, fake, fake, None, None, None, None,
                                None, None, fake, nbytes, None) == B.MOE_ERR_INVALID_ARG
+    # balance update: nothing to do is an error; a negative step is rejected
+    assert L.moe_balance_update(ctypes.byref(cfg), fake, None, ctypes.c_float(0.1), None, None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_balance_update(ctypes.byref(cfg), fake, fake, ctypes.c_float(-0.1), None, None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_balance_update(ctypes.byref(cfg), None, fake, ctypes.c_float(0.1), None, None) == B.MOE_ERR_INVALID_ARG
     # the timeout self-test needs a workspace and a positive bound
     assert L.moe_selftest_wait_timeout(None, 256, 1000, None) == B.MOE_ERR_INVALID_ARG
     assert L.moe_selftest_wait_timeout(fake, 256, 0, None) == B.MOE_ERR_INVALID_ARG
