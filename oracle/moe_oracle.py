@@ -17,7 +17,8 @@ Sources (web pages, cited by title and section):
         section "How it works": eq. 12 (residual form), the SwiGLU equation,
         the "Routing" paragraph and the "Packed forward (official)" paragraph.
 * [L2]  "Lesson 2 - From the Dense FFN to a Layer of Experts" (fanfani.net),
-        section 2 (boxed MoE equation) and section 4 (shared experts equation).
+        section 1 (dense FFN with phi), section 2 (expert definition and the
+        boxed MoE equation) and section 4 (shared experts equation).
 
 Everything is computed in float64 from the exact input values (bf16 inputs
 are widened exactly by the caller). No intermediate is rounded. Library
@@ -40,7 +41,9 @@ again in the design notes):
   arithmetic; ``moe_forward_dense_loop`` restates it and a test checks it.
 * Sigmoid mode always renormalises over the winners ([DS] "Routing").
 * W1 sits inside SiLU, W3 is the multiplier, W2 projects down ([DS] SwiGLU
-  equation); experts carry no bias vectors.
+  equation); SwiGLU experts carry no bias vectors. The generic experts of
+  [L2] section 2 (``gelu_ffn``) carry b1 and b2 and use the exact erf GELU;
+  their gate scales the whole expert output, b2 included.
 * The block returns shared + routed, without the residual ([DS] eq. 12 and
   the note under it).
 """
@@ -60,6 +63,7 @@ __all__ = [
     "silu", "swiglu_hidden", "swiglu_ffn", "expert_outputs", "moe_forward", "moe_forward_dense_loop",
     "expert_counts_offsets", "permutation_rows", "near_tie_tokens",
     "balance_target", "update_bias", "routing_entropy",
+    "gelu", "gelu_ffn", "expert_outputs_gelu", "moe_forward_gelu",
 ]
 
 
@@ -405,3 +409,54 @@ def routing_entropy(counts) -> float:
         return 0.0
     p = c[c > 0] / total
     return float(-(p * np.log(p)).sum())
+
+
+# ---------------------------------------------------------------------------
+# Generic experts: bias vectors and a GELU nonlinearity
+# ---------------------------------------------------------------------------
+
+def gelu(z) -> np.ndarray:
+    """GELU(z) = z * Phi(z), Phi the standard normal CDF = (1 + erf(z/sqrt 2))/2.
+
+    [L2] section 1 names GELU as the FFN nonlinearity phi without fixing a
+    form; this is the exact (erf) definition, not the tanh approximation.
+    ``math.erf`` is the library primitive, applied element by element.
+    """
+    z = _f64(z)
+    erf = np.vectorize(math.erf, otypes=[np.float64])
+    return 0.5 * z * (1.0 + erf(z / math.sqrt(2.0)))
+
+
+def gelu_ffn(u, w1, b1, w2, b2) -> np.ndarray:
+    """E_i(u) = W2 phi(W1 u + b1) + b2 with phi = GELU, row-wise over u.
+
+    [L2] section 2, the expert definition: W1 in R^{f x d}, b1 in R^f,
+    W2 in R^{d x f}, b2 in R^d. u: (n, d). Returns (n, d).
+    """
+    u = _f64(u)
+    return gelu(u @ _f64(w1).T + _f64(b1)) @ _f64(w2).T + _f64(b2)
+
+
+def expert_outputs_gelu(x, idx, gates, w1, b1, w2, b2) -> np.ndarray:
+    """MoE(x) = sum_{i in TopK(x)} g_i(x) E_i(x) with GELU experts.
+
+    [L2] section 2, boxed equation: the gate multiplies the whole expert
+    output, b2 included. No shared expert (the boxed form has none).
+    ``w1[e]`` etc. give expert e's parameters.
+    """
+    x = _f64(x)
+    idx = np.asarray(idx)
+    gates = _f64(gates)
+    y = np.zeros_like(x)
+    for e in np.unique(idx):
+        tok, slot = np.nonzero(idx == e)
+        out = gelu_ffn(x[tok], w1[e], b1[e], w2[e], b2[e])
+        np.add.at(y, tok, gates[tok, slot][:, None] * out)
+    return y
+
+
+def moe_forward_gelu(x, w_router, bias, w1, b1, w2, b2, k: int, gate_mode: int,
+                     n_groups: int = 1, topk_groups: int = 1, route_scale: float = 1.0) -> np.ndarray:
+    """Routing as in ``route`` followed by gated GELU experts ([L2] section 2)."""
+    r = route(x, w_router, bias, k, gate_mode, n_groups, topk_groups, route_scale)
+    return expert_outputs_gelu(x, r["idx"], r["gates"], w1, b1, w2, b2)

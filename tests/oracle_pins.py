@@ -408,4 +408,78 @@ def pin_balance_loop_raises_entropy():
     assert ent[-1] > 0.95 * math.log(E), ent
 
 
+# ------------------------------------------------ generic (GELU) experts
+# Standard normal CDF values from the printed normal table (textbook values).
+PHI_1 = 0.8413447460685429
+PHI_2 = 0.9772498680518208
+
+
+def pin_gelu_closed_forms():
+    _close(orc.gelu([0.0, 1.0, -1.0, 2.0]), [0.0, PHI_1, -(1.0 - PHI_1), 2.0 * PHI_2], tol=1e-15)
+    rng = np.random.default_rng(61)
+    z = rng.standard_normal(50) * 3
+    # Phi(-z) = 1 - Phi(z) gives GELU(z) - GELU(-z) = z.
+    _close(orc.gelu(z) - orc.gelu(-z), z, tol=1e-14)
+    # Far tails: GELU(z) -> z for z >> 0 and -> 0 for z << 0.
+    _close(orc.gelu([12.0, -12.0]), [12.0, 0.0], tol=1e-15)
+
+
+def pin_gelu_is_torch_exact_gelu():
+    rng = np.random.default_rng(62)
+    z = rng.standard_normal(200) * 4
+    ref = torch.nn.functional.gelu(torch.as_tensor(z, dtype=torch.float64), approximate="none").numpy()
+    _close(orc.gelu(z), ref, tol=1e-14)
+    tanh_form = torch.nn.functional.gelu(torch.as_tensor(z, dtype=torch.float64), approximate="tanh").numpy()
+    assert np.max(np.abs(orc.gelu(z) - tanh_form)) > 1e-5   # the erf form, not the tanh one
+
+
+def _torch_gelu_ffn(u, w1, b1, w2, b2):
+    u, w1, b1, w2, b2 = (torch.as_tensor(a, dtype=torch.float64) for a in (u, w1, b1, w2, b2))
+    F = torch.nn.functional
+    return F.linear(F.gelu(F.linear(u, w1, b1)), w2, b2).numpy()
+
+
+def pin_gelu_single_expert_is_dense_ffn():
+    rng = np.random.default_rng(63)
+    T, d, f = 9, 7, 5
+    x = rng.standard_normal((T, d))
+    w1, b1 = rng.standard_normal((1, f, d)), rng.standard_normal((1, f))
+    w2, b2 = rng.standard_normal((1, d, f)), rng.standard_normal((1, d))
+    ref = _torch_gelu_ffn(x, w1[0], b1[0], w2[0], b2[0])
+    _close(orc.gelu_ffn(x, w1[0], b1[0], w2[0], b2[0]), ref, tol=1e-12)
+    y = orc.moe_forward_gelu(x, rng.standard_normal((1, d)), None, w1, b1, w2, b2, 1, orc.GATE_SOFTMAX)
+    _close(y, ref, tol=1e-12)
+
+
+def pin_gelu_hand_case():
+    # Identity router and weights, expert 1 doubled; expert 1 has b1 = (1, -1)
+    # and b2 = (0.5, 0.5). Softmax, k = 1: tokens go to experts 0, 1, 0.
+    b1 = np.array([[0.0, 0.0], [1.0, -1.0]])
+    b2 = np.array([[0.0, 0.0], [0.5, 0.5]])
+    y = orc.moe_forward_gelu(HAND_X, HAND_WR, None, HAND_W1, b1, HAND_W2, b2, 1, orc.GATE_SOFTMAX)
+    want = np.array([
+        [PHI_1, 0.0],                             # GELU(1, 0)
+        [2.0 * PHI_1 + 0.5, 0.5],                 # 2 GELU((0, 1) + (1, -1)) + b2
+        [2.0 * PHI_2, -(1.0 - PHI_1)],            # GELU(2, -1)
+    ])
+    _close(y, want, tol=1e-15)
+
+
+def pin_gelu_b2_is_gated():
+    # The gate multiplies the whole expert output: shifting every b2 by c
+    # moves y by (sum of the token's gates) * c: route_scale * c in sigmoid
+    # mode, c in softmax mode.
+    rng = np.random.default_rng(64)
+    T, d, E, f = 10, 6, 8, 5
+    x = rng.standard_normal((T, d))
+    wr = rng.standard_normal((E, d))
+    w1, b1 = rng.standard_normal((E, f, d)), rng.standard_normal((E, f))
+    w2, b2 = rng.standard_normal((E, d, f)), rng.standard_normal((E, d))
+    c = rng.standard_normal(d)
+    for mode, scale in ((orc.GATE_SOFTMAX, 1.0), (orc.GATE_SIGMOID, 2.5)):
+        y0 = orc.moe_forward_gelu(x, wr, None, w1, b1, w2, b2, 3, mode, route_scale=scale)
+        y1 = orc.moe_forward_gelu(x, wr, None, w1, b1, w2, b2 + c, 3, mode, route_scale=scale)
+        _close(y1 - y0, np.tile(scale * c, (T, 1)), tol=1e-12)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]

@@ -138,6 +138,37 @@ def _target_no_k(T, k, E):
     return T / E
 
 
+def _gelu_tanh(z):
+    z = np.asarray(z, np.float64)
+    return 0.5 * z * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (z + 0.044715 * z ** 3)))
+
+
+def _gelu_cdf_only(z):
+    return _orig["gelu"](z) / np.where(np.asarray(z, np.float64) == 0, 1.0, np.asarray(z, np.float64))
+
+
+def _gelu_ffn_b1_outside(u, w1, b1, w2, b2):
+    u = np.asarray(u, np.float64)
+    h = orc.gelu(u @ np.asarray(w1, np.float64).T) + np.asarray(b1, np.float64)
+    return h @ np.asarray(w2, np.float64).T + np.asarray(b2, np.float64)
+
+
+def _gelu_ffn_no_b2(u, w1, b1, w2, b2):
+    return _orig["gelu_ffn"](u, w1, b1, w2, np.zeros_like(np.asarray(b2, np.float64)))
+
+
+def _gelu_ffn_down_transposed(u, w1, b1, w2, b2):
+    return _orig["gelu_ffn"](u, w1, b1, np.swapaxes(np.asarray(w2), -1, -2), b2)
+
+
+def _gelu_outputs_b2_ungated(x, idx, gates, w1, b1, w2, b2):
+    # b2 added once per routed expert instead of scaled by its gate.
+    y = _orig["expert_outputs_gelu"](x, idx, gates, w1, b1, w2, np.zeros_like(np.asarray(b2, np.float64)))
+    for j in range(np.asarray(idx).shape[1]):
+        y = y + np.asarray(b2, np.float64)[np.asarray(idx)[:, j]]
+    return y
+
+
 MUTATIONS = {
     "bias_update_wrong_sign": ("update_bias", _bias_update_wrong_sign),
     "entropy_in_bits": ("routing_entropy", _entropy_log2),
@@ -162,6 +193,12 @@ MUTATIONS = {
     "offsets_off_by_one": ("expert_counts_offsets", _counts_off_by_one),
     "near_ties_never_flagged": ("near_tie_tokens", _near_tie_none),
     "dense_loop_no_renorm": ("moe_forward_dense_loop", _loop_no_renorm),
+    "gelu_tanh_approximation": ("gelu", _gelu_tanh),
+    "gelu_drops_z": ("gelu", _gelu_cdf_only),
+    "gelu_b1_outside_phi": ("gelu_ffn", _gelu_ffn_b1_outside),
+    "gelu_b2_dropped": ("gelu_ffn", _gelu_ffn_no_b2),
+    "gelu_down_transposed": ("gelu_ffn", _gelu_ffn_down_transposed),
+    "gelu_b2_not_gated": ("expert_outputs_gelu", _gelu_outputs_b2_ungated),
 }
 
 
