@@ -64,6 +64,7 @@ __all__ = [
     "expert_counts_offsets", "permutation_rows", "near_tie_tokens",
     "balance_target", "update_bias", "routing_entropy",
     "gelu", "gelu_ffn", "expert_outputs_gelu", "moe_forward_gelu",
+    "silu_grad", "swiglu_ffn_backward", "gate_backward", "moe_backward",
 ]
 
 
@@ -460,3 +461,111 @@ def moe_forward_gelu(x, w_router, bias, w1, b1, w2, b2, k: int, gate_mode: int,
     """Routing as in ``route`` followed by gated GELU experts ([L2] section 2)."""
     r = route(x, w_router, bias, k, gate_mode, n_groups, topk_groups, route_scale)
     return expert_outputs_gelu(x, r["idx"], r["gates"], w1, b1, w2, b2)
+
+
+# ---------------------------------------------------------------------------
+# Backward pass of the block (training). The expert choice is piecewise
+# constant in the inputs, so gradients flow through the gates and the expert
+# FFNs only; the selection bias receives none (it is moved by the balance
+# step above, not by gradients: [CS] "Aux-loss-free balance loop").
+# ---------------------------------------------------------------------------
+
+def silu_grad(z) -> np.ndarray:
+    """d/dz [z sigma(z)] = sigma(z) (1 + z (1 - sigma(z)))."""
+    z = _f64(z)
+    with np.errstate(over="ignore"):
+        sig = 1.0 / (1.0 + np.exp(-z))
+    return sig * (1.0 + z * (1.0 - sig))
+
+
+def swiglu_ffn_backward(u, w1, w3, w2, dout):
+    """Gradients of FFN(u) = W2 (SiLU(W1 u) * W3 u) for a batch of rows u.
+
+    dout: (n, d), the gradient of the loss with respect to FFN(u).
+    Returns (du (n, d), dw1 (f, d), dw3 (f, d), dw2 (d, f)).
+    Chain rule through [DS]'s SwiGLU equation: a = W1 u, b = W3 u,
+    h = SiLU(a) * b, out = W2 h.
+    """
+    u, w1, w3, w2, dout = (_f64(v) for v in (u, w1, w3, w2, dout))
+    a = u @ w1.T
+    b = u @ w3.T
+    h = silu(a) * b
+    dw2 = dout.T @ h
+    dh = dout @ w2
+    da = dh * b * silu_grad(a)
+    db = dh * silu(a)
+    du = da @ w1 + db @ w3
+    return du, da.T @ u, db.T @ u, dw2
+
+
+def gate_backward(logits, scores, idx, gates, dgates, gate_mode: int, route_scale: float) -> np.ndarray:
+    """Gradient of the loss with respect to the router logits (T, E), given
+    the gradient with respect to the k gates of every token.
+
+    Sigmoid ([DS] "Routing"): g_j = rs * s_j / S with S the sum of the k
+    selected s, s = sigmoid(l): dL/ds_j = rs * (dg_j / S - sum_i dg_i s_i / S^2),
+    dL/dl_j = dL/ds_j * s_j (1 - s_j).
+    Softmax ([CS] "The router in code"): g_j = rs * p_j, p = softmax over the
+    k selected logits: dL/dl_j = rs * p_j (dg_j - sum_i p_i dg_i).
+    Experts that were not selected get 0.
+    """
+    T, k = idx.shape
+    E = _f64(logits).shape[1]
+    rows = np.arange(T)[:, None]
+    dg = _f64(dgates)
+    dl = np.zeros((T, E))
+    rs = float(route_scale)
+    if gate_mode == GATE_SIGMOID:
+        s = _f64(scores)[rows, idx]
+        S = s.sum(axis=1, keepdims=True)
+        ds = rs * (dg / S - (dg * s).sum(axis=1, keepdims=True) / S ** 2)
+        dl[rows, idx] = ds * s * (1.0 - s)
+    elif gate_mode == GATE_SOFTMAX:
+        p = _f64(gates) / rs
+        dl[rows, idx] = rs * p * (dg - (p * dg).sum(axis=1, keepdims=True))
+    else:
+        raise ValueError(f"unknown gate mode {gate_mode}")
+    return dl
+
+
+def moe_backward(x, w_router, bias, w1, w3, w2, k: int, gate_mode: int, dy,
+                 n_groups: int = 1, topk_groups: int = 1, route_scale: float = 1.0,
+                 ws1=None, ws3=None, ws2=None) -> dict:
+    """Gradients of <dy, MoE(x)> with respect to x and every weight.
+
+    The forward is ``moe_forward``: y_t = sum_j g_tj FFN_{e_tj}(x_t) + FFN_s(x_t).
+    Per token and slot: dL/dg_tj = <dy_t, FFN_{e_tj}(x_t)>, and the expert
+    sees dout = g_tj dy_t. The router adds dL/dl @ w_router to dx and
+    dL/dl^T x to its weight. Returns a dict with dx, dw_router, dw1, dw3, dw2
+    (stacked per expert; zero for unchosen experts), dws1, dws3, dws2 (None
+    without a shared expert), and the intermediates dgates, dlogits, idx, gates.
+    """
+    x = _f64(x)
+    dy = _f64(dy)
+    r = route(x, w_router, bias, k, gate_mode, n_groups, topk_groups, route_scale)
+    idx, gates = r["idx"], r["gates"]
+    T, d = x.shape
+    E = _f64(w_router).shape[0]
+    dx = np.zeros_like(x)
+    dgates = np.zeros_like(gates)
+    w1s, w3s, w2s = _f64(w1), _f64(w3), _f64(w2)
+    dw1, dw3, dw2 = np.zeros_like(w1s), np.zeros_like(w3s), np.zeros_like(w2s)
+    for e in np.unique(idx):
+        tok, slot = np.nonzero(idx == e)
+        out = swiglu_ffn(x[tok], w1s[e], w3s[e], w2s[e])
+        dgates[tok, slot] = (dy[tok] * out).sum(axis=1)
+        g = gates[tok, slot][:, None]
+        du, g1, g3, g2 = swiglu_ffn_backward(x[tok], w1s[e], w3s[e], w2s[e], g * dy[tok])
+        np.add.at(dx, tok, du)
+        dw1[e] += g1
+        dw3[e] += g3
+        dw2[e] += g2
+    dws1 = dws3 = dws2 = None
+    if ws1 is not None:
+        du, dws1, dws3, dws2 = swiglu_ffn_backward(x, ws1, ws3, ws2, dy)
+        dx += du
+    dlogits = gate_backward(r["logits"], r["scores"], idx, gates, dgates, gate_mode, route_scale)
+    dx += dlogits @ _f64(w_router)
+    dw_router = dlogits.T @ x
+    return dict(dx=dx, dw_router=dw_router, dw1=dw1, dw3=dw3, dw2=dw2, dws1=dws1, dws3=dws3,
+                dws2=dws2, dgates=dgates, dlogits=dlogits, idx=idx, gates=gates)

@@ -482,4 +482,129 @@ def pin_gelu_b2_is_gated():
         _close(y1 - y0, np.tile(scale * c, (T, 1)), tol=1e-12)
 
 
+# ---------------------------------------------------------------- backward
+def _bwd_case(rng, gate_mode, T=7, d=5, E=6, k=2, f=3, shared=4, n_groups=1, topk_groups=1):
+    c = _random_case(rng, T=T, d=d, E=E, f=f, shared=shared)
+    c.update(bias=rng.uniform(-0.2, 0.2, E), dy=rng.standard_normal((T, d)), k=k, mode=gate_mode,
+             n_groups=n_groups, topk_groups=topk_groups, rs=2.5 if gate_mode == orc.GATE_SIGMOID else 1.0)
+    return c
+
+
+def _loss(c, **override):
+    a = dict(c)
+    a.update(override)
+    y = orc.moe_forward(a["x"], a["wr"], a["bias"], a["w1"], a["w3"], a["w2"], a["k"], a["mode"],
+                        a["n_groups"], a["topk_groups"], a["rs"], a["ws1"], a["ws3"], a["ws2"])
+    idx = orc.route(a["x"], a["wr"], a["bias"], a["k"], a["mode"], a["n_groups"], a["topk_groups"],
+                    a["rs"])["idx"]
+    return float((np.asarray(a["dy"]) * y).sum()), idx
+
+
+def _bwd(c):
+    return orc.moe_backward(c["x"], c["wr"], c["bias"], c["w1"], c["w3"], c["w2"], c["k"], c["mode"], c["dy"],
+                            c["n_groups"], c["topk_groups"], c["rs"], c["ws1"], c["ws3"], c["ws2"])
+
+
+def pin_backward_finite_differences():
+    # Central differences of the (pinned) forward: the gradient's definition,
+    # exact up to O(h^2) while the expert choice does not move.
+    h = 1e-5
+    for seed, mode, ng, tg in ((71, orc.GATE_SIGMOID, 3, 2), (72, orc.GATE_SOFTMAX, 1, 1)):
+        rng = np.random.default_rng(seed)
+        c = _bwd_case(rng, mode, n_groups=ng, topk_groups=tg)
+        g = _bwd(c)
+        _, idx0 = _loss(c)
+        names = {"x": "dx", "wr": "dw_router", "w1": "dw1", "w3": "dw3", "w2": "dw2",
+                 "ws1": "dws1", "ws3": "dws3", "ws2": "dws2"}
+        for p, gname in names.items():
+            base = np.asarray(c[p], dtype=np.float64)
+            num = np.zeros_like(base)
+            for pos in np.ndindex(base.shape):
+                plus, minus = base.copy(), base.copy()
+                plus[pos] += h
+                minus[pos] -= h
+                lp, ip = _loss(c, **{p: plus})
+                lm, im = _loss(c, **{p: minus})
+                assert np.array_equal(ip, idx0) and np.array_equal(im, idx0), (p, pos)
+                num[pos] = (lp - lm) / (2 * h)
+            _close(g[gname], num, tol=1e-7)
+
+
+def _torch_moe_loss(c, idx):
+    """Independent fp64 torch statement of <dy, MoE(x)> for a fixed expert choice."""
+    t = lambda a: torch.tensor(np.asarray(a, dtype=np.float64), requires_grad=True)
+    P = {n: t(c[n]) for n in ("x", "wr", "w1", "w3", "w2", "ws1", "ws3", "ws2")}
+    F = torch.nn.functional
+    logits = P["x"] @ P["wr"].T
+    ii = torch.as_tensor(idx)
+    sel = torch.gather(logits, 1, ii)
+    if c["mode"] == orc.GATE_SIGMOID:
+        s = torch.sigmoid(sel)
+        gates = c["rs"] * s / s.sum(dim=1, keepdim=True)
+    else:
+        gates = c["rs"] * torch.softmax(sel, dim=1)
+    y = F.linear(F.silu(F.linear(P["x"], P["ws1"])) * F.linear(P["x"], P["ws3"]), P["ws2"])
+    for t_ in range(idx.shape[0]):
+        for j in range(idx.shape[1]):
+            e = int(idx[t_, j])
+            u = P["x"][t_]
+            o = P["w2"][e] @ (F.silu(P["w1"][e] @ u) * (P["w3"][e] @ u))
+            y = y + F.pad((gates[t_, j] * o)[None, :], (0, 0, t_, idx.shape[0] - t_ - 1))
+    loss = (torch.as_tensor(np.asarray(c["dy"])) * y).sum()
+    loss.backward()
+    return {n: P[n].grad.numpy() for n in P}
+
+
+def pin_backward_matches_torch_autograd():
+    names = {"x": "dx", "wr": "dw_router", "w1": "dw1", "w3": "dw3", "w2": "dw2",
+             "ws1": "dws1", "ws3": "dws3", "ws2": "dws2"}
+    for seed, mode in ((73, orc.GATE_SIGMOID), (74, orc.GATE_SOFTMAX)):
+        rng = np.random.default_rng(seed)
+        c = _bwd_case(rng, mode, T=9, d=6, E=8, k=3, f=4, shared=5)
+        g = _bwd(c)
+        ref = _torch_moe_loss(c, g["idx"])
+        for p, gname in names.items():
+            _close(g[gname], ref[p], tol=1e-12)
+
+
+def pin_silu_grad():
+    z = np.linspace(-8, 8, 41)
+    zt = torch.tensor(z, requires_grad=True)
+    torch.nn.functional.silu(zt).sum().backward()
+    _close(orc.silu_grad(z), zt.grad.numpy(), tol=1e-14)
+    _close(orc.silu_grad([0.0]), [0.5], tol=1e-15)
+
+
+def pin_constant_gate_gradient_moves_no_logit():
+    # Gates of a token sum to route_scale whatever the logits (both modes), so
+    # a gate gradient equal on all k slots has zero logit gradient.
+    rng = np.random.default_rng(75)
+    for mode, rs in ((orc.GATE_SIGMOID, 2.5), (orc.GATE_SOFTMAX, 1.0)):
+        c = _random_case(rng, T=10, E=8)
+        r = orc.route(c["x"], c["wr"], None, 3, mode, route_scale=rs)
+        dg = np.repeat(rng.standard_normal((10, 1)), 3, axis=1)
+        dl = orc.gate_backward(r["logits"], r["scores"], r["idx"], r["gates"], dg, mode, rs)
+        _close(dl, np.zeros_like(dl), tol=1e-14)
+
+
+def pin_single_expert_backward_is_dense():
+    # E = 1, k = 1, softmax: the gate is identically 1, the router gets no
+    # gradient and dx is the dense SwiGLU's input gradient (torch autograd).
+    rng = np.random.default_rng(76)
+    T, d, f = 6, 5, 4
+    x, dy = rng.standard_normal((T, d)), rng.standard_normal((T, d))
+    w1, w3, w2 = rng.standard_normal((1, f, d)), rng.standard_normal((1, f, d)), rng.standard_normal((1, d, f))
+    g = orc.moe_backward(x, rng.standard_normal((1, d)), None, w1, w3, w2, 1, orc.GATE_SOFTMAX, dy)
+    _close(g["dw_router"], np.zeros((1, d)), tol=1e-15)
+    xt = torch.tensor(x, requires_grad=True)
+    ws = [torch.tensor(w[0], requires_grad=True) for w in (w1, w3, w2)]
+    F = torch.nn.functional
+    y = F.linear(F.silu(F.linear(xt, ws[0])) * F.linear(xt, ws[1]), ws[2])
+    (torch.as_tensor(dy) * y).sum().backward()
+    _close(g["dx"], xt.grad.numpy(), tol=1e-12)
+    _close(g["dw1"][0], ws[0].grad.numpy(), tol=1e-12)
+    _close(g["dw3"][0], ws[1].grad.numpy(), tol=1e-12)
+    _close(g["dw2"][0], ws[2].grad.numpy(), tol=1e-12)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]

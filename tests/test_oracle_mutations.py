@@ -169,6 +169,51 @@ def _gelu_outputs_b2_ungated(x, idx, gates, w1, b1, w2, b2):
     return y
 
 
+def _silu_grad_sigma_only(z):
+    return 1.0 / (1.0 + np.exp(-np.asarray(z, np.float64)))
+
+
+def _swiglu_bwd_da_db_swapped(u, w1, w3, w2, dout):
+    du, g1, g3, g2 = _orig["swiglu_ffn_backward"](u, w1, w3, w2, dout)
+    return du, g3, g1, g2
+
+
+def _swiglu_bwd_no_up_factor(u, w1, w3, w2, dout):
+    # da forgets the multiplier b = W3 u.
+    u, w1, w3, w2, dout = (np.asarray(v, np.float64) for v in (u, w1, w3, w2, dout))
+    a, b = u @ w1.T, u @ w3.T
+    h = orc.silu(a) * b
+    dh = dout @ w2
+    da = dh * orc.silu_grad(a)
+    db = dh * orc.silu(a)
+    return da @ w1 + db @ w3, da.T @ u, db.T @ u, dout.T @ h
+
+
+def _gate_bwd_no_sigmoid_factor(logits, scores, idx, gates, dgates, gate_mode, route_scale):
+    dl = _orig["gate_backward"](logits, scores, idx, gates, dgates, gate_mode, route_scale)
+    if gate_mode == orc.GATE_SIGMOID:
+        s = np.asarray(scores, np.float64)
+        with np.errstate(divide="ignore", invalid="ignore"):
+            dl = np.where(dl != 0, dl / (s * (1 - s)), 0.0)
+    return dl
+
+
+def _gate_bwd_no_centering(logits, scores, idx, gates, dgates, gate_mode, route_scale):
+    T = idx.shape[0]
+    rows = np.arange(T)[:, None]
+    dl = np.zeros(np.asarray(logits).shape)
+    dl[rows, idx] = np.asarray(gates, np.float64) * np.asarray(dgates, np.float64)
+    return dl
+
+
+def _moe_bwd_no_router(*a, **kw):
+    g = _orig["moe_backward"](*a, **kw)
+    x = np.asarray(a[0], np.float64)
+    g["dx"] = g["dx"] - g["dlogits"] @ np.asarray(a[1], np.float64)
+    g["dw_router"] = np.zeros_like(g["dw_router"])
+    return g
+
+
 MUTATIONS = {
     "bias_update_wrong_sign": ("update_bias", _bias_update_wrong_sign),
     "entropy_in_bits": ("routing_entropy", _entropy_log2),
@@ -199,6 +244,12 @@ MUTATIONS = {
     "gelu_b2_dropped": ("gelu_ffn", _gelu_ffn_no_b2),
     "gelu_down_transposed": ("gelu_ffn", _gelu_ffn_down_transposed),
     "gelu_b2_not_gated": ("expert_outputs_gelu", _gelu_outputs_b2_ungated),
+    "silu_grad_sigma_only": ("silu_grad", _silu_grad_sigma_only),
+    "swiglu_bwd_dw1_dw3_swapped": ("swiglu_ffn_backward", _swiglu_bwd_da_db_swapped),
+    "swiglu_bwd_no_up_factor": ("swiglu_ffn_backward", _swiglu_bwd_no_up_factor),
+    "gate_bwd_no_sigmoid_factor": ("gate_backward", _gate_bwd_no_sigmoid_factor),
+    "gate_bwd_no_centering": ("gate_backward", _gate_bwd_no_centering),
+    "backward_drops_router": ("moe_backward", _moe_bwd_no_router),
 }
 
 
