@@ -164,7 +164,7 @@ def stage_work(cfg, counts):
     rows, srows = T * k, (T if fs else 0)
     w = {}
     w["route"] = dict(bytes=(T * d + E * d) * es + T * k * 8 + T * E * 4 * 2, flops=2.0 * T * E * d)
-    w["permute"] = dict(bytes=(T * d + rows * d) * es + rows * 8, flops=0.0)
+    w["permute"] = dict(bytes=(T * d + rows * d) * es + rows * 8 + T * k * 4, flops=0.0)
     w["gate_up"] = dict(bytes=(touched * 2 * f * d + 2 * fs * d) * es + (rows * d + srows * d) * es
                         + (rows * f + srows * fs) * es,
                         flops=4.0 * (rows * f + srows * fs) * d)
@@ -195,6 +195,75 @@ def traffic_for(workload, stage):
         return e["bytes_per_launch"]
     except Exception:
         return None
+
+
+def measure_gelu_experts(B, cfg, inp, counts, stream, reps):
+    """moe_forward_gelu (generic experts W2 GELU(W1 u + b1) + b2, no shared
+    expert) on this workload's x, router and w1/w2, timed over a CUDA graph."""
+    from mixture_experts_ffn_sigmoid_b200.inputs import make_expert_biases
+    gcfg = cfg.with_(f_shared=0)
+    dev = inp["x"].device
+    bb = make_expert_biases(gcfg, dev)
+    ws_g = B.alloc_workspace(gcfg, dev)
+    yg = torch.empty((cfg.T, cfg.d), dtype=cfg.torch_dtype, device=dev)
+
+    def fwd():   # on the current stream, so that the graph below captures it
+        B.moe_forward_gelu(gcfg, inp["x"], inp["w_router"], inp["bias"], inp["w1"], bb["b1"], inp["w2"],
+                           bb["b2"], yg, ws_g)
+
+    for _ in range(3):
+        fwd()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fwd()
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    del g
+    assert B.moe_get_device_error(ws_g) == B.MOE_OK
+    ms = e0.elapsed_time(e1) / reps
+    es = cfg.elem_bytes
+    T, d, E, k, f = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f
+    touched = int((counts > 0).sum())
+    flops = 2.0 * T * (E * d + k * 2 * d * f)
+    weight_bytes = touched * 2 * f * d * es + touched * (f + d) * 4
+    return {"workload": f"{cfg.name} routed experts as GELU FFNs with b1/b2 (no shared expert)",
+            "ms_per_step": ms, "tokens_per_s": T / (ms / 1e3),
+            "active_tflops": flops / (ms / 1e3) / 1e12,
+            "expert_weight_gbs": weight_bytes / (ms / 1e3) / 1e9, "graph_replays": reps}
+
+
+def measure_fused_permute(B, cfg, inp, idx, offsets, perm_src, inv_row, h, h_s, ws, stream, reps):
+    """The permute fused into the gate/up GEMM: maps-only permute, then the
+    GEMM gathering token rows from x (TMA gather4). Same h bytes as the
+    packed chain; timed with events like the stage breakdown."""
+    h2 = torch.empty_like(h)
+    hs2 = torch.empty_like(h_s) if h_s is not None else None
+    calls = [lambda: B.moe_permute(cfg, None, idx, offsets, None, perm_src, inv_row, ws),
+             lambda: B.moe_expert_gate_up_gather(cfg, inp["x"], perm_src, offsets, inp["w1"], inp["w3"],
+                                                 inp["ws1"], inp["ws3"], h2, hs2, ws)]
+    for _ in range(2):
+        for c in calls:
+            c()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+    for i in range(reps):
+        evs[i][0].record(stream)
+        for j, c in enumerate(calls):
+            c()
+            evs[i][j + 1].record(stream)
+    torch.cuda.synchronize()
+    assert torch.equal(h2, h), "gathered and packed gate/up disagree"
+    pm = statistics.mean(evs[i][0].elapsed_time(evs[i][1]) for i in range(reps))
+    gm = statistics.mean(evs[i][1].elapsed_time(evs[i][2]) for i in range(reps))
+    return {"permute_maps_ms": pm, "gate_up_gather_ms": gm, "fused_ms": pm + gm,
+            "note": "not used by moe_forward: slower than the packed copy plus gate/up"}
 
 
 # ---------------------------------------------------------------- oracle arm
@@ -375,6 +444,10 @@ def main():
     stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(n_stage))
                 for j, n in enumerate(names)}
     assert torch.equal(y2, y), "per-stage chain and moe_forward disagree"
+    fused = measure_fused_permute(B, cfg, inp, idx, offsets, perm_src, inv_row, h, h_s, ws, stream,
+                                  n_stage) if cfg.dtype == "bf16" else None
+    if fused is not None:
+        fused["packed_ms"] = stage_ms["permute"] + stage_ms["gate_up"]
     # ---- aux-loss-free balancing step that follows routing in training: one
     # small kernel over the E counts (launch-latency bound); timed on its own.
     bias_scratch = inp["bias"].clone() if inp["bias"] is not None else torch.zeros(E, device=dev)
@@ -398,8 +471,10 @@ def main():
     del bal_graph
     balance = {"us_per_call": b0.elapsed_time(b1) * 10.0, "entropy": ent.item(),
                "ln_E": math.log(E), "gamma": 0.15, "bound": "launch latency (E-element kernel)"}
+    gelu = measure_gelu_experts(B, cfg, inp, counts.cpu(), stream, max(3, min(args.steps, 20)))
     work, touched = stage_work(cfg, counts.cpu())
     peaks = measured_peaks()
+    gelu["expert_weight_frac_hbm"] = gelu["expert_weight_gbs"] / peaks["hbm"]
     dom = max(names, key=lambda n: stage_ms[n])
     wd = work[dom]
     t_dom = stage_ms[dom] / 1e3
@@ -496,6 +571,8 @@ def main():
                             "frac_hbm": expert_bytes / (expert_ms / 1e3) / 1e9 / peaks["hbm"]},
             "stages_ms": stage_ms,
             "balance_update": balance,
+            "gelu_experts": gelu,
+            "fused_permute_gather": fused,
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": {"value": whole_job_rate(T, world, e2e_ms), "unit": "tokens/s",

@@ -23,7 +23,9 @@
  *   [KB] "Mixture of experts and architecture families", "The router and
  *        load balancing": moe_layer(x, router, experts, k) over x: [tokens, d].
  *   [L2] "Lesson 2 - From the Dense FFN to a Layer of Experts", sections 2
- *        and 4 (routed sum; shared experts with unit weight).
+ *        and 4 (routed sum; shared experts with unit weight); sections 1-2
+ *        also define the generic expert W2 phi(W1 u + b1) + b2 (phi = GELU)
+ *        served by moe_expert_gelu / moe_forward_gelu.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -147,7 +149,10 @@ MOE_API moe_status moe_route(const moe_config* cfg, const void* x, const void* w
  *   topk_idx       [T][k]     int32   from moe_route (each row: k distinct ids)
  *   expert_offsets [E+1]      int32   from moe_route
  *   x_perm         [T*k][d]   dtype   OUT: row offsets[e] + r holds the r-th
- *                                     token (in token order) that chose e
+ *                                     token (in token order) that chose e;
+ *                                     NULL: only perm_src and inv_row are
+ *                                     written (x may then be NULL too), for
+ *                                     moe_expert_gate_up_gather
  *   perm_src       [T*k]      int32   OUT: source token of each packed row
  *   inv_row        [T][k]     int32   OUT: packed row of (token, slot)
  */
@@ -197,6 +202,28 @@ MOE_API moe_status moe_expert_gate_up(const moe_config* cfg, const void* x_perm,
                               void* h_shared, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * moe_expert_gate_up_gather - moe_expert_gate_up without the packed copy of
+ * the activations: the GEMM reads each packed row straight from x through
+ * perm_src (TMA tile::gather4, four rows per copy), so moe_permute can skip
+ * writing x_perm.  [DS] "Packed forward": gather the tokens of each expert.
+ *
+ *   x              [T][d]        bf16   activations (also the shared expert's input)
+ *   perm_src       [T*k]         int32  source token of each packed row (moe_permute)
+ *   expert_offsets, w1, w3, ws1, ws3, h, h_shared   as in moe_expert_gate_up
+ *
+ * bf16 only (MOE_ERR_UNSUPPORTED for fp32). Results are bit-identical to
+ * moe_permute + moe_expert_gate_up. It saves the permute's copy (T*k*d
+ * elements written, then read back) but fetches token rows 128 bytes per
+ * row and k-step instead of in 32-row boxes; on B200 the GEMM then runs
+ * slower by more than the copy costs, so moe_forward keeps the packed copy.
+ */
+MOE_API moe_status moe_expert_gate_up_gather(const moe_config* cfg, const void* x,
+                                     const int32_t* perm_src, const int32_t* expert_offsets,
+                                     const void* w1, const void* w3, const void* ws1,
+                                     const void* ws3, void* h, void* h_shared, void* workspace,
+                                     size_t ws_bytes, void* stream);
+
+/*
  * moe_expert_down - second half of moe_expert_swiglu: the down projection
  * W2 h of every segment.  [DS] SwiGLU equation, W2 in R^{d x f}.
  *
@@ -235,6 +262,70 @@ MOE_API moe_status moe_forward(const moe_config* cfg, const void* x, const void*
                        const float* bias, const void* w1, const void* w3, const void* w2,
                        const void* ws1, const void* ws3, const void* ws2, void* y,
                        void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * moe_expert_gelu - generic (Switch/GShard-style) experts on packed rows.
+ * [L2] section 2: E_i(u) = W2_i GELU(W1_i u + b1_i) + b2_i, the expert of
+ * section 1's dense FFN with its own weights; GELU(v) = v * Phi(v) with the
+ * standard normal CDF (the exact erf form, not the tanh approximation).
+ *
+ *   x_perm         [T*k][d]  dtype  packed rows (moe_permute's output)
+ *   expert_offsets [E+1]     int32  segment e = packed rows [off[e], off[e+1])
+ *   w1             [E][f][d] dtype  b1 [E][f] fp32 (NULL: zero)
+ *   w2             [E][d][f] dtype  b2 [E][d] fp32 (NULL: zero)
+ *   y_perm         [T*k][d]  dtype  OUT: E_e(x_perm[r]) for packed row r of segment e
+ *
+ * The hidden activation is kept in the workspace in dtype (one rounding
+ * after bias + GELU in fp32). Shared experts are not part of this form:
+ * cfg->f_shared > 0 returns MOE_ERR_UNSUPPORTED. bf16 runs on the tensor
+ * cores, fp32 on the FMA pipes.
+ */
+MOE_API moe_status moe_expert_gelu(const moe_config* cfg, const void* x_perm,
+                           const int32_t* expert_offsets, const void* w1, const float* b1,
+                           const void* w2, const float* b2, void* y_perm, void* workspace,
+                           size_t ws_bytes, void* stream);
+
+/*
+ * moe_forward_gelu - the whole block with generic experts: route (as
+ * moe_route), permute, moe_expert_gelu, combine without a shared row.
+ * [L2] section 2, boxed equation: MoE(u) = sum_{i in TopK} g_i E_i(u), the
+ * gate scaling the whole expert output, b2 included. y [T][d] dtype.
+ * cfg->f_shared must be 0 (else MOE_ERR_UNSUPPORTED).
+ */
+MOE_API moe_status moe_forward_gelu(const moe_config* cfg, const void* x, const void* w_router,
+                            const float* bias, const void* w1, const float* b1, const void* w2,
+                            const float* b2, void* y, void* workspace, size_t ws_bytes,
+                            void* stream);
+
+/*
+ * moe_backward - gradients of the block for training: given dy = dL/dy
+ * ([T][d], dtype), the gradients of L with respect to x and every weight.
+ * The expert choice is piecewise constant in the inputs, so gradients flow
+ * through the gates ([DS] "Routing": gates from the unbiased selected s,
+ * renormalised, times route_scale; [CS] "The router in code": softmax over
+ * the chosen raw scores) and the expert FFNs ([DS] SwiGLU equation); the
+ * selection bias gets none (it is moved by moe_balance_update).
+ *
+ *   x, w_router, bias, w1, w3, w2, ws1, ws3, ws2   as in moe_forward
+ *   dy        [T][d]         dtype  IN: gradient with respect to y
+ *   dx        [T][d]         dtype  OUT
+ *   dw_router [E][d]         dtype  OUT
+ *   dw1, dw3  [E][f][d]      dtype  OUT (zero for experts no token chose)
+ *   dw2       [E][d][f]      dtype  OUT
+ *   dws1, dws3 [f_shared][d], dws2 [d][f_shared]  dtype  OUT (NULL if f_shared == 0)
+ *
+ * The call recomputes the forward's routing and SwiGLU pre-activations
+ * (same kernels, same results as moe_forward), so it needs only the inputs
+ * and dy. Every accumulation is fp32; each output is rounded once to dtype.
+ * The workspace must hold moe_backward_workspace_size(cfg) bytes (larger
+ * than moe_workspace_size). T = 0 writes zero weight gradients.
+ */
+MOE_API size_t moe_backward_workspace_size(const moe_config* cfg);
+MOE_API moe_status moe_backward(const moe_config* cfg, const void* x, const void* w_router,
+                        const float* bias, const void* w1, const void* w3, const void* w2,
+                        const void* ws1, const void* ws3, const void* ws2, const void* dy, void* dx,
+                        void* dw_router, void* dw1, void* dw3, void* dw2, void* dws1, void* dws3,
+                        void* dws2, void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * moe_route_noalloc - moe_route for callers that cannot allocate device

@@ -30,8 +30,10 @@ MOE_DTYPE_F32 = 0
 MOE_DTYPE_BF16 = 1
 
 EXPORTED = ("moe_check_config", "moe_workspace_size", "moe_route", "moe_permute",
-            "moe_expert_swiglu", "moe_expert_gate_up", "moe_expert_down", "moe_combine", "moe_forward", "moe_get_device_error",
+            "moe_expert_swiglu", "moe_expert_gate_up", "moe_expert_gate_up_gather", "moe_expert_down",
+            "moe_combine", "moe_forward", "moe_get_device_error",
             "moe_selftest_wait_timeout", "moe_route_noalloc", "moe_balance_update",
+            "moe_expert_gelu", "moe_forward_gelu", "moe_backward_workspace_size", "moe_backward",
             "moe_status_string")
 
 
@@ -74,6 +76,8 @@ def lib() -> ctypes.CDLL:
             "moe_expert_swiglu": (ctypes.c_int, [cfgp, vp, i32p, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                                  vp, sz, vp]),
             "moe_expert_gate_up": (ctypes.c_int, [cfgp, vp, i32p, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+            "moe_expert_gate_up_gather": (ctypes.c_int, [cfgp, vp, i32p, i32p, vp, vp, vp, vp, vp, vp, vp,
+                                                         sz, vp]),
             "moe_expert_down": (ctypes.c_int, [cfgp, vp, i32p, vp, vp, vp, vp, vp, vp, sz, vp]),
             "moe_combine": (ctypes.c_int, [cfgp, vp, i32p, f32p, vp, vp, vp]),
             "moe_forward": (ctypes.c_int, [cfgp, vp, vp, f32p, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
@@ -81,6 +85,11 @@ def lib() -> ctypes.CDLL:
             "moe_selftest_wait_timeout": (ctypes.c_int, [vp, sz, ctypes.c_int64, vp]),
             "moe_route_noalloc": (ctypes.c_int, [cfgp, vp, vp, f32p, i32p, f32p, i32p, i32p, vp]),
             "moe_balance_update": (ctypes.c_int, [cfgp, i32p, f32p, ctypes.c_float, f32p, vp]),
+            "moe_expert_gelu": (ctypes.c_int, [cfgp, vp, i32p, vp, f32p, vp, f32p, vp, vp, sz, vp]),
+            "moe_forward_gelu": (ctypes.c_int, [cfgp, vp, vp, f32p, vp, f32p, vp, f32p, vp, vp, sz, vp]),
+            "moe_backward_workspace_size": (sz, [cfgp]),
+            "moe_backward": (ctypes.c_int, [cfgp, vp, vp, f32p, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                            vp, vp, vp, vp, sz, vp]),
             "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         }
         for name, (res, args) in sig.items():
@@ -175,6 +184,15 @@ def moe_expert_gate_up(cfg, x_perm, expert_offsets, w1, w3, x_shared, ws1, ws3, 
                                     _stream(stream)), "moe_expert_gate_up")
 
 
+def moe_expert_gate_up_gather(cfg, x, perm_src, expert_offsets, w1, w3, ws1, ws3, h, h_shared,
+                              workspace, stream=None):
+    c = _cfg(cfg)
+    _check(lib().moe_expert_gate_up_gather(ctypes.byref(c), _ptr(x), _ptr(perm_src), _ptr(expert_offsets),
+                                           _ptr(w1), _ptr(w3), _ptr(ws1), _ptr(ws3), _ptr(h),
+                                           _ptr(h_shared), _ptr(workspace), workspace.numel(),
+                                           _stream(stream)), "moe_expert_gate_up_gather")
+
+
 def moe_expert_down(cfg, h, expert_offsets, w2, h_shared, ws2, y_perm, y_shared, workspace,
                     stream=None):
     c = _cfg(cfg)
@@ -195,6 +213,44 @@ def moe_forward(cfg, x, w_router, bias, w1, w3, w2, ws1, ws3, ws2, y, workspace,
     _check(lib().moe_forward(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w1),
                              _ptr(w3), _ptr(w2), _ptr(ws1), _ptr(ws3), _ptr(ws2), _ptr(y),
                              _ptr(workspace), workspace.numel(), _stream(stream)), "moe_forward")
+
+
+def moe_expert_gelu(cfg, x_perm, expert_offsets, w1, b1, w2, b2, y_perm, workspace, stream=None):
+    """Generic experts on packed rows: y = W2 GELU(W1 x + b1) + b2 per segment."""
+    c = _cfg(cfg)
+    _check(lib().moe_expert_gelu(ctypes.byref(c), _ptr(x_perm), _ptr(expert_offsets), _ptr(w1), _ptr(b1),
+                                 _ptr(w2), _ptr(b2), _ptr(y_perm), _ptr(workspace), workspace.numel(),
+                                 _stream(stream)), "moe_expert_gelu")
+
+
+def moe_forward_gelu(cfg, x, w_router, bias, w1, b1, w2, b2, y, workspace, stream=None):
+    """The block with generic GELU experts (no shared expert)."""
+    c = _cfg(cfg)
+    _check(lib().moe_forward_gelu(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w1),
+                                  _ptr(b1), _ptr(w2), _ptr(b2), _ptr(y), _ptr(workspace),
+                                  workspace.numel(), _stream(stream)), "moe_forward_gelu")
+
+
+def backward_workspace_size(cfg) -> int:
+    c = _cfg(cfg)
+    return int(lib().moe_backward_workspace_size(ctypes.byref(c)))
+
+
+def alloc_backward_workspace(cfg, device="cuda") -> torch.Tensor:
+    n = backward_workspace_size(cfg)
+    if n == 0:
+        raise MoEError(MOE_ERR_INVALID_ARG, "moe_backward_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def moe_backward(cfg, x, w_router, bias, w1, w3, w2, ws1, ws3, ws2, dy, dx, dw_router, dw1, dw3, dw2,
+                 dws1, dws3, dws2, workspace, stream=None):
+    """Gradients of the block with respect to x and every weight, given dy."""
+    c = _cfg(cfg)
+    _check(lib().moe_backward(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w1), _ptr(w3),
+                              _ptr(w2), _ptr(ws1), _ptr(ws3), _ptr(ws2), _ptr(dy), _ptr(dx), _ptr(dw_router),
+                              _ptr(dw1), _ptr(dw3), _ptr(dw2), _ptr(dws1), _ptr(dws3), _ptr(dws2),
+                              _ptr(workspace), workspace.numel(), _stream(stream)), "moe_backward")
 
 
 def moe_route_noalloc(cfg, x, w_router, bias, topk_idx, topk_gate, expert_counts, expert_offsets,

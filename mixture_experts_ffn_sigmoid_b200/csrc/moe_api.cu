@@ -183,7 +183,8 @@ int expert_tile_n(const moe_config& c) {
 // SwiGLU inner activation of every segment: h = SiLU(x W1^T) * (x W3^T).
 moe_status enqueue_gate_up(const moe_config& c, const void* x_perm, const int* offsets, const void* w1,
                            const void* w3, const void* x_sh, const void* ws1, const void* ws3, void* h,
-                           void* h_s, uint32_t* err, cudaStream_t s) {
+                           void* h_s, uint32_t* err, cudaStream_t s, const int* gather_rows = nullptr,
+                           const void* gather_src = nullptr) {
   const bool shared = c.f_shared > 0;
   const int rows = c.T * c.k;
   if (c.dtype == MOE_DTYPE_BF16) {
@@ -207,6 +208,11 @@ moe_status enqueue_gate_up(const moe_config& c, const void* x_perm, const int* o
     g.err = err;
     g.timeout_ns = kDefaultTimeoutNs;
     g.max_routed_rows = rows;
+    if (gather_rows) {          // token rows read straight from x through the packed-row map
+      g.b_gather = gather_rows;
+      g.b_gather_src = gather_src;
+      g.b_gather_rows = c.T;
+    }
     MOE_CUDA(launch_umma_gemm(g, device_sm_count(), s));
   } else {
     SimtGemmParams g = {};
@@ -280,6 +286,306 @@ moe_status enqueue_experts(const moe_config& c, const void* x_perm, const int* o
   return enqueue_down(c, h, offsets, w2, h_s, ws2, y_perm, y_sh, err, s);
 }
 
+// Generic experts: h = GELU(x W1^T + b1), y = h W2^T + b2 (routed segments only).
+moe_status enqueue_gelu_experts(const moe_config& c, const void* x_perm, const int* offsets,
+                                const void* w1, const float* b1, const void* w2, const float* b2,
+                                void* y_perm, void* ws, cudaStream_t s) {
+  const Layout L = layout_of(c);
+  void* h = at<char>(ws, L.h);
+  uint32_t* err = at<uint32_t>(ws, L.err);
+  const int rows = c.T * c.k;
+  if (c.dtype == MOE_DTYPE_BF16) {
+    UmmaGemmParams g = {};
+    g.mode = kUmmaBiasAct;
+    g.n_routed = c.E;
+    g.offsets = offsets;
+    g.m_rows = c.f;
+    g.K = c.d;
+    g.bn_max = expert_tile_n(c);
+    g.max_inflight = inflight_for(g.bn_max);
+    g.a = w1; g.a3 = w1; g.b = x_perm;
+    g.a_rows_total = (long long)c.E * c.f;
+    g.b_rows_total = rows;
+    g.out = h; g.out_ld = c.f;
+    g.err = err;
+    g.timeout_ns = kDefaultTimeoutNs;
+    g.max_routed_rows = rows;
+    g.row_bias = b1;
+    g.act = kActGelu;
+    MOE_CUDA(launch_umma_gemm(g, device_sm_count(), s));
+    UmmaGemmParams q = g;
+    q.m_rows = c.d;
+    q.K = c.f;
+    q.a = w2; q.a3 = w2; q.b = h;
+    q.a_rows_total = (long long)c.E * c.d;
+    q.out = y_perm; q.out_ld = c.d;
+    q.row_bias = b2;
+    q.act = kActNone;
+    MOE_CUDA(launch_umma_gemm(q, device_sm_count(), s));
+  } else {
+    SimtGemmParams g = {};
+    g.dual = 0;
+    g.n_routed = c.E;
+    g.offsets = offsets;
+    g.a = x_perm; g.b1 = w1; g.out = h;
+    g.N = c.f; g.K = c.d;
+    g.max_rows = rows;
+    g.bias1 = b1;
+    g.act = kActGelu;
+    MOE_CUDA(launch_simt_gemm(c.dtype, 0, g, s));
+    SimtGemmParams q = g;
+    q.a = h; q.b1 = w2; q.out = y_perm;
+    q.N = c.d; q.K = c.f;
+    q.bias1 = b2;
+    q.act = kActNone;
+    MOE_CUDA(launch_simt_gemm(c.dtype, 0, q, s));
+  }
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------- backward
+// Regions of the backward workspace that follow the forward layout.
+struct BwdLayout {
+  size_t a, b, a_s, b_s, dyp, dhp, dhs, hg, hgs, dadb, dadbs, dgate, dl, dlb, dxp, dxs, dxr, total;
+  int f_pad, fs_pad;
+};
+
+BwdLayout bwd_layout_of(const moe_config& c) {
+  BwdLayout B;
+  size_t off = layout_of(c).total;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += (bytes + kAlign - 1) / kAlign * kAlign;
+    return o;
+  };
+  const size_t es = c.dtype == MOE_DTYPE_F32 ? 4 : 2;
+  const size_t T = (size_t)c.T, k = (size_t)c.k, E = (size_t)c.E, d = (size_t)c.d, f = (size_t)c.f;
+  const size_t fs = (size_t)c.f_shared, rows = T * k;
+  B.f_pad = (c.f + 63) / 64 * 64;
+  B.fs_pad = (c.f_shared + 63) / 64 * 64;
+  B.a = take(rows * f * es);
+  B.b = take(rows * f * es);
+  B.a_s = take(T * fs * es);
+  B.b_s = take(T * fs * es);
+  B.dyp = take(rows * d * es);
+  B.dhp = take(rows * f * 4);
+  B.dhs = take(T * fs * 4);
+  B.hg = take(rows * f * es);
+  B.hgs = take(T * fs * es);
+  B.dadb = take(rows * 2 * (size_t)B.f_pad * es);
+  B.dadbs = take(T * 2 * (size_t)B.fs_pad * es);
+  B.dgate = take(rows * 4);
+  B.dl = take(T * E * 4);
+  B.dlb = take(T * E * 2);
+  B.dxp = take(rows * d * 4);
+  B.dxs = take(fs > 0 ? T * d * 4 : 0);
+  B.dxr = take(T * d * 4);
+  B.total = off;
+  return B;
+}
+
+// C = A B^T through the strided SIMT kernel (see grad_gemm.cu for the
+// addressing); a helper to keep the call sites short.
+GradGemmParams gg(const moe_config& c, int seg_mode, int n_seg, const int* offsets) {
+  GradGemmParams g = {};
+  g.dtype = c.dtype;
+  g.seg_mode = seg_mode;
+  g.n_seg = n_seg;
+  g.offsets = offsets;
+  return g;
+}
+
+// Pre-activations a = W1 u and b = W3 u of every routed row and shared row.
+moe_status enqueue_preact(const moe_config& c, const void* x_perm, const int* offsets, const void* x,
+                          const void* w1, const void* w3, const void* ws1, const void* ws3, void* a,
+                          void* b, void* a_s, void* b_s, uint32_t* err, cudaStream_t s) {
+  const bool shared = c.f_shared > 0;
+  const int rows = c.T * c.k;
+  for (int which = 0; which < 2; ++which) {
+    const void* w = which ? w3 : w1;
+    const void* wsh = which ? ws3 : ws1;
+    void* out = which ? b : a;
+    void* out_s = which ? b_s : a_s;
+    if (c.dtype == MOE_DTYPE_BF16) {
+      UmmaGemmParams g = {};
+      g.mode = kUmmaBiasAct;
+      g.n_routed = c.E;
+      g.offsets = offsets;
+      g.m_rows = c.f;
+      g.K = c.d;
+      g.shared_rows = shared ? c.T : 0;
+      g.m_rows_s = c.f_shared;
+      g.K_s = c.d;
+      g.bn_max = expert_tile_n(c);
+      g.max_inflight = inflight_for(g.bn_max);
+      g.a = w; g.a3 = w; g.b = x_perm;
+      g.a_rows_total = (long long)c.E * c.f;
+      g.b_rows_total = rows;
+      g.a_s = wsh; g.a3_s = wsh; g.b_s = x;
+      g.out = out; g.out_ld = c.f;
+      g.out_s = out_s; g.out_s_ld = c.f_shared;
+      g.err = err;
+      g.timeout_ns = kDefaultTimeoutNs;
+      g.max_routed_rows = rows;
+      g.act = kActNone;
+      MOE_CUDA(launch_umma_gemm(g, device_sm_count(), s));
+    } else {
+      GradGemmParams g = gg(c, kSegRows, c.E, offsets);
+      g.N = c.f; g.K = c.d; g.max_rows = rows;
+      g.a = x_perm; g.a_si = c.d; g.a_sk = 1;
+      g.b = w; g.b_seg = (long long)c.f * c.d; g.b_sj = c.d; g.b_sk = 1;
+      g.c = out; g.c_si = c.f;
+      MOE_CUDA(launch_grad_gemm(g, s));
+      if (shared) {
+        GradGemmParams q = gg(c, kSegRows, 1, nullptr);
+        q.N = c.f_shared; q.K = c.d; q.max_rows = c.T;
+        q.a = x; q.a_si = c.d; q.a_sk = 1;
+        q.b = wsh; q.b_sj = c.d; q.b_sk = 1;
+        q.c = out_s; q.c_si = c.f_shared;
+        MOE_CUDA(launch_grad_gemm(q, s));
+      }
+    }
+  }
+  return MOE_OK;
+}
+
+moe_status enqueue_backward(const moe_config& c, const void* x, const void* w_router, const float* bias,
+                            const void* w1, const void* w3, const void* w2, const void* ws1,
+                            const void* ws3, const void* ws2, const void* dy, void* dx, void* dw_router,
+                            void* dw1, void* dw3, void* dw2, void* dws1, void* dws3, void* dws2,
+                            void* ws, cudaStream_t s) {
+  const Layout L = layout_of(c);
+  const BwdLayout Bw = bwd_layout_of(c);
+  const bool shared = c.f_shared > 0;
+  const int rows = c.T * c.k;
+  const long long d = c.d, f = c.f, fs = c.f_shared, E = c.E;
+  const int fp = Bw.f_pad, fsp = Bw.fs_pad;
+  uint32_t* err = at<uint32_t>(ws, L.err);
+  int* idx = at<int>(ws, L.idx);
+  float* gate = at<float>(ws, L.gate);
+  int* offsets = at<int>(ws, L.offsets);
+  int* inv_row = at<int>(ws, L.inv_row);
+  int* perm_src = at<int>(ws, L.perm_src);
+  char* x_perm = at<char>(ws, L.x_perm);
+  char* dyp = at<char>(ws, Bw.dyp);
+  const int nsm = device_sm_count();
+  // Forward state: routing, packed x, packed dy, pre-activations.
+  MOE_TRY(enqueue_route(c, x, w_router, bias, idx, gate, at<int>(ws, L.counts), offsets, ws, s));
+  MOE_CUDA(launch_permute(c.dtype, x, idx, offsets, at<int>(ws, L.cbase), c.T, c.d, c.E, c.k, x_perm,
+                          perm_src, inv_row, nsm, s, true));
+  MOE_CUDA(launch_permute(c.dtype, dy, idx, offsets, at<int>(ws, L.cbase), c.T, c.d, c.E, c.k, dyp,
+                          perm_src, inv_row, nsm, s, true));
+  MOE_TRY(enqueue_preact(c, x_perm, offsets, x, w1, w3, ws1, ws3, at<char>(ws, Bw.a), at<char>(ws, Bw.b),
+                         at<char>(ws, Bw.a_s), at<char>(ws, Bw.b_s), err, s));
+  // dh' = W2^T dy per packed row (gate not applied), and the shared expert's.
+  {
+    GradGemmParams g = gg(c, kSegRows, c.E, offsets);
+    g.c_f32 = 1;
+    g.N = c.f; g.K = c.d; g.max_rows = rows;
+    g.a = dyp; g.a_si = d; g.a_sk = 1;
+    g.b = w2; g.b_seg = d * f; g.b_sj = 1; g.b_sk = f;
+    g.c = at<char>(ws, Bw.dhp); g.c_si = f;
+    MOE_CUDA(launch_grad_gemm(g, s));
+    if (shared) {
+      GradGemmParams q = gg(c, kSegRows, 1, nullptr);
+      q.c_f32 = 1;
+      q.N = c.f_shared; q.K = c.d; q.max_rows = c.T;
+      q.a = dy; q.a_si = d; q.a_sk = 1;
+      q.b = ws2; q.b_sj = 1; q.b_sk = fs;
+      q.c = at<char>(ws, Bw.dhs); q.c_si = fs;
+      MOE_CUDA(launch_grad_gemm(q, s));
+    }
+  }
+  // SwiGLU backward: dgate, hg = g h, [da | db].
+  float* dgate = at<float>(ws, Bw.dgate);
+  MOE_CUDA(launch_swiglu_bwd(c.dtype, at<char>(ws, Bw.a), at<char>(ws, Bw.b), at<float>(ws, Bw.dhp), inv_row,
+                             gate, dgate, at<char>(ws, Bw.hg), at<char>(ws, Bw.dadb), rows, c.f, fp, s));
+  if (shared)
+    MOE_CUDA(launch_swiglu_bwd(c.dtype, at<char>(ws, Bw.a_s), at<char>(ws, Bw.b_s), at<float>(ws, Bw.dhs),
+                               nullptr, nullptr, nullptr, at<char>(ws, Bw.hgs), at<char>(ws, Bw.dadbs), c.T,
+                               c.f_shared, fsp, s));
+  // Gates -> router logits.
+  float* dl = at<float>(ws, Bw.dl);
+  MOE_CUDA(launch_gate_bwd(at<float>(ws, L.logits), idx, gate, dgate, dl, at<char>(ws, Bw.dlb), c.T, c.E,
+                           c.k, c.gate_mode, c.route_scale, s));
+  // Input gradients: dx_perm = da W1 + db W3 per packed row; shared; router.
+  const size_t es = c.dtype == MOE_DTYPE_F32 ? 4 : 2;
+  for (int which = 0; which < 2; ++which) {
+    GradGemmParams g = gg(c, kSegRows, c.E, offsets);
+    g.c_f32 = 1;
+    g.accumulate = which;
+    g.N = c.d; g.K = c.f; g.max_rows = rows;
+    g.a = at<char>(ws, Bw.dadb) + (size_t)which * fp * es; g.a_si = 2LL * fp; g.a_sk = 1;
+    g.b = which ? w3 : w1; g.b_seg = f * d; g.b_sj = 1; g.b_sk = d;
+    g.c = at<char>(ws, Bw.dxp); g.c_si = d;
+    MOE_CUDA(launch_grad_gemm(g, s));
+    if (shared) {
+      GradGemmParams q = gg(c, kSegRows, 1, nullptr);
+      q.c_f32 = 1;
+      q.accumulate = which;
+      q.N = c.d; q.K = c.f_shared; q.max_rows = c.T;
+      q.a = at<char>(ws, Bw.dadbs) + (size_t)which * fsp * es; q.a_si = 2LL * fsp; q.a_sk = 1;
+      q.b = which ? ws3 : ws1; q.b_sj = 1; q.b_sk = d;
+      q.c = at<char>(ws, Bw.dxs); q.c_si = d;
+      MOE_CUDA(launch_grad_gemm(q, s));
+    }
+  }
+  {
+    GradGemmParams q = gg(c, kSegRows, 1, nullptr);
+    q.a_f32 = 1; q.c_f32 = 1;
+    q.N = c.d; q.K = c.E; q.max_rows = c.T;
+    q.a = dl; q.a_si = E; q.a_sk = 1;
+    q.b = w_router; q.b_sj = 1; q.b_sk = d;
+    q.c = at<char>(ws, Bw.dxr); q.c_si = d;
+    MOE_CUDA(launch_grad_gemm(q, s));
+  }
+  MOE_CUDA(launch_unpermute_sum(c.dtype, at<float>(ws, Bw.dxp), inv_row, shared ? at<float>(ws, Bw.dxs) : nullptr,
+                                at<float>(ws, Bw.dxr), dx, c.T, c.d, c.k, s));
+  // Weight gradients, each a sum over the segment's tokens.
+  for (int which = 0; which < 2; ++which) {         // dW1, dW3 [E][f][d]
+    GradGemmParams g = gg(c, kSegK, c.E, offsets);
+    g.M = c.f; g.N = c.d;
+    g.a = at<char>(ws, Bw.dadb) + (size_t)which * fp * es; g.a_si = 1; g.a_sk = 2LL * fp;
+    g.b = x_perm; g.b_sj = 1; g.b_sk = d;
+    g.c = which ? dw3 : dw1; g.c_seg = f * d; g.c_si = d;
+    MOE_CUDA(launch_grad_gemm(g, s));
+    if (shared) {
+      GradGemmParams q = gg(c, kSegK, 1, nullptr);
+      q.M = c.f_shared; q.N = c.d; q.K = c.T;
+      q.a = at<char>(ws, Bw.dadbs) + (size_t)which * fsp * es; q.a_si = 1; q.a_sk = 2LL * fsp;
+      q.b = x; q.b_sj = 1; q.b_sk = d;
+      q.c = which ? dws3 : dws1; q.c_si = d;
+      MOE_CUDA(launch_grad_gemm(q, s));
+    }
+  }
+  {                                                  // dW2 [E][d][f]
+    GradGemmParams g = gg(c, kSegK, c.E, offsets);
+    g.M = c.d; g.N = c.f;
+    g.a = dyp; g.a_si = 1; g.a_sk = d;
+    g.b = at<char>(ws, Bw.hg); g.b_sj = 1; g.b_sk = f;
+    g.c = dw2; g.c_seg = d * f; g.c_si = f;
+    MOE_CUDA(launch_grad_gemm(g, s));
+    if (shared) {
+      GradGemmParams q = gg(c, kSegK, 1, nullptr);
+      q.M = c.d; q.N = c.f_shared; q.K = c.T;
+      q.a = dy; q.a_si = 1; q.a_sk = d;
+      q.b = at<char>(ws, Bw.hgs); q.b_sj = 1; q.b_sk = fs;
+      q.c = dws2; q.c_si = fs;
+      MOE_CUDA(launch_grad_gemm(q, s));
+    }
+  }
+  {                                                  // dW_router [E][d]
+    GradGemmParams q = gg(c, kSegK, 1, nullptr);
+    q.a_f32 = 1;
+    q.M = c.E; q.N = c.d; q.K = c.T;
+    q.a = dl; q.a_si = 1; q.a_sk = E;
+    q.b = x; q.b_sj = 1; q.b_sk = d;
+    q.c = dw_router; q.c_si = d;
+    MOE_CUDA(launch_grad_gemm(q, s));
+  }
+  return MOE_OK;
+}
+
 moe_status clear_error_word(void* ws, cudaStream_t s) {
   MOE_CUDA(cudaMemsetAsync(at<char>(ws, 0), 0, kAlign, s));
   return MOE_OK;
@@ -330,12 +636,15 @@ moe_status moe_permute(const moe_config* cfg, const void* x, const int32_t* topk
   const moe_config& c = *cfg;
   MOE_TRY(check_ws(c, workspace, ws_bytes));
   if (c.T == 0) return MOE_OK;
-  MOE_TRY(need(x));
-  MOE_TRY(need(x_perm));
   MOE_TRY(need4(topk_idx));
   MOE_TRY(need4(expert_offsets));
   MOE_TRY(need4(perm_src));
   MOE_TRY(need4(inv_row));
+  const bool copy = x_perm != nullptr;     // NULL: write the maps only
+  if (copy) {
+    MOE_TRY(need(x));
+    MOE_TRY(need(x_perm));
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   MOE_TRY(clear_error_word(workspace, s));
   const Layout L = layout_of(c);
@@ -344,7 +653,7 @@ moe_status moe_permute(const moe_config* cfg, const void* x, const int32_t* topk
   MOE_CUDA(launch_chunk_scan(at<int>(workspace, L.ccount), nch, c.E, at<int>(workspace, L.cbase),
                              at<int>(workspace, L.counts), s));
   MOE_CUDA(launch_permute(c.dtype, x, topk_idx, expert_offsets, at<int>(workspace, L.cbase), c.T, c.d,
-                          c.E, c.k, x_perm, perm_src, inv_row, device_sm_count(), s));
+                          c.E, c.k, x_perm, perm_src, inv_row, device_sm_count(), s, copy));
   return MOE_OK;
 }
 
@@ -398,6 +707,36 @@ moe_status moe_expert_gate_up(const moe_config* cfg, const void* x_perm, const i
   MOE_TRY(clear_error_word(workspace, s));
   return enqueue_gate_up(c, x_perm, expert_offsets, w1, w3, x_shared, ws1, ws3, h, h_shared,
                          at<uint32_t>(workspace, 0), s);
+}
+
+moe_status moe_expert_gate_up_gather(const moe_config* cfg, const void* x, const int32_t* perm_src,
+                                     const int32_t* expert_offsets, const void* w1, const void* w3,
+                                     const void* ws1, const void* ws3, void* h, void* h_shared,
+                                     void* workspace, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_config(cfg));
+  const moe_config& c = *cfg;
+  if (c.dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+  MOE_TRY(check_ws(c, workspace, ws_bytes));
+  if (c.T == 0) return MOE_OK;
+  MOE_TRY(need(x));
+  MOE_TRY(need4(perm_src));
+  MOE_TRY(need4(expert_offsets));
+  MOE_TRY(need(w1));
+  MOE_TRY(need(w3));
+  MOE_TRY(need(h));
+  if (c.f_shared > 0) {
+    MOE_TRY(need(ws1));
+    MOE_TRY(need(ws3));
+    MOE_TRY(need(h_shared));
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  MOE_TRY(clear_error_word(workspace, s));
+  const Layout L = layout_of(c);
+  // The routed B tensor map still needs a valid source; the workspace's packed
+  // region is never read on this path.
+  return enqueue_gate_up(c, at<char>(workspace, L.x_perm), expert_offsets, w1, w3,
+                         c.f_shared > 0 ? x : nullptr, ws1, ws3, h, h_shared,
+                         at<uint32_t>(workspace, 0), s, perm_src, x);
 }
 
 moe_status moe_expert_down(const moe_config* cfg, const void* h, const int32_t* expert_offsets,
@@ -465,9 +804,13 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
   float* gate = at<float>(ws, L.gate);
   int* offsets = at<int>(ws, L.offsets);
   MOE_TRY(enqueue_route(c, x, w_router, bias, idx, gate, at<int>(ws, L.counts), offsets, ws, s));
+  // Packed copy of the token rows, then GEMMs over contiguous segments. (The
+  // gate/up GEMM can instead gather rows from x with TMA gather4, see
+  // moe_expert_gate_up_gather; on B200 that costs more GEMM time than the
+  // copy it saves, so the block uses the packed copy.)
   MOE_CUDA(launch_permute(c.dtype, x, idx, offsets, at<int>(ws, L.cbase), c.T, c.d, c.E, c.k,
                           at<char>(ws, L.x_perm), at<int>(ws, L.perm_src), at<int>(ws, L.inv_row),
-                          device_sm_count(), s));
+                          device_sm_count(), s, true));
   const bool shared = c.f_shared > 0;
   void* y_s = shared ? at<char>(ws, L.y_s) : nullptr;
   MOE_TRY(enqueue_experts(c, at<char>(ws, L.x_perm), offsets, w1, w3, w2, shared ? x : nullptr, ws1,
@@ -475,6 +818,107 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
   MOE_CUDA(launch_combine(c.dtype, at<char>(ws, L.y_perm), at<int>(ws, L.inv_row), gate, y_s, y, c.T,
                           c.d, c.k, device_sm_count(), s));
   return MOE_OK;
+}
+
+moe_status moe_expert_gelu(const moe_config* cfg, const void* x_perm, const int32_t* expert_offsets,
+                           const void* w1, const float* b1, const void* w2, const float* b2,
+                           void* y_perm, void* workspace, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_config(cfg));
+  const moe_config& c = *cfg;
+  if (c.f_shared > 0) return MOE_ERR_UNSUPPORTED;
+  MOE_TRY(check_ws(c, workspace, ws_bytes));
+  if (c.T == 0) return MOE_OK;
+  MOE_TRY(need(x_perm));
+  MOE_TRY(need4(expert_offsets));
+  MOE_TRY(need(w1));
+  MOE_TRY(need(w2));
+  MOE_TRY(need(y_perm));
+  if (b1) MOE_TRY(need4(b1));
+  if (b2) MOE_TRY(need4(b2));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  MOE_TRY(clear_error_word(workspace, s));
+  return enqueue_gelu_experts(c, x_perm, expert_offsets, w1, b1, w2, b2, y_perm, workspace, s);
+}
+
+moe_status moe_forward_gelu(const moe_config* cfg, const void* x, const void* w_router,
+                            const float* bias, const void* w1, const float* b1, const void* w2,
+                            const float* b2, void* y, void* workspace, size_t ws_bytes,
+                            void* stream) {
+  MOE_TRY(check_config(cfg));
+  const moe_config& c = *cfg;
+  if (c.f_shared > 0) return MOE_ERR_UNSUPPORTED;
+  MOE_TRY(check_ws(c, workspace, ws_bytes));
+  if (c.T == 0) return MOE_OK;
+  MOE_TRY(need(x));
+  MOE_TRY(need(w_router));
+  if (bias) MOE_TRY(need4(bias));
+  MOE_TRY(need(w1));
+  MOE_TRY(need(w2));
+  MOE_TRY(need(y));
+  if (b1) MOE_TRY(need4(b1));
+  if (b2) MOE_TRY(need4(b2));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const Layout L = layout_of(c);
+  void* ws = workspace;
+  MOE_TRY(clear_error_word(ws, s));
+  int* idx = at<int>(ws, L.idx);
+  float* gate = at<float>(ws, L.gate);
+  int* offsets = at<int>(ws, L.offsets);
+  MOE_TRY(enqueue_route(c, x, w_router, bias, idx, gate, at<int>(ws, L.counts), offsets, ws, s));
+  MOE_CUDA(launch_permute(c.dtype, x, idx, offsets, at<int>(ws, L.cbase), c.T, c.d, c.E, c.k,
+                          at<char>(ws, L.x_perm), at<int>(ws, L.perm_src), at<int>(ws, L.inv_row),
+                          device_sm_count(), s, true));
+  MOE_TRY(enqueue_gelu_experts(c, at<char>(ws, L.x_perm), offsets, w1, b1, w2, b2,
+                               at<char>(ws, L.y_perm), ws, s));
+  MOE_CUDA(launch_combine(c.dtype, at<char>(ws, L.y_perm), at<int>(ws, L.inv_row), gate, nullptr, y,
+                          c.T, c.d, c.k, device_sm_count(), s));
+  return MOE_OK;
+}
+
+size_t moe_backward_workspace_size(const moe_config* cfg) {
+  if (check_config(cfg) != MOE_OK) return 0;
+  return bwd_layout_of(*cfg).total;
+}
+
+moe_status moe_backward(const moe_config* cfg, const void* x, const void* w_router, const float* bias,
+                        const void* w1, const void* w3, const void* w2, const void* ws1, const void* ws3,
+                        const void* ws2, const void* dy, void* dx, void* dw_router, void* dw1, void* dw3,
+                        void* dw2, void* dws1, void* dws3, void* dws2, void* workspace, size_t ws_bytes,
+                        void* stream) {
+  MOE_TRY(check_config(cfg));
+  const moe_config& c = *cfg;
+  MOE_TRY(need(workspace));
+  if (ws_bytes < bwd_layout_of(c).total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (c.T == 0) {
+    // No tokens: every weight gradient is zero.
+    MOE_TRY(need(dw_router)); MOE_TRY(need(dw1)); MOE_TRY(need(dw3)); MOE_TRY(need(dw2));
+    const size_t es = c.dtype == MOE_DTYPE_F32 ? 4 : 2;
+    MOE_CUDA(cudaMemsetAsync(dw_router, 0, (size_t)c.E * c.d * es, s));
+    MOE_CUDA(cudaMemsetAsync(dw1, 0, (size_t)c.E * c.f * c.d * es, s));
+    MOE_CUDA(cudaMemsetAsync(dw3, 0, (size_t)c.E * c.f * c.d * es, s));
+    MOE_CUDA(cudaMemsetAsync(dw2, 0, (size_t)c.E * c.d * c.f * es, s));
+    if (c.f_shared > 0) {
+      MOE_TRY(need(dws1)); MOE_TRY(need(dws3)); MOE_TRY(need(dws2));
+      MOE_CUDA(cudaMemsetAsync(dws1, 0, (size_t)c.f_shared * c.d * es, s));
+      MOE_CUDA(cudaMemsetAsync(dws3, 0, (size_t)c.f_shared * c.d * es, s));
+      MOE_CUDA(cudaMemsetAsync(dws2, 0, (size_t)c.d * c.f_shared * es, s));
+    }
+    return MOE_OK;
+  }
+  MOE_TRY(need(x));
+  MOE_TRY(need(w_router));
+  if (bias) MOE_TRY(need4(bias));
+  MOE_TRY(need(w1)); MOE_TRY(need(w3)); MOE_TRY(need(w2));
+  MOE_TRY(need(dy)); MOE_TRY(need(dx));
+  MOE_TRY(need(dw_router)); MOE_TRY(need(dw1)); MOE_TRY(need(dw3)); MOE_TRY(need(dw2));
+  if (c.f_shared > 0) {
+    MOE_TRY(need(ws1)); MOE_TRY(need(ws3)); MOE_TRY(need(ws2));
+    MOE_TRY(need(dws1)); MOE_TRY(need(dws3)); MOE_TRY(need(dws2));
+  }
+  MOE_TRY(clear_error_word(workspace, s));
+  return enqueue_backward(c, x, w_router, bias, w1, w3, w2, ws1, ws3, ws2, dy, dx, dw_router, dw1, dw3, dw2,
+                          dws1, dws3, dws2, workspace, s);
 }
 
 moe_status moe_balance_update(const moe_config* cfg, const int32_t* expert_counts, float* bias,

@@ -34,6 +34,14 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
   return __float2bfloat16_rn(v);
 }
 
+// Expert nonlinearities after a biased linear map (generic experts).
+constexpr int kActNone = 0;
+constexpr int kActGelu = 1;
+// GELU(v) = v * Phi(v), Phi the standard normal CDF, through erf.
+__device__ __forceinline__ float gelu_erf(float v) {
+  return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f));
+}
+
 // ---------------------------------------------------------------- launchers
 // Routing (route_kernels.cu)
 struct RouteParams {
@@ -57,7 +65,7 @@ cudaError_t launch_balance_update(const int* counts, int E, long long tk, float 
 // Permute / combine (permute_kernels.cu)
 cudaError_t launch_permute(int dtype, const void* x, const int* topk_idx, const int* offsets,
                            const int* chunk_base, int T, int d, int E, int k, void* x_perm,
-                           int* perm_src, int* inv_row, int num_sms, cudaStream_t s);
+                           int* perm_src, int* inv_row, int num_sms, cudaStream_t s, bool copy);
 cudaError_t launch_combine(int dtype, const void* y_perm, const int* inv_row, const float* gate,
                            const void* y_shared, void* y, int T, int d, int k, int num_sms,
                            cudaStream_t s);
@@ -76,11 +84,41 @@ struct SimtGemmParams {
   const void* a_s; const void* b1_s; const void* b3_s; void* out_s;
   int N_s, K_s;
   int max_rows;             // upper bound on routed rows (T*k) for the grid
+  // Single GEMM only: out = act(A B1^T + bias), bias fp32 [n_routed][N] / [N_s] or null.
+  const float* bias1; const float* bias1_s;
+  int act;                  // kActNone or kActGelu
 };
 cudaError_t launch_simt_gemm(int in_dtype, int out_f32, const SimtGemmParams& p, cudaStream_t s);
 
+// Strided grouped GEMM for the backward pass (grad_gemm.cu), fp32 FMA.
+enum GradSegMode { kSegRows = 0, kSegK = 1 };
+struct GradGemmParams {
+  int dtype;                // MOE_DTYPE_*: type of B and of A/C unless a_f32 / c_f32
+  int a_f32, c_f32;         // A / C held in fp32 regardless of dtype
+  int seg_mode;             // kSegRows or kSegK
+  int n_seg;
+  const int* offsets;       // [n_seg+1] row or reduction offsets (null: one segment)
+  int M, N, K;              // kSegK: output M x N per segment; kSegRows: N columns, K reduction
+  int max_rows;             // kSegRows: upper bound on rows (grid sizing / dense segment)
+  const void* a; long long a_si, a_sk;
+  const void* b; long long b_seg, b_sj, b_sk;
+  void* c; long long c_seg, c_si;
+  int accumulate;           // C += product instead of C = product
+};
+cudaError_t launch_grad_gemm(const GradGemmParams& p, cudaStream_t s);
+
+// Backward elementwise / per-token kernels (backward_kernels.cu)
+cudaError_t launch_swiglu_bwd(int dtype, const void* a, const void* b, const float* dhp,
+                              const int* inv_row, const float* gate, float* dgate, void* hg, void* dadb,
+                              int n_rows, int f, int f_pad, cudaStream_t s);
+cudaError_t launch_gate_bwd(const float* logits, const int* idx, const float* gate, const float* dgate,
+                            float* dl, void* dl_bf16, int T, int E, int k, int gate_mode,
+                            float route_scale, cudaStream_t s);
+cudaError_t launch_unpermute_sum(int dtype, const float* dxp, const int* inv_row, const float* dxs,
+                                 const float* dxr, void* dx, int T, int d, int k, cudaStream_t s);
+
 // tcgen05 grouped GEMM (umma_gemm.cu)
-enum UmmaMode { kUmmaRouter = 0, kUmmaSwiGLU = 1, kUmmaDown = 2 };
+enum UmmaMode { kUmmaRouter = 0, kUmmaSwiGLU = 1, kUmmaDown = 2, kUmmaBiasAct = 3 };
 struct UmmaGemmParams {
   int mode;
   int n_routed;             // routed segments
@@ -101,6 +139,15 @@ struct UmmaGemmParams {
   uint32_t* err;
   long long timeout_ns;
   int max_routed_rows;      // upper bound on routed rows (T*k) for the grid
+  // Optional gather of routed token rows: packed row r reads source row
+  // b_gather[r] of b_gather_src ([b_gather_rows][K]) instead of row r of b.
+  const int* b_gather;
+  const void* b_gather_src;
+  long long b_gather_rows;
+  // kUmmaBiasAct: out = act(acc + bias[weight row]); fp32 bias per segment
+  // ([n_routed][m_rows] routed, [m_rows_s] dense), null = no bias.
+  const float* row_bias; const float* row_bias_s;
+  int act;                  // kActNone or kActGelu
 };
 cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t s);
 cudaError_t launch_wait_timeout_selftest(uint32_t* err, long long timeout_ns, cudaStream_t s);

@@ -20,12 +20,14 @@ __device__ __forceinline__ void st16(void* p, uint4 v) { *reinterpret_cast<uint4
 
 // grid = (chunks of 32 tokens, column splits). Each block recomputes its
 // chunk's packed rows (cheap), then copies a column slice of the 32 rows to
-// their k destinations. Split 0 also writes inv_row / perm_src.
+// their k destinations. Split 0 also writes inv_row / perm_src. Without
+// `copy` only the maps are written (the GEMM then gathers rows from x).
 template <typename T>
 __global__ void __launch_bounds__(256) permute_kernel(
     const T* __restrict__ x, const int* __restrict__ idx, const int* __restrict__ offsets,
     const int* __restrict__ chunk_base, int n_tok, int d, int E, int k, T* __restrict__ x_perm,
-    int* __restrict__ perm_src, int* __restrict__ inv_row, int rows_total, int vec_per_split) {
+    int* __restrict__ perm_src, int* __restrict__ inv_row, int rows_total, int vec_per_split,
+    int copy) {
   constexpr int V = Vec16<T>::N;
   __shared__ uint32_t s_mask[kMaxExperts];
   __shared__ int s_row[kChunk * kMaxTopK];
@@ -58,6 +60,7 @@ __global__ void __launch_bounds__(256) permute_kernel(
       }
     }
   }
+  if (!copy) return;
   __syncthreads();
   const int nvec = d / V;
   const int v0 = blockIdx.y * vec_per_split;
@@ -146,12 +149,12 @@ __global__ void __launch_bounds__(128) combine_kernel(
 
 cudaError_t launch_permute(int dtype, const void* x, const int* topk_idx, const int* offsets,
                            const int* chunk_base, int T, int d, int E, int k, void* x_perm,
-                           int* perm_src, int* inv_row, int num_sms, cudaStream_t s) {
+                           int* perm_src, int* inv_row, int num_sms, cudaStream_t s, bool copy) {
   if (T <= 0) return cudaSuccess;
   const int V = dtype == MOE_DTYPE_F32 ? 4 : 8;
   const int nvec = d / V;
   const int nch = ceil_div(T, kChunk);
-  int nsplit = ceil_div(4 * num_sms, nch);
+  int nsplit = copy ? ceil_div(4 * num_sms, nch) : 1;
   if (nsplit < 1) nsplit = 1;
   if (nsplit > nvec) nsplit = nvec;
   const int vps = ceil_div(nvec, nsplit);
@@ -159,11 +162,11 @@ cudaError_t launch_permute(int dtype, const void* x, const int* topk_idx, const 
   dim3 grid(nch, nsplit);
   if (dtype == MOE_DTYPE_F32)
     permute_kernel<float><<<grid, 256, 0, s>>>((const float*)x, topk_idx, offsets, chunk_base, T, d,
-                                                E, k, (float*)x_perm, perm_src, inv_row, T * k, vps);
+                                                E, k, (float*)x_perm, perm_src, inv_row, T * k, vps, copy ? 1 : 0);
   else
     permute_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
         (const __nv_bfloat16*)x, topk_idx, offsets, chunk_base, T, d, E, k,
-        (__nv_bfloat16*)x_perm, perm_src, inv_row, T * k, vps);
+        (__nv_bfloat16*)x_perm, perm_src, inv_row, T * k, vps, copy ? 1 : 0);
   return cudaGetLastError();
 }
 

@@ -3,7 +3,9 @@
 // mantissa bits, too coarse for an fp32 path, so this kernel stays on FFMA.
 //
 //   dual:   out[r][n] = SiLU(sum_c A[r][c] B1[n][c]) * (sum_c A[r][c] B3[n][c])
-//   single: out[r][n] = sum_c A[r][c] B1[n][c]
+//   single: out[r][n] = act(sum_c A[r][c] B1[n][c] + bias[n]), act = identity or
+//           GELU, bias optional (the generic expert W2 phi(W1 u + b1) + b2 of
+//           "Lesson 2 - From the Dense FFN to a Layer of Experts", section 2)
 //
 // Segment s < n_routed covers packed rows [offsets[s], offsets[s+1]) of A and
 // uses expert s's matrices B1[s], B3[s] (N x K each). Segment n_routed, when
@@ -24,6 +26,7 @@ constexpr int TM = 64, TN = 64, TK = 16;
 struct Seg {
   const void* a; const void* b1; const void* b3; void* out;
   int row0, rows, N, K;
+  const float* bias;   // this segment's bias row [N], or null
 };
 
 template <typename TI, typename TO, bool DUAL>
@@ -42,7 +45,8 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGemmParams p) {
     if (bx < tiles) {
       sg = Seg{p.a, (const char*)p.b1 + (size_t)s * p.N * p.K * sizeof(TI),
                DUAL ? (const char*)p.b3 + (size_t)s * p.N * p.K * sizeof(TI) : nullptr,
-               p.out, r0 + bx * TM, min(TM, rows - bx * TM), p.N, p.K};
+               p.out, r0 + bx * TM, min(TM, rows - bx * TM), p.N, p.K,
+               p.bias1 ? p.bias1 + (size_t)s * p.N : nullptr};
       found = true;
       break;
     }
@@ -51,7 +55,8 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGemmParams p) {
   if (!found && p.shared_rows > 0) {
     const int tiles = (p.shared_rows + TM - 1) / TM;
     if (bx < tiles) {
-      sg = Seg{p.a_s, p.b1_s, p.b3_s, p.out_s, bx * TM, min(TM, p.shared_rows - bx * TM), p.N_s, p.K_s};
+      sg = Seg{p.a_s, p.b1_s, p.b3_s, p.out_s, bx * TM, min(TM, p.shared_rows - bx * TM), p.N_s, p.K_s,
+               p.bias1_s};
       found = true;
     }
   }
@@ -113,7 +118,12 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGemmParams p) {
       const int n = n0 + tx * 4 + j;
       if (n >= sg.N) continue;
       float v = acc1[i][j];
-      if (DUAL) v = (v / (1.0f + expf(-v))) * acc3[i][j];
+      if (DUAL) {
+        v = (v / (1.0f + expf(-v))) * acc3[i][j];
+      } else {
+        if (sg.bias) v += sg.bias[n];
+        if (p.act == kActGelu) v = gelu_erf(v);
+      }
       out[(size_t)(sg.row0 + r) * sg.N + n] = from_f32<TO>(v);
     }
   }

@@ -7,6 +7,9 @@
 //   kUmmaSwiGLU: h[r][m] = SiLU(sum_c W1_e[m][c] x[r][c]) * (sum_c W3_e[m][c] x[r][c])
 //   kUmmaDown:   y[r][m] = sum_c W2_e[m][c] h[r][c]
 //   kUmmaRouter: l[t][e] = sum_c Wr[e][c] x[t][c]            (fp32 out)
+//   kUmmaBiasAct: o[r][m] = act(sum_c W_e[m][c] u[r][c] + b_e[m]), act = GELU or
+//                identity (the generic expert of "Lesson 2 - From the Dense FFN
+//                to a Layer of Experts", section 2: W2 phi(W1 u + b1) + b2)
 //
 // for every packed row r of every segment. Segment e < n_routed is expert e
 // over packed rows [offsets[e], offsets[e+1]); segment n_routed is the dense
@@ -64,8 +67,10 @@ constexpr int NUM_THREADS = 192;
 constexpr int TMEM_COLS = 512;
 constexpr int NSLOT = 8;            // barrier pairs of the slot ring
 constexpr int SMEM_LIMIT = 232448;  // 227 KB of dynamic shared memory per block
+constexpr int HDR_BYTES = 2048;     // barriers, TMEM slot, slot records, gathered token rows
 
-// Shared-memory plan of one launch: [header page | tile tables | slot ring],
+// Shared-memory plan of one launch: [header (barriers, gathered token rows) |
+// tile tables | slot ring],
 // the ring 1024-byte aligned (128-byte swizzle atoms).
 struct SmemPlan {
   int table_bytes, ring_bytes, total;
@@ -74,8 +79,8 @@ struct SmemPlan {
 __host__ __device__ inline SmemPlan smem_plan(int n_routed, int nseg) {
   SmemPlan sp;
   sp.table_bytes = ((nseg + 1 + n_routed + 1) * 4 + 1023) / 1024 * 1024;
-  sp.ring_bytes = (SMEM_LIMIT - 1024 - 1024 - sp.table_bytes) / 1024 * 1024;
-  sp.total = 1024 + 1024 + sp.table_bytes + sp.ring_bytes;
+  sp.ring_bytes = (SMEM_LIMIT - 1024 - HDR_BYTES - sp.table_bytes) / 1024 * 1024;
+  sp.total = 1024 + HDR_BYTES + sp.table_bytes + sp.ring_bytes;
   return sp;
 }
 
@@ -253,6 +258,24 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(cluster_bar)
       : "memory");
 }
+// Four arbitrary rows (row0..row3) of a 2-D tensor, one 128-byte box row
+// each, written as four consecutive swizzled rows at dst (box height 1).
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* tm, int c0, int r0, int r1,
+                                            int r2, int r3, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tma_gather4_pair(uint32_t dst, const CUtensorMap* tm, int c0, int r0,
+                                                 int r1, int r2, int r3, uint32_t cluster_bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(cluster_bar)
+      : "memory");
+}
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t slot_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot_smem),
                "r"(ncols)
@@ -306,10 +329,14 @@ template <int MODE> struct Kind;
 template <> struct Kind<kUmmaRouter> { static constexpr int A_TILES = 1; static constexpr int ACC_STAGES = 2; };
 template <> struct Kind<kUmmaSwiGLU> { static constexpr int A_TILES = 2; static constexpr int ACC_STAGES = 1; };
 template <> struct Kind<kUmmaDown>   { static constexpr int A_TILES = 2; static constexpr int ACC_STAGES = 1; };
+template <> struct Kind<kUmmaBiasAct> { static constexpr int A_TILES = 2; static constexpr int ACC_STAGES = 1; };
+
+// Modes whose tile is two consecutive 128-row blocks of one weight matrix.
+__host__ __device__ constexpr bool two_blocks(int mode) { return mode == kUmmaDown || mode == kUmmaBiasAct; }
 
 // Weight rows covered by one tile (all CTAs of the group together).
 __host__ __device__ constexpr int tile_rows(int mode, bool pair) {
-  return (mode == kUmmaDown ? 256 : 128) * (pair ? 2 : 1);
+  return (two_blocks(mode) ? 256 : 128) * (pair ? 2 : 1);
 }
 
 struct Tile {
@@ -360,6 +387,10 @@ __device__ __forceinline__ Tile decode_tile(const UmmaGemmParams& p, const int* 
 // Token rows this CTA stages for a tile, and how many TMA boxes that takes.
 struct TokenSlice {
   int n_valid, n_mma, row, nbox;
+  int rows_gather;   // rows staged by gather4 (routed tiles of a gathered B), else 0
+  __device__ __forceinline__ uint32_t bytes() const {
+    return rows_gather > 0 ? (uint32_t)rows_gather * (BK * 2) : (uint32_t)nbox * BOX_BYTES;
+  }
 };
 template <bool PAIR>
 __device__ __forceinline__ TokenSlice token_slice(const UmmaGemmParams& p, const Tile& t, uint32_t rank) {
@@ -369,6 +400,8 @@ __device__ __forceinline__ TokenSlice token_slice(const UmmaGemmParams& p, const
   const int mine = PAIR ? ts.n_mma / 2 : ts.n_valid;
   ts.row = t.b_row0 + t.tt * p.bn_max + (PAIR ? (int)rank * (ts.n_mma / 2) : 0);
   ts.nbox = (mine + BOX_N - 1) / BOX_N;
+  // Gathered tiles stage exactly the rows the MMA reads (a multiple of 8).
+  ts.rows_gather = (p.b_gather && !t.dense) ? (PAIR ? ts.n_mma / 2 : ts.n_mma) : 0;
   return ts;
 }
 
@@ -377,13 +410,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA3,
                      const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmAs,
                      const __grid_constant__ CUtensorMap tmA3s, const __grid_constant__ CUtensorMap tmBs,
-                     const UmmaGemmParams p) {
+                     const __grid_constant__ CUtensorMap tmG, const UmmaGemmParams p) {
   using KD = Kind<MODE>;
   constexpr int A_TILES = KD::A_TILES;
   constexpr int ACC_STAGES = KD::ACC_STAGES;
   constexpr int WROWS = tile_rows(MODE, PAIR);
   // Row offset of weight block a (0 or 1) inside a tile, for CTA rank r.
-  constexpr int BLOCK_STEP = (MODE == kUmmaDown) ? (PAIR ? 256 : 128) : 0;
+  constexpr int BLOCK_STEP = two_blocks(MODE) ? (PAIR ? 256 : 128) : 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -400,9 +433,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   volatile uint32_t* abort_flag = tmem_slot + 1;
   uint32_t* fl_off = tmem_slot + 2;             // producer's record of slots in flight
   uint32_t* fl_size = fl_off + NSLOT;
-  int* s_start = reinterpret_cast<int*>(smem + 1024);
+  int* s_rows = reinterpret_cast<int*>(smem + 1024);    // token rows of the current tile (gather)
+  int* s_start = reinterpret_cast<int*>(smem + HDR_BYTES);
   int* s_off = s_start + (nseg + 1);
-  uint8_t* ring = smem + 1024 + sp.table_bytes;
+  uint8_t* ring = smem + HDR_BYTES + sp.table_bytes;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = PAIR ? cluster_rank() : 0u;
@@ -437,6 +471,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     tmap_prefetch(&tmA); tmap_prefetch(&tmB); tmap_prefetch(&tmAs); tmap_prefetch(&tmBs);
     if (MODE == kUmmaSwiGLU) { tmap_prefetch(&tmA3); tmap_prefetch(&tmA3s); }
+    if (p.b_gather) tmap_prefetch(&tmG);
   }
   __syncthreads();
   // Tiles per segment -> exclusive prefix s_start[0..nseg] (warp 0).
@@ -483,8 +518,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const CUtensorMap* mA3 = t.dense ? &tmA3s : &tmA3;
       const CUtensorMap* mB = t.dense ? &tmBs : &tmB;
       const int a_row = (t.dense ? 0 : t.seg * p.m_rows) + t.wt * WROWS + (int)rank * BM;
-      const uint32_t bytes = A_TILES * A_BYTES + ts.nbox * BOX_BYTES;
+      const uint32_t bytes = A_TILES * A_BYTES + ts.bytes();
       const int nk = ceil_div(t.K, BK);
+      if (ts.rows_gather > 0) {
+        // Token rows of this CTA's part of the tile: packed rows map to source
+        // tokens through b_gather; rows past the segment reuse its first token.
+        const int r_base = t.b_row0 + t.tt * p.bn_max + (PAIR ? (int)rank * ts.rows_gather : 0);
+        const int r_end = t.b_row0 + t.rows;
+        const int pad = p.b_gather[t.b_row0];
+        for (int j = 0; j < ts.rows_gather; ++j) {
+          const int r = r_base + j;
+          s_rows[j] = r < r_end ? p.b_gather[r] : pad;
+        }
+      }
       for (int kb = 0; kb < nk; ++kb) {
         // Make room: the barrier pair and the bytes of the new slot must be free.
         const uint32_t off_new = cur.peek(bytes, cap);
@@ -519,16 +565,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (leader) mbar_expect_tx(fb_local, 2 * bytes);
           tma_load_2d_pair(sb, mA, kb * BK, a_row, fb);
           if (MODE == kUmmaSwiGLU) tma_load_2d_pair(sb + A_BYTES, mA3, kb * BK, a_row, fb);
-          if (MODE == kUmmaDown) tma_load_2d_pair(sb + A_BYTES, mA, kb * BK, a_row + BLOCK_STEP, fb);
-          for (int bx = 0; bx < ts.nbox; ++bx)
-            tma_load_2d_pair(bb + bx * BOX_BYTES, mB, kb * BK, ts.row + bx * BOX_N, fb);
+          if (two_blocks(MODE)) tma_load_2d_pair(sb + A_BYTES, mA, kb * BK, a_row + BLOCK_STEP, fb);
+          if (ts.rows_gather > 0) {
+            for (int g = 0; g < ts.rows_gather; g += 4)
+              tma_gather4_pair(bb + g * (BK * 2), &tmG, kb * BK, s_rows[g], s_rows[g + 1], s_rows[g + 2],
+                               s_rows[g + 3], fb);
+          } else {
+            for (int bx = 0; bx < ts.nbox; ++bx)
+              tma_load_2d_pair(bb + bx * BOX_BYTES, mB, kb * BK, ts.row + bx * BOX_N, fb);
+          }
         } else {
           mbar_expect_tx(fb_local, bytes);
           tma_load_2d(sb, mA, kb * BK, a_row, fb_local);
           if (MODE == kUmmaSwiGLU) tma_load_2d(sb + A_BYTES, mA3, kb * BK, a_row, fb_local);
-          if (MODE == kUmmaDown) tma_load_2d(sb + A_BYTES, mA, kb * BK, a_row + BLOCK_STEP, fb_local);
-          for (int bx = 0; bx < ts.nbox; ++bx)
-            tma_load_2d(bb + bx * BOX_BYTES, mB, kb * BK, ts.row + bx * BOX_N, fb_local);
+          if (two_blocks(MODE)) tma_load_2d(sb + A_BYTES, mA, kb * BK, a_row + BLOCK_STEP, fb_local);
+          if (ts.rows_gather > 0) {
+            for (int g = 0; g < ts.rows_gather; g += 4)
+              tma_gather4(bb + g * (BK * 2), &tmG, kb * BK, s_rows[g], s_rows[g + 1], s_rows[g + 2],
+                          s_rows[g + 3], fb_local);
+          } else {
+            for (int bx = 0; bx < ts.nbox; ++bx)
+              tma_load_2d(bb + bx * BOX_BYTES, mB, kb * BK, ts.row + bx * BOX_N, fb_local);
+          }
         }
       }
     }
@@ -552,7 +610,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int tile = group; tile < total_tiles; tile += ngroups) {
       const Tile t = decode_tile(p, s_off, s_start, nseg, tile, WROWS);
       const TokenSlice ts = token_slice<PAIR>(p, t, 0);
-      const uint32_t bytes = A_TILES * A_BYTES + ts.nbox * BOX_BYTES;
+      const uint32_t bytes = A_TILES * A_BYTES + ts.bytes();
       const int nk = ceil_div(t.K, BK);
       if (!wait_bounded(smem_u32(&acce_bar[acc]), acc_phase ^ 1u, abort_flag, p.err, p.timeout_ns, true))
         break;
@@ -682,6 +740,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) { if (PAIR) mbar_arrive_cluster(acce); else mbar_arrive(acce); }
+      } else if (MODE == kUmmaBiasAct) {
+        // As kUmmaDown, with the weight row's bias added and the activation
+        // applied in fp32 before the one rounding to bf16.
+        const int m2 = m + BLOCK_STEP;
+        const bool m2_ok = m2 < t.mrows;
+        const float* rb = t.dense ? p.row_bias_s : p.row_bias;
+        const long long boff = t.dense ? 0 : (long long)t.seg * p.m_rows;
+        const float bias1 = (rb && m_ok) ? rb[boff + m] : 0.0f;
+        const float bias2 = (rb && m2_ok) ? rb[boff + m2] : 0.0f;
+        const bool gelu = p.act == kActGelu;
+        __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out) + r0 * ld;
+        for (int c0 = 0; c0 < n_mma; c0 += 16) {
+          uint32_t r1[16], r3[16];
+          tmem_ld16x2_wait(taddr + c0, taddr + BN_MAX + c0, r1, r3);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int col = c0 + j;
+            if (col < n_valid) {
+              float v1 = __uint_as_float(r1[j]) + bias1;
+              float v2 = __uint_as_float(r3[j]) + bias2;
+              if (gelu) { v1 = gelu_erf(v1); v2 = gelu_erf(v2); }
+              if (m_ok) o[(long long)col * ld + m] = __float2bfloat16_rn(v1);
+              if (m2_ok) o[(long long)col * ld + m2] = __float2bfloat16_rn(v2);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) { if (PAIR) mbar_arrive_cluster(acce); else mbar_arrive(acce); }
       } else {
         float* o = reinterpret_cast<float*>(out) + r0 * ld;
         for (int c0 = 0; c0 < n_mma; c0 += 16) {
@@ -775,11 +862,12 @@ cudaError_t ensure_smem_attr() {
 template <int MODE, bool PAIR>
 cudaError_t launch_mode(const CUtensorMap& tA, const CUtensorMap& tA3, const CUtensorMap& tB,
                         const CUtensorMap& tAs, const CUtensorMap& tA3s, const CUtensorMap& tBs,
-                        const UmmaGemmParams& p, int grid, int smem, cudaStream_t s) {
+                        const CUtensorMap& tG, const UmmaGemmParams& p, int grid, int smem,
+                        cudaStream_t s) {
   cudaError_t e = ensure_smem_attr<MODE, PAIR>();
   if (e != cudaSuccess) return e;
   if (!PAIR) {
-    umma_gemm_kernel<MODE, false><<<grid, NUM_THREADS, smem, s>>>(tA, tA3, tB, tAs, tA3s, tBs, p);
+    umma_gemm_kernel<MODE, false><<<grid, NUM_THREADS, smem, s>>>(tA, tA3, tB, tAs, tA3s, tBs, tG, p);
     return cudaGetLastError();
   }
   cudaLaunchConfig_t cfg = {};
@@ -794,7 +882,7 @@ cudaError_t launch_mode(const CUtensorMap& tA, const CUtensorMap& tA3, const CUt
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, umma_gemm_kernel<MODE, true>, tA, tA3, tB, tAs, tA3s, tBs, p);
+  return cudaLaunchKernelEx(&cfg, umma_gemm_kernel<MODE, true>, tA, tA3, tB, tAs, tA3s, tBs, tG, p);
 }
 
 }  // namespace
@@ -830,6 +918,9 @@ cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t 
     tA = tAs; tA3 = tA3s; tB = tBs;
   }
   if (!has_dense) { tAs = tA; tA3s = tA3; tBs = tB; }
+  // Gathered token rows: one-row boxes over the source activations.
+  CUtensorMap tG = tB;
+  if (p.b_gather && !make_tmap(&tG, p.b_gather_src, p.K, p.b_gather_rows, 1)) return cudaErrorInvalidValue;
 
   long long tiles = 0;
   if (p.n_routed > 0)
@@ -841,13 +932,16 @@ cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t 
   const int grid = pair ? 2 * ngroup : ngroup;
   switch (p.mode) {
     case kUmmaRouter:
-      return launch_mode<kUmmaRouter, false>(tA, tA3, tB, tAs, tA3s, tBs, p, grid, sp.total, s);
+      return launch_mode<kUmmaRouter, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s);
     case kUmmaSwiGLU:
-      return pair ? launch_mode<kUmmaSwiGLU, true>(tA, tA3, tB, tAs, tA3s, tBs, p, grid, sp.total, s)
-                  : launch_mode<kUmmaSwiGLU, false>(tA, tA3, tB, tAs, tA3s, tBs, p, grid, sp.total, s);
+      return pair ? launch_mode<kUmmaSwiGLU, true>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s)
+                  : launch_mode<kUmmaSwiGLU, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s);
     case kUmmaDown:
-      return pair ? launch_mode<kUmmaDown, true>(tA, tA3, tB, tAs, tA3s, tBs, p, grid, sp.total, s)
-                  : launch_mode<kUmmaDown, false>(tA, tA3, tB, tAs, tA3s, tBs, p, grid, sp.total, s);
+      return pair ? launch_mode<kUmmaDown, true>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s)
+                  : launch_mode<kUmmaDown, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s);
+    case kUmmaBiasAct:
+      return pair ? launch_mode<kUmmaBiasAct, true>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s)
+                  : launch_mode<kUmmaBiasAct, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s);
   }
   return cudaErrorInvalidValue;
 }

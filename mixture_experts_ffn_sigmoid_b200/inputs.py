@@ -30,6 +30,11 @@ w_router, w1, w3, ws1, ws3 ~ N(0, 1/d); w2 ~ N(0, 1/f); ws2 ~ N(0, 1/f_shared).
 Bias is fp32 (None for the workloads whose bias is 0). The values differ
 between a CPU and a CUDA generator; a parity check always copies the bytes one
 side produced to the other side.
+
+Generic (GELU) experts add two fp32 bias stacks, drawn by ``make_expert_biases``
+from a second generator seeded with seed + 1000 (so the draws above do not
+move): b1 [E][f] then b2 [E][d], both N(0, 0.5^2). The weights of such an
+expert are the w1 and w2 drawn above (w3 is unused).
 """
 from __future__ import annotations
 
@@ -143,6 +148,15 @@ def make_inputs(cfg: MoEConfig, device="cpu", seed: int = 0,
     else:
         out["ws1"] = out["ws3"] = out["ws2"] = None
     return out
+
+
+def make_expert_biases(cfg: MoEConfig, device="cpu", seed: int = 0) -> dict:
+    """b1 [E][f] and b2 [E][d], fp32, for generic experts (recipe above)."""
+    device = torch.device(device)
+    g = torch.Generator(device=device)
+    g.manual_seed(seed + 1000)
+    return {"b1": _normal(g, (cfg.E, cfg.f), 0.5, torch.float32, device),
+            "b2": _normal(g, (cfg.E, cfg.d), 0.5, torch.float32, device)}
 
 
 def sample_token_ids(T: int, n: int, seed: int = 1) -> torch.Tensor:

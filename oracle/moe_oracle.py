@@ -530,7 +530,7 @@ def gate_backward(logits, scores, idx, gates, dgates, gate_mode: int, route_scal
 
 def moe_backward(x, w_router, bias, w1, w3, w2, k: int, gate_mode: int, dy,
                  n_groups: int = 1, topk_groups: int = 1, route_scale: float = 1.0,
-                 ws1=None, ws3=None, ws2=None) -> dict:
+                 ws1=None, ws3=None, ws2=None, idx=None) -> dict:
     """Gradients of <dy, MoE(x)> with respect to x and every weight.
 
     The forward is ``moe_forward``: y_t = sum_j g_tj FFN_{e_tj}(x_t) + FFN_s(x_t).
@@ -539,10 +539,18 @@ def moe_backward(x, w_router, bias, w1, w3, w2, k: int, gate_mode: int, dy,
     dL/dl^T x to its weight. Returns a dict with dx, dw_router, dw1, dw3, dw2
     (stacked per expert; zero for unchosen experts), dws1, dws3, dws2 (None
     without a shared expert), and the intermediates dgates, dlogits, idx, gates.
+
+    ``idx`` (T, k), when given, fixes the expert choice (ascending ids per
+    token) instead of this routing's own; the gates are then those of that
+    choice. The gradient is defined for a fixed choice, so a caller whose
+    selection differs only on near-tie tokens can compare against it.
     """
     x = _f64(x)
     dy = _f64(dy)
     r = route(x, w_router, bias, k, gate_mode, n_groups, topk_groups, route_scale)
+    if idx is not None:
+        r["idx"] = np.asarray(idx, dtype=np.int64)
+        r["gates"] = gate_values(r["logits"], r["scores"], r["idx"], gate_mode, route_scale)
     idx, gates = r["idx"], r["gates"]
     T, d = x.shape
     E = _f64(w_router).shape[0]

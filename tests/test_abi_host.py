@@ -146,6 +146,21 @@ def test_host_side_rejections_before_any_launch():
     assert L.moe_balance_update(ctypes.byref(cfg), fake, None, ctypes.c_float(0.1), None, None) == B.MOE_ERR_INVALID_ARG
     assert L.moe_balance_update(ctypes.byref(cfg), fake, fake, ctypes.c_float(-0.1), None, None) == B.MOE_ERR_INVALID_ARG
     assert L.moe_balance_update(ctypes.byref(cfg), None, fake, ctypes.c_float(0.1), None, None) == B.MOE_ERR_INVALID_ARG
+    # generic (GELU) experts: no shared-expert form
+    assert L.moe_forward_gelu(ctypes.byref(cs), fake, fake, None, fake, None, fake, None, fake, fake, ns,
+                              None) == B.MOE_ERR_UNSUPPORTED
+    assert L.moe_expert_gelu(ctypes.byref(cs), fake, fake, fake, None, fake, None, fake, fake, ns,
+                             None) == B.MOE_ERR_UNSUPPORTED
+    assert L.moe_forward_gelu(ctypes.byref(cfg), fake, fake, None, None, None, fake, None, fake, fake,
+                              nbytes, None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_expert_gelu(ctypes.byref(cfg), fake, fake, fake, ctypes.c_void_p(0x10002), fake, None,
+                             fake, fake, nbytes, None) == B.MOE_ERR_MISALIGNED
+    # backward: its workspace is larger than the forward's
+    nb = L.moe_backward_workspace_size(ctypes.byref(cfg))
+    assert nb > nbytes
+    args = [fake] * 18
+    assert L.moe_backward(ctypes.byref(cfg), *args, fake, nb - 1, None) == B.MOE_ERR_WORKSPACE_TOO_SMALL
+    assert L.moe_backward(ctypes.byref(bad), *args, fake, nb, None) == B.MOE_ERR_INVALID_ARG
     # the timeout self-test needs a workspace and a positive bound
     assert L.moe_selftest_wait_timeout(None, 256, 1000, None) == B.MOE_ERR_INVALID_ARG
     assert L.moe_selftest_wait_timeout(fake, 256, 0, None) == B.MOE_ERR_INVALID_ARG

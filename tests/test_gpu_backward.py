@@ -1,0 +1,137 @@
+"""Backward pass on the GPU (moe_backward) against the oracle's chain rule.
+
+The oracle's gradients are pinned to central differences of the forward and
+to torch autograd (``oracle_pins``). The GPU recomputes the routing in fp32;
+where that choice differs from the oracle's on a near-tie token, the oracle
+is evaluated on the GPU's choice (the gradient is defined for a fixed
+choice; the choice itself is checked by the routing tests).
+
+Tolerances: fp32 storage, relative L2 <= 1e-5 per gradient tensor; bf16
+storage (bf16 pre-activations, hg and [da | db] rounded once, fp32
+accumulation), relative L2 <= 2e-2 and max-abs <= 5e-2 * RMS, like the
+forward. A weight gradient of an expert no token chose must be exactly 0.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.moe_oracle as orc
+from mixture_experts_ffn_sigmoid_b200 import binding as B
+from mixture_experts_ffn_sigmoid_b200.inputs import GATE_SIGMOID, MoEConfig, make_inputs
+
+import gpu_harness as H
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    "tiny_fp32": MoEConfig("tiny_bwd_f32", T=64, d=128, E=8, k=2, f=256, dtype="f32"),
+    "ragged_fp32": MoEConfig("ragged_bwd_f32", T=77, d=200, E=12, k=3, f=72, dtype="f32",
+                             gate_mode=GATE_SIGMOID, route_scale=2.5, f_shared=40, bias="uniform"),
+    "ragged_bf16": MoEConfig("ragged_bwd", T=77, d=200, E=12, k=3, f=72, gate_mode=GATE_SIGMOID,
+                             route_scale=1.0, f_shared=40, bias="uniform"),
+    "grouped_bf16": MoEConfig("grouped_bwd", T=300, d=256, E=32, k=4, f=384, gate_mode=GATE_SIGMOID,
+                              n_groups=8, topk_groups=4, route_scale=2.5, f_shared=256, bias="uniform"),
+    "softmax_bf16": MoEConfig("softmax_bwd", T=200, d=192, E=16, k=2, f=136),
+}
+
+
+def _dy(cfg, seed=9):
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    return torch.randn((cfg.T, cfg.d), generator=g, device="cuda").to(cfg.torch_dtype)
+
+
+def gpu_backward(cfg, inp, dy):
+    dt, dev = cfg.torch_dtype, "cuda"
+    nan = float("nan")
+    out = dict(dx=torch.full((cfg.T, cfg.d), nan, dtype=dt, device=dev),
+               dw_router=torch.full((cfg.E, cfg.d), nan, dtype=dt, device=dev),
+               dw1=torch.full((cfg.E, cfg.f, cfg.d), nan, dtype=dt, device=dev),
+               dw3=torch.full((cfg.E, cfg.f, cfg.d), nan, dtype=dt, device=dev),
+               dw2=torch.full((cfg.E, cfg.d, cfg.f), nan, dtype=dt, device=dev))
+    sh = cfg.f_shared > 0
+    out["dws1"] = torch.full((cfg.f_shared, cfg.d), nan, dtype=dt, device=dev) if sh else None
+    out["dws3"] = torch.full((cfg.f_shared, cfg.d), nan, dtype=dt, device=dev) if sh else None
+    out["dws2"] = torch.full((cfg.d, cfg.f_shared), nan, dtype=dt, device=dev) if sh else None
+    ws = B.alloc_backward_workspace(cfg)
+    B.moe_backward(cfg, inp["x"], inp["w_router"], inp["bias"], inp["w1"], inp["w3"], inp["w2"], inp["ws1"],
+                   inp["ws3"], inp["ws2"], dy, out["dx"], out["dw_router"], out["dw1"], out["dw3"], out["dw2"],
+                   out["dws1"], out["dws3"], out["dws2"], ws)
+    assert B.moe_get_device_error(ws) == B.MOE_OK
+    return out
+
+
+def oracle_backward(cfg, inp, dy, idx=None):
+    return orc.moe_backward(H.f64(inp["x"]), H.f64(inp["w_router"]), H.f64(inp["bias"]), H.f64(inp["w1"]),
+                            H.f64(inp["w3"]), H.f64(inp["w2"]), cfg.k, cfg.gate_mode, H.f64(dy), cfg.n_groups,
+                            cfg.topk_groups, cfg.route_scale, H.f64(inp["ws1"]), H.f64(inp["ws3"]),
+                            H.f64(inp["ws2"]), idx=idx)
+
+
+@pytest.fixture(scope="module")
+def results():
+    out = {}
+    for name, cfg in CASES.items():
+        inp = H.gpu_inputs(cfg)
+        dy = _dy(cfg)
+        got = gpu_backward(cfg, inp, dy)
+        gr = H.gpu_route(cfg, inp)
+        rep = H.check_route(cfg, H.oracle_route(cfg, inp), gr)
+        ref = oracle_backward(cfg, inp, dy, idx=gr["idx"].cpu().numpy())
+        out[name] = (cfg, inp, dy, got, ref, rep)
+    return out
+
+
+NAMES = ["dx", "dw_router", "dw1", "dw3", "dw2", "dws1", "dws3", "dws2"]
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+@pytest.mark.parametrize("grad", NAMES)
+def test_gradient_matches_oracle(results, name, grad):
+    cfg, inp, dy, got, ref, rep = results[name]
+    if ref[grad] is None:
+        assert got[grad] is None
+        return
+    H.compare_outputs(cfg, H.f64(got[grad]), ref[grad], grad)
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_unchosen_experts_get_zero_weight_gradient(results, name):
+    cfg, inp, dy, got, ref, rep = results[name]
+    chosen = np.zeros(cfg.E, dtype=bool)
+    chosen[np.unique(ref["idx"])] = True
+    for g in ("dw1", "dw3", "dw2"):
+        w = got[g].float()
+        for e in np.nonzero(~chosen)[0]:
+            assert torch.count_nonzero(w[int(e)]).item() == 0, (g, e)
+
+
+def test_backward_is_deterministic():
+    cfg = CASES["grouped_bf16"]
+    inp = H.gpu_inputs(cfg)
+    dy = _dy(cfg)
+    a = gpu_backward(cfg, inp, dy)
+    b = gpu_backward(cfg, inp, dy)
+    for n in NAMES:
+        if a[n] is not None:
+            assert torch.equal(a[n], b[n]), n
+
+
+def test_backward_empty_tokens():
+    cfg = CASES["ragged_bf16"].with_(T=0)
+    inp = make_inputs(CASES["ragged_bf16"], "cuda")
+    dt = cfg.torch_dtype
+    dw = dict(dw_router=torch.full((cfg.E, cfg.d), 1.0, dtype=dt, device="cuda"),
+              dw1=torch.full((cfg.E, cfg.f, cfg.d), 1.0, dtype=dt, device="cuda"),
+              dw3=torch.full((cfg.E, cfg.f, cfg.d), 1.0, dtype=dt, device="cuda"),
+              dw2=torch.full((cfg.E, cfg.d, cfg.f), 1.0, dtype=dt, device="cuda"),
+              dws1=torch.full((cfg.f_shared, cfg.d), 1.0, dtype=dt, device="cuda"),
+              dws3=torch.full((cfg.f_shared, cfg.d), 1.0, dtype=dt, device="cuda"),
+              dws2=torch.full((cfg.d, cfg.f_shared), 1.0, dtype=dt, device="cuda"))
+    ws = B.alloc_backward_workspace(cfg)
+    B.moe_backward(cfg, None, inp["w_router"], inp["bias"], inp["w1"], inp["w3"], inp["w2"], inp["ws1"],
+                   inp["ws3"], inp["ws2"], None, None, dw["dw_router"], dw["dw1"], dw["dw3"], dw["dw2"],
+                   dw["dws1"], dw["dws3"], dw["dws2"], ws)
+    torch.cuda.synchronize()
+    for n, t in dw.items():
+        assert torch.count_nonzero(t).item() == 0, n

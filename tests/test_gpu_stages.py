@@ -154,3 +154,36 @@ def test_forward_is_deterministic(cases):
     a = H.gpu_forward(cfg, inp)
     b = H.gpu_forward(cfg, inp)
     assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("name", sorted(STAGE_CASES))
+def test_gate_up_gather_matches_packed(cases, name):
+    # Reading token rows through perm_src (TMA gather4) gives bit-identical h
+    # to reading the packed copy x_perm; maps-only permute writes the same maps.
+    cfg, inp = cases[name]
+    got, x_perm, perm_src, inv_row = _packed(cfg, inp)
+    rows = cfg.T * cfg.k
+    src2 = torch.full((rows,), -7, dtype=torch.int32, device="cuda")
+    inv2 = torch.full((cfg.T, cfg.k), -7, dtype=torch.int32, device="cuda")
+    B.moe_permute(cfg, None, got["idx"], got["offsets"], None, src2, inv2, got["ws"])
+    torch.cuda.synchronize()
+    assert torch.equal(src2, perm_src) and torch.equal(inv2, inv_row)
+    sh = cfg.f_shared > 0
+    h_a = torch.full((rows, cfg.f), float("nan"), dtype=cfg.torch_dtype, device="cuda")
+    h_b = torch.full((rows, cfg.f), float("nan"), dtype=cfg.torch_dtype, device="cuda")
+    hs_a = torch.full((cfg.T, cfg.f_shared), float("nan"), dtype=cfg.torch_dtype, device="cuda") if sh else None
+    hs_b = torch.full((cfg.T, cfg.f_shared), float("nan"), dtype=cfg.torch_dtype, device="cuda") if sh else None
+    B.moe_expert_gate_up(cfg, x_perm, got["offsets"], inp["w1"], inp["w3"], inp["x"] if sh else None,
+                         inp["ws1"], inp["ws3"], h_a, hs_a, got["ws"])
+    if cfg.dtype == "f32":
+        with pytest.raises(B.MoEError) as ei:
+            B.moe_expert_gate_up_gather(cfg, inp["x"], perm_src, got["offsets"], inp["w1"], inp["w3"],
+                                        inp["ws1"], inp["ws3"], h_b, hs_b, got["ws"])
+        assert ei.value.status == B.MOE_ERR_UNSUPPORTED
+        return
+    B.moe_expert_gate_up_gather(cfg, inp["x"], perm_src, got["offsets"], inp["w1"], inp["w3"],
+                                inp["ws1"], inp["ws3"], h_b, hs_b, got["ws"])
+    assert B.moe_get_device_error(got["ws"]) == B.MOE_OK
+    assert torch.equal(h_a, h_b)
+    if sh:
+        assert torch.equal(hs_a, hs_b)
