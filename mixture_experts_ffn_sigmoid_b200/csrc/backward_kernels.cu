@@ -71,20 +71,20 @@ __global__ void __launch_bounds__(256) swiglu_bwd_kernel(
 
 // Gate gradients -> logit gradients, one warp per token (lanes over slots).
 // dl is [T][E], zero outside the token's k experts (written here for every
-// expert, so no separate clear is needed).
+// expert, so no separate clear is needed); the optional bf16 copy is
+// [T][e_pad] with zero columns past E.
 __global__ void __launch_bounds__(256) gate_bwd_kernel(
     const float* __restrict__ logits, const int* __restrict__ idx, const float* __restrict__ gate,
-    const float* __restrict__ dgate, float* __restrict__ dl, void* __restrict__ dl_bf16, int T, int E,
-    int k, int gate_mode, float route_scale) {
+    const float* __restrict__ dgate, float* __restrict__ dl, void* __restrict__ dl_bf16, int e_pad, int T,
+    int E, int k, int gate_mode, float route_scale) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= T) return;
   const int t = warp;
   float* row = dl + (size_t)t * E;
-  __nv_bfloat16* rowb = dl_bf16 ? static_cast<__nv_bfloat16*>(dl_bf16) + (size_t)t * E : nullptr;
-  for (int e = lane; e < E; e += 32) {
-    row[e] = 0.0f;
-    if (rowb) rowb[e] = __float2bfloat16_rn(0.0f);
-  }
+  __nv_bfloat16* rowb = dl_bf16 ? static_cast<__nv_bfloat16*>(dl_bf16) + (size_t)t * e_pad : nullptr;
+  for (int e = lane; e < E; e += 32) row[e] = 0.0f;
+  if (rowb)
+    for (int e = lane; e < e_pad; e += 32) rowb[e] = __float2bfloat16_rn(0.0f);
   __syncwarp();
   // Lanes j < k hold slot j (k <= 32).
   const bool act = lane < k;
@@ -151,11 +151,11 @@ cudaError_t launch_swiglu_bwd(int dtype, const void* a, const void* b, const flo
 }
 
 cudaError_t launch_gate_bwd(const float* logits, const int* idx, const float* gate, const float* dgate,
-                            float* dl, void* dl_bf16, int T, int E, int k, int gate_mode,
+                            float* dl, void* dl_bf16, int e_pad, int T, int E, int k, int gate_mode,
                             float route_scale, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  gate_bwd_kernel<<<ceil_div(T, 8), 256, 0, s>>>(logits, idx, gate, dgate, dl, dl_bf16, T, E, k, gate_mode,
-                                                 route_scale);
+  gate_bwd_kernel<<<ceil_div(T, 8), 256, 0, s>>>(logits, idx, gate, dgate, dl, dl_bf16, e_pad, T, E, k,
+                                                 gate_mode, route_scale);
   return cudaGetLastError();
 }
 

@@ -347,7 +347,7 @@ moe_status enqueue_gelu_experts(const moe_config& c, const void* x_perm, const i
 // Regions of the backward workspace that follow the forward layout.
 struct BwdLayout {
   size_t a, b, a_s, b_s, dyp, dhp, dhs, hg, hgs, dadb, dadbs, dgate, dl, dlb, dxp, dxs, dxr, total;
-  int f_pad, fs_pad;
+  int f_pad, fs_pad, e_pad;
 };
 
 BwdLayout bwd_layout_of(const moe_config& c) {
@@ -376,7 +376,8 @@ BwdLayout bwd_layout_of(const moe_config& c) {
   B.dadbs = take(T * 2 * (size_t)B.fs_pad * es);
   B.dgate = take(rows * 4);
   B.dl = take(T * E * 4);
-  B.dlb = take(T * E * 2);
+  B.e_pad = (c.E + 7) / 8 * 8;
+  B.dlb = take(T * (size_t)B.e_pad * 2);
   B.dxp = take(rows * d * 4);
   B.dxs = take(fs > 0 ? T * d * 4 : 0);
   B.dxr = take(T * d * 4);
@@ -393,6 +394,50 @@ GradGemmParams gg(const moe_config& c, int seg_mode, int n_seg, const int* offse
   g.n_seg = n_seg;
   g.offsets = offsets;
   return g;
+}
+
+// Input-gradient GEMM on the tensor cores: out[r][m] = sum_c W[c][m] g[r][c]
+// per routed segment (W stacked [E * c_rows][m_rows]) and, when sh_rows > 0,
+// the dense segment (W_s [c_rows_s][m_rows_s]); fp32 output. w2nd / ws2nd
+// take over after k_split / k_split_s 64-wide blocks of the contraction.
+struct DgradArgs {
+  const int* offsets; int n_routed;
+  const void* g; int K; const void* w; const void* w2nd; int c_rows; int m_rows; int k_split; float* out;
+  int sh_rows; const void* g_s; int K_s; const void* w_s; const void* ws2nd; int c_rows_s; int m_rows_s;
+  int k_split_s; float* out_s;
+  int bn;
+};
+moe_status enqueue_dgrad(const DgradArgs& a, int rows, uint32_t* err, cudaStream_t s) {
+  UmmaGemmParams g = {};
+  g.mode = kUmmaDgrad;
+  g.out_f32 = 1;
+  g.n_routed = a.n_routed;
+  g.offsets = a.offsets;
+  g.m_rows = a.m_rows;
+  g.K = a.K;
+  g.shared_rows = a.sh_rows;
+  g.m_rows_s = a.m_rows_s;
+  g.K_s = a.K_s;
+  g.bn_max = a.bn;
+  g.max_inflight = inflight_for(a.bn);
+  g.a = a.w; g.a3 = a.w2nd; g.b = a.g;
+  g.a_rows_total = (long long)a.n_routed * a.c_rows;
+  g.b_rows_total = rows;
+  g.a_s = a.w_s; g.a3_s = a.ws2nd; g.b_s = a.g_s;
+  g.a_k_rows = a.c_rows; g.a_k_rows_s = a.c_rows_s;
+  g.k_split = a.k_split; g.k_split_s = a.k_split_s;
+  g.out = a.out; g.out_ld = a.m_rows;
+  g.out_s = a.out_s; g.out_s_ld = a.m_rows_s;
+  g.err = err;
+  g.timeout_ns = kDefaultTimeoutNs;
+  g.max_routed_rows = rows;
+  MOE_CUDA(launch_umma_gemm(g, device_sm_count(), s));
+  return MOE_OK;
+}
+
+int dense_tile_n(int T) {
+  const int bn = (T + 15) / 16 * 16;
+  return bn > 256 ? 256 : (bn < 16 ? 16 : bn);
 }
 
 // Pre-activations a = W1 u and b = W3 u of every routed row and shared row.
@@ -478,7 +523,20 @@ moe_status enqueue_backward(const moe_config& c, const void* x, const void* w_ro
   MOE_TRY(enqueue_preact(c, x_perm, offsets, x, w1, w3, ws1, ws3, at<char>(ws, Bw.a), at<char>(ws, Bw.b),
                          at<char>(ws, Bw.a_s), at<char>(ws, Bw.b_s), err, s));
   // dh' = W2^T dy per packed row (gate not applied), and the shared expert's.
-  {
+  const bool tc = c.dtype == MOE_DTYPE_BF16;
+  constexpr int kNoSplit = 1 << 30;
+  if (tc) {
+    DgradArgs a = {};
+    a.offsets = offsets; a.n_routed = c.E;
+    a.g = dyp; a.K = c.d; a.w = w2; a.w2nd = nullptr; a.c_rows = c.d; a.m_rows = c.f; a.k_split = kNoSplit;
+    a.out = at<float>(ws, Bw.dhp);
+    if (shared) {
+      a.sh_rows = c.T; a.g_s = dy; a.K_s = c.d; a.w_s = ws2; a.ws2nd = nullptr; a.c_rows_s = c.d;
+      a.m_rows_s = c.f_shared; a.k_split_s = kNoSplit; a.out_s = at<float>(ws, Bw.dhs);
+    }
+    a.bn = expert_tile_n(c);
+    MOE_TRY(enqueue_dgrad(a, rows, err, s));
+  } else {
     GradGemmParams g = gg(c, kSegRows, c.E, offsets);
     g.c_f32 = 1;
     g.N = c.f; g.K = c.d; g.max_rows = rows;
@@ -506,11 +564,29 @@ moe_status enqueue_backward(const moe_config& c, const void* x, const void* w_ro
                                c.f_shared, fsp, s));
   // Gates -> router logits.
   float* dl = at<float>(ws, Bw.dl);
-  MOE_CUDA(launch_gate_bwd(at<float>(ws, L.logits), idx, gate, dgate, dl, at<char>(ws, Bw.dlb), c.T, c.E,
-                           c.k, c.gate_mode, c.route_scale, s));
+  MOE_CUDA(launch_gate_bwd(at<float>(ws, L.logits), idx, gate, dgate, dl, tc ? at<char>(ws, Bw.dlb) : nullptr,
+                           Bw.e_pad, c.T, c.E, c.k, c.gate_mode, c.route_scale, s));
   // Input gradients: dx_perm = da W1 + db W3 per packed row; shared; router.
   const size_t es = c.dtype == MOE_DTYPE_F32 ? 4 : 2;
-  for (int which = 0; which < 2; ++which) {
+  if (tc) {
+    DgradArgs a = {};
+    a.offsets = offsets; a.n_routed = c.E;
+    a.g = at<char>(ws, Bw.dadb); a.K = 2 * fp; a.w = w1; a.w2nd = w3; a.c_rows = c.f; a.m_rows = c.d;
+    a.k_split = fp / 64; a.out = at<float>(ws, Bw.dxp);
+    if (shared) {
+      a.sh_rows = c.T; a.g_s = at<char>(ws, Bw.dadbs); a.K_s = 2 * fsp; a.w_s = ws1; a.ws2nd = ws3;
+      a.c_rows_s = c.f_shared; a.m_rows_s = c.d; a.k_split_s = fsp / 64; a.out_s = at<float>(ws, Bw.dxs);
+    }
+    a.bn = expert_tile_n(c);
+    MOE_TRY(enqueue_dgrad(a, rows, err, s));
+    DgradArgs r = {};
+    r.n_routed = 0;
+    r.sh_rows = c.T; r.g_s = at<char>(ws, Bw.dlb); r.K_s = Bw.e_pad; r.w_s = w_router; r.ws2nd = nullptr;
+    r.c_rows_s = c.E; r.m_rows_s = c.d; r.k_split_s = kNoSplit; r.out_s = at<float>(ws, Bw.dxr);
+    r.bn = dense_tile_n(c.T);
+    MOE_TRY(enqueue_dgrad(r, c.T, err, s));
+  }
+  for (int which = 0; which < 2 && !tc; ++which) {
     GradGemmParams g = gg(c, kSegRows, c.E, offsets);
     g.c_f32 = 1;
     g.accumulate = which;
@@ -530,7 +606,7 @@ moe_status enqueue_backward(const moe_config& c, const void* x, const void* w_ro
       MOE_CUDA(launch_grad_gemm(q, s));
     }
   }
-  {
+  if (!tc) {
     GradGemmParams q = gg(c, kSegRows, 1, nullptr);
     q.a_f32 = 1; q.c_f32 = 1;
     q.N = c.d; q.K = c.E; q.max_rows = c.T;

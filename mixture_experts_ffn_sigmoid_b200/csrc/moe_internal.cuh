@@ -112,13 +112,13 @@ cudaError_t launch_swiglu_bwd(int dtype, const void* a, const void* b, const flo
                               const int* inv_row, const float* gate, float* dgate, void* hg, void* dadb,
                               int n_rows, int f, int f_pad, cudaStream_t s);
 cudaError_t launch_gate_bwd(const float* logits, const int* idx, const float* gate, const float* dgate,
-                            float* dl, void* dl_bf16, int T, int E, int k, int gate_mode,
+                            float* dl, void* dl_bf16, int e_pad, int T, int E, int k, int gate_mode,
                             float route_scale, cudaStream_t s);
 cudaError_t launch_unpermute_sum(int dtype, const float* dxp, const int* inv_row, const float* dxs,
                                  const float* dxr, void* dx, int T, int d, int k, cudaStream_t s);
 
 // tcgen05 grouped GEMM (umma_gemm.cu)
-enum UmmaMode { kUmmaRouter = 0, kUmmaSwiGLU = 1, kUmmaDown = 2, kUmmaBiasAct = 3 };
+enum UmmaMode { kUmmaRouter = 0, kUmmaSwiGLU = 1, kUmmaDown = 2, kUmmaBiasAct = 3, kUmmaDgrad = 4 };
 struct UmmaGemmParams {
   int mode;
   int n_routed;             // routed segments
@@ -148,6 +148,12 @@ struct UmmaGemmParams {
   // ([n_routed][m_rows] routed, [m_rows_s] dense), null = no bias.
   const float* row_bias; const float* row_bias_s;
   int act;                  // kActNone or kActGelu
+  // kUmmaDgrad: a / a3 (a_s / a3_s) are stored [rows c][m_rows] with m
+  // contiguous; a_k_rows (a_k_rows_s) rows of c per segment; the first
+  // k_split (k_split_s) 64-wide k blocks read a, the rest read a3 from row 0.
+  int a_k_rows, a_k_rows_s;
+  int k_split, k_split_s;
+  int out_f32;              // kUmmaDgrad: fp32 output instead of bf16
 };
 cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t s);
 cudaError_t launch_wait_timeout_selftest(uint32_t* err, long long timeout_ns, cudaStream_t s);

@@ -10,6 +10,10 @@
 //   kUmmaBiasAct: o[r][m] = act(sum_c W_e[m][c] u[r][c] + b_e[m]), act = GELU or
 //                identity (the generic expert of "Lesson 2 - From the Dense FFN
 //                to a Layer of Experts", section 2: W2 phi(W1 u + b1) + b2)
+//   kUmmaDgrad:  o[r][m] = sum_c W_e[c][m] g[r][c]   (the transposed weight:
+//                input gradients of the backward pass; W_e is read with m
+//                contiguous, an MN-major operand; the contraction may run
+//                over two stacked weights, W for c < k_split blocks, W' after)
 //
 // for every packed row r of every segment. Segment e < n_routed is expert e
 // over packed rows [offsets[e], offsets[e+1]); segment n_routed is the dense
@@ -314,8 +318,18 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) |
          ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
+// MN-major operand, 128-byte swizzle: each 128-byte row holds 64 consecutive
+// M (or N) elements of one k; 8 k-rows form a 1024-byte atom. Tiles are
+// staged as 64 x 64 TMA boxes (8 KB), so 64-element M groups lie 8192 bytes
+// apart (leading byte offset) and 8-row k groups 1024 bytes apart (stride
+// byte offset).
+constexpr int MN_BOX_BYTES = 64 * 64 * 2;
+__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(MN_BOX_BYTES >> 4) << 16) |
+         ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
 // Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
-// K-major, N >> 3 at bit 17, M >> 4 at bit 24.
+// K-major, N >> 3 at bit 17, M >> 4 at bit 24 (bit 15 set: A is MN-major).
 __device__ __forceinline__ uint32_t idesc_bf16_f32(int m, int n) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
          ((uint32_t)(m >> 4) << 24);
@@ -330,9 +344,12 @@ template <> struct Kind<kUmmaRouter> { static constexpr int A_TILES = 1; static 
 template <> struct Kind<kUmmaSwiGLU> { static constexpr int A_TILES = 2; static constexpr int ACC_STAGES = 1; };
 template <> struct Kind<kUmmaDown>   { static constexpr int A_TILES = 2; static constexpr int ACC_STAGES = 1; };
 template <> struct Kind<kUmmaBiasAct> { static constexpr int A_TILES = 2; static constexpr int ACC_STAGES = 1; };
+template <> struct Kind<kUmmaDgrad> { static constexpr int A_TILES = 2; static constexpr int ACC_STAGES = 1; };
 
 // Modes whose tile is two consecutive 128-row blocks of one weight matrix.
-__host__ __device__ constexpr bool two_blocks(int mode) { return mode == kUmmaDown || mode == kUmmaBiasAct; }
+__host__ __device__ constexpr bool two_blocks(int mode) {
+  return mode == kUmmaDown || mode == kUmmaBiasAct || mode == kUmmaDgrad;
+}
 
 // Weight rows covered by one tile (all CTAs of the group together).
 __host__ __device__ constexpr int tile_rows(int mode, bool pair) {
@@ -518,6 +535,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const CUtensorMap* mA3 = t.dense ? &tmA3s : &tmA3;
       const CUtensorMap* mB = t.dense ? &tmBs : &tmB;
       const int a_row = (t.dense ? 0 : t.seg * p.m_rows) + t.wt * WROWS + (int)rank * BM;
+      // kUmmaDgrad: output rows m of the stored weight's columns, contraction
+      // rows c of the stored weight (this segment's block of them).
+      const int m_row0 = t.wt * WROWS + (int)rank * BM;
+      const int c_row0 = t.dense ? 0 : t.seg * p.a_k_rows;
+      const int ksplit = t.dense ? p.k_split_s : p.k_split;
       const uint32_t bytes = A_TILES * A_BYTES + ts.bytes();
       const int nk = ceil_div(t.K, BK);
       if (ts.rows_gather > 0) {
@@ -563,9 +585,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // arms for both halves (the halves are the same size).
           const uint32_t fb = map_to_cta(fb_local, 0);
           if (leader) mbar_expect_tx(fb_local, 2 * bytes);
-          tma_load_2d_pair(sb, mA, kb * BK, a_row, fb);
-          if (MODE == kUmmaSwiGLU) tma_load_2d_pair(sb + A_BYTES, mA3, kb * BK, a_row, fb);
-          if (two_blocks(MODE)) tma_load_2d_pair(sb + A_BYTES, mA, kb * BK, a_row + BLOCK_STEP, fb);
+          if (MODE == kUmmaDgrad) {
+            const bool second = kb >= ksplit;
+            const int crow = c_row0 + (second ? kb - ksplit : kb) * BK;
+            const CUtensorMap* mk = second ? mA3 : mA;
+#pragma unroll
+            for (int blk = 0; blk < 2; ++blk)
+#pragma unroll
+              for (int h = 0; h < 2; ++h)
+                tma_load_2d_pair(sb + blk * A_BYTES + h * MN_BOX_BYTES, mk, m_row0 + blk * BLOCK_STEP + h * 64,
+                                 crow, fb);
+          } else {
+            tma_load_2d_pair(sb, mA, kb * BK, a_row, fb);
+            if (MODE == kUmmaSwiGLU) tma_load_2d_pair(sb + A_BYTES, mA3, kb * BK, a_row, fb);
+            if (two_blocks(MODE)) tma_load_2d_pair(sb + A_BYTES, mA, kb * BK, a_row + BLOCK_STEP, fb);
+          }
           if (ts.rows_gather > 0) {
             for (int g = 0; g < ts.rows_gather; g += 4)
               tma_gather4_pair(bb + g * (BK * 2), &tmG, kb * BK, s_rows[g], s_rows[g + 1], s_rows[g + 2],
@@ -576,9 +610,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         } else {
           mbar_expect_tx(fb_local, bytes);
-          tma_load_2d(sb, mA, kb * BK, a_row, fb_local);
-          if (MODE == kUmmaSwiGLU) tma_load_2d(sb + A_BYTES, mA3, kb * BK, a_row, fb_local);
-          if (two_blocks(MODE)) tma_load_2d(sb + A_BYTES, mA, kb * BK, a_row + BLOCK_STEP, fb_local);
+          if (MODE == kUmmaDgrad) {
+            const bool second = kb >= ksplit;
+            const int crow = c_row0 + (second ? kb - ksplit : kb) * BK;
+            const CUtensorMap* mk = second ? mA3 : mA;
+#pragma unroll
+            for (int blk = 0; blk < 2; ++blk)
+#pragma unroll
+              for (int h = 0; h < 2; ++h)
+                tma_load_2d(sb + blk * A_BYTES + h * MN_BOX_BYTES, mk, m_row0 + blk * BLOCK_STEP + h * 64, crow,
+                            fb_local);
+          } else {
+            tma_load_2d(sb, mA, kb * BK, a_row, fb_local);
+            if (MODE == kUmmaSwiGLU) tma_load_2d(sb + A_BYTES, mA3, kb * BK, a_row, fb_local);
+            if (two_blocks(MODE)) tma_load_2d(sb + A_BYTES, mA, kb * BK, a_row + BLOCK_STEP, fb_local);
+          }
           if (ts.rows_gather > 0) {
             for (int g = 0; g < ts.rows_gather; g += 4)
               tma_gather4(bb + g * (BK * 2), &tmG, kb * BK, s_rows[g], s_rows[g + 1], s_rows[g + 2],
@@ -615,7 +661,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!wait_bounded(smem_u32(&acce_bar[acc]), acc_phase ^ 1u, abort_flag, p.err, p.timeout_ns, true))
         break;
       tc_fence_after();
-      const uint32_t idesc = idesc_bf16_f32(PAIR ? 2 * BM : BM, ts.n_mma);
+      const uint32_t idesc = idesc_bf16_f32(PAIR ? 2 * BM : BM, ts.n_mma) | (MODE == kUmmaDgrad ? (1u << 15) : 0u);
       const uint32_t d1 = tmem_base + (uint32_t)(acc * BN_MAX);
       const uint32_t d3 = tmem_base + (uint32_t)BN_MAX;
       bool ok = true;
@@ -628,19 +674,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         tc_fence_after();
         const uint32_t sb = smem_u32(ring + off);
-        const uint64_t a_desc = sw128_desc(sb);
-        const uint64_t a3_desc = sw128_desc(sb + A_BYTES);
+        constexpr bool MN_A = MODE == kUmmaDgrad;
+        const uint64_t a_desc = MN_A ? sw128_mn_desc(sb) : sw128_desc(sb);
+        const uint64_t a3_desc = MN_A ? sw128_mn_desc(sb + A_BYTES) : sw128_desc(sb + A_BYTES);
         const uint64_t b_desc = sw128_desc(sb + A_TILES * A_BYTES);
 #pragma unroll
         for (int kk = 0; kk < BK / UMMA_K; ++kk) {
           const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+          // K-major: the next 16 k are 32 bytes along the row; MN-major: two
+          // 8-row k groups (2 x 1024 bytes) further on.
           const uint64_t koff = (uint64_t)((kk * UMMA_K * 2) >> 4);
+          const uint64_t koff_a = MN_A ? (uint64_t)((kk * 2 * 1024) >> 4) : koff;
           if (PAIR) {
-            umma_bf16_pair(d1, a_desc + koff, b_desc + koff, idesc, accum);
-            if (A_TILES == 2) umma_bf16_pair(d3, a3_desc + koff, b_desc + koff, idesc, accum);
+            umma_bf16_pair(d1, a_desc + koff_a, b_desc + koff, idesc, accum);
+            if (A_TILES == 2) umma_bf16_pair(d3, a3_desc + koff_a, b_desc + koff, idesc, accum);
           } else {
-            umma_bf16(d1, a_desc + koff, b_desc + koff, idesc, accum);
-            if (A_TILES == 2) umma_bf16(d3, a3_desc + koff, b_desc + koff, idesc, accum);
+            umma_bf16(d1, a_desc + koff_a, b_desc + koff, idesc, accum);
+            if (A_TILES == 2) umma_bf16(d3, a3_desc + koff_a, b_desc + koff, idesc, accum);
           }
         }
         issued = true;
@@ -720,7 +770,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
         }
-      } else if (MODE == kUmmaDown) {
+      } else if (MODE == kUmmaDgrad && p.out_f32) {
+        // Two 128-row blocks, BLOCK_STEP apart; fp32 output.
+        const int m2 = m + BLOCK_STEP;
+        const bool m2_ok = m2 < t.mrows;
+        float* o = reinterpret_cast<float*>(out) + r0 * ld;
+        for (int c0 = 0; c0 < n_mma; c0 += 16) {
+          uint32_t r1[16], r3[16];
+          tmem_ld16x2_wait(taddr + c0, taddr + BN_MAX + c0, r1, r3);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int col = c0 + j;
+            if (col < n_valid) {
+              if (m_ok) o[(long long)col * ld + m] = __uint_as_float(r1[j]);
+              if (m2_ok) o[(long long)col * ld + m2] = __uint_as_float(r3[j]);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) { if (PAIR) mbar_arrive_cluster(acce); else mbar_arrive(acce); }
+      } else if (MODE == kUmmaDown || MODE == kUmmaDgrad) {
         // Two 128-row blocks of the tile's weight rows, BLOCK_STEP apart.
         const int m2 = m + BLOCK_STEP;
         const bool m2_ok = m2 < t.mrows;
@@ -902,18 +972,29 @@ cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t 
   if (sp.ring_bytes < 2 * (a_tiles * A_BYTES + ceil_div(p.bn_max, BOX_N) * BOX_BYTES))
     return cudaErrorInvalidValue;
   const bool swiglu = p.mode == kUmmaSwiGLU;
+  const bool dgrad = p.mode == kUmmaDgrad;
   CUtensorMap tA, tA3, tB, tAs, tA3s, tBs;
   if (has_dense) {
-    if (!make_tmap(&tAs, p.a_s, p.K_s, p.m_rows_s, BM)) return cudaErrorInvalidValue;
+    if (dgrad) {   // stored weight [a_k_rows_s][m_rows_s], m contiguous: 64 x 64 boxes
+      if (!make_tmap(&tAs, p.a_s, p.m_rows_s, p.a_k_rows_s, 64)) return cudaErrorInvalidValue;
+      if (!make_tmap(&tA3s, p.a3_s ? p.a3_s : p.a_s, p.m_rows_s, p.a_k_rows_s, 64)) return cudaErrorInvalidValue;
+    } else {
+      if (!make_tmap(&tAs, p.a_s, p.K_s, p.m_rows_s, BM)) return cudaErrorInvalidValue;
+      if (swiglu && !make_tmap(&tA3s, p.a3_s, p.K_s, p.m_rows_s, BM)) return cudaErrorInvalidValue;
+      if (!swiglu) tA3s = tAs;
+    }
     if (!make_tmap(&tBs, p.b_s, p.K_s, p.shared_rows, BOX_N)) return cudaErrorInvalidValue;
-    if (swiglu && !make_tmap(&tA3s, p.a3_s, p.K_s, p.m_rows_s, BM)) return cudaErrorInvalidValue;
-    if (!swiglu) tA3s = tAs;
   }
   if (p.n_routed > 0) {
-    if (!make_tmap(&tA, p.a, p.K, p.a_rows_total, BM)) return cudaErrorInvalidValue;
+    if (dgrad) {   // stacked weights [n_routed * a_k_rows][m_rows], m contiguous
+      if (!make_tmap(&tA, p.a, p.m_rows, p.a_rows_total, 64)) return cudaErrorInvalidValue;
+      if (!make_tmap(&tA3, p.a3 ? p.a3 : p.a, p.m_rows, p.a_rows_total, 64)) return cudaErrorInvalidValue;
+    } else {
+      if (!make_tmap(&tA, p.a, p.K, p.a_rows_total, BM)) return cudaErrorInvalidValue;
+      if (swiglu && !make_tmap(&tA3, p.a3, p.K, p.a_rows_total, BM)) return cudaErrorInvalidValue;
+      if (!swiglu) tA3 = tA;
+    }
     if (!make_tmap(&tB, p.b, p.K, p.b_rows_total, BOX_N)) return cudaErrorInvalidValue;
-    if (swiglu && !make_tmap(&tA3, p.a3, p.K, p.a_rows_total, BM)) return cudaErrorInvalidValue;
-    if (!swiglu) tA3 = tA;
   } else {
     tA = tAs; tA3 = tA3s; tB = tBs;
   }
@@ -942,6 +1023,9 @@ cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t 
     case kUmmaBiasAct:
       return pair ? launch_mode<kUmmaBiasAct, true>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s)
                   : launch_mode<kUmmaBiasAct, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s);
+    case kUmmaDgrad:
+      return pair ? launch_mode<kUmmaDgrad, true>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s)
+                  : launch_mode<kUmmaDgrad, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s);
   }
   return cudaErrorInvalidValue;
 }
