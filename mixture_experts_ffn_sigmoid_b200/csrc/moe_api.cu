@@ -618,6 +618,30 @@ moe_status enqueue_backward(const moe_config& c, const void* x, const void* w_ro
   MOE_CUDA(launch_unpermute_sum(c.dtype, at<float>(ws, Bw.dxp), inv_row, shared ? at<float>(ws, Bw.dxs) : nullptr,
                                 at<float>(ws, Bw.dxr), dx, c.T, c.d, c.k, s));
   // Weight gradients, each a sum over the segment's tokens.
+  if (tc) {
+    const int nsm2 = device_sm_count();
+    auto wg = [&](int n_seg, const int* offs, int k_total, int M, int N, const void* P, long long ldP,
+                  long long p_rows, const void* Q, long long ldQ, long long q_rows, void* out) -> moe_status {
+      WgradParams w = {};
+      w.n_seg = n_seg; w.offsets = offs; w.k_total = k_total; w.M = M; w.N = N;
+      w.P = P; w.ldP = ldP; w.p_rows = p_rows; w.Q = Q; w.ldQ = ldQ; w.q_rows = q_rows; w.out = out;
+      w.err = err; w.timeout_ns = kDefaultTimeoutNs;
+      MOE_CUDA(launch_wgrad(w, nsm2, s));
+      return MOE_OK;
+    };
+    char* dadb = at<char>(ws, Bw.dadb);
+    MOE_TRY(wg(c.E, offsets, 0, c.f, c.d, dadb, 2LL * fp, rows, x_perm, d, rows, dw1));
+    MOE_TRY(wg(c.E, offsets, 0, c.f, c.d, dadb + (size_t)fp * es, 2LL * fp, rows, x_perm, d, rows, dw3));
+    MOE_TRY(wg(c.E, offsets, 0, c.d, c.f, dyp, d, rows, at<char>(ws, Bw.hg), f, rows, dw2));
+    if (shared) {
+      char* dadbs = at<char>(ws, Bw.dadbs);
+      MOE_TRY(wg(1, nullptr, c.T, c.f_shared, c.d, dadbs, 2LL * fsp, c.T, x, d, c.T, dws1));
+      MOE_TRY(wg(1, nullptr, c.T, c.f_shared, c.d, dadbs + (size_t)fsp * es, 2LL * fsp, c.T, x, d, c.T, dws3));
+      MOE_TRY(wg(1, nullptr, c.T, c.d, c.f_shared, dy, d, c.T, at<char>(ws, Bw.hgs), fs, c.T, dws2));
+    }
+    MOE_TRY(wg(1, nullptr, c.T, c.E, c.d, at<char>(ws, Bw.dlb), Bw.e_pad, c.T, x, d, c.T, dw_router));
+    return MOE_OK;
+  }
   for (int which = 0; which < 2; ++which) {         // dW1, dW3 [E][f][d]
     GradGemmParams g = gg(c, kSegK, c.E, offsets);
     g.M = c.f; g.N = c.d;

@@ -156,6 +156,21 @@ struct UmmaGemmParams {
   int out_f32;              // kUmmaDgrad: fp32 output instead of bf16
 };
 cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t s);
+
+// tcgen05 weight-gradient GEMM (umma_wgrad.cu): D_s[m][n] = sum over the
+// rows r of segment s of P[r][m] Q[r][n], bf16 in, fp32 accumulate, bf16 out.
+struct WgradParams {
+  int n_seg;
+  const int* offsets;       // [n_seg+1] row offsets; null: one segment of k_total rows
+  int k_total;
+  int M, N;
+  const void* P; long long ldP, p_rows;   // [p_rows][ldP] bf16, columns [0, M) used
+  const void* Q; long long ldQ, q_rows;   // [q_rows][ldQ] bf16, columns [0, N) used
+  void* out;                // bf16 [n_seg][M][N]
+  uint32_t* err;
+  long long timeout_ns;
+};
+cudaError_t launch_wgrad(const WgradParams& p, int num_sms, cudaStream_t s);
 cudaError_t launch_wait_timeout_selftest(uint32_t* err, long long timeout_ns, cudaStream_t s);
 
 int device_sm_count();

@@ -1,0 +1,285 @@
+// Weight gradients of the backward pass on the tensor cores (tcgen05):
+//
+//   D_s[m][n] = sum_{r in segment s} P[r][m] * Q[r][n]
+//
+// P and Q are row-major activations over the packed rows r (for dW1 of
+// expert e: P = da, Q = x_perm over the expert's rows; for dW2: P = dy
+// gathered in packed order, Q = g h). The contraction runs over a
+// segment's rows, so both operands are MN-major (m, n contiguous) and the
+// reduction length is ragged: expert s owns rows [offsets[s], offsets[s+1])
+// (Sparse MoE FFN note, "Packed forward": each expert sees the tokens that
+// chose it). Segments no row belongs to get D_s = 0.
+//
+// Tiles: 128 m x 256 n per CTA (one M=128, N=256 MMA per 16 rows), rows in
+// blocks of 64. Both operands arrive as 64 x 64 TMA boxes (128-byte swizzle,
+// MN-major: 64-element M/N groups 8 KB apart, 8-row groups 1 KB apart).
+// Rows of the last block past the segment's end belong to the next segment:
+// the MMA warp zeroes those rows of the P tile in shared memory before the
+// MMA, so they add nothing (Q's rows there are finite data or zero fill).
+//
+// Roles (192 threads, one CTA per SM, persistent over tiles ordered
+// segment-major, so CTAs running at once share a segment's rows in L2):
+//   warp 0 lane 0 : TMA producer into a 4-stage ring
+//   warp 1        : TMEM allocator; zero-fills partial blocks; lane 0 issues
+//                   tcgen05.mma and tcgen05.commit
+//   warps 2..5    : epilogue; two TMEM accumulators (2 x 256 columns), so a
+//                   tile's stores overlap the next tile's MMAs
+// Every wait is bounded, as in the forward GEMM.
+#include "umma_common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int WG_BM = 128;
+constexpr int WG_BN = 256;
+constexpr int WG_BK = 64;
+constexpr int WG_STAGES = 4;
+constexpr int WG_BOX = 64 * 64 * 2;                      // one 64 x 64 bf16 box
+constexpr int WG_A_BYTES = 2 * WG_BOX;                   // 128 m x 64 rows
+constexpr int WG_B_BYTES = 4 * WG_BOX;                   // 256 n x 64 rows
+constexpr int WG_STAGE_BYTES = WG_A_BYTES + WG_B_BYTES;
+constexpr int WG_THREADS = 192;
+constexpr int WG_SMEM = 1024 + 1024 + WG_STAGES * WG_STAGE_BYTES;
+constexpr int WG_TMEM_COLS = 512;
+
+struct WgTile {
+  int seg, m0, n0, r0, rows, nk;
+};
+
+__device__ __forceinline__ WgTile wg_tile(const WgradParams& p, int tile, int mt, int nt) {
+  WgTile t;
+  const int per_seg = mt * nt;
+  t.seg = tile / per_seg;
+  const int rem = tile - t.seg * per_seg;
+  t.m0 = (rem / nt) * WG_BM;
+  t.n0 = (rem - (rem / nt) * nt) * WG_BN;
+  if (p.offsets) {
+    t.r0 = p.offsets[t.seg];
+    t.rows = p.offsets[t.seg + 1] - t.r0;
+  } else {
+    t.r0 = 0;
+    t.rows = p.k_total;
+  }
+  t.nk = t.rows > 0 ? ceil_div(t.rows, WG_BK) : 0;
+  return t;
+}
+
+__device__ __forceinline__ void st_shared_zero16(uint32_t addr) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(WG_THREADS, 1)
+    wgrad_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
+                 const WgradParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty_bar = full_bar + WG_STAGES;
+  uint64_t* accf_bar = empty_bar + WG_STAGES;
+  uint64_t* acce_bar = accf_bar + 2;
+  uint64_t* drain_bar = acce_bar + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+  uint8_t* ring = smem + 1024;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < WG_STAGES; ++i) {
+      mbar_init(smem_u32(&full_bar[i]), 1);
+      mbar_init(smem_u32(&empty_bar[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&accf_bar[i]), 1);
+      mbar_init(smem_u32(&acce_bar[i]), 4);   // one arrival per epilogue warp
+    }
+    mbar_init(smem_u32(drain_bar), 1);
+    *abort_flag = 0u;
+    fence_mbar_init();
+    tmap_prefetch(&tmP);
+    tmap_prefetch(&tmQ);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), WG_TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int mt = ceil_div(p.M, WG_BM), nt = ceil_div(p.N, WG_BN);
+  const int total = p.n_seg * mt * nt;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      const WgTile t = wg_tile(p, tile, mt, nt);
+      for (int kb = 0; kb < t.nk; ++kb) {
+        if (!wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag, p.err, p.timeout_ns, true)) {
+          ok = false;
+          break;
+        }
+        const uint32_t fb = smem_u32(&full_bar[stage]);
+        const uint32_t sa = smem_u32(ring + stage * WG_STAGE_BYTES);
+        const uint32_t sbq = sa + WG_A_BYTES;
+        const int r = t.r0 + kb * WG_BK;
+        // Boxes wholly past M or N are not loaded: the rows (columns) of D
+        // they feed are never stored.
+        const int na = min(2, ceil_div(p.M - t.m0, 64)), nb = min(4, ceil_div(p.N - t.n0, 64));
+        mbar_expect_tx(fb, (uint32_t)(na + nb) * WG_BOX);
+        for (int h = 0; h < na; ++h) tma_load_2d(sa + h * WG_BOX, &tmP, t.m0 + h * 64, r, fb);
+        for (int h = 0; h < nb; ++h) tma_load_2d(sbq + h * WG_BOX, &tmQ, t.n0 + h * 64, r, fb);
+        if (++stage == WG_STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool issued = false, ok = true;
+    const uint32_t idesc = idesc_bf16_f32(WG_BM, WG_BN) | (1u << 15) | (1u << 16);
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      const WgTile t = wg_tile(p, tile, mt, nt);
+      if (t.nk == 0) continue;                  // the epilogue writes zeros
+      // Lane 0 waits; the outcome is broadcast so the warp stays converged.
+      int w_ok = lane == 0 ? (int)wait_bounded(smem_u32(&acce_bar[acc]), acc_phase ^ 1u, abort_flag, p.err,
+                                               p.timeout_ns, true) : 0;
+      if (!__shfl_sync(0xffffffffu, w_ok, 0)) break;
+      tc_fence_after();
+      const uint32_t d = tmem_base + (uint32_t)(acc * WG_BN);
+      const int na = min(2, ceil_div(p.M - t.m0, 64));
+      for (int kb = 0; kb < t.nk; ++kb) {
+        w_ok = lane == 0 ? (int)wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, p.err, p.timeout_ns,
+                                             true) : 0;
+        if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
+          ok = false;
+          break;
+        }
+        const uint32_t sa = smem_u32(ring + stage * WG_STAGE_BYTES);
+        const int valid = min(WG_BK, t.rows - kb * WG_BK);
+        if (valid < WG_BK) {
+          // Every lane sees the completed phase itself (it has completed, so
+          // the wait returns at once) before overwriting rows TMA wrote.
+          wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, p.err, p.timeout_ns, false);
+          // Rows valid..63 of the loaded 64-row P boxes: 128 bytes each, 8 x 16 B.
+          const int n16 = (WG_BK - valid) * na * 8;
+          for (int i = lane; i < n16; i += 32) {
+            const int h = i / ((WG_BK - valid) * 8);
+            const int rem = i - h * (WG_BK - valid) * 8;
+            st_shared_zero16(sa + h * WG_BOX + (valid + rem / 8) * 128 + (rem % 8) * 16);
+          }
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        tc_fence_after();
+        if (lane == 0) {
+          const uint64_t a_desc = sw128_mn_desc(sa);
+          const uint64_t b_desc = sw128_mn_desc(sa + WG_A_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < WG_BK / 16; ++kk) {
+            const uint64_t koff = (uint64_t)((kk * 2 * 1024) >> 4);   // two 8-row groups per 16 rows
+            umma_bf16(d, a_desc + koff, b_desc + koff, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(smem_u32(&empty_bar[stage]));
+        }
+        __syncwarp();
+        issued = true;
+        if (++stage == WG_STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+      if (lane == 0) umma_commit(smem_u32(&accf_bar[acc]));
+      __syncwarp();
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+    if (issued && lane == 0) {   // every MMA completes before TMEM is freed
+      umma_commit(smem_u32(drain_bar));
+      wait_bounded(smem_u32(drain_bar), 0u, abort_flag, p.err, p.timeout_ns, false);
+    }
+    __syncwarp();
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                    // TMEM lane quarter this warp may read
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      const WgTile t = wg_tile(p, tile, mt, nt);
+      const int m = t.m0 + q * 32 + lane;
+      __nv_bfloat16* orow = out + ((size_t)t.seg * p.M + (m < p.M ? m : 0)) * p.N;
+      if (t.nk == 0) {
+        if (m < p.M)
+          for (int c = 0; c < WG_BN && t.n0 + c < p.N; ++c) orow[t.n0 + c] = __float2bfloat16_rn(0.0f);
+        continue;
+      }
+      if (!wait_bounded(smem_u32(&accf_bar[acc]), acc_phase, abort_flag, p.err, p.timeout_ns, true)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * WG_BN);
+      for (int c0 = 0; c0 < WG_BN; c0 += 16) {
+        if (t.n0 + c0 >= p.N) break;
+        uint32_t r[16];
+        tmem_ld16_wait(taddr + c0, r);
+        if (m < p.M) {
+          uint32_t w[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+            w[j] = *reinterpret_cast<const uint32_t*>(&h);
+          }
+          __nv_bfloat16* dst = orow + t.n0 + c0;
+          if (t.n0 + c0 + 16 <= p.N) {
+            reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+          } else {
+            for (int j = 0; j < 16 && t.n0 + c0 + j < p.N; ++j)
+              dst[j] = __ushort_as_bfloat16((unsigned short)(w[j >> 1] >> ((j & 1) * 16)));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&acce_bar[acc]));
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, WG_TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_wgrad(const WgradParams& p, int num_sms, cudaStream_t s) {
+  if (p.n_seg <= 0 || p.M <= 0 || p.N <= 0) return cudaSuccess;
+  CUtensorMap tP, tQ;
+  if (!make_tmap_strided(&tP, p.P, p.M, p.p_rows, p.ldP * 2, 64)) return cudaErrorInvalidValue;
+  if (!make_tmap_strided(&tQ, p.Q, p.N, p.q_rows, p.ldQ * 2, 64)) return cudaErrorInvalidValue;
+  static int attr_done_mask = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (!(dev < 32 && ((attr_done_mask >> dev) & 1))) {
+    e = cudaFuncSetAttribute(wgrad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, WG_SMEM);
+    if (e != cudaSuccess) return e;
+    if (dev < 32) attr_done_mask |= 1 << dev;
+  }
+  const long long tiles = (long long)p.n_seg * ceil_div(p.M, WG_BM) * ceil_div(p.N, WG_BN);
+  const int grid = (int)(tiles < num_sms ? tiles : num_sms);
+  wgrad_kernel<<<grid, WG_THREADS, WG_SMEM, s>>>(tP, tQ, p);
+  return cudaGetLastError();
+}
+
+}  // namespace moe
