@@ -239,6 +239,72 @@ def measure_gelu_experts(B, cfg, inp, counts, stream, reps):
             "expert_weight_gbs": weight_bytes / (ms / 1e3) / 1e9, "graph_replays": reps}
 
 
+def backward_work(cfg, touched):
+    """Algorithmic flops and HBM bytes of one moe_backward call.
+
+    Flops: the router (logits, input and weight gradients: 3 x 2TEd) and, per
+    routed row (T k of them) and shared row (T), the recomputed
+    pre-activations (2 x 2df), dh' (2df), dx (2 x 2df) and the three weight
+    gradients (3 x 2df): 16 d f per row. Bytes: every touched expert's W1, W3
+    read twice (pre-activations, dx) and W2 once; every weight gradient
+    written once (untouched experts' as zeros); x and dy read, dx written.
+    """
+    es = cfg.elem_bytes
+    T, d, E, k, f, fs = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.f_shared
+    flops = 6.0 * T * E * d + 16.0 * d * (T * k * f + T * fs)
+    w_read = (touched * 5 * f * d + 5 * fs * d + E * d) * es
+    g_write = (E * 3 * f * d + 3 * fs * d + E * d) * es
+    act = 3 * T * d * es
+    return flops, w_read + g_write + act
+
+
+def measure_backward(B, cfg, inp, touched, stream, reps):
+    """moe_backward (routing and pre-activations recomputed, every gradient
+    written) timed over a CUDA graph on the workload's inputs and a seeded dy."""
+    dev = inp["x"].device
+    dt = cfg.torch_dtype
+    g = torch.Generator(device=dev)
+    g.manual_seed(9)
+    dy = torch.randn((cfg.T, cfg.d), generator=g, device=dev).to(dt)
+    sh = cfg.f_shared > 0
+    outs = [torch.empty((cfg.T, cfg.d), dtype=dt, device=dev), torch.empty((cfg.E, cfg.d), dtype=dt, device=dev),
+            torch.empty((cfg.E, cfg.f, cfg.d), dtype=dt, device=dev),
+            torch.empty((cfg.E, cfg.f, cfg.d), dtype=dt, device=dev),
+            torch.empty((cfg.E, cfg.d, cfg.f), dtype=dt, device=dev),
+            torch.empty((cfg.f_shared, cfg.d), dtype=dt, device=dev) if sh else None,
+            torch.empty((cfg.f_shared, cfg.d), dtype=dt, device=dev) if sh else None,
+            torch.empty((cfg.d, cfg.f_shared), dtype=dt, device=dev) if sh else None]
+    wsb = B.alloc_backward_workspace(cfg, dev)
+
+    def bwd():   # on the current stream, so that the graph below captures it
+        B.moe_backward(cfg, inp["x"], inp["w_router"], inp["bias"], inp["w1"], inp["w3"], inp["w2"], inp["ws1"],
+                       inp["ws3"], inp["ws2"], dy, *outs, wsb)
+
+    for _ in range(2):
+        bwd()
+    torch.cuda.synchronize()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        bwd()
+    gr.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        gr.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    del gr
+    assert B.moe_get_device_error(wsb) == B.MOE_OK
+    ms = e0.elapsed_time(e1) / reps
+    flops, nbytes = backward_work(cfg, touched)
+    del outs, wsb
+    return {"ms_per_step": ms, "tokens_per_s": cfg.T / (ms / 1e3), "tflops": flops / (ms / 1e3) / 1e12,
+            "gbs": nbytes / (ms / 1e3) / 1e9, "algorithmic_flops": flops, "algorithmic_bytes": nbytes,
+            "graph_replays": reps,
+            "note": "recomputes routing and SwiGLU pre-activations; writes dx and every weight gradient"}
+
+
 def measure_fused_permute(B, cfg, inp, idx, offsets, perm_src, inv_row, h, h_s, ws, stream, reps):
     """The permute fused into the gate/up GEMM: maps-only permute, then the
     GEMM gathering token rows from x (TMA gather4). Same h bytes as the
@@ -475,6 +541,9 @@ def main():
     work, touched = stage_work(cfg, counts.cpu())
     peaks = measured_peaks()
     gelu["expert_weight_frac_hbm"] = gelu["expert_weight_gbs"] / peaks["hbm"]
+    bwd = measure_backward(B, cfg, inp, touched, stream, max(3, min(args.steps, 10)))
+    bwd["frac_tensor"] = bwd["tflops"] / peaks["tensor_sustained"]
+    bwd["frac_hbm"] = bwd["gbs"] / peaks["hbm"]
     dom = max(names, key=lambda n: stage_ms[n])
     wd = work[dom]
     t_dom = stage_ms[dom] / 1e3
@@ -573,6 +642,7 @@ def main():
             "balance_update": balance,
             "gelu_experts": gelu,
             "fused_permute_gather": fused,
+            "backward": bwd,
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": {"value": whole_job_rate(T, world, e2e_ms), "unit": "tokens/s",

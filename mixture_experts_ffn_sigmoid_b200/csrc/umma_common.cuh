@@ -140,6 +140,22 @@ __device__ __forceinline__ void tmem_ld16x2_wait(uint32_t ta, uint32_t tb, uint3
       : "r"(ta), "r"(tb)
       : "memory");
 }
+// Four 16-column loads (64 consecutive columns from `ta`) under one wait.
+__device__ __forceinline__ void tmem_ld64_wait(uint32_t ta, uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%65];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47}, [%66];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%67];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : MOE_R16((&r[0])), MOE_R16((&r[16])), MOE_R16((&r[32])), MOE_R16((&r[48]))
+      : "r"(ta), "r"(ta + 16), "r"(ta + 32), "r"(ta + 48)
+      : "memory");
+}
 #undef MOE_R16
 
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row atoms
@@ -206,6 +222,40 @@ bool make_tmap_strided(CUtensorMap* tm, const void* base, long long inner, long 
                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// 3-D bf16 tensor [outer2][outer1][inner] (strides in bytes), 128-byte
+// swizzle, box = 64 x box1 x 1: stores clip at each dimension's bound.
+bool make_tmap_3d(CUtensorMap* tm, void* base, long long inner, long long outer1, long long outer2,
+                  long long stride1_bytes, long long stride2_bytes, int box1) {
+  auto fn = get_encode_fn();
+  if (!fn || inner <= 0 || outer1 <= 0 || outer2 <= 0 || stride1_bytes % 16 || stride2_bytes % 16) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)outer1, (cuuint64_t)outer2};
+  cuuint64_t strides[2] = {(cuuint64_t)stride1_bytes, (cuuint64_t)stride2_bytes};
+  cuuint32_t box[3] = {(cuuint32_t)UMMA_BK, (cuuint32_t)box1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// TMA store of a 3-D box from shared memory, tracked by the bulk-group
+// counters of the issuing thread.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* tm, uint32_t src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+                   reinterpret_cast<uint64_t>(tm)),
+               "r"(c0), "r"(c1), "r"(c2), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Every committed group has finished reading its shared-memory source.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 }  // namespace

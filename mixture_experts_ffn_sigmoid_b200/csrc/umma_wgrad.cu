@@ -17,13 +17,15 @@
 // the MMA warp zeroes those rows of the P tile in shared memory before the
 // MMA, so they add nothing (Q's rows there are finite data or zero fill).
 //
-// Roles (192 threads, one CTA per SM, persistent over tiles ordered
+// Roles (320 threads, one CTA per SM, persistent over tiles ordered
 // segment-major, so CTAs running at once share a segment's rows in L2):
 //   warp 0 lane 0 : TMA producer into a 4-stage ring
 //   warp 1        : TMEM allocator; zero-fills partial blocks; lane 0 issues
 //                   tcgen05.mma and tcgen05.commit
-//   warps 2..5    : epilogue; two TMEM accumulators (2 x 256 columns), so a
-//                   tile's stores overlap the next tile's MMAs
+//   warps 2..9    : epilogue; warp w reads TMEM lane quarter w % 4 and half
+//                   of the 256 columns, 64 columns per load wait; two TMEM
+//                   accumulators (2 x 256 columns), so a tile's stores
+//                   overlap the next tile's MMAs
 // Every wait is bounded, as in the forward GEMM.
 #include "umma_common.cuh"
 
@@ -38,8 +40,10 @@ constexpr int WG_BOX = 64 * 64 * 2;                      // one 64 x 64 bf16 box
 constexpr int WG_A_BYTES = 2 * WG_BOX;                   // 128 m x 64 rows
 constexpr int WG_B_BYTES = 4 * WG_BOX;                   // 256 n x 64 rows
 constexpr int WG_STAGE_BYTES = WG_A_BYTES + WG_B_BYTES;
-constexpr int WG_THREADS = 192;
-constexpr int WG_SMEM = 1024 + 1024 + WG_STAGES * WG_STAGE_BYTES;
+constexpr int WG_THREADS = 320;
+constexpr int WG_EPI_WARPS = 8;
+constexpr int WG_STG_BYTES = 32 * 64 * 2;                // one warp's 32 x 64 output box
+constexpr int WG_SMEM = 1024 + 1024 + WG_STAGES * WG_STAGE_BYTES + WG_EPI_WARPS * WG_STG_BYTES;
 constexpr int WG_TMEM_COLS = 512;
 
 struct WgTile {
@@ -67,13 +71,10 @@ __device__ __forceinline__ WgTile wg_tile(const WgradParams& p, int tile, int mt
 __device__ __forceinline__ void st_shared_zero16(uint32_t addr) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
 }
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 
 __global__ void __launch_bounds__(WG_THREADS, 1)
     wgrad_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
-                 const WgradParams p) {
+                 const __grid_constant__ CUtensorMap tmD, const WgradParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -85,6 +86,7 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   uint8_t* ring = smem + 1024;
+  uint8_t* stage_out = ring + WG_STAGES * WG_STAGE_BYTES;   // epilogue staging, one box per warp
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -94,13 +96,14 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&accf_bar[i]), 1);
-      mbar_init(smem_u32(&acce_bar[i]), 4);   // one arrival per epilogue warp
+      mbar_init(smem_u32(&acce_bar[i]), WG_EPI_WARPS);   // one arrival per epilogue warp
     }
     mbar_init(smem_u32(drain_bar), 1);
     *abort_flag = 0u;
     fence_mbar_init();
     tmap_prefetch(&tmP);
     tmap_prefetch(&tmQ);
+    tmap_prefetch(&tmD);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), WG_TMEM_COLS);
@@ -208,41 +211,66 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
     __syncwarp();
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue
+    // Each warp converts its 32 rows x 64 columns to bf16 into a swizzled
+    // staging box (row = lane, 16-byte chunk c at c ^ (row & 7), the layout
+    // TMA's 128-byte swizzle reads) and lane 0 stores the box with TMA: one
+    // bulk write per 4 KB instead of 32 scattered 16-byte stores per
+    // instruction. The 3-D output map clips rows past M and columns past N.
     const int q = warp & 3;                    // TMEM lane quarter this warp may read
+    const int half = (warp - 2) >> 2;          // columns [128 half, 128 half + 128)
+    const uint32_t box = smem_u32(stage_out + (warp - 2) * WG_STG_BYTES);
     int acc = 0;
     uint32_t acc_phase = 0;
-    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
       const WgTile t = wg_tile(p, tile, mt, nt);
-      const int m = t.m0 + q * 32 + lane;
-      __nv_bfloat16* orow = out + ((size_t)t.seg * p.M + (m < p.M ? m : 0)) * p.N;
+      const int mrow = t.m0 + q * 32;          // first row of this warp's boxes
+      const int nbeg = t.n0 + half * 128;
       if (t.nk == 0) {
-        if (m < p.M)
-          for (int c = 0; c < WG_BN && t.n0 + c < p.N; ++c) orow[t.n0 + c] = __float2bfloat16_rn(0.0f);
+        // No row chose this segment: its gradient is zero. Store a zeroed
+        // staging box over the warp's two 32 x 64 output boxes.
+        if (mrow < p.M && nbeg < p.N) {
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
+#pragma unroll
+          for (int c = 0; c < 8; ++c) st_shared_zero16(box + lane * 128 + c * 16);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            for (int c0 = 0; c0 < 128 && nbeg + c0 < p.N; c0 += 64) tma_store_3d(&tmD, box, nbeg + c0, mrow, t.seg);
+            bulk_commit();
+          }
+        }
         continue;
       }
       if (!wait_bounded(smem_u32(&accf_bar[acc]), acc_phase, abort_flag, p.err, p.timeout_ns, true)) break;
       tc_fence_after();
-      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * WG_BN);
-      for (int c0 = 0; c0 < WG_BN; c0 += 16) {
-        if (t.n0 + c0 >= p.N) break;
-        uint32_t r[16];
-        tmem_ld16_wait(taddr + c0, r);
-        if (m < p.M) {
-          uint32_t w[8];
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * WG_BN + half * 128);
+      for (int c0 = 0; c0 < 128; c0 += 64) {
+        if (nbeg + c0 >= p.N || mrow >= p.M) break;
+        uint32_t r[64];
+        tmem_ld64_wait(taddr + c0, r);
+        // The previous store must have read the staging box out.
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+        for (int c = 0; c < 8; ++c) {
+          uint32_t w[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[8 * c + 2 * j]),
+                                                           __uint_as_float(r[8 * c + 2 * j + 1]));
             w[j] = *reinterpret_cast<const uint32_t*>(&h);
           }
-          __nv_bfloat16* dst = orow + t.n0 + c0;
-          if (t.n0 + c0 + 16 <= p.N) {
-            reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
-            reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
-          } else {
-            for (int j = 0; j < 16 && t.n0 + c0 + j < p.N; ++j)
-              dst[j] = __ushort_as_bfloat16((unsigned short)(w[j >> 1] >> ((j & 1) * 16)));
-          }
+          const uint32_t dst = box + lane * 128 + ((c ^ (lane & 7)) * 16);
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+                       "r"(w[3])
+                       : "memory");
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&tmD, box, nbeg + c0, mrow, t.seg);
+          bulk_commit();
         }
       }
       tc_fence_before();
@@ -251,6 +279,8 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
+    if (lane == 0) bulk_wait_all();   // staging boxes stay live until written out
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
@@ -264,9 +294,11 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
 
 cudaError_t launch_wgrad(const WgradParams& p, int num_sms, cudaStream_t s) {
   if (p.n_seg <= 0 || p.M <= 0 || p.N <= 0) return cudaSuccess;
-  CUtensorMap tP, tQ;
+  CUtensorMap tP, tQ, tD;
   if (!make_tmap_strided(&tP, p.P, p.M, p.p_rows, p.ldP * 2, 64)) return cudaErrorInvalidValue;
   if (!make_tmap_strided(&tQ, p.Q, p.N, p.q_rows, p.ldQ * 2, 64)) return cudaErrorInvalidValue;
+  if (!make_tmap_3d(&tD, p.out, p.N, p.M, p.n_seg, (long long)p.N * 2, (long long)p.M * p.N * 2, 32))
+    return cudaErrorInvalidValue;
   static int attr_done_mask = 0;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -278,7 +310,7 @@ cudaError_t launch_wgrad(const WgradParams& p, int num_sms, cudaStream_t s) {
   }
   const long long tiles = (long long)p.n_seg * ceil_div(p.M, WG_BM) * ceil_div(p.N, WG_BN);
   const int grid = (int)(tiles < num_sms ? tiles : num_sms);
-  wgrad_kernel<<<grid, WG_THREADS, WG_SMEM, s>>>(tP, tQ, p);
+  wgrad_kernel<<<grid, WG_THREADS, WG_SMEM, s>>>(tP, tQ, tD, p);
   return cudaGetLastError();
 }
 

@@ -552,22 +552,27 @@ def moe_backward(x, w_router, bias, w1, w3, w2, k: int, gate_mode: int, dy,
         r["idx"] = np.asarray(idx, dtype=np.int64)
         r["gates"] = gate_values(r["logits"], r["scores"], r["idx"], gate_mode, route_scale)
     idx, gates = r["idx"], r["gates"]
-    T, d = x.shape
-    E = _f64(w_router).shape[0]
     dx = np.zeros_like(x)
     dgates = np.zeros_like(gates)
-    w1s, w3s, w2s = _f64(w1), _f64(w3), _f64(w2)
-    dw1, dw3, dw2 = np.zeros_like(w1s), np.zeros_like(w3s), np.zeros_like(w2s)
+    # Expert matrices are read one expert at a time (w1[e]), so a caller may
+    # pass lazily widened stacks; the weight gradients of chosen experts are
+    # collected per expert and stacked (zeros elsewhere) for array inputs.
+    g1s, g3s, g2s = {}, {}, {}
     for e in np.unique(idx):
+        e = int(e)
         tok, slot = np.nonzero(idx == e)
-        out = swiglu_ffn(x[tok], w1s[e], w3s[e], w2s[e])
+        w1e, w3e, w2e = _f64(w1[e]), _f64(w3[e]), _f64(w2[e])
+        out = swiglu_ffn(x[tok], w1e, w3e, w2e)
         dgates[tok, slot] = (dy[tok] * out).sum(axis=1)
         g = gates[tok, slot][:, None]
-        du, g1, g3, g2 = swiglu_ffn_backward(x[tok], w1s[e], w3s[e], w2s[e], g * dy[tok])
+        du, g1s[e], g3s[e], g2s[e] = swiglu_ffn_backward(x[tok], w1e, w3e, w2e, g * dy[tok])
         np.add.at(dx, tok, du)
-        dw1[e] += g1
-        dw3[e] += g3
-        dw2[e] += g2
+    if isinstance(w1, np.ndarray):
+        dw1, dw3, dw2 = np.zeros(w1.shape), np.zeros(w3.shape), np.zeros(w2.shape)
+        for e in g1s:
+            dw1[e], dw3[e], dw2[e] = g1s[e], g3s[e], g2s[e]
+    else:
+        dw1, dw3, dw2 = g1s, g3s, g2s
     dws1 = dws3 = dws2 = None
     if ws1 is not None:
         du, dws1, dws3, dws2 = swiglu_ffn_backward(x, ws1, ws3, ws2, dy)

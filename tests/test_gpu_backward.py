@@ -156,3 +156,54 @@ def test_backward_empty_tokens():
     torch.cuda.synchronize()
     for n, t in dw.items():
         assert torch.count_nonzero(t).item() == 0, n
+
+
+def test_backward_full_size_sampled():
+    # The DeepSeek-V3 workload the bench times, checked on outputs the oracle
+    # can compute one at a time:
+    #  * dx of sampled tokens: dx_t depends only on token t, so the oracle's
+    #    backward over those tokens (on the GPU's expert choice) gives it;
+    #  * the full dW1, dW3, dW2 of two experts (most and least loaded): each
+    #    depends only on the tokens that chose the expert, their gates and dy;
+    #  * rows of the shared expert's dWs1, dWs3 and columns of dWs2 for
+    #    sampled inner units: given dy, inner units are independent, so the
+    #    gradient of the FFN restricted to those units equals them.
+    # The router's weight gradient needs every token's expert outputs; the
+    # small cases above check it.
+    from mixture_experts_ffn_sigmoid_b200.inputs import CONFIGS, sample_token_ids
+    cfg = CONFIGS["deepseek_v3"]
+    inp = H.gpu_inputs(cfg)
+    dy = _dy(cfg)
+    got = gpu_backward(cfg, inp, dy)
+    gr = H.gpu_route(cfg, inp)
+    ref_route = H.oracle_route(cfg, inp)
+    rep = H.check_route(cfg, ref_route, gr)
+    gidx = gr["idx"].cpu().numpy().astype(np.int64)
+    w1, w3, w2 = H.LazyStack(inp["w1"]), H.LazyStack(inp["w3"]), H.LazyStack(inp["w2"])
+    x64, dy64 = H.f64(inp["x"]), H.f64(dy)
+    wr, bias = H.f64(inp["w_router"]), H.f64(inp["bias"])
+    # dx on sampled tokens
+    toks = sample_token_ids(cfg.T, 6).numpy()
+    ref = orc.moe_backward(x64[toks], wr, bias, w1, w3, w2, cfg.k, cfg.gate_mode, dy64[toks], cfg.n_groups,
+                           cfg.topk_groups, cfg.route_scale, H.f64(inp["ws1"]), H.f64(inp["ws3"]),
+                           H.f64(inp["ws2"]), idx=gidx[toks])
+    compare_grad(cfg, H.f64(got["dx"])[toks], ref["dx"], "dx (sampled tokens)")
+    # whole weight gradients of two experts
+    counts = np.bincount(gidx.ravel(), minlength=cfg.E)
+    gates = orc.gate_values(ref_route["logits"], ref_route["scores"], gidx, cfg.gate_mode, cfg.route_scale)
+    for e in (int(np.argmax(counts)), int(np.argmin(np.where(counts > 0, counts, 1 << 30)))):
+        tok, slot = np.nonzero(gidx == e)
+        g = gates[tok, slot][:, None]
+        _, d1, d3, d2 = orc.swiglu_ffn_backward(x64[tok], w1[e], w3[e], w2[e], g * dy64[tok])
+        compare_grad(cfg, H.f64(got["dw1"][e]), d1, f"dw1[{e}]")
+        compare_grad(cfg, H.f64(got["dw3"][e]), d3, f"dw3[{e}]")
+        compare_grad(cfg, H.f64(got["dw2"][e]), d2, f"dw2[{e}]")
+    # sampled inner units of the shared expert
+    units = np.sort(np.random.default_rng(3).choice(cfg.f_shared, 16, replace=False))
+    ws1, ws3, ws2 = H.f64(inp["ws1"]), H.f64(inp["ws3"]), H.f64(inp["ws2"])
+    _, s1, s3, s2 = orc.swiglu_ffn_backward(x64, ws1[units], ws3[units], ws2[:, units], dy64)
+    compare_grad(cfg, H.f64(got["dws1"])[units], s1, "dws1 (sampled rows)")
+    compare_grad(cfg, H.f64(got["dws3"])[units], s3, "dws3 (sampled rows)")
+    compare_grad(cfg, H.f64(got["dws2"])[:, units], s2, "dws2 (sampled columns)")
+    for n in NAMES:
+        assert torch.isfinite(got[n].float()).all().item(), n
