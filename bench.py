@@ -175,8 +175,12 @@ def stage_work(cfg, counts):
     return w, touched
 
 
-def source_sha(path):
-    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+def source_sha(paths):
+    """First 16 hex digits of the sha256 of the files' contents, in order."""
+    h = hashlib.sha256()
+    for path in ([paths] if isinstance(paths, str) else paths):
+        h.update(open(path, "rb").read())
+    return h.hexdigest()[:16]
 
 
 def traffic_for(workload, stage):
@@ -189,8 +193,8 @@ def traffic_for(workload, stage):
         e = d.get(workload, {}).get(stage)
         if not e:
             return None
-        src = os.path.join(ROOT, e["source"])
-        if source_sha(src) != e["source_sha256_16"]:
+        srcs = e["sources"] if "sources" in e else [e["source"]]
+        if source_sha([os.path.join(ROOT, x) for x in srcs]) != e["source_sha256_16"]:
             return None
         return e["bytes_per_launch"]
     except Exception:
