@@ -340,8 +340,10 @@ MOE_API moe_status moe_backward(const moe_config* cfg, const void* x, const void
  * and bases, error word) is one fixed 24 MiB array in the library's device
  * image, present on every GPU that loads the library until the process
  * exits; the call itself allocates nothing.
- *  - Capacity: the call needs 256 + 4*T*E + 8*E*ceil(T/32) bytes (each term
- *    rounded up to 256); beyond 24 MiB it returns MOE_ERR_WORKSPACE_TOO_SMALL
+ *  - Capacity: the call needs 256 + 4*S*T*E + 8*E*ceil(T/32) bytes (each term
+ *    rounded up to 256), where S is the number of router partial sums: 1 for
+ *    fp32; for bf16, S = min(8, ceil(d/64), max(1, floor(148 / (ceil(T/128) *
+ *    ceil(E/256))))). Beyond 24 MiB it returns MOE_ERR_WORKSPACE_TOO_SMALL
  *    before enqueuing anything.
  *  - The first call on each device looks up the array's device address
  *    (with that device current) and caches it; make that first call before

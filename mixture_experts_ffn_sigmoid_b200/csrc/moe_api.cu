@@ -43,7 +43,9 @@ Layout layout_of(const moe_config& c) {
   const size_t fs = (size_t)c.f_shared;
   const size_t nch = (T + kChunk - 1) / kChunk;
   L.err = take(kAlign);
-  L.logits = take(T * E * 4);
+  // bf16 router logits come as partial sums of a split contraction.
+  const size_t n_part = c.dtype == MOE_DTYPE_BF16 ? (size_t)router_gemm_splits(c.T, c.E, c.d) : 1;
+  L.logits = take(n_part * T * E * 4);
   L.ccount = take(nch * E * 4);
   L.cbase = take(nch * E * 4);
   L.idx = take(T * k * 4);
@@ -121,24 +123,10 @@ moe_status enqueue_route(const moe_config& c, const void* x, const void* w_route
   const Layout L = layout_of(c);
   float* logits = at<float>(ws, L.logits);
   const int num_sms = device_sm_count();
+  int n_part = 1;
   if (c.dtype == MOE_DTYPE_BF16) {
-    UmmaGemmParams g = {};
-    g.mode = kUmmaRouter;
-    g.n_routed = 0;
-    g.shared_rows = c.T;
-    g.m_rows_s = c.E;
-    g.K_s = c.d;
-    int bn = 256;
-    while (bn > 32 && (long long)ceil_div(c.E, 128) * ceil_div(c.T, bn) < num_sms) bn >>= 1;
-    g.bn_max = bn;
-    g.max_inflight = 3;
-    g.a_s = w_router;
-    g.b_s = x;
-    g.out_s = logits;
-    g.out_s_ld = c.E;
-    g.err = at<uint32_t>(ws, L.err);
-    g.timeout_ns = kDefaultTimeoutNs;
-    MOE_CUDA(launch_umma_gemm(g, num_sms, s));
+    n_part = router_gemm_splits(c.T, c.E, c.d);
+    MOE_CUDA(launch_router_gemm(x, w_router, c.T, c.E, c.d, logits, n_part, at<uint32_t>(ws, L.err), s));
   } else {
     SimtGemmParams g = {};
     g.dual = 0;
@@ -155,6 +143,8 @@ moe_status enqueue_route(const moe_config& c, const void* x, const void* w_route
   r.T = c.T; r.E = c.E; r.k = c.k; r.gate_mode = c.gate_mode;
   r.n_groups = c.n_groups; r.topk_groups = c.topk_groups; r.route_scale = c.route_scale;
   r.logits = logits; r.bias = bias; r.topk_idx = idx; r.topk_gate = gate;
+  r.n_partials = n_part;
+  r.partial_stride = (long long)c.T * c.E;
   r.chunk_counts = at<int>(ws, L.ccount);
   MOE_CUDA(launch_router_topk(r, s));
   const int nch = ceil_div(c.T, kChunk);

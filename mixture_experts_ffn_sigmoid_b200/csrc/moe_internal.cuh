@@ -47,7 +47,9 @@ __device__ __forceinline__ float gelu_erf(float v) {
 struct RouteParams {
   int T, E, k, gate_mode, n_groups, topk_groups;
   float route_scale;
-  const float* logits;     // [T][E]
+  float* logits;           // [T][E]; with n_partials > 1, partial 0 of n_partials
+  int n_partials;          // router partial sums to add (in order) per logit, >= 1
+  long long partial_stride;  // elements between partials (T * E)
   const float* bias;       // [E] or null
   int* topk_idx;           // [T][k]
   float* topk_gate;        // [T][k]
@@ -172,6 +174,12 @@ struct WgradParams {
 };
 cudaError_t launch_wgrad(const WgradParams& p, int num_sms, cudaStream_t s);
 cudaError_t launch_wait_timeout_selftest(uint32_t* err, long long timeout_ns, cudaStream_t s);
+
+// tcgen05 router logits with a split contraction (umma_router.cu): partial
+// [n_split][T][E] fp32, summed by the top-k kernel.
+int router_gemm_splits(int T, int E, int K);
+cudaError_t launch_router_gemm(const void* x, const void* w_router, int T, int E, int K, float* partial,
+                               int n_split, uint32_t* err, cudaStream_t s);
 
 int device_sm_count();
 

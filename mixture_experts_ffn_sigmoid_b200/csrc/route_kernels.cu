@@ -36,14 +36,18 @@ __global__ void __launch_bounds__(1024, 1) router_topk_kernel(RouteParams p) {
   __syncthreads();
 
   if (t < p.T) {                       // warp-uniform
-    const float* lrow = p.logits + (size_t)t * E;
+    float* lrow = p.logits + (size_t)t * E;
     float v[NPL];                      // biased selection score b' = s + bias
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
       const int e = lane + 32 * i;
       float b = -INFINITY;
       if (e < E) {
-        const float l = lrow[e];
+        // Router partial sums (a split contraction) add up in a fixed order;
+        // the total replaces partial 0, where later readers find the logit.
+        float l = lrow[e];
+        for (int q = 1; q < p.n_partials; ++q) l += lrow[(size_t)q * p.partial_stride + e];
+        if (p.n_partials > 1) lrow[e] = l;
         const float s = (p.gate_mode == MOE_GATE_SIGMOID) ? sigmoid_f32(l) : l;
         b = s + (p.bias ? p.bias[e] : 0.0f);
       }
