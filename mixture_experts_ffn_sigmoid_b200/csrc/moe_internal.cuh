@@ -120,7 +120,7 @@ cudaError_t launch_unpermute_sum(int dtype, const float* dxp, const int* inv_row
                                  const float* dxr, void* dx, int T, int d, int k, cudaStream_t s);
 
 // tcgen05 grouped GEMM (umma_gemm.cu)
-enum UmmaMode { kUmmaRouter = 0, kUmmaSwiGLU = 1, kUmmaDown = 2, kUmmaBiasAct = 3, kUmmaDgrad = 4 };
+enum UmmaMode { kUmmaSwiGLU = 1, kUmmaDown = 2, kUmmaBiasAct = 3, kUmmaDgrad = 4 };
 struct UmmaGemmParams {
   int mode;
   int n_routed;             // routed segments

@@ -2,11 +2,10 @@
 //
 // What it computes (SwiGLU equation of the Sparse MoE FFN note, "How it
 // works": FFN(u) = W2 (SiLU(W1 u) * W3 u), W1, W3 in R^{f x d}, W2 in
-// R^{d x f}; the router linear of the "Routing" paragraph, u . e_i):
+// R^{d x f}; the router logits have their own kernel, umma_router.cu):
 //
 //   kUmmaSwiGLU: h[r][m] = SiLU(sum_c W1_e[m][c] x[r][c]) * (sum_c W3_e[m][c] x[r][c])
 //   kUmmaDown:   y[r][m] = sum_c W2_e[m][c] h[r][c]
-//   kUmmaRouter: l[t][e] = sum_c Wr[e][c] x[t][c]            (fp32 out)
 //   kUmmaBiasAct: o[r][m] = act(sum_c W_e[m][c] u[r][c] + b_e[m]), act = GELU or
 //                identity (the generic expert of "Lesson 2 - From the Dense FFN
 //                to a Layer of Experts", section 2: W2 phi(W1 u + b1) + b2)
@@ -17,7 +16,8 @@
 //
 // for every packed row r of every segment. Segment e < n_routed is expert e
 // over packed rows [offsets[e], offsets[e+1]); segment n_routed is the dense
-// segment (the shared expert over all T tokens, or the router over all tokens).
+// segment (the shared expert over all T tokens, or a dense weight such as the
+// router's in the backward pass).
 //
 // Orientation ("swap AB"): weight rows are the MMA's M side (128 per MMA) and
 // tokens its N side (16..256 per tile, a multiple of 16). A DeepSeek-V3 expert
@@ -186,7 +186,6 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar, uint16_t mask) {
 // With PAIR the two CTAs of a cluster run one M=256 MMA: each holds 128 rows
 // of every weight block and half of the token tile.
 template <int MODE> struct Kind;
-template <> struct Kind<kUmmaRouter> { static constexpr int A_TILES = 1; static constexpr int ACC_STAGES = 2; };
 template <> struct Kind<kUmmaSwiGLU> { static constexpr int A_TILES = 2; static constexpr int ACC_STAGES = 1; };
 template <> struct Kind<kUmmaDown>   { static constexpr int A_TILES = 2; static constexpr int ACC_STAGES = 1; };
 template <> struct Kind<kUmmaBiasAct> { static constexpr int A_TILES = 2; static constexpr int ACC_STAGES = 1; };
@@ -685,22 +684,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) { if (PAIR) mbar_arrive_cluster(acce); else mbar_arrive(acce); }
-      } else {
-        float* o = reinterpret_cast<float*>(out) + r0 * ld;
-        for (int c0 = 0; c0 < n_mma; c0 += 16) {
-          uint32_t r1[16];
-          tmem_ld16_wait(taddr + c0, r1);
-          if (m_ok) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int col = c0 + j;
-              if (col < n_valid) o[(long long)col * ld + m] = __uint_as_float(r1[j]);
-            }
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) { if (PAIR) mbar_arrive_cluster(acce); else mbar_arrive(acce); }
       }
       if (ACC_STAGES == 2) {
         acc ^= 1;
@@ -783,11 +766,11 @@ cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t 
   if (p.bn_max < 16 || p.bn_max > BN_MAX || p.bn_max % 16) return cudaErrorInvalidValue;
   const int nseg = p.n_routed + (has_dense ? 1 : 0);
   const SmemPlan sp = smem_plan(p.n_routed, nseg);
-  const int a_tiles = p.mode == kUmmaRouter ? 1 : 2;
-  // Expert GEMMs with wide token tiles run on CTA pairs (M=256 MMAs: each CTA
-  // stages half the token tile, halving token traffic per weight byte). Narrow
-  // tiles (decode) and the router stay on single CTAs.
-  const bool pair = p.mode != kUmmaRouter && p.bn_max >= 128 && num_sms >= 2;
+  const int a_tiles = 2;
+  // Wide token tiles run on CTA pairs (M=256 MMAs: each CTA stages half the
+  // token tile, halving token traffic per weight byte). Narrow tiles (decode)
+  // stay on single CTAs.
+  const bool pair = p.bn_max >= 128 && num_sms >= 2;
   const int wrows = tile_rows(p.mode, pair);
   if (sp.ring_bytes < 2 * (a_tiles * A_BYTES + ceil_div(p.bn_max, BOX_N) * BOX_BYTES))
     return cudaErrorInvalidValue;
@@ -832,8 +815,6 @@ cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t 
   if (ngroup <= 0) return cudaSuccess;
   const int grid = pair ? 2 * ngroup : ngroup;
   switch (p.mode) {
-    case kUmmaRouter:
-      return launch_mode<kUmmaRouter, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s);
     case kUmmaSwiGLU:
       return pair ? launch_mode<kUmmaSwiGLU, true>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s)
                   : launch_mode<kUmmaSwiGLU, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s);
