@@ -302,11 +302,49 @@ def measure_backward(B, cfg, inp, touched, stream, reps):
     assert B.moe_get_device_error(wsb) == B.MOE_OK
     ms = e0.elapsed_time(e1) / reps
     flops, nbytes = backward_work(cfg, touched)
+
+    # Training step: moe_forward_train keeps routing and pre-activations in the
+    # workspace, moe_backward_saved uses them (no recomputation).
+    y = torch.empty((cfg.T, cfg.d), dtype=dt, device=dev)
+
+    def fwd_train():
+        B.moe_forward_train(cfg, inp["x"], inp["w_router"], inp["bias"], inp["w1"], inp["w3"], inp["w2"],
+                            inp["ws1"], inp["ws3"], inp["ws2"], y, wsb)
+
+    def bwd_saved():
+        B.moe_backward_saved(cfg, inp["x"], inp["w_router"], inp["w1"], inp["w3"], inp["w2"], inp["ws1"],
+                             inp["ws3"], inp["ws2"], dy, *outs, wsb)
+
+    def timed(fn):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        gg = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gg):
+            fn()
+        gg.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            gg.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        del gg
+        assert B.moe_get_device_error(wsb) == B.MOE_OK
+        return a.elapsed_time(b) / reps
+
+    fwd_train()
+    saved_ms = timed(bwd_saved)
+    step_ms = timed(lambda: (fwd_train(), bwd_saved()))
     del outs, wsb
     return {"ms_per_step": ms, "tokens_per_s": cfg.T / (ms / 1e3), "tflops": flops / (ms / 1e3) / 1e12,
             "gbs": nbytes / (ms / 1e3) / 1e9, "algorithmic_flops": flops, "algorithmic_bytes": nbytes,
             "graph_replays": reps,
-            "note": "recomputes routing and SwiGLU pre-activations; writes dx and every weight gradient"}
+            "note": "recomputes routing and SwiGLU pre-activations; writes dx and every weight gradient",
+            "saved_ms": saved_ms,
+            "train_step_ms": step_ms,
+            "train_step_note": "moe_forward_train + moe_backward_saved (pre-activations kept from the forward)"}
 
 
 def measure_fused_permute(B, cfg, inp, idx, offsets, perm_src, inv_row, h, h_s, ws, stream, reps):

@@ -328,6 +328,32 @@ MOE_API moe_status moe_backward(const moe_config* cfg, const void* x, const void
                         void* dws2, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * moe_forward_train - moe_forward for training: the same y, and the
+ * workspace (at least moe_backward_workspace_size(cfg) bytes) keeps what the
+ * backward pass would otherwise recompute: the routing (indices, gates,
+ * offsets, packed-row maps, router logits), the packed activations and the
+ * SwiGLU pre-activations W1 u and W3 u of every routed and shared row
+ * (dtype, written by the gate/up GEMM's epilogue).
+ */
+MOE_API moe_status moe_forward_train(const moe_config* cfg, const void* x, const void* w_router,
+                             const float* bias, const void* w1, const void* w3, const void* w2,
+                             const void* ws1, const void* ws3, const void* ws2, void* y,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * moe_backward_saved - moe_backward on the state moe_forward_train left in
+ * `workspace`: no routing, packing or pre-activation GEMMs are recomputed.
+ * x and the weights must be the ones that forward call used (they feed the
+ * weight gradients and the router's input gradient), and nothing may have
+ * written the workspace in between. Outputs as moe_backward's.
+ */
+MOE_API moe_status moe_backward_saved(const moe_config* cfg, const void* x, const void* w_router,
+                              const void* w1, const void* w3, const void* w2, const void* ws1,
+                              const void* ws3, const void* ws2, const void* dy, void* dx,
+                              void* dw_router, void* dw1, void* dw3, void* dw2, void* dws1, void* dws3,
+                              void* dws2, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * moe_route_noalloc - moe_route for callers that cannot allocate device
  * memory (no workspace argument). Same arguments and outputs as moe_route
  * minus the workspace. The pages have no counterpart: this entry point only

@@ -34,7 +34,7 @@ EXPORTED = ("moe_check_config", "moe_workspace_size", "moe_route", "moe_permute"
             "moe_combine", "moe_forward", "moe_get_device_error",
             "moe_selftest_wait_timeout", "moe_route_noalloc", "moe_balance_update",
             "moe_expert_gelu", "moe_forward_gelu", "moe_backward_workspace_size", "moe_backward",
-            "moe_status_string")
+            "moe_forward_train", "moe_backward_saved", "moe_status_string")
 
 
 class MoEError(RuntimeError):
@@ -88,6 +88,9 @@ def lib() -> ctypes.CDLL:
             "moe_expert_gelu": (ctypes.c_int, [cfgp, vp, i32p, vp, f32p, vp, f32p, vp, vp, sz, vp]),
             "moe_forward_gelu": (ctypes.c_int, [cfgp, vp, vp, f32p, vp, f32p, vp, f32p, vp, vp, sz, vp]),
             "moe_backward_workspace_size": (sz, [cfgp]),
+            "moe_forward_train": (ctypes.c_int, [cfgp, vp, vp, f32p, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+            "moe_backward_saved": (ctypes.c_int, [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                                  vp, vp, vp, vp, sz, vp]),
             "moe_backward": (ctypes.c_int, [cfgp, vp, vp, f32p, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                             vp, vp, vp, vp, sz, vp]),
             "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -251,6 +254,24 @@ def moe_backward(cfg, x, w_router, bias, w1, w3, w2, ws1, ws3, ws2, dy, dx, dw_r
                               _ptr(w2), _ptr(ws1), _ptr(ws3), _ptr(ws2), _ptr(dy), _ptr(dx), _ptr(dw_router),
                               _ptr(dw1), _ptr(dw3), _ptr(dw2), _ptr(dws1), _ptr(dws3), _ptr(dws2),
                               _ptr(workspace), workspace.numel(), _stream(stream)), "moe_backward")
+
+
+def moe_forward_train(cfg, x, w_router, bias, w1, w3, w2, ws1, ws3, ws2, y, workspace, stream=None):
+    """moe_forward that keeps routing and pre-activations in a backward-size workspace."""
+    c = _cfg(cfg)
+    _check(lib().moe_forward_train(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w1), _ptr(w3),
+                                   _ptr(w2), _ptr(ws1), _ptr(ws3), _ptr(ws2), _ptr(y), _ptr(workspace),
+                                   workspace.numel(), _stream(stream)), "moe_forward_train")
+
+
+def moe_backward_saved(cfg, x, w_router, w1, w3, w2, ws1, ws3, ws2, dy, dx, dw_router, dw1, dw3, dw2,
+                       dws1, dws3, dws2, workspace, stream=None):
+    """moe_backward on the state moe_forward_train left in `workspace`."""
+    c = _cfg(cfg)
+    _check(lib().moe_backward_saved(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(w1), _ptr(w3), _ptr(w2),
+                                    _ptr(ws1), _ptr(ws3), _ptr(ws2), _ptr(dy), _ptr(dx), _ptr(dw_router),
+                                    _ptr(dw1), _ptr(dw3), _ptr(dw2), _ptr(dws1), _ptr(dws3), _ptr(dws2),
+                                    _ptr(workspace), workspace.numel(), _stream(stream)), "moe_backward_saved")
 
 
 def moe_route_noalloc(cfg, x, w_router, bias, topk_idx, topk_gate, expert_counts, expert_offsets,

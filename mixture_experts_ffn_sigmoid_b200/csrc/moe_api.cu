@@ -174,7 +174,7 @@ int expert_tile_n(const moe_config& c) {
 moe_status enqueue_gate_up(const moe_config& c, const void* x_perm, const int* offsets, const void* w1,
                            const void* w3, const void* x_sh, const void* ws1, const void* ws3, void* h,
                            void* h_s, uint32_t* err, cudaStream_t s, const int* gather_rows = nullptr,
-                           const void* gather_src = nullptr) {
+                           const void* gather_src = nullptr, void* const* pre = nullptr) {
   const bool shared = c.f_shared > 0;
   const int rows = c.T * c.k;
   if (c.dtype == MOE_DTYPE_BF16) {
@@ -203,6 +203,10 @@ moe_status enqueue_gate_up(const moe_config& c, const void* x_perm, const int* o
       g.b_gather_src = gather_src;
       g.b_gather_rows = c.T;
     }
+    if (pre) {
+      g.mode = kUmmaSwiGLUSave;
+      g.pre_a = pre[0]; g.pre_b = pre[1]; g.pre_a_s = pre[2]; g.pre_b_s = pre[3];
+    }
     MOE_CUDA(launch_umma_gemm(g, device_sm_count(), s));
   } else {
     SimtGemmParams g = {};
@@ -215,6 +219,7 @@ moe_status enqueue_gate_up(const moe_config& c, const void* x_perm, const int* o
     g.a_s = x_sh; g.b1_s = ws1; g.b3_s = ws3; g.out_s = h_s;
     g.N_s = c.f_shared; g.K_s = c.d;
     g.max_rows = rows;
+    if (pre) { g.pre_a = pre[0]; g.pre_b = pre[1]; g.pre_a_s = pre[2]; g.pre_b_s = pre[3]; }
     MOE_CUDA(launch_simt_gemm(c.dtype, 0, g, s));
   }
   return MOE_OK;
@@ -267,12 +272,12 @@ moe_status enqueue_down(const moe_config& c, const void* h, const int* offsets, 
 moe_status enqueue_experts(const moe_config& c, const void* x_perm, const int* offsets, const void* w1,
                            const void* w3, const void* w2, const void* x_sh, const void* ws1,
                            const void* ws3, const void* ws2, void* y_perm, void* y_sh, void* ws,
-                           cudaStream_t s) {
+                           cudaStream_t s, void* const* pre = nullptr) {
   const Layout L = layout_of(c);
   void* h = at<char>(ws, L.h);
   void* h_s = at<char>(ws, L.h_s);
   uint32_t* err = at<uint32_t>(ws, L.err);
-  MOE_TRY(enqueue_gate_up(c, x_perm, offsets, w1, w3, x_sh, ws1, ws3, h, h_s, err, s));
+  MOE_TRY(enqueue_gate_up(c, x_perm, offsets, w1, w3, x_sh, ws1, ws3, h, h_s, err, s, nullptr, nullptr, pre));
   return enqueue_down(c, h, offsets, w2, h_s, ws2, y_perm, y_sh, err, s);
 }
 
@@ -484,11 +489,13 @@ moe_status enqueue_preact(const moe_config& c, const void* x_perm, const int* of
   return MOE_OK;
 }
 
+// recompute: route, pack x and compute the pre-activations here; otherwise
+// they are the state a training forward left in this workspace.
 moe_status enqueue_backward(const moe_config& c, const void* x, const void* w_router, const float* bias,
                             const void* w1, const void* w3, const void* w2, const void* ws1,
                             const void* ws3, const void* ws2, const void* dy, void* dx, void* dw_router,
                             void* dw1, void* dw3, void* dw2, void* dws1, void* dws3, void* dws2,
-                            void* ws, cudaStream_t s) {
+                            void* ws, cudaStream_t s, bool recompute = true) {
   const Layout L = layout_of(c);
   const BwdLayout Bw = bwd_layout_of(c);
   const bool shared = c.f_shared > 0;
@@ -504,14 +511,16 @@ moe_status enqueue_backward(const moe_config& c, const void* x, const void* w_ro
   char* x_perm = at<char>(ws, L.x_perm);
   char* dyp = at<char>(ws, Bw.dyp);
   const int nsm = device_sm_count();
-  // Forward state: routing, packed x, packed dy, pre-activations.
-  MOE_TRY(enqueue_route(c, x, w_router, bias, idx, gate, at<int>(ws, L.counts), offsets, ws, s));
-  MOE_CUDA(launch_permute(c.dtype, x, idx, offsets, at<int>(ws, L.cbase), c.T, c.d, c.E, c.k, x_perm,
-                          perm_src, inv_row, nsm, s, true));
+  // Forward state: routing, packed x, pre-activations; then packed dy.
+  if (recompute) {
+    MOE_TRY(enqueue_route(c, x, w_router, bias, idx, gate, at<int>(ws, L.counts), offsets, ws, s));
+    MOE_CUDA(launch_permute(c.dtype, x, idx, offsets, at<int>(ws, L.cbase), c.T, c.d, c.E, c.k, x_perm,
+                            perm_src, inv_row, nsm, s, true));
+    MOE_TRY(enqueue_preact(c, x_perm, offsets, x, w1, w3, ws1, ws3, at<char>(ws, Bw.a), at<char>(ws, Bw.b),
+                           at<char>(ws, Bw.a_s), at<char>(ws, Bw.b_s), err, s));
+  }
   MOE_CUDA(launch_permute(c.dtype, dy, idx, offsets, at<int>(ws, L.cbase), c.T, c.d, c.E, c.k, dyp,
                           perm_src, inv_row, nsm, s, true));
-  MOE_TRY(enqueue_preact(c, x_perm, offsets, x, w1, w3, ws1, ws3, at<char>(ws, Bw.a), at<char>(ws, Bw.b),
-                         at<char>(ws, Bw.a_s), at<char>(ws, Bw.b_s), err, s));
   // dh' = W2^T dy per packed row (gate not applied), and the shared expert's.
   const bool tc = c.dtype == MOE_DTYPE_BF16;
   constexpr int kNoSplit = 1 << 30;
@@ -970,11 +979,15 @@ size_t moe_backward_workspace_size(const moe_config* cfg) {
   return bwd_layout_of(*cfg).total;
 }
 
-moe_status moe_backward(const moe_config* cfg, const void* x, const void* w_router, const float* bias,
-                        const void* w1, const void* w3, const void* w2, const void* ws1, const void* ws3,
-                        const void* ws2, const void* dy, void* dx, void* dw_router, void* dw1, void* dw3,
-                        void* dw2, void* dws1, void* dws3, void* dws2, void* workspace, size_t ws_bytes,
-                        void* stream) {
+}  // extern "C"
+
+namespace moe {
+namespace {
+moe_status backward_entry(const moe_config* cfg, const void* x, const void* w_router, const float* bias,
+                          const void* w1, const void* w3, const void* w2, const void* ws1, const void* ws3,
+                          const void* ws2, const void* dy, void* dx, void* dw_router, void* dw1, void* dw3,
+                          void* dw2, void* dws1, void* dws3, void* dws2, void* workspace, size_t ws_bytes,
+                          void* stream, bool recompute) {
   MOE_TRY(check_config(cfg));
   const moe_config& c = *cfg;
   MOE_TRY(need(workspace));
@@ -1008,7 +1021,73 @@ moe_status moe_backward(const moe_config* cfg, const void* x, const void* w_rout
   }
   MOE_TRY(clear_error_word(workspace, s));
   return enqueue_backward(c, x, w_router, bias, w1, w3, w2, ws1, ws3, ws2, dy, dx, dw_router, dw1, dw3, dw2,
-                          dws1, dws3, dws2, workspace, s);
+                          dws1, dws3, dws2, workspace, s, recompute);
+}
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
+moe_status moe_backward(const moe_config* cfg, const void* x, const void* w_router, const float* bias,
+                        const void* w1, const void* w3, const void* w2, const void* ws1, const void* ws3,
+                        const void* ws2, const void* dy, void* dx, void* dw_router, void* dw1, void* dw3,
+                        void* dw2, void* dws1, void* dws3, void* dws2, void* workspace, size_t ws_bytes,
+                        void* stream) {
+  return backward_entry(cfg, x, w_router, bias, w1, w3, w2, ws1, ws3, ws2, dy, dx, dw_router, dw1, dw3, dw2,
+                        dws1, dws3, dws2, workspace, ws_bytes, stream, true);
+}
+
+moe_status moe_backward_saved(const moe_config* cfg, const void* x, const void* w_router, const void* w1,
+                              const void* w3, const void* w2, const void* ws1, const void* ws3,
+                              const void* ws2, const void* dy, void* dx, void* dw_router, void* dw1,
+                              void* dw3, void* dw2, void* dws1, void* dws3, void* dws2, void* workspace,
+                              size_t ws_bytes, void* stream) {
+  return backward_entry(cfg, x, w_router, nullptr, w1, w3, w2, ws1, ws3, ws2, dy, dx, dw_router, dw1, dw3,
+                        dw2, dws1, dws3, dws2, workspace, ws_bytes, stream, false);
+}
+
+moe_status moe_forward_train(const moe_config* cfg, const void* x, const void* w_router, const float* bias,
+                             const void* w1, const void* w3, const void* w2, const void* ws1,
+                             const void* ws3, const void* ws2, void* y, void* workspace, size_t ws_bytes,
+                             void* stream) {
+  MOE_TRY(check_config(cfg));
+  const moe_config& c = *cfg;
+  MOE_TRY(need(workspace));
+  if (ws_bytes < bwd_layout_of(c).total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (c.T == 0) return MOE_OK;
+  MOE_TRY(need(x));
+  MOE_TRY(need(w_router));
+  if (bias) MOE_TRY(need4(bias));
+  MOE_TRY(need(w1));
+  MOE_TRY(need(w3));
+  MOE_TRY(need(w2));
+  MOE_TRY(need(y));
+  if (c.f_shared > 0) {
+    MOE_TRY(need(ws1));
+    MOE_TRY(need(ws3));
+    MOE_TRY(need(ws2));
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const Layout L = layout_of(c);
+  const BwdLayout Bw = bwd_layout_of(c);
+  void* ws = workspace;
+  MOE_TRY(clear_error_word(ws, s));
+  int* idx = at<int>(ws, L.idx);
+  float* gate = at<float>(ws, L.gate);
+  int* offsets = at<int>(ws, L.offsets);
+  MOE_TRY(enqueue_route(c, x, w_router, bias, idx, gate, at<int>(ws, L.counts), offsets, ws, s));
+  MOE_CUDA(launch_permute(c.dtype, x, idx, offsets, at<int>(ws, L.cbase), c.T, c.d, c.E, c.k,
+                          at<char>(ws, L.x_perm), at<int>(ws, L.perm_src), at<int>(ws, L.inv_row),
+                          device_sm_count(), s, true));
+  const bool shared = c.f_shared > 0;
+  void* y_s = shared ? at<char>(ws, L.y_s) : nullptr;
+  void* pre[4] = {at<char>(ws, Bw.a), at<char>(ws, Bw.b), shared ? at<char>(ws, Bw.a_s) : nullptr,
+                  shared ? at<char>(ws, Bw.b_s) : nullptr};
+  MOE_TRY(enqueue_experts(c, at<char>(ws, L.x_perm), offsets, w1, w3, w2, shared ? x : nullptr, ws1, ws3, ws2,
+                          at<char>(ws, L.y_perm), y_s, ws, s, pre));
+  MOE_CUDA(launch_combine(c.dtype, at<char>(ws, L.y_perm), at<int>(ws, L.inv_row), gate, y_s, y, c.T, c.d, c.k,
+                          device_sm_count(), s));
+  return MOE_OK;
 }
 
 moe_status moe_balance_update(const moe_config* cfg, const int32_t* expert_counts, float* bias,

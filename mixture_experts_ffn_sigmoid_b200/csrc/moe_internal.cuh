@@ -86,6 +86,8 @@ struct SimtGemmParams {
   const void* a_s; const void* b1_s; const void* b3_s; void* out_s;
   int N_s, K_s;
   int max_rows;             // upper bound on routed rows (T*k) for the grid
+  // Dual GEMM, optional: also store A B1^T and A B3^T (pre-activations).
+  void* pre_a; void* pre_b; void* pre_a_s; void* pre_b_s;
   // Single GEMM only: out = act(A B1^T + bias), bias fp32 [n_routed][N] / [N_s] or null.
   const float* bias1; const float* bias1_s;
   int act;                  // kActNone or kActGelu
@@ -120,7 +122,7 @@ cudaError_t launch_unpermute_sum(int dtype, const float* dxp, const int* inv_row
                                  const float* dxr, void* dx, int T, int d, int k, cudaStream_t s);
 
 // tcgen05 grouped GEMM (umma_gemm.cu)
-enum UmmaMode { kUmmaSwiGLU = 1, kUmmaDown = 2, kUmmaBiasAct = 3, kUmmaDgrad = 4 };
+enum UmmaMode { kUmmaSwiGLU = 1, kUmmaDown = 2, kUmmaBiasAct = 3, kUmmaDgrad = 4, kUmmaSwiGLUSave = 5 };
 struct UmmaGemmParams {
   int mode;
   int n_routed;             // routed segments
@@ -156,6 +158,9 @@ struct UmmaGemmParams {
   int a_k_rows, a_k_rows_s;
   int k_split, k_split_s;
   int out_f32;              // kUmmaDgrad: fp32 output instead of bf16
+  // kUmmaSwiGLUSave: also store the pre-activations W1 u, W3 u (bf16, laid
+  // out like out / out_s) for a later backward pass.
+  void* pre_a; void* pre_b; void* pre_a_s; void* pre_b_s;
 };
 cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t s);
 

@@ -27,6 +27,7 @@ struct Seg {
   const void* a; const void* b1; const void* b3; void* out;
   int row0, rows, N, K;
   const float* bias;   // this segment's bias row [N], or null
+  void* pre_a; void* pre_b;   // dual: optional pre-activation outputs
 };
 
 template <typename TI, typename TO, bool DUAL>
@@ -46,7 +47,7 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGemmParams p) {
       sg = Seg{p.a, (const char*)p.b1 + (size_t)s * p.N * p.K * sizeof(TI),
                DUAL ? (const char*)p.b3 + (size_t)s * p.N * p.K * sizeof(TI) : nullptr,
                p.out, r0 + bx * TM, min(TM, rows - bx * TM), p.N, p.K,
-               p.bias1 ? p.bias1 + (size_t)s * p.N : nullptr};
+               p.bias1 ? p.bias1 + (size_t)s * p.N : nullptr, p.pre_a, p.pre_b};
       found = true;
       break;
     }
@@ -56,7 +57,7 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGemmParams p) {
     const int tiles = (p.shared_rows + TM - 1) / TM;
     if (bx < tiles) {
       sg = Seg{p.a_s, p.b1_s, p.b3_s, p.out_s, bx * TM, min(TM, p.shared_rows - bx * TM), p.N_s, p.K_s,
-               p.bias1_s};
+               p.bias1_s, p.pre_a_s, p.pre_b_s};
       found = true;
     }
   }
@@ -119,6 +120,11 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGemmParams p) {
       if (n >= sg.N) continue;
       float v = acc1[i][j];
       if (DUAL) {
+        if (sg.pre_a) {
+          const size_t o = (size_t)(sg.row0 + r) * sg.N + n;
+          static_cast<TO*>(sg.pre_a)[o] = from_f32<TO>(v);
+          static_cast<TO*>(sg.pre_b)[o] = from_f32<TO>(acc3[i][j]);
+        }
         v = (v / (1.0f + expf(-v))) * acc3[i][j];
       } else {
         if (sg.bias) v += sg.bias[n];

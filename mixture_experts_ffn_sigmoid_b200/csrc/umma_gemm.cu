@@ -5,6 +5,8 @@
 // R^{d x f}; the router logits have their own kernel, umma_router.cu):
 //
 //   kUmmaSwiGLU: h[r][m] = SiLU(sum_c W1_e[m][c] x[r][c]) * (sum_c W3_e[m][c] x[r][c])
+//   kUmmaSwiGLUSave: the same, also storing both sums (the pre-activations a
+//                training forward keeps for the backward pass)
 //   kUmmaDown:   y[r][m] = sum_c W2_e[m][c] h[r][c]
 //   kUmmaBiasAct: o[r][m] = act(sum_c W_e[m][c] u[r][c] + b_e[m]), act = GELU or
 //                identity (the generic expert of "Lesson 2 - From the Dense FFN
@@ -187,6 +189,10 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar, uint16_t mask) {
 // of every weight block and half of the token tile.
 template <int MODE> struct Kind;
 template <> struct Kind<kUmmaSwiGLU> { static constexpr int A_TILES = 2; static constexpr int ACC_STAGES = 1; };
+template <> struct Kind<kUmmaSwiGLUSave> { static constexpr int A_TILES = 2; static constexpr int ACC_STAGES = 1; };
+
+// Modes whose tile pairs the W1 and W3 rows of one range (SwiGLU).
+__host__ __device__ constexpr bool dual_a(int mode) { return mode == kUmmaSwiGLU || mode == kUmmaSwiGLUSave; }
 template <> struct Kind<kUmmaDown>   { static constexpr int A_TILES = 2; static constexpr int ACC_STAGES = 1; };
 template <> struct Kind<kUmmaBiasAct> { static constexpr int A_TILES = 2; static constexpr int ACC_STAGES = 1; };
 template <> struct Kind<kUmmaDgrad> { static constexpr int A_TILES = 2; static constexpr int ACC_STAGES = 1; };
@@ -332,7 +338,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
   if (threadIdx.x == 0) {
     tmap_prefetch(&tmA); tmap_prefetch(&tmB); tmap_prefetch(&tmAs); tmap_prefetch(&tmBs);
-    if (MODE == kUmmaSwiGLU) { tmap_prefetch(&tmA3); tmap_prefetch(&tmA3s); }
+    if (dual_a(MODE)) { tmap_prefetch(&tmA3); tmap_prefetch(&tmA3s); }
     if (p.b_gather) tmap_prefetch(&tmG);
   }
   __syncthreads();
@@ -442,7 +448,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                  crow, fb);
           } else {
             tma_load_2d_pair(sb, mA, kb * BK, a_row, fb);
-            if (MODE == kUmmaSwiGLU) tma_load_2d_pair(sb + A_BYTES, mA3, kb * BK, a_row, fb);
+            if (dual_a(MODE)) tma_load_2d_pair(sb + A_BYTES, mA3, kb * BK, a_row, fb);
             if (two_blocks(MODE)) tma_load_2d_pair(sb + A_BYTES, mA, kb * BK, a_row + BLOCK_STEP, fb);
           }
           if (ts.rows_gather > 0) {
@@ -467,7 +473,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             fb_local);
           } else {
             tma_load_2d(sb, mA, kb * BK, a_row, fb_local);
-            if (MODE == kUmmaSwiGLU) tma_load_2d(sb + A_BYTES, mA3, kb * BK, a_row, fb_local);
+            if (dual_a(MODE)) tma_load_2d(sb + A_BYTES, mA3, kb * BK, a_row, fb_local);
             if (two_blocks(MODE)) tma_load_2d(sb + A_BYTES, mA, kb * BK, a_row + BLOCK_STEP, fb_local);
           }
           if (ts.rows_gather > 0) {
@@ -579,15 +585,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const long long r0 = (long long)t.b_row0 + (long long)t.tt * p.bn_max;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MAX);
       const uint32_t acce = acce0 + (uint32_t)(acc * 8);
-      if (MODE == kUmmaSwiGLU) {
+      if (dual_a(MODE)) {
         // Drain both accumulators into registers as packed bf16 h, hand TMEM
         // back to the MMA warp, then store while the next tile accumulates.
+        __nv_bfloat16* pre_a = nullptr;
+        __nv_bfloat16* pre_b = nullptr;
+        if (MODE == kUmmaSwiGLUSave) {
+          pre_a = static_cast<__nv_bfloat16*>(t.dense ? p.pre_a_s : p.pre_a) + r0 * ld;
+          pre_b = static_cast<__nv_bfloat16*>(t.dense ? p.pre_b_s : p.pre_b) + r0 * ld;
+        }
         uint32_t hp[BN_MAX / 2];
 #pragma unroll
         for (int c = 0; c < BN_MAX / 16; ++c) {
           if (c * 16 < n_mma) {
             uint32_t r1[16], r3[16];
             tmem_ld16x2_wait(taddr + c * 16, taddr + BN_MAX + c * 16, r1, r3);
+            if (MODE == kUmmaSwiGLUSave && m_ok) {
+              // Training forward: keep W1 u and W3 u (bf16) for the backward.
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const int col = c * 16 + j;
+                if (col < n_valid) {
+                  pre_a[(long long)col * ld + m] = __float2bfloat16_rn(__uint_as_float(r1[j]));
+                  pre_b[(long long)col * ld + m] = __float2bfloat16_rn(__uint_as_float(r3[j]));
+                }
+              }
+            }
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
               const float g0 = __uint_as_float(r1[2 * j]), g1 = __uint_as_float(r1[2 * j + 1]);
@@ -774,7 +797,7 @@ cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t 
   const int wrows = tile_rows(p.mode, pair);
   if (sp.ring_bytes < 2 * (a_tiles * A_BYTES + ceil_div(p.bn_max, BOX_N) * BOX_BYTES))
     return cudaErrorInvalidValue;
-  const bool swiglu = p.mode == kUmmaSwiGLU;
+  const bool swiglu = dual_a(p.mode);
   const bool dgrad = p.mode == kUmmaDgrad;
   CUtensorMap tA, tA3, tB, tAs, tA3s, tBs;
   if (has_dense) {
@@ -818,6 +841,9 @@ cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t 
     case kUmmaSwiGLU:
       return pair ? launch_mode<kUmmaSwiGLU, true>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s)
                   : launch_mode<kUmmaSwiGLU, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s);
+    case kUmmaSwiGLUSave:
+      return pair ? launch_mode<kUmmaSwiGLUSave, true>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s)
+                  : launch_mode<kUmmaSwiGLUSave, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s);
     case kUmmaDown:
       return pair ? launch_mode<kUmmaDown, true>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s)
                   : launch_mode<kUmmaDown, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s);

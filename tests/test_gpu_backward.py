@@ -207,3 +207,26 @@ def test_backward_full_size_sampled():
     compare_grad(cfg, H.f64(got["dws2"])[:, units], s2, "dws2 (sampled columns)")
     for n in NAMES:
         assert torch.isfinite(got[n].float()).all().item(), n
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_training_forward_then_saved_backward(results, name):
+    # moe_forward_train gives moe_forward's bytes, and moe_backward_saved on
+    # its workspace gives moe_backward's bytes (same kernels, same operands:
+    # the pre-activations come from the gate/up epilogue instead of a
+    # recomputing GEMM with the same accumulation order).
+    cfg, inp, dy, got, ref, rep = results[name]
+    ws = B.alloc_backward_workspace(cfg)
+    y = torch.full((cfg.T, cfg.d), float("nan"), dtype=cfg.torch_dtype, device="cuda")
+    B.moe_forward_train(cfg, inp["x"], inp["w_router"], inp["bias"], inp["w1"], inp["w3"], inp["w2"], inp["ws1"],
+                        inp["ws3"], inp["ws2"], y, ws)
+    assert torch.equal(y, H.gpu_forward(cfg, inp))
+    dt = cfg.torch_dtype
+    out = {n: (torch.full_like(got[n], float("nan")) if got[n] is not None else None) for n in NAMES}
+    B.moe_backward_saved(cfg, inp["x"], inp["w_router"], inp["w1"], inp["w3"], inp["w2"], inp["ws1"], inp["ws3"],
+                         inp["ws2"], dy, out["dx"], out["dw_router"], out["dw1"], out["dw3"], out["dw2"],
+                         out["dws1"], out["dws3"], out["dws2"], ws)
+    assert B.moe_get_device_error(ws) == B.MOE_OK
+    for n in NAMES:
+        if got[n] is not None:
+            assert torch.equal(out[n], got[n]), n

@@ -27,6 +27,10 @@ STAGE_CASES = {
                                   route_scale=1.0, f_shared=40, bias="uniform"),
     "ragged_dims_fp32": MoEConfig("ragged_dims_f32", T=77, d=200, E=12, k=3, f=72, dtype="f32",
                                   gate_mode=GATE_SIGMOID, f_shared=40, bias="uniform"),
+    # More than 256 experts: the router's second expert tile; ragged T and
+    # segments of a handful of rows.
+    "wide_experts_bf16": MoEConfig("wide_experts", T=150, d=192, E=320, k=6, f=64, gate_mode=GATE_SIGMOID,
+                                   n_groups=8, topk_groups=4, route_scale=2.5, f_shared=64, bias="uniform"),
 }
 
 
