@@ -10,8 +10,8 @@
 // (Sparse MoE FFN note, "Packed forward": each expert sees the tokens that
 // chose it). Segments no row belongs to get D_s = 0.
 //
-// Tiles: 128 m x 256 n per CTA (one M=128, N=256 MMA per 16 rows), rows in
-// blocks of 64. Both operands arrive as 64 x 64 TMA boxes (128-byte swizzle,
+// Tiles: 256 m x 256 n per CTA (two M=128, N=256 MMAs per 16 rows, one
+// per 128-row M block, sharing the staged Q tile), rows in blocks of 64. Both operands arrive as 64 x 64 TMA boxes (128-byte swizzle,
 // MN-major: 64-element M/N groups 8 KB apart, 8-row groups 1 KB apart).
 // Rows of the last block past the segment's end belong to the next segment:
 // the MMA warp zeroes those rows of the P tile in shared memory before the
@@ -22,40 +22,50 @@
 //   warp 0 lane 0 : TMA producer into a 4-stage ring
 //   warp 1        : TMEM allocator; zero-fills partial blocks; lane 0 issues
 //                   tcgen05.mma and tcgen05.commit
-//   warps 2..9    : epilogue; warp w reads TMEM lane quarter w % 4 and half
-//                   of the 256 columns, 64 columns per load wait; two TMEM
-//                   accumulators (2 x 256 columns), so a tile's stores
-//                   overlap the next tile's MMAs
+//   warps 2..9    : epilogue; warp w reads TMEM lane quarter w % 4 of one M
+//                   block (or half the columns with one block), 64 columns per
+//                   load wait, and writes 32 x 64 boxes with TMA stores
 // Every wait is bounded, as in the forward GEMM.
 #include "umma_common.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int WG_BM = 128;
+// Tile shapes. WG_MB 128-row M blocks per tile: two blocks share each
+// staged Q tile, cutting the operands read per output byte by a third, but
+// their accumulators (2 x 256 TMEM columns) fill TMEM, so the next tile's
+// MMAs wait for the epilogue; one block keeps two accumulator stages. Long
+// contractions (hundreds of rows per segment) take two blocks, short ones one.
+template <int MB> struct WgShape {
+  static constexpr int BM = 128 * MB;
+  static constexpr int ACC_STAGES = MB == 1 ? 2 : 1;
+  static constexpr int STAGES = MB == 1 ? 4 : 3;
+};
 constexpr int WG_BN = 256;
 constexpr int WG_BK = 64;
-constexpr int WG_STAGES = 4;
 constexpr int WG_BOX = 64 * 64 * 2;                      // one 64 x 64 bf16 box
-constexpr int WG_A_BYTES = 2 * WG_BOX;                   // 128 m x 64 rows
 constexpr int WG_B_BYTES = 4 * WG_BOX;                   // 256 n x 64 rows
-constexpr int WG_STAGE_BYTES = WG_A_BYTES + WG_B_BYTES;
 constexpr int WG_THREADS = 320;
 constexpr int WG_EPI_WARPS = 8;
 constexpr int WG_STG_BYTES = 32 * 64 * 2;                // one warp's 32 x 64 output box
-constexpr int WG_SMEM = 1024 + 1024 + WG_STAGES * WG_STAGE_BYTES + WG_EPI_WARPS * WG_STG_BYTES;
 constexpr int WG_TMEM_COLS = 512;
+template <int MB> constexpr int wg_a_bytes() { return 2 * MB * WG_BOX; }
+template <int MB> constexpr int wg_stage_bytes() { return wg_a_bytes<MB>() + WG_B_BYTES; }
+template <int MB> constexpr int wg_smem() {
+  return 1024 + 1024 + WgShape<MB>::STAGES * wg_stage_bytes<MB>() + WG_EPI_WARPS * WG_STG_BYTES;
+}
 
 struct WgTile {
   int seg, m0, n0, r0, rows, nk;
 };
 
+template <int BM>
 __device__ __forceinline__ WgTile wg_tile(const WgradParams& p, int tile, int mt, int nt) {
   WgTile t;
   const int per_seg = mt * nt;
   t.seg = tile / per_seg;
   const int rem = tile - t.seg * per_seg;
-  t.m0 = (rem / nt) * WG_BM;
+  t.m0 = (rem / nt) * BM;
   t.n0 = (rem - (rem / nt) * nt) * WG_BN;
   if (p.offsets) {
     t.r0 = p.offsets[t.seg];
@@ -72,9 +82,15 @@ __device__ __forceinline__ void st_shared_zero16(uint32_t addr) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
 }
 
+template <int WG_MB>
 __global__ void __launch_bounds__(WG_THREADS, 1)
     wgrad_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                  const __grid_constant__ CUtensorMap tmD, const WgradParams p) {
+  constexpr int WG_BM = WgShape<WG_MB>::BM;
+  constexpr int WG_ACC_STAGES = WgShape<WG_MB>::ACC_STAGES;
+  constexpr int WG_STAGES = WgShape<WG_MB>::STAGES;
+  constexpr int WG_A_BYTES = wg_a_bytes<WG_MB>();
+  constexpr int WG_STAGE_BYTES = wg_stage_bytes<WG_MB>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -123,7 +139,7 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
     uint32_t phase = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-      const WgTile t = wg_tile(p, tile, mt, nt);
+      const WgTile t = wg_tile<WG_BM>(p, tile, mt, nt);
       for (int kb = 0; kb < t.nk; ++kb) {
         if (!wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag, p.err, p.timeout_ns, true)) {
           ok = false;
@@ -135,7 +151,7 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
         const int r = t.r0 + kb * WG_BK;
         // Boxes wholly past M or N are not loaded: the rows (columns) of D
         // they feed are never stored.
-        const int na = min(2, ceil_div(p.M - t.m0, 64)), nb = min(4, ceil_div(p.N - t.n0, 64));
+        const int na = min(2 * WG_MB, ceil_div(p.M - t.m0, 64)), nb = min(4, ceil_div(p.N - t.n0, 64));
         mbar_expect_tx(fb, (uint32_t)(na + nb) * WG_BOX);
         for (int h = 0; h < na; ++h) tma_load_2d(sa + h * WG_BOX, &tmP, t.m0 + h * 64, r, fb);
         for (int h = 0; h < nb; ++h) tma_load_2d(sbq + h * WG_BOX, &tmQ, t.n0 + h * 64, r, fb);
@@ -149,17 +165,17 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     bool issued = false, ok = true;
-    const uint32_t idesc = idesc_bf16_f32(WG_BM, WG_BN) | (1u << 15) | (1u << 16);
+    const uint32_t idesc = idesc_bf16_f32(128, WG_BN) | (1u << 15) | (1u << 16);
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-      const WgTile t = wg_tile(p, tile, mt, nt);
+      const WgTile t = wg_tile<WG_BM>(p, tile, mt, nt);
       if (t.nk == 0) continue;                  // the epilogue writes zeros
       // Lane 0 waits; the outcome is broadcast so the warp stays converged.
       int w_ok = lane == 0 ? (int)wait_bounded(smem_u32(&acce_bar[acc]), acc_phase ^ 1u, abort_flag, p.err,
                                                p.timeout_ns, true) : 0;
       if (!__shfl_sync(0xffffffffu, w_ok, 0)) break;
       tc_fence_after();
-      const uint32_t d = tmem_base + (uint32_t)(acc * WG_BN);
-      const int na = min(2, ceil_div(p.M - t.m0, 64));
+      const uint32_t d = tmem_base + (uint32_t)(acc * WG_BN);   // block b adds b * WG_BN (WG_MB == 2)
+      const int na = min(2 * WG_MB, ceil_div(p.M - t.m0, 64));
       for (int kb = 0; kb < t.nk; ++kb) {
         w_ok = lane == 0 ? (int)wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, p.err, p.timeout_ns,
                                              true) : 0;
@@ -185,12 +201,16 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
         __syncwarp();
         tc_fence_after();
         if (lane == 0) {
-          const uint64_t a_desc = sw128_mn_desc(sa);
           const uint64_t b_desc = sw128_mn_desc(sa + WG_A_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < WG_BK / 16; ++kk) {
-            const uint64_t koff = (uint64_t)((kk * 2 * 1024) >> 4);   // two 8-row groups per 16 rows
-            umma_bf16(d, a_desc + koff, b_desc + koff, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          for (int blk = 0; blk < WG_MB; ++blk) {
+            if (blk * 128 >= p.M - t.m0) break;   // block wholly past M: not loaded, not needed
+            const uint64_t a_desc = sw128_mn_desc(sa + blk * 2 * WG_BOX);
+#pragma unroll
+            for (int kk = 0; kk < WG_BK / 16; ++kk) {
+              const uint64_t koff = (uint64_t)((kk * 2 * 1024) >> 4);   // two 8-row groups per 16 rows
+              umma_bf16(d + blk * WG_BN, a_desc + koff, b_desc + koff, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            }
           }
           umma_commit(smem_u32(&empty_bar[stage]));
         }
@@ -201,8 +221,7 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
       if (!ok) break;
       if (lane == 0) umma_commit(smem_u32(&accf_bar[acc]));
       __syncwarp();
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
+      if (++acc == WG_ACC_STAGES) { acc = 0; acc_phase ^= 1u; }
     }
     if (issued && lane == 0) {   // every MMA completes before TMEM is freed
       umma_commit(smem_u32(drain_bar));
@@ -217,17 +236,22 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
     // bulk write per 4 KB instead of 32 scattered 16-byte stores per
     // instruction. The 3-D output map clips rows past M and columns past N.
     const int q = warp & 3;                    // TMEM lane quarter this warp may read
-    const int half = (warp - 2) >> 2;          // columns [128 half, 128 half + 128)
+    // Warps 2-5 and 6-9 split the tile: by M block when there are two (each
+    // warp then stores all 256 columns of its 32 rows), else by column half.
+    const int grp = (warp - 2) >> 2;
+    const int blk = WG_MB == 2 ? grp : 0;
+    const int ncol = WG_MB == 2 ? WG_BN : WG_BN / 2;
+    const int cbeg = WG_MB == 2 ? 0 : grp * (WG_BN / 2);
     const uint32_t box = smem_u32(stage_out + (warp - 2) * WG_STG_BYTES);
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      const WgTile t = wg_tile(p, tile, mt, nt);
-      const int mrow = t.m0 + q * 32;          // first row of this warp's boxes
-      const int nbeg = t.n0 + half * 128;
+      const WgTile t = wg_tile<WG_BM>(p, tile, mt, nt);
+      const int mrow = t.m0 + blk * 128 + q * 32;   // first row of this warp's boxes
+      const int nbeg = t.n0 + cbeg;
       if (t.nk == 0) {
         // No row chose this segment: its gradient is zero. Store a zeroed
-        // staging box over the warp's two 32 x 64 output boxes.
+        // staging box over the warp's 32 x 64 output boxes.
         if (mrow < p.M && nbeg < p.N) {
           if (lane == 0) bulk_wait_read_all();
           __syncwarp();
@@ -236,7 +260,7 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            for (int c0 = 0; c0 < 128 && nbeg + c0 < p.N; c0 += 64) tma_store_3d(&tmD, box, nbeg + c0, mrow, t.seg);
+            for (int c0 = 0; c0 < ncol && nbeg + c0 < p.N; c0 += 64) tma_store_3d(&tmD, box, nbeg + c0, mrow, t.seg);
             bulk_commit();
           }
         }
@@ -244,8 +268,9 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
       }
       if (!wait_bounded(smem_u32(&accf_bar[acc]), acc_phase, abort_flag, p.err, p.timeout_ns, true)) break;
       tc_fence_after();
-      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * WG_BN + half * 128);
-      for (int c0 = 0; c0 < 128; c0 += 64) {
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) +
+                             (uint32_t)((WG_MB == 2 ? blk : acc) * WG_BN + cbeg);
+      for (int c0 = 0; c0 < ncol; c0 += 64) {
         if (nbeg + c0 >= p.N || mrow >= p.M) break;
         uint32_t r[64];
         tmem_ld64_wait(taddr + c0, r);
@@ -276,8 +301,7 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&acce_bar[acc]));
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
+      if (++acc == WG_ACC_STAGES) { acc = 0; acc_phase ^= 1u; }
     }
     if (lane == 0) bulk_wait_all();   // staging boxes stay live until written out
     __syncwarp();
@@ -299,18 +323,25 @@ cudaError_t launch_wgrad(const WgradParams& p, int num_sms, cudaStream_t s) {
   if (!make_tmap_strided(&tQ, p.Q, p.N, p.q_rows, p.ldQ * 2, 64)) return cudaErrorInvalidValue;
   if (!make_tmap_3d(&tD, p.out, p.N, p.M, p.n_seg, (long long)p.N * 2, (long long)p.M * p.N * 2, 32))
     return cudaErrorInvalidValue;
-  static int attr_done_mask = 0;
+  // Two M blocks per tile once segments average more than 256 rows.
+  const long long rows_per_seg = (p.offsets ? (long long)p.p_rows : (long long)p.k_total) / p.n_seg;
+  const bool two = rows_per_seg > 256;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (!(dev < 32 && ((attr_done_mask >> dev) & 1))) {
-    e = cudaFuncSetAttribute(wgrad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, WG_SMEM);
+  static int attr_done_mask[2] = {0, 0};
+  int& mask = attr_done_mask[two ? 1 : 0];
+  if (!(dev < 32 && ((mask >> dev) & 1))) {
+    e = two ? cudaFuncSetAttribute(wgrad_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, wg_smem<2>())
+            : cudaFuncSetAttribute(wgrad_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, wg_smem<1>());
     if (e != cudaSuccess) return e;
-    if (dev < 32) attr_done_mask |= 1 << dev;
+    if (dev < 32) mask |= 1 << dev;
   }
-  const long long tiles = (long long)p.n_seg * ceil_div(p.M, WG_BM) * ceil_div(p.N, WG_BN);
+  const int bm = two ? WgShape<2>::BM : WgShape<1>::BM;
+  const long long tiles = (long long)p.n_seg * ceil_div(p.M, bm) * ceil_div(p.N, WG_BN);
   const int grid = (int)(tiles < num_sms ? tiles : num_sms);
-  wgrad_kernel<<<grid, WG_THREADS, WG_SMEM, s>>>(tP, tQ, tD, p);
+  if (two) wgrad_kernel<2><<<grid, WG_THREADS, wg_smem<2>(), s>>>(tP, tQ, tD, p);
+  else wgrad_kernel<1><<<grid, WG_THREADS, wg_smem<1>(), s>>>(tP, tQ, tD, p);
   return cudaGetLastError();
 }
 

@@ -39,6 +39,8 @@ CASES = {
     "grouped_bf16": MoEConfig("grouped_bwd", T=300, d=256, E=32, k=4, f=384, gate_mode=GATE_SIGMOID,
                               n_groups=8, topk_groups=4, route_scale=2.5, f_shared=256, bias="uniform"),
     "softmax_bf16": MoEConfig("softmax_bwd", T=200, d=192, E=16, k=2, f=136),
+    # ~512 rows per expert: the weight gradients take two 128-row M blocks per tile.
+    "long_segments_bf16": MoEConfig("long_bwd", T=1024, d=256, E=4, k=2, f=200, f_shared=64),
 }
 
 
