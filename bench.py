@@ -15,6 +15,13 @@ independent replica on its own GPU (the block has no exchange step on one
 node's data-parallel path): weak scaling, value = all ranks' tokens / the
 slowest rank's time. Rank 0 prints one JSON line.
 
+Besides the timed steps, the JSON line carries: the per-stage breakdown
+(CUDA events between the stage entry points), the roofline of the dominant
+kernel, the end-to-end rate through the public call with pinned host
+buffers, the aux-loss-free balance step, the same routing with generic GELU
+experts, the fused-permute variant, and the backward (recomputing, on saved
+state, and a whole training step), each on the same inputs.
+
 ``--impl reference`` times the CPU oracle (the plain fp64 statement of the
 block) on a bounded sample of the same workload: the reference arm.
 """

@@ -122,7 +122,6 @@ moe_status enqueue_route(const moe_config& c, const void* x, const void* w_route
                          int* idx, float* gate, int* counts, int* offsets, void* ws, cudaStream_t s) {
   const Layout L = layout_of(c);
   float* logits = at<float>(ws, L.logits);
-  const int num_sms = device_sm_count();
   int n_part = 1;
   if (c.dtype == MOE_DTYPE_BF16) {
     n_part = router_gemm_splits(c.T, c.E, c.d);
@@ -139,7 +138,7 @@ moe_status enqueue_route(const moe_config& c, const void* x, const void* w_route
     g.K_s = c.d;
     MOE_CUDA(launch_simt_gemm(c.dtype, 1, g, s));
   }
-  RouteParams r;
+  RouteParams r = {};
   r.T = c.T; r.E = c.E; r.k = c.k; r.gate_mode = c.gate_mode;
   r.n_groups = c.n_groups; r.topk_groups = c.topk_groups; r.route_scale = c.route_scale;
   r.logits = logits; r.bias = bias; r.topk_idx = idx; r.topk_gate = gate;
