@@ -604,6 +604,9 @@ def main():
     else:
         roof = {"bound": "hbm", "achieved": wd["bytes"] / t_dom / 1e9, "peak": peaks["hbm"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
+    # For context, against B200's nominal figures (HBM3e 7.7 TB/s HGX, dense bf16 2.25 PFLOP/s).
+    roof["nominal_peak"] = 7700.0 if roof["bound"] == "hbm" else 2250.0
+    roof["frac_nominal"] = roof["achieved"] / roof["nominal_peak"]
     roof["traffic"] = traffic_for(cfg.name, dom)
     roof.update({"kernel": dom, "peak_source": peaks["source"], "algorithmic_bytes": wd["bytes"],
                  "algorithmic_flops": wd["flops"], "kernel_ms": stage_ms[dom]})
