@@ -1,10 +1,27 @@
 /*
- * moe.h - C ABI of the sparse Mixture-of-Experts FFN forward pass on B200.
+ * moe.h - C ABI of the sparse Mixture-of-Experts FFN block on B200.
  *
  * The block computed here (the forward pass, without the residual):
  *
  *   MoE(u_t) = sum_{s in shared} FFN_s(u_t) + sum_{i in TopK(t)} g_{i,t} FFN_i(u_t)
  *   FFN(u)   = W2 (SiLU(W1 u) * W3 u)
+ *
+ * Entry points, in the order of the path:
+ *   moe_check_config, moe_workspace_size      validation and scratch size
+ *   moe_route (moe_route_noalloc)             router logits, biased group-limited
+ *                                             top-k, gates, counts, offsets
+ *   moe_permute                               tokens into expert-contiguous rows
+ *   moe_expert_swiglu = moe_expert_gate_up + moe_expert_down
+ *                                             every expert's FFN (+ the shared one)
+ *   moe_combine                               gate-weighted sum + shared row
+ *   moe_forward                               all of the above in one call
+ * and around it:
+ *   moe_balance_update                        aux-loss-free bias step, entropy
+ *   moe_expert_gate_up_gather                 gate/up reading rows of x directly
+ *   moe_expert_gelu, moe_forward_gelu         generic experts W2 GELU(W1 u + b1) + b2
+ *   moe_backward (_workspace_size), moe_forward_train, moe_backward_saved
+ *                                             gradients of the block for training
+ *   moe_get_device_error, moe_selftest_wait_timeout, moe_status_string
  *
  * Sources, cited by page title and section:
  *   [DS] "Sparse MoE FFN" DeepSeek-V3 study note, "How it works": eq. 12
