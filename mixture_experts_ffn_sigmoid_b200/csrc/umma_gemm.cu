@@ -29,12 +29,18 @@
 // (SwiGLU: the W1 and W3 rows of the same f range; down: 256 consecutive W2
 // rows), so two MMAs share every token tile that is staged.
 //
-// Roles (192 threads, one CTA per SM, persistent over a static tile list):
+// Roles (320 threads, one CTA per SM, persistent over a static tile list):
 //   warp 0 lane 0 : TMA producer into a ring of variable-size slots
 //   warp 1        : TMEM allocator; lane 0 issues tcgen05.mma (kind::f16,
 //                   bf16 x bf16 -> fp32 in TMEM) and tcgen05.commit
-//   warps 2..5    : epilogue; tcgen05.ld of their 32-lane quarter, SiLU * up
-//                   in fp32, one rounding to the output type, masked stores
+//   warps 2..9    : epilogue, two warps per 32-lane TMEM quarter (each takes
+//                   every other 16-column chunk); tcgen05.ld, SiLU * up in
+//                   fp32, one rounding to the output type, masked stores
+//
+// TMEM (512 columns) holds a tile's two accumulators. Tiles of at most 128
+// token columns alternate between the two 256-column halves, so the MMAs of
+// the next tile do not wait for the epilogue to drain this one; wider tiles
+// take all 512 columns.
 //
 // The slot ring: a k-step needs (weights) + (its token rows, rounded to 32)
 // bytes, so slots are sized per tile and packed into one shared-memory ring
@@ -66,7 +72,8 @@ constexpr int BN_MAX = 256;      // token columns per tile (MMA N), upper bound
 constexpr int BOX_N = 32;        // token rows per TMA box
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int BOX_BYTES = BOX_N * BK * 2;
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 320;
+constexpr int EPI_WARPS = 8;      // warps 2..9: two per TMEM lane quarter
 constexpr int TMEM_COLS = 512;
 constexpr int NSLOT = 8;            // barrier pairs of the slot ring
 constexpr int SMEM_LIMIT = 232448;  // 227 KB of dynamic shared memory per block
@@ -184,18 +191,35 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar, uint16_t mask) {
 }
 
 // ------------------------------------------------------------ tile list
-// Per mode: weight blocks (128 rows each) per CTA and accumulator stages.
-// With PAIR the two CTAs of a cluster run one M=256 MMA: each holds 128 rows
-// of every weight block and half of the token tile.
+// Per mode: weight blocks (128 rows each) per CTA. With PAIR the two CTAs of
+// a cluster run one M=256 MMA: each holds 128 rows of every weight block and
+// half of the token tile.
 template <int MODE> struct Kind;
-template <> struct Kind<kUmmaSwiGLU> { static constexpr int A_TILES = 2; static constexpr int ACC_STAGES = 1; };
-template <> struct Kind<kUmmaSwiGLUSave> { static constexpr int A_TILES = 2; static constexpr int ACC_STAGES = 1; };
+template <> struct Kind<kUmmaSwiGLU> { static constexpr int A_TILES = 2; };
+template <> struct Kind<kUmmaSwiGLUSave> { static constexpr int A_TILES = 2; };
 
 // Modes whose tile pairs the W1 and W3 rows of one range (SwiGLU).
 __host__ __device__ constexpr bool dual_a(int mode) { return mode == kUmmaSwiGLU || mode == kUmmaSwiGLUSave; }
-template <> struct Kind<kUmmaDown>   { static constexpr int A_TILES = 2; static constexpr int ACC_STAGES = 1; };
-template <> struct Kind<kUmmaBiasAct> { static constexpr int A_TILES = 2; static constexpr int ACC_STAGES = 1; };
-template <> struct Kind<kUmmaDgrad> { static constexpr int A_TILES = 2; static constexpr int ACC_STAGES = 1; };
+template <> struct Kind<kUmmaDown>   { static constexpr int A_TILES = 2; };
+template <> struct Kind<kUmmaBiasAct> { static constexpr int A_TILES = 2; };
+template <> struct Kind<kUmmaDgrad> { static constexpr int A_TILES = 2; };
+
+// Where a tile's two accumulators sit in the 512 TMEM columns. A tile of at
+// most 128 token columns takes one half (first accumulator at +0, second at
+// +128), alternating halves, so the next such tile accumulates while the
+// epilogue drains this one; a wider tile takes all 512 columns (second
+// accumulator at +256) once both halves are drained. The MMA issuer and the
+// epilogue walk the same tile sequence, so they derive the same placement.
+struct AccPlace {
+  uint32_t next = 0;   // half the next narrow tile takes
+  __device__ __forceinline__ void take(int n_mma, bool& wide, uint32_t& half) {
+    wide = n_mma > BN_MAX / 2;
+    half = wide ? 0u : next;
+    next = wide ? 0u : (next ^ 1u);
+  }
+  __device__ __forceinline__ static uint32_t col0(bool wide, uint32_t half) { return wide ? 0u : half * BN_MAX; }
+  __device__ __forceinline__ static uint32_t second(bool wide) { return wide ? BN_MAX : BN_MAX / 2; }
+};
 
 // Modes whose tile is two consecutive 128-row blocks of one weight matrix.
 __host__ __device__ constexpr bool two_blocks(int mode) {
@@ -281,7 +305,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                      const __grid_constant__ CUtensorMap tmG, const UmmaGemmParams p) {
   using KD = Kind<MODE>;
   constexpr int A_TILES = KD::A_TILES;
-  constexpr int ACC_STAGES = KD::ACC_STAGES;
   constexpr int WROWS = tile_rows(MODE, PAIR);
   // Row offset of weight block a (0 or 1) inside a tile, for CTA rank r.
   constexpr int BLOCK_STEP = two_blocks(MODE) ? (PAIR ? 256 : 128) : 0;
@@ -321,7 +344,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&accf_bar[i]), 1);
-      mbar_init(smem_u32(&acce_bar[i]), (PAIR ? 2 : 1) * 4);   // one arrival per epilogue warp
+      mbar_init(smem_u32(&acce_bar[i]), (PAIR ? 2 : 1) * EPI_WARPS);   // one arrival per epilogue warp
     }
     mbar_init(smem_u32(drain_bar), 1);
     *abort_flag = 0u;
@@ -501,21 +524,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1 && lane == 0 && leader) {
     // ------------------------------------------------------------ MMA issuer
     RingCursor cur;
-    int acc = 0;
-    uint32_t acc_phase = 0;
+    AccPlace place;
+    uint32_t uses0 = 0, uses1 = 0;   // tiles placed in each TMEM half so far
     bool issued = false;
     for (int tile = group; tile < total_tiles; tile += ngroups) {
       const Tile t = decode_tile(p, s_off, s_start, nseg, tile, WROWS);
       const TokenSlice ts = token_slice<PAIR>(p, t, 0);
       const uint32_t bytes = A_TILES * A_BYTES + ts.bytes();
       const int nk = ceil_div(t.K, BK);
-      if (!wait_bounded(smem_u32(&acce_bar[acc]), acc_phase ^ 1u, abort_flag, p.err, p.timeout_ns, true))
-        break;
+      bool wide;
+      uint32_t half;
+      place.take(ts.n_mma, wide, half);
+      // The half (both for a wide tile) must have been drained by the epilogue.
+      bool ok = true;
+      if (wide || half == 0u) {
+        ok = wait_bounded(smem_u32(&acce_bar[0]), (uses0 & 1u) ^ 1u, abort_flag, p.err, p.timeout_ns, true);
+        ++uses0;
+      }
+      if (ok && (wide || half == 1u)) {
+        ok = wait_bounded(smem_u32(&acce_bar[1]), (uses1 & 1u) ^ 1u, abort_flag, p.err, p.timeout_ns, true);
+        ++uses1;
+      }
+      if (!ok) break;
       tc_fence_after();
       const uint32_t idesc = idesc_bf16_f32(PAIR ? 2 * BM : BM, ts.n_mma) | (MODE == kUmmaDgrad ? (1u << 15) : 0u);
-      const uint32_t d1 = tmem_base + (uint32_t)(acc * BN_MAX);
-      const uint32_t d3 = tmem_base + (uint32_t)BN_MAX;
-      bool ok = true;
+      const uint32_t d1 = tmem_base + AccPlace::col0(wide, half);
+      const uint32_t d3 = d1 + AccPlace::second(wide);
       for (int kb = 0; kb < nk; ++kb) {
         uint32_t off, slot, parity;
         cur.take(bytes, cap, off, slot, parity);
@@ -549,14 +583,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         else umma_commit(smem_u32(&empty_bar[slot]));
       }
       if (!ok) break;
-      if (PAIR) umma_commit_pair(smem_u32(&accf_bar[acc]), 0x3);
-      else umma_commit(smem_u32(&accf_bar[acc]));
-      if (ACC_STAGES == 2) {
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
-      } else {
-        acc_phase ^= 1u;
-      }
+      if (PAIR) umma_commit_pair(smem_u32(&accf_bar[half]), 0x3);
+      else umma_commit(smem_u32(&accf_bar[half]));
     }
     if (issued) {   // every MMA this thread issued completes before TMEM is freed
       if (PAIR) umma_commit_pair(smem_u32(drain_bar), 0x1);
@@ -566,25 +594,43 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                  // TMEM lane quarter this warp may read
+    const int ch = (warp - 2) >> 2;          // which 16-column chunks: ch, ch + 2, ch + 4, ...
     const int row = q * 32 + lane;
     // The accumulator is released to the leader's barrier (remote for the peer).
     const uint32_t acce0 = PAIR ? map_to_cta(smem_u32(&acce_bar[0]), 0) : smem_u32(&acce_bar[0]);
-    int acc = 0;
-    uint32_t acc_phase = 0;
+    AccPlace place;
+    uint32_t fills0 = 0, fills1 = 0;   // accumulators consumed from each half so far
     for (int tile = group; tile < total_tiles; tile += ngroups) {
       const Tile t = decode_tile(p, s_off, s_start, nseg, tile, WROWS);
       const TokenSlice ts = token_slice<PAIR>(p, t, 0);
       const int n_valid = ts.n_valid, n_mma = ts.n_mma;
-      if (!wait_bounded(smem_u32(&accf_bar[acc]), acc_phase, abort_flag, p.err, p.timeout_ns, true))
+      bool wide;
+      uint32_t half;
+      place.take(n_mma, wide, half);
+      const uint32_t fill_parity = (half ? fills1 : fills0) & 1u;
+      if (!wait_bounded(smem_u32(&accf_bar[half]), fill_parity, abort_flag, p.err, p.timeout_ns, true))
         break;
+      if (half) ++fills1; else ++fills0;
       tc_fence_after();
       const int m = t.wt * WROWS + (int)rank * BM + row;
       const bool m_ok = m < t.mrows;
       const long long ld = t.dense ? p.out_s_ld : p.out_ld;
       void* out = t.dense ? p.out_s : p.out;
       const long long r0 = (long long)t.b_row0 + (long long)t.tt * p.bn_max;
-      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MAX);
-      const uint32_t acce = acce0 + (uint32_t)(acc * 8);
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + AccPlace::col0(wide, half);
+      const uint32_t off2 = AccPlace::second(wide);   // second accumulator's column offset
+      // Hand the tile's TMEM back: its half, or both halves for a wide tile.
+      auto release = [&]() {
+        if (lane == 0) {
+          if (PAIR) {
+            mbar_arrive_cluster(acce0 + half * 8u);
+            if (wide) mbar_arrive_cluster(acce0 + 8u);
+          } else {
+            mbar_arrive(acce0 + half * 8u);
+            if (wide) mbar_arrive(acce0 + 8u);
+          }
+        }
+      };
       if (dual_a(MODE)) {
         // Drain both accumulators into registers as packed bf16 h, hand TMEM
         // back to the MMA warp, then store while the next tile accumulates.
@@ -594,12 +640,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           pre_a = static_cast<__nv_bfloat16*>(t.dense ? p.pre_a_s : p.pre_a) + r0 * ld;
           pre_b = static_cast<__nv_bfloat16*>(t.dense ? p.pre_b_s : p.pre_b) + r0 * ld;
         }
-        uint32_t hp[BN_MAX / 2];
+        uint32_t hp[BN_MAX / 4];
 #pragma unroll
-        for (int c = 0; c < BN_MAX / 16; ++c) {
+        for (int cc = 0; cc < BN_MAX / 32; ++cc) {
+          const int c = 2 * cc + ch;
           if (c * 16 < n_mma) {
             uint32_t r1[16], r3[16];
-            tmem_ld16x2_wait(taddr + c * 16, taddr + BN_MAX + c * 16, r1, r3);
+            tmem_ld16x2_wait(taddr + c * 16, taddr + off2 + c * 16, r1, r3);
             if (MODE == kUmmaSwiGLUSave && m_ok) {
               // Training forward: keep W1 u and W3 u (bf16) for the backward.
 #pragma unroll
@@ -614,26 +661,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
               const float g0 = __uint_as_float(r1[2 * j]), g1 = __uint_as_float(r1[2 * j + 1]);
-              const float h0 = (g0 / (1.0f + __expf(-g0))) * __uint_as_float(r3[2 * j]);
-              const float h1 = (g1 / (1.0f + __expf(-g1))) * __uint_as_float(r3[2 * j + 1]);
+              // SiLU(g) = g / (1 + e^-g); the fast divide returns 0 once the
+              // denominator passes 2^126, where the exact quotient is below 1e-36.
+              const float h0 = __fdividef(g0, 1.0f + __expf(-g0)) * __uint_as_float(r3[2 * j]);
+              const float h1 = __fdividef(g1, 1.0f + __expf(-g1)) * __uint_as_float(r3[2 * j + 1]);
               const __nv_bfloat162 hb = __floats2bfloat162_rn(h0, h1);
-              hp[c * 8 + j] = *reinterpret_cast<const uint32_t*>(&hb);
+              hp[cc * 8 + j] = *reinterpret_cast<const uint32_t*>(&hb);
             }
           }
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) { if (PAIR) mbar_arrive_cluster(acce); else mbar_arrive(acce); }
+        release();
         if (m_ok) {
           unsigned short* o = reinterpret_cast<unsigned short*>(out) + r0 * ld + m;
 #pragma unroll
-          for (int c = 0; c < BN_MAX / 16; ++c) {
+          for (int cc = 0; cc < BN_MAX / 32; ++cc) {
+            const int c = 2 * cc + ch;
             if (c * 16 < n_valid) {
 #pragma unroll
               for (int j = 0; j < 16; ++j) {
                 const int col = c * 16 + j;
                 if (col < n_valid)
-                  o[(long long)col * ld] = (unsigned short)(hp[c * 8 + (j >> 1)] >> ((j & 1) * 16));
+                  o[(long long)col * ld] = (unsigned short)(hp[cc * 8 + (j >> 1)] >> ((j & 1) * 16));
               }
             }
           }
@@ -643,9 +693,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int m2 = m + BLOCK_STEP;
         const bool m2_ok = m2 < t.mrows;
         float* o = reinterpret_cast<float*>(out) + r0 * ld;
-        for (int c0 = 0; c0 < n_mma; c0 += 16) {
+        for (int c0 = ch * 16; c0 < n_mma; c0 += 32) {
           uint32_t r1[16], r3[16];
-          tmem_ld16x2_wait(taddr + c0, taddr + BN_MAX + c0, r1, r3);
+          tmem_ld16x2_wait(taddr + c0, taddr + off2 + c0, r1, r3);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int col = c0 + j;
@@ -657,15 +707,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) { if (PAIR) mbar_arrive_cluster(acce); else mbar_arrive(acce); }
+        release();
       } else if (MODE == kUmmaDown || MODE == kUmmaDgrad) {
         // Two 128-row blocks of the tile's weight rows, BLOCK_STEP apart.
         const int m2 = m + BLOCK_STEP;
         const bool m2_ok = m2 < t.mrows;
         __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out) + r0 * ld;
-        for (int c0 = 0; c0 < n_mma; c0 += 16) {
+        for (int c0 = ch * 16; c0 < n_mma; c0 += 32) {
           uint32_t r1[16], r3[16];
-          tmem_ld16x2_wait(taddr + c0, taddr + BN_MAX + c0, r1, r3);
+          tmem_ld16x2_wait(taddr + c0, taddr + off2 + c0, r1, r3);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int col = c0 + j;
@@ -677,7 +727,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) { if (PAIR) mbar_arrive_cluster(acce); else mbar_arrive(acce); }
+        release();
       } else if (MODE == kUmmaBiasAct) {
         // As kUmmaDown, with the weight row's bias added and the activation
         // applied in fp32 before the one rounding to bf16.
@@ -689,9 +739,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const float bias2 = (rb && m2_ok) ? rb[boff + m2] : 0.0f;
         const bool gelu = p.act == kActGelu;
         __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out) + r0 * ld;
-        for (int c0 = 0; c0 < n_mma; c0 += 16) {
+        for (int c0 = ch * 16; c0 < n_mma; c0 += 32) {
           uint32_t r1[16], r3[16];
-          tmem_ld16x2_wait(taddr + c0, taddr + BN_MAX + c0, r1, r3);
+          tmem_ld16x2_wait(taddr + c0, taddr + off2 + c0, r1, r3);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int col = c0 + j;
@@ -706,13 +756,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) { if (PAIR) mbar_arrive_cluster(acce); else mbar_arrive(acce); }
-      }
-      if (ACC_STAGES == 2) {
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
-      } else {
-        acc_phase ^= 1u;
+        release();
       }
     }
   }
