@@ -86,21 +86,77 @@ def measured_peaks():
 
 # --------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while work runs."""
+    """SM clock, power and clock-event reasons sampled while work runs: from NVML
+    every 20 ms when the library answers for this GPU, else from an `nvidia-smi`
+    query loop every 100 ms. Both only read the GPU's state."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NVML_PERIOD_S = 0.02
 
     def __init__(self, device_index: int):
         self.samples = []
         self.proc = None
         self.dev = device_index
+        self.source = None
+        self._nvml = None
+        self._stop_evt = None
+        self.thread = None
+
+    def _uuid(self):
+        uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+        return uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+
+    def _nvml_row(self):
+        """One sample in the column order of FIELDS (reasons as Active / Not Active)."""
+        n, h = self._nvml, self._handle
+        sm = n.nvmlDeviceGetClockInfo(h, n.NVML_CLOCK_SM)
+        mx = n.nvmlDeviceGetMaxClockInfo(h, n.NVML_CLOCK_SM)
+        watts = n.nvmlDeviceGetPowerUsage(h) / 1000.0
+        mask = n.nvmlDeviceGetCurrentClocksEventReasons(h)
+        bits = (n.nvmlClocksEventReasonHwSlowdown, n.nvmlClocksEventReasonHwThermalSlowdown,
+                n.nvmlClocksEventReasonSwThermalSlowdown, n.nvmlClocksEventReasonSwPowerCap)
+        return [str(sm), str(mx), f"{watts:.2f}", hex(mask)] + \
+            ["Active" if mask & b else "Not Active" for b in bits]
+
+    def _start_nvml(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._handle = pynvml.nvmlDeviceGetHandleByUUID(self._uuid())
+            self.samples.append((time.time(), self._nvml_row()))   # the first read must work
+        except Exception:
+            self._shutdown_nvml()
+            self.samples = []
+            return False
+        self._stop_evt = threading.Event()
+        self.thread = threading.Thread(target=self._poll_nvml, daemon=True)
+        self.thread.start()
+        self.source = "nvml"
+        return True
+
+    def _poll_nvml(self):
+        while not self._stop_evt.wait(self.NVML_PERIOD_S):
+            try:
+                self.samples.append((time.time(), self._nvml_row()))
+            except Exception:
+                return
+
+    def _shutdown_nvml(self):
+        if self._nvml is not None:
+            try:
+                self._nvml.nvmlShutdown()
+            except Exception:
+                pass
+            self._nvml = None
 
     def start(self):
+        if self._start_nvml():
+            return
         try:
-            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
-            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            sel = self._uuid()
         except Exception:
             sel = str(self.dev)
         try:
@@ -110,6 +166,7 @@ class ClockSampler:
         except Exception:
             self.proc = None
             return
+        self.source = "nvidia-smi"
         self.thread = threading.Thread(target=self._read, daemon=True)
         self.thread.start()
 
@@ -118,6 +175,11 @@ class ClockSampler:
             self.samples.append((time.time(), [v.strip() for v in line.split(",")]))
 
     def stop(self):
+        if self._stop_evt is not None:
+            self._stop_evt.set()
+            if self.thread is not None:
+                self.thread.join(timeout=2)
+            self._shutdown_nvml()
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -144,7 +206,7 @@ class ClockSampler:
         reasons = sorted({names[i] for r in rows for i in range(4) if len(r) > 4 + i and r[4 + i] == "Active"})
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": num(rows[0][1]), "reasons": reasons, "samples": len(rows), "window": window,
-                "power_w_max": max((num(r[2]) or 0.0) for r in rows)}
+                "source": self.source, "power_w_max": max((num(r[2]) or 0.0) for r in rows)}
 
 
 # ------------------------------------------------------- multi-rank timing
