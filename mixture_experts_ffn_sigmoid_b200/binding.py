@@ -1,9 +1,11 @@
 """ctypes binding of ``libmoe_b200.so`` (declared in ``include/moe.h``).
 
-Argument marshalling only: every function here checks shapes and dtypes of
-torch tensors, passes their device pointers and the current CUDA stream to
-the C entry point of the same name, and raises ``MoEError`` on a non-OK
-status. All compute runs in the library's CUDA kernels; there is no other
+Argument marshalling only: every function here checks that each torch
+tensor has the dtype the entry point expects and at least as many elements as
+the library will read or write through it (a short buffer would be an
+out-of-bounds access on the GPU), that it is a contiguous CUDA tensor, passes
+the device pointers and the current CUDA stream to the C entry point of the
+same name, and raises ``MoEError`` on a non-OK status. All compute runs in the library's CUDA kernels; there is no other
 path. If the library is missing or cannot be loaded, every call raises.
 """
 from __future__ import annotations
@@ -118,6 +120,78 @@ def _cfg(c) -> CConfig:
     return c if isinstance(c, CConfig) else make_config(c)
 
 
+_I32, _F32, _U8 = torch.int32, torch.float32, torch.uint8
+
+
+def _dt(c: CConfig) -> torch.dtype:
+    return torch.float32 if c.dtype == MOE_DTYPE_F32 else torch.bfloat16
+
+
+def _need(t, name: str, numel: int, dtype: torch.dtype, required: bool = True):
+    """Refuse a tensor the library would overrun or misread: wrong dtype, or
+    fewer than ``numel`` elements. None passes where the C entry point takes
+    NULL (``required=False``) and where it reads or writes nothing through the
+    pointer (``numel == 0``, e.g. token arrays when T = 0)."""
+    if t is None:
+        if required and numel > 0:
+            raise ValueError(f"{name} is required")
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor, not {type(t).__name__}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if t.numel() < numel:
+        raise ValueError(f"{name}: {t.numel()} elements, needs at least {numel}")
+
+
+def _need_routing_io(c: CConfig, x, w_router, bias, topk_idx, topk_gate, expert_counts, expert_offsets):
+    T, d, E, k, dt = c.T, c.d, c.E, c.k, _dt(c)
+    _need(x, "x", T * d, dt)
+    _need(w_router, "w_router", E * d, dt)
+    _need(bias, "bias", E, _F32, required=False)
+    _need(topk_idx, "topk_idx", T * k, _I32)
+    _need(topk_gate, "topk_gate", T * k, _F32)
+    _need(expert_counts, "expert_counts", E, _I32)
+    _need(expert_offsets, "expert_offsets", E + 1, _I32)
+
+
+def _need_weights(c: CConfig, w1, w3, w2, ws1, ws3, ws2, prefix: str = ""):
+    d, E, f, fs, dt = c.d, c.E, c.f, c.f_shared, _dt(c)
+    sh = fs > 0
+    _need(w1, prefix + "w1", E * f * d, dt)
+    _need(w3, prefix + "w3", E * f * d, dt)
+    _need(w2, prefix + "w2", E * d * f, dt)
+    _need(ws1, prefix + "ws1", fs * d, dt, required=sh)
+    _need(ws3, prefix + "ws3", fs * d, dt, required=sh)
+    _need(ws2, prefix + "ws2", d * fs, dt, required=sh)
+
+
+def _need_ws(workspace):
+    if workspace is None:
+        raise ValueError("workspace is required")
+    _need(workspace, "workspace", 0, _U8)
+
+
+def _need_block(c: CConfig, x, w_router, bias, w1, w3, w2, ws1, ws3, ws2, y, workspace):
+    """Inputs of the whole block (y checked unless None is passed for it)."""
+    dt = _dt(c)
+    _need(x, "x", c.T * c.d, dt)
+    _need(w_router, "w_router", c.E * c.d, dt)
+    _need(bias, "bias", c.E, _F32, required=False)
+    _need_weights(c, w1, w3, w2, ws1, ws3, ws2)
+    if y is not None:
+        _need(y, "y", c.T * c.d, dt)
+    _need_ws(workspace)
+
+
+def _need_grads(c: CConfig, dy, dx, dw_router, dw1, dw3, dw2, dws1, dws3, dws2):
+    dt = _dt(c)
+    _need(dy, "dy", c.T * c.d, dt)
+    _need(dx, "dx", c.T * c.d, dt)
+    _need(dw_router, "dw_router", c.E * c.d, dt)
+    _need_weights(c, dw1, dw3, dw2, dws1, dws3, dws2, prefix="d")
+
+
 def _ptr(t: Optional[torch.Tensor]):
     if t is None:
         return None
@@ -157,6 +231,8 @@ def alloc_workspace(cfg, device="cuda") -> torch.Tensor:
 def moe_route(cfg, x, w_router, bias, topk_idx, topk_gate, expert_counts, expert_offsets,
               workspace, stream=None):
     c = _cfg(cfg)
+    _need_routing_io(c, x, w_router, bias, topk_idx, topk_gate, expert_counts, expert_offsets)
+    _need_ws(workspace)
     _check(lib().moe_route(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(topk_idx),
                            _ptr(topk_gate), _ptr(expert_counts), _ptr(expert_offsets),
                            _ptr(workspace), workspace.numel(), _stream(stream)), "moe_route")
@@ -164,6 +240,14 @@ def moe_route(cfg, x, w_router, bias, topk_idx, topk_gate, expert_counts, expert
 
 def moe_permute(cfg, x, topk_idx, expert_offsets, x_perm, perm_src, inv_row, workspace, stream=None):
     c = _cfg(cfg)
+    R, dt = c.T * c.k, _dt(c)
+    _need(x, "x", c.T * c.d, dt, required=x_perm is not None)
+    _need(topk_idx, "topk_idx", R, _I32)
+    _need(expert_offsets, "expert_offsets", c.E + 1, _I32)
+    _need(x_perm, "x_perm", R * c.d, dt, required=False)
+    _need(perm_src, "perm_src", R, _I32)
+    _need(inv_row, "inv_row", R, _I32)
+    _need_ws(workspace)
     _check(lib().moe_permute(ctypes.byref(c), _ptr(x), _ptr(topk_idx), _ptr(expert_offsets),
                              _ptr(x_perm), _ptr(perm_src), _ptr(inv_row), _ptr(workspace),
                              workspace.numel(), _stream(stream)), "moe_permute")
@@ -172,6 +256,14 @@ def moe_permute(cfg, x, topk_idx, expert_offsets, x_perm, perm_src, inv_row, wor
 def moe_expert_swiglu(cfg, x_perm, expert_offsets, w1, w3, w2, x_shared, ws1, ws3, ws2, y_perm,
                       y_shared, workspace, stream=None):
     c = _cfg(cfg)
+    R, dt, sh = c.T * c.k, _dt(c), c.f_shared > 0
+    _need(x_perm, "x_perm", R * c.d, dt)
+    _need(expert_offsets, "expert_offsets", c.E + 1, _I32)
+    _need_weights(c, w1, w3, w2, ws1, ws3, ws2)
+    _need(x_shared, "x_shared", c.T * c.d, dt, required=sh)
+    _need(y_perm, "y_perm", R * c.d, dt)
+    _need(y_shared, "y_shared", c.T * c.d, dt, required=sh)
+    _need_ws(workspace)
     _check(lib().moe_expert_swiglu(ctypes.byref(c), _ptr(x_perm), _ptr(expert_offsets), _ptr(w1),
                                    _ptr(w3), _ptr(w2), _ptr(x_shared), _ptr(ws1), _ptr(ws3),
                                    _ptr(ws2), _ptr(y_perm), _ptr(y_shared), _ptr(workspace),
@@ -181,6 +273,17 @@ def moe_expert_swiglu(cfg, x_perm, expert_offsets, w1, w3, w2, x_shared, ws1, ws
 def moe_expert_gate_up(cfg, x_perm, expert_offsets, w1, w3, x_shared, ws1, ws3, h, h_shared,
                        workspace, stream=None):
     c = _cfg(cfg)
+    R, dt, sh, fs = c.T * c.k, _dt(c), c.f_shared > 0, c.f_shared
+    _need(x_perm, "x_perm", R * c.d, dt)
+    _need(expert_offsets, "expert_offsets", c.E + 1, _I32)
+    _need(w1, "w1", c.E * c.f * c.d, dt)
+    _need(w3, "w3", c.E * c.f * c.d, dt)
+    _need(x_shared, "x_shared", c.T * c.d, dt, required=sh)
+    _need(ws1, "ws1", fs * c.d, dt, required=sh)
+    _need(ws3, "ws3", fs * c.d, dt, required=sh)
+    _need(h, "h", R * c.f, dt)
+    _need(h_shared, "h_shared", c.T * fs, dt, required=sh)
+    _need_ws(workspace)
     _check(lib().moe_expert_gate_up(ctypes.byref(c), _ptr(x_perm), _ptr(expert_offsets), _ptr(w1),
                                     _ptr(w3), _ptr(x_shared), _ptr(ws1), _ptr(ws3), _ptr(h),
                                     _ptr(h_shared), _ptr(workspace), workspace.numel(),
@@ -190,6 +293,17 @@ def moe_expert_gate_up(cfg, x_perm, expert_offsets, w1, w3, x_shared, ws1, ws3, 
 def moe_expert_gate_up_gather(cfg, x, perm_src, expert_offsets, w1, w3, ws1, ws3, h, h_shared,
                               workspace, stream=None):
     c = _cfg(cfg)
+    R, dt, sh, fs = c.T * c.k, _dt(c), c.f_shared > 0, c.f_shared
+    _need(x, "x", c.T * c.d, dt)
+    _need(perm_src, "perm_src", R, _I32)
+    _need(expert_offsets, "expert_offsets", c.E + 1, _I32)
+    _need(w1, "w1", c.E * c.f * c.d, dt)
+    _need(w3, "w3", c.E * c.f * c.d, dt)
+    _need(ws1, "ws1", fs * c.d, dt, required=sh)
+    _need(ws3, "ws3", fs * c.d, dt, required=sh)
+    _need(h, "h", R * c.f, dt)
+    _need(h_shared, "h_shared", c.T * fs, dt, required=sh)
+    _need_ws(workspace)
     _check(lib().moe_expert_gate_up_gather(ctypes.byref(c), _ptr(x), _ptr(perm_src), _ptr(expert_offsets),
                                            _ptr(w1), _ptr(w3), _ptr(ws1), _ptr(ws3), _ptr(h),
                                            _ptr(h_shared), _ptr(workspace), workspace.numel(),
@@ -199,6 +313,15 @@ def moe_expert_gate_up_gather(cfg, x, perm_src, expert_offsets, w1, w3, ws1, ws3
 def moe_expert_down(cfg, h, expert_offsets, w2, h_shared, ws2, y_perm, y_shared, workspace,
                     stream=None):
     c = _cfg(cfg)
+    R, dt, sh, fs = c.T * c.k, _dt(c), c.f_shared > 0, c.f_shared
+    _need(h, "h", R * c.f, dt)
+    _need(expert_offsets, "expert_offsets", c.E + 1, _I32)
+    _need(w2, "w2", c.E * c.d * c.f, dt)
+    _need(h_shared, "h_shared", c.T * fs, dt, required=sh)
+    _need(ws2, "ws2", c.d * fs, dt, required=sh)
+    _need(y_perm, "y_perm", R * c.d, dt)
+    _need(y_shared, "y_shared", c.T * c.d, dt, required=sh)
+    _need_ws(workspace)
     _check(lib().moe_expert_down(ctypes.byref(c), _ptr(h), _ptr(expert_offsets), _ptr(w2),
                                  _ptr(h_shared), _ptr(ws2), _ptr(y_perm), _ptr(y_shared),
                                  _ptr(workspace), workspace.numel(), _stream(stream)),
@@ -207,12 +330,19 @@ def moe_expert_down(cfg, h, expert_offsets, w2, h_shared, ws2, y_perm, y_shared,
 
 def moe_combine(cfg, y_perm, inv_row, topk_gate, y_shared, y, stream=None):
     c = _cfg(cfg)
+    R, dt = c.T * c.k, _dt(c)
+    _need(y_perm, "y_perm", R * c.d, dt)
+    _need(inv_row, "inv_row", R, _I32)
+    _need(topk_gate, "topk_gate", R, _F32)
+    _need(y_shared, "y_shared", c.T * c.d, dt, required=False)
+    _need(y, "y", c.T * c.d, dt)
     _check(lib().moe_combine(ctypes.byref(c), _ptr(y_perm), _ptr(inv_row), _ptr(topk_gate),
                              _ptr(y_shared), _ptr(y), _stream(stream)), "moe_combine")
 
 
 def moe_forward(cfg, x, w_router, bias, w1, w3, w2, ws1, ws3, ws2, y, workspace, stream=None):
     c = _cfg(cfg)
+    _need_block(c, x, w_router, bias, w1, w3, w2, ws1, ws3, ws2, y, workspace)
     _check(lib().moe_forward(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w1),
                              _ptr(w3), _ptr(w2), _ptr(ws1), _ptr(ws3), _ptr(ws2), _ptr(y),
                              _ptr(workspace), workspace.numel(), _stream(stream)), "moe_forward")
@@ -221,6 +351,15 @@ def moe_forward(cfg, x, w_router, bias, w1, w3, w2, ws1, ws3, ws2, y, workspace,
 def moe_expert_gelu(cfg, x_perm, expert_offsets, w1, b1, w2, b2, y_perm, workspace, stream=None):
     """Generic experts on packed rows: y = W2 GELU(W1 x + b1) + b2 per segment."""
     c = _cfg(cfg)
+    R, dt = c.T * c.k, _dt(c)
+    _need(x_perm, "x_perm", R * c.d, dt)
+    _need(expert_offsets, "expert_offsets", c.E + 1, _I32)
+    _need(w1, "w1", c.E * c.f * c.d, dt)
+    _need(b1, "b1", c.E * c.f, _F32, required=False)
+    _need(w2, "w2", c.E * c.d * c.f, dt)
+    _need(b2, "b2", c.E * c.d, _F32, required=False)
+    _need(y_perm, "y_perm", R * c.d, dt)
+    _need_ws(workspace)
     _check(lib().moe_expert_gelu(ctypes.byref(c), _ptr(x_perm), _ptr(expert_offsets), _ptr(w1), _ptr(b1),
                                  _ptr(w2), _ptr(b2), _ptr(y_perm), _ptr(workspace), workspace.numel(),
                                  _stream(stream)), "moe_expert_gelu")
@@ -229,6 +368,16 @@ def moe_expert_gelu(cfg, x_perm, expert_offsets, w1, b1, w2, b2, y_perm, workspa
 def moe_forward_gelu(cfg, x, w_router, bias, w1, b1, w2, b2, y, workspace, stream=None):
     """The block with generic GELU experts (no shared expert)."""
     c = _cfg(cfg)
+    dt = _dt(c)
+    _need(x, "x", c.T * c.d, dt)
+    _need(w_router, "w_router", c.E * c.d, dt)
+    _need(bias, "bias", c.E, _F32, required=False)
+    _need(w1, "w1", c.E * c.f * c.d, dt)
+    _need(b1, "b1", c.E * c.f, _F32, required=False)
+    _need(w2, "w2", c.E * c.d * c.f, dt)
+    _need(b2, "b2", c.E * c.d, _F32, required=False)
+    _need(y, "y", c.T * c.d, dt)
+    _need_ws(workspace)
     _check(lib().moe_forward_gelu(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w1),
                                   _ptr(b1), _ptr(w2), _ptr(b2), _ptr(y), _ptr(workspace),
                                   workspace.numel(), _stream(stream)), "moe_forward_gelu")
@@ -250,6 +399,8 @@ def moe_backward(cfg, x, w_router, bias, w1, w3, w2, ws1, ws3, ws2, dy, dx, dw_r
                  dws1, dws3, dws2, workspace, stream=None):
     """Gradients of the block with respect to x and every weight, given dy."""
     c = _cfg(cfg)
+    _need_block(c, x, w_router, bias, w1, w3, w2, ws1, ws3, ws2, None, workspace)
+    _need_grads(c, dy, dx, dw_router, dw1, dw3, dw2, dws1, dws3, dws2)
     _check(lib().moe_backward(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w1), _ptr(w3),
                               _ptr(w2), _ptr(ws1), _ptr(ws3), _ptr(ws2), _ptr(dy), _ptr(dx), _ptr(dw_router),
                               _ptr(dw1), _ptr(dw3), _ptr(dw2), _ptr(dws1), _ptr(dws3), _ptr(dws2),
@@ -259,6 +410,7 @@ def moe_backward(cfg, x, w_router, bias, w1, w3, w2, ws1, ws3, ws2, dy, dx, dw_r
 def moe_forward_train(cfg, x, w_router, bias, w1, w3, w2, ws1, ws3, ws2, y, workspace, stream=None):
     """moe_forward that keeps routing and pre-activations in a backward-size workspace."""
     c = _cfg(cfg)
+    _need_block(c, x, w_router, bias, w1, w3, w2, ws1, ws3, ws2, y, workspace)
     _check(lib().moe_forward_train(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w1), _ptr(w3),
                                    _ptr(w2), _ptr(ws1), _ptr(ws3), _ptr(ws2), _ptr(y), _ptr(workspace),
                                    workspace.numel(), _stream(stream)), "moe_forward_train")
@@ -268,6 +420,8 @@ def moe_backward_saved(cfg, x, w_router, w1, w3, w2, ws1, ws3, ws2, dy, dx, dw_r
                        dws1, dws3, dws2, workspace, stream=None):
     """moe_backward on the state moe_forward_train left in `workspace`."""
     c = _cfg(cfg)
+    _need_block(c, x, w_router, None, w1, w3, w2, ws1, ws3, ws2, None, workspace)
+    _need_grads(c, dy, dx, dw_router, dw1, dw3, dw2, dws1, dws3, dws2)
     _check(lib().moe_backward_saved(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(w1), _ptr(w3), _ptr(w2),
                                     _ptr(ws1), _ptr(ws3), _ptr(ws2), _ptr(dy), _ptr(dx), _ptr(dw_router),
                                     _ptr(dw1), _ptr(dw3), _ptr(dw2), _ptr(dws1), _ptr(dws3), _ptr(dws2),
@@ -278,6 +432,7 @@ def moe_route_noalloc(cfg, x, w_router, bias, topk_idx, topk_gate, expert_counts
                       stream=None):
     """moe_route with the router's scratch in the library's fixed device array."""
     c = _cfg(cfg)
+    _need_routing_io(c, x, w_router, bias, topk_idx, topk_gate, expert_counts, expert_offsets)
     _check(lib().moe_route_noalloc(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(bias),
                                    _ptr(topk_idx), _ptr(topk_gate), _ptr(expert_counts),
                                    _ptr(expert_offsets), _stream(stream)), "moe_route_noalloc")
@@ -286,15 +441,20 @@ def moe_route_noalloc(cfg, x, w_router, bias, topk_idx, topk_gate, expert_counts
 def moe_balance_update(cfg, expert_counts, bias, gamma: float, entropy=None, stream=None):
     """Aux-loss-free bias step in place on `bias` and/or the routing entropy."""
     c = _cfg(cfg)
+    _need(expert_counts, "expert_counts", c.E, _I32)
+    _need(bias, "bias", c.E, _F32, required=False)
+    _need(entropy, "entropy", 1, _F32, required=False)
     _check(lib().moe_balance_update(ctypes.byref(c), _ptr(expert_counts), _ptr(bias), float(gamma),
                                     _ptr(entropy), _stream(stream)), "moe_balance_update")
 
 
 def moe_get_device_error(workspace, stream=None) -> int:
+    _need_ws(workspace)
     return lib().moe_get_device_error(_ptr(workspace), _stream(stream))
 
 
 def moe_selftest_wait_timeout(workspace, timeout_ns: int, stream=None):
+    _need_ws(workspace)
     _check(lib().moe_selftest_wait_timeout(_ptr(workspace), workspace.numel(), int(timeout_ns),
                                            _stream(stream)), "moe_selftest_wait_timeout")
 

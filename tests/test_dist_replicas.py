@@ -38,7 +38,10 @@ def _worker(rank, world, port, out):
 def test_two_rank_replica_timing():
     world = 2
     port = _free_port()
-    with mp.Manager() as mgr:
+    # The result dict's server process is started with spawn too: the test
+    # process may already run threads (torch's pools), and a forked child
+    # would inherit any lock one of them held.
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)
