@@ -272,6 +272,24 @@ def pin_brute_force_group_limited():
         assert got[0].tolist() == _brute_group_route(vals.tolist(), n_groups, tg, k), (vals, n_groups, tg, k)
 
 
+def pin_group_score_uses_biased_scores():
+    # The Sparse MoE FFN note's "Routing": the group score is the sum of the two
+    # largest *biased* scores. Scores s = (0.4, 0.4 | 0.6, 0.5) in two groups of
+    # two: unbiased, group 1 leads (1.1 > 0.8) and keeps expert 2; a +0.3 bias on
+    # group 0 lifts its pair to 0.7 + 0.7 = 1.4 > 1.1, so the choice moves into
+    # group 0 (the 0.7 / 0.7 tie goes to the lower id), and the gate is still
+    # the unbiased score renormalised over the one selected expert, 1.
+    s = np.array([[0.4, 0.4, 0.6, 0.5]])
+    logits = np.log(s / (1.0 - s))                       # sigmoid(logits) = s
+    eye = np.eye(4)
+    r0 = orc.route(logits, eye, np.zeros(4), 1, orc.GATE_SIGMOID, 2, 1, 1.0)
+    assert r0["idx"].tolist() == [[2]]
+    r = orc.route(logits, eye, np.array([0.3, 0.3, 0.0, 0.0]), 1, orc.GATE_SIGMOID, 2, 1, 1.0)
+    assert r["idx"].tolist() == [[0]]
+    assert np.allclose(r["gates"], [[1.0]], rtol=0, atol=1e-15)
+    assert r["eligible"][0].tolist() == [True, True, False, False]
+
+
 # --------------------------------------------------- library special cases
 def _torch_swiglu(u, w1, w3, w2):
     u, w1, w3, w2 = (torch.as_tensor(a, dtype=torch.float64) for a in (u, w1, w3, w2))

@@ -206,6 +206,40 @@ def _gate_bwd_no_centering(logits, scores, idx, gates, dgates, gate_mode, route_
     return dl
 
 
+def _route_groups_from_unbiased(x, w_router, bias, k, gate_mode, n_groups=1, topk_groups=1,
+                                route_scale=1.0):
+    # Group scores from the unbiased affinities (the bias then moves only the
+    # choice inside the kept groups).
+    logits = _orig["router_logits"](x, w_router)
+    scores = _orig["affinity"](logits, gate_mode)
+    biased = _orig["biased_scores"](scores, bias)
+    eligible = _orig["group_eligibility"](scores, n_groups, topk_groups)
+    idx = _orig["select_experts"](biased, eligible, k)
+    gates = _orig["gate_values"](logits, scores, idx, gate_mode, route_scale)
+    return dict(idx=idx, gates=gates, logits=logits, scores=scores, biased=biased, eligible=eligible)
+
+
+def _gate_bwd_no_route_scale(logits, scores, idx, gates, dgates, gate_mode, route_scale):
+    if gate_mode == orc.GATE_SIGMOID:
+        return _orig["gate_backward"](logits, scores, idx, gates, dgates, gate_mode, 1.0)
+    return _orig["gate_backward"](logits, scores, idx, np.asarray(gates, np.float64) / route_scale, dgates,
+                                  gate_mode, 1.0)
+
+
+def _gate_bwd_softmax_over_all(logits, scores, idx, gates, dgates, gate_mode, route_scale):
+    # Softmax Jacobian taken over all E logits instead of the k selected ones.
+    if gate_mode != orc.GATE_SOFTMAX:
+        return _orig["gate_backward"](logits, scores, idx, gates, dgates, gate_mode, route_scale)
+    l = np.asarray(logits, np.float64)
+    T, k = idx.shape
+    rows = np.arange(T)[:, None]
+    p_all = np.exp(l - l.max(axis=1, keepdims=True))
+    p_all /= p_all.sum(axis=1, keepdims=True)
+    dp = np.zeros_like(l)
+    dp[rows, idx] = route_scale * np.asarray(dgates, np.float64)
+    return p_all * (dp - (p_all * dp).sum(axis=1, keepdims=True))
+
+
 def _moe_bwd_no_router(*a, **kw):
     g = _orig["moe_backward"](*a, **kw)
     x = np.asarray(a[0], np.float64)
@@ -250,6 +284,9 @@ MUTATIONS = {
     "gate_bwd_no_sigmoid_factor": ("gate_backward", _gate_bwd_no_sigmoid_factor),
     "gate_bwd_no_centering": ("gate_backward", _gate_bwd_no_centering),
     "backward_drops_router": ("moe_backward", _moe_bwd_no_router),
+    "group_score_unbiased": ("route", _route_groups_from_unbiased),
+    "gate_bwd_no_route_scale": ("gate_backward", _gate_bwd_no_route_scale),
+    "gate_bwd_softmax_over_all": ("gate_backward", _gate_bwd_softmax_over_all),
 }
 
 
