@@ -387,6 +387,17 @@ def pin_near_tie_flags():
     assert orc.near_tie_tokens(r, 2, 3, 2).tolist() == [False, False]
 
 
+def pin_near_tie_gap_is_on_biased_scores():
+    # The near-tie rule measures the k-th / (k+1)-th gap of the selection
+    # scores s + b, the values top-k ranks. Token 0: the raw scores tie (1, 1)
+    # but the bias separates them (1.5 vs 1) -> not a near tie. Token 1: the
+    # raw scores differ (0.5 vs 1) but the bias closes the gap (1 vs 1) -> a
+    # near tie. k = 1, softmax mode (s = raw logit).
+    lg = np.array([[1.0, 1.0, -1.0, -2.0], [0.5, 1.0, -1.0, -2.0]])
+    r = orc.route(lg, np.eye(4), np.array([0.5, 0.0, 0.0, 0.0]), 1, orc.GATE_SOFTMAX)
+    assert orc.near_tie_tokens(r, 1).tolist() == [False, True]
+
+
 # ------------------------------------------------------- balance loop
 def pin_entropy_closed_forms():
     for E in (1, 2, 7, 256):

@@ -240,6 +240,33 @@ def _gate_bwd_softmax_over_all(logits, scores, idx, gates, dgates, gate_mode, ro
     return p_all * (dp - (p_all * dp).sum(axis=1, keepdims=True))
 
 
+def _biased_softmax_of_logits(scores, bias):
+    # Softmax-mode bias added to softmax probabilities over all experts
+    # instead of to the raw logit (sigmoid mode unchanged).
+    sc = np.asarray(scores, np.float64)
+    if bias is None:
+        return sc.copy()
+    p = np.exp(sc - sc.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    return p + np.asarray(bias, np.float64)[None, :]
+
+
+def _gates_sigmoid_over_all(logits, scores, idx, gate_mode, route_scale):
+    # Sigmoid gates renormalised over all E scores instead of the k selected.
+    if gate_mode != orc.GATE_SIGMOID:
+        return _orig["gate_values"](logits, scores, idx, gate_mode, route_scale)
+    sc = np.asarray(scores, np.float64)
+    rows = np.arange(idx.shape[0])[:, None]
+    return sc[rows, idx] / sc.sum(axis=1, keepdims=True) * route_scale
+
+
+def _near_tie_unbiased(routed, k, n_groups=1, topk_groups=1, eps=1e-5):
+    # Gap measured on the unbiased scores instead of the selection scores.
+    r = dict(routed)
+    r["biased"] = routed["scores"]
+    return _orig["near_tie_tokens"](r, k, n_groups, topk_groups, eps)
+
+
 def _moe_bwd_no_router(*a, **kw):
     g = _orig["moe_backward"](*a, **kw)
     x = np.asarray(a[0], np.float64)
@@ -287,6 +314,9 @@ MUTATIONS = {
     "group_score_unbiased": ("route", _route_groups_from_unbiased),
     "gate_bwd_no_route_scale": ("gate_backward", _gate_bwd_no_route_scale),
     "gate_bwd_softmax_over_all": ("gate_backward", _gate_bwd_softmax_over_all),
+    "softmax_bias_on_probabilities": ("biased_scores", _biased_softmax_of_logits),
+    "sigmoid_gates_over_all_experts": ("gate_values", _gates_sigmoid_over_all),
+    "near_tie_gap_unbiased": ("near_tie_tokens", _near_tie_unbiased),
 }
 
 
