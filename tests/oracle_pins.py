@@ -260,6 +260,12 @@ def pin_brute_force_group_limited():
     # top-2 sum (0.6 + 0.5 > 0.9 + 0.0); keeping one group selects expert 2.
     b = np.array([[0.9, 0.0, 0.6, 0.5]])
     assert orc.select_experts(b, orc.group_eligibility(b, 2, 1), 1)[0].tolist() == [2]
+    # Groups of three: the score counts the two best members only, so a weak
+    # third member does not pull group 0 (0.9 + 0.8 = 1.7) below group 1
+    # (0.5 + 0.5 = 1.0, whose three members would sum to 1.5 > -3.3).
+    b = np.array([[0.9, 0.8, -5.0, 0.5, 0.5, 0.5]])
+    assert np.allclose(orc.group_scores(b, 2)[0], [1.7, 1.0], rtol=0, atol=1e-15)
+    assert orc.select_experts(b, orc.group_eligibility(b, 2, 1), 1)[0].tolist() == [0]
     rng = np.random.default_rng(22)
     for trial in range(60):
         n_groups = int(rng.choice([2, 4]))

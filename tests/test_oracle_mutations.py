@@ -5,6 +5,8 @@ so the oracle's own callers see it) with a variant that carries one error:
 a dropped term, a wrong sign or index, a transposed or swapped operand, a
 missing step. The pins must fail (raise) for every one of them.
 """
+import inspect
+
 import numpy as np
 import pytest
 
@@ -267,6 +269,46 @@ def _near_tie_unbiased(routed, k, n_groups=1, topk_groups=1, eps=1e-5):
     return _orig["near_tie_tokens"](r, k, n_groups, topk_groups, eps)
 
 
+def _bias_update_proportional(bias, counts, target, gamma):
+    # A step proportional to the miss instead of a fixed +-gamma.
+    b = np.asarray(bias, np.float64).copy()
+    return b - gamma * (np.asarray(counts, np.float64) - target)
+
+
+def _moe_bwd_no_shared_dx(*a, **kw):
+    g = _orig["moe_backward"](*a, **kw)
+    bound = inspect.signature(_orig["moe_backward"]).bind(*a, **kw)
+    bound.apply_defaults()
+    ar = bound.arguments
+    if ar["ws1"] is not None:
+        du = _orig["swiglu_ffn_backward"](np.asarray(ar["x"], np.float64), ar["ws1"], ar["ws3"], ar["ws2"],
+                                          np.asarray(ar["dy"], np.float64))[0]
+        g["dx"] = g["dx"] - du
+    return g
+
+
+def _moe_bwd_shared_dw_swapped(*a, **kw):
+    g = _orig["moe_backward"](*a, **kw)
+    if g["dws1"] is not None:
+        g["dws1"], g["dws3"] = g["dws3"], g["dws1"]
+    return g
+
+
+def _rows_slots_swapped(idx, offsets):
+    # inv_row of a token's first two slots exchanged (perm_src unchanged).
+    inv_row, perm_src = _orig["permutation_rows"](idx, offsets)
+    if inv_row.shape[1] >= 2:
+        inv_row = inv_row.copy()
+        inv_row[:, [0, 1]] = inv_row[:, [1, 0]]
+    return inv_row, perm_src
+
+
+def _group_sum_all(biased, n_groups):
+    b = np.asarray(biased, np.float64)
+    T, E = b.shape
+    return b.reshape(T, n_groups, E // n_groups).sum(axis=2)
+
+
 def _moe_bwd_no_router(*a, **kw):
     g = _orig["moe_backward"](*a, **kw)
     x = np.asarray(a[0], np.float64)
@@ -317,6 +359,11 @@ MUTATIONS = {
     "softmax_bias_on_probabilities": ("biased_scores", _biased_softmax_of_logits),
     "sigmoid_gates_over_all_experts": ("gate_values", _gates_sigmoid_over_all),
     "near_tie_gap_unbiased": ("near_tie_tokens", _near_tie_unbiased),
+    "bias_update_proportional": ("update_bias", _bias_update_proportional),
+    "inv_row_slots_swapped": ("permutation_rows", _rows_slots_swapped),
+    "group_score_sum_of_all": ("group_scores", _group_sum_all),
+    "backward_drops_shared_dx": ("moe_backward", _moe_bwd_no_shared_dx),
+    "backward_shared_dw1_dw3_swapped": ("moe_backward", _moe_bwd_shared_dw_swapped),
 }
 
 
