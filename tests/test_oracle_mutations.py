@@ -309,6 +309,27 @@ def _group_sum_all(biased, n_groups):
     return b.reshape(T, n_groups, E // n_groups).sum(axis=2)
 
 
+def _silu_grad_no_sigma_term(z):
+    # The derivative of z * sigma(z) without its first term sigma(z).
+    z = np.asarray(z, np.float64)
+    sig = 1.0 / (1.0 + np.exp(-z))
+    return z * sig * (1.0 - sig)
+
+
+def _outputs_first_slot_only(x, idx, gates, w1, w3, w2, ws1=None, ws3=None, ws2=None):
+    idx = np.asarray(idx)
+    return _orig["expert_outputs"](x, idx[:, :1], np.asarray(gates)[:, :1], w1, w3, w2, ws1, ws3, ws2)
+
+
+def _swiglu_bwd_du_w1_only(u, w1, w3, w2, dout):
+    # Input gradient through the W1 branch only (the W3 branch's da/db term dropped).
+    du, dw1, dw3, dw2 = _orig["swiglu_ffn_backward"](u, w1, w3, w2, dout)
+    u64, w1_, w3_, w2_, d64 = (np.asarray(v, np.float64) for v in (u, w1, w3, w2, dout))
+    a = u64 @ w1_.T
+    db = (d64 @ w2_) * _orig["silu"](a)
+    return du - db @ w3_, dw1, dw3, dw2
+
+
 def _moe_bwd_no_router(*a, **kw):
     g = _orig["moe_backward"](*a, **kw)
     x = np.asarray(a[0], np.float64)
@@ -361,6 +382,9 @@ MUTATIONS = {
     "near_tie_gap_unbiased": ("near_tie_tokens", _near_tie_unbiased),
     "bias_update_proportional": ("update_bias", _bias_update_proportional),
     "inv_row_slots_swapped": ("permutation_rows", _rows_slots_swapped),
+    "silu_grad_no_sigma_term": ("silu_grad", _silu_grad_no_sigma_term),
+    "routed_sum_first_slot_only": ("expert_outputs", _outputs_first_slot_only),
+    "swiglu_bwd_du_drops_w3_branch": ("swiglu_ffn_backward", _swiglu_bwd_du_w1_only),
     "group_score_sum_of_all": ("group_scores", _group_sum_all),
     "backward_drops_shared_dx": ("moe_backward", _moe_bwd_no_shared_dx),
     "backward_shared_dw1_dw3_swapped": ("moe_backward", _moe_bwd_shared_dw_swapped),
