@@ -330,6 +330,37 @@ def _swiglu_bwd_du_w1_only(u, w1, w3, w2, dout):
     return du - db @ w3_, dw1, dw3, dw2
 
 
+def _select_descending(biased, eligible, k):
+    # Winners left in descending-score order instead of ascending expert id.
+    masked = np.where(eligible, np.asarray(biased, np.float64), -np.inf)
+    return np.argsort(-masked, axis=1, kind="stable")[:, :k]
+
+
+def _affinity_softmax_probs(logits, gate_mode):
+    # Softmax mode scores as probabilities over all E instead of raw logits.
+    if gate_mode != orc.GATE_SOFTMAX:
+        return _orig["affinity"](logits, gate_mode)
+    l = np.asarray(logits, np.float64)
+    p = np.exp(l - l.max(axis=1, keepdims=True))
+    return p / p.sum(axis=1, keepdims=True)
+
+
+def _rows_slot_major(idx, offsets):
+    # Packed rows filled slot by slot (all tokens' slot 0, then slot 1, ...).
+    idx = np.asarray(idx)
+    T, k = idx.shape
+    nxt = np.asarray(offsets[:-1], dtype=np.int64).copy()
+    inv_row = np.empty((T, k), dtype=np.int64)
+    perm_src = np.full(int(offsets[-1]), -1, dtype=np.int64)
+    for j in range(k):
+        for t in range(T):
+            e = idx[t, j]
+            inv_row[t, j] = nxt[e]
+            perm_src[nxt[e]] = t
+            nxt[e] += 1
+    return inv_row, perm_src
+
+
 def _moe_bwd_no_router(*a, **kw):
     g = _orig["moe_backward"](*a, **kw)
     x = np.asarray(a[0], np.float64)
@@ -383,6 +414,9 @@ MUTATIONS = {
     "bias_update_proportional": ("update_bias", _bias_update_proportional),
     "inv_row_slots_swapped": ("permutation_rows", _rows_slots_swapped),
     "silu_grad_no_sigma_term": ("silu_grad", _silu_grad_no_sigma_term),
+    "winners_in_score_order": ("select_experts", _select_descending),
+    "softmax_scores_as_probabilities": ("affinity", _affinity_softmax_probs),
+    "rows_filled_slot_major": ("permutation_rows", _rows_slot_major),
     "routed_sum_first_slot_only": ("expert_outputs", _outputs_first_slot_only),
     "swiglu_bwd_du_drops_w3_branch": ("swiglu_ffn_backward", _swiglu_bwd_du_w1_only),
     "group_score_sum_of_all": ("group_scores", _group_sum_all),
