@@ -119,3 +119,28 @@ def test_output_check_bounds(dtype):
     y[1] = np.nan
     with pytest.raises(AssertionError):
         H.compare_outputs(cfg, y, y_ref)
+
+
+def test_gradient_check_bounds():
+    from test_gpu_backward import compare_grad
+    cfg = CFG.with_(dtype="bf16")
+    rng = np.random.default_rng(9)
+    g_ref = rng.standard_t(3, size=(48, 40))          # heavy-tailed, like weight gradients
+    rms = float(np.sqrt(np.mean(g_ref ** 2)))
+    compare_grad(cfg, g_ref.copy(), g_ref, "g")
+    # every element off by a quarter of its own bound, in a random direction:
+    # inside the elementwise rule and the relative L2 bound
+    bound = 5e-2 * rms + 1e-2 * np.abs(g_ref)
+    within = g_ref + 0.25 * bound * np.sign(rng.standard_normal(g_ref.shape))
+    compare_grad(cfg, within, g_ref, "g")
+    # one element beyond its bound
+    y = g_ref.copy()
+    y[4, 4] += 2 * (5e-2 * rms + 1e-2 * abs(g_ref[4, 4]))
+    with pytest.raises(AssertionError, match="elementwise"):
+        compare_grad(cfg, y, g_ref, "g")
+    # a uniform 3% error: above the relative L2 bound
+    with pytest.raises(AssertionError, match="relative L2"):
+        compare_grad(cfg, g_ref * 1.03, g_ref, "g")
+    # fp32 gradients use the 1e-5 relative L2 bound
+    with pytest.raises(AssertionError, match="relative L2"):
+        compare_grad(cfg.with_(dtype="f32"), g_ref * (1 + 1e-4), g_ref, "g")
