@@ -422,6 +422,17 @@ def pin_bias_update_direction():
     _close(b, [0.35, -0.25, 0.15, 1.0], tol=1e-15)
 
 
+def pin_balance_target_is_not_rounded():
+    # The cheat sheet's "Aux-loss-free balance loop", step 1: target usage =
+    # n_tokens * top_k / n_experts, a real number. 10 tokens x top-3 over 4
+    # experts target 7.5 each, so counts of 7 and 8 are under and over target
+    # (none is on target) and every bias moves.
+    t = orc.balance_target(10, 3, 4)
+    assert t == 7.5
+    b = orc.update_bias([0.0, 0.0, 0.0, 0.0], [7, 8, 8, 7], t, 0.25)
+    assert np.array_equal(b, [0.25, -0.25, -0.25, 0.25])
+
+
 def pin_balance_loop_raises_entropy():
     # The cheat sheet's loop: route with scores + bias, count, update with
     # gamma = 0.15, 10 iterations; entropy rises toward ln(E). A router whose

@@ -361,6 +361,16 @@ def _rows_slot_major(idx, offsets):
     return inv_row, perm_src
 
 
+def _gelu_erf_without_sqrt2(z):
+    from math import erf
+    z = np.asarray(z, np.float64)
+    return 0.5 * z * (1.0 + np.vectorize(erf)(z))
+
+
+def _target_integer_division(T, k, E):
+    return float((T * k) // E)
+
+
 def _moe_bwd_no_router(*a, **kw):
     g = _orig["moe_backward"](*a, **kw)
     x = np.asarray(a[0], np.float64)
@@ -415,6 +425,8 @@ MUTATIONS = {
     "inv_row_slots_swapped": ("permutation_rows", _rows_slots_swapped),
     "silu_grad_no_sigma_term": ("silu_grad", _silu_grad_no_sigma_term),
     "winners_in_score_order": ("select_experts", _select_descending),
+    "gelu_erf_without_sqrt2": ("gelu", _gelu_erf_without_sqrt2),
+    "target_integer_division": ("balance_target", _target_integer_division),
     "softmax_scores_as_probabilities": ("affinity", _affinity_softmax_probs),
     "rows_filled_slot_major": ("permutation_rows", _rows_slot_major),
     "routed_sum_first_slot_only": ("expert_outputs", _outputs_first_slot_only),
