@@ -393,6 +393,18 @@ def pin_near_tie_flags():
     assert orc.near_tie_tokens(r, 2, 3, 2).tolist() == [False, False]
 
 
+def pin_near_tie_ignores_dropped_groups():
+    # Top-k chooses among the experts of the kept groups only, so an expert of a
+    # dropped group that ties the k-th winner cannot change the selection: not
+    # a near tie. Groups {0,1} (1.0 + 0.9) and {2,3} (1.0 - 3.0), keep one,
+    # k = 1: expert 0 wins against 0.9 inside its group; expert 2's 1.0 does
+    # not count, and the group scores are far apart.
+    lg = np.array([[1.0, 0.9, 1.0, -3.0]])
+    r = orc.route(lg, np.eye(4), None, 1, orc.GATE_SOFTMAX, n_groups=2, topk_groups=1)
+    assert r["idx"].tolist() == [[0]]
+    assert orc.near_tie_tokens(r, 1, 2, 1).tolist() == [False]
+
+
 def pin_near_tie_gap_is_on_biased_scores():
     # The near-tie rule measures the k-th / (k+1)-th gap of the selection
     # scores s + b, the values top-k ranks. Token 0: the raw scores tie (1, 1)

@@ -371,6 +371,19 @@ def _target_integer_division(T, k, E):
     return float((T * k) // E)
 
 
+def _near_tie_ignores_eligibility(routed, k, n_groups=1, topk_groups=1, eps=1e-5):
+    # k-th / (k+1)-th gap taken over all experts, dropped groups included.
+    r = dict(routed)
+    r["eligible"] = np.ones_like(np.asarray(routed["eligible"]), dtype=bool)
+    return _orig["near_tie_tokens"](r, k, n_groups, topk_groups, eps)
+
+
+def _logits_with_bias_inside(x, w_router):
+    # A constant offset folded into the router linear (as if the selection
+    # bias were a linear-layer bias): shifts every logit by the same amount.
+    return _orig["router_logits"](x, w_router) + 0.1
+
+
 def _moe_bwd_no_router(*a, **kw):
     g = _orig["moe_backward"](*a, **kw)
     x = np.asarray(a[0], np.float64)
@@ -426,6 +439,8 @@ MUTATIONS = {
     "silu_grad_no_sigma_term": ("silu_grad", _silu_grad_no_sigma_term),
     "winners_in_score_order": ("select_experts", _select_descending),
     "gelu_erf_without_sqrt2": ("gelu", _gelu_erf_without_sqrt2),
+    "near_tie_ignores_group_mask": ("near_tie_tokens", _near_tie_ignores_eligibility),
+    "router_logits_offset": ("router_logits", _logits_with_bias_inside),
     "target_integer_division": ("balance_target", _target_integer_division),
     "softmax_scores_as_probabilities": ("affinity", _affinity_softmax_probs),
     "rows_filled_slot_major": ("permutation_rows", _rows_slot_major),
