@@ -384,6 +384,33 @@ def _logits_with_bias_inside(x, w_router):
     return _orig["router_logits"](x, w_router) + 0.1
 
 
+def _moe_bwd_dgate_with_gate(*a, **kw):
+    # dL/dg taken as <dy, g * FFN(x)> instead of <dy, FFN(x)>: the logit
+    # gradient is recomputed from the scaled dgates.
+    g = _orig["moe_backward"](*a, **kw)
+    bound = inspect.signature(_orig["moe_backward"]).bind(*a, **kw)
+    bound.apply_defaults()
+    ar = bound.arguments
+    dg = g["dgates"] * g["gates"]
+    r = _orig["route"](ar["x"], ar["w_router"], ar["bias"], ar["k"], ar["gate_mode"], ar["n_groups"],
+                       ar["topk_groups"], ar["route_scale"])
+    dl = _orig["gate_backward"](r["logits"], r["scores"], g["idx"], g["gates"], dg, ar["gate_mode"],
+                                ar["route_scale"])
+    x = np.asarray(ar["x"], np.float64)
+    w = np.asarray(ar["w_router"], np.float64)
+    g["dx"] = g["dx"] - g["dlogits"] @ w + dl @ w
+    g["dw_router"] = dl.T @ x
+    g["dgates"], g["dlogits"] = dg, dl
+    return g
+
+
+def _rows_first_row_of_expert(idx, offsets):
+    # inv_row points at the expert's first packed row for every token.
+    inv_row, perm_src = _orig["permutation_rows"](idx, offsets)
+    idx = np.asarray(idx)
+    return np.asarray(offsets)[idx].astype(np.int64), perm_src
+
+
 def _moe_bwd_no_router(*a, **kw):
     g = _orig["moe_backward"](*a, **kw)
     x = np.asarray(a[0], np.float64)
@@ -440,6 +467,8 @@ MUTATIONS = {
     "winners_in_score_order": ("select_experts", _select_descending),
     "gelu_erf_without_sqrt2": ("gelu", _gelu_erf_without_sqrt2),
     "near_tie_ignores_group_mask": ("near_tie_tokens", _near_tie_ignores_eligibility),
+    "backward_dgate_includes_gate": ("moe_backward", _moe_bwd_dgate_with_gate),
+    "inv_row_first_row_of_expert": ("permutation_rows", _rows_first_row_of_expert),
     "router_logits_offset": ("router_logits", _logits_with_bias_inside),
     "target_integer_division": ("balance_target", _target_integer_division),
     "softmax_scores_as_probabilities": ("affinity", _affinity_softmax_probs),
