@@ -411,6 +411,21 @@ def _rows_first_row_of_expert(idx, offsets):
     return np.asarray(offsets)[idx].astype(np.int64), perm_src
 
 
+def _hidden_both_gated(u, w1, w3):
+    # SiLU applied to both branches.
+    u = np.asarray(u, np.float64)
+    return _orig["silu"](u @ np.asarray(w1, np.float64).T) * _orig["silu"](u @ np.asarray(w3, np.float64).T)
+
+
+def _silu_wrong_sign(z):
+    z = np.asarray(z, np.float64)
+    return z / (1.0 + np.exp(z))
+
+
+def _groups_keep_one_more(biased, n_groups, topk_groups):
+    return _orig["group_eligibility"](biased, n_groups, min(n_groups, topk_groups + 1))
+
+
 def _moe_bwd_no_router(*a, **kw):
     g = _orig["moe_backward"](*a, **kw)
     x = np.asarray(a[0], np.float64)
@@ -468,6 +483,9 @@ MUTATIONS = {
     "gelu_erf_without_sqrt2": ("gelu", _gelu_erf_without_sqrt2),
     "near_tie_ignores_group_mask": ("near_tie_tokens", _near_tie_ignores_eligibility),
     "backward_dgate_includes_gate": ("moe_backward", _moe_bwd_dgate_with_gate),
+    "hidden_silu_on_both_branches": ("swiglu_hidden", _hidden_both_gated),
+    "silu_wrong_sign": ("silu", _silu_wrong_sign),
+    "groups_keep_one_more": ("group_eligibility", _groups_keep_one_more),
     "inv_row_first_row_of_expert": ("permutation_rows", _rows_first_row_of_expert),
     "router_logits_offset": ("router_logits", _logits_with_bias_inside),
     "target_integer_division": ("balance_target", _target_integer_division),
