@@ -49,6 +49,7 @@ again in the design notes):
 """
 from __future__ import annotations
 
+import itertools
 import math
 from typing import Optional, Sequence
 
@@ -342,8 +343,12 @@ def near_tie_tokens(routed: dict, k: int, n_groups: int = 1, topk_groups: int = 
 
     A token is flagged when the k-th and (k+1)-th largest eligible biased
     scores differ by less than ``eps``, or, with group-limited routing, when
-    the last kept and first dropped group scores differ by less than ``eps``
-    AND swapping those two groups changes the selected set.
+    the group ranking is ambiguous at its boundary and that can change the
+    selected set: the near groups are the kept ones less than ``eps`` above
+    the first dropped score and the dropped ones less than ``eps`` below the
+    last kept score; every way of filling the kept places those near groups
+    compete for is tried, and the token is flagged if any of them selects a
+    different set of experts.
     """
     biased = routed["biased"]
     eligible = routed["eligible"]
@@ -360,15 +365,21 @@ def near_tie_tokens(routed: dict, k: int, n_groups: int = 1, topk_groups: int = 
         order = np.argsort(-gscore, axis=1, kind="stable")
         size = E // n_groups
         for t in range(T):
-            last, first_out = order[t, topk_groups - 1], order[t, topk_groups]
-            if gscore[t, last] - gscore[t, first_out] >= eps:
+            kept, dropped = list(order[t, :topk_groups]), list(order[t, topk_groups:])
+            hi, lo = gscore[t, kept[-1]], gscore[t, dropped[0]]
+            if hi - lo >= eps:
                 continue
-            alt = np.zeros(E, dtype=bool)
-            for g in list(order[t, :topk_groups - 1]) + [first_out]:
-                alt[g * size:(g + 1) * size] = True
-            alt_sel = select_experts(biased[t:t + 1], alt[None, :], k)[0]
-            if not np.array_equal(alt_sel, routed["idx"][t]):
-                flags[t] = True
+            near = [g for g in kept if gscore[t, g] - lo < eps] + \
+                   [g for g in dropped if hi - gscore[t, g] < eps]
+            sure = [g for g in kept if g not in near]
+            for pick in itertools.combinations(near, topk_groups - len(sure)):
+                alt = np.zeros(E, dtype=bool)
+                for g in sure + list(pick):
+                    alt[g * size:(g + 1) * size] = True
+                alt_sel = select_experts(biased[t:t + 1], alt[None, :], k)[0]
+                if not np.array_equal(alt_sel, routed["idx"][t]):
+                    flags[t] = True
+                    break
     return flags
 
 

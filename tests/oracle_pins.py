@@ -393,6 +393,24 @@ def pin_near_tie_flags():
     assert orc.near_tie_tokens(r, 2, 3, 2).tolist() == [False, False]
 
 
+def pin_near_tie_three_groups_at_the_boundary():
+    # Three groups within 1e-5 of one another, keep two, k = 1. Groups are
+    # {0,1}, {2,3}, {4,5}; their scores (sums of both members) are 1.0,
+    # 1.0 - 2e-6 and 1.0 - 4e-6, so groups 0 and 1 are kept and expert 0
+    # (0.9) wins. Exchanging the last kept and first dropped group (1 and 2)
+    # leaves expert 0 the winner, but another rounding could rank group 0
+    # last and drop it, and then expert 4 (0.6) would win: a near tie.
+    lg = np.array([[0.9, 0.1, 0.5, 0.5 - 2e-6, 0.6, 0.4 - 4e-6]])
+    r = orc.route(lg, np.eye(6), None, 1, orc.GATE_SOFTMAX, n_groups=3, topk_groups=2)
+    assert r["idx"].tolist() == [[0]]
+    assert orc.near_tie_tokens(r, 1, 3, 2).tolist() == [True]
+    # The same scores with group 0 well ahead (1.2): only groups 1 and 2 are
+    # near the boundary, and either keeps expert 0 the winner: no near tie.
+    lg2 = np.array([[0.9, 0.3, 0.5, 0.5 - 2e-6, 0.6, 0.4 - 4e-6]])
+    r2 = orc.route(lg2, np.eye(6), None, 1, orc.GATE_SOFTMAX, n_groups=3, topk_groups=2)
+    assert orc.near_tie_tokens(r2, 1, 3, 2).tolist() == [False]
+
+
 def pin_near_tie_ignores_dropped_groups():
     # Top-k chooses among the experts of the kept groups only, so an expert of a
     # dropped group that ties the k-th winner cannot change the selection: not

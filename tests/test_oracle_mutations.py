@@ -371,6 +371,28 @@ def _target_integer_division(T, k, E):
     return float((T * k) // E)
 
 
+def _near_tie_pair_swap_only(routed, k, n_groups=1, topk_groups=1, eps=1e-5):
+    # Group boundary checked by exchanging only the last kept and the first
+    # dropped group.
+    flags = _orig["near_tie_tokens"](routed, k, 1, 1, eps)
+    if n_groups > 1 and topk_groups < n_groups:
+        biased = routed["biased"]
+        T, E = biased.shape
+        gscore = orc.group_scores(biased, n_groups)
+        order = np.argsort(-gscore, axis=1, kind="stable")
+        size = E // n_groups
+        for t in range(T):
+            last, first_out = order[t, topk_groups - 1], order[t, topk_groups]
+            if gscore[t, last] - gscore[t, first_out] >= eps:
+                continue
+            alt = np.zeros(E, dtype=bool)
+            for g in list(order[t, :topk_groups - 1]) + [first_out]:
+                alt[g * size:(g + 1) * size] = True
+            if not np.array_equal(orc.select_experts(biased[t:t + 1], alt[None, :], k)[0], routed["idx"][t]):
+                flags[t] = True
+    return flags
+
+
 def _near_tie_ignores_eligibility(routed, k, n_groups=1, topk_groups=1, eps=1e-5):
     # k-th / (k+1)-th gap taken over all experts, dropped groups included.
     r = dict(routed)
@@ -482,6 +504,7 @@ MUTATIONS = {
     "winners_in_score_order": ("select_experts", _select_descending),
     "gelu_erf_without_sqrt2": ("gelu", _gelu_erf_without_sqrt2),
     "near_tie_ignores_group_mask": ("near_tie_tokens", _near_tie_ignores_eligibility),
+    "near_tie_group_pair_swap_only": ("near_tie_tokens", _near_tie_pair_swap_only),
     "backward_dgate_includes_gate": ("moe_backward", _moe_bwd_dgate_with_gate),
     "hidden_silu_on_both_branches": ("swiglu_hidden", _hidden_both_gated),
     "silu_wrong_sign": ("silu", _silu_wrong_sign),
