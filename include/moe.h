@@ -21,7 +21,8 @@
  *   moe_expert_gelu, moe_forward_gelu         generic experts W2 GELU(W1 u + b1) + b2
  *   moe_backward (_workspace_size), moe_forward_train, moe_backward_saved
  *                                             gradients of the block for training
- *   moe_get_device_error, moe_selftest_wait_timeout, moe_status_string
+ *   moe_get_device_error, moe_route_noalloc_device_error,
+ *   moe_selftest_wait_timeout, moe_status_string
  *
  * Sources, cited by page title and section:
  *   [DS] "Sparse MoE FFN" DeepSeek-V3 study note, "How it works": eq. 12
@@ -399,6 +400,22 @@ MOE_API moe_status moe_backward_saved(const moe_config* cfg, const void* x, cons
 MOE_API moe_status moe_route_noalloc(const moe_config* cfg, const void* x, const void* w_router,
                              const float* bias, int32_t* topk_idx, float* topk_gate,
                              int32_t* expert_counts, int32_t* expert_offsets, void* stream);
+
+/*
+ * moe_route_noalloc_device_error - the error word of moe_route_noalloc's
+ * fixed array on the current device, which no workspace pointer reaches.
+ * The pages have no counterpart: like moe_get_device_error, this only reports
+ * on the call's own bounded device waits.
+ *
+ * Synchronises `stream`, reads the word, clears it and returns MOE_OK or
+ * MOE_ERR_TIMEOUT (a device wait of a moe_route_noalloc call on this device
+ * ran out, so its routing is not to be trusted); MOE_ERR_CUDA if a CUDA call
+ * fails, MOE_ERR_UNSUPPORTED for a device ordinal of 64 or more. Allocates
+ * nothing. Call it on the stream of the moe_route_noalloc calls it checks,
+ * with their device current; like those calls it must not overlap another
+ * moe_route_noalloc on the same device.
+ */
+MOE_API moe_status moe_route_noalloc_device_error(void* stream);
 
 /*
  * moe_balance_update - the aux-loss-free balancing step that follows routing

@@ -34,7 +34,8 @@ MOE_DTYPE_BF16 = 1
 EXPORTED = ("moe_check_config", "moe_workspace_size", "moe_route", "moe_permute",
             "moe_expert_swiglu", "moe_expert_gate_up", "moe_expert_gate_up_gather", "moe_expert_down",
             "moe_combine", "moe_forward", "moe_get_device_error",
-            "moe_selftest_wait_timeout", "moe_route_noalloc", "moe_balance_update",
+            "moe_selftest_wait_timeout", "moe_route_noalloc", "moe_route_noalloc_device_error",
+            "moe_balance_update",
             "moe_expert_gelu", "moe_forward_gelu", "moe_backward_workspace_size", "moe_backward",
             "moe_forward_train", "moe_backward_saved", "moe_status_string")
 
@@ -86,6 +87,7 @@ def lib() -> ctypes.CDLL:
             "moe_get_device_error": (ctypes.c_int, [vp, vp]),
             "moe_selftest_wait_timeout": (ctypes.c_int, [vp, sz, ctypes.c_int64, vp]),
             "moe_route_noalloc": (ctypes.c_int, [cfgp, vp, vp, f32p, i32p, f32p, i32p, i32p, vp]),
+            "moe_route_noalloc_device_error": (ctypes.c_int, [vp]),
             "moe_balance_update": (ctypes.c_int, [cfgp, i32p, f32p, ctypes.c_float, f32p, vp]),
             "moe_expert_gelu": (ctypes.c_int, [cfgp, vp, i32p, vp, f32p, vp, f32p, vp, vp, sz, vp]),
             "moe_forward_gelu": (ctypes.c_int, [cfgp, vp, vp, f32p, vp, f32p, vp, f32p, vp, vp, sz, vp]),
@@ -436,6 +438,13 @@ def moe_route_noalloc(cfg, x, w_router, bias, topk_idx, topk_gate, expert_counts
     _check(lib().moe_route_noalloc(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(bias),
                                    _ptr(topk_idx), _ptr(topk_gate), _ptr(expert_counts),
                                    _ptr(expert_offsets), _stream(stream)), "moe_route_noalloc")
+
+
+def moe_route_noalloc_device_error(stream=None) -> int:
+    """Status of moe_route_noalloc's bounded device waits on the current
+    device (synchronises the stream, then reads and clears the fixed array's
+    error word): MOE_OK or MOE_ERR_TIMEOUT."""
+    return lib().moe_route_noalloc_device_error(_stream(stream))
 
 
 def moe_balance_update(cfg, expert_counts, bias, gamma: float, entropy=None, stream=None):

@@ -86,9 +86,11 @@ __global__ void __launch_bounds__(256) gate_bwd_kernel(
   if (rowb)
     for (int e = lane; e < e_pad; e += 32) rowb[e] = __float2bfloat16_rn(0.0f);
   __syncwarp();
-  // Lanes j < k hold slot j (k <= 32).
-  const bool act = lane < k;
-  const int e = act ? idx[(size_t)t * k + lane] : 0;
+  // Lanes j < k hold slot j (k <= 32). A slot whose id lies outside [0, E)
+  // (a caller-supplied topk_idx) is skipped before anything is read through it.
+  const int e_in = lane < k ? idx[(size_t)t * k + lane] : -1;
+  const bool act = lane < k && e_in >= 0 && e_in < E;
+  const int e = act ? e_in : 0;
   const float dg = act ? dgate[(size_t)t * k + lane] : 0.0f;
   float out = 0.0f;
   if (gate_mode == MOE_GATE_SIGMOID) {
@@ -106,7 +108,7 @@ __global__ void __launch_bounds__(256) gate_bwd_kernel(
     for (int o = 16; o > 0; o >>= 1) PD += __shfl_xor_sync(0xffffffffu, PD, o);
     out = route_scale * p * (dg - PD);
   }
-  if (act && e >= 0 && e < E) {
+  if (act) {
     row[e] = out;
     if (rowb) rowb[e] = __float2bfloat16_rn(out);
   }

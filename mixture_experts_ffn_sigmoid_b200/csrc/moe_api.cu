@@ -1209,3 +1209,17 @@ extern "C" moe_status moe_route_noalloc(const moe_config* cfg, const void* x, co
   return enqueue_route(c, x, w_router, bias, topk_idx, topk_gate, expert_counts, expert_offsets,
                        scratch, s);
 }
+
+// The fixed array's error word (its first bytes) on the current device:
+// synchronise the stream, read the word, clear it.
+extern "C" moe_status moe_route_noalloc_device_error(void* stream) {
+  void* scratch = nullptr;
+  MOE_TRY(route_scratch(&scratch));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t word = 0;
+  MOE_CUDA(cudaStreamSynchronize(s));
+  MOE_CUDA(cudaMemcpyAsync(&word, scratch, sizeof(word), cudaMemcpyDeviceToHost, s));
+  MOE_CUDA(cudaMemsetAsync(scratch, 0, sizeof(word), s));
+  MOE_CUDA(cudaStreamSynchronize(s));
+  return (word & kErrTimeoutWait) ? MOE_ERR_TIMEOUT : MOE_OK;
+}

@@ -50,6 +50,10 @@ __global__ void __launch_bounds__(1024, 1) router_topk_kernel(RouteParams p) {
         if (p.n_partials > 1) lrow[e] = l;
         const float s = (p.gate_mode == MOE_GATE_SIGMOID) ? sigmoid_f32(l) : l;
         b = s + (p.bias ? p.bias[e] : 0.0f);
+        // A NaN score (NaN or infinite input, NaN bias) ranks below every
+        // number, so it can neither win over a real score nor lose every
+        // comparison and leave the arg-max without a candidate.
+        if (isnan(b)) b = -INFINITY;
       }
       v[i] = b;
     }
@@ -78,7 +82,7 @@ __global__ void __launch_bounds__(1024, 1) router_topk_kernel(RouteParams p) {
           m1 = hi;
           m2 = lo;
         }
-        if (lane == G) my_gscore = m1 + m2;
+        if (lane == G) my_gscore = isnan(m1 + m2) ? -INFINITY : m1 + m2;   // +inf + -inf
       }
       // Keep the topk_groups best groups; ties go to the lower group index.
       int rank = 0;
@@ -95,24 +99,30 @@ __global__ void __launch_bounds__(1024, 1) router_topk_kernel(RouteParams p) {
     }
 
     // k rounds of a warp arg-max: largest b' first, equal b' to the lower id.
+    // kNone marks "no candidate yet": the first untaken in-range expert a lane
+    // sees always becomes its candidate, and a real candidate always beats
+    // kNone in the reduction. Round r < k <= E leaves at least one untaken
+    // expert, so every winner is an id in [0, E) whatever the scores hold.
+    constexpr int kNone = 0x7fffffff;
     unsigned taken = 0u;
     int my_e = -1;                     // lane j < k ends with the j-th winner
     for (int r = 0; r < k; ++r) {
       float bv = -INFINITY;
-      int be = 0x7fffffff;
+      int be = kNone;
 #pragma unroll
       for (int i = 0; i < NPL; ++i) {
         const int e = lane + 32 * i;
         if (e < E && !((taken >> i) & 1u)) {
-          if (v[i] > bv || (v[i] == bv && e < be)) { bv = v[i]; be = e; }
+          if (be == kNone || v[i] > bv || (v[i] == bv && e < be)) { bv = v[i]; be = e; }
         }
       }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) {
         const float ov = __shfl_xor_sync(kFull, bv, off);
         const int oe = __shfl_xor_sync(kFull, be, off);
-        if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+        if (oe != kNone && (be == kNone || ov > bv || (ov == bv && oe < be))) { bv = ov; be = oe; }
       }
+      if (be == kNone) be = 0;         // unreachable (k <= E); keeps the id in range regardless
       if ((be & 31) == lane) taken |= 1u << (be >> 5);
       if (lane == r) my_e = be;
     }

@@ -2,7 +2,8 @@
 one token, a token count that leaves a ragged 32-token chunk, k = E (every
 expert fires, bias irrelevant), all tokens on one expert (all other experts
 empty), a single expert (a dense SwiGLU), group limits that keep one group,
-no tokens at all, and the bounded-wait error path."""
+no tokens at all, a token whose scores are NaN or infinite, and the
+bounded-wait error path."""
 import numpy as np
 import pytest
 import torch
@@ -102,3 +103,35 @@ def test_bad_indices_are_skipped_not_dereferenced():
     inv = inv_row.cpu().numpy()
     assert inv[5, 1] == -1 and inv[7, 0] == -1
     assert inv.max() < rows
+
+
+NAN_CASES = {
+    "grouped_sigmoid": MoEConfig("nan_grouped", T=70, d=256, E=64, k=6, f=64, gate_mode=GATE_SIGMOID,
+                                 n_groups=8, topk_groups=4, route_scale=2.5, bias="uniform"),
+    "softmax": MoEConfig("nan_softmax", T=70, d=256, E=16, k=4, f=64),
+}
+
+
+@pytest.mark.parametrize("name", sorted(NAN_CASES))
+@pytest.mark.parametrize("bad", ["nan", "inf"])
+def test_non_finite_token_gets_valid_expert_ids(name, bad):
+    # One token row of NaN (or +inf) scores: its winners must still be k
+    # distinct in-range ids in ascending order (no index derived from a NaN
+    # comparison may leave [0, E)), counts still add up to T*k, and every
+    # other token is routed exactly as without the bad row.
+    cfg = NAN_CASES[name]
+    inp = H.gpu_inputs(cfg)
+    clean = H.gpu_route(cfg, inp)
+    inp["x"][5] = float(bad)
+    got = H.gpu_route(cfg, inp)
+    gi = got["idx"].cpu().numpy()
+    assert gi.min() >= 0 and gi.max() < cfg.E
+    assert np.all(np.diff(gi, axis=1) > 0)
+    assert int(got["counts"].sum().item()) == cfg.T * cfg.k
+    c, o = orc.expert_counts_offsets(gi, cfg.E)
+    assert np.array_equal(got["counts"].cpu().numpy(), c)
+    assert np.array_equal(got["offsets"].cpu().numpy(), o)
+    others = np.arange(cfg.T) != 5
+    assert np.array_equal(gi[others], clean["idx"].cpu().numpy()[others])
+    assert torch.equal(got["gate"][torch.as_tensor(others, device="cuda")],
+                       clean["gate"][torch.as_tensor(others, device="cuda")])

@@ -27,6 +27,8 @@ def _route_both(cfg, seed):
     counts = torch.full((E,), -7, dtype=torch.int32, device="cuda")
     offsets = torch.full((E + 1,), -7, dtype=torch.int32, device="cuda")
     B.moe_route_noalloc(cfg, inp["x"], inp["w_router"], inp["bias"], idx, gate, counts, offsets)
+    # The fixed array's error word: no bounded device wait of the call ran out.
+    assert B.moe_route_noalloc_device_error() == B.MOE_OK
     torch.cuda.synchronize()
     return ref, dict(idx=idx, gate=gate, counts=counts, offsets=offsets)
 
