@@ -63,6 +63,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--T", type=int, default=None, help="override the token count (profiling cases)")
     ap.add_argument("--E", type=int, default=None, help="override the routed expert count (profiling cases)")
+    ap.add_argument("--no-extra-workloads", action="store_true",
+                    help="time the headline workload only (the others run at N=1 by default)")
     return ap.parse_args()
 
 
@@ -443,6 +445,138 @@ def measure_fused_permute(B, cfg, inp, idx, offsets, perm_src, inv_row, h, h_s, 
             "note": "not used by moe_forward: slower than the packed copy plus gate/up"}
 
 
+def layer_bytes(cfg, touched):
+    """The layer's own compulsory HBM bytes for one forward: x, the router
+    matrix (and bias), every touched expert's three matrices, the shared
+    expert's, and y. Intermediates of this implementation are not counted."""
+    es = cfg.elem_bytes
+    T, d, E, f, fs = cfg.T, cfg.d, cfg.E, cfg.f, cfg.f_shared
+    return (2 * T * d + E * d + touched * 3 * f * d + 3 * fs * d) * es + (E * 4 if cfg.bias else 0)
+
+
+def stage_breakdown(B, cfg, inp, ws, stream, n):
+    """The forward through the per-stage entry points, one CUDA event between
+    stages on the launching stream, averaged over n passes. Returns the mean
+    milliseconds per stage and the stage outputs of the last pass."""
+    dev = inp["x"].device
+    T, d, E, k = cfg.T, cfg.d, cfg.E, cfg.k
+    rows = T * k
+    dt = cfg.torch_dtype
+    sh = cfg.f_shared > 0
+    o = dict(idx=torch.empty((T, k), dtype=torch.int32, device=dev),
+             gate=torch.empty((T, k), dtype=torch.float32, device=dev),
+             counts=torch.empty((E,), dtype=torch.int32, device=dev),
+             offsets=torch.empty((E + 1,), dtype=torch.int32, device=dev),
+             x_perm=torch.empty((rows, d), dtype=dt, device=dev),
+             perm_src=torch.empty((rows,), dtype=torch.int32, device=dev),
+             inv_row=torch.empty((T, k), dtype=torch.int32, device=dev),
+             h=torch.empty((rows, cfg.f), dtype=dt, device=dev),
+             h_s=torch.empty((T, cfg.f_shared), dtype=dt, device=dev) if sh else None,
+             y_perm=torch.empty((rows, d), dtype=dt, device=dev),
+             y_s=torch.empty((T, d), dtype=dt, device=dev) if sh else None,
+             y=torch.empty((T, d), dtype=dt, device=dev))
+    names = ["route", "permute", "gate_up", "down", "combine"]
+    calls = [
+        lambda: B.moe_route(cfg, inp["x"], inp["w_router"], inp["bias"], o["idx"], o["gate"], o["counts"],
+                            o["offsets"], ws),
+        lambda: B.moe_permute(cfg, inp["x"], o["idx"], o["offsets"], o["x_perm"], o["perm_src"], o["inv_row"], ws),
+        lambda: B.moe_expert_gate_up(cfg, o["x_perm"], o["offsets"], inp["w1"], inp["w3"], inp["x"] if sh else None,
+                                     inp["ws1"], inp["ws3"], o["h"], o["h_s"], ws),
+        lambda: B.moe_expert_down(cfg, o["h"], o["offsets"], inp["w2"], o["h_s"], inp["ws2"], o["y_perm"],
+                                  o["y_s"], ws),
+        lambda: B.moe_combine(cfg, o["y_perm"], o["inv_row"], o["gate"], o["y_s"], o["y"]),
+    ]
+    for _ in range(2):
+        for c in calls:
+            c()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(n)]
+    for i in range(n):
+        evs[i][0].record(stream)
+        for j, c in enumerate(calls):
+            c()
+            evs[i][j + 1].record(stream)
+    torch.cuda.synchronize()
+    assert B.moe_get_device_error(ws) == B.MOE_OK
+    stage_ms = {nm: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(n))
+                for j, nm in enumerate(names)}
+    return stage_ms, o
+
+
+def graph_step_ms(B, cfg, inp, ws, y, stream, steps, warmup):
+    """Milliseconds per moe_forward replayed from a CUDA graph, after warm-up."""
+    def fwd():
+        B.moe_forward(cfg, inp["x"], inp["w_router"], inp["bias"], inp["w1"], inp["w3"], inp["w2"],
+                      inp["ws1"], inp["ws3"], inp["ws2"], y, ws)
+
+    for _ in range(max(warmup, 3)):
+        fwd()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fwd()
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.time()
+    e0.record(stream)
+    for _ in range(steps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    del g
+    assert B.moe_get_device_error(ws) == B.MOE_OK
+    return e0.elapsed_time(e1) / steps, t0, t1
+
+
+def measure_workload(B, name, dev, stream, steps, warmup, sampler, peaks):
+    """One more workload of the pages, on its own inputs: the CUDA-graph step,
+    its stage times, and the fraction of the roof that binds it (HBM for the
+    weight-streaming shapes, the sustained tensor peak for the expert GEMMs of
+    the compute-bound ones), with the clock samples of its own timed region."""
+    from mixture_experts_ffn_sigmoid_b200.inputs import CONFIGS, make_inputs
+    cfg = CONFIGS[name]
+    inp = make_inputs(cfg, dev, seed=0)
+    ws = B.alloc_workspace(cfg, dev)
+    y = torch.empty((cfg.T, cfg.d), dtype=cfg.torch_dtype, device=dev)
+    ms, t0, t1 = graph_step_ms(B, cfg, inp, ws, y, stream, steps, warmup)
+    stage_ms, o = stage_breakdown(B, cfg, inp, ws, stream, max(3, min(steps, 50)))
+    assert torch.equal(o["y"], y), f"{name}: per-stage chain and moe_forward disagree"
+    work, touched = stage_work(cfg, o["counts"].cpu())
+    expert_ms = stage_ms["gate_up"] + stage_ms["down"]
+    expert_flops = work["gate_up"]["flops"] + work["down"]["flops"]
+    expert_bytes = work["gate_up"]["bytes"] + work["down"]["bytes"]
+    lb = layer_bytes(cfg, touched)
+    flops = cfg.active_flops()
+    r = {"config": {"T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k, "f": cfg.f, "f_shared": cfg.f_shared,
+                    "gate": "sigmoid" if cfg.gate_mode else "softmax", "n_groups": cfg.n_groups,
+                    "topk_groups": cfg.topk_groups, "route_scale": cfg.route_scale, "dtype": cfg.dtype},
+         "ms_per_step": ms, "steps": steps, "cuda_graph": True,
+         "tokens_per_s": cfg.T / (ms / 1e3), "active_tflops": flops / (ms / 1e3) / 1e12,
+         "experts_touched": touched, "stages_ms": stage_ms,
+         "layer_bytes": lb, "step_gbs": lb / (ms / 1e3) / 1e9,
+         "step_frac_hbm": lb / (ms / 1e3) / 1e9 / peaks["hbm"],
+         "expert_gemm": {"ms": expert_ms, "tflops": expert_flops / (expert_ms / 1e3) / 1e12,
+                         "frac_tensor_sustained": expert_flops / (expert_ms / 1e3) / 1e12 / peaks["tensor_sustained"],
+                         "gbs": expert_bytes / (expert_ms / 1e3) / 1e9,
+                         "frac_hbm": expert_bytes / (expert_ms / 1e3) / 1e9 / peaks["hbm"]},
+         "clocks": sampler.summary(t0, t1)}
+    hbm_t = lb / (peaks["hbm"] * 1e9)
+    tc_t = flops / (peaks["tensor_sustained"] * 1e12)
+    if cfg.dtype != "bf16":
+        r["binding_roof"] = "launch latency (parity-sized workload)"
+    elif tc_t > hbm_t:
+        r["binding_roof"] = "tensor"
+        r["binding_frac"] = r["expert_gemm"]["frac_tensor_sustained"]
+    else:
+        r["binding_roof"] = "hbm"
+        r["binding_frac"] = r["step_frac_hbm"]
+    del inp, ws, y, o
+    torch.cuda.empty_cache()
+    return r
+
+
 # ---------------------------------------------------------------- oracle arm
 def oracle_sample_time(cfg, inp, n_tokens, seed):
     """Run the CPU oracle on ``n_tokens`` seeded tokens; returns (seconds, threads)."""
@@ -577,50 +711,17 @@ def main():
     ms_step = ms_total / args.steps
     value = whole_job_rate(T, world, ms_step)
     assert B.moe_get_device_error(ws) == B.MOE_OK
-    sampler.stop()
     clocks = sampler.summary(t_wall0, t_wall1)
 
     # ---- stage breakdown: the same kernels through the per-stage entry points,
     # one CUDA event between stages on the launching stream ----------------------
     k, E = cfg.k, cfg.E
-    rows = T * k
-    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
-    gate = torch.empty((T, k), dtype=torch.float32, device=dev)
-    counts = torch.empty((E,), dtype=torch.int32, device=dev)
-    offsets = torch.empty((E + 1,), dtype=torch.int32, device=dev)
-    x_perm = torch.empty((rows, d), dtype=cfg.torch_dtype, device=dev)
-    perm_src = torch.empty((rows,), dtype=torch.int32, device=dev)
-    inv_row = torch.empty((T, k), dtype=torch.int32, device=dev)
-    h = torch.empty((rows, cfg.f), dtype=cfg.torch_dtype, device=dev)
-    sh = cfg.f_shared > 0
-    h_s = torch.empty((T, cfg.f_shared), dtype=cfg.torch_dtype, device=dev) if sh else None
-    y_perm = torch.empty((rows, d), dtype=cfg.torch_dtype, device=dev)
-    y_s = torch.empty((T, d), dtype=cfg.torch_dtype, device=dev) if sh else None
-    y2 = torch.empty_like(y)
-    names = ["route", "permute", "gate_up", "down", "combine"]
-    calls = [
-        lambda: B.moe_route(cfg, inp["x"], inp["w_router"], inp["bias"], idx, gate, counts, offsets, ws),
-        lambda: B.moe_permute(cfg, inp["x"], idx, offsets, x_perm, perm_src, inv_row, ws),
-        lambda: B.moe_expert_gate_up(cfg, x_perm, offsets, inp["w1"], inp["w3"], inp["x"] if sh else None,
-                                     inp["ws1"], inp["ws3"], h, h_s, ws),
-        lambda: B.moe_expert_down(cfg, h, offsets, inp["w2"], h_s, inp["ws2"], y_perm, y_s, ws),
-        lambda: B.moe_combine(cfg, y_perm, inv_row, gate, y_s, y2),
-    ]
-    for _ in range(2):
-        for c in calls:
-            c()
-    torch.cuda.synchronize()
     n_stage = max(3, min(args.steps, 50))
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(n_stage)]
-    for i in range(n_stage):
-        evs[i][0].record(stream)
-        for j, c in enumerate(calls):
-            c()
-            evs[i][j + 1].record(stream)
-    torch.cuda.synchronize()
-    stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(n_stage))
-                for j, n in enumerate(names)}
-    assert torch.equal(y2, y), "per-stage chain and moe_forward disagree"
+    names = ["route", "permute", "gate_up", "down", "combine"]
+    stage_ms, so = stage_breakdown(B, cfg, inp, ws, stream, n_stage)
+    idx, gate, counts, offsets = so["idx"], so["gate"], so["counts"], so["offsets"]
+    perm_src, inv_row, h, h_s = so["perm_src"], so["inv_row"], so["h"], so["h_s"]
+    assert torch.equal(so["y"], y), "per-stage chain and moe_forward disagree"
     fused = measure_fused_permute(B, cfg, inp, idx, offsets, perm_src, inv_row, h, h_s, ws, stream,
                                   n_stage) if cfg.dtype == "bf16" else None
     if fused is not None:
@@ -734,6 +835,20 @@ def main():
                "sample": f"{n} seeded tokens of {cfg.name}: fp64 routing over all {E} experts and the "
                          f"FFN of each selected and shared expert ({dt:.1f} s)"}
 
+    # ---- the pages' other workloads (one GPU only): each on its own inputs,
+    # CUDA-graph step, stage times, binding-roof fraction, its own clocks -------
+    extra = None
+    if world == 1 and not args.no_extra_workloads and args.T is None and args.E is None:
+        from mixture_experts_ffn_sigmoid_b200.inputs import CONFIGS
+        del x_host, y_host, x_dev, y_dev
+        torch.cuda.empty_cache()
+        extra = {}
+        for name in CONFIGS:
+            if name != cfg.name:
+                extra[name] = measure_workload(B, name, dev, stream, max(3, min(args.steps, 50)), args.warmup,
+                                               sampler, peaks)
+    sampler.stop()
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -762,6 +877,7 @@ def main():
             "e2e": {"value": whole_job_rate(T, world, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": T * d * cfg.elem_bytes, "d2h_bytes_per_step": T * d * cfg.elem_bytes,
                     "ms_per_step": e2e_ms},
+            "workloads": extra,
             "gpu_launches": KERNELS_PER_FORWARD * args.steps,
             "clocks": clocks,
         }

@@ -133,5 +133,15 @@ def test_non_finite_token_gets_valid_expert_ids(name, bad):
     assert np.array_equal(got["offsets"].cpu().numpy(), o)
     others = np.arange(cfg.T) != 5
     assert np.array_equal(gi[others], clean["idx"].cpu().numpy()[others])
-    assert torch.equal(got["gate"][torch.as_tensor(others, device="cuda")],
-                       clean["gate"][torch.as_tensor(others, device="cuda")])
+    keep = torch.as_tensor(others, device="cuda")
+    assert torch.equal(got["gate"][keep], clean["gate"][keep])
+    # The whole block: the bad row stays in its own outputs. Every other
+    # token's output is finite and bitwise that of the clean input (each output
+    # element is one token row's dot products, whatever the packing).
+    y_bad = H.gpu_forward(cfg, inp)
+    x_clean = inp["x"].clone()
+    x_clean[5] = H.gpu_inputs(cfg)["x"][5]
+    inp["x"] = x_clean
+    y_clean = H.gpu_forward(cfg, inp)
+    assert torch.isfinite(y_bad[keep].float()).all().item()
+    assert torch.equal(y_bad[keep], y_clean[keep])
