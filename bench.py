@@ -45,7 +45,12 @@ sys.path.insert(0, ROOT)
 import torch  # noqa: E402
 
 METRIC = "MoE-layer tokens/s and active TFLOP/s at DeepSeek-V3 shape; % bf16 / HBM roofline"
-KERNELS_PER_FORWARD = 8   # router GEMM, top-k, chunk scan, offsets, permute, gate/up, down, combine
+def kernels_per_forward(cfg) -> int:
+    """Kernel launches of one moe_forward: the fused router (bf16, E <= 256)
+    or router GEMM + top-k + chunk scan + offsets, then permute, gate/up,
+    down and combine."""
+    fused = cfg.dtype == "bf16" and cfg.E <= 256
+    return (1 if fused else 4) + 4
 CPU_SAMPLE_TOKENS = {"tiny_fp32": 64, "decode_fine": 32, "deepseek_v3": 16, "mixtral_8x7b": 8,
                      "deepseek_v3_skewed": 64}
 REF_STEP_TOKENS = {"tiny_fp32": 64, "decode_fine": 8, "deepseek_v3": 2, "mixtral_8x7b": 2,
@@ -63,6 +68,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--T", type=int, default=None, help="override the token count (profiling cases)")
     ap.add_argument("--E", type=int, default=None, help="override the routed expert count (profiling cases)")
+    ap.add_argument("--f", type=int, default=None, help="override the expert inner width (profiling cases)")
+    ap.add_argument("--forward-only", action="store_true",
+                    help="stop after the timed forward steps and the stage breakdown (profiling runs)")
     ap.add_argument("--no-extra-workloads", action="store_true",
                     help="time the headline workload only (the others run at N=1 by default)")
     return ap.parse_args()
@@ -71,9 +79,11 @@ def parse_args():
 def workload(args):
     from mixture_experts_ffn_sigmoid_b200.inputs import CONFIGS
     cfg = CONFIGS[args.config]
-    if args.T is not None or args.E is not None:
-        cfg = cfg.with_(T=args.T or cfg.T, E=args.E or cfg.E,
-                        name=f"{cfg.name}_T{args.T or cfg.T}_E{args.E or cfg.E}")
+    if args.T is not None or args.E is not None or args.f is not None:
+        f = args.f or cfg.f
+        cfg = cfg.with_(T=args.T or cfg.T, E=args.E or cfg.E, f=f,
+                        f_shared=(f if cfg.f_shared else 0),
+                        name=f"{cfg.name}_T{args.T or cfg.T}_E{args.E or cfg.E}" + (f"_f{f}" if args.f else ""))
     return cfg
 
 
@@ -234,7 +244,9 @@ def stage_work(cfg, counts):
     touched = int((counts > 0).sum())
     rows, srows = T * k, (T if fs else 0)
     w = {}
-    w["route"] = dict(bytes=(T * d + E * d) * es + T * k * 8 + T * E * 4 * 2, flops=2.0 * T * E * d)
+    # route: x and the router read, the summed fp32 logits written once (kept
+    # for the backward pass), indices and gates written.
+    w["route"] = dict(bytes=(T * d + E * d) * es + T * k * 8 + T * E * 4, flops=2.0 * T * E * d)
     w["permute"] = dict(bytes=(T * d + rows * d) * es + rows * 8 + T * k * 4, flops=0.0)
     w["gate_up"] = dict(bytes=(touched * 2 * f * d + 2 * fs * d) * es + (rows * d + srows * d) * es
                         + (rows * f + srows * fs) * es,
@@ -722,6 +734,16 @@ def main():
     idx, gate, counts, offsets = so["idx"], so["gate"], so["counts"], so["offsets"]
     perm_src, inv_row, h, h_s = so["perm_src"], so["inv_row"], so["h"], so["h_s"]
     assert torch.equal(so["y"], y), "per-stage chain and moe_forward disagree"
+    if args.forward_only:
+        sampler.stop()
+        if rank == 0:
+            print(json.dumps({"profiling_run": cfg.name, "ms_per_step": ms_step, "stages_ms": stage_ms,
+                              "clocks": clocks}), flush=True)
+        if graph is not None:
+            del graph
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
     fused = measure_fused_permute(B, cfg, inp, idx, offsets, perm_src, inv_row, h, h_s, ws, stream,
                                   n_stage) if cfg.dtype == "bf16" else None
     if fused is not None:
@@ -838,7 +860,7 @@ def main():
     # ---- the pages' other workloads (one GPU only): each on its own inputs,
     # CUDA-graph step, stage times, binding-roof fraction, its own clocks -------
     extra = None
-    if world == 1 and not args.no_extra_workloads and args.T is None and args.E is None:
+    if world == 1 and not args.no_extra_workloads and args.T is None and args.E is None and args.f is None:
         from mixture_experts_ffn_sigmoid_b200.inputs import CONFIGS
         del x_host, y_host, x_dev, y_dev
         torch.cuda.empty_cache()
@@ -878,7 +900,7 @@ def main():
                     "h2d_bytes_per_step": T * d * cfg.elem_bytes, "d2h_bytes_per_step": T * d * cfg.elem_bytes,
                     "ms_per_step": e2e_ms},
             "workloads": extra,
-            "gpu_launches": KERNELS_PER_FORWARD * args.steps,
+            "gpu_launches": kernels_per_forward(cfg) * args.steps,
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

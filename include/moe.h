@@ -68,7 +68,11 @@
  *    exception crosses this interface.
  *  - Device-side waits are bounded (about 2 s). A wait that runs out records
  *    MOE_ERR_TIMEOUT in the workspace's error word and its kernel returns;
- *    moe_get_device_error() reports it.
+ *    moe_get_device_error() reports it. Caller-supplied indices (topk_idx,
+ *    expert_offsets, inv_row) are bounds-checked on the device: out-of-range
+ *    values are skipped or clamped, never dereferenced, and flagged in the
+ *    same word where the call has one (moe_combine has none: it skips a
+ *    row past T*k silently).
  */
 #ifndef MOE_B200_H_
 #define MOE_B200_H_
@@ -151,7 +155,9 @@ MOE_API size_t moe_workspace_size(const moe_config* cfg);
  * or s = logit (MOE_GATE_SOFTMAX). With n_groups > 1, group G = experts
  * [G*E/n_groups, (G+1)*E/n_groups) scores the sum of its two largest b';
  * only the topk_groups best groups stay eligible. Then the k largest
- * eligible b' win.
+ * eligible b' win. For bf16 with E <= 256 the whole call is one kernel (the
+ * router logits never leave the chip as partial sums); the workspace keeps
+ * the summed logits [T][E] fp32 either way.
  */
 MOE_API moe_status moe_route(const moe_config* cfg, const void* x, const void* w_router,
                      const float* bias, int32_t* topk_idx, float* topk_gate,
@@ -384,11 +390,13 @@ MOE_API moe_status moe_backward_saved(const moe_config* cfg, const void* x, cons
  * and bases, error word) is one fixed 24 MiB array in the library's device
  * image, present on every GPU that loads the library until the process
  * exits; the call itself allocates nothing.
- *  - Capacity: the call needs 256 + 4*S*T*E + 8*E*ceil(T/32) bytes (each term
- *    rounded up to 256), where S is the number of router partial sums: 1 for
- *    fp32; for bf16, S = min(8, ceil(d/64), max(1, floor(148 / (ceil(T/128) *
- *    ceil(E/256))))). Beyond 24 MiB it returns MOE_ERR_WORKSPACE_TOO_SMALL
- *    before enqueuing anything.
+ *  - Capacity: the call needs 256 + 4*S*T*E + 8*E*ceil(T/32) + 8*E*ceil(T/128)
+ *    bytes (each term rounded up to 256), where S is the number of router
+ *    partial sums kept in memory: 1 for fp32 and for bf16 with E <= 256 (one
+ *    fused kernel adds the partial sums on chip); for bf16 with more experts,
+ *    S = min(8, ceil(d/64), max(1, floor(148 / (ceil(T/128) * ceil(E/256))))).
+ *    Beyond 24 MiB it returns MOE_ERR_WORKSPACE_TOO_SMALL before enqueuing
+ *    anything.
  *  - The first call on each device looks up the array's device address
  *    (with that device current) and caches it; make that first call before
  *    any stream capture on the device.
@@ -438,8 +446,13 @@ MOE_API moe_status moe_balance_update(const moe_config* cfg, const int32_t* expe
 
 /* Synchronises `stream`, reads and clears the workspace's device error word.
  * Returns MOE_OK, MOE_ERR_TIMEOUT (a bounded device wait ran out during an
- * earlier call on this workspace) or MOE_ERR_CUDA. Every entry point that
- * takes a workspace clears the word when it starts. */
+ * earlier call on this workspace), MOE_ERR_INVALID_ARG (a device-side check
+ * found a caller index out of range: an expert id outside [0, E) or a
+ * packed row outside [0, T*k) in moe_permute, or an expert_offsets entry
+ * outside [0, T*k) or below its predecessor in the expert calls; such ids
+ * and rows are skipped and such offsets clamped, so no access leaves the
+ * caller's buffers, but the outputs are not defined) or MOE_ERR_CUDA. Every
+ * entry point that takes a workspace clears the word when it starts. */
 MOE_API moe_status moe_get_device_error(void* workspace, void* stream);
 
 /* Launches one kernel that waits on a barrier nothing ever arrives at,

@@ -4,6 +4,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -23,10 +25,27 @@ namespace {
 
 constexpr size_t kAlign = 256;
 
+// A named NVTX range over the host-side enqueue of an entry point or stage,
+// for timeline tools (a no-op unless one is attached).
+struct TraceRange {
+  explicit TraceRange(const char* name) { nvtxRangePushA(name); }
+  ~TraceRange() { nvtxRangePop(); }
+  TraceRange(const TraceRange&) = delete;
+  TraceRange& operator=(const TraceRange&) = delete;
+};
+
 struct Layout {
-  size_t err, logits, ccount, cbase, idx, gate, counts, offsets, inv_row, perm_src;
+  size_t err, logits, ccount, cbase, thist, tbase, idx, gate, counts, offsets, inv_row, perm_src;
   size_t x_perm, h, h_s, y_perm, y_s, total;
 };
+
+// Byte offset, inside the error region (cleared at the start of every call),
+// of the fused router's device-wide tile counter.
+constexpr size_t kDoneCountOffset = 64;
+
+// The bf16 router of up to 256 experts runs as one fused kernel; otherwise
+// a GEMM (split contraction for bf16) feeds the separate top-k and scans.
+bool fused_route(const moe_config& c) { return router_fused_supported(c.dtype, c.E); }
 
 // Workspace regions, each 256-byte aligned. Sizes cover the worst case of
 // T*k packed rows plus T shared rows.
@@ -43,11 +62,15 @@ Layout layout_of(const moe_config& c) {
   const size_t fs = (size_t)c.f_shared;
   const size_t nch = (T + kChunk - 1) / kChunk;
   L.err = take(kAlign);
-  // bf16 router logits come as partial sums of a split contraction.
-  const size_t n_part = c.dtype == MOE_DTYPE_BF16 ? (size_t)router_gemm_splits(c.T, c.E, c.d) : 1;
+  // Unfused bf16 router logits come as partial sums of a split contraction.
+  const size_t n_part =
+      (c.dtype == MOE_DTYPE_BF16 && !fused_route(c)) ? (size_t)router_gemm_splits(c.T, c.E, c.d) : 1;
+  const size_t ntiles = (T + (size_t)(kChunk * kTileChunks) - 1) / (kChunk * kTileChunks);
   L.logits = take(n_part * T * E * 4);
   L.ccount = take(nch * E * 4);
   L.cbase = take(nch * E * 4);
+  L.thist = take(ntiles * E * 4);
+  L.tbase = take(ntiles * E * 4);
   L.idx = take(T * k * 4);
   L.gate = take(T * k * 4);
   L.counts = take(E * 4);
@@ -122,6 +145,14 @@ moe_status enqueue_route(const moe_config& c, const void* x, const void* w_route
                          int* idx, float* gate, int* counts, int* offsets, void* ws, cudaStream_t s) {
   const Layout L = layout_of(c);
   float* logits = at<float>(ws, L.logits);
+  const TopkArgs tk = {c.E, c.k, c.gate_mode, c.n_groups, c.topk_groups, c.route_scale, bias};
+  if (fused_route(c)) {
+    const FusedRouterLaunch a = {x, w_router, c.T, c.E, c.d, tk, logits, idx, gate, at<int>(ws, L.cbase),
+                                 at<int>(ws, L.thist), at<int>(ws, L.tbase), counts, offsets,
+                                 at<uint32_t>(ws, L.err), at<uint32_t>(ws, L.err + kDoneCountOffset)};
+    MOE_CUDA(launch_router_fused(a, s));
+    return MOE_OK;
+  }
   int n_part = 1;
   if (c.dtype == MOE_DTYPE_BF16) {
     n_part = router_gemm_splits(c.T, c.E, c.d);
@@ -150,6 +181,13 @@ moe_status enqueue_route(const moe_config& c, const void* x, const void* w_route
   MOE_CUDA(launch_chunk_scan(at<int>(ws, L.ccount), nch, c.E, at<int>(ws, L.cbase), counts, s));
   MOE_CUDA(launch_offsets(counts, c.E, offsets, s));
   return MOE_OK;
+}
+
+// Tile bases to add to the chunk bases enqueue_route left in the workspace
+// (the fused router's chunk bases count from the start of their tile), or
+// null when the chunk bases are already global.
+const int* route_tile_base(const moe_config& c, void* ws) {
+  return fused_route(c) ? at<int>(ws, layout_of(c).tbase) : nullptr;
 }
 
 // Token-tile width of the expert GEMMs. Weight bytes dominate: every token
@@ -218,6 +256,7 @@ moe_status enqueue_gate_up(const moe_config& c, const void* x_perm, const int* o
     g.a_s = x_sh; g.b1_s = ws1; g.b3_s = ws3; g.out_s = h_s;
     g.N_s = c.f_shared; g.K_s = c.d;
     g.max_rows = rows;
+    g.err = err;
     if (pre) { g.pre_a = pre[0]; g.pre_b = pre[1]; g.pre_a_s = pre[2]; g.pre_b_s = pre[3]; }
     MOE_CUDA(launch_simt_gemm(c.dtype, 0, g, s));
   }
@@ -263,6 +302,7 @@ moe_status enqueue_down(const moe_config& c, const void* h, const int* offsets, 
     q.a_s = h_s; q.b1_s = ws2; q.out_s = y_sh;
     q.N_s = c.d; q.K_s = c.f_shared;
     q.max_rows = rows;
+    q.err = err;
     MOE_CUDA(launch_simt_gemm(c.dtype, 0, q, s));
   }
   return MOE_OK;
@@ -324,6 +364,7 @@ moe_status enqueue_gelu_experts(const moe_config& c, const void* x_perm, const i
     g.a = x_perm; g.b1 = w1; g.out = h;
     g.N = c.f; g.K = c.d;
     g.max_rows = rows;
+    g.err = err;
     g.bias1 = b1;
     g.act = kActGelu;
     MOE_CUDA(launch_simt_gemm(c.dtype, 0, g, s));
@@ -513,13 +554,13 @@ moe_status enqueue_backward(const moe_config& c, const void* x, const void* w_ro
   // Forward state: routing, packed x, pre-activations; then packed dy.
   if (recompute) {
     MOE_TRY(enqueue_route(c, x, w_router, bias, idx, gate, at<int>(ws, L.counts), offsets, ws, s));
-    MOE_CUDA(launch_permute(c.dtype, x, idx, offsets, at<int>(ws, L.cbase), c.T, c.d, c.E, c.k, x_perm,
-                            perm_src, inv_row, nsm, s, true));
+    MOE_CUDA(launch_permute(c.dtype, x, idx, offsets, at<int>(ws, L.cbase), route_tile_base(c, ws), c.T, c.d,
+                            c.E, c.k, x_perm, perm_src, inv_row, nsm, s, true, err));
     MOE_TRY(enqueue_preact(c, x_perm, offsets, x, w1, w3, ws1, ws3, at<char>(ws, Bw.a), at<char>(ws, Bw.b),
                            at<char>(ws, Bw.a_s), at<char>(ws, Bw.b_s), err, s));
   }
-  MOE_CUDA(launch_permute(c.dtype, dy, idx, offsets, at<int>(ws, L.cbase), c.T, c.d, c.E, c.k, dyp,
-                          perm_src, inv_row, nsm, s, true));
+  MOE_CUDA(launch_permute(c.dtype, dy, idx, offsets, at<int>(ws, L.cbase), route_tile_base(c, ws), c.T, c.d,
+                          c.E, c.k, dyp, perm_src, inv_row, nsm, s, true, err));
   // dh' = W2^T dy per packed row (gate not applied), and the shared expert's.
   const bool tc = c.dtype == MOE_DTYPE_BF16;
   constexpr int kNoSplit = 1 << 30;
@@ -706,6 +747,7 @@ size_t moe_workspace_size(const moe_config* cfg) {
 moe_status moe_route(const moe_config* cfg, const void* x, const void* w_router, const float* bias,
                      int32_t* topk_idx, float* topk_gate, int32_t* expert_counts,
                      int32_t* expert_offsets, void* workspace, size_t ws_bytes, void* stream) {
+  TraceRange trace("moe_route");
   MOE_TRY(check_config(cfg));
   const moe_config& c = *cfg;
   MOE_TRY(need4(expert_counts));
@@ -730,6 +772,7 @@ moe_status moe_route(const moe_config* cfg, const void* x, const void* w_router,
 moe_status moe_permute(const moe_config* cfg, const void* x, const int32_t* topk_idx,
                        const int32_t* expert_offsets, void* x_perm, int32_t* perm_src,
                        int32_t* inv_row, void* workspace, size_t ws_bytes, void* stream) {
+  TraceRange trace("moe_permute");
   MOE_TRY(check_config(cfg));
   const moe_config& c = *cfg;
   MOE_TRY(check_ws(c, workspace, ws_bytes));
@@ -750,8 +793,9 @@ moe_status moe_permute(const moe_config* cfg, const void* x, const int32_t* topk
   MOE_CUDA(launch_chunk_counts(topk_idx, c.T, c.k, c.E, at<int>(workspace, L.ccount), s));
   MOE_CUDA(launch_chunk_scan(at<int>(workspace, L.ccount), nch, c.E, at<int>(workspace, L.cbase),
                              at<int>(workspace, L.counts), s));
-  MOE_CUDA(launch_permute(c.dtype, x, topk_idx, expert_offsets, at<int>(workspace, L.cbase), c.T, c.d,
-                          c.E, c.k, x_perm, perm_src, inv_row, device_sm_count(), s, copy));
+  MOE_CUDA(launch_permute(c.dtype, x, topk_idx, expert_offsets, at<int>(workspace, L.cbase), nullptr, c.T,
+                          c.d, c.E, c.k, x_perm, perm_src, inv_row, device_sm_count(), s, copy,
+                          at<uint32_t>(workspace, L.err)));
   return MOE_OK;
 }
 
@@ -759,6 +803,7 @@ moe_status moe_expert_swiglu(const moe_config* cfg, const void* x_perm, const in
                              const void* w1, const void* w3, const void* w2, const void* x_shared,
                              const void* ws1, const void* ws3, const void* ws2, void* y_perm,
                              void* y_shared, void* workspace, size_t ws_bytes, void* stream) {
+  TraceRange trace("moe_expert_swiglu");
   MOE_TRY(check_config(cfg));
   const moe_config& c = *cfg;
   MOE_TRY(check_ws(c, workspace, ws_bytes));
@@ -786,6 +831,7 @@ moe_status moe_expert_gate_up(const moe_config* cfg, const void* x_perm, const i
                               const void* w1, const void* w3, const void* x_shared, const void* ws1,
                               const void* ws3, void* h, void* h_shared, void* workspace,
                               size_t ws_bytes, void* stream) {
+  TraceRange trace("moe_expert_gate_up");
   MOE_TRY(check_config(cfg));
   const moe_config& c = *cfg;
   MOE_TRY(check_ws(c, workspace, ws_bytes));
@@ -811,6 +857,7 @@ moe_status moe_expert_gate_up_gather(const moe_config* cfg, const void* x, const
                                      const int32_t* expert_offsets, const void* w1, const void* w3,
                                      const void* ws1, const void* ws3, void* h, void* h_shared,
                                      void* workspace, size_t ws_bytes, void* stream) {
+  TraceRange trace("moe_expert_gate_up_gather");
   MOE_TRY(check_config(cfg));
   const moe_config& c = *cfg;
   if (c.dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
@@ -840,6 +887,7 @@ moe_status moe_expert_gate_up_gather(const moe_config* cfg, const void* x, const
 moe_status moe_expert_down(const moe_config* cfg, const void* h, const int32_t* expert_offsets,
                            const void* w2, const void* h_shared, const void* ws2, void* y_perm,
                            void* y_shared, void* workspace, size_t ws_bytes, void* stream) {
+  TraceRange trace("moe_expert_down");
   MOE_TRY(check_config(cfg));
   const moe_config& c = *cfg;
   MOE_TRY(check_ws(c, workspace, ws_bytes));
@@ -861,6 +909,7 @@ moe_status moe_expert_down(const moe_config* cfg, const void* h, const int32_t* 
 
 moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t* inv_row,
                        const float* topk_gate, const void* y_shared, void* y, void* stream) {
+  TraceRange trace("moe_combine");
   MOE_TRY(check_config(cfg));
   const moe_config& c = *cfg;
   if (c.T == 0) return MOE_OK;
@@ -878,6 +927,7 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
                        const void* w1, const void* w3, const void* w2, const void* ws1,
                        const void* ws3, const void* ws2, void* y, void* workspace, size_t ws_bytes,
                        void* stream) {
+  TraceRange trace("moe_forward");
   MOE_TRY(check_config(cfg));
   const moe_config& c = *cfg;
   MOE_TRY(check_ws(c, workspace, ws_bytes));
@@ -901,18 +951,28 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
   int* idx = at<int>(ws, L.idx);
   float* gate = at<float>(ws, L.gate);
   int* offsets = at<int>(ws, L.offsets);
-  MOE_TRY(enqueue_route(c, x, w_router, bias, idx, gate, at<int>(ws, L.counts), offsets, ws, s));
+  {
+    TraceRange stage("moe_forward.route");
+    MOE_TRY(enqueue_route(c, x, w_router, bias, idx, gate, at<int>(ws, L.counts), offsets, ws, s));
+  }
   // Packed copy of the token rows, then GEMMs over contiguous segments. (The
   // gate/up GEMM can instead gather rows from x with TMA gather4, see
   // moe_expert_gate_up_gather; on B200 that costs more GEMM time than the
   // copy it saves, so the block uses the packed copy.)
-  MOE_CUDA(launch_permute(c.dtype, x, idx, offsets, at<int>(ws, L.cbase), c.T, c.d, c.E, c.k,
-                          at<char>(ws, L.x_perm), at<int>(ws, L.perm_src), at<int>(ws, L.inv_row),
-                          device_sm_count(), s, true));
+  {
+    TraceRange stage("moe_forward.permute");
+    MOE_CUDA(launch_permute(c.dtype, x, idx, offsets, at<int>(ws, L.cbase), route_tile_base(c, ws), c.T, c.d,
+                            c.E, c.k, at<char>(ws, L.x_perm), at<int>(ws, L.perm_src), at<int>(ws, L.inv_row),
+                            device_sm_count(), s, true, at<uint32_t>(ws, L.err)));
+  }
   const bool shared = c.f_shared > 0;
   void* y_s = shared ? at<char>(ws, L.y_s) : nullptr;
-  MOE_TRY(enqueue_experts(c, at<char>(ws, L.x_perm), offsets, w1, w3, w2, shared ? x : nullptr, ws1,
-                          ws3, ws2, at<char>(ws, L.y_perm), y_s, ws, s));
+  {
+    TraceRange stage("moe_forward.experts");
+    MOE_TRY(enqueue_experts(c, at<char>(ws, L.x_perm), offsets, w1, w3, w2, shared ? x : nullptr, ws1,
+                            ws3, ws2, at<char>(ws, L.y_perm), y_s, ws, s));
+  }
+  TraceRange stage("moe_forward.combine");
   MOE_CUDA(launch_combine(c.dtype, at<char>(ws, L.y_perm), at<int>(ws, L.inv_row), gate, y_s, y, c.T,
                           c.d, c.k, device_sm_count(), s));
   return MOE_OK;
@@ -921,6 +981,7 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
 moe_status moe_expert_gelu(const moe_config* cfg, const void* x_perm, const int32_t* expert_offsets,
                            const void* w1, const float* b1, const void* w2, const float* b2,
                            void* y_perm, void* workspace, size_t ws_bytes, void* stream) {
+  TraceRange trace("moe_expert_gelu");
   MOE_TRY(check_config(cfg));
   const moe_config& c = *cfg;
   if (c.f_shared > 0) return MOE_ERR_UNSUPPORTED;
@@ -942,6 +1003,7 @@ moe_status moe_forward_gelu(const moe_config* cfg, const void* x, const void* w_
                             const float* bias, const void* w1, const float* b1, const void* w2,
                             const float* b2, void* y, void* workspace, size_t ws_bytes,
                             void* stream) {
+  TraceRange trace("moe_forward_gelu");
   MOE_TRY(check_config(cfg));
   const moe_config& c = *cfg;
   if (c.f_shared > 0) return MOE_ERR_UNSUPPORTED;
@@ -963,9 +1025,9 @@ moe_status moe_forward_gelu(const moe_config* cfg, const void* x, const void* w_
   float* gate = at<float>(ws, L.gate);
   int* offsets = at<int>(ws, L.offsets);
   MOE_TRY(enqueue_route(c, x, w_router, bias, idx, gate, at<int>(ws, L.counts), offsets, ws, s));
-  MOE_CUDA(launch_permute(c.dtype, x, idx, offsets, at<int>(ws, L.cbase), c.T, c.d, c.E, c.k,
-                          at<char>(ws, L.x_perm), at<int>(ws, L.perm_src), at<int>(ws, L.inv_row),
-                          device_sm_count(), s, true));
+  MOE_CUDA(launch_permute(c.dtype, x, idx, offsets, at<int>(ws, L.cbase), route_tile_base(c, ws), c.T, c.d,
+                          c.E, c.k, at<char>(ws, L.x_perm), at<int>(ws, L.perm_src), at<int>(ws, L.inv_row),
+                          device_sm_count(), s, true, at<uint32_t>(ws, L.err)));
   MOE_TRY(enqueue_gelu_experts(c, at<char>(ws, L.x_perm), offsets, w1, b1, w2, b2,
                                at<char>(ws, L.y_perm), ws, s));
   MOE_CUDA(launch_combine(c.dtype, at<char>(ws, L.y_perm), at<int>(ws, L.inv_row), gate, nullptr, y,
@@ -1032,6 +1094,7 @@ moe_status moe_backward(const moe_config* cfg, const void* x, const void* w_rout
                         const void* ws2, const void* dy, void* dx, void* dw_router, void* dw1, void* dw3,
                         void* dw2, void* dws1, void* dws3, void* dws2, void* workspace, size_t ws_bytes,
                         void* stream) {
+  TraceRange trace("moe_backward");
   return backward_entry(cfg, x, w_router, bias, w1, w3, w2, ws1, ws3, ws2, dy, dx, dw_router, dw1, dw3, dw2,
                         dws1, dws3, dws2, workspace, ws_bytes, stream, true);
 }
@@ -1041,6 +1104,7 @@ moe_status moe_backward_saved(const moe_config* cfg, const void* x, const void* 
                               const void* ws2, const void* dy, void* dx, void* dw_router, void* dw1,
                               void* dw3, void* dw2, void* dws1, void* dws3, void* dws2, void* workspace,
                               size_t ws_bytes, void* stream) {
+  TraceRange trace("moe_backward_saved");
   return backward_entry(cfg, x, w_router, nullptr, w1, w3, w2, ws1, ws3, ws2, dy, dx, dw_router, dw1, dw3,
                         dw2, dws1, dws3, dws2, workspace, ws_bytes, stream, false);
 }
@@ -1049,6 +1113,7 @@ moe_status moe_forward_train(const moe_config* cfg, const void* x, const void* w
                              const void* w1, const void* w3, const void* w2, const void* ws1,
                              const void* ws3, const void* ws2, void* y, void* workspace, size_t ws_bytes,
                              void* stream) {
+  TraceRange trace("moe_forward_train");
   MOE_TRY(check_config(cfg));
   const moe_config& c = *cfg;
   MOE_TRY(need(workspace));
@@ -1075,9 +1140,9 @@ moe_status moe_forward_train(const moe_config* cfg, const void* x, const void* w
   float* gate = at<float>(ws, L.gate);
   int* offsets = at<int>(ws, L.offsets);
   MOE_TRY(enqueue_route(c, x, w_router, bias, idx, gate, at<int>(ws, L.counts), offsets, ws, s));
-  MOE_CUDA(launch_permute(c.dtype, x, idx, offsets, at<int>(ws, L.cbase), c.T, c.d, c.E, c.k,
-                          at<char>(ws, L.x_perm), at<int>(ws, L.perm_src), at<int>(ws, L.inv_row),
-                          device_sm_count(), s, true));
+  MOE_CUDA(launch_permute(c.dtype, x, idx, offsets, at<int>(ws, L.cbase), route_tile_base(c, ws), c.T, c.d,
+                          c.E, c.k, at<char>(ws, L.x_perm), at<int>(ws, L.perm_src), at<int>(ws, L.inv_row),
+                          device_sm_count(), s, true, at<uint32_t>(ws, L.err)));
   const bool shared = c.f_shared > 0;
   void* y_s = shared ? at<char>(ws, L.y_s) : nullptr;
   void* pre[4] = {at<char>(ws, Bw.a), at<char>(ws, Bw.b), shared ? at<char>(ws, Bw.a_s) : nullptr,
@@ -1091,6 +1156,7 @@ moe_status moe_forward_train(const moe_config* cfg, const void* x, const void* w
 
 moe_status moe_balance_update(const moe_config* cfg, const int32_t* expert_counts, float* bias,
                               float gamma, float* entropy, void* stream) {
+  TraceRange trace("moe_balance_update");
   MOE_TRY(check_config(cfg));
   const moe_config& c = *cfg;
   MOE_TRY(need4(expert_counts));
@@ -1112,6 +1178,7 @@ moe_status moe_get_device_error(void* workspace, void* stream) {
     return MOE_ERR_CUDA;
   if (cudaMemset(workspace, 0, sizeof(word)) != cudaSuccess) return MOE_ERR_CUDA;
   if (word & kErrTimeoutWait) return MOE_ERR_TIMEOUT;
+  if (word & kErrBadIndex) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 
@@ -1185,6 +1252,7 @@ extern "C" moe_status moe_route_noalloc(const moe_config* cfg, const void* x, co
                                         const float* bias, int32_t* topk_idx, float* topk_gate,
                                         int32_t* expert_counts, int32_t* expert_offsets,
                                         void* stream) {
+  TraceRange trace("moe_route_noalloc");
   MOE_TRY(check_config(cfg));
   const moe_config& c = *cfg;
   MOE_TRY(need4(expert_counts));
@@ -1221,5 +1289,6 @@ extern "C" moe_status moe_route_noalloc_device_error(void* stream) {
   MOE_CUDA(cudaMemcpyAsync(&word, scratch, sizeof(word), cudaMemcpyDeviceToHost, s));
   MOE_CUDA(cudaMemsetAsync(scratch, 0, sizeof(word), s));
   MOE_CUDA(cudaStreamSynchronize(s));
-  return (word & kErrTimeoutWait) ? MOE_ERR_TIMEOUT : MOE_OK;
+  if (word & kErrTimeoutWait) return MOE_ERR_TIMEOUT;
+  return (word & kErrBadIndex) ? MOE_ERR_INVALID_ARG : MOE_OK;
 }

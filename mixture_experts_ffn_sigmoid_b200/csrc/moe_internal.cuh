@@ -10,6 +10,7 @@
 namespace moe {
 
 constexpr int kChunk = 32;            // tokens per routing chunk (one warp's worth)
+constexpr int kTileChunks = 4;        // chunks per 128-token tile of the fused router
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopK = 32;
 constexpr int kMaxGroups = 32;
@@ -20,6 +21,17 @@ constexpr uint32_t kErrTimeoutWait = 1u << 0;
 constexpr uint32_t kErrBadIndex = 1u << 1;
 
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// A caller-supplied segment offset, clamped into [0, hi] so that every row a
+// kernel derives from it stays inside the packed arrays; a value that needed
+// clamping is recorded in the error word (when there is one).
+__device__ __forceinline__ int clamp_offset(int v, int hi, uint32_t* err) {
+  if (v < 0 || v > hi) {
+    if (err) atomicOr(err, kErrBadIndex);
+    return v < 0 ? 0 : hi;
+  }
+  return v;
+}
 __host__ __device__ inline long long ceil_div_ll(long long a, long long b) { return (a + b - 1) / b; }
 
 template <typename T> struct Vec16;            // 16-byte vector of T
@@ -43,6 +55,13 @@ __device__ __forceinline__ float gelu_erf(float v) {
 }
 
 // ---------------------------------------------------------------- launchers
+// Per-token routing settings (route_topk.cuh).
+struct TopkArgs {
+  int E, k, gate_mode, n_groups, topk_groups;
+  float route_scale;
+  const float* bias;   // [E] or null
+};
+
 // Routing (route_kernels.cu)
 struct RouteParams {
   int T, E, k, gate_mode, n_groups, topk_groups;
@@ -65,9 +84,14 @@ cudaError_t launch_balance_update(const int* counts, int E, long long tk, float 
                                   float* entropy, cudaStream_t s);
 
 // Permute / combine (permute_kernels.cu)
+// A token's packed row: offsets[e] + tile_base[chunk / kTileChunks][e] (null:
+// 0) + chunk_base[chunk][e] + its rank among the chunk's tokens that chose e.
+// Ids outside [0, E) and rows outside [0, T*k) are skipped (row -1) and
+// recorded in `err` (nullable).
 cudaError_t launch_permute(int dtype, const void* x, const int* topk_idx, const int* offsets,
-                           const int* chunk_base, int T, int d, int E, int k, void* x_perm,
-                           int* perm_src, int* inv_row, int num_sms, cudaStream_t s, bool copy);
+                           const int* chunk_base, const int* tile_base, int T, int d, int E, int k,
+                           void* x_perm, int* perm_src, int* inv_row, int num_sms, cudaStream_t s, bool copy,
+                           uint32_t* err);
 cudaError_t launch_combine(int dtype, const void* y_perm, const int* inv_row, const float* gate,
                            const void* y_shared, void* y, int T, int d, int k, int num_sms,
                            cudaStream_t s);
@@ -85,7 +109,8 @@ struct SimtGemmParams {
   int shared_rows;          // rows of the dense (shared) segment, 0 = none
   const void* a_s; const void* b1_s; const void* b3_s; void* out_s;
   int N_s, K_s;
-  int max_rows;             // upper bound on routed rows (T*k) for the grid
+  int max_rows;             // routed rows (T*k): grid size, and the bound offsets are clamped to
+  uint32_t* err;            // error word for out-of-range offsets, or null
   // Dual GEMM, optional: also store A B1^T and A B3^T (pre-activations).
   void* pre_a; void* pre_b; void* pre_a_s; void* pre_b_s;
   // Single GEMM only: out = act(A B1^T + bias), bias fp32 [n_routed][N] / [N_s] or null.
@@ -179,6 +204,21 @@ struct WgradParams {
 };
 cudaError_t launch_wgrad(const WgradParams& p, int num_sms, cudaStream_t s);
 cudaError_t launch_wait_timeout_selftest(uint32_t* err, long long timeout_ns, cudaStream_t s);
+
+// The whole router in one kernel (router_fused.cu), bf16 and E <= 256:
+// logits, top-k, gates, chunk bases within 128-token tiles, tile bases,
+// counts and offsets. `done_count` must be zero before the launch.
+struct FusedRouterLaunch {
+  const void* x; const void* w_router;
+  int T, E, K;
+  TopkArgs topk;
+  float* logits; int* topk_idx; float* topk_gate;
+  int* chunk_base; int* tile_hist; int* tile_base; int* counts; int* offsets;
+  uint32_t* err; uint32_t* done_count;
+};
+bool router_fused_supported(int dtype, int E);
+int router_fused_cluster(int T, int K);
+cudaError_t launch_router_fused(const FusedRouterLaunch& a, cudaStream_t s);
 
 // tcgen05 router logits with a split contraction (umma_router.cu): partial
 // [n_split][T][E] fp32, summed by the top-k kernel.

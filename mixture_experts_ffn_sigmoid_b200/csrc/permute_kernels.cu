@@ -19,15 +19,18 @@ __device__ __forceinline__ uint4 ld16(const void* p) { return __ldg(reinterpret_
 __device__ __forceinline__ void st16(void* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
 
 // grid = (chunks of 32 tokens, column splits). Each block recomputes its
-// chunk's packed rows (cheap), then copies a column slice of the 32 rows to
-// their k destinations. Split 0 also writes inv_row / perm_src. Without
+// chunk's packed rows (cheap: offsets[e] + the chunk's base for e, plus the
+// base of its 128-token tile when the chunk bases count from the tile's
+// start, + the token's rank in the chunk), then copies a column slice of the
+// 32 rows to their k destinations. Split 0 also writes inv_row / perm_src. Without
 // `copy` only the maps are written (the GEMM then gathers rows from x).
 template <typename T>
 __global__ void __launch_bounds__(256) permute_kernel(
     const T* __restrict__ x, const int* __restrict__ idx, const int* __restrict__ offsets,
-    const int* __restrict__ chunk_base, int n_tok, int d, int E, int k, T* __restrict__ x_perm,
+    const int* __restrict__ chunk_base, const int* __restrict__ tile_base, int n_tok, int d, int E, int k,
+    T* __restrict__ x_perm,
     int* __restrict__ perm_src, int* __restrict__ inv_row, int rows_total, int vec_per_split,
-    int copy) {
+    int copy, uint32_t* __restrict__ err) {
   constexpr int V = Vec16<T>::N;
   __shared__ uint32_t s_mask[kMaxExperts];
   __shared__ int s_row[kChunk * kMaxTopK];
@@ -51,8 +54,10 @@ __global__ void __launch_bounds__(256) permute_kernel(
       if (e >= 0 && e < E) {
         const int rank = __popc(s_mask[e] & ((1u << tid) - 1u));
         row = offsets[e] + chunk_base[(size_t)c * E + e] + rank;
+        if (tile_base) row += tile_base[(size_t)(c / kTileChunks) * E + e];
         if (row < 0 || row >= rows_total) row = -1;
       }
+      if (row < 0 && err && blockIdx.y == 0) atomicOr(err, kErrBadIndex);
       s_row[tid * k + j] = row;
       if (blockIdx.y == 0) {
         inv_row[(size_t)t * k + j] = row;
@@ -68,13 +73,31 @@ __global__ void __launch_bounds__(256) permute_kernel(
   const int nv = v1 - v0;
   const int ntok = min(kChunk, n_tok - c * kChunk);
   if (nv <= 0) return;
-  for (int item = tid; item < ntok * nv; item += blockDim.x) {
-    const int tl = item / nv;
-    const int v = v0 + item - tl * nv;
-    const uint4 val = ld16(x + (size_t)(c * kChunk + tl) * d + (size_t)v * V);
-    for (int j = 0; j < k; ++j) {
-      const int row = s_row[tl * k + j];
-      if (row >= 0) st16(x_perm + (size_t)row * d + (size_t)v * V, val);
+  // Four independent 16-byte loads in flight per thread before their stores
+  // (each load feeds k stores, so the copy is bound by how many loads wait).
+  constexpr int U = 4;
+  const int n_items = ntok * nv;
+  for (int base = tid; base < n_items; base += U * blockDim.x) {
+    uint4 val[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int item = base + u * blockDim.x;
+      if (item < n_items) {
+        const int tl = item / nv;
+        val[u] = ld16(x + (size_t)(c * kChunk + tl) * d + (size_t)(v0 + item - tl * nv) * V);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int item = base + u * blockDim.x;
+      if (item < n_items) {
+        const int tl = item / nv;
+        const int v = v0 + item - tl * nv;
+        for (int j = 0; j < k; ++j) {
+          const int row = s_row[tl * k + j];
+          if (row >= 0) st16(x_perm + (size_t)row * d + (size_t)v * V, val[u]);
+        }
+      }
     }
   }
 }
@@ -119,13 +142,14 @@ template <> __device__ __forceinline__ uint4 pack<__nv_bfloat16>(const float* ac
 template <typename T>
 __global__ void __launch_bounds__(128) combine_kernel(
     const T* __restrict__ y_perm, const int* __restrict__ inv_row, const float* __restrict__ gate,
-    const T* __restrict__ y_shared, T* __restrict__ y, int d, int k, int vec_per_split) {
+    const T* __restrict__ y_shared, T* __restrict__ y, int d, int k, int vec_per_split, int rows_total) {
   constexpr int V = Vec16<T>::N;
   __shared__ int s_row[kMaxTopK];
   __shared__ float s_g[kMaxTopK];
   const int t = blockIdx.x;
   if (threadIdx.x < k) {
-    s_row[threadIdx.x] = inv_row[(size_t)t * k + threadIdx.x];
+    const int r = inv_row[(size_t)t * k + threadIdx.x];
+    s_row[threadIdx.x] = r < rows_total ? r : -1;   // a caller row past the packed rows is skipped
     s_g[threadIdx.x] = gate[(size_t)t * k + threadIdx.x];
   }
   __syncthreads();
@@ -148,8 +172,9 @@ __global__ void __launch_bounds__(128) combine_kernel(
 }  // namespace
 
 cudaError_t launch_permute(int dtype, const void* x, const int* topk_idx, const int* offsets,
-                           const int* chunk_base, int T, int d, int E, int k, void* x_perm,
-                           int* perm_src, int* inv_row, int num_sms, cudaStream_t s, bool copy) {
+                           const int* chunk_base, const int* tile_base, int T, int d, int E, int k,
+                           void* x_perm, int* perm_src, int* inv_row, int num_sms, cudaStream_t s, bool copy,
+                           uint32_t* err) {
   if (T <= 0) return cudaSuccess;
   const int V = dtype == MOE_DTYPE_F32 ? 4 : 8;
   const int nvec = d / V;
@@ -161,12 +186,13 @@ cudaError_t launch_permute(int dtype, const void* x, const int* topk_idx, const 
   nsplit = ceil_div(nvec, vps);
   dim3 grid(nch, nsplit);
   if (dtype == MOE_DTYPE_F32)
-    permute_kernel<float><<<grid, 256, 0, s>>>((const float*)x, topk_idx, offsets, chunk_base, T, d,
-                                                E, k, (float*)x_perm, perm_src, inv_row, T * k, vps, copy ? 1 : 0);
+    permute_kernel<float><<<grid, 256, 0, s>>>((const float*)x, topk_idx, offsets, chunk_base, tile_base, T,
+                                                d, E, k, (float*)x_perm, perm_src, inv_row, T * k, vps,
+                                                copy ? 1 : 0, err);
   else
     permute_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-        (const __nv_bfloat16*)x, topk_idx, offsets, chunk_base, T, d, E, k,
-        (__nv_bfloat16*)x_perm, perm_src, inv_row, T * k, vps, copy ? 1 : 0);
+        (const __nv_bfloat16*)x, topk_idx, offsets, chunk_base, tile_base, T, d, E, k,
+        (__nv_bfloat16*)x_perm, perm_src, inv_row, T * k, vps, copy ? 1 : 0, err);
   return cudaGetLastError();
 }
 
@@ -185,11 +211,11 @@ cudaError_t launch_combine(int dtype, const void* y_perm, const int* inv_row, co
   dim3 grid(T, nsplit);
   if (dtype == MOE_DTYPE_F32)
     combine_kernel<float><<<grid, 128, 0, s>>>((const float*)y_perm, inv_row, gate,
-                                               (const float*)y_shared, (float*)y, d, k, vps);
+                                               (const float*)y_shared, (float*)y, d, k, vps, T * k);
   else
     combine_kernel<__nv_bfloat16><<<grid, 128, 0, s>>>(
         (const __nv_bfloat16*)y_perm, inv_row, gate, (const __nv_bfloat16*)y_shared,
-        (__nv_bfloat16*)y, d, k, vps);
+        (__nv_bfloat16*)y, d, k, vps, T * k);
   return cudaGetLastError();
 }
 

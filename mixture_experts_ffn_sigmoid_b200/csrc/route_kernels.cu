@@ -1,12 +1,9 @@
-// Routing kernels: biased, optionally group-limited top-k over router logits,
+// Routing kernels: biased, optionally group-limited top-k over router logits
+// held in memory (the per-token logic of route_topk.cuh: the Sparse MoE FFN
+// note's Routing paragraph and the MoE cheat sheet's "The router in code"),
 // gates from the unbiased affinities, and the deterministic packing offsets.
-//
-// Sparse MoE FFN (DeepSeek-V3 note), "How it works", Routing paragraph:
-//   s = sigmoid(u . e_i); top-K on s + b (after group masking: 8 groups,
-//   keep 4, group score = sum of top-2); gates = unbiased selected s,
-//   renormalised over the winners, times route_scale.
-// MoE cheat sheet, "The router in code": bias moves selection only; softmax
-//   over the chosen raw scores (max-subtracted), which sums to 1.
+// Used for fp32 inputs and for more than 256 experts; the bf16 router of up
+// to 256 experts runs fused with its GEMM (router_fused.cu).
 //
 // Layout: one warp per token, lane l holds experts l, l+32, l+64, ...; a
 // block of 32 warps is one chunk of 32 tokens, so the same block can also
@@ -16,14 +13,12 @@
 // offsets[e] + #{earlier tokens that chose e}: deterministic, atomic-free.
 #include <math.h>
 
-#include "moe_internal.cuh"
+#include "route_topk.cuh"
 
 namespace moe {
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
-
-__device__ __forceinline__ float sigmoid_f32(float l) { return 1.0f / (1.0f + expf(-l)); }
 
 template <int NPL>
 __global__ void __launch_bounds__(1024, 1) router_topk_kernel(RouteParams p) {
@@ -37,120 +32,27 @@ __global__ void __launch_bounds__(1024, 1) router_topk_kernel(RouteParams p) {
 
   if (t < p.T) {                       // warp-uniform
     float* lrow = p.logits + (size_t)t * E;
-    float v[NPL];                      // biased selection score b' = s + bias
+    float lg[NPL];
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
       const int e = lane + 32 * i;
-      float b = -INFINITY;
+      float l = 0.0f;
       if (e < E) {
         // Router partial sums (a split contraction) add up in a fixed order;
         // the total replaces partial 0, where later readers find the logit.
-        float l = lrow[e];
+        l = lrow[e];
         for (int q = 1; q < p.n_partials; ++q) l += lrow[(size_t)q * p.partial_stride + e];
         if (p.n_partials > 1) lrow[e] = l;
-        const float s = (p.gate_mode == MOE_GATE_SIGMOID) ? sigmoid_f32(l) : l;
-        b = s + (p.bias ? p.bias[e] : 0.0f);
-        // A NaN score (NaN or infinite input, NaN bias) ranks below every
-        // number, so it can neither win over a real score nor lose every
-        // comparison and leave the arg-max without a candidate.
-        if (isnan(b)) b = -INFINITY;
       }
-      v[i] = b;
+      lg[i] = l;
     }
-
-    if (p.n_groups > 1) {
-      // Group score = sum of the two largest b' of the group; lane G ends up
-      // holding group G's score.
-      const int gsz = E / p.n_groups;
-      float my_gscore = -INFINITY;
-      for (int G = 0; G < p.n_groups; ++G) {
-        float m1 = -INFINITY, m2 = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < NPL; ++i) {
-          const int e = lane + 32 * i;
-          if (e < E && e / gsz == G) {
-            const float x = v[i];
-            if (x > m1) { m2 = m1; m1 = x; } else if (x > m2) { m2 = x; }
-          }
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          const float o1 = __shfl_xor_sync(kFull, m1, off);
-          const float o2 = __shfl_xor_sync(kFull, m2, off);
-          const float hi = fmaxf(m1, o1);
-          const float lo = fmaxf(fminf(m1, o1), fmaxf(m2, o2));
-          m1 = hi;
-          m2 = lo;
-        }
-        if (lane == G) my_gscore = isnan(m1 + m2) ? -INFINITY : m1 + m2;   // +inf + -inf
-      }
-      // Keep the topk_groups best groups; ties go to the lower group index.
-      int rank = 0;
-      for (int G = 0; G < p.n_groups; ++G) {
-        const float o = __shfl_sync(kFull, my_gscore, G);
-        if (o > my_gscore || (o == my_gscore && G < lane)) ++rank;
-      }
-      const unsigned kept = __ballot_sync(kFull, lane < p.n_groups && rank < p.topk_groups);
-#pragma unroll
-      for (int i = 0; i < NPL; ++i) {
-        const int e = lane + 32 * i;
-        if (e < E && !((kept >> (e / gsz)) & 1u)) v[i] = -INFINITY;
-      }
-    }
-
-    // k rounds of a warp arg-max: largest b' first, equal b' to the lower id.
-    // kNone marks "no candidate yet": the first untaken in-range expert a lane
-    // sees always becomes its candidate, and a real candidate always beats
-    // kNone in the reduction. Round r < k <= E leaves at least one untaken
-    // expert, so every winner is an id in [0, E) whatever the scores hold.
-    constexpr int kNone = 0x7fffffff;
-    unsigned taken = 0u;
-    int my_e = -1;                     // lane j < k ends with the j-th winner
-    for (int r = 0; r < k; ++r) {
-      float bv = -INFINITY;
-      int be = kNone;
-#pragma unroll
-      for (int i = 0; i < NPL; ++i) {
-        const int e = lane + 32 * i;
-        if (e < E && !((taken >> i) & 1u)) {
-          if (be == kNone || v[i] > bv || (v[i] == bv && e < be)) { bv = v[i]; be = e; }
-        }
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(kFull, bv, off);
-        const int oe = __shfl_xor_sync(kFull, be, off);
-        if (oe != kNone && (be == kNone || ov > bv || (ov == bv && oe < be))) { bv = ov; be = oe; }
-      }
-      if (be == kNone) be = 0;         // unreachable (k <= E); keeps the id in range regardless
-      if ((be & 31) == lane) taken |= 1u << (be >> 5);
-      if (lane == r) my_e = be;
-    }
-
-    // Report winners in ascending expert id.
-    int pos = 0;
-    for (int j = 0; j < k; ++j) {
-      const int o = __shfl_sync(kFull, my_e, j);
-      if (o < my_e) ++pos;
-    }
-    // Gates from the UNBIASED value of each winner.
-    const bool act = lane < k;
-    const float l = act ? lrow[my_e] : 0.0f;
-    float num;
-    if (p.gate_mode == MOE_GATE_SIGMOID) {
-      num = act ? sigmoid_f32(l) : 0.0f;
-    } else {
-      float m = act ? l : -INFINITY;
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
-      num = act ? expf(l - m) : 0.0f;
-    }
-    float sum = num;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(kFull, sum, off);
-    if (act) {
+    const TopkArgs a = {E, k, p.gate_mode, p.n_groups, p.topk_groups, p.route_scale, p.bias};
+    int my_e, pos;
+    float gate;
+    route_token<NPL>(lg, lane, a, my_e, pos, gate);
+    if (lane < k) {
       p.topk_idx[(size_t)t * k + pos] = my_e;
-      p.topk_gate[(size_t)t * k + pos] = p.route_scale * (num / sum);
+      p.topk_gate[(size_t)t * k + pos] = gate;
       atomicOr(&s_mask[my_e], 1u << warp);
     }
   }

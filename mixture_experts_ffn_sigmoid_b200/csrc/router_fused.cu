@@ -1,0 +1,390 @@
+// The router of the block in one kernel (bf16 inputs, up to 256 experts):
+// logits, affinities, biased group-limited top-k, gates, per-expert counts
+// and packing offsets.
+//
+//   l[t][e] = sum_c x[t][c] w_router[e][c]         (the router linear: the
+//     Sparse MoE FFN note's Routing paragraph, u_t . e_i; the MoE cheat
+//     sheet's "The router in code": one dot product per router row)
+//   then per token the biased, group-limited top-k and the gates of
+//   route_topk.cuh, and the counts and offsets that pack every token's rows
+//   expert by expert, tokens in order (the note's "Packed forward
+//   (official)": each expert gathers the tokens that chose it).
+//
+// One 128-token tile per cluster of S CTAs (S = 1, 2, 4 or 8). CTA r of the
+// cluster runs its share of the contraction on the tensor cores: TMA stages
+// x and w_router tiles (128-byte swizzle) into a 4-stage ring, one lane
+// issues tcgen05.mma (kind::f16, M = 128 tokens, N = the expert count
+// rounded up to 16, fp32 accumulator in TMEM). The 32 warps then copy the
+// partial logits from TMEM into the CTA's shared memory (over the ring,
+// which is no longer needed), and after a cluster barrier the CTAs add the
+// S partial sums through distributed shared memory in rank order (a fixed
+// order: the logits are the same bits on every run). The tile's four
+// 32-token chunks are shared among the CTAs; in each, warp w routes token w
+// and the chunk's per-expert bit mask records which tokens chose each
+// expert. CTA 0 turns the four masks into each chunk's base within the tile
+// and the tile's histogram. The last tile to finish (a device-wide counter)
+// scans the tile histograms into each tile's base, the per-expert counts
+// and the offsets. A token's packed row is then
+//   offsets[e] + tile_base[tile][e] + chunk_base[chunk][e] + (earlier tokens
+//   of its chunk that chose e),
+// which the permute kernel computes.
+//
+// No fp32 partial logits go through HBM; the summed logits are written once
+// ([T][E], kept for the backward pass). Every mbarrier wait is bounded; on
+// expiry the CTA records the timeout in the error word and still reaches
+// every cluster barrier, so no CTA waits for an aborted peer.
+#include "route_topk.cuh"
+#include "umma_common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int FR_BM = 128;                        // tokens per tile (one cluster)
+constexpr int FR_BK = 64;
+constexpr int FR_STAGES = 4;
+constexpr int FR_THREADS = 1024;                  // 32 warps: one token each when routing
+constexpr int FR_BN_MAX = 256;
+constexpr int FR_A_BYTES = FR_BM * FR_BK * 2;     // 16 KB of x per stage
+constexpr int FR_HDR = 1024;
+constexpr int FR_TMEM_COLS = 256;
+
+static_assert(FR_BM == kTileChunks * kChunk, "a tile is kTileChunks chunks");
+
+struct FusedRouterArgs {
+  int T, E, K;
+  int n_pad;          // MMA N: E rounded up to 16
+  int kb_per_split;   // 64-wide k blocks per CTA of a cluster
+  int ntiles;
+  TopkArgs topk;
+  float* logits;      // [T][E] summed router logits
+  int* topk_idx;      // [T][k]
+  float* topk_gate;   // [T][k]
+  int* chunk_base;    // [ceil(T/32)][E]: base of each chunk within its tile
+  int* tile_hist;     // [ntiles][E]
+  int* tile_base;     // [ntiles][E]: base of each tile
+  int* counts;        // [E]
+  int* offsets;       // [E + 1]
+  uint32_t* err;
+  uint32_t* done_count;   // zero before the launch; the last tile sets it back to zero
+  long long timeout_ns;
+};
+
+__host__ __device__ inline int fr_stage_bytes(int n_pad) { return FR_A_BYTES + n_pad * FR_BK * 2; }
+__host__ __device__ inline int fr_smem_bytes(int n_pad) {
+  // alignment slack, header, ring (also the partial-logit buffer), the tile's
+  // chunk masks [kTileChunks][256] and the scan's partial sums [4][256]
+  return 1024 + FR_HDR + FR_STAGES * fr_stage_bytes(n_pad) + kTileChunks * 256 * 4 + 4 * 256 * 4 + 256;
+}
+
+template <int NPL>
+__global__ void __launch_bounds__(FR_THREADS, 1)
+    router_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                        const FusedRouterArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty_bar = full_bar + FR_STAGES;
+  uint64_t* done_bar = empty_bar + FR_STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+  volatile int* s_last = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  int* s_warp = reinterpret_cast<int*>(tmem_slot + 4);          // [32]
+  uint8_t* ring = smem + FR_HDR;
+  const int stage_bytes = fr_stage_bytes(p.n_pad);
+  float* s_log = reinterpret_cast<float*>(ring);                // [128][ld_log] after the MMAs
+  const int ld_log = p.n_pad + 4;                               // 16-byte rows, conflict-free float4 stores
+  uint32_t* s_mask = reinterpret_cast<uint32_t*>(ring + FR_STAGES * stage_bytes);   // [kTileChunks][256]
+  int* s_part = reinterpret_cast<int*>(s_mask + kTileChunks * 256);                 // [4][256]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const uint32_t S = cluster_ncta();
+  const int tile = (int)(blockIdx.x / S);
+  const int t0 = tile * FR_BM;
+  const int E = p.E;
+  const int nkb = ceil_div(p.K, FR_BK);
+  const int kb0 = (int)rank * p.kb_per_split;
+  const int kb1 = min(nkb, kb0 + p.kb_per_split);
+  const int nk = max(0, kb1 - kb0);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < FR_STAGES; ++i) {
+      mbar_init(smem_u32(&full_bar[i]), 1);
+      mbar_init(smem_u32(&empty_bar[i]), 1);
+    }
+    mbar_init(smem_u32(done_bar), 1);
+    *abort_flag = 0u;
+    fence_mbar_init();
+    tmap_prefetch(&tmX);
+    tmap_prefetch(&tmW);
+  }
+  for (int i = threadIdx.x; i < kTileChunks * 256; i += blockDim.x) s_mask[i] = 0u;
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), FR_TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  // ------------------------------------------------------------ partial logits
+  if (warp == 0 && lane == 0) {
+    // producer: x [128 tokens][64] and w_router [n_pad experts][64] per k block
+    int n_issued = 0;
+    for (int i = 0; i < nk; ++i) {
+      const int stage = i % FR_STAGES;
+      const uint32_t parity = ((i / FR_STAGES) & 1u) ^ 1u;
+      if (!wait_bounded(smem_u32(&empty_bar[stage]), parity, abort_flag, p.err, p.timeout_ns, true)) break;
+      const uint32_t fb = smem_u32(&full_bar[stage]);
+      const uint32_t sa = smem_u32(ring + stage * stage_bytes);
+      mbar_expect_tx(fb, (uint32_t)stage_bytes);   // whole boxes; rows past T or E read as zeros
+      tma_load_2d(sa, &tmX, (kb0 + i) * FR_BK, t0, fb);
+      tma_load_2d(sa + FR_A_BYTES, &tmW, (kb0 + i) * FR_BK, 0, fb);
+      n_issued = i + 1;
+    }
+    // Every copy this thread started has landed before the ring is reused
+    // for the partial logits (on an abort some may not have been consumed).
+    for (int i = max(0, n_issued - FR_STAGES); i < n_issued; ++i)
+      wait_bounded(smem_u32(&full_bar[i % FR_STAGES]), (i / FR_STAGES) & 1u, abort_flag, p.err, p.timeout_ns,
+                   false);
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // MMA issuer
+      bool issued = false;
+      const uint32_t idesc = idesc_bf16_f32(FR_BM, p.n_pad);
+      for (int i = 0; i < nk; ++i) {
+        const int stage = i % FR_STAGES;
+        if (!wait_bounded(smem_u32(&full_bar[stage]), (i / FR_STAGES) & 1u, abort_flag, p.err, p.timeout_ns,
+                          true))
+          break;
+        tc_fence_after();
+        const uint32_t sa = smem_u32(ring + stage * stage_bytes);
+        const uint64_t a_desc = sw128_desc(sa);
+        const uint64_t b_desc = sw128_desc(sa + FR_A_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < FR_BK / 16; ++kk) {
+          const uint64_t koff = (uint64_t)((kk * 32) >> 4);
+          umma_bf16(tmem_base, a_desc + koff, b_desc + koff, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(smem_u32(&empty_bar[stage]));
+        issued = true;
+      }
+      if (issued) umma_commit(smem_u32(done_bar));   // completion of every MMA releases the drain
+      else mbar_arrive(smem_u32(done_bar));
+    }
+    __syncwarp();
+  }
+  __syncwarp();
+  const bool ok = __all_sync(0xffffffffu,
+                             wait_bounded(smem_u32(done_bar), 0u, abort_flag, p.err, p.timeout_ns, false));
+  tc_fence_after();
+  __syncthreads();      // the producer's copies have landed: the ring may be overwritten
+  // TMEM -> shared memory: warp w reads lane quarter w & 3 (32 tokens) and
+  // 32 columns starting at 32 * (w >> 2).
+  {
+    const int q = warp & 3, c0 = (warp >> 2) * 32;
+    if (c0 < p.n_pad) {
+      uint32_t ra[16], rb[16];
+      if (ok && nk > 0) {
+        const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)c0;
+        tmem_ld16x2_wait(ta, ta + 16, ra, rb);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) { ra[j] = 0u; rb[j] = 0u; }   // empty share (or a failed wait): zeros
+      }
+      float* row = s_log + (q * 32 + lane) * ld_log + c0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        reinterpret_cast<float4*>(row)[j] = make_float4(__uint_as_float(ra[4 * j]), __uint_as_float(ra[4 * j + 1]),
+                                                        __uint_as_float(ra[4 * j + 2]), __uint_as_float(ra[4 * j + 3]));
+      if (c0 + 16 < p.n_pad) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          reinterpret_cast<float4*>(row + 16)[j] =
+              make_float4(__uint_as_float(rb[4 * j]), __uint_as_float(rb[4 * j + 1]), __uint_as_float(rb[4 * j + 2]),
+                          __uint_as_float(rb[4 * j + 3]));
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, FR_TMEM_COLS);
+  }
+  cluster_sync_all();   // every CTA's partial logits are in its shared memory
+
+  // ------------------------------------------------------------ routing
+  const int nch_tile = min(kTileChunks, ceil_div(p.T - t0, kChunk));
+  const int k = p.topk.k;
+  for (int j = (int)rank; j < nch_tile; j += (int)S) {
+    const int tl = j * kChunk + warp;       // token of the tile this warp routes
+    const int t = t0 + tl;
+    if (t < p.T) {                          // warp-uniform
+      float lg[NPL];
+#pragma unroll
+      for (int i = 0; i < NPL; ++i) {
+        const int e = lane + 32 * i;
+        float l = 0.0f;
+        if (e < E) {
+          const uint32_t a = smem_u32(s_log + tl * ld_log + e);
+          l = ld_cluster_f32(map_to_cta(a, 0));
+          for (uint32_t q = 1; q < S; ++q) l += ld_cluster_f32(map_to_cta(a, q));
+          p.logits[(size_t)t * E + e] = l;
+        }
+        lg[i] = l;
+      }
+      int my_e, pos;
+      float gate;
+      route_token<NPL>(lg, lane, p.topk, my_e, pos, gate);
+      if (lane < k) {
+        p.topk_idx[(size_t)t * k + pos] = my_e;
+        p.topk_gate[(size_t)t * k + pos] = gate;
+        atomicOr(&s_mask[j * 256 + my_e], 1u << warp);
+      }
+    }
+  }
+  __syncthreads();
+  cluster_sync_all();   // chunk masks complete; no CTA reads a peer's logits any more
+
+  // ------------------------------------------------------------ tile histogram (CTA 0)
+  if (rank == 0) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      int run = 0;
+      for (int j = 0; j < nch_tile; ++j) {
+        const uint32_t m = ld_cluster_u32(map_to_cta(smem_u32(&s_mask[j * 256 + e]), (uint32_t)j % S));
+        p.chunk_base[(size_t)(tile * kTileChunks + j) * E + e] = run;
+        run += __popc(m);
+      }
+      p.tile_hist[(size_t)tile * E + e] = run;
+    }
+  }
+  cluster_sync_all();   // CTA 0 has read its peers' masks: they may exit
+  if (rank != 0) return;
+
+  // ------------------------------------------------------------ last tile: scan
+  __threadfence();      // this CTA's chunk bases and tile histogram before its arrival
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t prev = atomicAdd(p.done_count, 1u);
+    *s_last = prev == (uint32_t)(p.ntiles - 1) ? 1 : 0;
+  }
+  __syncthreads();
+  if (!*s_last) return;
+  __threadfence();
+  // Four groups of 256 threads, each over a quarter of the tiles: its partial
+  // per-expert sums, then each tile's base from the groups before it.
+  const int g = threadIdx.x >> 8, e = threadIdx.x & 255;
+  const int per = ceil_div(p.ntiles, 4);
+  const int i0 = min(p.ntiles, g * per), i1 = min(p.ntiles, i0 + per);
+  int part = 0;
+  if (e < E)
+    for (int i = i0; i < i1; ++i) part += __ldcg(&p.tile_hist[(size_t)i * E + e]);
+  s_part[g * 256 + e] = part;
+  __syncthreads();
+  if (e < E) {
+    int run = 0;
+    for (int gg = 0; gg < g; ++gg) run += s_part[gg * 256 + e];
+    for (int i = i0; i < i1; ++i) {
+      p.tile_base[(size_t)i * E + e] = run;
+      run += __ldcg(&p.tile_hist[(size_t)i * E + e]);
+    }
+  }
+  // Counts, then offsets = exclusive scan of the counts over experts (threads 0..255).
+  int cnt = 0;
+  if (g == 0 && e < E) {
+    cnt = s_part[e] + s_part[256 + e] + s_part[512 + e] + s_part[768 + e];
+    p.counts[e] = cnt;
+  }
+  int incl = cnt;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (g == 0 && lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (g == 0) {
+    int before = 0;
+    for (int w = 0; w < warp; ++w) before += s_warp[w];
+    if (e < E) p.offsets[e] = before + incl - cnt;
+    if (e == 0) {
+      int total = 0;
+      for (int w = 0; w < 8; ++w) total += s_warp[w];
+      p.offsets[E] = total;
+      *p.done_count = 0u;   // ready for the next launch
+    }
+  }
+}
+
+}  // namespace
+
+bool router_fused_supported(int dtype, int E) { return dtype == MOE_DTYPE_BF16 && E >= 1 && E <= FR_BN_MAX; }
+
+// CTAs per tile: the largest of 8, 4, 2, 1 that keeps every CTA at least one
+// k block and the grid within B200's 148 SMs (one CTA per SM). A function of
+// the shape only.
+int router_fused_cluster(int T, int K) {
+  constexpr int num_sms = 148;
+  const int ntiles = ceil_div(T, FR_BM);
+  const int nkb = ceil_div(K, FR_BK);
+  int s = 8;
+  while (s > 1 && (s > nkb || ntiles * s > num_sms)) s >>= 1;
+  return s;
+}
+
+cudaError_t launch_router_fused(const FusedRouterLaunch& a, cudaStream_t s) {
+  if (a.T <= 0) return cudaSuccess;
+  if (!router_fused_supported(MOE_DTYPE_BF16, a.E)) return cudaErrorInvalidValue;
+  const int n_pad = (a.E + 15) / 16 * 16;
+  CUtensorMap tX, tW;
+  if (!make_tmap(&tX, a.x, a.K, a.T, FR_BM)) return cudaErrorInvalidValue;
+  if (!make_tmap(&tW, a.w_router, a.K, a.E, n_pad)) return cudaErrorInvalidValue;
+  const int smem = fr_smem_bytes(n_pad);
+  const int npl = ceil_div(a.E, 32);
+  auto kernel = npl <= 1 ? router_fused_kernel<1>
+              : npl <= 2 ? router_fused_kernel<2>
+              : npl <= 4 ? router_fused_kernel<4>
+                         : router_fused_kernel<8>;
+  static int attr_done[4] = {0, 0, 0, 0};   // one bit per device ordinal (< 32), per instantiation
+  const int which = npl <= 1 ? 0 : npl <= 2 ? 1 : npl <= 4 ? 2 : 3;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (!(dev < 32 && ((attr_done[which] >> dev) & 1))) {
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fr_smem_bytes(FR_BN_MAX));
+    if (e != cudaSuccess) return e;
+    if (dev < 32) attr_done[which] |= 1 << dev;
+  }
+  FusedRouterArgs p = {};
+  p.T = a.T; p.E = a.E; p.K = a.K;
+  p.n_pad = n_pad;
+  const int S = router_fused_cluster(a.T, a.K);
+  p.kb_per_split = ceil_div(ceil_div(a.K, FR_BK), S);
+  p.ntiles = ceil_div(a.T, FR_BM);
+  p.topk = a.topk;
+  p.logits = a.logits;
+  p.topk_idx = a.topk_idx; p.topk_gate = a.topk_gate;
+  p.chunk_base = a.chunk_base; p.tile_hist = a.tile_hist; p.tile_base = a.tile_base;
+  p.counts = a.counts; p.offsets = a.offsets;
+  p.err = a.err; p.done_count = a.done_count;
+  p.timeout_ns = kDefaultTimeoutNs;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.ntiles * S);
+  cfg.blockDim = dim3(FR_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, tX, tW, p);
+}
+
+}  // namespace moe

@@ -41,7 +41,11 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGemmParams p) {
   Seg sg;
   bool found = false;
   for (int s = 0; s < p.n_routed; ++s) {
-    const int r0 = p.offsets[s], rows = p.offsets[s + 1] - r0;
+    // Caller offsets clamped into the packed rows (block 0 records a bad one);
+    // a decreasing pair is an empty segment.
+    uint32_t* err = blockIdx.x == 0 && blockIdx.y == 0 ? p.err : nullptr;
+    const int r0 = clamp_offset(p.offsets[s], p.max_rows, err);
+    const int rows = max(0, clamp_offset(p.offsets[s + 1], p.max_rows, err) - r0);
     const int tiles = (rows + TM - 1) / TM;
     if (bx < tiles) {
       sg = Seg{p.a, (const char*)p.b1 + (size_t)s * p.N * p.K * sizeof(TI),

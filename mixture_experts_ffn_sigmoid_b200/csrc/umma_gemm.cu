@@ -112,20 +112,6 @@ struct RingCursor {
 };
 
 // ---- CTA-pair (cluster of 2) forms used by the two-SM MMA path.
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
-}
-// Address of the same shared-memory location in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t map_to_cta(uint32_t saddr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-  return r;
-}
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
@@ -190,6 +176,30 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar, uint16_t mask) {
       : "memory");
 }
 
+// SiLU(g) * u for four accumulator pairs (g, u), in fp32. sigma(g) =
+// 1 / q with q = 1 + e^-g; the four reciprocals come from one (Montgomery's
+// batch-inversion trick: 1/q0 = q1 q2 q3 / (q0 q1 q2 q3), and so on), so the
+// epilogue issues 1.25 special-function operations per element instead of 2
+// (an exponential and a reciprocal each). g is clamped at -21 inside the
+// exponential only: the product of four q stays below 2^122, where the fast
+// reciprocal is accurate, and below g = -21 the clamp moves SiLU(g) by less
+// than |g| * 1e-9. A NaN g makes the clamp return -21, so only its own
+// product is NaN (through the factor g), never its three neighbours'.
+__device__ __forceinline__ void silu_mul4(const uint32_t* g32, const uint32_t* u32, float (&h)[4]) {
+  float g[4], q[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    g[i] = __uint_as_float(g32[i]);
+    q[i] = 1.0f + __expf(-fmaxf(g[i], -21.0f));
+  }
+  const float q01 = q[0] * q[1], q23 = q[2] * q[3];
+  const float r = __fdividef(1.0f, q01 * q23);
+  const float r23 = r * q23, r01 = r * q01;
+  const float sg[4] = {r23 * q[1], r23 * q[0], r01 * q[3], r01 * q[2]};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = g[i] * sg[i] * __uint_as_float(u32[i]);
+}
+
 // ------------------------------------------------------------ tile list
 // Per mode: weight blocks (128 rows each) per CTA. With PAIR the two CTAs of
 // a cluster run one M=256 MMA: each holds 128 rows of every weight block and
@@ -204,12 +214,16 @@ template <> struct Kind<kUmmaDown>   { static constexpr int A_TILES = 2; };
 template <> struct Kind<kUmmaBiasAct> { static constexpr int A_TILES = 2; };
 template <> struct Kind<kUmmaDgrad> { static constexpr int A_TILES = 2; };
 
-// Where a tile's two accumulators sit in the 512 TMEM columns. A tile of at
-// most 128 token columns takes one half (first accumulator at +0, second at
-// +128), alternating halves, so the next such tile accumulates while the
-// epilogue drains this one; a wider tile takes all 512 columns (second
-// accumulator at +256) once both halves are drained. The MMA issuer and the
-// epilogue walk the same tile sequence, so they derive the same placement.
+// Where a tile's two accumulators sit in the 512 TMEM columns. Half h is
+// columns [128h, 128h + 128) and [256 + 128h, 256 + 128h + 128). A tile of at
+// most 128 token columns takes one half (first accumulator at 128h, second
+// at 256 + 128h), alternating halves, so the next such tile accumulates
+// while the epilogue drains this one. A wider tile takes both halves (first
+// accumulator at 0, second at 256): its token columns 0..127 are half 0, so
+// its epilogue can hand half 0 back as soon as it has drained those columns
+// of both accumulators, and a following narrow tile starts while the rest
+// drains. The MMA issuer and the epilogue walk the same tile sequence, so
+// they derive the same placement.
 struct AccPlace {
   uint32_t next = 0;   // half the next narrow tile takes
   __device__ __forceinline__ void take(int n_mma, bool& wide, uint32_t& half) {
@@ -217,8 +231,8 @@ struct AccPlace {
     half = wide ? 0u : next;
     next = wide ? 0u : (next ^ 1u);
   }
-  __device__ __forceinline__ static uint32_t col0(bool wide, uint32_t half) { return wide ? 0u : half * BN_MAX; }
-  __device__ __forceinline__ static uint32_t second(bool wide) { return wide ? BN_MAX : BN_MAX / 2; }
+  __device__ __forceinline__ static uint32_t col0(bool wide, uint32_t half) { return wide ? 0u : half * (BN_MAX / 2); }
+  __device__ __forceinline__ static uint32_t second(bool) { return BN_MAX; }
 };
 
 // Modes whose tile is two consecutive 128-row blocks of one weight matrix.
@@ -335,8 +349,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int group = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int ngroups = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
+  // Segment offsets come from the caller: each is clamped into the packed
+  // rows (and a decreasing pair makes an empty segment), so no tile can reach
+  // past them; CTA 0 records any offset that was out of range.
   for (int s = threadIdx.x; s <= p.n_routed; s += blockDim.x)
-    s_off[s] = p.n_routed > 0 ? p.offsets[s] : 0;
+    s_off[s] = p.n_routed > 0 ? clamp_offset(p.offsets[s], p.max_routed_rows, blockIdx.x == 0 ? p.err : nullptr)
+                              : 0;
   if (threadIdx.x == 64) {
     for (int i = 0; i < NSLOT; ++i) {
       mbar_init(smem_u32(&full_bar[i]), 1);
@@ -390,6 +408,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     if (lane == 31) s_start[nseg] = incl;
   }
+  if (blockIdx.x == 0 && p.err)
+    for (int s = threadIdx.x; s < p.n_routed; s += blockDim.x)
+      if (s_off[s + 1] < s_off[s]) atomicOr(p.err, kErrBadIndex);
   tc_fence_before();
   if (PAIR) cluster_sync_all(); else __syncthreads();   // barriers of both CTAs exist from here on
   tc_fence_after();
@@ -619,18 +640,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const long long r0 = (long long)t.b_row0 + (long long)t.tt * p.bn_max;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + AccPlace::col0(wide, half);
       const uint32_t off2 = AccPlace::second(wide);   // second accumulator's column offset
-      // Hand the tile's TMEM back: its half, or both halves for a wide tile.
-      auto release = [&]() {
+      // Hand TMEM half h back to the MMA warp (after this warp's last read of it).
+      auto release_half = [&](uint32_t h) {
+        tc_fence_before();
+        __syncwarp();
         if (lane == 0) {
-          if (PAIR) {
-            mbar_arrive_cluster(acce0 + half * 8u);
-            if (wide) mbar_arrive_cluster(acce0 + 8u);
-          } else {
-            mbar_arrive(acce0 + half * 8u);
-            if (wide) mbar_arrive(acce0 + 8u);
-          }
+          if (PAIR) mbar_arrive_cluster(acce0 + h * 8u);
+          else mbar_arrive(acce0 + h * 8u);
         }
       };
+      // Hand the tile's TMEM back: its half, or both halves for a wide tile.
+      auto release = [&]() {
+        release_half(half);
+        if (wide) release_half(1u);
+      };
+      // The same for epilogues that already handed half 0 of a wide tile back
+      // once its token columns 0..127 were drained (the first four chunk
+      // pairs of each warp).
+      auto release_rest = [&]() { release_half(wide ? 1u : half); };
       if (dual_a(MODE)) {
         // Drain both accumulators into registers as packed bf16 h, hand TMEM
         // back to the MMA warp, then store while the next tile accumulates.
@@ -659,20 +686,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               }
             }
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const float g0 = __uint_as_float(r1[2 * j]), g1 = __uint_as_float(r1[2 * j + 1]);
-              // SiLU(g) = g / (1 + e^-g); the fast divide returns 0 once the
-              // denominator passes 2^126, where the exact quotient is below 1e-36.
-              const float h0 = __fdividef(g0, 1.0f + __expf(-g0)) * __uint_as_float(r3[2 * j]);
-              const float h1 = __fdividef(g1, 1.0f + __expf(-g1)) * __uint_as_float(r3[2 * j + 1]);
-              const __nv_bfloat162 hb = __floats2bfloat162_rn(h0, h1);
-              hp[cc * 8 + j] = *reinterpret_cast<const uint32_t*>(&hb);
+            for (int j = 0; j < 4; ++j) {
+              float hv[4];
+              silu_mul4(&r1[4 * j], &r3[4 * j], hv);
+              const __nv_bfloat162 h01 = __floats2bfloat162_rn(hv[0], hv[1]);
+              const __nv_bfloat162 h23 = __floats2bfloat162_rn(hv[2], hv[3]);
+              hp[cc * 8 + 2 * j] = *reinterpret_cast<const uint32_t*>(&h01);
+              hp[cc * 8 + 2 * j + 1] = *reinterpret_cast<const uint32_t*>(&h23);
             }
           }
+          if (cc == BN_MAX / 64 - 1 && wide) release_half(0u);   // token columns 0..127 drained
         }
-        tc_fence_before();
-        __syncwarp();
-        release();
+        release_rest();
         if (m_ok) {
           unsigned short* o = reinterpret_cast<unsigned short*>(out) + r0 * ld + m;
 #pragma unroll
@@ -705,11 +730,51 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
         }
-        tc_fence_before();
-        __syncwarp();
         release();
-      } else if (MODE == kUmmaDown || MODE == kUmmaDgrad) {
-        // Two 128-row blocks of the tile's weight rows, BLOCK_STEP apart.
+      } else if (MODE == kUmmaDown) {
+        // Two 128-row blocks of W2, BLOCK_STEP apart. Both accumulators are
+        // drained into packed bf16 registers first, TMEM goes back to the MMA
+        // warp, and the stores run while the next tile accumulates (down
+        // tiles are short, 32 k-steps at f = 2048, so a TMEM hold over the
+        // stores would stop the weight stream for a large share of a tile).
+        const int m2 = m + BLOCK_STEP;
+        const bool m2_ok = m2 < t.mrows;
+        uint32_t q1[BN_MAX / 4], q2[BN_MAX / 4];
+#pragma unroll
+        for (int cc = 0; cc < BN_MAX / 32; ++cc) {
+          const int c = 2 * cc + ch;
+          if (c * 16 < n_mma) {
+            uint32_t r1[16], r3[16];
+            tmem_ld16x2_wait(taddr + c * 16, taddr + off2 + c * 16, r1, r3);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const __nv_bfloat162 pa = __floats2bfloat162_rn(__uint_as_float(r1[2 * j]), __uint_as_float(r1[2 * j + 1]));
+              const __nv_bfloat162 pb = __floats2bfloat162_rn(__uint_as_float(r3[2 * j]), __uint_as_float(r3[2 * j + 1]));
+              q1[cc * 8 + j] = *reinterpret_cast<const uint32_t*>(&pa);
+              q2[cc * 8 + j] = *reinterpret_cast<const uint32_t*>(&pb);
+            }
+          }
+          if (cc == BN_MAX / 64 - 1 && wide) release_half(0u);   // token columns 0..127 drained
+        }
+        release_rest();
+        unsigned short* o = reinterpret_cast<unsigned short*>(out) + r0 * ld;
+#pragma unroll
+        for (int cc = 0; cc < BN_MAX / 32; ++cc) {
+          const int c = 2 * cc + ch;
+          if (c * 16 < n_valid) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int col = c * 16 + j;
+              if (col < n_valid) {
+                const int sh = (j & 1) * 16;
+                if (m_ok) o[(long long)col * ld + m] = (unsigned short)(q1[cc * 8 + (j >> 1)] >> sh);
+                if (m2_ok) o[(long long)col * ld + m2] = (unsigned short)(q2[cc * 8 + (j >> 1)] >> sh);
+              }
+            }
+          }
+        }
+      } else if (MODE == kUmmaDgrad) {
+        // Two 128-row blocks, BLOCK_STEP apart; bf16 output.
         const int m2 = m + BLOCK_STEP;
         const bool m2_ok = m2 < t.mrows;
         __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out) + r0 * ld;
@@ -725,12 +790,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
         }
-        tc_fence_before();
-        __syncwarp();
         release();
       } else if (MODE == kUmmaBiasAct) {
-        // As kUmmaDown, with the weight row's bias added and the activation
-        // applied in fp32 before the one rounding to bf16.
+        // As the bf16 input gradients, with the weight row's bias added and the
+        // activation applied in fp32 before the one rounding to bf16.
         const int m2 = m + BLOCK_STEP;
         const bool m2_ok = m2 < t.mrows;
         const float* rb = t.dense ? p.row_bias_s : p.row_bias;
@@ -754,8 +817,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
         }
-        tc_fence_before();
-        __syncwarp();
         release();
       }
     }

@@ -56,8 +56,8 @@ def test_stage_bytes_are_the_operands_touched_once(shared):
     assert work["permute"]["bytes"] == nbytes(inp["x"], x_perm) + 2 * rows * 4 + nbytes(idx32)
     # combine: packed rows and shared rows read, y written, int32 row map and fp32 gates read.
     assert work["combine"]["bytes"] == nbytes(y_perm, y_s, y) + nbytes(idx32, gate32)
-    # route: x and the router read, fp32 logits written and read back, indices and gates written.
-    assert work["route"]["bytes"] == nbytes(inp["x"], inp["w_router"], logits, logits, idx32, gate32)
+    # route: x and the router read, the summed fp32 logits written once, indices and gates written.
+    assert work["route"]["bytes"] == nbytes(inp["x"], inp["w_router"], logits, idx32, gate32)
 
     # flops: 2 per multiply-add of each matmul the stage performs.
     def mm(m, n, kk):
