@@ -176,30 +176,6 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar, uint16_t mask) {
       : "memory");
 }
 
-// SiLU(g) * u for four accumulator pairs (g, u), in fp32. sigma(g) =
-// 1 / q with q = 1 + e^-g; the four reciprocals come from one (Montgomery's
-// batch-inversion trick: 1/q0 = q1 q2 q3 / (q0 q1 q2 q3), and so on), so the
-// epilogue issues 1.25 special-function operations per element instead of 2
-// (an exponential and a reciprocal each). g is clamped at -21 inside the
-// exponential only: the product of four q stays below 2^122, where the fast
-// reciprocal is accurate, and below g = -21 the clamp moves SiLU(g) by less
-// than |g| * 1e-9. A NaN g makes the clamp return -21, so only its own
-// product is NaN (through the factor g), never its three neighbours'.
-__device__ __forceinline__ void silu_mul4(const uint32_t* g32, const uint32_t* u32, float (&h)[4]) {
-  float g[4], q[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    g[i] = __uint_as_float(g32[i]);
-    q[i] = 1.0f + __expf(-fmaxf(g[i], -21.0f));
-  }
-  const float q01 = q[0] * q[1], q23 = q[2] * q[3];
-  const float r = __fdividef(1.0f, q01 * q23);
-  const float r23 = r * q23, r01 = r * q01;
-  const float sg[4] = {r23 * q[1], r23 * q[0], r01 * q[3], r01 * q[2]};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) h[i] = g[i] * sg[i] * __uint_as_float(u32[i]);
-}
-
 // ------------------------------------------------------------ tile list
 // Per mode: weight blocks (128 rows each) per CTA. With PAIR the two CTAs of
 // a cluster run one M=256 MMA: each holds 128 rows of every weight block and
@@ -686,13 +662,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               }
             }
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              float hv[4];
-              silu_mul4(&r1[4 * j], &r3[4 * j], hv);
-              const __nv_bfloat162 h01 = __floats2bfloat162_rn(hv[0], hv[1]);
-              const __nv_bfloat162 h23 = __floats2bfloat162_rn(hv[2], hv[3]);
-              hp[cc * 8 + 2 * j] = *reinterpret_cast<const uint32_t*>(&h01);
-              hp[cc * 8 + 2 * j + 1] = *reinterpret_cast<const uint32_t*>(&h23);
+            for (int j = 0; j < 8; ++j) {
+              const float g0 = __uint_as_float(r1[2 * j]), g1 = __uint_as_float(r1[2 * j + 1]);
+              // SiLU(g) = g / (1 + e^-g), element by element (a token's h
+              // depends on nothing but its own accumulators); the fast divide
+              // returns 0 once the denominator passes 2^126, where the exact
+              // quotient is below 1e-36.
+              const float h0 = __fdividef(g0, 1.0f + __expf(-g0)) * __uint_as_float(r3[2 * j]);
+              const float h1 = __fdividef(g1, 1.0f + __expf(-g1)) * __uint_as_float(r3[2 * j + 1]);
+              const __nv_bfloat162 hb = __floats2bfloat162_rn(h0, h1);
+              hp[cc * 8 + j] = *reinterpret_cast<const uint32_t*>(&hb);
             }
           }
           if (cc == BN_MAX / 64 - 1 && wide) release_half(0u);   // token columns 0..127 drained

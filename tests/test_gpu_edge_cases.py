@@ -188,14 +188,14 @@ def test_non_finite_token_gets_valid_expert_ids(name, bad):
     keep = torch.as_tensor(others, device="cuda")
     assert torch.equal(got["gate"][keep], clean["gate"][keep])
     # The whole block: the bad row stays in its own outputs. Every other
-    # token's output is finite and matches the clean input's within the bf16
-    # output bound (the bad token's expert choice moves other tokens to other
-    # packed rows, and the SiLU epilogue shares one reciprocal among four
-    # neighbouring token columns, so the last bits may differ).
+    # token's output is finite and bitwise that of the clean input: the bad
+    # token's expert choice moves other tokens to other packed rows, but each
+    # output element depends only on its own token's row (no step mixes
+    # neighbouring tokens' values, not even in rounding).
     y_bad = H.gpu_forward(cfg, inp)
     x_clean = inp["x"].clone()
     x_clean[5] = H.gpu_inputs(cfg)["x"][5]
     inp["x"] = x_clean
     y_clean = H.gpu_forward(cfg, inp)
     assert torch.isfinite(y_bad[keep].float()).all().item()
-    H.compare_outputs(cfg, H.f64(y_bad[keep]), H.f64(y_clean[keep]), "other tokens' outputs")
+    assert torch.equal(y_bad[keep], y_clean[keep])
