@@ -194,11 +194,17 @@ const int* route_tile_base(const moe_config& c, void* ws) {
 // tile of an expert streams that expert's weights once more, so tiles are as
 // wide as the MMA allows (256) unless experts see only a handful of tokens
 // (decode), where a narrow tile leaves shared memory for deeper pipelining.
-// Slots in flight per CTA. With wide token tiles every slot also carries
-// L2-resident token rows, and measurements on B200 (DeepSeek-V3 shape) show
-// more than three outstanding weight slots slowing those loads down; narrow
-// tiles (decode) carry almost only weights and gain from a deeper queue.
-int inflight_for(int bn) { return bn >= 128 ? 3 : 8; }
+// Slots in flight per CTA. Narrow token tiles (decode) carry almost only
+// weights and gain from a deep queue (8). Wide tiles also carry L2-resident
+// token rows in every slot: with few tokens per expert (at most 256 on
+// average, weight streaming that waits on HBM latency) a fourth slot measured
+// 1% faster on the DeepSeek-V3 shape; with many (Mixtral: 1024 per expert,
+// tensor-bound tiles) it measured 5% slower, so three stay there.
+int inflight_for(int bn, double tokens_per_expert = 1e9) {
+  if (bn < 128) return 8;
+  return tokens_per_expert <= 256.0 ? 4 : 3;
+}
+double tokens_per_expert(const moe_config& c) { return (double)c.T * c.k / c.E; }
 
 int expert_tile_n(const moe_config& c) {
   const double m = (double)c.T * c.k / c.E;
@@ -225,7 +231,7 @@ moe_status enqueue_gate_up(const moe_config& c, const void* x_perm, const int* o
     g.m_rows_s = c.f_shared;
     g.K_s = c.d;
     g.bn_max = expert_tile_n(c);
-    g.max_inflight = inflight_for(g.bn_max);
+    g.max_inflight = inflight_for(g.bn_max, tokens_per_expert(c));
     g.a = w1; g.a3 = w3; g.b = x_perm;
     g.a_rows_total = (long long)c.E * c.f;
     g.b_rows_total = rows;
@@ -280,7 +286,7 @@ moe_status enqueue_down(const moe_config& c, const void* h, const int* offsets, 
     q.m_rows_s = c.d;
     q.K_s = c.f_shared;
     q.bn_max = expert_tile_n(c);
-    q.max_inflight = inflight_for(q.bn_max);
+    q.max_inflight = inflight_for(q.bn_max, tokens_per_expert(c));
     q.a = w2; q.b = h;
     q.a_rows_total = (long long)c.E * c.d;
     q.b_rows_total = rows;

@@ -49,7 +49,7 @@ __global__ void __launch_bounds__(1024, 1) router_topk_kernel(RouteParams p) {
     const TopkArgs a = {E, k, p.gate_mode, p.n_groups, p.topk_groups, p.route_scale, p.bias};
     int my_e, pos;
     float gate;
-    route_token<NPL>(lg, lane, a, my_e, pos, gate);
+    route_token<NPL>(lg, lane, a, my_e, pos, gate, lrow);
     if (lane < k) {
       p.topk_idx[(size_t)t * k + pos] = my_e;
       p.topk_gate[(size_t)t * k + pos] = gate;

@@ -22,10 +22,30 @@
 namespace moe {
 
 __device__ __forceinline__ float route_sigmoid(float l) { return 1.0f / (1.0f + expf(-l)); }
+// The same with the fast exponential and divide (a few ulp): used for the
+// selection scores only, where it is far below the fp32 logits' own error;
+// the gates use route_sigmoid. Large |l| saturate to 0 and 1 as they should.
+__device__ __forceinline__ float select_sigmoid(float l) { return __fdividef(1.0f, 1.0f + __expf(-l)); }
 
+// An fp32 score as an unsigned key with the same order: a > b exactly when
+// key(a) > key(b), for every non-NaN pair (-0 is folded into +0 first, since
+// the two compare equal). Keys of real scores, -inf included, are > 0, so 0
+// can mark "no candidate". A warp can then reduce scores with the hardware
+// integer reductions (redux.sync) instead of shuffle trees.
+__device__ __forceinline__ uint32_t score_key(float v) {
+  const uint32_t u = __float_as_uint(v == 0.0f ? 0.0f : v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_score(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// `lrow` holds the same logits in memory, [E] for this token; with more than
+// 256 experts (NPL > 8) the winners' logits are read back from it rather
+// than kept in registers, and it must not be null.
 template <int NPL>
 __device__ __forceinline__ void route_token(const float (&lg)[NPL], int lane, const TopkArgs& p, int& my_e,
-                                            int& pos, float& gate) {
+                                            int& pos, float& gate, const float* lrow = nullptr) {
   constexpr unsigned kFull = 0xffffffffu;
   const int E = p.E, k = p.k;
   float v[NPL];                      // biased selection score b' = s + bias
@@ -34,7 +54,7 @@ __device__ __forceinline__ void route_token(const float (&lg)[NPL], int lane, co
     const int e = lane + 32 * i;
     float b = -INFINITY;
     if (e < E) {
-      const float s = (p.gate_mode == MOE_GATE_SIGMOID) ? route_sigmoid(lg[i]) : lg[i];
+      const float s = (p.gate_mode == MOE_GATE_SIGMOID) ? select_sigmoid(lg[i]) : lg[i];
       b = s + (p.bias ? p.bias[e] : 0.0f);
       // A NaN score (NaN or infinite input, NaN bias) ranks below every
       // number, so it can neither win over a real score nor lose every
@@ -46,29 +66,56 @@ __device__ __forceinline__ void route_token(const float (&lg)[NPL], int lane, co
 
   if (p.n_groups > 1) {
     // Group score = sum of the two largest b' of the group; lane G ends up
-    // holding group G's score.
+    // holding group G's score. Each held expert's group is worked out once.
     const int gsz = E / p.n_groups;
+    // Group of held expert i (-1 past E): kept in registers for up to 256
+    // experts, recomputed where more experts would crowd the registers.
+    constexpr bool kKeepGid = NPL <= 8;
+    constexpr int kGidRegs = kKeepGid ? NPL : 1;
+    int gid_reg[kGidRegs];
+#pragma unroll
+    for (int i = 0; i < kGidRegs; ++i) {
+      const int e = lane + 32 * i;
+      gid_reg[i] = e < E ? e / gsz : -1;
+    }
+    auto gid = [&](int i) -> int {
+      if (kKeepGid) return gid_reg[i];
+      const int e = lane + 32 * i;
+      return e < E ? e / gsz : -1;
+    };
     float my_gscore = -INFINITY;
+    if (gsz == 32 && p.n_groups == NPL) {
+      // Groups of 32: lane l holds exactly one expert of group G (l + 32 G),
+      // so the group's two largest are the two largest lane values.
+#pragma unroll
+      for (int G = 0; G < NPL; ++G) {
+        const uint32_t k1 = score_key(v[G]);
+        const uint32_t g1 = __reduce_max_sync(kFull, k1);
+        const unsigned at_max = __ballot_sync(kFull, k1 == g1);
+        const uint32_t g2 = __popc(at_max) > 1 ? g1 : __reduce_max_sync(kFull, k1 == g1 ? 0u : k1);
+        const float gs = key_score(g1) + key_score(g2);
+        if (lane == G) my_gscore = isnan(gs) ? -INFINITY : gs;
+      }
+    } else
     for (int G = 0; G < p.n_groups; ++G) {
+      // This lane's two largest b' of group G, then the group's: its largest
+      // is the largest lane maximum; its second is that again when two lanes
+      // hold it, else the larger of that lane's second and every other
+      // lane's maximum.
       float m1 = -INFINITY, m2 = -INFINITY;
 #pragma unroll
       for (int i = 0; i < NPL; ++i) {
-        const int e = lane + 32 * i;
-        if (e < E && e / gsz == G) {
+        if (gid(i) == G) {
           const float x = v[i];
           if (x > m1) { m2 = m1; m1 = x; } else if (x > m2) { m2 = x; }
         }
       }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float o1 = __shfl_xor_sync(kFull, m1, off);
-        const float o2 = __shfl_xor_sync(kFull, m2, off);
-        const float hi = fmaxf(m1, o1);
-        const float lo = fmaxf(fminf(m1, o1), fmaxf(m2, o2));
-        m1 = hi;
-        m2 = lo;
-      }
-      if (lane == G) my_gscore = isnan(m1 + m2) ? -INFINITY : m1 + m2;   // +inf + -inf
+      const uint32_t k1 = score_key(m1), k2 = score_key(m2);
+      const uint32_t g1 = __reduce_max_sync(kFull, k1);
+      const unsigned at_max = __ballot_sync(kFull, k1 == g1);
+      const uint32_t g2 = __popc(at_max) > 1 ? g1 : __reduce_max_sync(kFull, k1 == g1 ? k2 : k1);
+      const float gs = key_score(g1) + key_score(g2);
+      if (lane == G) my_gscore = isnan(gs) ? -INFINITY : gs;   // +inf + -inf
     }
     // Keep the topk_groups best groups; ties go to the lower group index.
     int rank = 0;
@@ -78,10 +125,8 @@ __device__ __forceinline__ void route_token(const float (&lg)[NPL], int lane, co
     }
     const unsigned kept = __ballot_sync(kFull, lane < p.n_groups && rank < p.topk_groups);
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !((kept >> (e / gsz)) & 1u)) v[i] = -INFINITY;
-    }
+    for (int i = 0; i < NPL; ++i)
+      if (gid(i) >= 0 && !((kept >> gid(i)) & 1u)) v[i] = -INFINITY;
   }
 
   // k rounds of a warp arg-max: largest b' first, equal b' to the lower id.
@@ -102,13 +147,11 @@ __device__ __forceinline__ void route_token(const float (&lg)[NPL], int lane, co
         if (be == kNone || v[i] > bv || (v[i] == bv && e < be)) { bv = v[i]; be = e; }
       }
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ov = __shfl_xor_sync(kFull, bv, off);
-      const int oe = __shfl_xor_sync(kFull, be, off);
-      if (oe != kNone && (be == kNone || ov > bv || (ov == bv && oe < be))) { bv = ov; be = oe; }
-    }
-    if (be == kNone) be = 0;         // unreachable (k <= E); keeps the id in range regardless
+    // The warp's largest candidate score, then the lowest id holding it.
+    const uint32_t key = be == kNone ? 0u : score_key(bv);
+    const uint32_t best = __reduce_max_sync(kFull, key);
+    be = (int)__reduce_min_sync(kFull, (key == best && be != kNone) ? (uint32_t)be : 0xffffffffu);
+    if (be < 0 || be >= E) be = 0;   // unreachable (k <= E); keeps the id in range regardless
     if ((be & 31) == lane) taken |= 1u << (be >> 5);
     if (lane == r) my_e = be;
   }
@@ -119,14 +162,20 @@ __device__ __forceinline__ void route_token(const float (&lg)[NPL], int lane, co
     const int o = __shfl_sync(kFull, my_e, j);
     if (o < my_e) ++pos;
   }
-  // The unbiased logit of each winner, from the lane that holds it.
+  // The unbiased logit of each winner, from the lane that holds it (or from
+  // memory, once every lane's stores are visible to the warp).
   const bool act = lane < k;
-  const int src = act ? (my_e & 31) : lane, slot = act ? (my_e >> 5) : 0;
   float l = 0.0f;
+  if (NPL > 8) {             // callers with more than 256 experts pass lrow
+    __syncwarp();
+    if (act) l = lrow[my_e];
+  } else {
+    const int src = act ? (my_e & 31) : lane, slot = act ? (my_e >> 5) : 0;
 #pragma unroll
-  for (int i = 0; i < NPL; ++i) {
-    const float o = __shfl_sync(kFull, lg[i], src);
-    if (slot == i) l = o;
+    for (int i = 0; i < NPL; ++i) {
+      const float o = __shfl_sync(kFull, lg[i], src);
+      if (slot == i) l = o;
+    }
   }
   // Gates from the UNBIASED value of each winner.
   float num;

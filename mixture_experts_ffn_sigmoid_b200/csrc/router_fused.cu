@@ -89,6 +89,7 @@ __global__ void __launch_bounds__(FR_THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   volatile int* s_last = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  volatile int* s_ok = reinterpret_cast<volatile int*>(tmem_slot + 3);
   int* s_warp = reinterpret_cast<int*>(tmem_slot + 4);          // [32]
   uint8_t* ring = smem + FR_HDR;
   const int stage_bytes = fr_stage_bytes(p.n_pad);
@@ -175,12 +176,14 @@ __global__ void __launch_bounds__(FR_THREADS, 1)
       else mbar_arrive(smem_u32(done_bar));
     }
     __syncwarp();
+  } else if (warp == 2 && lane == 0) {
+    // One thread waits for the MMAs; the other threads wait in the block
+    // barrier below instead of polling the mbarrier.
+    *s_ok = wait_bounded(smem_u32(done_bar), 0u, abort_flag, p.err, p.timeout_ns, false) ? 1 : 0;
   }
-  __syncwarp();
-  const bool ok = __all_sync(0xffffffffu,
-                             wait_bounded(smem_u32(done_bar), 0u, abort_flag, p.err, p.timeout_ns, false));
+  __syncthreads();      // MMAs complete, and the producer's copies have landed: the ring may be overwritten
   tc_fence_after();
-  __syncthreads();      // the producer's copies have landed: the ring may be overwritten
+  const bool ok = *s_ok != 0;
   // TMEM -> shared memory: warp w reads lane quarter w & 3 (32 tokens) and
   // 32 columns starting at 32 * (w >> 2).
   {
@@ -223,19 +226,24 @@ __global__ void __launch_bounds__(FR_THREADS, 1)
     const int tl = j * kChunk + warp;       // token of the tile this warp routes
     const int t = t0 + tl;
     if (t < p.T) {                          // warp-uniform
+      // Partial sums of the NPL held experts, CTA by CTA in rank order; the
+      // NPL loads of one CTA are issued back to back.
       float lg[NPL];
+      const uint32_t row = smem_u32(s_log + tl * ld_log + lane);
+      for (uint32_t q = 0; q < S; ++q) {
+        const uint32_t base = map_to_cta(row, q);
+        float part[NPL];
 #pragma unroll
-      for (int i = 0; i < NPL; ++i) {
-        const int e = lane + 32 * i;
-        float l = 0.0f;
-        if (e < E) {
-          const uint32_t a = smem_u32(s_log + tl * ld_log + e);
-          l = ld_cluster_f32(map_to_cta(a, 0));
-          for (uint32_t q = 1; q < S; ++q) l += ld_cluster_f32(map_to_cta(a, q));
-          p.logits[(size_t)t * E + e] = l;
-        }
-        lg[i] = l;
+        for (int i = 0; i < NPL; ++i) part[i] = lane + 32 * i < E ? ld_cluster_f32(base + 128u * i) : 0.0f;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) lg[i] = q == 0 ? part[i] : lg[i] + part[i];
       }
+      // The sums replace this CTA's own partials of the token (only this CTA
+      // reads its own chunks' rows), to be copied out after the handshake.
+      float* own = s_log + tl * ld_log;
+#pragma unroll
+      for (int i = 0; i < NPL; ++i)
+        if (lane + 32 * i < E) own[lane + 32 * i] = lg[i];
       int my_e, pos;
       float gate;
       route_token<NPL>(lg, lane, p.topk, my_e, pos, gate);
@@ -262,7 +270,21 @@ __global__ void __launch_bounds__(FR_THREADS, 1)
     }
   }
   cluster_sync_all();   // CTA 0 has read its peers' masks: they may exit
-  if (rank != 0) return;
+
+  // The summed logits of this CTA's chunks ([T][E] fp32, kept for the
+  // backward pass), one warp per token row. CTA 0 first makes its tile
+  // histogram visible, so that its fence waits on those few stores only.
+  auto store_logits = [&]() {
+    for (int j = (int)rank; j < nch_tile; j += (int)S) {
+      const int tl = j * kChunk + warp, t = t0 + tl;
+      if (t < p.T)
+        for (int e = lane; e < E; e += 32) p.logits[(size_t)t * E + e] = s_log[tl * ld_log + e];
+    }
+  };
+  if (rank != 0) {
+    store_logits();
+    return;
+  }
 
   // ------------------------------------------------------------ last tile: scan
   __threadfence();      // this CTA's chunk bases and tile histogram before its arrival
@@ -272,6 +294,7 @@ __global__ void __launch_bounds__(FR_THREADS, 1)
     *s_last = prev == (uint32_t)(p.ntiles - 1) ? 1 : 0;
   }
   __syncthreads();
+  store_logits();
   if (!*s_last) return;
   __threadfence();
   // Four groups of 256 threads, each over a quarter of the tiles: its partial
