@@ -129,8 +129,12 @@ class ClockSampler:
         mask = n.nvmlDeviceGetCurrentClocksEventReasons(h)
         bits = (n.nvmlClocksEventReasonHwSlowdown, n.nvmlClocksEventReasonHwThermalSlowdown,
                 n.nvmlClocksEventReasonSwThermalSlowdown, n.nvmlClocksEventReasonSwPowerCap)
+        try:   # the memory clock, when this NVML reports it
+            mem = n.nvmlDeviceGetClockInfo(h, n.NVML_CLOCK_MEM)
+        except Exception:
+            mem = ""
         return [str(sm), str(mx), f"{watts:.2f}", hex(mask)] + \
-            ["Active" if mask & b else "Not Active" for b in bits]
+            ["Active" if mask & b else "Not Active" for b in bits] + [str(mem)]
 
     def _start_nvml(self):
         try:
@@ -216,9 +220,11 @@ class ClockSampler:
         sm = [num(r[0]) for r in rows if num(r[0]) is not None]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if len(r) > 4 + i and r[4 + i] == "Active"})
+        mem = [num(r[8]) for r in rows if len(r) > 8 and num(r[8]) is not None]
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": num(rows[0][1]), "reasons": reasons, "samples": len(rows), "window": window,
-                "source": self.source, "power_w_max": max((num(r[2]) or 0.0) for r in rows)}
+                "source": self.source, "power_w_max": max((num(r[2]) or 0.0) for r in rows),
+                "mem_mhz": statistics.median(mem) if mem else None}
 
 
 # ------------------------------------------------------- multi-rank timing
@@ -744,6 +750,19 @@ def main():
         if world > 1:
             torch.distributed.destroy_process_group()
         return
+    # ---- the pages' other workloads (one GPU only): each on its own inputs,
+    # CUDA-graph step, stage times, binding-roof fraction, its own clocks. They
+    # run right after the headline's own timing, before the long backward and
+    # end-to-end measurements heat the GPU. ---------------------------------------
+    peaks = measured_peaks()
+    extra = None
+    if world == 1 and not args.no_extra_workloads and args.T is None and args.E is None and args.f is None:
+        from mixture_experts_ffn_sigmoid_b200.inputs import CONFIGS
+        extra = {}
+        for name in CONFIGS:
+            if name != cfg.name:
+                extra[name] = measure_workload(B, name, dev, stream, max(3, min(args.steps, 50)), args.warmup,
+                                               sampler, peaks)
     fused = measure_fused_permute(B, cfg, inp, idx, offsets, perm_src, inv_row, h, h_s, ws, stream,
                                   n_stage) if cfg.dtype == "bf16" else None
     if fused is not None:
@@ -773,7 +792,6 @@ def main():
                "ln_E": math.log(E), "gamma": 0.15, "bound": "launch latency (E-element kernel)"}
     gelu = measure_gelu_experts(B, cfg, inp, counts.cpu(), stream, max(3, min(args.steps, 20)))
     work, touched = stage_work(cfg, counts.cpu())
-    peaks = measured_peaks()
     gelu["expert_weight_frac_hbm"] = gelu["expert_weight_gbs"] / peaks["hbm"]
     bwd = measure_backward(B, cfg, inp, touched, stream, max(3, min(args.steps, 10)))
     bwd["frac_tensor"] = bwd["tflops"] / peaks["tensor_sustained"]
@@ -857,18 +875,6 @@ def main():
                "sample": f"{n} seeded tokens of {cfg.name}: fp64 routing over all {E} experts and the "
                          f"FFN of each selected and shared expert ({dt:.1f} s)"}
 
-    # ---- the pages' other workloads (one GPU only): each on its own inputs,
-    # CUDA-graph step, stage times, binding-roof fraction, its own clocks -------
-    extra = None
-    if world == 1 and not args.no_extra_workloads and args.T is None and args.E is None and args.f is None:
-        from mixture_experts_ffn_sigmoid_b200.inputs import CONFIGS
-        del x_host, y_host, x_dev, y_dev
-        torch.cuda.empty_cache()
-        extra = {}
-        for name in CONFIGS:
-            if name != cfg.name:
-                extra[name] = measure_workload(B, name, dev, stream, max(3, min(args.steps, 50)), args.warmup,
-                                               sampler, peaks)
     sampler.stop()
 
     if rank == 0:

@@ -23,8 +23,9 @@ namespace moe {
 
 __device__ __forceinline__ float route_sigmoid(float l) { return 1.0f / (1.0f + expf(-l)); }
 // The same with the fast exponential and divide (a few ulp): used for the
-// selection scores only, where it is far below the fp32 logits' own error;
-// the gates use route_sigmoid. Large |l| saturate to 0 and 1 as they should.
+// selection scores of up to 256 experts, where it is far below the fp32
+// logits' own error; the gates use route_sigmoid. Large |l| saturate to 0
+// and 1 as they should.
 __device__ __forceinline__ float select_sigmoid(float l) { return __fdividef(1.0f, 1.0f + __expf(-l)); }
 
 // An fp32 score as an unsigned key with the same order: a > b exactly when
@@ -54,7 +55,8 @@ __device__ __forceinline__ void route_token(const float (&lg)[NPL], int lane, co
     const int e = lane + 32 * i;
     float b = -INFINITY;
     if (e < E) {
-      const float s = (p.gate_mode == MOE_GATE_SIGMOID) ? select_sigmoid(lg[i]) : lg[i];
+      const float s = (p.gate_mode == MOE_GATE_SIGMOID) ? (NPL <= 8 ? select_sigmoid(lg[i]) : route_sigmoid(lg[i]))
+                                                        : lg[i];
       b = s + (p.bias ? p.bias[e] : 0.0f);
       // A NaN score (NaN or infinite input, NaN bias) ranks below every
       // number, so it can neither win over a real score nor lose every
@@ -84,7 +86,7 @@ __device__ __forceinline__ void route_token(const float (&lg)[NPL], int lane, co
       return e < E ? e / gsz : -1;
     };
     float my_gscore = -INFINITY;
-    if (gsz == 32 && p.n_groups == NPL) {
+    if (NPL <= 8 && gsz == 32 && p.n_groups == NPL) {
       // Groups of 32: lane l holds exactly one expert of group G (l + 32 G),
       // so the group's two largest are the two largest lane values.
 #pragma unroll
@@ -129,6 +131,55 @@ __device__ __forceinline__ void route_token(const float (&lg)[NPL], int lane, co
       if (gid(i) >= 0 && !((kept >> gid(i)) & 1u)) v[i] = -INFINITY;
   }
 
+  if constexpr (NPL <= 8) {
+    // Each lane sorts its (b', id) pairs once, best first (larger b', then
+    // the lower id; ids past E last), and each of the k rounds looks at the
+    // lanes' heads only: the warp's largest head score, then the lowest id
+    // holding it, and the winning lane shifts its list by one. A lane's head
+    // is its best untaken expert, so the winners are those of a full rescan.
+    constexpr int kNoId = 0x7fffffff;
+    float sv[NPL];
+    int se[NPL];
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      const int e = lane + 32 * i;
+      sv[i] = e < E ? v[i] : -INFINITY;
+      se[i] = e < E ? e : kNoId;
+    }
+    auto cmp_swap = [&](int a, int b) {   // after it, position a holds the better pair
+      const bool b_first = se[b] != kNoId && (se[a] == kNoId || sv[b] > sv[a] || (sv[b] == sv[a] && se[b] < se[a]));
+      const float fv = b_first ? sv[b] : sv[a], gv = b_first ? sv[a] : sv[b];
+      const int fe = b_first ? se[b] : se[a], ge = b_first ? se[a] : se[b];
+      sv[a] = fv; sv[b] = gv; se[a] = fe; se[b] = ge;
+    };
+    if constexpr (NPL == 2) {
+      cmp_swap(0, 1);
+    } else if constexpr (NPL == 4) {
+      cmp_swap(0, 1); cmp_swap(2, 3); cmp_swap(0, 2); cmp_swap(1, 3); cmp_swap(1, 2);
+    } else if constexpr (NPL == 8) {   // Batcher's odd-even merge sort of 8
+      cmp_swap(0, 1); cmp_swap(2, 3); cmp_swap(4, 5); cmp_swap(6, 7);
+      cmp_swap(0, 2); cmp_swap(1, 3); cmp_swap(4, 6); cmp_swap(5, 7);
+      cmp_swap(1, 2); cmp_swap(5, 6);
+      cmp_swap(0, 4); cmp_swap(1, 5); cmp_swap(2, 6); cmp_swap(3, 7);
+      cmp_swap(2, 4); cmp_swap(3, 5);
+      cmp_swap(1, 2); cmp_swap(3, 4); cmp_swap(5, 6);
+    }
+    my_e = -1;
+    for (int r = 0; r < k; ++r) {
+      const bool has = se[0] != kNoId;
+      const uint32_t key = has ? score_key(sv[0]) : 0u;
+      const uint32_t best = __reduce_max_sync(kFull, key);
+      int be = (int)__reduce_min_sync(kFull, (has && key == best) ? (uint32_t)se[0] : 0xffffffffu);
+      if (be < 0 || be >= E) be = 0;   // unreachable (k <= E); keeps the id in range regardless
+      if (has && se[0] == be) {        // this lane's head won: drop it
+#pragma unroll
+        for (int i = 0; i + 1 < NPL; ++i) { sv[i] = sv[i + 1]; se[i] = se[i + 1]; }
+        sv[NPL - 1] = -INFINITY;
+        se[NPL - 1] = kNoId;
+      }
+      if (lane == r) my_e = be;
+    }
+  } else {
   // k rounds of a warp arg-max: largest b' first, equal b' to the lower id.
   // kNone marks "no candidate yet": the first untaken in-range expert a lane
   // sees always becomes its candidate, and a real candidate always beats
@@ -154,6 +205,7 @@ __device__ __forceinline__ void route_token(const float (&lg)[NPL], int lane, co
     if (be < 0 || be >= E) be = 0;   // unreachable (k <= E); keeps the id in range regardless
     if ((be & 31) == lane) taken |= 1u << (be >> 5);
     if (lane == r) my_e = be;
+  }
   }
 
   // Winners in ascending expert id.

@@ -18,11 +18,11 @@
 // partial logits from TMEM into the CTA's shared memory (over the ring,
 // which is no longer needed), and after a cluster barrier the CTAs add the
 // S partial sums through distributed shared memory in rank order (a fixed
-// order: the logits are the same bits on every run). The tile's four
-// 32-token chunks are shared among the CTAs; in each, warp w routes token w
-// and the chunk's per-expert bit mask records which tokens chose each
-// expert. CTA 0 turns the four masks into each chunk's base within the tile
-// and the tile's histogram. The last tile to finish (a device-wide counter)
+// order: the logits are the same bits on every run). The tile's tokens are
+// shared among the CTAs' warps (one warp per token, token tl on CTA tl % S),
+// and per-expert bit masks record which tokens of each 32-token chunk chose
+// each expert. CTA 0 ORs the CTAs' masks and turns them into each chunk's
+// base within the tile and the tile's histogram. The last tile to finish (a device-wide counter)
 // scans the tile histograms into each tile's base, the per-expert counts
 // and the offsets. A token's packed row is then
 //   offsets[e] + tile_base[tile][e] + chunk_base[chunk][e] + (earlier tokens
@@ -220,12 +220,17 @@ __global__ void __launch_bounds__(FR_THREADS, 1)
   cluster_sync_all();   // every CTA's partial logits are in its shared memory
 
   // ------------------------------------------------------------ routing
+  // Token tl of the tile is routed by CTA tl % S, warp (tl / S) % 32, so a
+  // short tile (decode) spreads its tokens over every CTA of the cluster
+  // rather than queueing them on one SM. Each CTA records, per chunk, which
+  // of the tokens it routed chose each expert; CTA 0 ORs those masks below.
   const int nch_tile = min(kTileChunks, ceil_div(p.T - t0, kChunk));
+  const int tile_tokens = min(FR_BM, p.T - t0);
   const int k = p.topk.k;
-  for (int j = (int)rank; j < nch_tile; j += (int)S) {
-    const int tl = j * kChunk + warp;       // token of the tile this warp routes
+  for (int tl = (int)rank + (int)S * warp; tl < tile_tokens; tl += (int)S * 32) {
     const int t = t0 + tl;
-    if (t < p.T) {                          // warp-uniform
+    const int j = tl / kChunk;
+    {   // one warp, one token
       // Partial sums of the NPL held experts, CTA by CTA in rank order; the
       // NPL loads of one CTA are issued back to back.
       float lg[NPL];
@@ -238,8 +243,9 @@ __global__ void __launch_bounds__(FR_THREADS, 1)
 #pragma unroll
         for (int i = 0; i < NPL; ++i) lg[i] = q == 0 ? part[i] : lg[i] + part[i];
       }
-      // The sums replace this CTA's own partials of the token (only this CTA
-      // reads its own chunks' rows), to be copied out after the handshake.
+      // The sums replace this CTA's own partials of the token (a token's
+      // rows are read only by the CTA that routes it), to be copied out after
+      // the handshake.
       float* own = s_log + tl * ld_log;
 #pragma unroll
       for (int i = 0; i < NPL; ++i)
@@ -250,7 +256,7 @@ __global__ void __launch_bounds__(FR_THREADS, 1)
       if (lane < k) {
         p.topk_idx[(size_t)t * k + pos] = my_e;
         p.topk_gate[(size_t)t * k + pos] = gate;
-        atomicOr(&s_mask[j * 256 + my_e], 1u << warp);
+        atomicOr(&s_mask[j * 256 + my_e], 1u << (tl % kChunk));
       }
     }
   }
@@ -262,7 +268,9 @@ __global__ void __launch_bounds__(FR_THREADS, 1)
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
       int run = 0;
       for (int j = 0; j < nch_tile; ++j) {
-        const uint32_t m = ld_cluster_u32(map_to_cta(smem_u32(&s_mask[j * 256 + e]), (uint32_t)j % S));
+        const uint32_t a = smem_u32(&s_mask[j * 256 + e]);
+        uint32_t m = 0u;
+        for (uint32_t q = 0; q < S; ++q) m |= ld_cluster_u32(map_to_cta(a, q));
         p.chunk_base[(size_t)(tile * kTileChunks + j) * E + e] = run;
         run += __popc(m);
       }
@@ -271,15 +279,13 @@ __global__ void __launch_bounds__(FR_THREADS, 1)
   }
   cluster_sync_all();   // CTA 0 has read its peers' masks: they may exit
 
-  // The summed logits of this CTA's chunks ([T][E] fp32, kept for the
-  // backward pass), one warp per token row. CTA 0 first makes its tile
-  // histogram visible, so that its fence waits on those few stores only.
+  // The summed logits of the tokens this CTA routed ([T][E] fp32, kept for
+  // the backward pass), one warp per token row. CTA 0 first publishes its
+  // tile histogram (and, on the last tile, runs the scan), so neither waits
+  // on these stores.
   auto store_logits = [&]() {
-    for (int j = (int)rank; j < nch_tile; j += (int)S) {
-      const int tl = j * kChunk + warp, t = t0 + tl;
-      if (t < p.T)
-        for (int e = lane; e < E; e += 32) p.logits[(size_t)t * E + e] = s_log[tl * ld_log + e];
-    }
+    for (int tl = (int)rank + (int)S * warp; tl < tile_tokens; tl += (int)S * 32)
+      for (int e = lane; e < E; e += 32) p.logits[(size_t)(t0 + tl) * E + e] = s_log[tl * ld_log + e];
   };
   if (rank != 0) {
     store_logits();
@@ -287,15 +293,20 @@ __global__ void __launch_bounds__(FR_THREADS, 1)
   }
 
   // ------------------------------------------------------------ last tile: scan
-  __threadfence();      // this CTA's chunk bases and tile histogram before its arrival
+  // The block barrier orders every thread's chunk bases and tile-histogram
+  // stores before thread 0's fence (a cumulative gpu-scope fence), which
+  // orders them before the counter increment that publishes them.
   __syncthreads();
   if (threadIdx.x == 0) {
+    __threadfence();
     const uint32_t prev = atomicAdd(p.done_count, 1u);
     *s_last = prev == (uint32_t)(p.ntiles - 1) ? 1 : 0;
   }
   __syncthreads();
-  store_logits();
-  if (!*s_last) return;
+  if (!*s_last) {
+    store_logits();
+    return;
+  }
   __threadfence();
   // Four groups of 256 threads, each over a quarter of the tiles: its partial
   // per-expert sums, then each tile's base from the groups before it.
@@ -340,6 +351,7 @@ __global__ void __launch_bounds__(FR_THREADS, 1)
       *p.done_count = 0u;   // ready for the next launch
     }
   }
+  store_logits();
 }
 
 }  // namespace

@@ -22,6 +22,7 @@ def fake_nvml(mask, init_fails=False, sm_mhz=1965):
     calls = {"handle_uuid": None, "shutdown": 0}
     m = types.ModuleType("pynvml")
     m.NVML_CLOCK_SM = 1
+    m.NVML_CLOCK_MEM = 2
     m.nvmlClocksEventReasonHwSlowdown = HW_SLOWDOWN
     m.nvmlClocksEventReasonHwThermalSlowdown = HW_THERMAL
     m.nvmlClocksEventReasonSwThermalSlowdown = SW_THERMAL
@@ -40,7 +41,7 @@ def fake_nvml(mask, init_fails=False, sm_mhz=1965):
         calls["handle_uuid"] = u
         return "handle"
     m.nvmlDeviceGetHandleByUUID = by_uuid
-    m.nvmlDeviceGetClockInfo = lambda h, t: sm_mhz
+    m.nvmlDeviceGetClockInfo = lambda h, t: sm_mhz if t == m.NVML_CLOCK_SM else 3996
     m.nvmlDeviceGetMaxClockInfo = lambda h, t: 1965
     m.nvmlDeviceGetPowerUsage = lambda h: 987_000   # milliwatts
     m.nvmlDeviceGetCurrentClocksEventReasons = lambda h: mask
@@ -69,6 +70,7 @@ def test_nvml_samples_during_the_timed_region(monkeypatch, fake_device):
     s, summ = run_sampler(monkeypatch, mod)
     assert calls["handle_uuid"] == b"GPU-" + UUID.encode() or calls["handle_uuid"] == "GPU-" + UUID
     assert summ["source"] == "nvml"
+    assert summ["mem_mhz"] == 3996
     assert summ["window"] == "timed region" and summ["samples"] >= 3
     assert summ["sm_mhz"] == 1650 and summ["sm_max_mhz"] == 1965
     assert summ["reasons"] == ["sw_power_cap"]
