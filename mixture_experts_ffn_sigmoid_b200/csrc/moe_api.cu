@@ -194,17 +194,13 @@ const int* route_tile_base(const moe_config& c, void* ws) {
 // tile of an expert streams that expert's weights once more, so tiles are as
 // wide as the MMA allows (256) unless experts see only a handful of tokens
 // (decode), where a narrow tile leaves shared memory for deeper pipelining.
-// Slots in flight per CTA. Narrow token tiles (decode) carry almost only
-// weights and gain from a deep queue (8). Wide tiles also carry L2-resident
-// token rows in every slot: with few tokens per expert (at most 256 on
-// average, weight streaming that waits on HBM latency) a fourth slot measured
-// 1% faster on the DeepSeek-V3 shape; with many (Mixtral: 1024 per expert,
-// tensor-bound tiles) it measured 5% slower, so three stay there.
-int inflight_for(int bn, double tokens_per_expert = 1e9) {
-  if (bn < 128) return 8;
-  return tokens_per_expert <= 256.0 ? 4 : 3;
-}
-double tokens_per_expert(const moe_config& c) { return (double)c.T * c.k / c.E; }
+// Slots in flight per CTA: four, so each SM keeps 4 x 32 KB of weight rows
+// (plus the slots' token rows) on the way. A read stream of TMA copies on
+// B200 peaks there (about 7.3 TB/s from HBM with 128 KB in flight per SM)
+// and loses throughput with more (6.6 TB/s at 192 KB); in the GEMMs four
+// measured faster than three, five or eight on the decode, DeepSeek-V3 and
+// Mixtral shapes alike.
+int inflight_for() { return 4; }
 
 int expert_tile_n(const moe_config& c) {
   const double m = (double)c.T * c.k / c.E;
@@ -231,7 +227,7 @@ moe_status enqueue_gate_up(const moe_config& c, const void* x_perm, const int* o
     g.m_rows_s = c.f_shared;
     g.K_s = c.d;
     g.bn_max = expert_tile_n(c);
-    g.max_inflight = inflight_for(g.bn_max, tokens_per_expert(c));
+    g.max_inflight = inflight_for();
     g.a = w1; g.a3 = w3; g.b = x_perm;
     g.a_rows_total = (long long)c.E * c.f;
     g.b_rows_total = rows;
@@ -286,7 +282,7 @@ moe_status enqueue_down(const moe_config& c, const void* h, const int* offsets, 
     q.m_rows_s = c.d;
     q.K_s = c.f_shared;
     q.bn_max = expert_tile_n(c);
-    q.max_inflight = inflight_for(q.bn_max, tokens_per_expert(c));
+    q.max_inflight = inflight_for();
     q.a = w2; q.b = h;
     q.a_rows_total = (long long)c.E * c.d;
     q.b_rows_total = rows;
@@ -342,7 +338,7 @@ moe_status enqueue_gelu_experts(const moe_config& c, const void* x_perm, const i
     g.m_rows = c.f;
     g.K = c.d;
     g.bn_max = expert_tile_n(c);
-    g.max_inflight = inflight_for(g.bn_max);
+    g.max_inflight = inflight_for();
     g.a = w1; g.a3 = w1; g.b = x_perm;
     g.a_rows_total = (long long)c.E * c.f;
     g.b_rows_total = rows;
@@ -460,7 +456,7 @@ moe_status enqueue_dgrad(const DgradArgs& a, int rows, uint32_t* err, cudaStream
   g.m_rows_s = a.m_rows_s;
   g.K_s = a.K_s;
   g.bn_max = a.bn;
-  g.max_inflight = inflight_for(a.bn);
+  g.max_inflight = inflight_for();
   g.a = a.w; g.a3 = a.w2nd; g.b = a.g;
   g.a_rows_total = (long long)a.n_routed * a.c_rows;
   g.b_rows_total = rows;
@@ -503,7 +499,7 @@ moe_status enqueue_preact(const moe_config& c, const void* x_perm, const int* of
       g.m_rows_s = c.f_shared;
       g.K_s = c.d;
       g.bn_max = expert_tile_n(c);
-      g.max_inflight = inflight_for(g.bn_max);
+      g.max_inflight = inflight_for();
       g.a = w; g.a3 = w; g.b = x_perm;
       g.a_rows_total = (long long)c.E * c.f;
       g.b_rows_total = rows;

@@ -69,9 +69,8 @@ constexpr int BM = 128;          // weight rows per MMA (M)
 constexpr int BK = 64;           // K per slot: one 128-byte swizzle row of bf16
 constexpr int UMMA_K = 16;       // K per tcgen05.mma for 16-bit inputs
 constexpr int BN_MAX = 256;      // token columns per tile (MMA N), upper bound
-constexpr int BOX_N = 32;        // token rows per TMA box
+constexpr int BOX_N_MAX = 128;   // token rows per TMA box, at most
 constexpr int A_BYTES = BM * BK * 2;
-constexpr int BOX_BYTES = BOX_N * BK * 2;
 constexpr int NUM_THREADS = 320;
 constexpr int EPI_WARPS = 8;      // warps 2..9: two per TMEM lane quarter
 constexpr int TMEM_COLS = 512;
@@ -221,6 +220,14 @@ __host__ __device__ constexpr int tile_rows(int mode, bool pair) {
   return (two_blocks(mode) ? 256 : 128) * (pair ? 2 : 1);
 }
 
+// The parameters as launched: the caller's, plus what the launcher derives.
+// Each TMA copy costs the issuing thread and the copy engine a fixed
+// overhead whatever its size, and a slot completes only when all of its
+// copies have, so a CTA's token rows of a slot come in one copy.
+struct UmmaLaunch : UmmaGemmParams {
+  int box_n;   // token rows per copy of B: a multiple of 8, at most 128
+};
+
 struct Tile {
   int seg, wt, tt;
   int rows;      // tokens in the segment
@@ -269,19 +276,21 @@ __device__ __forceinline__ Tile decode_tile(const UmmaGemmParams& p, const int* 
 // Token rows this CTA stages for a tile, and how many TMA boxes that takes.
 struct TokenSlice {
   int n_valid, n_mma, row, nbox;
-  int rows_gather;   // rows staged by gather4 (routed tiles of a gathered B), else 0
+  uint32_t box_bytes;   // bytes of one copy of B
+  int rows_gather;      // rows staged by gather4 (routed tiles of a gathered B), else 0
   __device__ __forceinline__ uint32_t bytes() const {
-    return rows_gather > 0 ? (uint32_t)rows_gather * (BK * 2) : (uint32_t)nbox * BOX_BYTES;
+    return rows_gather > 0 ? (uint32_t)rows_gather * (BK * 2) : (uint32_t)nbox * box_bytes;
   }
 };
 template <bool PAIR>
-__device__ __forceinline__ TokenSlice token_slice(const UmmaGemmParams& p, const Tile& t, uint32_t rank) {
+__device__ __forceinline__ TokenSlice token_slice(const UmmaLaunch& p, const Tile& t, uint32_t rank) {
   TokenSlice ts;
   ts.n_valid = min(p.bn_max, t.rows - t.tt * p.bn_max);
   ts.n_mma = (ts.n_valid + 15) & ~15;
   const int mine = PAIR ? ts.n_mma / 2 : ts.n_valid;
   ts.row = t.b_row0 + t.tt * p.bn_max + (PAIR ? (int)rank * (ts.n_mma / 2) : 0);
-  ts.nbox = (mine + BOX_N - 1) / BOX_N;
+  ts.nbox = (mine + p.box_n - 1) / p.box_n;
+  ts.box_bytes = (uint32_t)p.box_n * (BK * 2);
   // Gathered tiles stage exactly the rows the MMA reads (a multiple of 8).
   ts.rows_gather = (p.b_gather && !t.dense) ? (PAIR ? ts.n_mma / 2 : ts.n_mma) : 0;
   return ts;
@@ -292,7 +301,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA3,
                      const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmAs,
                      const __grid_constant__ CUtensorMap tmA3s, const __grid_constant__ CUtensorMap tmBs,
-                     const __grid_constant__ CUtensorMap tmG, const UmmaGemmParams p) {
+                     const __grid_constant__ CUtensorMap tmG, const UmmaLaunch p) {
   using KD = Kind<MODE>;
   constexpr int A_TILES = KD::A_TILES;
   constexpr int WROWS = tile_rows(MODE, PAIR);
@@ -477,7 +486,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                s_rows[g + 3], fb);
           } else {
             for (int bx = 0; bx < ts.nbox; ++bx)
-              tma_load_2d_pair(bb + bx * BOX_BYTES, mB, kb * BK, ts.row + bx * BOX_N, fb);
+              tma_load_2d_pair(bb + bx * ts.box_bytes, mB, kb * BK, ts.row + bx * p.box_n, fb);
           }
         } else {
           mbar_expect_tx(fb_local, bytes);
@@ -502,7 +511,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                           s_rows[g + 3], fb_local);
           } else {
             for (int bx = 0; bx < ts.nbox; ++bx)
-              tma_load_2d(bb + bx * BOX_BYTES, mB, kb * BK, ts.row + bx * BOX_N, fb_local);
+              tma_load_2d(bb + bx * ts.box_bytes, mB, kb * BK, ts.row + bx * p.box_n, fb_local);
           }
         }
       }
@@ -842,7 +851,7 @@ cudaError_t ensure_smem_attr() {
 template <int MODE, bool PAIR>
 cudaError_t launch_mode(const CUtensorMap& tA, const CUtensorMap& tA3, const CUtensorMap& tB,
                         const CUtensorMap& tAs, const CUtensorMap& tA3s, const CUtensorMap& tBs,
-                        const CUtensorMap& tG, const UmmaGemmParams& p, int grid, int smem,
+                        const CUtensorMap& tG, const UmmaLaunch& p, int grid, int smem,
                         cudaStream_t s) {
   cudaError_t e = ensure_smem_attr<MODE, PAIR>();
   if (e != cudaSuccess) return e;
@@ -879,7 +888,13 @@ cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t 
   // stay on single CTAs.
   const bool pair = p.bn_max >= 128 && num_sms >= 2;
   const int wrows = tile_rows(p.mode, pair);
-  if (sp.ring_bytes < 2 * (a_tiles * A_BYTES + ceil_div(p.bn_max, BOX_N) * BOX_BYTES))
+  UmmaLaunch q;
+  static_cast<UmmaGemmParams&>(q) = p;
+  // One copy of B per CTA and slot: a box as tall as the most token rows a
+  // CTA stages (rounded to the 8-row swizzle atom), at most 128 rows.
+  const int mine_max = pair ? p.bn_max / 2 : p.bn_max;
+  q.box_n = ((mine_max + 7) & ~7) < BOX_N_MAX ? ((mine_max + 7) & ~7) : BOX_N_MAX;
+  if (sp.ring_bytes < 2 * (a_tiles * A_BYTES + ceil_div(mine_max, q.box_n) * q.box_n * BK * 2))
     return cudaErrorInvalidValue;
   const bool swiglu = dual_a(p.mode);
   const bool dgrad = p.mode == kUmmaDgrad;
@@ -893,7 +908,7 @@ cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t 
       if (swiglu && !make_tmap(&tA3s, p.a3_s, p.K_s, p.m_rows_s, BM)) return cudaErrorInvalidValue;
       if (!swiglu) tA3s = tAs;
     }
-    if (!make_tmap(&tBs, p.b_s, p.K_s, p.shared_rows, BOX_N)) return cudaErrorInvalidValue;
+    if (!make_tmap(&tBs, p.b_s, p.K_s, p.shared_rows, q.box_n)) return cudaErrorInvalidValue;
   }
   if (p.n_routed > 0) {
     if (dgrad) {   // stacked weights [n_routed * a_k_rows][m_rows], m contiguous
@@ -904,7 +919,7 @@ cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t 
       if (swiglu && !make_tmap(&tA3, p.a3, p.K, p.a_rows_total, BM)) return cudaErrorInvalidValue;
       if (!swiglu) tA3 = tA;
     }
-    if (!make_tmap(&tB, p.b, p.K, p.b_rows_total, BOX_N)) return cudaErrorInvalidValue;
+    if (!make_tmap(&tB, p.b, p.K, p.b_rows_total, q.box_n)) return cudaErrorInvalidValue;
   } else {
     tA = tAs; tA3 = tA3s; tB = tBs;
   }
@@ -923,20 +938,20 @@ cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t 
   const int grid = pair ? 2 * ngroup : ngroup;
   switch (p.mode) {
     case kUmmaSwiGLU:
-      return pair ? launch_mode<kUmmaSwiGLU, true>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s)
-                  : launch_mode<kUmmaSwiGLU, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s);
+      return pair ? launch_mode<kUmmaSwiGLU, true>(tA, tA3, tB, tAs, tA3s, tBs, tG, q, grid, sp.total, s)
+                  : launch_mode<kUmmaSwiGLU, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, q, grid, sp.total, s);
     case kUmmaSwiGLUSave:
-      return pair ? launch_mode<kUmmaSwiGLUSave, true>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s)
-                  : launch_mode<kUmmaSwiGLUSave, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s);
+      return pair ? launch_mode<kUmmaSwiGLUSave, true>(tA, tA3, tB, tAs, tA3s, tBs, tG, q, grid, sp.total, s)
+                  : launch_mode<kUmmaSwiGLUSave, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, q, grid, sp.total, s);
     case kUmmaDown:
-      return pair ? launch_mode<kUmmaDown, true>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s)
-                  : launch_mode<kUmmaDown, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s);
+      return pair ? launch_mode<kUmmaDown, true>(tA, tA3, tB, tAs, tA3s, tBs, tG, q, grid, sp.total, s)
+                  : launch_mode<kUmmaDown, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, q, grid, sp.total, s);
     case kUmmaBiasAct:
-      return pair ? launch_mode<kUmmaBiasAct, true>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s)
-                  : launch_mode<kUmmaBiasAct, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s);
+      return pair ? launch_mode<kUmmaBiasAct, true>(tA, tA3, tB, tAs, tA3s, tBs, tG, q, grid, sp.total, s)
+                  : launch_mode<kUmmaBiasAct, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, q, grid, sp.total, s);
     case kUmmaDgrad:
-      return pair ? launch_mode<kUmmaDgrad, true>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s)
-                  : launch_mode<kUmmaDgrad, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, p, grid, sp.total, s);
+      return pair ? launch_mode<kUmmaDgrad, true>(tA, tA3, tB, tAs, tA3s, tBs, tG, q, grid, sp.total, s)
+                  : launch_mode<kUmmaDgrad, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, q, grid, sp.total, s);
   }
   return cudaErrorInvalidValue;
 }

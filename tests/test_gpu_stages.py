@@ -31,6 +31,13 @@ STAGE_CASES = {
     # segments of a handful of rows.
     "wide_experts_bf16": MoEConfig("wide_experts", T=150, d=192, E=320, k=6, f=64, gate_mode=GATE_SIGMOID,
                                    n_groups=8, topk_groups=4, route_scale=2.5, f_shared=64, bias="uniform"),
+    # d a multiple of the down tile's rows (512 on CTA pairs, 256 on single
+    # CTAs), so no weight tile is ragged; token tiles of up to 256 rows (one
+    # 128-row copy per CTA of a pair) and of 64 rows (single CTAs).
+    "fused_blocks_pair_bf16": MoEConfig("fused_blocks_pair", T=256, d=512, E=8, k=2, f=256,
+                                        gate_mode=GATE_SIGMOID, route_scale=1.0, f_shared=128, bias="uniform"),
+    "fused_blocks_single_bf16": MoEConfig("fused_blocks_single", T=40, d=256, E=16, k=2, f=128,
+                                          gate_mode=GATE_SIGMOID, route_scale=1.0, f_shared=64, bias="uniform"),
 }
 
 
@@ -232,3 +239,43 @@ def test_gate_up_hidden_matches_oracle(cases, name):
         if sh:
             ref_s = orc.swiglu_hidden(x64, H.f64(inp["ws1"]), H.f64(inp["ws3"]))
             H.compare_outputs(cfg, H.f64(h_s), ref_s, f"{v} shared h")
+
+
+@pytest.mark.parametrize("name", sorted(STAGE_CASES))
+def test_gate_up_weight_storage_order(cases, name):
+    # W1 and W3 are two caller buffers at any addresses. h must not depend on
+    # their order in memory: the same weights stored W1-then-W3 and
+    # W3-then-W1 in one allocation give bit-identical h, and that h matches
+    # the oracle (SwiGLU equation of the Sparse MoE FFN note).
+    cfg, inp = cases[name]
+    got, x_perm, _, _ = _packed(cfg, inp)
+    rows = cfg.T * cfg.k
+    sh = cfg.f_shared > 0
+    outs = []
+    for order in ("w1_first", "w3_first"):
+        pair = torch.empty((2,) + tuple(inp["w1"].shape), dtype=inp["w1"].dtype, device="cuda")
+        pair_s = torch.empty((2,) + tuple(inp["ws1"].shape), dtype=inp["ws1"].dtype, device="cuda") if sh else None
+        i1, i3 = (0, 1) if order == "w1_first" else (1, 0)
+        pair[i1].copy_(inp["w1"])
+        pair[i3].copy_(inp["w3"])
+        if sh:
+            pair_s[i1].copy_(inp["ws1"])
+            pair_s[i3].copy_(inp["ws3"])
+        assert (pair[i3].data_ptr() < pair[i1].data_ptr()) == (order == "w3_first")
+        h = torch.full((rows, cfg.f), float("nan"), dtype=cfg.torch_dtype, device="cuda")
+        h_s = torch.full((cfg.T, cfg.f_shared), float("nan"), dtype=cfg.torch_dtype, device="cuda") if sh else None
+        B.moe_expert_gate_up(cfg, x_perm, got["offsets"], pair[i1], pair[i3], inp["x"] if sh else None,
+                             pair_s[i1] if sh else None, pair_s[i3] if sh else None, h, h_s, got["ws"])
+        assert B.moe_get_device_error(got["ws"]) == B.MOE_OK
+        outs.append((h, h_s))
+    assert torch.equal(outs[0][0], outs[1][0])
+    if sh:
+        assert torch.equal(outs[0][1], outs[1][1])
+    offs = got["offsets"].cpu().numpy()
+    _, src = orc.permutation_rows(got["idx"].cpu().numpy(), offs)
+    x64, h64 = H.f64(inp["x"]), H.f64(outs[1][0])
+    for e in range(cfg.E):
+        a, b = offs[e], offs[e + 1]
+        if b > a:
+            ref = orc.swiglu_hidden(x64[src[a:b]], H.f64(inp["w1"])[e], H.f64(inp["w3"])[e])
+            H.compare_outputs(cfg, h64[a:b], ref, f"w3-first h of expert {e}")
