@@ -243,8 +243,10 @@ def whole_job_rate(tokens_per_rank: int, world: int, ms_per_step: float) -> floa
 
 
 # ------------------------------------------------------------ work accounting
-def stage_work(cfg, counts):
-    """Algorithmic bytes (compulsory HBM traffic) and flops of each stage for one forward."""
+def stage_work(cfg, counts, gather=False):
+    """Algorithmic bytes (compulsory HBM traffic) and flops of each stage for one forward.
+    gather: the gate/up GEMM reads token rows from x itself and the permute
+    writes the maps only (moe_forward_gathers_rows)."""
     es = cfg.elem_bytes
     T, d, E, k, f, fs = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.f_shared
     touched = int((counts > 0).sum())
@@ -253,7 +255,7 @@ def stage_work(cfg, counts):
     # route: x and the router read, the summed fp32 logits written once (kept
     # for the backward pass), indices and gates written.
     w["route"] = dict(bytes=(T * d + E * d) * es + T * k * 8 + T * E * 4, flops=2.0 * T * E * d)
-    w["permute"] = dict(bytes=(T * d + rows * d) * es + rows * 8 + T * k * 4, flops=0.0)
+    w["permute"] = dict(bytes=(0 if gather else (T * d + rows * d) * es) + rows * 8 + T * k * 4, flops=0.0)
     w["gate_up"] = dict(bytes=(touched * 2 * f * d + 2 * fs * d) * es + (rows * d + srows * d) * es
                         + (rows * f + srows * fs) * es,
                         flops=4.0 * (rows * f + srows * fs) * d)
@@ -438,8 +440,8 @@ def measure_backward(B, cfg, inp, touched, stream, reps):
 
 def measure_fused_permute(B, cfg, inp, idx, offsets, perm_src, inv_row, h, h_s, ws, stream, reps):
     """The permute fused into the gate/up GEMM: maps-only permute, then the
-    GEMM gathering token rows from x (TMA gather4). Same h bytes as the
-    packed chain; timed with events like the stage breakdown."""
+    GEMM gathering token rows from x (cp.async gather warps). Same h bytes as
+    the packed chain; timed with events like the stage breakdown."""
     h2 = torch.empty_like(h)
     hs2 = torch.empty_like(h_s) if h_s is not None else None
     calls = [lambda: B.moe_permute(cfg, None, idx, offsets, None, perm_src, inv_row, ws),
@@ -460,7 +462,8 @@ def measure_fused_permute(B, cfg, inp, idx, offsets, perm_src, inv_row, h, h_s, 
     pm = statistics.mean(evs[i][0].elapsed_time(evs[i][1]) for i in range(reps))
     gm = statistics.mean(evs[i][1].elapsed_time(evs[i][2]) for i in range(reps))
     return {"permute_maps_ms": pm, "gate_up_gather_ms": gm, "fused_ms": pm + gm,
-            "note": "not used by moe_forward: slower than the packed copy plus gate/up"}
+            "note": "moe_forward gathers only with single-CTA token tiles (under 128 rows); "
+                    "this shape runs CTA pairs, where the packed copy plus gate/up is faster"}
 
 
 def layer_bytes(cfg, touched):
@@ -494,12 +497,19 @@ def stage_breakdown(B, cfg, inp, ws, stream, n):
              y_s=torch.empty((T, d), dtype=dt, device=dev) if sh else None,
              y=torch.empty((T, d), dtype=dt, device=dev))
     names = ["route", "permute", "gate_up", "down", "combine"]
+    # The same path moe_forward takes: packed rows, or (single-CTA token
+    # tiles) the maps-only permute and the GEMM gathering rows from x.
+    gather = B.moe_forward_gathers_rows(cfg, inp["x"])
     calls = [
         lambda: B.moe_route(cfg, inp["x"], inp["w_router"], inp["bias"], o["idx"], o["gate"], o["counts"],
                             o["offsets"], ws),
-        lambda: B.moe_permute(cfg, inp["x"], o["idx"], o["offsets"], o["x_perm"], o["perm_src"], o["inv_row"], ws),
-        lambda: B.moe_expert_gate_up(cfg, o["x_perm"], o["offsets"], inp["w1"], inp["w3"], inp["x"] if sh else None,
-                                     inp["ws1"], inp["ws3"], o["h"], o["h_s"], ws),
+        (lambda: B.moe_permute(cfg, None, o["idx"], o["offsets"], None, o["perm_src"], o["inv_row"], ws)) if gather
+        else (lambda: B.moe_permute(cfg, inp["x"], o["idx"], o["offsets"], o["x_perm"], o["perm_src"],
+                                    o["inv_row"], ws)),
+        (lambda: B.moe_expert_gate_up_gather(cfg, inp["x"], o["perm_src"], o["offsets"], inp["w1"], inp["w3"],
+                                             inp["ws1"], inp["ws3"], o["h"], o["h_s"], ws)) if gather
+        else (lambda: B.moe_expert_gate_up(cfg, o["x_perm"], o["offsets"], inp["w1"], inp["w3"],
+                                           inp["x"] if sh else None, inp["ws1"], inp["ws3"], o["h"], o["h_s"], ws)),
         lambda: B.moe_expert_down(cfg, o["h"], o["offsets"], inp["w2"], o["h_s"], inp["ws2"], o["y_perm"],
                                   o["y_s"], ws),
         lambda: B.moe_combine(cfg, o["y_perm"], o["inv_row"], o["gate"], o["y_s"], o["y"]),
@@ -561,7 +571,7 @@ def measure_workload(B, name, dev, stream, steps, warmup, sampler, peaks):
     ms, t0, t1 = graph_step_ms(B, cfg, inp, ws, y, stream, steps, warmup)
     stage_ms, o = stage_breakdown(B, cfg, inp, ws, stream, max(3, min(steps, 50)))
     assert torch.equal(o["y"], y), f"{name}: per-stage chain and moe_forward disagree"
-    work, touched = stage_work(cfg, o["counts"].cpu())
+    work, touched = stage_work(cfg, o["counts"].cpu(), B.moe_forward_gathers_rows(cfg, inp["x"]))
     expert_ms = stage_ms["gate_up"] + stage_ms["down"]
     expert_flops = work["gate_up"]["flops"] + work["down"]["flops"]
     expert_bytes = work["gate_up"]["bytes"] + work["down"]["bytes"]
@@ -759,10 +769,14 @@ def main():
     if world == 1 and not args.no_extra_workloads and args.T is None and args.E is None and args.f is None:
         from mixture_experts_ffn_sigmoid_b200.inputs import CONFIGS
         extra = {}
-        for name in CONFIGS:
-            if name != cfg.name:
-                extra[name] = measure_workload(B, name, dev, stream, max(3, min(args.steps, 50)), args.warmup,
-                                               sampler, peaks)
+        # Lightest first, each after a second of idle GPU: the power cap that a
+        # heavy workload engages (sw_power_cap) then does not carry over into
+        # the next one's clocks, which each line reports for its own window.
+        for name in sorted((n for n in CONFIGS if n != cfg.name), key=lambda n: CONFIGS[n].active_flops()):
+            torch.cuda.synchronize()
+            time.sleep(1.0)
+            extra[name] = measure_workload(B, name, dev, stream, max(3, min(args.steps, 50)), args.warmup,
+                                           sampler, peaks)
     fused = measure_fused_permute(B, cfg, inp, idx, offsets, perm_src, inv_row, h, h_s, ws, stream,
                                   n_stage) if cfg.dtype == "bf16" else None
     if fused is not None:
@@ -791,7 +805,7 @@ def main():
     balance = {"us_per_call": b0.elapsed_time(b1) * 10.0, "entropy": ent.item(),
                "ln_E": math.log(E), "gamma": 0.15, "bound": "launch latency (E-element kernel)"}
     gelu = measure_gelu_experts(B, cfg, inp, counts.cpu(), stream, max(3, min(args.steps, 20)))
-    work, touched = stage_work(cfg, counts.cpu())
+    work, touched = stage_work(cfg, counts.cpu(), B.moe_forward_gathers_rows(cfg, inp["x"]))
     gelu["expert_weight_frac_hbm"] = gelu["expert_weight_gbs"] / peaks["hbm"]
     bwd = measure_backward(B, cfg, inp, touched, stream, max(3, min(args.steps, 10)))
     bwd["frac_tensor"] = bwd["tflops"] / peaks["tensor_sustained"]

@@ -22,7 +22,7 @@
  *   moe_backward (_workspace_size), moe_forward_train, moe_backward_saved
  *                                             gradients of the block for training
  *   moe_get_device_error, moe_route_noalloc_device_error,
- *   moe_selftest_wait_timeout, moe_status_string
+ *   moe_forward_gathers_rows, moe_selftest_wait_timeout, moe_status_string
  *
  * Sources, cited by page title and section:
  *   [DS] "Sparse MoE FFN" DeepSeek-V3 study note, "How it works": eq. 12
@@ -228,18 +228,23 @@ MOE_API moe_status moe_expert_gate_up(const moe_config* cfg, const void* x_perm,
 /*
  * moe_expert_gate_up_gather - moe_expert_gate_up without the packed copy of
  * the activations: the GEMM reads each packed row straight from x through
- * perm_src (TMA tile::gather4, four rows per copy), so moe_permute can skip
- * writing x_perm.  [DS] "Packed forward": gather the tokens of each expert.
+ * perm_src (two gather warps per CTA copy the rows with cp.async into the
+ * GEMM's shared-memory slots), so moe_permute can skip writing x_perm.
+ * [DS] "Packed forward": gather the tokens of each expert.
  *
- *   x              [T][d]        bf16   activations (also the shared expert's input)
- *   perm_src       [T*k]         int32  source token of each packed row (moe_permute)
+ *   x              [T][d]        bf16   activations (also the shared expert's input),
+ *                                       16-byte aligned, T*d*2 < 4 GiB
+ *   perm_src       [T*k]         int32  source token of each packed row (moe_permute);
+ *                                       an entry outside [0, T) reads row 0 and
+ *                                       sets MOE_ERR_INVALID_ARG in the error word
  *   expert_offsets, w1, w3, ws1, ws3, h, h_shared   as in moe_expert_gate_up
  *
- * bf16 only (MOE_ERR_UNSUPPORTED for fp32). Results are bit-identical to
- * moe_permute + moe_expert_gate_up. It saves the permute's copy (T*k*d
- * elements written, then read back) but fetches token rows 128 bytes per
- * row and k-step instead of in 32-row boxes; on B200 the GEMM then runs
- * slower by more than the copy costs, so moe_forward keeps the packed copy.
+ * bf16 only (MOE_ERR_UNSUPPORTED for fp32, or when x breaks the limits
+ * above). Results are bit-identical to moe_permute + moe_expert_gate_up.
+ * moe_forward takes this path itself when the token tiles run on single
+ * CTAs (fewer than 128 token rows per tile, e.g. decode), where it is as
+ * fast as reading packed rows and saves the permute's copy; on CTA pairs
+ * the packed copy is faster and moe_forward uses it.
  */
 MOE_API moe_status moe_expert_gate_up_gather(const moe_config* cfg, const void* x,
                                      const int32_t* perm_src, const int32_t* expert_offsets,
@@ -280,7 +285,10 @@ MOE_API moe_status moe_combine(const moe_config* cfg, const void* y_perm, const 
 /*
  * moe_forward - the whole block: route, permute, experts, combine.
  * Inputs as above; y [T][d] dtype receives shared + routed (no residual,
- * [DS] eq. 12). ws1/ws3/ws2 are NULL when f_shared == 0.
+ * [DS] eq. 12). ws1/ws3/ws2 are NULL when f_shared == 0. The gate/up GEMM
+ * reads the token rows either from the permute's packed copy or, with
+ * single-CTA token tiles, gathered straight from x (moe_forward_gathers_rows
+ * says which); the bytes of y are the same either way.
  */
 MOE_API moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_router,
                        const float* bias, const void* w1, const void* w3, const void* w2,
@@ -424,6 +432,18 @@ MOE_API moe_status moe_route_noalloc(const moe_config* cfg, const void* x, const
  * moe_route_noalloc on the same device.
  */
 MOE_API moe_status moe_route_noalloc_device_error(void* stream);
+
+/*
+ * moe_forward_gathers_rows - 1 if moe_forward, for this configuration and
+ * activation pointer x, has its gate/up GEMM gather the token rows from x
+ * (moe_permute writing the maps only, as moe_expert_gate_up_gather), 0 if it
+ * reads the permute's packed copy; -1 for an invalid configuration. The
+ * pages have no counterpart: the two paths give the same bytes, this tells
+ * a caller timing the stages which one to time. The rule: bf16, token tiles
+ * of fewer than 128 rows (single-CTA GEMM tiles, e.g. decode), x 16-byte
+ * aligned, T*d*2 under 4 GiB.
+ */
+MOE_API int moe_forward_gathers_rows(const moe_config* cfg, const void* x);
 
 /*
  * moe_balance_update - the aux-loss-free balancing step that follows routing

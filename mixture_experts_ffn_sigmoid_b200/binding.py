@@ -35,6 +35,7 @@ EXPORTED = ("moe_check_config", "moe_workspace_size", "moe_route", "moe_permute"
             "moe_expert_swiglu", "moe_expert_gate_up", "moe_expert_gate_up_gather", "moe_expert_down",
             "moe_combine", "moe_forward", "moe_get_device_error",
             "moe_selftest_wait_timeout", "moe_route_noalloc", "moe_route_noalloc_device_error",
+            "moe_forward_gathers_rows",
             "moe_balance_update",
             "moe_expert_gelu", "moe_forward_gelu", "moe_backward_workspace_size", "moe_backward",
             "moe_forward_train", "moe_backward_saved", "moe_status_string")
@@ -88,6 +89,7 @@ def lib() -> ctypes.CDLL:
             "moe_selftest_wait_timeout": (ctypes.c_int, [vp, sz, ctypes.c_int64, vp]),
             "moe_route_noalloc": (ctypes.c_int, [cfgp, vp, vp, f32p, i32p, f32p, i32p, i32p, vp]),
             "moe_route_noalloc_device_error": (ctypes.c_int, [vp]),
+            "moe_forward_gathers_rows": (ctypes.c_int, [cfgp, vp]),
             "moe_balance_update": (ctypes.c_int, [cfgp, i32p, f32p, ctypes.c_float, f32p, vp]),
             "moe_expert_gelu": (ctypes.c_int, [cfgp, vp, i32p, vp, f32p, vp, f32p, vp, vp, sz, vp]),
             "moe_forward_gelu": (ctypes.c_int, [cfgp, vp, vp, f32p, vp, f32p, vp, f32p, vp, vp, sz, vp]),
@@ -445,6 +447,15 @@ def moe_route_noalloc_device_error(stream=None) -> int:
     device (synchronises the stream, then reads and clears the fixed array's
     error word): MOE_OK or MOE_ERR_TIMEOUT."""
     return lib().moe_route_noalloc_device_error(_stream(stream))
+
+
+def moe_forward_gathers_rows(cfg, x) -> bool:
+    """Whether moe_forward's gate/up GEMM gathers the token rows of x itself
+    (the permute then writes the maps only) rather than reading a packed copy."""
+    r = lib().moe_forward_gathers_rows(ctypes.byref(_cfg(cfg)), _ptr(x))
+    if r < 0:
+        raise MoEError(MOE_ERR_INVALID_ARG, "moe_forward_gathers_rows")
+    return r == 1
 
 
 def moe_balance_update(cfg, expert_counts, bias, gamma: float, entropy=None, stream=None):

@@ -202,6 +202,17 @@ const int* route_tile_base(const moe_config& c, void* ws) {
 // Mixtral shapes alike.
 int inflight_for() { return 4; }
 
+// Whether moe_forward's gate/up GEMM gathers token rows from x (cp.async,
+// single-CTA tiles) instead of reading a packed copy: bf16, token tiles
+// under 128 (no CTA pairs), 16-byte aligned rows, x under 4 GB. Measured on
+// B200: as fast as the packed rows at these shapes, and the permute's copy
+// is saved; on CTA pairs the packed copy wins.
+int expert_tile_n(const moe_config& c);
+bool gather_rows_in_gemm(const moe_config& c, const void* x) {
+  return c.dtype == MOE_DTYPE_BF16 && expert_tile_n(c) < 128 && (reinterpret_cast<uintptr_t>(x) & 15u) == 0 &&
+         c.d % 8 == 0 && (long long)c.T * c.d * 2 <= 0xffffffffll;
+}
+
 int expert_tile_n(const moe_config& c) {
   const double m = (double)c.T * c.k / c.E;
   int bn = (int)ceil(4.0 * m + 16.0);
@@ -313,12 +324,14 @@ moe_status enqueue_down(const moe_config& c, const void* h, const int* offsets, 
 moe_status enqueue_experts(const moe_config& c, const void* x_perm, const int* offsets, const void* w1,
                            const void* w3, const void* w2, const void* x_sh, const void* ws1,
                            const void* ws3, const void* ws2, void* y_perm, void* y_sh, void* ws,
-                           cudaStream_t s, void* const* pre = nullptr) {
+                           cudaStream_t s, void* const* pre = nullptr, const int* gather_rows = nullptr,
+                           const void* gather_src = nullptr) {
   const Layout L = layout_of(c);
   void* h = at<char>(ws, L.h);
   void* h_s = at<char>(ws, L.h_s);
   uint32_t* err = at<uint32_t>(ws, L.err);
-  MOE_TRY(enqueue_gate_up(c, x_perm, offsets, w1, w3, x_sh, ws1, ws3, h, h_s, err, s, nullptr, nullptr, pre));
+  MOE_TRY(enqueue_gate_up(c, x_perm, offsets, w1, w3, x_sh, ws1, ws3, h, h_s, err, s, gather_rows, gather_src,
+                          pre));
   return enqueue_down(c, h, offsets, w2, h_s, ws2, y_perm, y_sh, err, s);
 }
 
@@ -863,6 +876,9 @@ moe_status moe_expert_gate_up_gather(const moe_config* cfg, const void* x, const
   MOE_TRY(check_config(cfg));
   const moe_config& c = *cfg;
   if (c.dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+  // cp.async reads 16-byte pieces of the rows at 32-bit offsets
+  if ((reinterpret_cast<uintptr_t>(x) & 15u) || c.d % 8 || (long long)c.T * c.d * 2 > 0xffffffffll)
+    return MOE_ERR_UNSUPPORTED;
   MOE_TRY(check_ws(c, workspace, ws_bytes));
   if (c.T == 0) return MOE_OK;
   MOE_TRY(need(x));
@@ -957,27 +973,36 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
     TraceRange stage("moe_forward.route");
     MOE_TRY(enqueue_route(c, x, w_router, bias, idx, gate, at<int>(ws, L.counts), offsets, ws, s));
   }
-  // Packed copy of the token rows, then GEMMs over contiguous segments. (The
-  // gate/up GEMM can instead gather rows from x with TMA gather4, see
-  // moe_expert_gate_up_gather; on B200 that costs more GEMM time than the
-  // copy it saves, so the block uses the packed copy.)
+  // Token rows for the gate/up GEMM. With single-CTA token tiles (few
+  // tokens per expert, e.g. decode) the GEMM gathers each expert's rows from
+  // x through perm_src, and the permute writes the maps only; with CTA pairs
+  // the packed copy plus TMA rows is faster, so the permute copies the rows.
+  const bool gather = gather_rows_in_gemm(c, x);
   {
     TraceRange stage("moe_forward.permute");
     MOE_CUDA(launch_permute(c.dtype, x, idx, offsets, at<int>(ws, L.cbase), route_tile_base(c, ws), c.T, c.d,
                             c.E, c.k, at<char>(ws, L.x_perm), at<int>(ws, L.perm_src), at<int>(ws, L.inv_row),
-                            device_sm_count(), s, true, at<uint32_t>(ws, L.err)));
+                            device_sm_count(), s, !gather, at<uint32_t>(ws, L.err)));
   }
   const bool shared = c.f_shared > 0;
   void* y_s = shared ? at<char>(ws, L.y_s) : nullptr;
   {
     TraceRange stage("moe_forward.experts");
+    // On the gather path the routed B tensor map still needs a valid
+    // source: the workspace's packed region, never read.
     MOE_TRY(enqueue_experts(c, at<char>(ws, L.x_perm), offsets, w1, w3, w2, shared ? x : nullptr, ws1,
-                            ws3, ws2, at<char>(ws, L.y_perm), y_s, ws, s));
+                            ws3, ws2, at<char>(ws, L.y_perm), y_s, ws, s, nullptr,
+                            gather ? at<int>(ws, L.perm_src) : nullptr, gather ? x : nullptr));
   }
   TraceRange stage("moe_forward.combine");
   MOE_CUDA(launch_combine(c.dtype, at<char>(ws, L.y_perm), at<int>(ws, L.inv_row), gate, y_s, y, c.T,
                           c.d, c.k, device_sm_count(), s));
   return MOE_OK;
+}
+
+int moe_forward_gathers_rows(const moe_config* cfg, const void* x) {
+  if (check_config(cfg) != MOE_OK) return -1;
+  return gather_rows_in_gemm(*cfg, x) ? 1 : 0;
 }
 
 moe_status moe_expert_gelu(const moe_config* cfg, const void* x_perm, const int32_t* expert_offsets,

@@ -71,12 +71,19 @@ constexpr int UMMA_K = 16;       // K per tcgen05.mma for 16-bit inputs
 constexpr int BN_MAX = 256;      // token columns per tile (MMA N), upper bound
 constexpr int BOX_N_MAX = 128;   // token rows per TMA box, at most
 constexpr int A_BYTES = BM * BK * 2;
-constexpr int NUM_THREADS = 320;
 constexpr int EPI_WARPS = 8;      // warps 2..9: two per TMEM lane quarter
+constexpr int GATHER_WARPS = 2;   // warps 10..11, launched only when B is gathered
+constexpr int NUM_THREADS = 32 * (2 + EPI_WARPS);                   // without gather warps
+constexpr int NUM_THREADS_GATHER = 32 * (2 + EPI_WARPS + GATHER_WARPS);
 constexpr int TMEM_COLS = 512;
 constexpr int NSLOT = 8;            // barrier pairs of the slot ring
 constexpr int SMEM_LIMIT = 232448;  // 227 KB of dynamic shared memory per block
-constexpr int HDR_BYTES = 2048;     // barriers, TMEM slot, slot records, gathered token rows
+// Gathered token rows per gather lane and tile: a CTA stages at most 128
+// rows, each gather warp half of them, four rows per 32 lanes at a time.
+constexpr int kGatherRowsPerLane = 128 / GATHER_WARPS / 4;
+// barriers, TMEM slot, slot records (first 1 KB); per gather warp the source
+// offsets of its token rows, [kGatherRowsPerLane][32 lanes] words
+constexpr int HDR_BYTES = 1024 + GATHER_WARPS * kGatherRowsPerLane * 32 * 4;
 
 // Shared-memory plan of one launch: [header (barriers, gathered token rows) |
 // tile tables | slot ring],
@@ -125,24 +132,18 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(cluster_bar)
       : "memory");
 }
-// Four arbitrary rows (row0..row3) of a 2-D tensor, one 128-byte box row
-// each, written as four consecutive swizzled rows at dst (box height 1).
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* tm, int c0, int r0, int r1,
-                                            int r2, int r3, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar)
-      : "memory");
+// 16 bytes from global memory into shared memory (cp.async, L2 only);
+// bytes past src_bytes (0..16) are zero.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
 }
-__device__ __forceinline__ void tma_gather4_pair(uint32_t dst, const CUtensorMap* tm, int c0, int r0,
-                                                 int r1, int r2, int r3, uint32_t cluster_bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(cluster_bar)
-      : "memory");
+// One arrival on the barrier once this thread's earlier cp.async copies have
+// landed; the arrival is not added to the barrier's expected count.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t slot_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot_smem),
                "r"(ncols)
@@ -297,11 +298,11 @@ __device__ __forceinline__ TokenSlice token_slice(const UmmaLaunch& p, const Til
 }
 
 template <int MODE, bool PAIR>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(NUM_THREADS_GATHER, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA3,
                      const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmAs,
                      const __grid_constant__ CUtensorMap tmA3s, const __grid_constant__ CUtensorMap tmBs,
-                     const __grid_constant__ CUtensorMap tmG, const UmmaLaunch p) {
+                     const UmmaLaunch p) {
   using KD = Kind<MODE>;
   constexpr int A_TILES = KD::A_TILES;
   constexpr int WROWS = tile_rows(MODE, PAIR);
@@ -323,7 +324,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   volatile uint32_t* abort_flag = tmem_slot + 1;
   uint32_t* fl_off = tmem_slot + 2;             // producer's record of slots in flight
   uint32_t* fl_size = fl_off + NSLOT;
-  int* s_rows = reinterpret_cast<int*>(smem + 1024);    // token rows of the current tile (gather)
+  uint64_t* gbar = reinterpret_cast<uint64_t*>(smem + 256);   // peer CTA: its gathered rows landed
+  uint64_t* acq_bar = gbar + NSLOT;                            // slot claimed by the TMA issuer
+  uint32_t* s_goff = reinterpret_cast<uint32_t*>(smem + 1024);   // gathered rows' byte offsets in the source
   int* s_start = reinterpret_cast<int*>(smem + HDR_BYTES);
   int* s_off = s_start + (nseg + 1);
   uint8_t* ring = smem + HDR_BYTES + sp.table_bytes;
@@ -331,6 +334,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = PAIR ? cluster_rank() : 0u;
   const bool leader = rank == 0;
+  const bool gather = p.b_gather != nullptr;
   const int group = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int ngroups = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
@@ -341,9 +345,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     s_off[s] = p.n_routed > 0 ? clamp_offset(p.offsets[s], p.max_routed_rows, blockIdx.x == 0 ? p.err : nullptr)
                               : 0;
   if (threadIdx.x == 64) {
+    // Full barrier arrivals per slot: the arming TMA issuer; with a gathered
+    // B also every gather lane, and on a pair the peer's forwarder.
+    constexpr uint32_t kGatherLanes = 32 * GATHER_WARPS;
+    const uint32_t full_count = gather ? (PAIR ? (leader ? 2u + kGatherLanes : 1u) : 1u + kGatherLanes) : 1u;
     for (int i = 0; i < NSLOT; ++i) {
-      mbar_init(smem_u32(&full_bar[i]), 1);
+      mbar_init(smem_u32(&full_bar[i]), full_count);
       mbar_init(smem_u32(&empty_bar[i]), 1);
+      mbar_init(smem_u32(&gbar[i]), kGatherLanes);
+      mbar_init(smem_u32(&acq_bar[i]), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&accf_bar[i]), 1);
@@ -365,7 +375,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     tmap_prefetch(&tmA); tmap_prefetch(&tmB); tmap_prefetch(&tmAs); tmap_prefetch(&tmBs);
     if (dual_a(MODE)) { tmap_prefetch(&tmA3); tmap_prefetch(&tmA3s); }
-    if (p.b_gather) tmap_prefetch(&tmG);
   }
   __syncthreads();
   // Tiles per segment -> exclusive prefix s_start[0..nseg] (warp 0).
@@ -404,6 +413,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
+    // Claims ring slots and issues the TMA copies. A gathered B (routed
+    // token rows read from the source activations through b_gather) is
+    // copied by the gather warps: each claimed slot is announced on its
+    // acq_bar.
     RingCursor cur;
     uint32_t inflight = 0;
     const uint32_t max_inflight = (uint32_t)min(max(p.max_inflight, 2), NSLOT);
@@ -421,19 +434,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int c_row0 = t.dense ? 0 : t.seg * p.a_k_rows;
       const int ksplit = t.dense ? p.k_split_s : p.k_split;
       const uint32_t bytes = A_TILES * A_BYTES + ts.bytes();
+      // Bytes the TMA delivers: the weights, and B unless it is gathered.
+      const uint32_t tx = A_TILES * A_BYTES + (ts.rows_gather > 0 ? 0u : ts.bytes());
       const int nk = ceil_div(t.K, BK);
-      if (ts.rows_gather > 0) {
-        // Token rows of this CTA's part of the tile: packed rows map to source
-        // tokens through b_gather; rows past the segment reuse its first token.
-        const int r_base = t.b_row0 + t.tt * p.bn_max + (PAIR ? (int)rank * ts.rows_gather : 0);
-        const int r_end = t.b_row0 + t.rows;
-        const int pad = p.b_gather[t.b_row0];
-        for (int j = 0; j < ts.rows_gather; ++j) {
-          const int r = r_base + j;
-          s_rows[j] = r < r_end ? p.b_gather[r] : pad;
-        }
-      }
-      for (int kb = 0; kb < nk; ++kb) {
+      for (int kb = 0; kb < nk && ok; ++kb) {
         // Make room: the barrier pair and the bytes of the new slot must be free.
         const uint32_t off_new = cur.peek(bytes, cap);
         while (true) {
@@ -457,14 +461,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         fl_off[slot] = off;
         fl_size[slot] = bytes;
         ++inflight;
+        if (gather) mbar_arrive(smem_u32(&acq_bar[slot]));
         const uint32_t fb_local = smem_u32(&full_bar[slot]);
         const uint32_t sb = smem_u32(ring + off);
         const uint32_t bb = sb + A_TILES * A_BYTES;
         if (PAIR) {
-          // Both CTAs' copies complete on the leader's barrier, which the leader
-          // arms for both halves (the halves are the same size).
+          // Both CTAs' copies complete on the leader's barrier, which the
+          // leader arms for both halves (the halves are the same size).
           const uint32_t fb = map_to_cta(fb_local, 0);
-          if (leader) mbar_expect_tx(fb_local, 2 * bytes);
+          if (leader) mbar_expect_tx(fb_local, 2 * tx);
           if (MODE == kUmmaDgrad) {
             const bool second = kb >= ksplit;
             const int crow = c_row0 + (second ? kb - ksplit : kb) * BK;
@@ -480,16 +485,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (dual_a(MODE)) tma_load_2d_pair(sb + A_BYTES, mA3, kb * BK, a_row, fb);
             if (two_blocks(MODE)) tma_load_2d_pair(sb + A_BYTES, mA, kb * BK, a_row + BLOCK_STEP, fb);
           }
-          if (ts.rows_gather > 0) {
-            for (int g = 0; g < ts.rows_gather; g += 4)
-              tma_gather4_pair(bb + g * (BK * 2), &tmG, kb * BK, s_rows[g], s_rows[g + 1], s_rows[g + 2],
-                               s_rows[g + 3], fb);
-          } else {
+          if (ts.rows_gather == 0)
             for (int bx = 0; bx < ts.nbox; ++bx)
               tma_load_2d_pair(bb + bx * ts.box_bytes, mB, kb * BK, ts.row + bx * p.box_n, fb);
-          }
         } else {
-          mbar_expect_tx(fb_local, bytes);
+          mbar_expect_tx(fb_local, tx);
           if (MODE == kUmmaDgrad) {
             const bool second = kb >= ksplit;
             const int crow = c_row0 + (second ? kb - ksplit : kb) * BK;
@@ -505,14 +505,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (dual_a(MODE)) tma_load_2d(sb + A_BYTES, mA3, kb * BK, a_row, fb_local);
             if (two_blocks(MODE)) tma_load_2d(sb + A_BYTES, mA, kb * BK, a_row + BLOCK_STEP, fb_local);
           }
-          if (ts.rows_gather > 0) {
-            for (int g = 0; g < ts.rows_gather; g += 4)
-              tma_gather4(bb + g * (BK * 2), &tmG, kb * BK, s_rows[g], s_rows[g + 1], s_rows[g + 2],
-                          s_rows[g + 3], fb_local);
-          } else {
+          if (ts.rows_gather == 0)
             for (int bx = 0; bx < ts.nbox; ++bx)
               tma_load_2d(bb + bx * ts.box_bytes, mB, kb * BK, ts.row + bx * p.box_n, fb_local);
-          }
         }
       }
     }
@@ -526,6 +521,92 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       else
         wait_bounded(smem_u32(&full_bar[u % NSLOT]), (u / NSLOT) & 1u, abort_flag, p.err,
                      p.timeout_ns, false);
+    }
+  } else if (gather && warp >= 2 + EPI_WARPS) {
+    // ------------------------------------------------------------ gather
+    // Gather warp g copies rows [g R/2, (g+1) R/2) of the CTA's R gathered
+    // token rows into each slot the issuer claims (same ring walk, so the
+    // same offsets): lane l takes 16-byte column chunk l % 8 of rows
+    // l / 8 + 4i, whose source offsets are fixed per tile. Each lane's
+    // completion is one arrival on the slot's full barrier (in a pair's peer
+    // CTA on its gather barrier, which the forwarder passes on).
+    const int gw = warp - (2 + EPI_WARPS);
+    uint32_t* goff = s_goff + gw * kGatherRowsPerLane * 32;
+    const char* src = static_cast<const char*>(p.b_gather_src);
+    RingCursor cur;
+    bool ok = true;
+    for (int tile = group; tile < total_tiles && ok; tile += ngroups) {
+      const Tile t = decode_tile(p, s_off, s_start, nseg, tile, WROWS);
+      const TokenSlice ts = token_slice<PAIR>(p, t, rank);
+      const uint32_t bytes = A_TILES * A_BYTES + ts.bytes();
+      const int nk = ceil_div(t.K, BK);
+      const int half_rows = ts.rows_gather / GATHER_WARPS;   // a multiple of 4
+      const int g_n = half_rows / 4;                          // rows per lane, at most kGatherRowsPerLane
+      if (g_n > 0) {
+        // Packed rows map to source tokens through b_gather; rows past the
+        // segment reuse its first token. A source row outside
+        // [0, b_gather_rows) is recorded and replaced by row 0.
+        const int r_base = t.b_row0 + t.tt * p.bn_max + (PAIR ? (int)rank * ts.rows_gather : 0) + gw * half_rows;
+        const int r_end = t.b_row0 + t.rows;
+        for (int i = 0; i < g_n; ++i) {
+          const int r = r_base + (lane >> 3) + 4 * i;
+          int tok = p.b_gather[r < r_end ? r : t.b_row0];
+          if (tok < 0 || (long long)tok >= p.b_gather_rows) {
+            if (p.err) atomicOr(p.err, kErrBadIndex);
+            tok = 0;
+          }
+          goff[i * 32 + lane] = (uint32_t)(((long long)tok * t.K + (lane & 7) * 8) * 2);
+        }
+        __syncwarp();
+      }
+      // Row r = gw R/2 + lane / 8 + 4i lands at r * 128 in the 128-byte
+      // swizzle, its chunk c at (c ^ (r % 8)) * 16.
+      const int c = lane & 7;
+      const int rb = gw * half_rows + (lane >> 3);
+      for (int kb = 0; kb < nk; ++kb) {
+        const uint32_t u = cur.count;
+        uint32_t off, slot, parity;
+        cur.take(bytes, cap, off, slot, parity);
+        if (!wait_bounded(smem_u32(&acq_bar[slot]), (u / NSLOT) & 1u, abort_flag, p.err, p.timeout_ns, true)) {
+          ok = false;
+          break;
+        }
+        if (g_n > 0) {
+          const uint32_t bb = smem_u32(ring + off) + A_TILES * A_BYTES;
+          const bool in_k = kb * BK + c * 8 < t.K;   // K is a multiple of 8
+          const long long koff = in_k ? (long long)kb * BK * 2 : 0;
+          const uint32_t src_bytes = in_k ? 16u : 0u;
+#pragma unroll
+          for (int i = 0; i < kGatherRowsPerLane; ++i)
+            if (i < g_n) {
+              const int r = rb + 4 * i;
+              cp_async_16(bb + (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)), src + goff[i * 32 + lane] + koff,
+                          src_bytes);
+            }
+        }
+        cp_async_arrive_noinc(PAIR && !leader ? smem_u32(&gbar[slot]) : smem_u32(&full_bar[slot]));
+      }
+    }
+    cp_async_wait_all();
+  } else if (PAIR && gather && warp == 1 && lane == 0 && !leader) {
+    // ------------------------------------------------------------ forwarder
+    // The peer CTA's gathered rows land in its own shared memory; once all
+    // 32 lanes' copies of a slot are done, make them visible to the tensor
+    // core's (async) proxy and count them on the leader's full barrier.
+    uint32_t u = 0;
+    bool ok = true;
+    for (int tile = group; tile < total_tiles && ok; tile += ngroups) {
+      const Tile t = decode_tile(p, s_off, s_start, nseg, tile, WROWS);
+      const int nk = ceil_div(t.K, BK);
+      for (int kb = 0; kb < nk; ++kb, ++u) {
+        if (!wait_bounded(smem_u32(&gbar[u % NSLOT]), (u / NSLOT) & 1u, abort_flag, p.err, p.timeout_ns,
+                          true)) {
+          ok = false;
+          break;
+        }
+        fence_proxy_async_smem();
+        mbar_arrive_cluster(map_to_cta(smem_u32(&full_bar[u % NSLOT]), 0));
+      }
     }
   } else if (warp == 1 && lane == 0 && leader) {
     // ------------------------------------------------------------ MMA issuer
@@ -563,6 +644,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ok = false;
           break;
         }
+        // Rows gathered with cp.async were written through the generic proxy;
+        // the tensor core reads shared memory through the async proxy.
+        if (gather) fence_proxy_async_smem();
         tc_fence_after();
         const uint32_t sb = smem_u32(ring + off);
         constexpr bool MN_A = MODE == kUmmaDgrad;
@@ -597,7 +681,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       else umma_commit(smem_u32(drain_bar));
       wait_bounded(smem_u32(drain_bar), 0u, abort_flag, p.err, p.timeout_ns, false);
     }
-  } else if (warp >= 2) {
+  } else if (warp >= 2 && warp < 2 + EPI_WARPS) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                  // TMEM lane quarter this warp may read
     const int ch = (warp - 2) >> 2;          // which 16-column chunks: ch, ch + 2, ch + 4, ...
@@ -851,17 +935,18 @@ cudaError_t ensure_smem_attr() {
 template <int MODE, bool PAIR>
 cudaError_t launch_mode(const CUtensorMap& tA, const CUtensorMap& tA3, const CUtensorMap& tB,
                         const CUtensorMap& tAs, const CUtensorMap& tA3s, const CUtensorMap& tBs,
-                        const CUtensorMap& tG, const UmmaLaunch& p, int grid, int smem,
+                        const UmmaLaunch& p, int grid, int smem,
                         cudaStream_t s) {
   cudaError_t e = ensure_smem_attr<MODE, PAIR>();
   if (e != cudaSuccess) return e;
+  const int threads = p.b_gather ? NUM_THREADS_GATHER : NUM_THREADS;
   if (!PAIR) {
-    umma_gemm_kernel<MODE, false><<<grid, NUM_THREADS, smem, s>>>(tA, tA3, tB, tAs, tA3s, tBs, tG, p);
+    umma_gemm_kernel<MODE, false><<<grid, threads, smem, s>>>(tA, tA3, tB, tAs, tA3s, tBs, p);
     return cudaGetLastError();
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -871,7 +956,7 @@ cudaError_t launch_mode(const CUtensorMap& tA, const CUtensorMap& tA3, const CUt
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, umma_gemm_kernel<MODE, true>, tA, tA3, tB, tAs, tA3s, tBs, tG, p);
+  return cudaLaunchKernelEx(&cfg, umma_gemm_kernel<MODE, true>, tA, tA3, tB, tAs, tA3s, tBs, p);
 }
 
 }  // namespace
@@ -924,9 +1009,12 @@ cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t 
     tA = tAs; tA3 = tA3s; tB = tBs;
   }
   if (!has_dense) { tAs = tA; tA3s = tA3; tBs = tB; }
-  // Gathered token rows: one-row boxes over the source activations.
-  CUtensorMap tG = tB;
-  if (p.b_gather && !make_tmap(&tG, p.b_gather_src, p.K, p.b_gather_rows, 1)) return cudaErrorInvalidValue;
+  // Gathered token rows are copied with cp.async: the source rows must be
+  // 16-byte aligned.
+  if (p.b_gather && (!p.b_gather_src || p.b_gather_rows <= 0 ||
+                     (reinterpret_cast<uintptr_t>(p.b_gather_src) & 15u) || (p.K * 2) % 16 ||
+                     mine_max > GATHER_WARPS * 4 * kGatherRowsPerLane || p.b_gather_rows * p.K * 2 > 0xffffffffll))
+    return cudaErrorInvalidValue;
 
   long long tiles = 0;
   if (p.n_routed > 0)
@@ -938,20 +1026,20 @@ cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t 
   const int grid = pair ? 2 * ngroup : ngroup;
   switch (p.mode) {
     case kUmmaSwiGLU:
-      return pair ? launch_mode<kUmmaSwiGLU, true>(tA, tA3, tB, tAs, tA3s, tBs, tG, q, grid, sp.total, s)
-                  : launch_mode<kUmmaSwiGLU, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, q, grid, sp.total, s);
+      return pair ? launch_mode<kUmmaSwiGLU, true>(tA, tA3, tB, tAs, tA3s, tBs, q, grid, sp.total, s)
+                  : launch_mode<kUmmaSwiGLU, false>(tA, tA3, tB, tAs, tA3s, tBs, q, grid, sp.total, s);
     case kUmmaSwiGLUSave:
-      return pair ? launch_mode<kUmmaSwiGLUSave, true>(tA, tA3, tB, tAs, tA3s, tBs, tG, q, grid, sp.total, s)
-                  : launch_mode<kUmmaSwiGLUSave, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, q, grid, sp.total, s);
+      return pair ? launch_mode<kUmmaSwiGLUSave, true>(tA, tA3, tB, tAs, tA3s, tBs, q, grid, sp.total, s)
+                  : launch_mode<kUmmaSwiGLUSave, false>(tA, tA3, tB, tAs, tA3s, tBs, q, grid, sp.total, s);
     case kUmmaDown:
-      return pair ? launch_mode<kUmmaDown, true>(tA, tA3, tB, tAs, tA3s, tBs, tG, q, grid, sp.total, s)
-                  : launch_mode<kUmmaDown, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, q, grid, sp.total, s);
+      return pair ? launch_mode<kUmmaDown, true>(tA, tA3, tB, tAs, tA3s, tBs, q, grid, sp.total, s)
+                  : launch_mode<kUmmaDown, false>(tA, tA3, tB, tAs, tA3s, tBs, q, grid, sp.total, s);
     case kUmmaBiasAct:
-      return pair ? launch_mode<kUmmaBiasAct, true>(tA, tA3, tB, tAs, tA3s, tBs, tG, q, grid, sp.total, s)
-                  : launch_mode<kUmmaBiasAct, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, q, grid, sp.total, s);
+      return pair ? launch_mode<kUmmaBiasAct, true>(tA, tA3, tB, tAs, tA3s, tBs, q, grid, sp.total, s)
+                  : launch_mode<kUmmaBiasAct, false>(tA, tA3, tB, tAs, tA3s, tBs, q, grid, sp.total, s);
     case kUmmaDgrad:
-      return pair ? launch_mode<kUmmaDgrad, true>(tA, tA3, tB, tAs, tA3s, tBs, tG, q, grid, sp.total, s)
-                  : launch_mode<kUmmaDgrad, false>(tA, tA3, tB, tAs, tA3s, tBs, tG, q, grid, sp.total, s);
+      return pair ? launch_mode<kUmmaDgrad, true>(tA, tA3, tB, tAs, tA3s, tBs, q, grid, sp.total, s)
+                  : launch_mode<kUmmaDgrad, false>(tA, tA3, tB, tAs, tA3s, tBs, q, grid, sp.total, s);
   }
   return cudaErrorInvalidValue;
 }

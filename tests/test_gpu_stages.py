@@ -144,9 +144,13 @@ def test_forward_full_oracle(cases, name):
     assert rep["compared"] >= cfg.T - max(1, cfg.T // 100)
 
 
-def test_forward_equals_stage_chain(cases):
+# ds_like_small runs its expert GEMMs on CTA pairs (moe_forward reads a packed
+# copy of the token rows); fused_blocks_single on single CTAs (moe_forward's
+# gate/up GEMM gathers the rows from x, the permute writes the maps only).
+@pytest.mark.parametrize("name", ["ds_like_small_bf16", "fused_blocks_single_bf16"])
+def test_forward_equals_stage_chain(cases, name):
     # moe_forward and the four stage calls give the same bytes.
-    cfg, inp = cases["ds_like_small_bf16"]
+    cfg, inp = cases[name]
     y_fwd = H.gpu_forward(cfg, inp)
     got, x_perm, perm_src, inv_row = _packed(cfg, inp)
     rows = cfg.T * cfg.k
@@ -160,8 +164,9 @@ def test_forward_equals_stage_chain(cases):
     assert torch.equal(y, y_fwd)
 
 
-def test_forward_is_deterministic(cases):
-    cfg, inp = cases["ds_like_small_bf16"]
+@pytest.mark.parametrize("name", ["ds_like_small_bf16", "fused_blocks_single_bf16"])
+def test_forward_is_deterministic(cases, name):
+    cfg, inp = cases[name]
     a = H.gpu_forward(cfg, inp)
     b = H.gpu_forward(cfg, inp)
     assert torch.equal(a, b)
@@ -169,7 +174,7 @@ def test_forward_is_deterministic(cases):
 
 @pytest.mark.parametrize("name", sorted(STAGE_CASES))
 def test_gate_up_gather_matches_packed(cases, name):
-    # Reading token rows through perm_src (TMA gather4) gives bit-identical h
+    # Reading token rows through perm_src (cp.async gather) gives bit-identical h
     # to reading the packed copy x_perm; maps-only permute writes the same maps.
     cfg, inp = cases[name]
     got, x_perm, perm_src, inv_row = _packed(cfg, inp)
