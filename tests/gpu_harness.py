@@ -94,6 +94,11 @@ def check_route(cfg: MoEConfig, ref: dict, got: dict) -> dict:
     return dict(near_ties=int(flags.sum()), gate_err=float(err), flags=flags)
 
 
+# Relative part of the bf16 elementwise bound: 2.6x the 2^-8 worst case of one
+# round-to-nearest into bf16 (the backward tests use the same form).
+BF16_REL = 1e-2
+
+
 def compare_outputs(cfg: MoEConfig, y: np.ndarray, y_ref: np.ndarray, what: str = "y") -> dict:
     rel_tol, max_tol = out_tol(cfg)
     diff = y.astype(np.float64) - y_ref
@@ -104,7 +109,15 @@ def compare_outputs(cfg: MoEConfig, y: np.ndarray, y_ref: np.ndarray, what: str 
     assert np.all(np.isfinite(y)), f"{what}: non-finite values (unwritten rows?)"
     assert rel <= rel_tol, f"{what}: relative L2 error {rel:.3e} > {rel_tol}"
     if max_tol is not None:
-        assert mx <= max_tol * rms, f"{what}: max abs error {mx:.3e} > {max_tol} * rms {rms:.3e}"
+        # Elementwise: max_tol * RMS for the accumulated error, plus 1e-2 * |ref|
+        # for the final rounding to bf16, which moves a stored value by up to
+        # 2^-8 of its own magnitude (half an ulp at the bottom of its binade),
+        # so large entries carry a proportionally larger error.
+        bound = max_tol * rms + BF16_REL * np.abs(y_ref)
+        worst = int(np.argmax(np.abs(diff) - bound)) if diff.size else 0
+        assert np.all(np.abs(diff) <= bound), (
+            f"{what}: max abs error {np.abs(diff).flat[worst]:.3e} at |ref| {np.abs(y_ref).flat[worst]:.3e} > "
+            f"{max_tol} * rms {rms:.3e} + {BF16_REL} * |ref|")
     return dict(rel_l2=rel, max_abs=mx, rms=rms)
 
 
