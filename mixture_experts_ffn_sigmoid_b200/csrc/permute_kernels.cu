@@ -10,7 +10,9 @@
 //
 // Both kernels move whole rows with 16-byte vector loads and stores; rows
 // are d * sizeof(T) bytes, a multiple of 16 (checked by the C ABI).
-#include "moe_internal.cuh"
+#include <algorithm>
+
+#include "umma_common.cuh"
 
 namespace moe {
 namespace {
@@ -24,17 +26,14 @@ __device__ __forceinline__ void st16(void* p, uint4 v) { *reinterpret_cast<uint4
 // start, + the token's rank in the chunk), then copies a column slice of the
 // 32 rows to their k destinations. Split 0 also writes inv_row / perm_src. Without
 // `copy` only the maps are written (the GEMM then gathers rows from x).
-template <typename T>
-__global__ void __launch_bounds__(256) permute_kernel(
-    const T* __restrict__ x, const int* __restrict__ idx, const int* __restrict__ offsets,
-    const int* __restrict__ chunk_base, const int* __restrict__ tile_base, int n_tok, int d, int E, int k,
-    T* __restrict__ x_perm,
-    int* __restrict__ perm_src, int* __restrict__ inv_row, int rows_total, int vec_per_split,
-    int copy, uint32_t* __restrict__ err) {
-  constexpr int V = Vec16<T>::N;
-  __shared__ uint32_t s_mask[kMaxExperts];
-  __shared__ int s_row[kChunk * kMaxTopK];
-  const int c = blockIdx.x;
+// Packed rows of chunk c's tokens into s_row[token * k + j] (-1 for an id
+// outside [0, E) or a row outside [0, rows_total), recorded in err); with
+// write_maps also inv_row and perm_src. Called by every thread of the block;
+// ends with the block synchronised.
+__device__ void chunk_rows(int c, const int* __restrict__ idx, const int* __restrict__ offsets,
+                           const int* __restrict__ chunk_base, const int* __restrict__ tile_base, int n_tok, int E,
+                           int k, int rows_total, bool write_maps, int* __restrict__ perm_src,
+                           int* __restrict__ inv_row, uint32_t* __restrict__ err, uint32_t* s_mask, int* s_row) {
   const int tid = threadIdx.x;
   for (int e = tid; e < E; e += blockDim.x) s_mask[e] = 0u;
   __syncthreads();
@@ -57,16 +56,32 @@ __global__ void __launch_bounds__(256) permute_kernel(
         if (tile_base) row += tile_base[(size_t)(c / kTileChunks) * E + e];
         if (row < 0 || row >= rows_total) row = -1;
       }
-      if (row < 0 && err && blockIdx.y == 0) atomicOr(err, kErrBadIndex);
+      if (row < 0 && err && write_maps) atomicOr(err, kErrBadIndex);
       s_row[tid * k + j] = row;
-      if (blockIdx.y == 0) {
+      if (write_maps) {
         inv_row[(size_t)t * k + j] = row;
         if (row >= 0) perm_src[row] = t;
       }
     }
   }
-  if (!copy) return;
   __syncthreads();
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) permute_kernel(
+    const T* __restrict__ x, const int* __restrict__ idx, const int* __restrict__ offsets,
+    const int* __restrict__ chunk_base, const int* __restrict__ tile_base, int n_tok, int d, int E, int k,
+    T* __restrict__ x_perm,
+    int* __restrict__ perm_src, int* __restrict__ inv_row, int rows_total, int vec_per_split,
+    int copy, uint32_t* __restrict__ err) {
+  constexpr int V = Vec16<T>::N;
+  __shared__ uint32_t s_mask[kMaxExperts];
+  __shared__ int s_row[kChunk * kMaxTopK];
+  const int c = blockIdx.x;
+  const int tid = threadIdx.x;
+  chunk_rows(c, idx, offsets, chunk_base, tile_base, n_tok, E, k, rows_total, blockIdx.y == 0, perm_src, inv_row,
+             err, s_mask, s_row);
+  if (!copy) return;
   const int nvec = d / V;
   const int v0 = blockIdx.y * vec_per_split;
   const int v1 = min(nvec, v0 + vec_per_split);
@@ -100,6 +115,83 @@ __global__ void __launch_bounds__(256) permute_kernel(
       }
     }
   }
+}
+
+constexpr int kMaxBulkBufs = 8;
+
+__device__ __forceinline__ void bulk_load_row(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_store_row(void* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
+               : "memory");
+}
+// All but the newest committed group have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_but_one() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
+// The same permute moving whole rows with bulk copies: grid = one block per
+// chunk of 32 tokens. After the row maps, one thread streams the chunk's
+// rows through a ring of nbuf shared-memory buffers: one copy brings a row
+// (row_bytes, a multiple of 16) in, k copies write it to its packed rows. A
+// row's buffer is refilled once the copies out of it have read it, so up to
+// nbuf - 1 rows are on their way in while one goes out. Every wait is
+// bounded; on expiry the block records kErrTimeoutWait, waits (bounded) for
+// the rows it still has coming in, and stops.
+__global__ void __launch_bounds__(128) permute_bulk_kernel(
+    const char* __restrict__ x, const int* __restrict__ idx, const int* __restrict__ offsets,
+    const int* __restrict__ chunk_base, const int* __restrict__ tile_base, int n_tok, int E, int k,
+    uint32_t row_bytes, int nbuf, char* __restrict__ x_perm, int* __restrict__ perm_src, int* __restrict__ inv_row,
+    int rows_total, uint32_t* __restrict__ err, long long timeout_ns) {
+  extern __shared__ __align__(128) uint8_t ring[];
+  __shared__ uint32_t s_mask[kMaxExperts];
+  __shared__ int s_row[kChunk * kMaxTopK];
+  __shared__ __align__(8) uint64_t bars[kMaxBulkBufs];
+  __shared__ uint32_t s_abort;
+  const int c = blockIdx.x;
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < nbuf; ++b) mbar_init(smem_u32(&bars[b]), 1);
+    s_abort = 0u;
+    fence_mbar_init();
+  }
+  chunk_rows(c, idx, offsets, chunk_base, tile_base, n_tok, E, k, rows_total, true, perm_src, inv_row, err, s_mask,
+             s_row);
+  if (threadIdx.x != 0) return;
+  const int ntok = min(kChunk, n_tok - c * kChunk);
+  const uint32_t ring0 = smem_u32(ring);
+  auto load = [&](int i) {
+    const int b = i % nbuf;
+    mbar_expect_tx(smem_u32(&bars[b]), row_bytes);
+    bulk_load_row(ring0 + (uint32_t)b * row_bytes, x + (size_t)(c * kChunk + i) * row_bytes, row_bytes,
+                  smem_u32(&bars[b]));
+  };
+  int issued = min(nbuf, ntok);
+  for (int i = 0; i < issued; ++i) load(i);
+  int done = 0;   // rows whose load has been waited for
+  for (int i = 0; i < ntok; ++i) {
+    const int b = i % nbuf;
+    if (!wait_bounded(smem_u32(&bars[b]), (uint32_t)(i / nbuf) & 1u, (volatile uint32_t*)&s_abort, err, timeout_ns,
+                      true))
+      break;
+    done = i + 1;
+    for (int j = 0; j < k; ++j) {
+      const int row = s_row[i * k + j];
+      if (row >= 0) bulk_store_row(x_perm + (size_t)row * row_bytes, ring0 + (uint32_t)b * row_bytes, row_bytes);
+    }
+    bulk_commit();
+    // Refill the previous row's buffer once its copies out have read it.
+    if (i >= 1 && issued < ntok) {
+      bulk_wait_read_but_one();
+      load(issued++);
+    }
+  }
+  for (int i = done; i < issued; ++i)   // only after a timeout: let the rows in flight land
+    wait_bounded(smem_u32(&bars[i % nbuf]), (uint32_t)(i / nbuf) & 1u, (volatile uint32_t*)&s_abort, err,
+                 timeout_ns, false);
+  bulk_wait_all();
 }
 
 template <typename T>
@@ -160,9 +252,21 @@ __global__ void __launch_bounds__(128) combine_kernel(
     float acc[V];
 #pragma unroll
     for (int i = 0; i < V; ++i) acc[i] = 0.0f;
-    for (int j = 0; j < k; ++j) {
-      const int row = s_row[j];
-      if (row >= 0) unpack_add<T>(acc, ld16(y_perm + (size_t)row * d + (size_t)v * V), s_g[j]);
+    // The k expert rows' loads go out eight at a time before any is summed
+    // (the sum itself keeps slot order), so eight wait in parallel.
+    for (int j0 = 0; j0 < k; j0 += 8) {
+      uint4 raw[8];
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        const int j = j0 + jj;
+        const int row = j < k ? s_row[j] : -1;
+        raw[jj] = row >= 0 ? ld16(y_perm + (size_t)row * d + (size_t)v * V) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        const int j = j0 + jj;
+        if (j < k && s_row[j] >= 0) unpack_add<T>(acc, raw[jj], s_g[j]);
+      }
     }
     if (y_shared) unpack_add<T>(acc, ld16(y_shared + (size_t)t * d + (size_t)v * V), 1.0f);
     st16(y + (size_t)t * d + (size_t)v * V, pack<T>(acc));
@@ -179,6 +283,30 @@ cudaError_t launch_permute(int dtype, const void* x, const int* topk_idx, const 
   const int V = dtype == MOE_DTYPE_F32 ? 4 : 8;
   const int nvec = d / V;
   const int nch = ceil_div(T, kChunk);
+  // Whole rows by bulk copies when each row goes to at least four packed
+  // rows and there are at least 64 chunks (measured on B200: 12% faster at
+  // k = 8 with 128 or 512 chunks, slower at k = 2 or with a handful of
+  // chunks, where one thread's per-row chain dominates), a ring of at least
+  // two rows fits in kBulkRingBytes and both row arrays are 16-byte aligned.
+  constexpr int kBulkRingBytes = 96 * 1024;
+  const long long row_bytes = (long long)d * (dtype == MOE_DTYPE_F32 ? 4 : 2);
+  const int nbuf = (int)std::min<long long>(kMaxBulkBufs, kBulkRingBytes / row_bytes);
+  if (copy && k >= 4 && nch >= 64 && nbuf >= 2 && row_bytes % 16 == 0 &&
+      ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(x_perm)) & 15u) == 0) {
+    static int attr_done = 0;   // one bit per device ordinal (< 32)
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (!(dev < 32 && ((attr_done >> dev) & 1))) {
+      e = cudaFuncSetAttribute(permute_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kBulkRingBytes);
+      if (e != cudaSuccess) return e;
+      if (dev < 32) attr_done |= 1 << dev;
+    }
+    permute_bulk_kernel<<<nch, 128, nbuf * row_bytes, s>>>(
+        static_cast<const char*>(x), topk_idx, offsets, chunk_base, tile_base, T, E, k, (uint32_t)row_bytes, nbuf,
+        static_cast<char*>(x_perm), perm_src, inv_row, T * k, err, kDefaultTimeoutNs);
+    return cudaGetLastError();
+  }
   int nsplit = copy ? ceil_div(4 * num_sms, nch) : 1;
   if (nsplit < 1) nsplit = 1;
   if (nsplit > nvec) nsplit = nvec;
