@@ -476,9 +476,12 @@ def layer_bytes(cfg, touched):
 
 
 def stage_breakdown(B, cfg, inp, ws, stream, n):
-    """The forward through the per-stage entry points, one CUDA event between
-    stages on the launching stream, averaged over n passes. Returns the mean
-    milliseconds per stage and the stage outputs of the last pass."""
+    """The forward through the per-stage entry points, captured once as a CUDA
+    graph with a CUDA event recorded between consecutive stage calls (event
+    nodes inside the graph), replayed n times; each replay is read back before
+    the next. A stage's time is the device time between its events in a chain
+    that runs like moe_forward's graph, once per pass. Returns the mean
+    milliseconds per stage and the stage outputs (of the last pass)."""
     dev = inp["x"].device
     T, d, E, k = cfg.T, cfg.d, cfg.E, cfg.k
     rows = T * k
@@ -518,17 +521,25 @@ def stage_breakdown(B, cfg, inp, ws, stream, n):
         for c in calls:
             c()
     torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(n)]
-    for i in range(n):
-        evs[i][0].record(stream)
+    # external: recorded inside the capture as timing event nodes
+    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(calls) + 1)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        evs[0].record()
         for j, c in enumerate(calls):
             c()
-            evs[i][j + 1].record(stream)
+            evs[j + 1].record()
+    g.replay()
     torch.cuda.synchronize()
+    acc = [0.0] * len(calls)
+    for _ in range(n):
+        g.replay()
+        torch.cuda.synchronize()
+        for j in range(len(calls)):
+            acc[j] += evs[j].elapsed_time(evs[j + 1])
+    del g
     assert B.moe_get_device_error(ws) == B.MOE_OK
-    stage_ms = {nm: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(n))
-                for j, nm in enumerate(names)}
-    return stage_ms, o
+    return {nm: acc[j] / n for j, nm in enumerate(names)}, o
 
 
 def graph_step_ms(B, cfg, inp, ws, y, stream, steps, warmup):
