@@ -33,9 +33,10 @@
 //   warp 0 lane 0 : TMA producer into a ring of variable-size slots
 //   warp 1        : TMEM allocator; lane 0 issues tcgen05.mma (kind::f16,
 //                   bf16 x bf16 -> fp32 in TMEM) and tcgen05.commit
-//   warps 2..9    : epilogue, two warps per 32-lane TMEM quarter (each takes
-//                   every other 16-column chunk); tcgen05.ld, SiLU * up in
-//                   fp32, one rounding to the output type, masked stores
+//   warps 2..     : epilogue, EPI_WPQ warps per 32-lane TMEM quarter (each
+//                   takes every EPI_WPQ-th 16-column chunk); tcgen05.ld, SiLU
+//                   * up in fp32, one rounding to the output type, masked
+//                   stores
 //
 // TMEM (512 columns) holds a tile's two accumulators. Tiles of at most 128
 // token columns alternate between the two 256-column halves, so the MMAs of
@@ -71,7 +72,9 @@ constexpr int UMMA_K = 16;       // K per tcgen05.mma for 16-bit inputs
 constexpr int BN_MAX = 256;      // token columns per tile (MMA N), upper bound
 constexpr int BOX_N_MAX = 128;   // token rows per TMA box, at most
 constexpr int A_BYTES = BM * BK * 2;
-constexpr int EPI_WARPS = 8;      // warps 2..9: two per TMEM lane quarter
+constexpr int EPI_WPQ = 2;                  // epilogue warps per 32-lane TMEM quarter
+constexpr int EPI_WARPS = 4 * EPI_WPQ;      // warps 2 .. 1 + EPI_WARPS
+constexpr int EPI_CPW = (16 + EPI_WPQ - 1) / EPI_WPQ;   // 16-column chunks per warp and accumulator (256 / 16 = 16 in all)
 constexpr int GATHER_WARPS = 2;   // warps 10..11, launched only when B is gathered
 constexpr int NUM_THREADS = 32 * (2 + EPI_WARPS);                   // without gather warps
 constexpr int NUM_THREADS_GATHER = 32 * (2 + EPI_WARPS + GATHER_WARPS);
@@ -297,8 +300,12 @@ __device__ __forceinline__ TokenSlice token_slice(const UmmaLaunch& p, const Til
   return ts;
 }
 
+// Only the SwiGLU forward gathers its token rows (and launches the two
+// gather warps); the other modes keep the register budget of NUM_THREADS.
+template <int MODE> constexpr int max_threads() { return MODE == kUmmaSwiGLU ? NUM_THREADS_GATHER : NUM_THREADS; }
+
 template <int MODE, bool PAIR>
-__global__ void __launch_bounds__(NUM_THREADS_GATHER, 1)
+__global__ void __launch_bounds__(max_threads<MODE>(), 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA3,
                      const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmAs,
                      const __grid_constant__ CUtensorMap tmA3s, const __grid_constant__ CUtensorMap tmBs,
@@ -684,7 +691,7 @@ __global__ void __launch_bounds__(NUM_THREADS_GATHER, 1)
   } else if (warp >= 2 && warp < 2 + EPI_WARPS) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                  // TMEM lane quarter this warp may read
-    const int ch = (warp - 2) >> 2;          // which 16-column chunks: ch, ch + 2, ch + 4, ...
+    const int ch = (warp - 2) >> 2;          // which 16-column chunks: ch, ch + EPI_WPQ, ch + 2 EPI_WPQ, ...
     const int row = q * 32 + lane;
     // The accumulator is released to the leader's barrier (remote for the peer).
     const uint32_t acce0 = PAIR ? map_to_cta(smem_u32(&acce_bar[0]), 0) : smem_u32(&acce_bar[0]);
@@ -724,9 +731,10 @@ __global__ void __launch_bounds__(NUM_THREADS_GATHER, 1)
         if (wide) release_half(1u);
       };
       // The same for epilogues that already handed half 0 of a wide tile back
-      // once its token columns 0..127 were drained (the first four chunk
-      // pairs of each warp).
+      // once its token columns 0..127 (chunks 0..7) were drained.
       auto release_rest = [&]() { release_half(wide ? 1u : half); };
+      // Chunk cc of this warp is its last one among chunks 0..7.
+      auto last_low_chunk = [&](int cc) { return EPI_WPQ * cc + ch < 8 && EPI_WPQ * (cc + 1) + ch >= 8; };
       if (dual_a(MODE)) {
         // Drain both accumulators into registers as packed bf16 h, hand TMEM
         // back to the MMA warp, then store while the next tile accumulates.
@@ -736,11 +744,11 @@ __global__ void __launch_bounds__(NUM_THREADS_GATHER, 1)
           pre_a = static_cast<__nv_bfloat16*>(t.dense ? p.pre_a_s : p.pre_a) + r0 * ld;
           pre_b = static_cast<__nv_bfloat16*>(t.dense ? p.pre_b_s : p.pre_b) + r0 * ld;
         }
-        uint32_t hp[BN_MAX / 4];
+        uint32_t hp[EPI_CPW * 8];
 #pragma unroll
-        for (int cc = 0; cc < BN_MAX / 32; ++cc) {
-          const int c = 2 * cc + ch;
-          if (c * 16 < n_mma) {
+        for (int cc = 0; cc < EPI_CPW; ++cc) {
+          const int c = EPI_WPQ * cc + ch;
+          if (c < 16 && c * 16 < n_mma) {
             uint32_t r1[16], r3[16];
             tmem_ld16x2_wait(taddr + c * 16, taddr + off2 + c * 16, r1, r3);
             if (MODE == kUmmaSwiGLUSave && m_ok) {
@@ -767,15 +775,15 @@ __global__ void __launch_bounds__(NUM_THREADS_GATHER, 1)
               hp[cc * 8 + j] = *reinterpret_cast<const uint32_t*>(&hb);
             }
           }
-          if (cc == BN_MAX / 64 - 1 && wide) release_half(0u);   // token columns 0..127 drained
+          if (wide && last_low_chunk(cc)) release_half(0u);   // token columns 0..127 drained
         }
         release_rest();
         if (m_ok) {
           unsigned short* o = reinterpret_cast<unsigned short*>(out) + r0 * ld + m;
 #pragma unroll
-          for (int cc = 0; cc < BN_MAX / 32; ++cc) {
-            const int c = 2 * cc + ch;
-            if (c * 16 < n_valid) {
+          for (int cc = 0; cc < EPI_CPW; ++cc) {
+            const int c = EPI_WPQ * cc + ch;
+            if (c < 16 && c * 16 < n_valid) {
 #pragma unroll
               for (int j = 0; j < 16; ++j) {
                 const int col = c * 16 + j;
@@ -790,7 +798,7 @@ __global__ void __launch_bounds__(NUM_THREADS_GATHER, 1)
         const int m2 = m + BLOCK_STEP;
         const bool m2_ok = m2 < t.mrows;
         float* o = reinterpret_cast<float*>(out) + r0 * ld;
-        for (int c0 = ch * 16; c0 < n_mma; c0 += 32) {
+        for (int c0 = ch * 16; c0 < n_mma; c0 += 16 * EPI_WPQ) {
           uint32_t r1[16], r3[16];
           tmem_ld16x2_wait(taddr + c0, taddr + off2 + c0, r1, r3);
 #pragma unroll
@@ -811,11 +819,11 @@ __global__ void __launch_bounds__(NUM_THREADS_GATHER, 1)
         // stores would stop the weight stream for a large share of a tile).
         const int m2 = m + BLOCK_STEP;
         const bool m2_ok = m2 < t.mrows;
-        uint32_t q1[BN_MAX / 4], q2[BN_MAX / 4];
+        uint32_t q1[EPI_CPW * 8], q2[EPI_CPW * 8];
 #pragma unroll
-        for (int cc = 0; cc < BN_MAX / 32; ++cc) {
-          const int c = 2 * cc + ch;
-          if (c * 16 < n_mma) {
+        for (int cc = 0; cc < EPI_CPW; ++cc) {
+          const int c = EPI_WPQ * cc + ch;
+          if (c < 16 && c * 16 < n_mma) {
             uint32_t r1[16], r3[16];
             tmem_ld16x2_wait(taddr + c * 16, taddr + off2 + c * 16, r1, r3);
 #pragma unroll
@@ -826,14 +834,14 @@ __global__ void __launch_bounds__(NUM_THREADS_GATHER, 1)
               q2[cc * 8 + j] = *reinterpret_cast<const uint32_t*>(&pb);
             }
           }
-          if (cc == BN_MAX / 64 - 1 && wide) release_half(0u);   // token columns 0..127 drained
+          if (wide && last_low_chunk(cc)) release_half(0u);   // token columns 0..127 drained
         }
         release_rest();
         unsigned short* o = reinterpret_cast<unsigned short*>(out) + r0 * ld;
 #pragma unroll
-        for (int cc = 0; cc < BN_MAX / 32; ++cc) {
-          const int c = 2 * cc + ch;
-          if (c * 16 < n_valid) {
+        for (int cc = 0; cc < EPI_CPW; ++cc) {
+          const int c = EPI_WPQ * cc + ch;
+          if (c < 16 && c * 16 < n_valid) {
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               const int col = c * 16 + j;
@@ -850,7 +858,7 @@ __global__ void __launch_bounds__(NUM_THREADS_GATHER, 1)
         const int m2 = m + BLOCK_STEP;
         const bool m2_ok = m2 < t.mrows;
         __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out) + r0 * ld;
-        for (int c0 = ch * 16; c0 < n_mma; c0 += 32) {
+        for (int c0 = ch * 16; c0 < n_mma; c0 += 16 * EPI_WPQ) {
           uint32_t r1[16], r3[16];
           tmem_ld16x2_wait(taddr + c0, taddr + off2 + c0, r1, r3);
 #pragma unroll
@@ -874,7 +882,7 @@ __global__ void __launch_bounds__(NUM_THREADS_GATHER, 1)
         const float bias2 = (rb && m2_ok) ? rb[boff + m2] : 0.0f;
         const bool gelu = p.act == kActGelu;
         __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out) + r0 * ld;
-        for (int c0 = ch * 16; c0 < n_mma; c0 += 32) {
+        for (int c0 = ch * 16; c0 < n_mma; c0 += 16 * EPI_WPQ) {
           uint32_t r1[16], r3[16];
           tmem_ld16x2_wait(taddr + c0, taddr + off2 + c0, r1, r3);
 #pragma unroll
@@ -1011,7 +1019,7 @@ cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t 
   if (!has_dense) { tAs = tA; tA3s = tA3; tBs = tB; }
   // Gathered token rows are copied with cp.async: the source rows must be
   // 16-byte aligned.
-  if (p.b_gather && (!p.b_gather_src || p.b_gather_rows <= 0 ||
+  if (p.b_gather && (p.mode != kUmmaSwiGLU || !p.b_gather_src || p.b_gather_rows <= 0 ||
                      (reinterpret_cast<uintptr_t>(p.b_gather_src) & 15u) || (p.K * 2) % 16 ||
                      mine_max > GATHER_WARPS * 4 * kGatherRowsPerLane || p.b_gather_rows * p.K * 2 > 0xffffffffll))
     return cudaErrorInvalidValue;
