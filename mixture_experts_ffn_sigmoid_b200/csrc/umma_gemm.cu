@@ -29,14 +29,18 @@
 // (SwiGLU: the W1 and W3 rows of the same f range; down: 256 consecutive W2
 // rows), so two MMAs share every token tile that is staged.
 //
-// Roles (320 threads, one CTA per SM, persistent over a static tile list):
+// Roles (one CTA per SM, persistent over a static tile list):
 //   warp 0 lane 0 : TMA producer into a ring of variable-size slots
 //   warp 1        : TMEM allocator; lane 0 issues tcgen05.mma (kind::f16,
-//                   bf16 x bf16 -> fp32 in TMEM) and tcgen05.commit
-//   warps 2..     : epilogue, EPI_WPQ warps per 32-lane TMEM quarter (each
+//                   bf16 x bf16 -> fp32 in TMEM) and tcgen05.commit; in a
+//                   pair's peer CTA lane 0 forwards gathered rows' arrivals
+//   warps 2..9    : epilogue, EPI_WPQ warps per 32-lane TMEM quarter (each
 //                   takes every EPI_WPQ-th 16-column chunk); tcgen05.ld, SiLU
 //                   * up in fp32, one rounding to the output type, masked
 //                   stores
+//   warps 10..11  : launched for CTA pairs and gathered rows: lane 0 of warp
+//                   10 issues each slot's second weight block and packed token
+//                   rows, or both warps gather token rows with cp.async
 //
 // TMEM (512 columns) holds a tile's two accumulators. Tiles of at most 128
 // token columns alternate between the two 256-column halves, so the MMAs of
@@ -71,6 +75,7 @@ constexpr int BK = 64;           // K per slot: one 128-byte swizzle row of bf16
 constexpr int UMMA_K = 16;       // K per tcgen05.mma for 16-bit inputs
 constexpr int BN_MAX = 256;      // token columns per tile (MMA N), upper bound
 constexpr int BOX_N_MAX = 128;   // token rows per TMA box, at most
+constexpr int kSplitB = 1;       // CTA pairs: a second thread issues part of each slot's copies
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int EPI_WPQ = 2;                  // epilogue warps per 32-lane TMEM quarter
 constexpr int EPI_WARPS = 4 * EPI_WPQ;      // warps 2 .. 1 + EPI_WARPS
@@ -229,7 +234,9 @@ __host__ __device__ constexpr int tile_rows(int mode, bool pair) {
 // overhead whatever its size, and a slot completes only when all of its
 // copies have, so a CTA's token rows of a slot come in one copy.
 struct UmmaLaunch : UmmaGemmParams {
-  int box_n;   // token rows per copy of B: a multiple of 8, at most 128
+  int box_n;     // token rows per copy of B: a multiple of 8, at most 128
+  int split_b;   // a second thread (warp 2 + EPI_WARPS, lane 0) issues each slot's second
+                 // weight block and its packed token rows (CTA pairs only)
 };
 
 struct Tile {
@@ -300,9 +307,9 @@ __device__ __forceinline__ TokenSlice token_slice(const UmmaLaunch& p, const Til
   return ts;
 }
 
-// Only the SwiGLU forward gathers its token rows (and launches the two
-// gather warps); the other modes keep the register budget of NUM_THREADS.
-template <int MODE> constexpr int max_threads() { return MODE == kUmmaSwiGLU ? NUM_THREADS_GATHER : NUM_THREADS; }
+// The warps after the epilogue's gather the SwiGLU forward's token rows,
+// or (split_b) the first of them issues the packed token rows' copies.
+template <int MODE> constexpr int max_threads() { return NUM_THREADS_GATHER; }
 
 template <int MODE, bool PAIR>
 __global__ void __launch_bounds__(max_threads<MODE>(), 1)
@@ -468,7 +475,7 @@ __global__ void __launch_bounds__(max_threads<MODE>(), 1)
         fl_off[slot] = off;
         fl_size[slot] = bytes;
         ++inflight;
-        if (gather) mbar_arrive(smem_u32(&acq_bar[slot]));
+        if (gather || p.split_b) mbar_arrive(smem_u32(&acq_bar[slot]));
         const uint32_t fb_local = smem_u32(&full_bar[slot]);
         const uint32_t sb = smem_u32(ring + off);
         const uint32_t bb = sb + A_TILES * A_BYTES;
@@ -489,10 +496,10 @@ __global__ void __launch_bounds__(max_threads<MODE>(), 1)
                                  crow, fb);
           } else {
             tma_load_2d_pair(sb, mA, kb * BK, a_row, fb);
-            if (dual_a(MODE)) tma_load_2d_pair(sb + A_BYTES, mA3, kb * BK, a_row, fb);
-            if (two_blocks(MODE)) tma_load_2d_pair(sb + A_BYTES, mA, kb * BK, a_row + BLOCK_STEP, fb);
+            if (dual_a(MODE) && !p.split_b) tma_load_2d_pair(sb + A_BYTES, mA3, kb * BK, a_row, fb);
+            if (two_blocks(MODE) && !p.split_b) tma_load_2d_pair(sb + A_BYTES, mA, kb * BK, a_row + BLOCK_STEP, fb);
           }
-          if (ts.rows_gather == 0)
+          if (ts.rows_gather == 0 && !p.split_b)
             for (int bx = 0; bx < ts.nbox; ++bx)
               tma_load_2d_pair(bb + bx * ts.box_bytes, mB, kb * BK, ts.row + bx * p.box_n, fb);
         } else {
@@ -512,7 +519,7 @@ __global__ void __launch_bounds__(max_threads<MODE>(), 1)
             if (dual_a(MODE)) tma_load_2d(sb + A_BYTES, mA3, kb * BK, a_row, fb_local);
             if (two_blocks(MODE)) tma_load_2d(sb + A_BYTES, mA, kb * BK, a_row + BLOCK_STEP, fb_local);
           }
-          if (ts.rows_gather == 0)
+          if (ts.rows_gather == 0 && !p.split_b)
             for (int bx = 0; bx < ts.nbox; ++bx)
               tma_load_2d(bb + bx * ts.box_bytes, mB, kb * BK, ts.row + bx * p.box_n, fb_local);
         }
@@ -528,6 +535,48 @@ __global__ void __launch_bounds__(max_threads<MODE>(), 1)
       else
         wait_bounded(smem_u32(&full_bar[u % NSLOT]), (u / NSLOT) & 1u, abort_flag, p.err,
                      p.timeout_ns, false);
+    }
+  } else if (p.split_b && warp == 2 + EPI_WARPS && lane == 0) {
+    // ------------------------------------------------------------ second issuer
+    // One thread's copy issue paces the weight stream (each copy costs its
+    // issuer a fixed time, whatever the size), so on CTA pairs a second
+    // thread takes the slot's second weight block (W3, or down's block a
+    // block step further) and its packed token rows, once the producer has
+    // claimed the slot (same ring walk, so the same offsets). The copies
+    // complete on the slot's full barrier, which the producer armed for all.
+    RingCursor cur;
+    bool ok = true;
+    for (int tile = group; tile < total_tiles && ok; tile += ngroups) {
+      const Tile t = decode_tile(p, s_off, s_start, nseg, tile, WROWS);
+      const TokenSlice ts = token_slice<PAIR>(p, t, rank);
+      const CUtensorMap* mB = t.dense ? &tmBs : &tmB;
+      const uint32_t bytes = A_TILES * A_BYTES + ts.bytes();
+      const int nk = ceil_div(t.K, BK);
+      for (int kb = 0; kb < nk; ++kb) {
+        const uint32_t u = cur.count;
+        uint32_t off, slot, parity;
+        cur.take(bytes, cap, off, slot, parity);
+        if (!wait_bounded(smem_u32(&acq_bar[slot]), (u / NSLOT) & 1u, abort_flag, p.err, p.timeout_ns, true)) {
+          ok = false;
+          break;
+        }
+        const uint32_t bb = smem_u32(ring + off) + A_TILES * A_BYTES;
+        const uint32_t fb_local = smem_u32(&full_bar[slot]);
+        if (PAIR && MODE != kUmmaDgrad) {   // the slot's second weight block
+          const int a_row = (t.dense ? 0 : t.seg * p.m_rows) + t.wt * WROWS + (int)rank * BM;
+          const CUtensorMap* mA = t.dense ? &tmAs : &tmA;
+          const CUtensorMap* mA3 = t.dense ? &tmA3s : &tmA3;
+          const uint32_t sb = smem_u32(ring + off);
+          if (dual_a(MODE)) tma_load_2d_pair(sb + A_BYTES, mA3, kb * BK, a_row, map_to_cta(fb_local, 0));
+          if (two_blocks(MODE)) tma_load_2d_pair(sb + A_BYTES, mA, kb * BK, a_row + BLOCK_STEP, map_to_cta(fb_local, 0));
+        }
+        for (int bx = 0; bx < ts.nbox; ++bx) {
+          if (PAIR)
+            tma_load_2d_pair(bb + bx * ts.box_bytes, mB, kb * BK, ts.row + bx * p.box_n, map_to_cta(fb_local, 0));
+          else
+            tma_load_2d(bb + bx * ts.box_bytes, mB, kb * BK, ts.row + bx * p.box_n, fb_local);
+        }
+      }
     }
   } else if (gather && warp >= 2 + EPI_WARPS) {
     // ------------------------------------------------------------ gather
@@ -947,7 +996,7 @@ cudaError_t launch_mode(const CUtensorMap& tA, const CUtensorMap& tA3, const CUt
                         cudaStream_t s) {
   cudaError_t e = ensure_smem_attr<MODE, PAIR>();
   if (e != cudaSuccess) return e;
-  const int threads = p.b_gather ? NUM_THREADS_GATHER : NUM_THREADS;
+  const int threads = (p.b_gather || p.split_b) ? NUM_THREADS_GATHER : NUM_THREADS;
   if (!PAIR) {
     umma_gemm_kernel<MODE, false><<<grid, threads, smem, s>>>(tA, tA3, tB, tAs, tA3s, tBs, p);
     return cudaGetLastError();
@@ -987,6 +1036,10 @@ cudaError_t launch_umma_gemm(const UmmaGemmParams& p, int num_sms, cudaStream_t 
   // CTA stages (rounded to the 8-row swizzle atom), at most 128 rows.
   const int mine_max = pair ? p.bn_max / 2 : p.bn_max;
   q.box_n = ((mine_max + 7) & ~7) < BOX_N_MAX ? ((mine_max + 7) & ~7) : BOX_N_MAX;
+  // Second issuing thread on CTA pairs (wide token tiles), where a slot's
+  // copies are many bytes and the issuing thread paces the stream; single
+  // CTAs (decode) stage a few token rows per slot and keep one issuer.
+  q.split_b = (p.b_gather || !pair) ? 0 : kSplitB;
   if (sp.ring_bytes < 2 * (a_tiles * A_BYTES + ceil_div(mine_max, q.box_n) * q.box_n * BK * 2))
     return cudaErrorInvalidValue;
   const bool swiglu = dual_a(p.mode);
