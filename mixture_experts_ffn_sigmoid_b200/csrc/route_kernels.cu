@@ -5,7 +5,8 @@
 // Used for fp32 inputs and for more than 256 experts; the bf16 router of up
 // to 256 experts runs fused with its GEMM (router_fused.cu).
 //
-// Layout: one warp per token, lane l holds experts l, l+32, l+64, ...; a
+// Layout: one warp per token, each lane holding the experts route_expert
+// gives it (NPL consecutive experts up to 256, else l, l+32, ...); a
 // block of 32 warps is one chunk of 32 tokens, so the same block can also
 // emit the chunk's per-expert histogram (a bit mask per expert: bit w set
 // when token w of the chunk chose the expert). Histograms are exact and the
@@ -35,7 +36,7 @@ __global__ void __launch_bounds__(1024, 1) router_topk_kernel(RouteParams p) {
     float lg[NPL];
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
-      const int e = lane + 32 * i;
+      const int e = route_expert<NPL>(lane, i);
       float l = 0.0f;
       if (e < E) {
         // Router partial sums (a split contraction) add up in a fixed order;
@@ -49,7 +50,7 @@ __global__ void __launch_bounds__(1024, 1) router_topk_kernel(RouteParams p) {
     const TopkArgs a = {E, k, p.gate_mode, p.n_groups, p.topk_groups, p.route_scale, p.bias};
     int my_e, pos;
     float gate;
-    route_token<NPL>(lg, lane, a, my_e, pos, gate, lrow);
+    route_token<NPL>(lg, lane, a, my_e, pos, gate, NPL > 8 ? lrow : nullptr);
     if (lane < k) {
       p.topk_idx[(size_t)t * k + pos] = my_e;
       p.topk_gate[(size_t)t * k + pos] = gate;

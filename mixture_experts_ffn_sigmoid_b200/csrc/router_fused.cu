@@ -72,8 +72,39 @@ struct FusedRouterArgs {
 __host__ __device__ inline int fr_stage_bytes(int n_pad) { return FR_A_BYTES + n_pad * FR_BK * 2; }
 __host__ __device__ inline int fr_smem_bytes(int n_pad) {
   // alignment slack, header, ring (also the partial-logit buffer), the tile's
-  // chunk masks [kTileChunks][256] and the scan's partial sums [4][256]
-  return 1024 + FR_HDR + FR_STAGES * fr_stage_bytes(n_pad) + kTileChunks * 256 * 4 + 4 * 256 * 4 + 256;
+  // chunk masks [kTileChunks][256], the scan's partial sums [4][256] and the
+  // selection bias [256]
+  return 1024 + FR_HDR + FR_STAGES * fr_stage_bytes(n_pad) + kTileChunks * 256 * 4 + 4 * 256 * 4 + 256 * 4 + 256;
+}
+
+// NPL consecutive fp32 values (NPL = 1, 2, 4 or 8) from the shared memory of
+// a CTA of the cluster; the address is aligned to min(NPL, 4) * 4 bytes.
+template <int NPL>
+__device__ __forceinline__ void ld_cluster_vec(uint32_t a, float (&v)[NPL]) {
+  if constexpr (NPL == 1) {
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v[0]) : "r"(a) : "memory");
+  } else if constexpr (NPL == 2) {
+    asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v[0]), "=f"(v[1]) : "r"(a) : "memory");
+  } else {
+#pragma unroll
+    for (int h = 0; h < NPL / 4; ++h)
+      asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                   : "=f"(v[4 * h]), "=f"(v[4 * h + 1]), "=f"(v[4 * h + 2]), "=f"(v[4 * h + 3])
+                   : "r"(a + 16u * h) : "memory");
+  }
+}
+// The same number of values to this CTA's shared memory, same alignment.
+template <int NPL>
+__device__ __forceinline__ void st_shared_vec(float* dst, const float (&v)[NPL]) {
+  if constexpr (NPL == 1) {
+    dst[0] = v[0];
+  } else if constexpr (NPL == 2) {
+    *reinterpret_cast<float2*>(dst) = make_float2(v[0], v[1]);
+  } else {
+#pragma unroll
+    for (int h = 0; h < NPL / 4; ++h)
+      reinterpret_cast<float4*>(dst)[h] = make_float4(v[4 * h], v[4 * h + 1], v[4 * h + 2], v[4 * h + 3]);
+  }
 }
 
 template <int NPL>
@@ -97,6 +128,7 @@ __global__ void __launch_bounds__(FR_THREADS, 1)
   const int ld_log = p.n_pad + 4;                               // 16-byte rows, conflict-free float4 stores
   uint32_t* s_mask = reinterpret_cast<uint32_t*>(ring + FR_STAGES * stage_bytes);   // [kTileChunks][256]
   int* s_part = reinterpret_cast<int*>(s_mask + kTileChunks * 256);                 // [4][256]
+  float* s_bias = reinterpret_cast<float*>(s_part + 4 * 256);                       // [256]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
@@ -121,6 +153,8 @@ __global__ void __launch_bounds__(FR_THREADS, 1)
     tmap_prefetch(&tmW);
   }
   for (int i = threadIdx.x; i < kTileChunks * 256; i += blockDim.x) s_mask[i] = 0u;
+  if (p.topk.bias)   // every token of the tile reads all of it
+    for (int i = threadIdx.x; i < E; i += blockDim.x) s_bias[i] = p.topk.bias[i];
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), FR_TMEM_COLS);
     tmem_relinquish();
@@ -227,32 +261,77 @@ __global__ void __launch_bounds__(FR_THREADS, 1)
   const int nch_tile = min(kTileChunks, ceil_div(p.T - t0, kChunk));
   const int tile_tokens = min(FR_BM, p.T - t0);
   const int k = p.topk.k;
+  TopkArgs tk = p.topk;
+  if (tk.bias) tk.bias = s_bias;
+  // route_token takes lane l's experts l*NPL .. l*NPL + NPL - 1 (its blocked
+  // layout); columns past n_pad are not there, and columns E .. n_pad - 1
+  // hold zeros the routing ignores.
   for (int tl = (int)rank + (int)S * warp; tl < tile_tokens; tl += (int)S * 32) {
     const int t = t0 + tl;
     const int j = tl / kChunk;
     {   // one warp, one token
-      // Partial sums of the NPL held experts, CTA by CTA in rank order; the
-      // NPL loads of one CTA are issued back to back.
+      // Partial sums, CTA by CTA in rank order; the shares of up to QB CTAs
+      // are requested before the first of them is added (QB * NPL values in
+      // registers). Each load instruction of the warp reads one contiguous
+      // run of the row (lane l: columns 4l .. 4l + 3 of each 128-column
+      // half with eight per lane), so no two lanes share a bank; with eight
+      // per lane the sums then go through this CTA's row into the blocked
+      // layout.
+      constexpr uint32_t QB = NPL >= 8 ? 4 : 8;
+      constexpr int VW = NPL >= 4 ? 4 : NPL;       // values per vector
       float lg[NPL];
-      const uint32_t row = smem_u32(s_log + tl * ld_log + lane);
-      for (uint32_t q = 0; q < S; ++q) {
-        const uint32_t base = map_to_cta(row, q);
-        float part[NPL];
+      float* own = s_log + tl * ld_log;
+      auto col = [&](int h) { return NPL >= 8 ? 128 * h + 4 * lane : lane * NPL; };
+      bool hv[NPL / VW];
 #pragma unroll
-        for (int i = 0; i < NPL; ++i) part[i] = lane + 32 * i < E ? ld_cluster_f32(base + 128u * i) : 0.0f;
+      for (int h = 0; h < NPL / VW; ++h) hv[h] = col(h) < p.n_pad;
 #pragma unroll
-        for (int i = 0; i < NPL; ++i) lg[i] = q == 0 ? part[i] : lg[i] + part[i];
+      for (int i = 0; i < NPL; ++i) lg[i] = 0.0f;
+#pragma unroll
+      for (uint32_t q0 = 0; q0 < 8; q0 += QB) {
+        if (q0 < S) {
+          float part[QB][NPL];
+#pragma unroll
+          for (uint32_t b = 0; b < QB; ++b) {
+#pragma unroll
+            for (int h = 0; h < NPL / VW; ++h) {
+              float* dst = &part[b][h * VW];
+              if (hv[h] && q0 + b < S) {
+                ld_cluster_vec<VW>(map_to_cta(smem_u32(own + col(h)), q0 + b),
+                                   *reinterpret_cast<float(*)[VW]>(dst));
+              } else {
+#pragma unroll
+                for (int i = 0; i < VW; ++i) dst[i] = 0.0f;
+              }
+            }
+          }
+#pragma unroll
+          for (uint32_t b = 0; b < QB; ++b) {
+            if (q0 + b < S) {
+#pragma unroll
+              for (int i = 0; i < NPL; ++i) lg[i] = q0 + b == 0 ? part[b][i] : lg[i] + part[b][i];
+            }
+          }
+        }
       }
       // The sums replace this CTA's own partials of the token (a token's
       // rows are read only by the CTA that routes it), to be copied out after
       // the handshake.
-      float* own = s_log + tl * ld_log;
 #pragma unroll
-      for (int i = 0; i < NPL; ++i)
-        if (lane + 32 * i < E) own[lane + 32 * i] = lg[i];
+      for (int h = 0; h < NPL / VW; ++h)
+        if (hv[h]) st_shared_vec<VW>(own + col(h), *reinterpret_cast<const float(*)[VW]>(&lg[h * VW]));
+      if constexpr (NPL >= 8) {   // into the blocked layout
+        __syncwarp();
+        const bool have = lane * NPL < p.n_pad;
+#pragma unroll
+        for (int h = 0; h < NPL / 4; ++h) {
+          const float4 v = have ? reinterpret_cast<const float4*>(own + lane * NPL)[h] : make_float4(0.f, 0.f, 0.f, 0.f);
+          lg[4 * h] = v.x; lg[4 * h + 1] = v.y; lg[4 * h + 2] = v.z; lg[4 * h + 3] = v.w;
+        }
+      }
       int my_e, pos;
       float gate;
-      route_token<NPL>(lg, lane, p.topk, my_e, pos, gate);
+      route_token<NPL>(lg, lane, tk, my_e, pos, gate, own);
       if (lane < k) {
         p.topk_idx[(size_t)t * k + pos] = my_e;
         p.topk_gate[(size_t)t * k + pos] = gate;
@@ -266,13 +345,25 @@ __global__ void __launch_bounds__(FR_THREADS, 1)
   // ------------------------------------------------------------ tile histogram (CTA 0)
   if (rank == 0) {
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      // every CTA's masks of every chunk requested before any is used
+      uint32_t m[kTileChunks];
+#pragma unroll
+      for (int j = 0; j < kTileChunks; ++j) m[j] = 0u;
+#pragma unroll
+      for (uint32_t q = 0; q < 8; ++q) {
+        if (q < S) {
+#pragma unroll
+          for (int j = 0; j < kTileChunks; ++j)
+            if (j < nch_tile) m[j] |= ld_cluster_u32(map_to_cta(smem_u32(&s_mask[j * 256 + e]), q));
+        }
+      }
       int run = 0;
-      for (int j = 0; j < nch_tile; ++j) {
-        const uint32_t a = smem_u32(&s_mask[j * 256 + e]);
-        uint32_t m = 0u;
-        for (uint32_t q = 0; q < S; ++q) m |= ld_cluster_u32(map_to_cta(a, q));
-        p.chunk_base[(size_t)(tile * kTileChunks + j) * E + e] = run;
-        run += __popc(m);
+#pragma unroll
+      for (int j = 0; j < kTileChunks; ++j) {
+        if (j < nch_tile) {
+          p.chunk_base[(size_t)(tile * kTileChunks + j) * E + e] = run;
+          run += __popc(m[j]);
+        }
       }
       p.tile_hist[(size_t)tile * E + e] = run;
     }
@@ -295,35 +386,56 @@ __global__ void __launch_bounds__(FR_THREADS, 1)
   // ------------------------------------------------------------ last tile: scan
   // The block barrier orders every thread's chunk bases and tile-histogram
   // stores before thread 0's fence (a cumulative gpu-scope fence), which
-  // orders them before the counter increment that publishes them.
+  // orders them before the counter increment that publishes them. On the
+  // last tile thread 0 fences again after reading the counter, and the block
+  // barrier after it passes that ordering on to every thread, so the other
+  // tiles' histograms are visible to the scan. (One fence per CTA: a fence
+  // in each of the 1024 threads costs microseconds.)
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
     const uint32_t prev = atomicAdd(p.done_count, 1u);
-    *s_last = prev == (uint32_t)(p.ntiles - 1) ? 1 : 0;
+    const bool last = prev == (uint32_t)(p.ntiles - 1);
+    if (last) __threadfence();
+    *s_last = last ? 1 : 0;
   }
   __syncthreads();
   if (!*s_last) {
     store_logits();
     return;
   }
-  __threadfence();
   // Four groups of 256 threads, each over a quarter of the tiles: its partial
   // per-expert sums, then each tile's base from the groups before it.
   const int g = threadIdx.x >> 8, e = threadIdx.x & 255;
+  // Loads go out eight at a time before any is added; with at most eight
+  // tiles per group (up to 32 tiles) they stay in registers for the bases.
+  constexpr int kBatch = 8;
   const int per = ceil_div(p.ntiles, 4);
   const int i0 = min(p.ntiles, g * per), i1 = min(p.ntiles, i0 + per);
+  int h[kBatch];
   int part = 0;
   if (e < E)
-    for (int i = i0; i < i1; ++i) part += __ldcg(&p.tile_hist[(size_t)i * E + e]);
+    for (int i = i0; i < i1; i += kBatch) {
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) h[u] = i + u < i1 ? __ldcg(&p.tile_hist[(size_t)(i + u) * E + e]) : 0;
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) part += h[u];
+    }
   s_part[g * 256 + e] = part;
   __syncthreads();
   if (e < E) {
     int run = 0;
     for (int gg = 0; gg < g; ++gg) run += s_part[gg * 256 + e];
-    for (int i = i0; i < i1; ++i) {
-      p.tile_base[(size_t)i * E + e] = run;
-      run += __ldcg(&p.tile_hist[(size_t)i * E + e]);
+    for (int i = i0; i < i1; i += kBatch) {
+      if (per > kBatch) {   // the registers hold the last batch only: reload
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) h[u] = i + u < i1 ? __ldcg(&p.tile_hist[(size_t)(i + u) * E + e]) : 0;
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        if (i + u < i1) p.tile_base[(size_t)(i + u) * E + e] = run;
+        run += h[u];
+      }
     }
   }
   // Counts, then offsets = exclusive scan of the counts over experts (threads 0..255).
