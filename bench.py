@@ -45,12 +45,13 @@ sys.path.insert(0, ROOT)
 import torch  # noqa: E402
 
 METRIC = "MoE-layer tokens/s and active TFLOP/s at DeepSeek-V3 shape; % bf16 / HBM roofline"
-def kernels_per_forward(cfg) -> int:
+def kernels_per_forward(B, cfg, x) -> int:
     """Kernel launches of one moe_forward: the fused router (bf16, E <= 256)
-    or router GEMM + top-k + chunk scan + offsets, then permute, gate/up,
-    down and combine."""
+    or router GEMM + top-k + chunk scan + offsets, then permute (left out
+    when the router writes the row maps itself), gate/up, down and combine."""
     fused = cfg.dtype == "bf16" and cfg.E <= 256
-    return (1 if fused else 4) + 4
+    maps_in_route = B.moe_forward_gathers_rows(cfg, x) and B.moe_route_maps_supported(cfg)
+    return (1 if fused else 4) + (3 if maps_in_route else 4)
 CPU_SAMPLE_TOKENS = {"tiny_fp32": 64, "decode_fine": 32, "deepseek_v3": 16, "mixtral_8x7b": 8,
                      "deepseek_v3_skewed": 64}
 REF_STEP_TOKENS = {"tiny_fp32": 64, "decode_fine": 8, "deepseek_v3": 2, "mixtral_8x7b": 2,
@@ -501,12 +502,19 @@ def stage_breakdown(B, cfg, inp, ws, stream, n):
              y=torch.empty((T, d), dtype=dt, device=dev))
     names = ["route", "permute", "gate_up", "down", "combine"]
     # The same path moe_forward takes: packed rows, or (single-CTA token
-    # tiles) the maps-only permute and the GEMM gathering rows from x.
+    # tiles) the row maps only and the GEMM gathering rows from x; the maps
+    # come from the router itself when the batch is one router tile (the
+    # permute stage is then empty: the time between two adjacent events).
     gather = B.moe_forward_gathers_rows(cfg, inp["x"])
+    maps_in_route = gather and B.moe_route_maps_supported(cfg)
     calls = [
-        lambda: B.moe_route(cfg, inp["x"], inp["w_router"], inp["bias"], o["idx"], o["gate"], o["counts"],
-                            o["offsets"], ws),
-        (lambda: B.moe_permute(cfg, None, o["idx"], o["offsets"], None, o["perm_src"], o["inv_row"], ws)) if gather
+        (lambda: B.moe_route_maps(cfg, inp["x"], inp["w_router"], inp["bias"], o["idx"], o["gate"], o["counts"],
+                                  o["offsets"], o["perm_src"], o["inv_row"], ws)) if maps_in_route
+        else (lambda: B.moe_route(cfg, inp["x"], inp["w_router"], inp["bias"], o["idx"], o["gate"], o["counts"],
+                                  o["offsets"], ws)),
+        (lambda: None) if maps_in_route
+        else (lambda: B.moe_permute(cfg, None, o["idx"], o["offsets"], None, o["perm_src"], o["inv_row"], ws))
+        if gather
         else (lambda: B.moe_permute(cfg, inp["x"], o["idx"], o["offsets"], o["x_perm"], o["perm_src"],
                                     o["inv_row"], ws)),
         (lambda: B.moe_expert_gate_up_gather(cfg, inp["x"], o["perm_src"], o["offsets"], inp["w1"], inp["w3"],
@@ -931,7 +939,7 @@ def main():
                     "h2d_bytes_per_step": T * d * cfg.elem_bytes, "d2h_bytes_per_step": T * d * cfg.elem_bytes,
                     "ms_per_step": e2e_ms},
             "workloads": extra,
-            "gpu_launches": kernels_per_forward(cfg) * args.steps,
+            "gpu_launches": kernels_per_forward(B, cfg, inp["x"]) * args.steps,
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

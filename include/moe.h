@@ -165,6 +165,31 @@ MOE_API moe_status moe_route(const moe_config* cfg, const void* x, const void* w
                      void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * moe_route_maps - moe_route plus the row maps of moe_permute's x_perm = NULL
+ * form, from the same single launch: for a batch that is one tile of the
+ * fused router (bf16, E <= 256, T <= 128), whose last step already holds the
+ * offsets and every chunk's selections. moe_forward takes this path when its
+ * gate/up GEMM gathers the token rows (decode-sized batches). [DS]
+ * "Routing" and "Packed forward".
+ *
+ *   x .. expert_offsets   as moe_route
+ *   perm_src       [T*k]      int32   OUT: source token of each packed row
+ *   inv_row        [T][k]     int32   OUT: packed row of (token, slot)
+ *
+ * The results equal moe_route followed by moe_permute(x_perm = NULL).
+ * Anywhere else (fp32, E > 256, T > 128) it returns MOE_ERR_UNSUPPORTED and
+ * writes nothing; moe_route_maps_supported says beforehand.
+ */
+MOE_API moe_status moe_route_maps(const moe_config* cfg, const void* x, const void* w_router,
+                          const float* bias, int32_t* topk_idx, float* topk_gate,
+                          int32_t* expert_counts, int32_t* expert_offsets, int32_t* perm_src,
+                          int32_t* inv_row, void* workspace, size_t ws_bytes, void* stream);
+
+/* 1 when moe_route_maps runs for cfg, 0 when it would return
+ * MOE_ERR_UNSUPPORTED, -1 for an invalid cfg. Host-only. */
+MOE_API int moe_route_maps_supported(const moe_config* cfg);
+
+/*
  * moe_permute - gather token rows into expert-contiguous order.
  * [DS] "Packed forward": for each expert, gather the tokens whose indices
  * equal it; [KB] the per-expert mask loop.

@@ -35,7 +35,7 @@ EXPORTED = ("moe_check_config", "moe_workspace_size", "moe_route", "moe_permute"
             "moe_expert_swiglu", "moe_expert_gate_up", "moe_expert_gate_up_gather", "moe_expert_down",
             "moe_combine", "moe_forward", "moe_get_device_error",
             "moe_selftest_wait_timeout", "moe_route_noalloc", "moe_route_noalloc_device_error",
-            "moe_forward_gathers_rows",
+            "moe_forward_gathers_rows", "moe_route_maps", "moe_route_maps_supported",
             "moe_balance_update",
             "moe_expert_gelu", "moe_forward_gelu", "moe_backward_workspace_size", "moe_backward",
             "moe_forward_train", "moe_backward_saved", "moe_status_string")
@@ -90,6 +90,8 @@ def lib() -> ctypes.CDLL:
             "moe_route_noalloc": (ctypes.c_int, [cfgp, vp, vp, f32p, i32p, f32p, i32p, i32p, vp]),
             "moe_route_noalloc_device_error": (ctypes.c_int, [vp]),
             "moe_forward_gathers_rows": (ctypes.c_int, [cfgp, vp]),
+            "moe_route_maps": (ctypes.c_int, [cfgp, vp, vp, f32p, i32p, f32p, i32p, i32p, i32p, i32p, vp, sz, vp]),
+            "moe_route_maps_supported": (ctypes.c_int, [cfgp]),
             "moe_balance_update": (ctypes.c_int, [cfgp, i32p, f32p, ctypes.c_float, f32p, vp]),
             "moe_expert_gelu": (ctypes.c_int, [cfgp, vp, i32p, vp, f32p, vp, f32p, vp, vp, sz, vp]),
             "moe_forward_gelu": (ctypes.c_int, [cfgp, vp, vp, f32p, vp, f32p, vp, f32p, vp, vp, sz, vp]),
@@ -240,6 +242,28 @@ def moe_route(cfg, x, w_router, bias, topk_idx, topk_gate, expert_counts, expert
     _check(lib().moe_route(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(topk_idx),
                            _ptr(topk_gate), _ptr(expert_counts), _ptr(expert_offsets),
                            _ptr(workspace), workspace.numel(), _stream(stream)), "moe_route")
+
+
+def moe_route_maps(cfg, x, w_router, bias, topk_idx, topk_gate, expert_counts, expert_offsets, perm_src,
+                   inv_row, workspace, stream=None):
+    """moe_route plus the maps-only permute in one launch (one-tile batches)."""
+    c = _cfg(cfg)
+    _need_routing_io(c, x, w_router, bias, topk_idx, topk_gate, expert_counts, expert_offsets)
+    _need(perm_src, "perm_src", c.T * c.k, _I32)
+    _need(inv_row, "inv_row", c.T * c.k, _I32)
+    _need_ws(workspace)
+    _check(lib().moe_route_maps(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(topk_idx),
+                                _ptr(topk_gate), _ptr(expert_counts), _ptr(expert_offsets), _ptr(perm_src),
+                                _ptr(inv_row), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "moe_route_maps")
+
+
+def moe_route_maps_supported(cfg) -> bool:
+    """Whether moe_route_maps runs for cfg (else it returns MOE_ERR_UNSUPPORTED)."""
+    r = lib().moe_route_maps_supported(ctypes.byref(_cfg(cfg)))
+    if r < 0:
+        raise MoEError(MOE_ERR_INVALID_ARG, "moe_route_maps_supported")
+    return r == 1
 
 
 def moe_permute(cfg, x, topk_idx, expert_offsets, x_perm, perm_src, inv_row, workspace, stream=None):

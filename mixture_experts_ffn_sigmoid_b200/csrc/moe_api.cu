@@ -140,16 +140,27 @@ moe_status check_ws(const moe_config& c, void* ws, size_t ws_bytes) {
   return MOE_OK;
 }
 
-// Router logits -> top-k, gates, chunk histograms -> counts, chunk bases, offsets.
+// Whether enqueue_route can also write the permute's row maps: the fused
+// router with a single 128-token tile, whose last step knows the offsets and
+// every chunk's masks (decode-sized batches).
+bool route_writes_maps(const moe_config& c) { return fused_route(c) && c.T <= 128; }
+
+// Router logits -> top-k, gates, chunk histograms -> counts, chunk bases,
+// offsets; with inv_row and perm_src (only where route_writes_maps) also the
+// row maps the permute would write.
 moe_status enqueue_route(const moe_config& c, const void* x, const void* w_router, const float* bias,
-                         int* idx, float* gate, int* counts, int* offsets, void* ws, cudaStream_t s) {
+                         int* idx, float* gate, int* counts, int* offsets, void* ws, cudaStream_t s,
+                         int* inv_row = nullptr, int* perm_src = nullptr) {
   const Layout L = layout_of(c);
   float* logits = at<float>(ws, L.logits);
   const TopkArgs tk = {c.E, c.k, c.gate_mode, c.n_groups, c.topk_groups, c.route_scale, bias};
+  if ((inv_row || perm_src) && !route_writes_maps(c)) return MOE_ERR_INVALID_ARG;
   if (fused_route(c)) {
-    const FusedRouterLaunch a = {x, w_router, c.T, c.E, c.d, tk, logits, idx, gate, at<int>(ws, L.cbase),
-                                 at<int>(ws, L.thist), at<int>(ws, L.tbase), counts, offsets,
-                                 at<uint32_t>(ws, L.err), at<uint32_t>(ws, L.err + kDoneCountOffset)};
+    FusedRouterLaunch a = {x, w_router, c.T, c.E, c.d, tk, logits, idx, gate, at<int>(ws, L.cbase),
+                           at<int>(ws, L.thist), at<int>(ws, L.tbase), counts, offsets,
+                           at<uint32_t>(ws, L.err), at<uint32_t>(ws, L.err + kDoneCountOffset)};
+    a.inv_row = inv_row;
+    a.perm_src = perm_src;
     MOE_CUDA(launch_router_fused(a, s));
     return MOE_OK;
   }
@@ -784,6 +795,40 @@ moe_status moe_route(const moe_config* cfg, const void* x, const void* w_router,
                        workspace, s);
 }
 
+moe_status moe_route_maps(const moe_config* cfg, const void* x, const void* w_router, const float* bias,
+                          int32_t* topk_idx, float* topk_gate, int32_t* expert_counts,
+                          int32_t* expert_offsets, int32_t* perm_src, int32_t* inv_row, void* workspace,
+                          size_t ws_bytes, void* stream) {
+  TraceRange trace("moe_route_maps");
+  MOE_TRY(check_config(cfg));
+  const moe_config& c = *cfg;
+  if (!route_writes_maps(c)) return MOE_ERR_UNSUPPORTED;
+  MOE_TRY(need4(expert_counts));
+  MOE_TRY(need4(expert_offsets));
+  MOE_TRY(check_ws(c, workspace, ws_bytes));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (c.T == 0) {
+    MOE_CUDA(cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * c.E, s));
+    MOE_CUDA(cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (c.E + 1), s));
+    return MOE_OK;
+  }
+  MOE_TRY(need(x));
+  MOE_TRY(need(w_router));
+  MOE_TRY(need4(topk_idx));
+  MOE_TRY(need4(topk_gate));
+  MOE_TRY(need4(perm_src));
+  MOE_TRY(need4(inv_row));
+  if (bias) MOE_TRY(need4(bias));
+  MOE_TRY(clear_error_word(workspace, s));
+  return enqueue_route(c, x, w_router, bias, topk_idx, topk_gate, expert_counts, expert_offsets,
+                       workspace, s, inv_row, perm_src);
+}
+
+int moe_route_maps_supported(const moe_config* cfg) {
+  if (check_config(cfg) != MOE_OK) return -1;
+  return route_writes_maps(*cfg) ? 1 : 0;
+}
+
 moe_status moe_permute(const moe_config* cfg, const void* x, const int32_t* topk_idx,
                        const int32_t* expert_offsets, void* x_perm, int32_t* perm_src,
                        int32_t* inv_row, void* workspace, size_t ws_bytes, void* stream) {
@@ -969,16 +1014,21 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
   int* idx = at<int>(ws, L.idx);
   float* gate = at<float>(ws, L.gate);
   int* offsets = at<int>(ws, L.offsets);
-  {
-    TraceRange stage("moe_forward.route");
-    MOE_TRY(enqueue_route(c, x, w_router, bias, idx, gate, at<int>(ws, L.counts), offsets, ws, s));
-  }
   // Token rows for the gate/up GEMM. With single-CTA token tiles (few
   // tokens per expert, e.g. decode) the GEMM gathers each expert's rows from
-  // x through perm_src, and the permute writes the maps only; with CTA pairs
-  // the packed copy plus TMA rows is faster, so the permute copies the rows.
+  // x through perm_src, and only the row maps are needed: the router writes
+  // them itself when the batch is one tile, else the permute writes them.
+  // With CTA pairs the packed copy plus TMA rows is faster, so the permute
+  // copies the rows.
   const bool gather = gather_rows_in_gemm(c, x);
+  const bool maps_in_route = gather && route_writes_maps(c);
   {
+    TraceRange stage("moe_forward.route");
+    MOE_TRY(enqueue_route(c, x, w_router, bias, idx, gate, at<int>(ws, L.counts), offsets, ws, s,
+                          maps_in_route ? at<int>(ws, L.inv_row) : nullptr,
+                          maps_in_route ? at<int>(ws, L.perm_src) : nullptr));
+  }
+  if (!maps_in_route) {
     TraceRange stage("moe_forward.permute");
     MOE_CUDA(launch_permute(c.dtype, x, idx, offsets, at<int>(ws, L.cbase), route_tile_base(c, ws), c.T, c.d,
                             c.E, c.k, at<char>(ws, L.x_perm), at<int>(ws, L.perm_src), at<int>(ws, L.inv_row),

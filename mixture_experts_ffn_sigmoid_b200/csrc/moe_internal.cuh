@@ -215,6 +215,8 @@ struct FusedRouterLaunch {
   float* logits; int* topk_idx; float* topk_gate;
   int* chunk_base; int* tile_hist; int* tile_base; int* counts; int* offsets;
   uint32_t* err; uint32_t* done_count;
+  int* inv_row = nullptr;    // with perm_src: the permute's row maps too (T <= 128 only)
+  int* perm_src = nullptr;
 };
 bool router_fused_supported(int dtype, int E);
 int router_fused_cluster(int T, int K);

@@ -67,14 +67,20 @@ struct FusedRouterArgs {
   uint32_t* err;
   uint32_t* done_count;   // zero before the launch; the last tile sets it back to zero
   long long timeout_ns;
+  // With one tile (T <= 128) and these set, the row maps of the permute as
+  // well: inv_row [T][k] (each token's packed rows) and perm_src [T * k]
+  // (each packed row's token).
+  int* inv_row;
+  int* perm_src;
 };
 
 __host__ __device__ inline int fr_stage_bytes(int n_pad) { return FR_A_BYTES + n_pad * FR_BK * 2; }
 __host__ __device__ inline int fr_smem_bytes(int n_pad) {
   // alignment slack, header, ring (also the partial-logit buffer), the tile's
-  // chunk masks [kTileChunks][256], the scan's partial sums [4][256] and the
-  // selection bias [256]
-  return 1024 + FR_HDR + FR_STAGES * fr_stage_bytes(n_pad) + kTileChunks * 256 * 4 + 4 * 256 * 4 + 256 * 4 + 256;
+  // chunk masks [kTileChunks][256], the scan's partial sums [4][256], the
+  // selection bias [256] and the tile's chunk bases [kTileChunks][256]
+  return 1024 + FR_HDR + FR_STAGES * fr_stage_bytes(n_pad) + kTileChunks * 256 * 4 + 4 * 256 * 4 + 256 * 4 +
+         kTileChunks * 256 * 4 + 256;
 }
 
 // NPL consecutive fp32 values (NPL = 1, 2, 4 or 8) from the shared memory of
@@ -129,6 +135,7 @@ __global__ void __launch_bounds__(FR_THREADS, 1)
   uint32_t* s_mask = reinterpret_cast<uint32_t*>(ring + FR_STAGES * stage_bytes);   // [kTileChunks][256]
   int* s_part = reinterpret_cast<int*>(s_mask + kTileChunks * 256);                 // [4][256]
   float* s_bias = reinterpret_cast<float*>(s_part + 4 * 256);                       // [256]
+  int* s_cbase = reinterpret_cast<int*>(s_bias + 256);                               // [kTileChunks][256]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
@@ -362,6 +369,10 @@ __global__ void __launch_bounds__(FR_THREADS, 1)
       for (int j = 0; j < kTileChunks; ++j) {
         if (j < nch_tile) {
           p.chunk_base[(size_t)(tile * kTileChunks + j) * E + e] = run;
+          if (p.inv_row) {   // kept for the row maps: this thread's own entries
+            s_mask[j * 256 + e] = m[j];
+            s_cbase[j * 256 + e] = run;
+          }
           run += __popc(m[j]);
         }
       }
@@ -455,12 +466,30 @@ __global__ void __launch_bounds__(FR_THREADS, 1)
   if (g == 0) {
     int before = 0;
     for (int w = 0; w < warp; ++w) before += s_warp[w];
-    if (e < E) p.offsets[e] = before + incl - cnt;
+    if (e < E) {
+      p.offsets[e] = before + incl - cnt;
+      s_part[e] = before + incl - cnt;   // the partial sums are no longer read
+    }
     if (e == 0) {
       int total = 0;
       for (int w = 0; w < 8; ++w) total += s_warp[w];
       p.offsets[E] = total;
       *p.done_count = 0u;   // ready for the next launch
+    }
+  }
+  if (p.inv_row) {
+    // One tile: the rows of token t, j-th choice e = offsets[e] + its chunk's
+    // base for e + the earlier tokens of its chunk that chose e (the tile's
+    // base is zero). The other CTAs' index stores are visible after the
+    // cluster barriers; read them from L2.
+    __syncthreads();
+    for (int i = threadIdx.x; i < tile_tokens * k; i += blockDim.x) {
+      const int tl = i / k;
+      const int e = __ldcg(&p.topk_idx[(size_t)(t0 + tl) * k + (i - tl * k)]);
+      const int c = tl / kChunk;
+      const int row = s_part[e] + s_cbase[c * 256 + e] + __popc(s_mask[c * 256 + e] & ((1u << (tl % kChunk)) - 1u));
+      p.inv_row[(size_t)(t0 + tl) * k + (i - tl * k)] = row;
+      p.perm_src[row] = t0 + tl;
     }
   }
   store_logits();
@@ -519,6 +548,11 @@ cudaError_t launch_router_fused(const FusedRouterLaunch& a, cudaStream_t s) {
   p.counts = a.counts; p.offsets = a.offsets;
   p.err = a.err; p.done_count = a.done_count;
   p.timeout_ns = kDefaultTimeoutNs;
+  if (a.inv_row || a.perm_src) {
+    if (!(a.inv_row && a.perm_src) || p.ntiles != 1) return cudaErrorInvalidValue;
+    p.inv_row = a.inv_row;
+    p.perm_src = a.perm_src;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.ntiles * S);
   cfg.blockDim = dim3(FR_THREADS);

@@ -176,3 +176,22 @@ def test_binding_requires_cuda_tensors():
     x = torch.zeros(64, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         B._ptr(x)
+
+
+def test_route_maps_support_and_host_rejections():
+    L = B.lib()
+    # one tile of the fused router: bf16, E <= 256, T <= 128
+    assert L.moe_route_maps_supported(ctypes.byref(_cfg(T=128))) == 1
+    assert L.moe_route_maps_supported(ctypes.byref(_cfg(T=129))) == 0
+    assert L.moe_route_maps_supported(ctypes.byref(_cfg(T=64, dtype=B.MOE_DTYPE_F32))) == 0
+    assert L.moe_route_maps_supported(ctypes.byref(_cfg(T=64, E=320))) == 0
+    assert L.moe_route_maps_supported(ctypes.byref(_cfg(k=9))) == -1
+    fake = ctypes.c_void_p(0x10000)        # never dereferenced: every case fails on the host
+    for cfg in (_cfg(T=129), _cfg(T=64, dtype=B.MOE_DTYPE_F32)):
+        nbytes = L.moe_workspace_size(ctypes.byref(cfg))
+        assert L.moe_route_maps(ctypes.byref(cfg), fake, fake, None, fake, fake, fake, fake, fake, fake, fake,
+                                nbytes, None) == B.MOE_ERR_UNSUPPORTED
+    cfg = _cfg(T=64)
+    nbytes = L.moe_workspace_size(ctypes.byref(cfg))
+    assert L.moe_route_maps(ctypes.byref(cfg), fake, fake, None, fake, fake, fake, fake, None, fake, fake,
+                            nbytes, None) == B.MOE_ERR_INVALID_ARG

@@ -23,6 +23,7 @@ import torch
 from mixture_experts_ffn_sigmoid_b200.inputs import GATE_SIGMOID, GATE_SOFTMAX, MoEConfig
 
 import gpu_harness as H
+from mixture_experts_ffn_sigmoid_b200 import binding as B
 
 pytestmark = pytest.mark.gpu
 
@@ -120,3 +121,60 @@ def test_all_scores_equal_pick_the_lowest_groups_and_ids(dtype):
     assert np.abs(gg - cfg.route_scale / cfg.k).max() <= H.gate_tol(cfg)
     ref = H.oracle_route(cfg, inp)
     assert np.array_equal(ref["idx"], gi)
+
+
+# moe_route_maps: the fused router of a one-tile batch also writes the row
+# maps; they must equal moe_route followed by the maps-only moe_permute.
+MAPS = {
+    "maps_t1": _cfg("maps_t1", 16, 4, T=1),
+    "maps_t33_e256_g8": _cfg("maps_t33", 256, 8, 8, 4, T=33),
+    "maps_t128_e128_softmax": _cfg("maps_t128", 128, 8, gate=GATE_SOFTMAX, T=128),
+    "maps_t100_e72_g24": _cfg("maps_t100", 72, 6, 24, 4, T=100),
+    "maps_t64_e8_k8": _cfg("maps_t64_k8", 8, 8, T=64),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MAPS))
+def test_route_maps_equal_route_then_permute(name):
+    cfg = MAPS[name]
+    inp = H.gpu_inputs(cfg, seed=7)
+    assert B.moe_route_maps_supported(cfg)
+    ref = H.gpu_route(cfg, inp)
+    rows = cfg.T * cfg.k
+    src_a = torch.full((rows,), -7, dtype=torch.int32, device="cuda")
+    inv_a = torch.full((cfg.T, cfg.k), -7, dtype=torch.int32, device="cuda")
+    B.moe_permute(cfg, None, ref["idx"], ref["offsets"], None, src_a, inv_a, ref["ws"])
+    ws = B.alloc_workspace(cfg)
+    idx = torch.full((cfg.T, cfg.k), -7, dtype=torch.int32, device="cuda")
+    gate = torch.full((cfg.T, cfg.k), float("nan"), dtype=torch.float32, device="cuda")
+    counts = torch.full((cfg.E,), -7, dtype=torch.int32, device="cuda")
+    offsets = torch.full((cfg.E + 1,), -7, dtype=torch.int32, device="cuda")
+    src_b = torch.full((rows,), -7, dtype=torch.int32, device="cuda")
+    inv_b = torch.full((cfg.T, cfg.k), -7, dtype=torch.int32, device="cuda")
+    B.moe_route_maps(cfg, inp["x"], inp["w_router"], inp["bias"], idx, gate, counts, offsets, src_b, inv_b, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, ref["idx"]) and torch.equal(gate, ref["gate"])
+    assert torch.equal(counts, ref["counts"]) and torch.equal(offsets, ref["offsets"])
+    assert torch.equal(src_b, src_a) and torch.equal(inv_b, inv_a)
+    assert B.moe_get_device_error(ws) == B.MOE_OK
+    H.check_route(cfg, H.oracle_route(cfg, inp), ref)
+
+
+@pytest.mark.parametrize("cfg", [_cfg("maps_t129", 64, 4, T=129), _cfg("maps_f32", 64, 4, dtype="f32", T=64),
+                                 _cfg("maps_e320", 320, 4, T=64)], ids=lambda c: c.name)
+def test_route_maps_unsupported_writes_nothing(cfg):
+    assert not B.moe_route_maps_supported(cfg)
+    inp = H.gpu_inputs(cfg, seed=7)
+    ws = B.alloc_workspace(cfg)
+    rows = cfg.T * cfg.k
+    idx = torch.full((cfg.T, cfg.k), -7, dtype=torch.int32, device="cuda")
+    gate = torch.zeros((cfg.T, cfg.k), dtype=torch.float32, device="cuda")
+    counts = torch.full((cfg.E,), -7, dtype=torch.int32, device="cuda")
+    offsets = torch.full((cfg.E + 1,), -7, dtype=torch.int32, device="cuda")
+    src = torch.full((rows,), -7, dtype=torch.int32, device="cuda")
+    inv = torch.full((cfg.T, cfg.k), -7, dtype=torch.int32, device="cuda")
+    with pytest.raises(B.MoEError) as e:
+        B.moe_route_maps(cfg, inp["x"], inp["w_router"], inp["bias"], idx, gate, counts, offsets, src, inv, ws)
+    assert e.value.status == B.MOE_ERR_UNSUPPORTED
+    torch.cuda.synchronize()
+    assert int(idx.min()) == -7 and int(src.max()) == -7 and int(counts.max()) == -7
