@@ -36,6 +36,26 @@ namespace {
 // their accumulators (2 x 256 TMEM columns) fill TMEM, so the next tile's
 // MMAs wait for the epilogue; one block keeps two accumulator stages. Long
 // contractions (hundreds of rows per segment) take two blocks, short ones one.
+// All but the newest committed bulk group have read their shared memory.
+__device__ __forceinline__ void bulk_wait_read_but_one() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
+// The output map: bf16 [n_seg][M][N], 64-byte swizzle, 32 x 32 x 1 boxes
+// (stores clip at each dimension's bound).
+bool make_out_tmap(CUtensorMap* tm, void* base, long long n, long long m, long long segs) {
+  auto fn = get_encode_fn();
+  if (!fn || n <= 0 || m <= 0 || segs <= 0 || (n * 2) % 16) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)n, (cuuint64_t)m, (cuuint64_t)segs};
+  cuuint64_t strides[2] = {(cuuint64_t)(n * 2), (cuuint64_t)(m * n * 2)};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <int MB> struct WgShape {
   static constexpr int BM = 128 * MB;
   static constexpr int ACC_STAGES = MB == 1 ? 2 : 1;
@@ -47,7 +67,8 @@ constexpr int WG_BOX = 64 * 64 * 2;                      // one 64 x 64 bf16 box
 constexpr int WG_B_BYTES = 4 * WG_BOX;                   // 256 n x 64 rows
 constexpr int WG_THREADS = 320;
 constexpr int WG_EPI_WARPS = 8;
-constexpr int WG_STG_BYTES = 32 * 64 * 2;                // one warp's 32 x 64 output box
+constexpr int WG_STG_BYTES = 2 * 32 * 32 * 2;            // one warp's two 32 x 32 output boxes
+constexpr int WG_OBOX = 32 * 32 * 2;                     // one 32 x 32 bf16 output box (64-byte rows)
 constexpr int WG_TMEM_COLS = 512;
 template <int MB> constexpr int wg_a_bytes() { return 2 * MB * WG_BOX; }
 template <int MB> constexpr int wg_stage_bytes() { return wg_a_bytes<MB>() + WG_B_BYTES; }
@@ -230,11 +251,13 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
     __syncwarp();
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue
-    // Each warp converts its 32 rows x 64 columns to bf16 into a swizzled
-    // staging box (row = lane, 16-byte chunk c at c ^ (row & 7), the layout
-    // TMA's 128-byte swizzle reads) and lane 0 stores the box with TMA: one
-    // bulk write per 4 KB instead of 32 scattered 16-byte stores per
-    // instruction. The 3-D output map clips rows past M and columns past N.
+    // Each warp converts its 32 rows x 32 columns at a time to bf16 into one
+    // of two staging boxes (row = lane, 16-byte chunk c at c ^ ((row >> 1) & 3),
+    // the layout TMA's 64-byte swizzle reads) and lane 0 stores the box with
+    // TMA. With two boxes a chunk waits only for the store issued two chunks
+    // earlier to have read its box out, so the stores overlap the next
+    // chunk's TMEM loads and conversion. The 3-D output map clips rows past M
+    // and columns past N.
     const int q = warp & 3;                    // TMEM lane quarter this warp may read
     // Warps 2-5 and 6-9 split the tile: by M block when there are two (each
     // warp then stores all 256 columns of its 32 rows), else by column half.
@@ -242,27 +265,29 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
     const int blk = WG_MB == 2 ? grp : 0;
     const int ncol = WG_MB == 2 ? WG_BN : WG_BN / 2;
     const int cbeg = WG_MB == 2 ? 0 : grp * (WG_BN / 2);
-    const uint32_t box = smem_u32(stage_out + (warp - 2) * WG_STG_BYTES);
+    const uint32_t box0 = smem_u32(stage_out + (warp - 2) * WG_STG_BYTES);
     int acc = 0;
     uint32_t acc_phase = 0;
+    uint32_t nbox = 0;                         // boxes this warp has stored (selects the buffer)
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
       const WgTile t = wg_tile<WG_BM>(p, tile, mt, nt);
       const int mrow = t.m0 + blk * 128 + q * 32;   // first row of this warp's boxes
       const int nbeg = t.n0 + cbeg;
       if (t.nk == 0) {
         // No row chose this segment: its gradient is zero. Store a zeroed
-        // staging box over the warp's 32 x 64 output boxes.
+        // staging box over the warp's 32 x 32 output boxes.
         if (mrow < p.M && nbeg < p.N) {
           if (lane == 0) bulk_wait_read_all();
           __syncwarp();
 #pragma unroll
-          for (int c = 0; c < 8; ++c) st_shared_zero16(box + lane * 128 + c * 16);
+          for (int c = 0; c < 4; ++c) st_shared_zero16(box0 + lane * 64 + c * 16);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            for (int c0 = 0; c0 < ncol && nbeg + c0 < p.N; c0 += 64) tma_store_3d(&tmD, box, nbeg + c0, mrow, t.seg);
+            for (int c0 = 0; c0 < ncol && nbeg + c0 < p.N; c0 += 32) tma_store_3d(&tmD, box0, nbeg + c0, mrow, t.seg);
             bulk_commit();
           }
+          nbox = 1;   // the next box written is the second one
         }
         continue;
       }
@@ -270,23 +295,26 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) +
                              (uint32_t)((WG_MB == 2 ? blk : acc) * WG_BN + cbeg);
-      for (int c0 = 0; c0 < ncol; c0 += 64) {
+      for (int c0 = 0; c0 < ncol; c0 += 32) {
         if (nbeg + c0 >= p.N || mrow >= p.M) break;
-        uint32_t r[64];
-        tmem_ld64_wait(taddr + c0, r);
-        // The previous store must have read the staging box out.
-        if (lane == 0) bulk_wait_read_all();
+        uint32_t ra[16], rb[16];
+        tmem_ld16x2_wait(taddr + c0, taddr + c0 + 16, ra, rb);
+        const uint32_t box = box0 + (nbox & 1u) * WG_OBOX;
+        // The store of two boxes ago (same buffer) must have read it out.
+        if (lane == 0) bulk_wait_read_but_one();
         __syncwarp();
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t w[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[8 * c + 2 * j]),
-                                                           __uint_as_float(r[8 * c + 2 * j + 1]));
+            const int i = 8 * c + 2 * j;   // columns i, i + 1 of the 32
+            const float lo = __uint_as_float(i < 16 ? ra[i] : rb[i - 16]);
+            const float hi = __uint_as_float(i + 1 < 16 ? ra[i + 1] : rb[i + 1 - 16]);
+            const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
             w[j] = *reinterpret_cast<const uint32_t*>(&h);
           }
-          const uint32_t dst = box + lane * 128 + ((c ^ (lane & 7)) * 16);
+          const uint32_t dst = box + lane * 64 + ((c ^ ((lane >> 1) & 3)) * 16);
           asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(w[0]), "r"(w[1]), "r"(w[2]),
                        "r"(w[3])
                        : "memory");
@@ -297,6 +325,7 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
           tma_store_3d(&tmD, box, nbeg + c0, mrow, t.seg);
           bulk_commit();
         }
+        ++nbox;
       }
       tc_fence_before();
       __syncwarp();
@@ -321,8 +350,7 @@ cudaError_t launch_wgrad(const WgradParams& p, int num_sms, cudaStream_t s) {
   CUtensorMap tP, tQ, tD;
   if (!make_tmap_strided(&tP, p.P, p.M, p.p_rows, p.ldP * 2, 64)) return cudaErrorInvalidValue;
   if (!make_tmap_strided(&tQ, p.Q, p.N, p.q_rows, p.ldQ * 2, 64)) return cudaErrorInvalidValue;
-  if (!make_tmap_3d(&tD, p.out, p.N, p.M, p.n_seg, (long long)p.N * 2, (long long)p.M * p.N * 2, 32))
-    return cudaErrorInvalidValue;
+  if (!make_out_tmap(&tD, p.out, p.N, p.M, p.n_seg)) return cudaErrorInvalidValue;
   // Two M blocks per tile once segments average more than 256 rows.
   const long long rows_per_seg = (p.offsets ? (long long)p.p_rows : (long long)p.k_total) / p.n_seg;
   const bool two = rows_per_seg > 256;
