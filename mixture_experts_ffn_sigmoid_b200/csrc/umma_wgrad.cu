@@ -14,8 +14,10 @@
 // per 128-row M block, sharing the staged Q tile), rows in blocks of 64. Both operands arrive as 64 x 64 TMA boxes (128-byte swizzle,
 // MN-major: 64-element M/N groups 8 KB apart, 8-row groups 1 KB apart).
 // Rows of the last block past the segment's end belong to the next segment:
-// the MMA warp zeroes those rows of the P tile in shared memory before the
-// MMA, so they add nothing (Q's rows there are finite data or zero fill).
+// the MMAs (16 rows each) stop at the one holding the segment's last row,
+// and the MMA warp zeroes that MMA's rows past the end in the P tile in
+// shared memory, so they add nothing (Q's rows there are finite data or
+// zero fill).
 //
 // Roles (320 threads, one CTA per SM, persistent over tiles ordered
 // segment-major, so CTAs running at once share a segment's rows in L2):
@@ -206,15 +208,20 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
         }
         const uint32_t sa = smem_u32(ring + stage * WG_STAGE_BYTES);
         const int valid = min(WG_BK, t.rows - kb * WG_BK);
-        if (valid < WG_BK) {
+        // MMAs of 16 rows each: only those that reach a valid row run, and
+        // only the rows past `valid` inside the last of them are zeroed.
+        const int n_kk = (valid + 15) / 16;
+        const int pad = n_kk * 16 - valid;
+        if (pad > 0) {
           // Every lane sees the completed phase itself (it has completed, so
           // the wait returns at once) before overwriting rows TMA wrote.
           wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, p.err, p.timeout_ns, false);
-          // Rows valid..63 of the loaded 64-row P boxes: 128 bytes each, 8 x 16 B.
-          const int n16 = (WG_BK - valid) * na * 8;
+          // Rows valid .. valid + pad - 1 of the loaded 64-row P boxes: 128
+          // bytes each, 8 x 16 B.
+          const int n16 = pad * na * 8;
           for (int i = lane; i < n16; i += 32) {
-            const int h = i / ((WG_BK - valid) * 8);
-            const int rem = i - h * (WG_BK - valid) * 8;
+            const int h = i / (pad * 8);
+            const int rem = i - h * pad * 8;
             st_shared_zero16(sa + h * WG_BOX + (valid + rem / 8) * 128 + (rem % 8) * 16);
           }
           fence_proxy_async_smem();
@@ -229,6 +236,7 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
             const uint64_t a_desc = sw128_mn_desc(sa + blk * 2 * WG_BOX);
 #pragma unroll
             for (int kk = 0; kk < WG_BK / 16; ++kk) {
+              if (kk >= n_kk) break;
               const uint64_t koff = (uint64_t)((kk * 2 * 1024) >> 4);   // two 8-row groups per 16 rows
               umma_bf16(d + blk * WG_BN, a_desc + koff, b_desc + koff, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
             }
