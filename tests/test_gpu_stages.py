@@ -44,6 +44,11 @@ STAGE_CASES = {
                                    n_groups=8, topk_groups=4, route_scale=2.5, f_shared=128, bias="uniform"),
     "bulk_permute_fp32": MoEConfig("bulk_permute_f32", T=2040, d=136, E=32, k=4, f=64, dtype="f32",
                                    gate_mode=GATE_SIGMOID, route_scale=1.0, bias="uniform"),
+    # More chunks than SMs (150 > 148): each chunk's rows are split over
+    # eight four-token blocks, and the last chunk holds two tokens.
+    "bulk_permute_split_bf16": MoEConfig("bulk_permute_split", T=4770, d=128, E=64, k=4, f=64,
+                                         gate_mode=GATE_SIGMOID, n_groups=8, topk_groups=4, route_scale=2.5,
+                                         f_shared=64, bias="uniform"),
 }
 
 
