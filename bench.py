@@ -482,7 +482,10 @@ def stage_breakdown(B, cfg, inp, ws, stream, n):
     nodes inside the graph), replayed n times; each replay is read back before
     the next. A stage's time is the device time between its events in a chain
     that runs like moe_forward's graph, once per pass. Returns the mean
-    milliseconds per stage and the stage outputs (of the last pass)."""
+    milliseconds per stage, the stage outputs (of the last pass), and each
+    short stage's (route, permute, combine) milliseconds per call when its
+    entry point runs back to back in a graph of its own (no event node
+    between launches)."""
     dev = inp["x"].device
     T, d, E, k = cfg.T, cfg.d, cfg.E, cfg.k
     rows = T * k
@@ -512,7 +515,7 @@ def stage_breakdown(B, cfg, inp, ws, stream, n):
                                   o["offsets"], o["perm_src"], o["inv_row"], ws)) if maps_in_route
         else (lambda: B.moe_route(cfg, inp["x"], inp["w_router"], inp["bias"], o["idx"], o["gate"], o["counts"],
                                   o["offsets"], ws)),
-        (lambda: None) if maps_in_route
+        None if maps_in_route
         else (lambda: B.moe_permute(cfg, None, o["idx"], o["offsets"], None, o["perm_src"], o["inv_row"], ws))
         if gather
         else (lambda: B.moe_permute(cfg, inp["x"], o["idx"], o["offsets"], o["x_perm"], o["perm_src"],
@@ -527,7 +530,8 @@ def stage_breakdown(B, cfg, inp, ws, stream, n):
     ]
     for _ in range(2):
         for c in calls:
-            c()
+            if c:
+                c()
     torch.cuda.synchronize()
     # external: recorded inside the capture as timing event nodes
     evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(calls) + 1)]
@@ -535,7 +539,8 @@ def stage_breakdown(B, cfg, inp, ws, stream, n):
     with torch.cuda.graph(g):
         evs[0].record()
         for j, c in enumerate(calls):
-            c()
+            if c:
+                c()
             evs[j + 1].record()
     g.replay()
     torch.cuda.synchronize()
@@ -546,8 +551,37 @@ def stage_breakdown(B, cfg, inp, ws, stream, n):
         for j in range(len(calls)):
             acc[j] += evs[j].elapsed_time(evs[j + 1])
     del g
+    # The short stages alone: `reps` calls of the entry point back to back in
+    # one CUDA graph (launches pipelined as inside moe_forward's graph, no
+    # event node between them), device time per call. Every call redoes the
+    # whole stage on the same inputs. The event nodes of the chain above add
+    # a few microseconds per stage, which is a large share of these; the
+    # expert GEMMs are left out (eight of them back to back run under the
+    # power cap, below the clock they run at in the step).
+    reps = 8
+    iso = {}
+    for j, c in enumerate(calls):
+        if names[j] not in ("route", "permute", "combine"):
+            continue
+        if c is None:   # no launch of its own on this path
+            iso[names[j]] = 0.0
+            continue
+        gj = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gj):
+            for _ in range(reps):
+                c()
+        gj.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(2):
+            gj.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        iso[names[j]] = e0.elapsed_time(e1) / (2 * reps)
+        del gj
     assert B.moe_get_device_error(ws) == B.MOE_OK
-    return {nm: acc[j] / n for j, nm in enumerate(names)}, o
+    return {nm: acc[j] / n for j, nm in enumerate(names)}, o, iso
 
 
 def graph_step_ms(B, cfg, inp, ws, y, stream, steps, warmup):
@@ -588,7 +622,7 @@ def measure_workload(B, name, dev, stream, steps, warmup, sampler, peaks):
     ws = B.alloc_workspace(cfg, dev)
     y = torch.empty((cfg.T, cfg.d), dtype=cfg.torch_dtype, device=dev)
     ms, t0, t1 = graph_step_ms(B, cfg, inp, ws, y, stream, steps, warmup)
-    stage_ms, o = stage_breakdown(B, cfg, inp, ws, stream, max(3, min(steps, 50)))
+    stage_ms, o, stage_iso = stage_breakdown(B, cfg, inp, ws, stream, max(3, min(steps, 50)))
     assert torch.equal(o["y"], y), f"{name}: per-stage chain and moe_forward disagree"
     work, touched = stage_work(cfg, o["counts"].cpu(), B.moe_forward_gathers_rows(cfg, inp["x"]))
     expert_ms = stage_ms["gate_up"] + stage_ms["down"]
@@ -601,7 +635,7 @@ def measure_workload(B, name, dev, stream, steps, warmup, sampler, peaks):
                     "topk_groups": cfg.topk_groups, "route_scale": cfg.route_scale, "dtype": cfg.dtype},
          "ms_per_step": ms, "steps": steps, "cuda_graph": True,
          "tokens_per_s": cfg.T / (ms / 1e3), "active_tflops": flops / (ms / 1e3) / 1e12,
-         "experts_touched": touched, "stages_ms": stage_ms,
+         "experts_touched": touched, "stages_ms": stage_ms, "stages_ms_back_to_back": stage_iso,
          "layer_bytes": lb, "step_gbs": lb / (ms / 1e3) / 1e9,
          "step_frac_hbm": lb / (ms / 1e3) / 1e9 / peaks["hbm"],
          "expert_gemm": {"ms": expert_ms, "tflops": expert_flops / (expert_ms / 1e3) / 1e12,
@@ -765,7 +799,7 @@ def main():
     k, E = cfg.k, cfg.E
     n_stage = max(3, min(args.steps, 50))
     names = ["route", "permute", "gate_up", "down", "combine"]
-    stage_ms, so = stage_breakdown(B, cfg, inp, ws, stream, n_stage)
+    stage_ms, so, stage_iso = stage_breakdown(B, cfg, inp, ws, stream, n_stage)
     idx, gate, counts, offsets = so["idx"], so["gate"], so["counts"], so["offsets"]
     perm_src, inv_row, h, h_s = so["perm_src"], so["inv_row"], so["h"], so["h_s"]
     assert torch.equal(so["y"], y), "per-stage chain and moe_forward disagree"
@@ -773,6 +807,7 @@ def main():
         sampler.stop()
         if rank == 0:
             print(json.dumps({"profiling_run": cfg.name, "ms_per_step": ms_step, "stages_ms": stage_ms,
+                              "stages_ms_back_to_back": stage_iso,
                               "clocks": clocks}), flush=True)
         if graph is not None:
             del graph
@@ -929,6 +964,7 @@ def main():
                             "frac_tensor": expert_flops / (expert_ms / 1e3) / 1e12 / peaks["tensor_sustained"],
                             "frac_hbm": expert_bytes / (expert_ms / 1e3) / 1e9 / peaks["hbm"]},
             "stages_ms": stage_ms,
+            "stages_ms_back_to_back": stage_iso,
             "balance_update": balance,
             "gelu_experts": gelu,
             "fused_permute_gather": fused,
