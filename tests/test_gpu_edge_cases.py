@@ -28,6 +28,11 @@ EDGE = {
                                 n_groups=8, topk_groups=1, route_scale=2.5, bias="uniform"),
     "k1_fp32": MoEConfig("k1_fp32", T=50, d=64, E=5, k=1, f=48, dtype="f32"),
     "many_experts": MoEConfig("many_experts", T=64, d=128, E=1024, k=32, f=64),
+    # One full router tile of a DeepSeek-V3-style routing (grouped sigmoid,
+    # shared expert) at decode size: moe_forward routes and writes the row
+    # maps in one launch and its gate/up GEMM gathers the rows from x.
+    "one_tile_grouped": MoEConfig("one_tile_grouped", T=128, d=512, E=256, k=8, f=256, gate_mode=GATE_SIGMOID,
+                                  n_groups=8, topk_groups=4, route_scale=2.5, f_shared=256, bias="uniform"),
 }
 
 
@@ -35,6 +40,8 @@ EDGE = {
 def test_edge_forward(name):
     cfg = EDGE[name]
     inp = H.gpu_inputs(cfg)
+    if name == "one_tile_grouped":
+        assert B.moe_forward_gathers_rows(cfg, inp["x"]) and B.moe_route_maps_supported(cfg)
     got = H.gpu_route(cfg, inp)
     H.check_route(cfg, H.oracle_route(cfg, inp), got)
     y = H.gpu_forward(cfg, inp)
