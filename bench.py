@@ -693,6 +693,16 @@ def oracle_sample_time(cfg, inp, n_tokens, seed):
     return dt, threads
 
 
+def workload_config(cfg, world: int) -> dict:
+    """The JSON line's `config`: the workload, identical on both arms."""
+    return {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k, "f": cfg.f,
+            "f_shared": cfg.f_shared, "gate": "sigmoid" if cfg.gate_mode else "softmax",
+            "n_groups": cfg.n_groups, "topk_groups": cfg.topk_groups, "route_scale": cfg.route_scale,
+            "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2: every step streams the layer's expert weights "
+                  f"({(cfg.E * 3 * cfg.f * cfg.d + 3 * cfg.f_shared * cfg.d) * cfg.elem_bytes / 1e9:.2f} GB)"}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -717,8 +727,7 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k, "f": cfg.f,
-                       "f_shared": cfg.f_shared},
+            "config": workload_config(cfg, args.gpus),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -950,13 +959,7 @@ def main():
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "f32", "data": "synthetic",
-            "config": {"workload": cfg.name, "T": T, "d": d, "E": E, "k": k, "f": cfg.f,
-                       "f_shared": cfg.f_shared, "gate": "sigmoid" if cfg.gate_mode else "softmax",
-                       "n_groups": cfg.n_groups, "topk_groups": cfg.topk_groups,
-                       "route_scale": cfg.route_scale, "parallelism": f"replicas x{world}",
-                       "cuda_graph": graph is not None,
-                       "l2": "inputs larger than L2: every step streams the touched expert weights "
-                             f"({(touched * 3 * cfg.f * d + 3 * cfg.f_shared * d) * cfg.elem_bytes / 1e9:.2f} GB)"},
+            "config": workload_config(cfg, world), "cuda_graph": graph is not None,
             "active_tflops": cfg.active_flops() * world / (ms_step / 1e3) / 1e12,
             "experts_touched": touched,
             "expert_gemm": {"ms": expert_ms, "tflops": expert_flops / (expert_ms / 1e3) / 1e12,
