@@ -10,8 +10,9 @@
 // (Sparse MoE FFN note, "Packed forward": each expert sees the tokens that
 // chose it). Segments no row belongs to get D_s = 0.
 //
-// Tiles: 256 m x 256 n per CTA (two M=128, N=256 MMAs per 16 rows, one
-// per 128-row M block, sharing the staged Q tile), rows in blocks of 64. Both operands arrive as 64 x 64 TMA boxes (128-byte swizzle,
+// Tiles: 128 or 256 m x 256 n per CTA (one M=128, N=256 MMA per 16 rows for
+// each 128-row M block; two blocks share the staged Q tile), rows in blocks
+// of 64. Both operands arrive as 64 x 64 TMA boxes (128-byte swizzle,
 // MN-major: 64-element M/N groups 8 KB apart, 8-row groups 1 KB apart).
 // Rows of the last block past the segment's end belong to the next segment:
 // the MMAs (16 rows each) stop at the one holding the segment's last row,
@@ -21,23 +22,18 @@
 //
 // Roles (320 threads, one CTA per SM, persistent over tiles ordered
 // segment-major, so CTAs running at once share a segment's rows in L2):
-//   warp 0 lane 0 : TMA producer into a 4-stage ring
+//   warp 0 lane 0 : TMA producer into a 4-stage ring (3 with two M blocks)
 //   warp 1        : TMEM allocator; zero-fills partial blocks; lane 0 issues
 //                   tcgen05.mma and tcgen05.commit
 //   warps 2..9    : epilogue; warp w reads TMEM lane quarter w % 4 of one M
-//                   block (or half the columns with one block), 64 columns per
-//                   load wait, and writes 32 x 64 boxes with TMA stores
+//                   block (or half the columns with one block), 32 columns per
+//                   load wait, and writes 32 x 32 boxes with TMA stores
 // Every wait is bounded, as in the forward GEMM.
 #include "umma_common.cuh"
 
 namespace moe {
 namespace {
 
-// Tile shapes. WG_MB 128-row M blocks per tile: two blocks share each
-// staged Q tile, cutting the operands read per output byte by a third, but
-// their accumulators (2 x 256 TMEM columns) fill TMEM, so the next tile's
-// MMAs wait for the epilogue; one block keeps two accumulator stages. Long
-// contractions (hundreds of rows per segment) take two blocks, short ones one.
 // All but the newest committed bulk group have read their shared memory.
 __device__ __forceinline__ void bulk_wait_read_but_one() {
   asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
@@ -58,6 +54,11 @@ bool make_out_tmap(CUtensorMap* tm, void* base, long long n, long long m, long l
   return r == CUDA_SUCCESS;
 }
 
+// Tile shapes. WG_MB 128-row M blocks per tile: two blocks share each
+// staged Q tile, cutting the operands read per output byte by a third, but
+// their accumulators (2 x 256 TMEM columns) fill TMEM, so the next tile's
+// MMAs wait for the epilogue; one block keeps two accumulator stages. Long
+// contractions (hundreds of rows per segment) take two blocks, short ones one.
 template <int MB> struct WgShape {
   static constexpr int BM = 128 * MB;
   static constexpr int ACC_STAGES = MB == 1 ? 2 : 1;
